@@ -1,0 +1,375 @@
+"""Plain fp64 CPU oracle of the single-device MoE layer forward.
+
+TEST INFRASTRUCTURE.  Nothing on the product path may import, call or run
+this module: only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline
+leg of ``bench.py`` use it.  It is written for a reader who wants to check it
+against the pages by eye: every step is the textbook definition, one expert
+or one token at a time, with NumPy float64 matmuls and sorts as the only
+library primitives.  No blocking, fusion or reordering beyond that.
+
+Sources (page title, then the function or section on it):
+
+* [HP]  hyper_parallel ``platform/torch/common/moe.py`` coverage page --
+  ``TokenChoiceTopKRouter.forward``, ``MoE.permutation``,
+  ``MoE.unpermutation``, ``_run_experts_for_loop``, ``MoE.forward``.
+* [QO]  QwenLM/Qwen3-Omni issue #115 "Training: Extremely Slow Deepspeed
+  Engine initialization ..." -- ``SpeedupMoeExperts.forward`` (training
+  branch: per-expert ``index_add_``; eval branch: dense ``bmm`` over all
+  experts) and ``SpeedupMoeSparseMoeBlock.forward`` (``norm_topk_prob``).
+* [EP]  huggingface/transformers PR #41053 "Qwen3 moe" --
+  ``Ep2DpParallel._token_dispatch`` (per-rank counts, all-to-all, the
+  received buffer that "needs to be reshuffled back").
+
+Readings taken where the pages are silent or disagree (each is repeated in
+the design notes):
+
+* top-k order: descending score, ties to the lower expert index; selection is
+  on the router logits (softmax is strictly increasing, so the selected set
+  and its order are the same as on the probabilities).
+* the order of copies inside one expert's segment is the order of the flat
+  index ``t*k + j`` ([HP] ``MoE.permutation`` uses a stable argsort).
+* the routing weight multiplies the expert output (after ``w2``), as in [QO]
+  ``weighted_output``; [HP] applies it to the hidden activation before ``w2``,
+  which is the same number by linearity of ``w2``.
+* ``offsets`` has ``E + 1`` entries (exclusive scan including the total).
+* the received EP buffer is source-rank-major: for each destination block,
+  source rank outer and local expert inner; the regroup output is local
+  expert outer and source rank inner.
+
+Parity pins: every function here is pinned by a ``-m "not gpu"`` test that
+does not re-derive it (hand cases, closed forms, brute force, invariants, a
+second formulation).  No function is "parity unpinned".
+"""
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "as_f64", "router_logits", "topk_select", "softmax", "router_topk",
+    "expert_counts", "dispatch", "permute_rows", "ep_dispatch_rank_major",
+    "ep_local_regroup", "apply_row_perm", "silu", "swiglu_ffn",
+    "grouped_swiglu", "combine", "moe_forward", "dense_moe", "moe_tokens",
+]
+
+
+def as_f64(a) -> np.ndarray:
+    """Exact conversion of a torch tensor (fp32/bf16) or array to float64."""
+    try:
+        import torch
+        if isinstance(a, torch.Tensor):
+            a = a.detach().to("cpu")
+            if a.dtype in (torch.bfloat16, torch.float16):
+                a = a.to(torch.float32)          # exact widening
+            return a.numpy().astype(np.float64)
+    except ImportError:  # pragma: no cover
+        pass
+    return np.asarray(a, dtype=np.float64)
+
+
+def _i64(a) -> np.ndarray:
+    try:
+        import torch
+        if isinstance(a, torch.Tensor):
+            return a.detach().to("cpu").numpy().astype(np.int64)
+    except ImportError:  # pragma: no cover
+        pass
+    return np.asarray(a, dtype=np.int64)
+
+
+# --------------------------------------------------------------------------
+# Router  ([HP] TokenChoiceTopKRouter.forward; [QO] SpeedupMoeSparseMoeBlock)
+# --------------------------------------------------------------------------
+
+def router_logits(x, w_router) -> np.ndarray:
+    """Gate logits ``x @ w_router^T`` in fp64 (the gate is a bias-free
+    ``nn.Linear(d, E)`` whose weight is ``w_router[E, d]``)."""
+    return as_f64(x) @ as_f64(w_router).T
+
+
+def topk_select(scores, top_k: int) -> np.ndarray:
+    """Indices of the ``top_k`` largest scores per row, largest first, ties
+    broken towards the lower expert index.  ``int64 [T, k]``.
+
+    A stable sort of the negated scores keeps equal scores in index order.
+    """
+    s = as_f64(scores)
+    order = np.argsort(-s, axis=1, kind="stable")
+    return order[:, :top_k]
+
+
+def softmax(L) -> np.ndarray:
+    """Row softmax ``exp(L - max) / sum`` in fp64."""
+    L = as_f64(L)
+    z = np.exp(L - L.max(axis=1, keepdims=True))
+    return z / z.sum(axis=1, keepdims=True)
+
+
+def router_topk(top_k: int, renormalize: bool, x=None, w_router=None, logits=None):
+    """Token-choice top-k router.
+
+    Scores are the fp32 gate logits if ``logits`` is given (consumed exactly),
+    else the fp64 ``x @ w_router^T``.  Returns ``(idx[T,k] int64,
+    w[T,k] fp64, counts[E] int64, logits[T,E] fp64)``.
+
+    [HP] ``TokenChoiceTopKRouter.forward``: softmax over all experts, top-k,
+    gather of the (unbiased) probabilities, bincount.  [QO]
+    ``SpeedupMoeSparseMoeBlock.forward``: with ``norm_topk_prob`` the k
+    weights are divided by their sum.
+    """
+    L = as_f64(logits) if logits is not None else router_logits(x, w_router)
+    idx = topk_select(L, top_k)
+    p = softmax(L)
+    w = np.take_along_axis(p, idx, axis=1)
+    if renormalize:
+        w = w / w.sum(axis=1, keepdims=True)
+    counts = expert_counts(idx, L.shape[1])
+    return idx, w, counts, L
+
+
+def expert_counts(idx, E: int) -> np.ndarray:
+    """``counts[e] = #{(t, j): idx[t, j] == e}`` ([HP] ``torch.bincount``)."""
+    return np.bincount(_i64(idx).ravel(), minlength=E).astype(np.int64)
+
+
+# --------------------------------------------------------------------------
+# Dispatch  ([HP] MoE.permutation and the gather in MoE.forward)
+# --------------------------------------------------------------------------
+
+def dispatch(idx, E: int):
+    """Expert-major permutation of the routed copies.
+
+    Flattening ``idx[T, k]`` gives flat index ``f = t*k + j``; a stable sort of
+    the flat expert ids lists the copies expert by expert, and inside one
+    expert in increasing ``f`` ([HP] ``MoE.permutation``).  Returns
+
+    * ``counts[E]``, ``offsets[E+1]`` (exclusive scan, ``offsets[E] = T*k``),
+    * ``src_row[N]``: the token of each expert-major slot (``f // k``),
+    * ``dst_pos[T, k]``: the slot of each copy (inverse of the sort).
+    """
+    idx = _i64(idx)
+    T, k = idx.shape
+    flat = idx.ravel()
+    order = np.argsort(flat, kind="stable")       # slot -> flat index
+    counts = np.bincount(flat, minlength=E).astype(np.int64)
+    offsets = np.zeros(E + 1, dtype=np.int64)
+    offsets[1:] = np.cumsum(counts)
+    src_row = order // k
+    dst = np.empty(T * k, dtype=np.int64)
+    dst[order] = np.arange(T * k)
+    return counts, offsets, src_row, dst.reshape(T, k)
+
+
+def permute_rows(x, src_row) -> np.ndarray:
+    """``x_perm[s] = x[src_row[s]]`` ([HP] ``routed_x = x_flat[token_indices]``)."""
+    return as_f64(x)[_i64(src_row)]
+
+
+# --------------------------------------------------------------------------
+# Expert-parallel layout and local regroup ([EP] Ep2DpParallel._token_dispatch)
+# --------------------------------------------------------------------------
+
+def ep_dispatch_rank_major(idx, E: int, R: int):
+    """Layout of the routed copies as EP ranks would receive them.
+
+    Source rank ``r`` owns the contiguous token shard
+    ``[r*S, min(T, (r+1)*S))`` with ``S = ceil(T / R)`` and dispatches it into
+    its own expert-major order.  Destination block ``g`` owns the local
+    experts ``g*L .. g*L + L - 1`` (``L = E // R``); the all-to-all
+    concatenates, for every ``g``, source rank after source rank, the rows each
+    source holds for those experts (source rank outer, local expert inner).
+
+    Returns ``counts_rm[G, R, L]``, ``src_row[N]`` (token of every received
+    row), ``dst_pos[T, k]`` (received row of every copy).
+    """
+    idx = _i64(idx)
+    T, k = idx.shape
+    G = R
+    L = E // G
+    S = -(-T // R) if T else 0
+    counts_rm = np.zeros((G, R, L), dtype=np.int64)
+    src_row = []
+    dst_pos = np.full((T, k), -1, dtype=np.int64)
+    local = []
+    for r in range(R):
+        t0, t1 = min(T, r * S), min(T, (r + 1) * S)
+        c, off, srow, dpos = dispatch(idx[t0:t1], E)
+        local.append((t0, c, off, srow, dpos))
+    pos = 0
+    for g in range(G):
+        for r in range(R):
+            t0, c, off, srow, dpos = local[r]
+            for l in range(L):
+                e = g * L + l
+                counts_rm[g, r, l] = c[e]
+            lo, hi = off[g * L], off[(g + 1) * L]
+            # rows [lo, hi) of rank r's buffer land at [pos, pos + hi - lo)
+            src_row.append(srow[lo:hi] + t0)
+            sel = (dpos >= lo) & (dpos < hi)
+            tt, jj = np.nonzero(sel)
+            dst_pos[tt + t0, jj] = dpos[tt, jj] - lo + pos
+            pos += hi - lo
+    src_row = np.concatenate(src_row) if src_row else np.zeros(0, np.int64)
+    return counts_rm, src_row, dst_pos
+
+
+def ep_local_regroup(counts_rm):
+    """Regroup of a rank-major received buffer into expert-major order.
+
+    For each destination block ``g`` and local expert ``l``, the segments of
+    source ranks ``r = 0 .. R-1`` are appended in order.  Returns
+    ``perm[rows]`` (output row -> input row), ``counts_em[G*L]`` (summed over
+    source ranks) and ``offsets_em[G*L + 1]``.
+    """
+    c = _i64(counts_rm)
+    G, R, L = c.shape
+    in_off = np.zeros(G * R * L + 1, dtype=np.int64)
+    in_off[1:] = np.cumsum(c.ravel())              # (g, r, l) order
+    perm = []
+    for g in range(G):
+        for l in range(L):
+            for r in range(R):
+                s = (g * R + r) * L + l
+                perm.append(np.arange(in_off[s], in_off[s + 1]))
+    perm = np.concatenate(perm) if perm else np.zeros(0, np.int64)
+    counts_em = c.sum(axis=1).reshape(G * L)
+    offsets_em = np.zeros(G * L + 1, dtype=np.int64)
+    offsets_em[1:] = np.cumsum(counts_em)
+    return perm, counts_em, offsets_em
+
+
+def apply_row_perm(rows, perm) -> np.ndarray:
+    """``out[i] = rows[perm[i]]``."""
+    return np.asarray(rows)[_i64(perm)]
+
+
+# --------------------------------------------------------------------------
+# Experts ([HP] _run_experts_for_loop / FeedForward; [QO] training branch)
+# --------------------------------------------------------------------------
+
+def silu(z) -> np.ndarray:
+    """``silu(z) = z / (1 + exp(-z))``."""
+    z = as_f64(z)
+    with np.errstate(over="ignore"):
+        return z / (1.0 + np.exp(-z))
+
+
+def swiglu_ffn(S, w1e, w3e, w2e) -> np.ndarray:
+    """One expert: ``(silu(S w1^T) * (S w3^T)) w2^T`` with ``[out, in]``
+    weights ([HP] ``FeedForward.forward``)."""
+    S = as_f64(S)
+    A = silu(S @ as_f64(w1e).T) * (S @ as_f64(w3e).T)
+    return A @ as_f64(w2e).T
+
+
+def grouped_swiglu(x_perm, offsets, w1, w3, w2, row_scale=None) -> np.ndarray:
+    """Per-expert SwiGLU over expert-major segments ([HP]
+    ``_run_experts_for_loop``): experts with no rows are skipped; an optional
+    per-row ``row_scale`` multiplies the hidden activation before ``w2``.
+    Converts one expert's weights to fp64 at a time."""
+    xp = as_f64(x_perm)
+    off = _i64(offsets)
+    E = len(off) - 1
+    d = w2.shape[1]
+    y = np.zeros((xp.shape[0], d), dtype=np.float64)
+    rs = None if row_scale is None else as_f64(row_scale)
+    for e in range(E):
+        lo, hi = int(off[e]), int(off[e + 1])
+        if hi == lo:
+            continue
+        S = xp[lo:hi]
+        A = silu(S @ as_f64(w1[e]).T) * (S @ as_f64(w3[e]).T)
+        if rs is not None:
+            A = A * rs[lo:hi, None]
+        y[lo:hi] = A @ as_f64(w2[e]).T
+    return y
+
+
+# --------------------------------------------------------------------------
+# Combine ([QO] index_add_; [HP] MoE.unpermutation scatter_add)
+# --------------------------------------------------------------------------
+
+def combine(y, dst_pos, topk_w=None) -> np.ndarray:
+    """``out[t] = sum_j w[t, j] * y[dst_pos[t, j]]`` (``w = 1`` if None).
+
+    The sum over ``j`` is the scatter-add of every copy's output into its
+    token row.
+    """
+    y = as_f64(y)
+    dp = _i64(dst_pos)
+    T, k = dp.shape
+    out = np.zeros((T, y.shape[1]), dtype=np.float64)
+    w = np.ones((T, k)) if topk_w is None else as_f64(topk_w)
+    for j in range(k):
+        out += w[:, j:j + 1] * y[dp[:, j]]
+    return out
+
+
+# --------------------------------------------------------------------------
+# Whole layer ([HP] MoE.forward with score_before_experts=False)
+# --------------------------------------------------------------------------
+
+def moe_forward(x, w_router, w1, w3, w2, top_k: int, renormalize: bool = True,
+                logits=None, ep_ranks: int = 1):
+    """Router -> dispatch -> (EP regroup) -> grouped SwiGLU -> combine.
+
+    Returns a dict with every intermediate (fp64 / int64).  With
+    ``ep_ranks > 1`` the routed rows are first laid out as received by
+    ``ep_ranks`` simulated EP ranks and regrouped before the experts.
+    """
+    E = w1.shape[0]
+    idx, w, counts, L = router_topk(top_k, renormalize, x=x, w_router=w_router,
+                                    logits=logits)
+    res = {"logits": L, "topk_idx": idx, "topk_w": w}
+    if ep_ranks == 1:
+        c, off, src_row, dst_pos = dispatch(idx, E)
+        res.update(counts=c, offsets=off, src_row=src_row, dst_pos=dst_pos)
+        x_perm = permute_rows(x, src_row)
+        y = grouped_swiglu(x_perm, off, w1, w3, w2)
+        res.update(x_perm=x_perm, y=y, out=combine(y, dst_pos, w))
+        return res
+    counts_rm, src_rm, dst_rm = ep_dispatch_rank_major(idx, E, ep_ranks)
+    x_rm = permute_rows(x, src_rm)
+    perm, counts_em, off_em = ep_local_regroup(counts_rm)
+    x_em = apply_row_perm(x_rm, perm)
+    inv = np.empty_like(perm)
+    inv[perm] = np.arange(len(perm))
+    dst_em = inv[dst_rm]
+    y = grouped_swiglu(x_em, off_em, w1, w3, w2)
+    res.update(counts_rm=counts_rm, src_row_rm=src_rm, dst_pos_rm=dst_rm,
+               perm=perm, counts=counts_em, offsets=off_em, dst_pos=dst_em,
+               src_row=src_rm[perm], x_perm=x_em, y=y,
+               out=combine(y, dst_em, w))
+    return res
+
+
+def dense_moe(x, idx, w, w1, w3, w2) -> np.ndarray:
+    """Brute-force dense formulation ([QO] eval branch): every expert runs
+    on every token and the outputs are summed with the mask
+    ``M[t, e] = sum_j w[t, j] [idx[t, j] == e]``."""
+    x = as_f64(x)
+    idx = _i64(idx)
+    w = as_f64(w)
+    T = x.shape[0]
+    E = w1.shape[0]
+    M = np.zeros((T, E))
+    for j in range(idx.shape[1]):
+        np.add.at(M, (np.arange(T), idx[:, j]), w[:, j])
+    out = np.zeros((T, w2.shape[1]))
+    for e in range(E):
+        out += M[:, e:e + 1] * swiglu_ffn(x, w1[e], w3[e], w2[e])
+    return out
+
+
+def moe_tokens(x_rows, idx_rows, w_rows, w1, w3, w2) -> np.ndarray:
+    """Token-by-token definition for a sample of tokens:
+    ``out[t] = sum_j w[t, j] * FFN_{idx[t, j]}(x[t])``.  Used to check sampled
+    outputs of layers too large for the full oracle."""
+    x_rows = as_f64(x_rows)
+    idx_rows = _i64(idx_rows)
+    w_rows = as_f64(w_rows)
+    out = np.zeros((x_rows.shape[0], w2.shape[1]))
+    for t in range(x_rows.shape[0]):
+        for j in range(idx_rows.shape[1]):
+            e = int(idx_rows[t, j])
+            out[t] += w_rows[t, j] * swiglu_ffn(x_rows[t:t + 1], w1[e], w3[e], w2[e])[0]
+    return out
