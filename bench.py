@@ -1,0 +1,393 @@
+"""Benchmark of the MoE layer forward on B200 (one JSON line on rank 0).
+
+A step is one pass of the whole hot path over one batch of synthetic tokens
+resident in HBM: router top-k -> dispatch -> grouped SwiGLU -> combine, run
+through the C ABI (the four entry points moe_forward chains, each bracketed
+by CUDA events on the launching stream so the grouped-GEMM time is measured
+live).  L2 is flushed (256 MB write) between timed steps, outside the step's
+events.  ``value`` is tokens/s of the whole job (all ranks; ranks run
+independent token batches, weak scaling, no data-path collective).
+
+``--impl reference`` times the fp64 CPU oracle on the host cores instead
+(a bounded token sample per step) and prints the same metric.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "MoE-layer routed tokens/s (bf16); grouped-GEMM TFLOP/s as % of tensor peak"
+UNIT = "tokens/s"
+FLUSH_BYTES = 256 << 20
+LAUNCHES_PER_STEP = {"router": 1, "dispatch": 3, "grouped_swiglu": 2, "combine": 1}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.t:
+            self.t.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(n_gpus):
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v, ws):
+    if ws == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------- CPU oracle
+def cpu_oracle_step(cfg, lay_cpu, tokens):
+    """One oracle pass (router -> dispatch -> experts -> combine) on `tokens`
+    rows; returns wall seconds."""
+    import oracle as O
+    x = lay_cpu["x"][:tokens]
+    t0 = time.perf_counter()
+    O.moe_forward(x, lay_cpu["w_router"], lay_cpu["w1"], lay_cpu["w3"], lay_cpu["w2"],
+                  cfg.top_k, cfg.renormalize, ep_ranks=cfg.ep_ranks)
+    return time.perf_counter() - t0
+
+
+def cpu_layer(cfg, tokens):
+    lay = W.make_layer(cfg, "cpu", T=tokens)
+    return lay
+
+
+def cpu_baseline(cfg, tokens=256, reps=1):
+    lay = cpu_layer(cfg, tokens)
+    cpu_oracle_step(cfg, lay, min(tokens, 16))          # warm-up (BLAS init)
+    secs = [cpu_oracle_step(cfg, lay, tokens) for _ in range(reps)]
+    s = sum(secs)
+    return {"value": tokens * reps / s, "unit": UNIT, "cores": os.cpu_count(), "kind": "oracle",
+            "sample": f"{tokens} tokens of {cfg.name} per pass, {reps} pass(es), fp64 NumPy "
+                      f"(BLAS threads = all host cores), {s:.1f} s"}
+
+
+def run_reference(args, ws, rank):
+    """Reference arm: the fp64 CPU oracle, rank 0 only."""
+    if rank != 0:
+        return
+    cfg = W.config(args.config)
+    tokens = args.ref_tokens
+    lay = cpu_layer(cfg, tokens)
+    for _ in range(args.warmup):
+        cpu_oracle_step(cfg, lay, tokens)
+    secs = [cpu_oracle_step(cfg, lay, tokens) for _ in range(args.steps)]
+    total = sum(secs)
+    value = tokens * args.steps / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "E": cfg.E, "top_k": cfg.top_k,
+                   "h": cfg.h, "sample_tokens_per_step": tokens},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": os.cpu_count(), "kind": "oracle",
+                         "sample": f"{tokens} tokens of {cfg.name} per step"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------- GPU arm
+def run_ours(args, ws, rank, local):
+    import routing_dispatch_grouped_topk_b200 as M
+    M.lib()  # fails loudly if the CUDA library is missing
+    cfg = W.config(args.config)
+    T, d, E, k, h, R = cfg.T, cfg.d, cfg.E, cfg.top_k, cfg.h, cfg.ep_ranks
+    N = T * k
+    dev = torch.device("cuda", local)
+    lay = W.make_layer(cfg, dev)
+    if rank:   # independent token batch per rank
+        lay["x"] = W.make_layer(W.MoEConfig(**{**cfg.__dict__, "seed": cfg.seed + 1000 * rank}),
+                                dev, experts=False)["x"]
+    x, wr, w1, w3, w2 = lay["x"], lay["w_router"], lay["w1"], lay["w3"], lay["w2"]
+    dt = M.MOE_BF16 if cfg.dtype == "bf16" else M.MOE_F32
+    stream = torch.cuda.current_stream()
+
+    # buffers of the four stages (the same sequence moe_forward runs)
+    idx = torch.empty(T, k, dtype=torch.int32, device=dev)
+    w = torch.empty(T, k, dtype=torch.float32, device=dev)
+    rws = torch.empty(M.router_workspace_size(T, d, E, dt), dtype=torch.uint8, device=dev)
+    nb = E * R
+    counts = torch.empty(nb, dtype=torch.int32, device=dev)
+    offsets = torch.empty(nb + 1, dtype=torch.int32, device=dev)
+    src_row = torch.empty(N, dtype=torch.int32, device=dev)
+    dst_pos = torch.empty(T, k, dtype=torch.int32, device=dev)
+    x_perm = torch.empty(N, d, dtype=x.dtype, device=dev)
+    dws = torch.empty(M.ep_dispatch_workspace_size(T, E, k, R), dtype=torch.uint8, device=dev)
+    if R > 1:
+        x_em = torch.empty_like(x_perm)
+        cem = torch.empty(E, dtype=torch.int32, device=dev)
+        oem = torch.empty(E + 1, dtype=torch.int32, device=dev)
+        perm = torch.empty(N, dtype=torch.int32, device=dev)
+        pinv = torch.empty(N, dtype=torch.int32, device=dev)
+        gws = torch.empty(M.regroup_workspace_size(R, R, E // R), dtype=torch.uint8, device=dev)
+    y = torch.empty(N, d, dtype=x.dtype, device=dev)
+    sws = torch.empty(M.grouped_swiglu_workspace_size(N, d, h, E, dt), dtype=torch.uint8,
+                      device=dev)
+    out = torch.empty(T, d, dtype=x.dtype, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    stages = ["router", "dispatch"] + (["regroup"] if R > 1 else []) + ["grouped_swiglu",
+                                                                        "combine"]
+
+    def step(ev=None):
+        def mark(i):
+            if ev is not None:
+                ev[i].record(stream)
+        mark(0)
+        M.moe_router_topk(x, wr, None, T, d, E, k, M.MOE_SCORE_SOFTMAX, cfg.renormalize, dt, None,
+                          idx, w, None, rws)
+        mark(1)
+        if R == 1:
+            M.moe_dispatch(x, idx, T, d, E, k, dt, counts, offsets, src_row, dst_pos, x_perm, dws)
+        else:
+            M.moe_ep_dispatch_rank_major(x, idx, T, d, E, k, R, dt, counts, offsets, src_row,
+                                         dst_pos, x_perm, dws)
+        mark(2)
+        i = 2
+        xe, off, rmap = x_perm, offsets, None
+        if R > 1:
+            M.moe_ep_local_regroup(x_perm, counts, R, R, E // R, N, d, dt, x_em, cem, oem, perm,
+                                   pinv, gws)
+            i += 1
+            mark(i)
+            xe, off, rmap = x_em, oem, pinv
+        M.moe_grouped_swiglu(xe, off, w1, w3, w2, None, N, d, h, E, dt, y, sws)
+        mark(i + 1)
+        M.moe_combine(y, dst_pos, rmap, w, T, d, N, k, dt, out)
+        mark(i + 2)
+
+    nmarks = len(stages) + 1
+    for _ in range(args.warmup):
+        step()
+        flush.zero_()
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(local)
+    if rank == 0:
+        sampler.start()
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(nmarks)]
+              for _ in range(args.steps)]
+    barrier(ws)
+    torch.cuda.synchronize()
+    region0 = torch.cuda.Event(enable_timing=True)
+    region1 = torch.cuda.Event(enable_timing=True)
+    region0.record(stream)
+    for s in range(args.steps):
+        step(events[s])
+        flush.zero_()          # L2 flush between steps, outside the step's events
+    region1.record(stream)
+    torch.cuda.synchronize()
+    barrier(ws)
+    clocks = sampler.stop() if rank == 0 else None
+
+    per_stage = {n: [] for n in stages}
+    step_ms = []
+    for ev in events:
+        for i, n in enumerate(stages):
+            per_stage[n].append(ev[i].elapsed_time(ev[i + 1]))
+        step_ms.append(ev[0].elapsed_time(ev[-1]))
+    total_ms = sum(step_ms)
+    total_ms_max = max_over_ranks(total_ms, ws)
+    ms_per_step = total_ms_max / args.steps
+    value = T * ws * args.steps / (total_ms_max / 1e3)
+
+    # e2e: host buffers through the public moe_forward call, copies included
+    x_host = x.cpu().pin_memory()
+    out_host = torch.empty(T, d, dtype=x.dtype).pin_memory()
+    fws = torch.empty(M.forward_workspace_size(T, d, E, k, h, R, dt), dtype=torch.uint8,
+                      device=dev)
+    x_dev = torch.empty_like(x)
+    out_dev = torch.empty_like(out)
+
+    def e2e_step():
+        x_dev.copy_(x_host, non_blocking=True)
+        M.moe_forward(x_dev, wr, None, w1, w3, w2, T, d, E, k, h, M.MOE_SCORE_SOFTMAX,
+                      cfg.renormalize, R, dt, out_dev, None, None, None, None, fws)
+        out_host.copy_(out_dev, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+        flush.zero_()
+    torch.cuda.synchronize()
+    e2e_ms = []
+    barrier(ws)
+    for _ in range(args.steps):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        e2e_step()
+        b.record(stream)
+        flush.zero_()
+        e2e_ms.append((a, b))
+    torch.cuda.synchronize()
+    barrier(ws)
+    e2e_total = max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ms), ws)
+    e2e_value = T * ws * args.steps / (e2e_total / 1e3)
+    # the e2e output equals the device-resident step's output
+    e2e_match = bool(torch.equal(out_host.to(dev), out))
+
+    if rank != 0:
+        return
+    pk = peaks()
+    sw_ms = statistics.mean(per_stage["grouped_swiglu"])
+    flops = cfg.gemm_flops()
+    achieved = flops / (sw_ms / 1e3) / 1e12
+    peak = pk["bf16_tflops_sustained"]
+    stage_ms = {n: statistics.mean(v) for n, v in per_stage.items()}
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
+        "config": {"workload": cfg.name, "T": T, "d": d, "E": E, "top_k": k, "h": h,
+                   "ep_ranks": R, "global_batch": T * ws, "parallelism": f"dp{ws}",
+                   "l2": "flushed between steps (256 MB write, outside step events)",
+                   "inputs": "seeded synthetic, resident in HBM"},
+        "roofline": {"kernel": "moe_grouped_swiglu (GEMM1 w1|w3 + SiLU*up, GEMM2 w2)",
+                     "bound": "tensor", "achieved": achieved, "peak": peak,
+                     "peak_kind": f"bf16 sustained, {pk['source']}", "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "algorithmic_flops_per_launch": flops},
+        "stage_ms": stage_ms,
+        "copies_per_s": value * k,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": x.numel() * x.element_size(),
+                "d2h_bytes_per_step": out.numel() * out.element_size(),
+                "output_matches_device_step": e2e_match},
+        "gpu_launches": args.steps * (sum(LAUNCHES_PER_STEP.values()) + (2 if R > 1 else 0)),
+        "clocks": clocks,
+    }
+    if not args.no_cpu_baseline and ws == 1:
+        line["cpu_baseline"] = cpu_baseline(cfg, tokens=args.cpu_tokens)
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", type=int, default=1, help="workload index (default: the "
+                    "Qwen3-30B-A3B-shaped layer, T=4096)")
+    ap.add_argument("--cpu-tokens", type=int, default=256)
+    ap.add_argument("--ref-tokens", type=int, default=128)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        ws = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, ws, rank)
+        return
+    ws, rank, local = dist_setup(args.gpus)
+    try:
+        run_ours(args, ws, rank, local)
+    finally:
+        if ws > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

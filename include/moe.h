@@ -1,0 +1,256 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) MoE layer forward library (libmoe.so).
+ *
+ * The library computes the single-device forward of a token-choice top-k
+ * mixture-of-experts layer with SwiGLU experts:
+ *
+ *   router (fp32 logits, softmax, top-k, optional renormalisation)
+ *   -> dispatch of the routed copies into expert-major order
+ *   -> [expert-parallel local regroup of a rank-major buffer]
+ *   -> grouped SwiGLU  y = (silu(x w1^T) * (x w3^T)) w2^T  per expert segment
+ *   -> weighted combine (scatter-add of every copy back to its token).
+ *
+ * Sources, by page and section:
+ *   [HP] hyper_parallel platform/torch/common/moe.py coverage page:
+ *        TokenChoiceTopKRouter.forward, MoE.permutation, MoE.unpermutation,
+ *        _run_experts_for_loop, _run_experts_grouped_mm_gpu, GroupedExperts,
+ *        MoE.forward.
+ *   [QO] QwenLM/Qwen3-Omni issue #115: SpeedupMoeExperts.forward (training
+ *        branch with index_add_), SpeedupMoeSparseMoeBlock.forward
+ *        (norm_topk_prob renormalisation).
+ *   [EP] huggingface/transformers PR #41053 "Qwen3 moe":
+ *        Ep2DpParallel._token_dispatch (rank-major received buffer that has to
+ *        be reshuffled back into expert order).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Ownership: every array argument is a DEVICE pointer owned by the caller,
+ *   except where a comment says "host".  The library keeps no state between
+ *   calls and allocates no device memory; scratch space is the caller's
+ *   workspace `ws` of at least the size the matching *_workspace_size()
+ *   returns (256-byte aligned).
+ * Layout: row-major, contiguous.  `dt` is the element type of x, the expert
+ *   weights, x_perm, the hidden activation, y and out.  Router logits and
+ *   routing weights are always fp32; indices and counts are int32.
+ * Streams: `stream` is a cudaStream_t (NULL = legacy default stream).  All
+ *   work is asynchronous on it and no entry point synchronises the host,
+ *   except moe_get_device_status.
+ * Errors: arguments are checked on the host before anything is launched;
+ *   a bad argument returns MOE_ERR_INVALID_ARG and launches nothing.  Shapes
+ *   the sm_100a kernels do not cover return MOE_ERR_UNSUPPORTED (there is no
+ *   CPU fallback).  A failed launch returns MOE_ERR_CUDA.  Bad *data* found
+ *   on the device (an expert id outside [0,E), regroup counts that do not sum
+ *   to the row count, offsets that are not a valid segmentation, a pipeline
+ *   wait that ran out of time) never traps: the kernels skip the offending
+ *   element, keep every access in bounds and OR a MOE_DEV_* bit into the
+ *   status word at the start of the workspace.  Each entry point that takes
+ *   `ws` clears that word when it starts; read it with
+ *   moe_get_device_status.  moe_last_error() describes the last host-side
+ *   error of the calling thread.
+ * Empty inputs: T == 0 (or N == 0) is a valid no-op that still writes the
+ *   zero counts / offsets it is asked for.
+ */
+#ifndef MOE_B200_MOE_H
+#define MOE_B200_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,
+  MOE_ERR_UNSUPPORTED = 2,
+  MOE_ERR_CUDA = 3,
+  MOE_ERR_WORKSPACE = 4,
+  MOE_ERR_DEVICE = 5
+} moe_status_t;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype_t;
+
+/* Score function of the router.  Only softmax is defined by the layers this
+ * library targets ([HP] TokenChoiceTopKRouter with score_func="softmax",
+ * [QO] SpeedupMoeSparseMoeBlock).  Other values return MOE_ERR_UNSUPPORTED. */
+typedef enum { MOE_SCORE_SOFTMAX = 0 } moe_score_t;
+
+/* Bits of the device status word. */
+#define MOE_DEV_BAD_EXPERT 1   /* dispatch: expert id outside [0, E)            */
+#define MOE_DEV_BAD_COUNTS 2   /* regroup: counts negative or not summing to rows */
+#define MOE_DEV_BAD_OFFSETS 4  /* grouped_swiglu: offsets not 0..N non-decreasing */
+#define MOE_DEV_TIMEOUT 8      /* a pipeline wait exceeded its time limit        */
+
+/* Limits of this build. */
+#define MOE_MAX_EXPERTS 512
+#define MOE_MAX_TOPK 16
+
+/* ------------------------------------------------------------------------
+ * moe_router_topk -- [HP] TokenChoiceTopKRouter.forward, softmax branch;
+ * [QO] SpeedupMoeSparseMoeBlock.forward (norm_topk_prob).
+ *
+ *   scores  = logits_in            if logits_in != NULL
+ *           = x @ w_router^T (fp32 accumulation, no rounding of the logits)
+ *   p       = softmax(scores) over all E experts
+ *   topk_idx[t, 0..k-1] = the k largest scores, largest first; equal scores
+ *             go to the lower expert index (selection is made on the fp32
+ *             scores; softmax is increasing so this is the top-k of p)
+ *   topk_w[t, j] = p[t, topk_idx[t, j]], divided by their sum over j when
+ *             renormalize != 0
+ *   counts[e] = number of (t, j) with topk_idx[t, j] == e
+ *
+ * x        [T, d]  dt, may be NULL when logits_in is given
+ * w_router [E, d]  dt (the bias-free gate nn.Linear(d, E) weight)
+ * logits_in  [T, E] fp32 or NULL
+ * logits_out [T, E] fp32 or NULL (written when the GEMM runs)
+ * topk_idx [T, k] int32, topk_w [T, k] fp32, counts [E] int32 or NULL.
+ * NaN scores are treated as -inf for the selection.
+ * Requires 1 <= top_k <= min(E, 16), E <= 512, d % 8 == 0 for bf16 (whole
+ * 16-byte rows), 16-byte aligned x / w_router.
+ * ---------------------------------------------------------------------- */
+MOE_API size_t moe_router_workspace_size(int T, int d, int E, moe_dtype_t dt);
+MOE_API moe_status_t moe_router_topk(const void* x, const void* w_router, const float* logits_in,
+                             int T, int d, int E, int top_k, moe_score_t score,
+                             int renormalize, moe_dtype_t dt, float* logits_out,
+                             int32_t* topk_idx, float* topk_w, int32_t* counts,
+                             void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * moe_dispatch -- [HP] MoE.permutation (stable argsort of the flat expert
+ * ids, bincount) and the gather routed_x = x_flat[token_indices].
+ *
+ * With f = t*k + j the flat index of copy (t, j):
+ *   counts[e]    = #{f : topk_idx[f] == e}
+ *   offsets[e]   = sum_{e' < e} counts[e'],  offsets[E] = T*k
+ *   dst_pos[t,j] = offsets[e] + #{f' < f : topk_idx[f'] == e}   (slot of the copy)
+ *   src_row[s]   = t for the copy in slot s
+ *   x_perm[s, :] = x[src_row[s], :]   (skipped when x_perm == NULL)
+ * The order inside an expert segment is increasing f, so the result is
+ * unique and bit-exact.  topk_idx [T, k] int32; counts [E]; offsets [E+1];
+ * src_row [T*k]; dst_pos [T, k]; x [T, d] and x_perm [T*k, d] dt.
+ * Ids outside [0, E) set MOE_DEV_BAD_EXPERT; such copies get dst_pos = -1,
+ * take no slot, and the unused tail slots of src_row are -1.
+ * ---------------------------------------------------------------------- */
+MOE_API size_t moe_dispatch_workspace_size(int T, int E, int top_k);
+MOE_API moe_status_t moe_dispatch(const void* x, const int32_t* topk_idx, int T, int d, int E,
+                          int top_k, moe_dtype_t dt, int32_t* counts, int32_t* offsets,
+                          int32_t* src_row, int32_t* dst_pos, void* x_perm, void* ws,
+                          size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * moe_ep_dispatch_rank_major -- the layout in which R expert-parallel ranks
+ * receive the routed copies ([EP] Ep2DpParallel._token_dispatch): source
+ * rank r owns tokens [r*S, min(T, (r+1)*S)), S = ceil(T/R), and destination
+ * rank g owns experts [g*L, (g+1)*L), L = E / R.  The buffer lists, for
+ * g = 0..R-1, for r = 0..R-1, for l = 0..L-1, the copies of source r for
+ * expert g*L + l in increasing flat index.  Produced on one GPU as if after
+ * the all-to-all (no communication).
+ *   counts_rm [R, R, L] (indexed [g][r][l]); offsets_rm [R*R*L + 1];
+ *   src_row [T*k]; dst_pos [T, k]; x_rm [T*k, d] or NULL.
+ * Requires E % R == 0 and E*R <= 8192.  Other rules as moe_dispatch.
+ * ---------------------------------------------------------------------- */
+MOE_API size_t moe_ep_dispatch_workspace_size(int T, int E, int top_k, int R);
+MOE_API moe_status_t moe_ep_dispatch_rank_major(const void* x, const int32_t* topk_idx, int T, int d,
+                                        int E, int top_k, int R, moe_dtype_t dt,
+                                        int32_t* counts_rm, int32_t* offsets_rm,
+                                        int32_t* src_row, int32_t* dst_pos, void* x_rm,
+                                        void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * moe_ep_local_regroup -- [EP] Ep2DpParallel._token_dispatch: the received
+ * buffer "is not sorted by expert anymore" and "needs to be reshuffled back".
+ *
+ * in [rows, d] holds, for each destination block g, segments (r, l) in
+ * source-rank-major order (r outer, l inner) of counts_rm[g][r][l] rows.
+ * out [rows, d] holds the same rows local-expert-major (l outer, r inner):
+ *   for g, for l, for r: segment (g, r, l)
+ * perm [rows]: out row -> in row.  counts_em [G*L] = sum_r counts_rm[g][r][l];
+ * offsets_em [G*L + 1].  perm_inv [rows] (in row -> out row) or NULL.
+ * counts_rm [G, R, L] int32 device array.  If the counts are negative or do
+ * not sum to rows, MOE_DEV_BAD_COUNTS is set and nothing is copied.
+ * G*R*L <= 8192.
+ * ---------------------------------------------------------------------- */
+MOE_API size_t moe_regroup_workspace_size(int G, int R, int L);
+MOE_API moe_status_t moe_ep_local_regroup(const void* in, const int32_t* counts_rm, int G, int R,
+                                  int L, int rows, int d, moe_dtype_t dt, void* out,
+                                  int32_t* counts_em, int32_t* offsets_em, int32_t* perm,
+                                  int32_t* perm_inv, void* ws, size_t ws_bytes,
+                                  void* stream);
+
+/* ------------------------------------------------------------------------
+ * moe_grouped_swiglu -- [HP] _run_experts_for_loop / _run_experts_grouped_mm_gpu
+ * (GroupedExperts weights [E, out, in]).
+ *
+ * For every expert e with rows s in [offsets[e], offsets[e+1]):
+ *   H[s] = silu(x_perm[s] . w1[e]^T) * (x_perm[s] . w3[e]^T)      (fp32 acc)
+ *   y[s] = (H[s] . w2[e]^T) * (row_scale ? row_scale[s] : 1)        (fp32 acc)
+ * bf16: H is rounded to bf16 once (it is the GEMM2 operand), y once.
+ * fp32: everything in fp32.  Experts with no rows are skipped.
+ * x_perm [N, d]; offsets [E+1] int32 (device); w1, w3 [E, h, d]; w2 [E, d, h];
+ * row_scale [N] fp32 or NULL; y [N, d].
+ * bf16 requires d % 64 == 0 and h % 64 == 0 (tcgen05 path); fp32 requires
+ * d % 4 == 0 and h % 4 == 0.
+ * ---------------------------------------------------------------------- */
+MOE_API size_t moe_grouped_swiglu_workspace_size(int N, int d, int h, int E, moe_dtype_t dt);
+MOE_API moe_status_t moe_grouped_swiglu(const void* x_perm, const int32_t* offsets, const void* w1,
+                                const void* w3, const void* w2, const float* row_scale,
+                                int N, int d, int h, int E, moe_dtype_t dt, void* y,
+                                void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * moe_combine -- [QO] SpeedupMoeExperts.forward training branch
+ * (weighted index_add_); [HP] MoE.unpermutation (scatter_add).
+ *
+ *   out[t, :] = sum_{j=0..k-1} w[t, j] * y[r(t, j), :]
+ *   r(t, j)   = row_map ? row_map[dst_pos[t, j]] : dst_pos[t, j]
+ *   w         = topk_w (fp32) or 1 when topk_w == NULL
+ * Accumulated in fp32 over j = 0..k-1 in order, rounded once to dt.
+ * y [N, d]; dst_pos [T, k]; row_map [N] or NULL; out [T, d].  Positions
+ * outside [0, N) (e.g. -1 from a bad expert id) contribute nothing.
+ * ---------------------------------------------------------------------- */
+MOE_API moe_status_t moe_combine(const void* y, const int32_t* dst_pos, const int32_t* row_map,
+                         const float* topk_w, int T, int d, int N, int top_k,
+                         moe_dtype_t dt, void* out, void* stream);
+
+/* ------------------------------------------------------------------------
+ * moe_forward -- [HP] MoE.forward with score_before_experts=False and no
+ * shared expert: router -> dispatch -> grouped SwiGLU -> combine.
+ * With ep_ranks R > 1 the routed rows are laid out as R simulated EP ranks
+ * would receive them (moe_ep_dispatch_rank_major), regrouped
+ * (moe_ep_local_regroup) and then run through the experts; the result is
+ * the same function.  out [T, d]; topk_idx/topk_w/counts/logits_out are
+ * optional copies of the router outputs.
+ * ---------------------------------------------------------------------- */
+MOE_API size_t moe_forward_workspace_size(int T, int d, int E, int top_k, int h, int ep_ranks,
+                                  moe_dtype_t dt);
+MOE_API moe_status_t moe_forward(const void* x, const void* w_router, const float* logits_in,
+                         const void* w1, const void* w3, const void* w2, int T, int d, int E,
+                         int top_k, int h, moe_score_t score, int renormalize, int ep_ranks,
+                         moe_dtype_t dt, void* out, float* logits_out, int32_t* topk_idx,
+                         float* topk_w, int32_t* counts, void* ws, size_t ws_bytes,
+                         void* stream);
+
+/* Synchronises `stream`, then copies the status word at the start of `ws`
+ * into *code (host).  Returns MOE_ERR_CUDA if the copy fails. */
+MOE_API moe_status_t moe_get_device_status(const void* ws, int* code, void* stream);
+
+/* Static description of a status code (never NULL). */
+MOE_API const char* moe_status_string(moe_status_t s);
+
+/* Text of the last host-side error raised on the calling thread ("" if none). */
+MOE_API const char* moe_last_error(void);
+
+/* Library version as major*10000 + minor*100 + patch. */
+MOE_API int moe_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_B200_MOE_H */

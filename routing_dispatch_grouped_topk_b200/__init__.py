@@ -1,0 +1,368 @@
+"""B200 (sm_100a) MoE layer forward: thin Python binding of libmoe.so.
+
+Every step of the layer (router, dispatch, EP regroup, grouped SwiGLU,
+combine) runs in the CUDA kernels of ``libmoe.so``; this module only
+marshals torch tensors into the C ABI of ``include/moe.h`` (pointers, sizes,
+the current CUDA stream) and raises on a non-zero status.  There is no CPU
+fallback: importing the binding without the built library raises.
+
+Two layers of API:
+
+* ``moe_router_topk``, ``moe_dispatch``, ``moe_ep_dispatch_rank_major``,
+  ``moe_ep_local_regroup``, ``moe_grouped_swiglu``, ``moe_combine``,
+  ``moe_forward`` -- same names and argument order as the C functions, with
+  torch tensors (or None) in place of pointers; outputs are caller-allocated.
+* ``router_topk``, ``dispatch``, ``ep_dispatch_rank_major``,
+  ``ep_local_regroup``, ``grouped_swiglu``, ``combine``, ``forward`` --
+  allocate their outputs and workspace with torch and return them.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+__all__ = [
+    "MoEError", "lib", "LIB_PATH", "MOE_F32", "MOE_BF16", "MOE_SCORE_SOFTMAX",
+    "MOE_DEV_BAD_EXPERT", "MOE_DEV_BAD_COUNTS", "MOE_DEV_BAD_OFFSETS", "MOE_DEV_TIMEOUT",
+    "EXPORTED_SYMBOLS",
+    "moe_router_topk", "moe_dispatch", "moe_ep_dispatch_rank_major", "moe_ep_local_regroup",
+    "moe_grouped_swiglu", "moe_combine", "moe_forward", "moe_get_device_status",
+    "router_workspace_size", "dispatch_workspace_size", "ep_dispatch_workspace_size",
+    "regroup_workspace_size", "grouped_swiglu_workspace_size", "forward_workspace_size",
+    "router_topk", "dispatch", "ep_dispatch_rank_major", "ep_local_regroup",
+    "grouped_swiglu", "combine", "forward", "device_status",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe.so")
+
+MOE_F32, MOE_BF16 = 0, 1
+MOE_SCORE_SOFTMAX = 0
+MOE_DEV_BAD_EXPERT, MOE_DEV_BAD_COUNTS, MOE_DEV_BAD_OFFSETS, MOE_DEV_TIMEOUT = 1, 2, 4, 8
+
+EXPORTED_SYMBOLS = [
+    "moe_router_workspace_size", "moe_router_topk",
+    "moe_dispatch_workspace_size", "moe_dispatch",
+    "moe_ep_dispatch_workspace_size", "moe_ep_dispatch_rank_major",
+    "moe_regroup_workspace_size", "moe_ep_local_regroup",
+    "moe_grouped_swiglu_workspace_size", "moe_grouped_swiglu",
+    "moe_combine",
+    "moe_forward_workspace_size", "moe_forward",
+    "moe_get_device_status", "moe_status_string", "moe_last_error", "moe_version",
+]
+
+
+class MoEError(RuntimeError):
+    pass
+
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_Z = ctypes.c_size_t
+_SIGS = {
+    "moe_router_workspace_size": (_Z, [_I, _I, _I, _I]),
+    "moe_router_topk": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _Z, _P]),
+    "moe_dispatch_workspace_size": (_Z, [_I, _I, _I]),
+    "moe_dispatch": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _Z, _P]),
+    "moe_ep_dispatch_workspace_size": (_Z, [_I, _I, _I, _I]),
+    "moe_ep_dispatch_rank_major": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P,
+                                        _Z, _P]),
+    "moe_regroup_workspace_size": (_Z, [_I, _I, _I]),
+    "moe_ep_local_regroup": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _Z,
+                                  _P]),
+    "moe_grouped_swiglu_workspace_size": (_Z, [_I, _I, _I, _I, _I]),
+    "moe_grouped_swiglu": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _Z, _P]),
+    "moe_combine": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P]),
+    "moe_forward_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I, _I]),
+    "moe_forward": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P,
+                         _P, _P, _P, _Z, _P]),
+    "moe_get_device_status": (_I, [_P, ctypes.POINTER(_I), _P]),
+    "moe_status_string": (ctypes.c_char_p, [_I]),
+    "moe_last_error": (ctypes.c_char_p, []),
+    "moe_version": (_I, []),
+}
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libmoe.so.  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise MoEError(
+                f"{LIB_PATH} is missing: build it with "
+                "`python -m routing_dispatch_grouped_topk_b200.build` (there is no CPU fallback)")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+# ------------------------------------------------------------------ helpers
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return MOE_BF16
+    if t.dtype == torch.float32:
+        return MOE_F32
+    raise MoEError(f"unsupported dtype {t.dtype}")
+
+
+def _ptr(t: Optional[torch.Tensor], dtype=None, name="tensor") -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise MoEError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise MoEError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise MoEError(f"{name} must be {dtype}, got {t.dtype}")
+    return t.data_ptr() or None
+
+
+def _stream(stream=None) -> Optional[int]:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream or None
+
+
+def _check(code: int, fn: str):
+    if code != 0:
+        L = lib()
+        msg = L.moe_last_error().decode()
+        raise MoEError(f"{fn}: {L.moe_status_string(code).decode()} ({msg})")
+
+
+def _nbytes(t: Optional[torch.Tensor]) -> int:
+    return 0 if t is None else t.numel() * t.element_size()
+
+
+def _ws(nbytes: int, device) -> torch.Tensor:
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+# ------------------------------------------------------ C-ABI mirror (1:1)
+def router_workspace_size(T, d, E, dt) -> int:
+    return lib().moe_router_workspace_size(T, d, E, dt)
+
+
+def dispatch_workspace_size(T, E, top_k) -> int:
+    return lib().moe_dispatch_workspace_size(T, E, top_k)
+
+
+def ep_dispatch_workspace_size(T, E, top_k, R) -> int:
+    return lib().moe_ep_dispatch_workspace_size(T, E, top_k, R)
+
+
+def regroup_workspace_size(G, R, L) -> int:
+    return lib().moe_regroup_workspace_size(G, R, L)
+
+
+def grouped_swiglu_workspace_size(N, d, h, E, dt) -> int:
+    return lib().moe_grouped_swiglu_workspace_size(N, d, h, E, dt)
+
+
+def forward_workspace_size(T, d, E, top_k, h, ep_ranks, dt) -> int:
+    return lib().moe_forward_workspace_size(T, d, E, top_k, h, ep_ranks, dt)
+
+
+def moe_router_topk(x, w_router, logits_in, T, d, E, top_k, score, renormalize, dt, logits_out,
+                    topk_idx, topk_w, counts, ws, stream=None):
+    _check(lib().moe_router_topk(
+        _ptr(x, name="x"), _ptr(w_router, name="w_router"),
+        _ptr(logits_in, torch.float32, "logits_in"), T, d, E, top_k, score, int(renormalize), dt,
+        _ptr(logits_out, torch.float32, "logits_out"), _ptr(topk_idx, torch.int32, "topk_idx"),
+        _ptr(topk_w, torch.float32, "topk_w"), _ptr(counts, torch.int32, "counts"),
+        _ptr(ws, name="ws"), _nbytes(ws), _stream(stream)), "moe_router_topk")
+
+
+def moe_dispatch(x, topk_idx, T, d, E, top_k, dt, counts, offsets, src_row, dst_pos, x_perm, ws,
+                 stream=None):
+    _check(lib().moe_dispatch(
+        _ptr(x, name="x"), _ptr(topk_idx, torch.int32, "topk_idx"), T, d, E, top_k, dt,
+        _ptr(counts, torch.int32, "counts"), _ptr(offsets, torch.int32, "offsets"),
+        _ptr(src_row, torch.int32, "src_row"), _ptr(dst_pos, torch.int32, "dst_pos"),
+        _ptr(x_perm, name="x_perm"), _ptr(ws, name="ws"), _nbytes(ws), _stream(stream)),
+        "moe_dispatch")
+
+
+def moe_ep_dispatch_rank_major(x, topk_idx, T, d, E, top_k, R, dt, counts_rm, offsets_rm,
+                               src_row, dst_pos, x_rm, ws, stream=None):
+    _check(lib().moe_ep_dispatch_rank_major(
+        _ptr(x, name="x"), _ptr(topk_idx, torch.int32, "topk_idx"), T, d, E, top_k, R, dt,
+        _ptr(counts_rm, torch.int32, "counts_rm"), _ptr(offsets_rm, torch.int32, "offsets_rm"),
+        _ptr(src_row, torch.int32, "src_row"), _ptr(dst_pos, torch.int32, "dst_pos"),
+        _ptr(x_rm, name="x_rm"), _ptr(ws, name="ws"), _nbytes(ws), _stream(stream)),
+        "moe_ep_dispatch_rank_major")
+
+
+def moe_ep_local_regroup(inp, counts_rm, G, R, L, rows, d, dt, out, counts_em, offsets_em, perm,
+                         perm_inv, ws, stream=None):
+    _check(lib().moe_ep_local_regroup(
+        _ptr(inp, name="in"), _ptr(counts_rm, torch.int32, "counts_rm"), G, R, L, rows, d, dt,
+        _ptr(out, name="out"), _ptr(counts_em, torch.int32, "counts_em"),
+        _ptr(offsets_em, torch.int32, "offsets_em"), _ptr(perm, torch.int32, "perm"),
+        _ptr(perm_inv, torch.int32, "perm_inv"), _ptr(ws, name="ws"), _nbytes(ws),
+        _stream(stream)), "moe_ep_local_regroup")
+
+
+def moe_grouped_swiglu(x_perm, offsets, w1, w3, w2, row_scale, N, d, h, E, dt, y, ws,
+                       stream=None):
+    _check(lib().moe_grouped_swiglu(
+        _ptr(x_perm, name="x_perm"), _ptr(offsets, torch.int32, "offsets"), _ptr(w1, name="w1"),
+        _ptr(w3, name="w3"), _ptr(w2, name="w2"), _ptr(row_scale, torch.float32, "row_scale"),
+        N, d, h, E, dt, _ptr(y, name="y"), _ptr(ws, name="ws"), _nbytes(ws), _stream(stream)),
+        "moe_grouped_swiglu")
+
+
+def moe_combine(y, dst_pos, row_map, topk_w, T, d, N, top_k, dt, out, stream=None):
+    _check(lib().moe_combine(
+        _ptr(y, name="y"), _ptr(dst_pos, torch.int32, "dst_pos"),
+        _ptr(row_map, torch.int32, "row_map"), _ptr(topk_w, torch.float32, "topk_w"), T, d, N,
+        top_k, dt, _ptr(out, name="out"), _stream(stream)), "moe_combine")
+
+
+def moe_forward(x, w_router, logits_in, w1, w3, w2, T, d, E, top_k, h, score, renormalize,
+                ep_ranks, dt, out, logits_out, topk_idx, topk_w, counts, ws, stream=None):
+    _check(lib().moe_forward(
+        _ptr(x, name="x"), _ptr(w_router, name="w_router"),
+        _ptr(logits_in, torch.float32, "logits_in"), _ptr(w1, name="w1"), _ptr(w3, name="w3"),
+        _ptr(w2, name="w2"), T, d, E, top_k, h, score, int(renormalize), ep_ranks, dt,
+        _ptr(out, name="out"), _ptr(logits_out, torch.float32, "logits_out"),
+        _ptr(topk_idx, torch.int32, "topk_idx"), _ptr(topk_w, torch.float32, "topk_w"),
+        _ptr(counts, torch.int32, "counts"), _ptr(ws, name="ws"), _nbytes(ws), _stream(stream)),
+        "moe_forward")
+
+
+def moe_get_device_status(ws, stream=None) -> int:
+    code = _I(0)
+    _check(lib().moe_get_device_status(_ptr(ws, name="ws"), ctypes.byref(code), _stream(stream)),
+           "moe_get_device_status")
+    return code.value
+
+
+device_status = moe_get_device_status
+
+
+# --------------------------------------------------- allocating wrappers
+def router_topk(x=None, w_router=None, top_k=1, renormalize=True, logits_in=None,
+                want_logits=False, E=None):
+    """Returns (topk_idx int32 [T,k], topk_w fp32 [T,k], counts int32 [E],
+    logits fp32 [T,E] or None, ws)."""
+    src = logits_in if logits_in is not None else x
+    dev = src.device
+    if logits_in is not None:
+        T, E = logits_in.shape
+        d = x.shape[1] if x is not None else 8
+        dt = _dt(x) if x is not None else MOE_BF16
+    else:
+        T, d = x.shape
+        E = w_router.shape[0]
+        dt = _dt(x)
+    idx = torch.empty(T, top_k, dtype=torch.int32, device=dev)
+    w = torch.empty(T, top_k, dtype=torch.float32, device=dev)
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    logits = torch.empty(T, E, dtype=torch.float32, device=dev) if (
+        want_logits and logits_in is None) else None
+    ws = _ws(router_workspace_size(T, d, E, dt), dev)
+    moe_router_topk(x, w_router, logits_in, T, d, E, top_k, MOE_SCORE_SOFTMAX, renormalize, dt,
+                    logits, idx, w, counts, ws)
+    return idx, w, counts, logits, ws
+
+
+def dispatch(x, topk_idx, E, materialize=True):
+    """Returns (counts [E], offsets [E+1], src_row [N], dst_pos [T,k], x_perm [N,d] or None, ws)."""
+    T, k = topk_idx.shape
+    d = x.shape[1]
+    dev = topk_idx.device
+    N = T * k
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    src_row = torch.empty(N, dtype=torch.int32, device=dev)
+    dst_pos = torch.empty(T, k, dtype=torch.int32, device=dev)
+    x_perm = torch.empty(N, d, dtype=x.dtype, device=dev) if materialize else None
+    ws = _ws(dispatch_workspace_size(T, E, k), dev)
+    moe_dispatch(x, topk_idx, T, d, E, k, _dt(x), counts, offsets, src_row, dst_pos, x_perm, ws)
+    return counts, offsets, src_row, dst_pos, x_perm, ws
+
+
+def ep_dispatch_rank_major(x, topk_idx, E, R, materialize=True):
+    """Returns (counts_rm [R,R,E/R], offsets_rm, src_row, dst_pos, x_rm or None, ws)."""
+    T, k = topk_idx.shape
+    d = x.shape[1]
+    dev = topk_idx.device
+    N = T * k
+    counts = torch.empty(R, R, E // R, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E * R + 1, dtype=torch.int32, device=dev)
+    src_row = torch.empty(N, dtype=torch.int32, device=dev)
+    dst_pos = torch.empty(T, k, dtype=torch.int32, device=dev)
+    x_rm = torch.empty(N, d, dtype=x.dtype, device=dev) if materialize else None
+    ws = _ws(ep_dispatch_workspace_size(T, E, k, R), dev)
+    moe_ep_dispatch_rank_major(x, topk_idx, T, d, E, k, R, _dt(x), counts, offsets, src_row,
+                               dst_pos, x_rm, ws)
+    return counts, offsets, src_row, dst_pos, x_rm, ws
+
+
+def ep_local_regroup(inp, counts_rm):
+    """Returns (out [rows,d], counts_em [G*L], offsets_em [G*L+1], perm, perm_inv, ws)."""
+    G, R, L = counts_rm.shape
+    rows, d = inp.shape
+    dev = inp.device
+    out = torch.empty_like(inp)
+    counts_em = torch.empty(G * L, dtype=torch.int32, device=dev)
+    offsets_em = torch.empty(G * L + 1, dtype=torch.int32, device=dev)
+    perm = torch.empty(rows, dtype=torch.int32, device=dev)
+    perm_inv = torch.empty(rows, dtype=torch.int32, device=dev)
+    ws = _ws(regroup_workspace_size(G, R, L), dev)
+    moe_ep_local_regroup(inp, counts_rm, G, R, L, rows, d, _dt(inp), out, counts_em, offsets_em,
+                         perm, perm_inv, ws)
+    return out, counts_em, offsets_em, perm, perm_inv, ws
+
+
+def grouped_swiglu(x_perm, offsets, w1, w3, w2, row_scale=None):
+    """Returns (y [N,d], ws)."""
+    N, d = x_perm.shape
+    E, h, _ = w1.shape
+    y = torch.empty(N, d, dtype=x_perm.dtype, device=x_perm.device)
+    ws = _ws(grouped_swiglu_workspace_size(N, d, h, E, _dt(x_perm)), x_perm.device)
+    moe_grouped_swiglu(x_perm, offsets, w1, w3, w2, row_scale, N, d, h, E, _dt(x_perm), y, ws)
+    return y, ws
+
+
+def combine(y, dst_pos, topk_w=None, row_map=None):
+    T, k = dst_pos.shape
+    N, d = y.shape
+    out = torch.empty(T, d, dtype=y.dtype, device=y.device)
+    moe_combine(y, dst_pos, row_map, topk_w, T, d, N, k, _dt(y), out)
+    return out
+
+
+def forward(x, w_router, w1, w3, w2, top_k, renormalize=True, ep_ranks=1, logits_in=None,
+            want_router=False, ws=None, out=None):
+    """Whole layer.  Returns ``out`` ([T, d], x's dtype), or with
+    ``want_router`` a dict with out, topk_idx, topk_w, counts, logits, ws."""
+    T, d = x.shape
+    E, h, _ = w1.shape
+    dt = _dt(x)
+    dev = x.device
+    need = forward_workspace_size(T, d, E, top_k, h, ep_ranks, dt)
+    if ws is None or _nbytes(ws) < need:
+        ws = _ws(need, dev)
+    if out is None:
+        out = torch.empty(T, d, dtype=x.dtype, device=dev)
+    idx = w = counts = logits = None
+    if want_router:
+        idx = torch.empty(T, top_k, dtype=torch.int32, device=dev)
+        w = torch.empty(T, top_k, dtype=torch.float32, device=dev)
+        counts = torch.empty(E, dtype=torch.int32, device=dev)
+        logits = torch.empty(T, E, dtype=torch.float32, device=dev) if logits_in is None else None
+    moe_forward(x, w_router, logits_in, w1, w3, w2, T, d, E, top_k, h, MOE_SCORE_SOFTMAX,
+                renormalize, ep_ranks, dt, out, logits, idx, w, counts, ws)
+    if want_router:
+        return {"out": out, "topk_idx": idx, "topk_w": w, "counts": counts, "logits": logits,
+                "ws": ws}
+    return out

@@ -1,0 +1,500 @@
+// C ABI of libmoe (include/moe.h): host-side argument checks, workspace
+// layout and the launch sequence of every entry point.  Nothing here
+// computes on the host: every step of the layer runs in the kernels.
+#include <stdarg.h>
+#include <stdio.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+static thread_local char g_err[512] = "";
+
+void set_last_error(const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+}
+
+int num_sms() {
+  static int cache[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64) {
+    if (!cache[dev]) {
+      int n = 0;
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+      cache[dev] = n > 0 ? n : 1;
+    }
+    return cache[dev];
+  }
+  int n = 0;
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 1;
+}
+
+namespace {
+
+constexpr size_t kStatusBytes = 256;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+size_t elt_bytes(moe_dtype_t dt) { return dt == MOE_BF16 ? 2 : 4; }
+
+#define MOE_CHECK_ARG(cond, ...)            \
+  do {                                      \
+    if (!(cond)) {                          \
+      set_last_error(__VA_ARGS__);          \
+      return MOE_ERR_INVALID_ARG;           \
+    }                                       \
+  } while (0)
+
+moe_status_t cuda_status(cudaError_t e, const char* where) {
+  if (e == cudaSuccess) return MOE_OK;
+  set_last_error("%s: %s", where, cudaGetErrorString(e));
+  return MOE_ERR_CUDA;
+}
+
+moe_status_t check_dtype(moe_dtype_t dt) {
+  MOE_CHECK_ARG(dt == MOE_F32 || dt == MOE_BF16, "dt must be MOE_F32 or MOE_BF16");
+  return MOE_OK;
+}
+
+// Row length in bytes must be whole 16-byte vectors.
+moe_status_t check_rows(int d, moe_dtype_t dt, const char* name) {
+  MOE_CHECK_ARG(d >= 1 && (static_cast<size_t>(d) * elt_bytes(dt)) % 16 == 0,
+                "%s: d=%d must be >= 1 and a multiple of %d for this dtype", name, d,
+                static_cast<int>(16 / elt_bytes(dt)));
+  return MOE_OK;
+}
+
+bool router_uses_tc(int E, moe_dtype_t dt) { return dt == MOE_BF16 && E <= 256; }
+
+size_t router_ws(int T, int E, moe_dtype_t dt) {
+  size_t b = kStatusBytes;
+  if (!router_uses_tc(E, dt)) b += align_up(static_cast<size_t>(T) * E * sizeof(float), 256);
+  return b;
+}
+
+moe_status_t check_router(const void* x, const void* w_router, const float* logits_in, int T,
+                          int d, int E, int top_k, moe_score_t score, moe_dtype_t dt,
+                          const int32_t* topk_idx, const float* topk_w) {
+  if (moe_status_t s = check_dtype(dt)) return s;
+  MOE_CHECK_ARG(score == MOE_SCORE_SOFTMAX, "score: only MOE_SCORE_SOFTMAX is defined");
+  MOE_CHECK_ARG(T >= 0, "T=%d must be >= 0", T);
+  MOE_CHECK_ARG(E >= 1 && E <= kMaxExperts, "E=%d must be in [1, %d]", E, kMaxExperts);
+  MOE_CHECK_ARG(top_k >= 1 && top_k <= std::min(E, kMaxTopK), "top_k=%d must be in [1, min(E, %d)]",
+                top_k, kMaxTopK);
+  if (T > 0) {
+    MOE_CHECK_ARG(topk_idx && topk_w, "topk_idx and topk_w are required");
+    if (!logits_in) {
+      MOE_CHECK_ARG(x && w_router, "x and w_router are required without logits_in");
+      MOE_CHECK_ARG(aligned16(x) && aligned16(w_router), "x / w_router must be 16-byte aligned");
+      if (moe_status_t s = check_rows(d, dt, "router")) return s;
+    }
+  }
+  return MOE_OK;
+}
+
+// Router launch sequence (status and counts already cleared by the caller).
+cudaError_t run_router(const void* x, const void* w_router, const float* logits_in, int T, int d,
+                       int E, int top_k, int renorm, moe_dtype_t dt, float* logits_out,
+                       int32_t* topk_idx, float* topk_w, int32_t* counts, void* scratch,
+                       int* status, cudaStream_t s) {
+  if (T == 0) return cudaSuccess;
+  if (logits_in)
+    return launch_topk_from_logits(logits_in, T, E, top_k, renorm, topk_idx, topk_w, counts, s);
+  if (router_uses_tc(E, dt))
+    return launch_router_tc(x, w_router, T, d, E, top_k, renorm, logits_out, topk_idx, topk_w,
+                            counts, status, s);
+  float* L = logits_out ? logits_out : static_cast<float*>(scratch);
+  cudaError_t e = launch_router_logits_simt(x, w_router, T, d, E, dt, L, s);
+  if (e != cudaSuccess) return e;
+  return launch_topk_from_logits(L, T, E, top_k, renorm, topk_idx, topk_w, counts, s);
+}
+
+size_t swiglu_ws(int N, int h, moe_dtype_t dt) {
+  return kStatusBytes + align_up(static_cast<size_t>(N) * h * elt_bytes(dt), 256);
+}
+
+moe_status_t check_swiglu_shape(int N, int d, int h, int E, moe_dtype_t dt) {
+  if (moe_status_t s = check_dtype(dt)) return s;
+  MOE_CHECK_ARG(N >= 0 && E >= 1 && E <= kMaxExperts && d >= 1 && h >= 1,
+                "bad sizes N=%d d=%d h=%d E=%d", N, d, h, E);
+  if (dt == MOE_BF16) {
+    if (d % 64 != 0 || h % 64 != 0) {
+      set_last_error("bf16 grouped SwiGLU needs d %% 64 == 0 and h %% 64 == 0 (d=%d h=%d)", d, h);
+      return MOE_ERR_UNSUPPORTED;
+    }
+  } else {
+    MOE_CHECK_ARG(d % 4 == 0 && h % 4 == 0, "fp32 grouped SwiGLU needs d, h multiples of 4");
+  }
+  return MOE_OK;
+}
+
+cudaError_t run_swiglu(const void* x_perm, const int32_t* offsets, const void* w1, const void* w3,
+                       const void* w2, const float* row_scale, int N, int d, int h, int E,
+                       moe_dtype_t dt, void* y, void* H, int* status, cudaStream_t s) {
+  if (N == 0) return cudaSuccess;
+  if (dt == MOE_BF16)
+    return launch_swiglu_tc(x_perm, offsets, w1, w3, w2, row_scale, N, d, h, E, y, H, status, s);
+  return launch_swiglu_simt_f32(static_cast<const float*>(x_perm), offsets,
+                                static_cast<const float*>(w1), static_cast<const float*>(w3),
+                                static_cast<const float*>(w2), row_scale, N, d, h, E,
+                                static_cast<float*>(y), static_cast<float*>(H), status, s);
+}
+
+struct Carve {
+  char* base;
+  size_t off = 0;
+  explicit Carve(void* p) : base(static_cast<char*>(p)) {}
+  template <typename T>
+  T* take(size_t count) {
+    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+    off += align_up(count * sizeof(T), 256);
+    return p;
+  }
+};
+
+// Workspace of moe_forward.  The same function sizes it (base = null) and
+// carves it, so the two can never disagree.
+struct ForwardWs {
+  int* status;
+  void* router_scratch;
+  int32_t* idx;
+  float* w;
+  int32_t* counts_a;    // counts (R = 1) or counts_rm (R > 1)
+  int32_t* offsets_a;   // offsets or offsets_rm
+  int32_t* src_row;
+  int32_t* dst_pos;
+  void* disp_ws;
+  void* x_a;            // x_perm (R = 1) or rank-major rows (R > 1)
+  void* x_em;
+  int32_t* counts_em;
+  int32_t* offsets_em;
+  int32_t* perm;
+  int32_t* perm_inv;
+  void* reg_ws;
+  void* y;
+  void* H;
+  size_t bytes;
+};
+
+ForwardWs carve_forward(void* ws, int T, int d, int E, int k, int h, int R, moe_dtype_t dt) {
+  ForwardWs f{};
+  Carve c(ws);
+  const size_t N = static_cast<size_t>(T) * k;
+  const size_t row = static_cast<size_t>(d) * elt_bytes(dt);
+  f.status = c.take<int>(kStatusBytes / sizeof(int));
+  f.router_scratch = c.take<char>(router_ws(T, E, dt) - kStatusBytes);
+  f.idx = c.take<int32_t>(N);
+  f.w = c.take<float>(N);
+  const DispatchPlan p = make_dispatch_plan(T, E, k, R);
+  f.counts_a = c.take<int32_t>(static_cast<size_t>(p.nbins));
+  f.offsets_a = c.take<int32_t>(static_cast<size_t>(p.nbins) + 1);
+  f.src_row = c.take<int32_t>(N);
+  f.dst_pos = c.take<int32_t>(N);
+  f.disp_ws = c.take<char>(dispatch_ws_bytes(p));
+  f.x_a = c.take<char>(N * row);
+  if (R > 1) {
+    f.x_em = c.take<char>(N * row);
+    f.counts_em = c.take<int32_t>(E);
+    f.offsets_em = c.take<int32_t>(static_cast<size_t>(E) + 1);
+    f.perm = c.take<int32_t>(N);
+    f.perm_inv = c.take<int32_t>(N);
+    f.reg_ws = c.take<char>(regroup_ws_bytes(R, R, E / R));
+  }
+  f.y = c.take<char>(N * row);
+  f.H = c.take<char>(N * static_cast<size_t>(h) * elt_bytes(dt));
+  f.bytes = c.off;
+  return f;
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+int moe_version(void) { return 1 * 10000 + 0 * 100 + 0; }
+
+const char* moe_last_error(void) { return g_err; }
+
+const char* moe_status_string(moe_status_t s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported shape or option";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_WORKSPACE: return "workspace too small";
+    case MOE_ERR_DEVICE: return "device-side error";
+  }
+  return "unknown status";
+}
+
+moe_status_t moe_get_device_status(const void* ws, int* code, void* stream) {
+  if (!ws || !code) {
+    set_last_error("ws and code are required");
+    return MOE_ERR_INVALID_ARG;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int v = 0;
+  cudaError_t e = cudaMemcpyAsync(&v, ws, sizeof(int), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_status(e, "moe_get_device_status");
+  *code = v;
+  return MOE_OK;
+}
+
+// ------------------------------------------------------------------ router
+size_t moe_router_workspace_size(int T, int d, int E, moe_dtype_t dt) {
+  (void)d;
+  if (T < 0 || E < 1) return kStatusBytes;
+  return router_ws(T, E, dt);
+}
+
+moe_status_t moe_router_topk(const void* x, const void* w_router, const float* logits_in, int T,
+                             int d, int E, int top_k, moe_score_t score, int renormalize,
+                             moe_dtype_t dt, float* logits_out, int32_t* topk_idx, float* topk_w,
+                             int32_t* counts, void* ws, size_t ws_bytes, void* stream) {
+  if (moe_status_t st = check_router(x, w_router, logits_in, T, d, E, top_k, score, dt, topk_idx,
+                                     topk_w))
+    return st;
+  MOE_CHECK_ARG(ws != nullptr, "ws is required");
+  if (ws_bytes < router_ws(T, E, dt)) {
+    set_last_error("router workspace %zu < %zu", ws_bytes, router_ws(T, E, dt));
+    return MOE_ERR_WORKSPACE;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* status = static_cast<int*>(ws);
+  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), s);
+  if (e == cudaSuccess && counts) e = cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, s);
+  if (e == cudaSuccess)
+    e = run_router(x, w_router, logits_in, T, d, E, top_k, renormalize, dt, logits_out, topk_idx,
+                   topk_w, counts, static_cast<char*>(ws) + kStatusBytes, status, s);
+  return cuda_status(e, "moe_router_topk");
+}
+
+// ----------------------------------------------------------------- dispatch
+static moe_status_t dispatch_common(const void* x, const int32_t* topk_idx, int T, int d, int E,
+                                    int top_k, int R, moe_dtype_t dt, int32_t* counts,
+                                    int32_t* offsets, int32_t* src_row, int32_t* dst_pos,
+                                    void* x_perm, void* ws, size_t ws_bytes, void* stream) {
+  if (moe_status_t st = check_dtype(dt)) return st;
+  MOE_CHECK_ARG(T >= 0, "T must be >= 0");
+  MOE_CHECK_ARG(E >= 1 && E <= kMaxExperts, "E=%d must be in [1, %d]", E, kMaxExperts);
+  MOE_CHECK_ARG(top_k >= 1 && top_k <= std::min(E, kMaxTopK), "top_k=%d out of range", top_k);
+  MOE_CHECK_ARG(R >= 1 && E % R == 0 && E * R <= kMaxBins, "R=%d must divide E and E*R <= %d", R,
+                kMaxBins);
+  MOE_CHECK_ARG(counts && offsets, "counts and offsets are required");
+  if (T > 0) {
+    MOE_CHECK_ARG(topk_idx && src_row && dst_pos, "topk_idx, src_row, dst_pos are required");
+    if (x_perm) {
+      MOE_CHECK_ARG(x != nullptr, "x is required when x_perm is given");
+      MOE_CHECK_ARG(aligned16(x) && aligned16(x_perm), "x / x_perm must be 16-byte aligned");
+      if (moe_status_t st = check_rows(d, dt, "dispatch")) return st;
+    }
+  }
+  MOE_CHECK_ARG(ws != nullptr, "ws is required");
+  const DispatchPlan p = make_dispatch_plan(T, E, top_k, R);
+  const size_t need = kStatusBytes + dispatch_ws_bytes(p);
+  if (ws_bytes < need) {
+    set_last_error("dispatch workspace %zu < %zu", ws_bytes, need);
+    return MOE_ERR_WORKSPACE;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* status = static_cast<int*>(ws);
+  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), s);
+  if (e == cudaSuccess)
+    e = launch_dispatch(p, x, topk_idx, d, dt, counts, offsets, src_row, dst_pos,
+                        x ? x_perm : nullptr, static_cast<char*>(ws) + kStatusBytes, status, s);
+  return cuda_status(e, "moe_dispatch");
+}
+
+size_t moe_dispatch_workspace_size(int T, int E, int top_k) {
+  if (T < 0 || E < 1 || top_k < 1) return kStatusBytes;
+  return kStatusBytes + dispatch_ws_bytes(make_dispatch_plan(T, E, top_k, 1));
+}
+
+moe_status_t moe_dispatch(const void* x, const int32_t* topk_idx, int T, int d, int E, int top_k,
+                          moe_dtype_t dt, int32_t* counts, int32_t* offsets, int32_t* src_row,
+                          int32_t* dst_pos, void* x_perm, void* ws, size_t ws_bytes,
+                          void* stream) {
+  return dispatch_common(x, topk_idx, T, d, E, top_k, 1, dt, counts, offsets, src_row, dst_pos,
+                         x_perm, ws, ws_bytes, stream);
+}
+
+size_t moe_ep_dispatch_workspace_size(int T, int E, int top_k, int R) {
+  if (T < 0 || E < 1 || top_k < 1 || R < 1 || E % R) return kStatusBytes;
+  return kStatusBytes + dispatch_ws_bytes(make_dispatch_plan(T, E, top_k, R));
+}
+
+moe_status_t moe_ep_dispatch_rank_major(const void* x, const int32_t* topk_idx, int T, int d,
+                                        int E, int top_k, int R, moe_dtype_t dt,
+                                        int32_t* counts_rm, int32_t* offsets_rm,
+                                        int32_t* src_row, int32_t* dst_pos, void* x_rm, void* ws,
+                                        size_t ws_bytes, void* stream) {
+  return dispatch_common(x, topk_idx, T, d, E, top_k, R, dt, counts_rm, offsets_rm, src_row,
+                         dst_pos, x_rm, ws, ws_bytes, stream);
+}
+
+// ------------------------------------------------------------------ regroup
+size_t moe_regroup_workspace_size(int G, int R, int L) {
+  if (G < 1 || R < 1 || L < 1) return kStatusBytes;
+  return kStatusBytes + regroup_ws_bytes(G, R, L);
+}
+
+moe_status_t moe_ep_local_regroup(const void* in, const int32_t* counts_rm, int G, int R, int L,
+                                  int rows, int d, moe_dtype_t dt, void* out,
+                                  int32_t* counts_em, int32_t* offsets_em, int32_t* perm,
+                                  int32_t* perm_inv, void* ws, size_t ws_bytes, void* stream) {
+  if (moe_status_t st = check_dtype(dt)) return st;
+  MOE_CHECK_ARG(G >= 1 && R >= 1 && L >= 1 && 1LL * G * R * L <= kMaxSegments,
+                "G*R*L must be in [1, %d]", kMaxSegments);
+  MOE_CHECK_ARG(rows >= 0, "rows must be >= 0");
+  MOE_CHECK_ARG(counts_rm && counts_em && offsets_em, "counts_rm, counts_em, offsets_em required");
+  if (rows > 0) {
+    MOE_CHECK_ARG(in && out && perm, "in, out, perm are required");
+    MOE_CHECK_ARG(aligned16(in) && aligned16(out), "in / out must be 16-byte aligned");
+    if (moe_status_t st = check_rows(d, dt, "regroup")) return st;
+  }
+  MOE_CHECK_ARG(ws != nullptr, "ws is required");
+  const size_t need = kStatusBytes + regroup_ws_bytes(G, R, L);
+  if (ws_bytes < need) {
+    set_last_error("regroup workspace %zu < %zu", ws_bytes, need);
+    return MOE_ERR_WORKSPACE;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* status = static_cast<int*>(ws);
+  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), s);
+  if (e == cudaSuccess)
+    e = launch_regroup(in, counts_rm, G, R, L, rows, d, dt, out, counts_em, offsets_em, perm,
+                       perm_inv, static_cast<char*>(ws) + kStatusBytes, status, s);
+  return cuda_status(e, "moe_ep_local_regroup");
+}
+
+// ----------------------------------------------------------- grouped SwiGLU
+size_t moe_grouped_swiglu_workspace_size(int N, int d, int h, int E, moe_dtype_t dt) {
+  (void)d;
+  (void)E;
+  if (N < 0 || h < 1) return kStatusBytes;
+  return swiglu_ws(N, h, dt);
+}
+
+moe_status_t moe_grouped_swiglu(const void* x_perm, const int32_t* offsets, const void* w1,
+                                const void* w3, const void* w2, const float* row_scale, int N,
+                                int d, int h, int E, moe_dtype_t dt, void* y, void* ws,
+                                size_t ws_bytes, void* stream) {
+  if (moe_status_t st = check_swiglu_shape(N, d, h, E, dt)) return st;
+  if (N > 0) {
+    MOE_CHECK_ARG(x_perm && offsets && w1 && w3 && w2 && y, "x_perm, offsets, w1, w3, w2, y required");
+    MOE_CHECK_ARG(aligned16(x_perm) && aligned16(w1) && aligned16(w3) && aligned16(w2) &&
+                      aligned16(y),
+                  "x_perm, w1, w3, w2, y must be 16-byte aligned");
+  }
+  MOE_CHECK_ARG(ws != nullptr, "ws is required");
+  const size_t need = swiglu_ws(N, h, dt);
+  if (ws_bytes < need) {
+    set_last_error("grouped_swiglu workspace %zu < %zu", ws_bytes, need);
+    return MOE_ERR_WORKSPACE;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* status = static_cast<int*>(ws);
+  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), s);
+  if (e == cudaSuccess)
+    e = run_swiglu(x_perm, offsets, w1, w3, w2, row_scale, N, d, h, E, dt, y,
+                   static_cast<char*>(ws) + kStatusBytes, status, s);
+  return cuda_status(e, "moe_grouped_swiglu");
+}
+
+// ------------------------------------------------------------------ combine
+moe_status_t moe_combine(const void* y, const int32_t* dst_pos, const int32_t* row_map,
+                         const float* topk_w, int T, int d, int N, int top_k, moe_dtype_t dt,
+                         void* out, void* stream) {
+  if (moe_status_t st = check_dtype(dt)) return st;
+  MOE_CHECK_ARG(T >= 0 && N >= 0, "T, N must be >= 0");
+  MOE_CHECK_ARG(top_k >= 1 && top_k <= kMaxTopK, "top_k=%d out of range", top_k);
+  if (T > 0) {
+    MOE_CHECK_ARG(out && dst_pos, "out and dst_pos are required");
+    MOE_CHECK_ARG(N == 0 || y, "y is required");
+    MOE_CHECK_ARG(aligned16(out) && aligned16(y), "y / out must be 16-byte aligned");
+    if (moe_status_t st = check_rows(d, dt, "combine")) return st;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return cuda_status(launch_combine(y, dst_pos, row_map, topk_w, T, d, N, top_k, dt, out, s),
+                     "moe_combine");
+}
+
+// ------------------------------------------------------------------ forward
+size_t moe_forward_workspace_size(int T, int d, int E, int top_k, int h, int ep_ranks,
+                                  moe_dtype_t dt) {
+  if (T < 0 || d < 1 || E < 1 || top_k < 1 || h < 1 || ep_ranks < 1 || E % ep_ranks)
+    return kStatusBytes;
+  return carve_forward(nullptr, T, d, E, top_k, h, ep_ranks, dt).bytes;
+}
+
+moe_status_t moe_forward(const void* x, const void* w_router, const float* logits_in,
+                         const void* w1, const void* w3, const void* w2, int T, int d, int E,
+                         int top_k, int h, moe_score_t score, int renormalize, int ep_ranks,
+                         moe_dtype_t dt, void* out, float* logits_out, int32_t* topk_idx,
+                         float* topk_w, int32_t* counts, void* ws, size_t ws_bytes,
+                         void* stream) {
+  if (moe_status_t st = check_router(x, w_router, logits_in, T, d, E, top_k, score, dt,
+                                     reinterpret_cast<int32_t*>(1), reinterpret_cast<float*>(1)))
+    return st;
+  const int N = T * top_k;
+  if (moe_status_t st = check_swiglu_shape(N, d, h, E, dt)) return st;
+  MOE_CHECK_ARG(ep_ranks >= 1 && E % ep_ranks == 0 && E * ep_ranks <= kMaxBins &&
+                    1LL * ep_ranks * E <= kMaxSegments,
+                "ep_ranks=%d must divide E with E*ep_ranks <= %d", ep_ranks, kMaxBins);
+  if (T > 0) {
+    MOE_CHECK_ARG(x && w1 && w3 && w2 && out, "x, w1, w3, w2, out are required");
+    MOE_CHECK_ARG(aligned16(x) && aligned16(w1) && aligned16(w3) && aligned16(w2) &&
+                      aligned16(out),
+                  "x, w1, w3, w2, out must be 16-byte aligned");
+    if (moe_status_t st = check_rows(d, dt, "forward")) return st;
+  }
+  MOE_CHECK_ARG(ws != nullptr, "ws is required");
+  const ForwardWs need = carve_forward(nullptr, T, d, E, top_k, h, ep_ranks, dt);
+  if (ws_bytes < need.bytes) {
+    set_last_error("forward workspace %zu < %zu", ws_bytes, need.bytes);
+    return MOE_ERR_WORKSPACE;
+  }
+  const ForwardWs f = carve_forward(ws, T, d, E, top_k, h, ep_ranks, dt);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t* idx = topk_idx ? topk_idx : f.idx;
+  float* w = topk_w ? topk_w : f.w;
+  const int R = ep_ranks;
+  cudaError_t e = cudaMemsetAsync(f.status, 0, sizeof(int), s);
+  if (e == cudaSuccess)
+    e = run_router(x, w_router, logits_in, T, d, E, top_k, renormalize, dt, logits_out, idx, w,
+                   nullptr, f.router_scratch, f.status, s);
+  if (e != cudaSuccess) return cuda_status(e, "moe_forward/router");
+  const DispatchPlan p = make_dispatch_plan(T, E, top_k, R);
+  int32_t* cnt_a = (R == 1 && counts) ? counts : f.counts_a;
+  e = launch_dispatch(p, x, idx, d, dt, cnt_a, f.offsets_a, f.src_row, f.dst_pos, f.x_a,
+                      f.disp_ws, f.status, s);
+  if (e != cudaSuccess) return cuda_status(e, "moe_forward/dispatch");
+  const void* xe = f.x_a;
+  const int32_t* off = f.offsets_a;
+  const int32_t* row_map = nullptr;
+  if (R > 1) {
+    int32_t* cem = counts ? counts : f.counts_em;
+    e = launch_regroup(f.x_a, f.counts_a, R, R, E / R, N, d, dt, f.x_em, cem, f.offsets_em,
+                       f.perm, f.perm_inv, f.reg_ws, f.status, s);
+    if (e != cudaSuccess) return cuda_status(e, "moe_forward/regroup");
+    xe = f.x_em;
+    off = f.offsets_em;
+    row_map = f.perm_inv;
+  }
+  e = run_swiglu(xe, off, w1, w3, w2, nullptr, N, d, h, E, dt, f.y, f.H, f.status, s);
+  if (e != cudaSuccess) return cuda_status(e, "moe_forward/grouped_swiglu");
+  e = launch_combine(f.y, f.dst_pos, row_map, w, T, d, N, top_k, dt, out, s);
+  return cuda_status(e, "moe_forward/combine");
+}
+
+}  // extern "C"

@@ -1,0 +1,68 @@
+// Internal (non-exported) launchers shared by the translation units of libmoe.
+// Every launcher enqueues on `stream`, never synchronises, and returns the
+// cudaError_t of its launches.  `status` points at the device status word.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+int num_sms();                               // SM count of the current device
+void set_last_error(const char* fmt, ...);   // thread-local text for moe_last_error
+
+// ---- router -------------------------------------------------------------
+// tcgen05 router GEMM with the top-k/softmax epilogue (bf16, E <= 256).
+cudaError_t launch_router_tc(const void* x, const void* w_router, int T, int d, int E,
+                             int top_k, int renorm, float* logits_out, int32_t* topk_idx,
+                             float* topk_w, int32_t* counts, int* status, cudaStream_t s);
+// CUDA-core fp32 logits (x fp32 or bf16) into `logits` [T, E].
+cudaError_t launch_router_logits_simt(const void* x, const void* w_router, int T, int d, int E,
+                                      moe_dtype_t dt, float* logits, cudaStream_t s);
+// top-k / softmax / renormalisation / counts from fp32 logits.
+cudaError_t launch_topk_from_logits(const float* logits, int T, int E, int top_k, int renorm,
+                                    int32_t* topk_idx, float* topk_w, int32_t* counts,
+                                    cudaStream_t s);
+
+// ---- dispatch -------------------------------------------------------------
+struct DispatchPlan {
+  int T, k, E, R, L, S;   // R = 1: plain dispatch; R > 1: rank-major EP layout
+  int nbins;              // E or E * R
+  int tb;                 // tokens per block
+  int nblk;
+};
+DispatchPlan make_dispatch_plan(int T, int E, int top_k, int R);
+size_t dispatch_ws_bytes(const DispatchPlan& p);
+cudaError_t launch_dispatch(const DispatchPlan& p, const void* x, const int32_t* topk_idx,
+                            int d, moe_dtype_t dt, int32_t* counts, int32_t* offsets,
+                            int32_t* src_row, int32_t* dst_pos, void* x_perm, void* ws,
+                            int* status, cudaStream_t s);
+
+// ---- regroup ----------------------------------------------------------------
+size_t regroup_ws_bytes(int G, int R, int L);
+cudaError_t launch_regroup(const void* in, const int32_t* counts_rm, int G, int R, int L,
+                           int rows, int d, moe_dtype_t dt, void* out, int32_t* counts_em,
+                           int32_t* offsets_em, int32_t* perm, int32_t* perm_inv, void* ws,
+                           int* status, cudaStream_t s);
+
+// ---- combine ----------------------------------------------------------------
+cudaError_t launch_combine(const void* y, const int32_t* dst_pos, const int32_t* row_map,
+                           const float* topk_w, int T, int d, int N, int top_k, moe_dtype_t dt,
+                           void* out, cudaStream_t s);
+
+// ---- grouped SwiGLU -----------------------------------------------------
+// bf16 tcgen05 path: H (bf16 [N, h]) is scratch.
+cudaError_t launch_swiglu_tc(const void* x_perm, const int32_t* offsets, const void* w1,
+                             const void* w3, const void* w2, const float* row_scale, int N,
+                             int d, int h, int E, void* y, void* H, int* status,
+                             cudaStream_t s);
+// fp32 CUDA-core path: H (fp32 [N, h]) is scratch.
+cudaError_t launch_swiglu_simt_f32(const float* x_perm, const int32_t* offsets,
+                                   const float* w1, const float* w3, const float* w2,
+                                   const float* row_scale, int N, int d, int h, int E, float* y,
+                                   float* H, int* status, cudaStream_t s);
+
+}  // namespace moe

@@ -1,0 +1,514 @@
+// CUDA-core kernels of libmoe: dispatch (histogram, scan, stable rank,
+// 16-byte row scatter), EP local regroup, combine, and the fp32 router.
+//
+// Dispatch follows [HP] MoE.permutation: the expert-major order is a stable
+// sort of the flat expert ids, computed here without a sort and without
+// global atomics: per-block histograms, one scan over (block, bin), then a
+// warp-synchronous stable rank (match.any + popc) inside each block.
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+// --------------------------------------------------------------- dispatch
+__device__ __forceinline__ int dispatch_key(int e, int t, int R, int L, int S) {
+  if (R == 1) return e;
+  const int g = e / L, l = e - g * L, r = t / S;
+  return (g * R + r) * L + l;
+}
+
+// K1: histogram of the keys of each block of `tb` tokens.
+__global__ void dispatch_hist_kernel(const int32_t* __restrict__ idx, int T, int k, int E, int R,
+                                     int L, int S, int tb, int nbins, int32_t* __restrict__ blk,
+                                     int* status) {
+  extern __shared__ int hist[];
+  for (int i = threadIdx.x; i < nbins; i += blockDim.x) hist[i] = 0;
+  __syncthreads();
+  const int t0 = blockIdx.x * tb;
+  const int t1 = min(T, t0 + tb);
+  const long long f0 = 1LL * t0 * k, f1 = 1LL * t1 * k;
+  for (long long f = f0 + threadIdx.x; f < f1; f += blockDim.x) {
+    const int e = idx[f];
+    if (static_cast<unsigned>(e) >= static_cast<unsigned>(E)) {
+      set_status(status, MOE_DEV_BAD_EXPERT);
+      continue;
+    }
+    atomicAdd(&hist[dispatch_key(e, static_cast<int>(f / k), R, L, S)], 1);
+  }
+  __syncthreads();
+  int32_t* out = blk + static_cast<size_t>(blockIdx.x) * nbins;
+  for (int i = threadIdx.x; i < nbins; i += blockDim.x) out[i] = hist[i];
+}
+
+// Block-wide exclusive scan of `n` ints held in shared memory `a` (in place);
+// returns the total.  blockDim.x must be a multiple of 32 and <= 1024.
+__device__ int block_exclusive_scan(int* a, int n, int* warp_sums) {
+  const int nt = blockDim.x;
+  const int per = (n + nt - 1) / nt;
+  const int i0 = min(n, threadIdx.x * per), i1 = min(n, i0 + per);
+  int local = 0;
+  for (int i = i0; i < i1; ++i) local += a[i];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  int incl = local;
+#pragma unroll
+  for (int sh = 1; sh < 32; sh <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, sh);
+    if (lane >= sh) incl += v;
+  }
+  if (lane == 31) warp_sums[w] = incl;
+  __syncthreads();
+  if (w == 0) {
+    const int nw = nt >> 5;
+    int s = lane < nw ? warp_sums[lane] : 0;
+    int si = s;
+#pragma unroll
+    for (int sh = 1; sh < 32; sh <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, si, sh);
+      if (lane >= sh) si += v;
+    }
+    if (lane < nw) warp_sums[lane] = si - s;   // exclusive warp offsets
+    if (lane == 31) warp_sums[32] = si;        // total
+  }
+  __syncthreads();
+  int run = warp_sums[w] + incl - local;
+  for (int i = i0; i < i1; ++i) {
+    const int v = a[i];
+    a[i] = run;
+    run += v;
+  }
+  const int total = warp_sums[32];
+  __syncthreads();
+  return total;
+}
+
+// K2 (one block): per-bin prefix over blocks, totals -> counts, exclusive scan
+// over bins -> offsets, and the absolute base of every (block, bin).
+__global__ void dispatch_scan_kernel(int32_t* __restrict__ blk, int nblk, int nbins, int N,
+                                     int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                                     int32_t* __restrict__ src_row) {
+  extern __shared__ int sm[];
+  int* tot = sm;                 // nbins
+  int* wsum = sm + nbins;        // 33
+  for (int b = threadIdx.x; b < nbins; b += blockDim.x) {
+    int run = 0;
+    for (int k = 0; k < nblk; ++k) {
+      int32_t* p = blk + static_cast<size_t>(k) * nbins + b;
+      const int v = *p;
+      *p = run;
+      run += v;
+    }
+    tot[b] = run;
+    counts[b] = run;
+  }
+  __syncthreads();
+  const int total = block_exclusive_scan(tot, nbins, wsum);
+  for (int b = threadIdx.x; b < nbins; b += blockDim.x) offsets[b] = tot[b];
+  if (threadIdx.x == 0) offsets[nbins] = total;
+  __syncthreads();
+  for (int b = threadIdx.x; b < nbins; b += blockDim.x) {
+    const int base = tot[b];
+    for (int k = 0; k < nblk; ++k) blk[static_cast<size_t>(k) * nbins + b] += base;
+  }
+  // slots left empty by invalid expert ids
+  for (int s = total + threadIdx.x; s < N; s += blockDim.x) src_row[s] = -1;
+}
+
+// K3: stable slot of every copy (warp 0), then the row copies (all warps):
+// each token row is read once and written to its k slots with 16-byte stores.
+__global__ void dispatch_scatter_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ idx,
+                                        int T, int k, int E, int R, int L, int S, int tb,
+                                        int nbins, const int32_t* __restrict__ blk,
+                                        int32_t* __restrict__ src_row,
+                                        int32_t* __restrict__ dst_pos, uint4* __restrict__ x_perm,
+                                        int row_vec) {
+  extern __shared__ int sm[];
+  int* run = sm;              // nbins
+  int* slot = sm + nbins;     // tb * k
+  const int t0 = blockIdx.x * tb;
+  const int t1 = min(T, t0 + tb);
+  const int nf = (t1 - t0) * k;
+  const int32_t* base = blk + static_cast<size_t>(blockIdx.x) * nbins;
+  for (int i = threadIdx.x; i < nbins; i += blockDim.x) run[i] = base[i];
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    const unsigned lt = (1u << lane) - 1u;
+    for (int c0 = 0; c0 < nf; c0 += 32) {
+      const int i = c0 + lane;
+      const long long f = 1LL * t0 * k + i;
+      int key = -1 - lane;                       // unique: never matches
+      if (i < nf) {
+        const int e = idx[f];
+        if (static_cast<unsigned>(e) < static_cast<unsigned>(E))
+          key = dispatch_key(e, static_cast<int>(f / k), R, L, S);
+      }
+      const unsigned peers = __match_any_sync(0xffffffffu, key);
+      const int rank = __popc(peers & lt);
+      const int leader = __ffs(peers) - 1;
+      int s = -1;
+      if (key >= 0) s = run[key] + rank;
+      __syncwarp();
+      if (key >= 0 && lane == leader) run[key] += __popc(peers);
+      __syncwarp();
+      if (i < nf) {
+        dst_pos[f] = s;
+        slot[i] = s;
+        if (s >= 0) src_row[s] = static_cast<int>(f / k);
+      }
+    }
+  }
+  __syncthreads();
+  if (!x_perm) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  for (int t = t0 + warp; t < t1; t += nw) {
+    const uint4* src = x + static_cast<size_t>(t) * row_vec;
+    const int* sl = slot + (t - t0) * k;
+    for (int c = lane; c < row_vec; c += 32) {
+      const uint4 v = src[c];
+      for (int j = 0; j < k; ++j) {
+        const int s = sl[j];
+        if (s >= 0) x_perm[static_cast<size_t>(s) * row_vec + c] = v;
+      }
+    }
+  }
+}
+
+DispatchPlan make_dispatch_plan(int T, int E, int top_k, int R) {
+  DispatchPlan p{};
+  p.T = T;
+  p.k = top_k;
+  p.E = E;
+  p.R = R;
+  p.L = E / R;
+  p.S = R > 1 ? std::max(1, cdiv(T, R)) : std::max(T, 1);
+  p.nbins = E * R;
+  // Enough blocks to cover the SMs about twice; small blocks keep the
+  // warp-serial ranking short.
+  int tb = 16;
+  while (tb < 128 && cdiv(T, tb * 2) >= 2 * 148) tb *= 2;
+  p.tb = tb;
+  p.nblk = std::max(1, cdiv(T, tb));
+  return p;
+}
+
+size_t dispatch_ws_bytes(const DispatchPlan& p) {
+  return align_up(static_cast<size_t>(p.nblk) * p.nbins * sizeof(int32_t), 256);
+}
+
+cudaError_t launch_dispatch(const DispatchPlan& p, const void* x, const int32_t* topk_idx,
+                            int d, moe_dtype_t dt, int32_t* counts, int32_t* offsets,
+                            int32_t* src_row, int32_t* dst_pos, void* x_perm, void* ws,
+                            int* status, cudaStream_t s) {
+  int32_t* blk = static_cast<int32_t*>(ws);
+  const int N = p.T * p.k;
+  if (p.T == 0) {
+    cudaError_t e = cudaMemsetAsync(counts, 0, sizeof(int32_t) * p.nbins, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (p.nbins + 1), s);
+    return e;
+  }
+  dispatch_hist_kernel<<<p.nblk, 256, p.nbins * sizeof(int), s>>>(
+      topk_idx, p.T, p.k, p.E, p.R, p.L, p.S, p.tb, p.nbins, blk, status);
+  dispatch_scan_kernel<<<1, 1024, (p.nbins + 33) * sizeof(int), s>>>(blk, p.nblk, p.nbins, N,
+                                                                     counts, offsets, src_row);
+  const int elt = dt == MOE_BF16 ? 2 : 4;
+  const int row_vec = d * elt / 16;
+  const size_t sm3 = (p.nbins + p.tb * p.k) * sizeof(int);
+  dispatch_scatter_kernel<<<p.nblk, 256, sm3, s>>>(
+      static_cast<const uint4*>(x), topk_idx, p.T, p.k, p.E, p.R, p.L, p.S, p.tb, p.nbins, blk,
+      src_row, dst_pos, static_cast<uint4*>(x_perm), row_vec);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- regroup
+// Segment tables (one block): segments are numbered in OUTPUT order
+// o = (g*L + l)*R + r; in_start[o] is where segment (g, r, l) starts in the
+// rank-major input, out_start[o] (o = 0..S) where it starts in the output.
+__global__ void regroup_scan_kernel(const int32_t* __restrict__ counts_rm, int G, int R, int L,
+                                    int rows, int32_t* __restrict__ in_start,
+                                    int32_t* __restrict__ out_start,
+                                    int32_t* __restrict__ counts_em,
+                                    int32_t* __restrict__ offsets_em, int* flag, int* status) {
+  extern __shared__ int sm[];
+  const int S = G * R * L;
+  int* a = sm;            // S
+  int* wsum = sm + S;     // 33
+  __shared__ int bad;
+  if (threadIdx.x == 0) bad = 0;
+  __syncthreads();
+  // input order (g, r, l): exclusive scan of the counts as given
+  for (int i = threadIdx.x; i < S; i += blockDim.x) {
+    const int c = counts_rm[i];
+    if (c < 0) atomicOr(&bad, 1);
+    a[i] = max(c, 0);
+  }
+  __syncthreads();
+  const int total = block_exclusive_scan(a, S, wsum);
+  // scatter the input starts into output numbering
+  for (int i = threadIdx.x; i < S; i += blockDim.x) {
+    const int g = i / (R * L), r = (i / L) % R, l = i % L;
+    in_start[(g * L + l) * R + r] = a[i];
+  }
+  __syncthreads();
+  for (int o = threadIdx.x; o < S; o += blockDim.x) {
+    const int g = o / (L * R), l = (o / R) % L, r = o % R;
+    a[o] = max(counts_rm[(g * R + r) * L + l], 0);
+  }
+  __syncthreads();
+  block_exclusive_scan(a, S, wsum);
+  for (int o = threadIdx.x; o < S; o += blockDim.x) out_start[o] = a[o];
+  if (threadIdx.x == 0) {
+    out_start[S] = total;
+    const int ok = (bad == 0) && (total == rows);
+    *flag = ok;
+    if (!ok) set_status(status, MOE_DEV_BAD_COUNTS);
+  }
+  // expert-major counts / offsets: sum over r
+  for (int gl = threadIdx.x; gl < G * L; gl += blockDim.x) {
+    int c = 0;
+    for (int r = 0; r < R; ++r) c += max(counts_rm[((gl / L) * R + r) * L + gl % L], 0);
+    counts_em[gl] = c;
+    offsets_em[gl] = a[gl * R];
+  }
+  if (threadIdx.x == 0) offsets_em[G * L] = total;
+}
+
+__global__ void regroup_copy_kernel(const uint4* __restrict__ in, int rows, int row_vec, int S,
+                                    const int32_t* __restrict__ in_start,
+                                    const int32_t* __restrict__ out_start, const int* flag,
+                                    uint4* __restrict__ out, int32_t* __restrict__ perm,
+                                    int32_t* __restrict__ perm_inv) {
+  if (!*flag) return;
+  const int lane = threadIdx.x & 31;
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int nw = (gridDim.x * blockDim.x) >> 5;
+  for (int o = gw; o < rows; o += nw) {
+    int lo = 0, hi = S - 1;     // last segment with out_start <= o
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (out_start[mid] <= o) lo = mid; else hi = mid - 1;
+    }
+    const int src = in_start[lo] + (o - out_start[lo]);
+    if (lane == 0) {
+      perm[o] = src;
+      if (perm_inv) perm_inv[src] = o;
+    }
+    const uint4* s = in + static_cast<size_t>(src) * row_vec;
+    uint4* dst = out + static_cast<size_t>(o) * row_vec;
+    for (int c = lane; c < row_vec; c += 32) dst[c] = s[c];
+  }
+}
+
+size_t regroup_ws_bytes(int G, int R, int L) {
+  const size_t S = static_cast<size_t>(G) * R * L;
+  return align_up((2 * S + 1) * sizeof(int32_t) + 16, 256);
+}
+
+cudaError_t launch_regroup(const void* in, const int32_t* counts_rm, int G, int R, int L,
+                           int rows, int d, moe_dtype_t dt, void* out, int32_t* counts_em,
+                           int32_t* offsets_em, int32_t* perm, int32_t* perm_inv, void* ws,
+                           int* status, cudaStream_t s) {
+  const int S = G * R * L;
+  int32_t* in_start = static_cast<int32_t*>(ws);
+  int32_t* out_start = in_start + S;
+  int* flag = reinterpret_cast<int*>(out_start + S + 1);
+  regroup_scan_kernel<<<1, 1024, (S + 33) * sizeof(int), s>>>(
+      counts_rm, G, R, L, rows, in_start, out_start, counts_em, offsets_em, flag, status);
+  if (rows > 0) {
+    const int elt = dt == MOE_BF16 ? 2 : 4;
+    const int row_vec = d * elt / 16;
+    const int blocks = std::min(cdiv(rows, 8), num_sms() * 8);
+    regroup_copy_kernel<<<blocks, 256, 0, s>>>(static_cast<const uint4*>(in), rows, row_vec, S,
+                                               in_start, out_start, flag,
+                                               static_cast<uint4*>(out), perm, perm_inv);
+  }
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- combine
+// out[t] = sum_j w[t,j] * y[r(t,j)] in fp32, one 16-byte chunk per thread.
+template <bool BF16>
+__global__ void combine_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ dst_pos,
+                               const int32_t* __restrict__ row_map,
+                               const float* __restrict__ w, int T, int row_vec, int N, int k,
+                               uint4* __restrict__ out) {
+  const long long total = 1LL * T * row_vec;
+  for (long long i = blockIdx.x * 1LL * blockDim.x + threadIdx.x; i < total;
+       i += 1LL * gridDim.x * blockDim.x) {
+    const int t = static_cast<int>(i / row_vec);
+    const int c = static_cast<int>(i - 1LL * t * row_vec);
+    float acc[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) acc[q] = 0.f;
+    for (int j = 0; j < k; ++j) {
+      int p = dst_pos[static_cast<size_t>(t) * k + j];
+      if (row_map && static_cast<unsigned>(p) < static_cast<unsigned>(N)) p = row_map[p];
+      if (static_cast<unsigned>(p) >= static_cast<unsigned>(N)) continue;
+      const float wj = w ? w[static_cast<size_t>(t) * k + j] : 1.0f;
+      const uint4 v = y[static_cast<size_t>(p) * row_vec + c];
+      if (BF16) {
+        acc[0] = fmaf(wj, bf16_lo(v.x), acc[0]);
+        acc[1] = fmaf(wj, bf16_hi(v.x), acc[1]);
+        acc[2] = fmaf(wj, bf16_lo(v.y), acc[2]);
+        acc[3] = fmaf(wj, bf16_hi(v.y), acc[3]);
+        acc[4] = fmaf(wj, bf16_lo(v.z), acc[4]);
+        acc[5] = fmaf(wj, bf16_hi(v.z), acc[5]);
+        acc[6] = fmaf(wj, bf16_lo(v.w), acc[6]);
+        acc[7] = fmaf(wj, bf16_hi(v.w), acc[7]);
+      } else {
+        acc[0] = fmaf(wj, __uint_as_float(v.x), acc[0]);
+        acc[1] = fmaf(wj, __uint_as_float(v.y), acc[1]);
+        acc[2] = fmaf(wj, __uint_as_float(v.z), acc[2]);
+        acc[3] = fmaf(wj, __uint_as_float(v.w), acc[3]);
+      }
+    }
+    uint4 o;
+    if (BF16) {
+      o = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
+                     pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
+    } else {
+      o = make_uint4(__float_as_uint(acc[0]), __float_as_uint(acc[1]), __float_as_uint(acc[2]),
+                     __float_as_uint(acc[3]));
+    }
+    out[i] = o;
+  }
+}
+
+cudaError_t launch_combine(const void* y, const int32_t* dst_pos, const int32_t* row_map,
+                           const float* topk_w, int T, int d, int N, int top_k, moe_dtype_t dt,
+                           void* out, cudaStream_t s) {
+  if (T == 0) return cudaSuccess;
+  const int elt = dt == MOE_BF16 ? 2 : 4;
+  const int row_vec = d * elt / 16;
+  const long long total = 1LL * T * row_vec;
+  const int blocks = static_cast<int>(std::min<long long>(cdiv(static_cast<int>(std::min<long long>(total, 1LL << 30)), 256),
+                                                          1LL * num_sms() * 16));
+  if (dt == MOE_BF16)
+    combine_kernel<true><<<blocks, 256, 0, s>>>(static_cast<const uint4*>(y), dst_pos, row_map,
+                                                topk_w, T, row_vec, N, top_k,
+                                                static_cast<uint4*>(out));
+  else
+    combine_kernel<false><<<blocks, 256, 0, s>>>(static_cast<const uint4*>(y), dst_pos, row_map,
+                                                 topk_w, T, row_vec, N, top_k,
+                                                 static_cast<uint4*>(out));
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------- fp32 / SIMT router
+template <typename TX>
+__device__ __forceinline__ float to_f(TX v);
+template <>
+__device__ __forceinline__ float to_f<float>(float v) { return v; }
+template <>
+__device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+// logits[t, e] = sum_i x[t, i] * w[e, i], sequential fp32 FMA over i.
+template <typename TX>
+__global__ void router_logits_kernel(const TX* __restrict__ x, const TX* __restrict__ w, int T,
+                                     int d, int E, float* __restrict__ logits) {
+  const long long total = 1LL * T * E;
+  for (long long i = blockIdx.x * 1LL * blockDim.x + threadIdx.x; i < total;
+       i += 1LL * gridDim.x * blockDim.x) {
+    const int t = static_cast<int>(i / E), e = static_cast<int>(i % E);
+    const TX* xr = x + static_cast<size_t>(t) * d;
+    const TX* wr = w + static_cast<size_t>(e) * d;
+    float acc = 0.f;
+    for (int q = 0; q < d; ++q) acc = fmaf(to_f<TX>(xr[q]), to_f<TX>(wr[q]), acc);
+    logits[i] = acc;
+  }
+}
+
+cudaError_t launch_router_logits_simt(const void* x, const void* w_router, int T, int d, int E,
+                                      moe_dtype_t dt, float* logits, cudaStream_t s) {
+  const long long total = 1LL * T * E;
+  if (total == 0) return cudaSuccess;
+  const int blocks = static_cast<int>(std::min<long long>((total + 255) / 256, 1LL * num_sms() * 32));
+  if (dt == MOE_BF16)
+    router_logits_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(w_router), T, d,
+        E, logits);
+  else
+    router_logits_kernel<float><<<blocks, 256, 0, s>>>(static_cast<const float*>(x),
+                                                       static_cast<const float*>(w_router), T, d,
+                                                       E, logits);
+  return cudaGetLastError();
+}
+
+// One thread per token: top-KMAX in registers (score desc, index asc; NaN as
+// -inf), softmax denominator over all E, weights, counts.
+template <int KMAX>
+__global__ void topk_from_logits_kernel(const float* __restrict__ logits, int T, int E, int k,
+                                        int renorm, int32_t* __restrict__ topk_idx,
+                                        float* __restrict__ topk_w, int32_t* __restrict__ counts) {
+  for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < T; t += gridDim.x * blockDim.x) {
+    const float* L = logits + static_cast<size_t>(t) * E;
+    float v[KMAX];
+    int id[KMAX];
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      v[j] = -INFINITY;
+      id[j] = E + j;
+    }
+    float mx = -INFINITY;
+    for (int e = 0; e < E; ++e) {
+      float s = L[e];
+      if (s != s) s = -INFINITY;
+      mx = fmaxf(mx, s);
+      float cv = s;
+      int ci = e;
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j) {
+        const bool sw = (cv > v[j]) || (cv == v[j] && ci < id[j]);
+        const float tv = v[j];
+        const int ti = id[j];
+        v[j] = sw ? cv : tv;
+        id[j] = sw ? ci : ti;
+        cv = sw ? tv : cv;
+        ci = sw ? ti : ci;
+      }
+    }
+    float sum = 0.f;
+    for (int e = 0; e < E; ++e) {
+      float s = L[e];
+      if (s != s) s = -INFINITY;
+      sum += expf(s - mx);
+    }
+    float ex[KMAX];
+    float sel = 0.f;
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      ex[j] = expf(v[j] - mx);
+      if (j < k) sel += ex[j];
+    }
+    const float denom = renorm ? sel : sum;
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      if (j < k) {
+        topk_idx[static_cast<size_t>(t) * k + j] = id[j];
+        topk_w[static_cast<size_t>(t) * k + j] = ex[j] / denom;
+        if (counts) atomicAdd(&counts[id[j]], 1);
+      }
+    }
+  }
+}
+
+cudaError_t launch_topk_from_logits(const float* logits, int T, int E, int top_k, int renorm,
+                                    int32_t* topk_idx, float* topk_w, int32_t* counts,
+                                    cudaStream_t s) {
+  if (T == 0) return cudaSuccess;
+  const int blocks = std::min(cdiv(T, 128), num_sms() * 8);
+  if (top_k <= 1)
+    topk_from_logits_kernel<1><<<blocks, 128, 0, s>>>(logits, T, E, top_k, renorm, topk_idx, topk_w, counts);
+  else if (top_k <= 2)
+    topk_from_logits_kernel<2><<<blocks, 128, 0, s>>>(logits, T, E, top_k, renorm, topk_idx, topk_w, counts);
+  else if (top_k <= 4)
+    topk_from_logits_kernel<4><<<blocks, 128, 0, s>>>(logits, T, E, top_k, renorm, topk_idx, topk_w, counts);
+  else if (top_k <= 8)
+    topk_from_logits_kernel<8><<<blocks, 128, 0, s>>>(logits, T, E, top_k, renorm, topk_idx, topk_w, counts);
+  else
+    topk_from_logits_kernel<16><<<blocks, 128, 0, s>>>(logits, T, E, top_k, renorm, topk_idx, topk_w, counts);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,670 @@
+// tcgen05 (5th-generation tensor core) GEMMs of the MoE layer on sm_100a.
+//
+// One warp-specialised, persistent kernel skeleton serves three problems:
+//   * the router        logits[T, E] = x[T, d] . w_router[E, d]^T, with the
+//                       softmax / top-k / renormalisation / histogram done in
+//                       the epilogue straight out of TMEM
+//                       ([HP] TokenChoiceTopKRouter.forward);
+//   * GEMM1 (up)        for every expert segment, one 128 x 256 accumulator
+//                       holds x . w1^T (columns 0..127) and x . w3^T
+//                       (columns 128..255) for the same 128 hidden units; the
+//                       epilogue writes H = silu(G) * U in bf16
+//                       ([HP] _run_experts_for_loop, silu(x w1^T) * (x w3^T));
+//   * GEMM2 (down)      y = H . w2^T (times an optional row scale).
+//
+// Roles (192 threads): warp 0 issues TMA loads into a STAGES-deep ring of
+// shared-memory stages, warp 1 allocates TMEM and issues tcgen05.mma from one
+// thread, warps 2..5 drain the accumulator (tcgen05.ld) and write results.
+// Two TMEM accumulators let the epilogue of tile i overlap the MMAs of tile
+// i + 1.  Tiles are 128 rows (BM) x BN columns, K in steps of 64 bf16 (one
+// 128-byte swizzle row).  The expert tile schedule is built on the device
+// from the offsets array: no host synchronisation, no per-expert launches.
+// Tiles of one expert that share a weight tile are adjacent in the schedule,
+// so the CTAs that read the same weight tile run at the same time and the
+// second read hits L2.
+//
+// Every mbarrier wait is bounded (2 s), sets MOE_DEV_TIMEOUT and unwinds;
+// the kernel then waits (bounded) for its own loads and MMAs and frees TMEM.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+namespace tc {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int kThreads = 192;
+constexpr int kATileBytes = BM * BK * 2;   // 16 KB
+constexpr int kSmemBudget = 200 * 1024;    // stages; the rest is barriers + schedule
+
+struct TileInfo {
+  int a_row;     // first A row (token or routed copy)
+  int b_row;     // first B row in the [E * n, K] view of the weights
+  int m_valid;   // rows of this tile that belong to the problem / expert
+  int n0;        // first output column
+};
+
+struct Args {
+  int M;                     // rows of A: T (router) or N (grouped)
+  int K;                     // reduction length
+  int E;
+  int n_out;                 // output columns: E (router), h (up), d (down)
+  const int32_t* offsets;    // [E+1] expert segments (grouped)
+  int* status;
+  // router
+  float* logits_out;
+  int32_t* topk_idx;
+  float* topk_w;
+  int32_t* counts;
+  int top_k;
+  int renorm;
+  // grouped
+  __nv_bfloat16* out;        // H [N, h] (up) or y [N, d] (down)
+  const float* row_scale;    // down only, may be null
+};
+
+__host__ __device__ constexpr int stages_for(int bn) {
+  return (kSmemBudget / (kATileBytes + bn * BK * 2)) > 8 ? 8
+                                                          : (kSmemBudget / (kATileBytes + bn * BK * 2));
+}
+__host__ __device__ constexpr uint32_t tmem_cols_for(int bn) {
+  return (2 * bn <= 32) ? 32u : (2 * bn <= 64) ? 64u : (2 * bn <= 128) ? 128u
+                                                     : (2 * bn <= 256) ? 256u : 512u;
+}
+
+// ---------------------------------------------------------------- top-k
+// Running top-KMAX of (score, expert) pairs ordered by score descending then
+// expert ascending; NaN scores count as -inf.  Sentinels carry indices E..
+// so that any real expert, even at -inf, displaces them.
+template <int KMAX>
+struct TopK {
+  float v[KMAX];
+  int i[KMAX];
+  float mx;
+  __device__ __forceinline__ void init(int E) {
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      v[j] = -INFINITY;
+      i[j] = E + j;
+    }
+    mx = -INFINITY;
+  }
+  __device__ __forceinline__ void push(float s, int e) {
+    if (s != s) s = -INFINITY;
+    mx = fmaxf(mx, s);
+    float cv = s;
+    int ci = e;
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      const bool sw = (cv > v[j]) || (cv == v[j] && ci < i[j]);
+      const float tv = v[j];
+      const int ti = i[j];
+      v[j] = sw ? cv : tv;
+      i[j] = sw ? ci : ti;
+      cv = sw ? tv : cv;
+      ci = sw ? ti : ci;
+    }
+  }
+};
+
+__device__ __forceinline__ float nan_to_neginf(float s) { return (s != s) ? -INFINITY : s; }
+
+// ---------------------------------------------------------------- policies
+// Router: A = x [T, d], B = w_router [E, d] (rows >= E are zero-filled by TMA).
+template <int BN_, int KMAX>
+struct RouterPolicy {
+  static constexpr int BN = BN_;
+  static constexpr int NUM_B = 1;
+  static constexpr int SCHED_INTS = kMaxExperts + 8;   // per-CTA expert histogram
+
+  static __device__ void prologue(const Args& a, int* sched) {
+    for (int i = threadIdx.x; i < a.E; i += blockDim.x) sched[i] = 0;
+  }
+  static __device__ int num_tiles(const Args& a, const int*) { return cdiv(a.M, BM); }
+  static __device__ TileInfo tile_info(const Args& a, const int*, int tile) {
+    TileInfo t;
+    t.a_row = tile * BM;
+    t.b_row = 0;
+    t.m_valid = min(BM, a.M - t.a_row);
+    t.n0 = 0;
+    return t;
+  }
+  static __device__ void epilogue(const Args& a, int* sched, const TileInfo& ti, uint32_t taddr,
+                                  int row) {
+    const int E = a.E;
+    const bool valid = row < ti.m_valid;
+    const int t = ti.a_row + row;
+    TopK<KMAX> tk;
+    tk.init(E);
+    const int nch = cdiv(E, 32);
+    // pass 1: logits out, running max, top-k
+    for (int c = 0; c < nch; ++c) {
+      uint32_t r[32];
+      tmem_ld32(taddr + c * 32, r);
+      tmem_ld_wait();
+      if (valid && a.logits_out) {
+        float* dst = a.logits_out + static_cast<size_t>(t) * E + c * 32;
+        const int ncol = min(32, E - c * 32);
+        if (ncol == 32 && (reinterpret_cast<uintptr_t>(dst) & 15u) == 0) {
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            reinterpret_cast<float4*>(dst)[q] =
+                make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
+                            __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3]));
+        } else {
+          for (int q = 0; q < ncol; ++q) dst[q] = __uint_as_float(r[q]);
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < 32; ++q)
+        if (c * 32 + q < E) tk.push(__uint_as_float(r[q]), c * 32 + q);
+    }
+    // pass 2: softmax denominator over all E
+    float sum = 0.f;
+    for (int c = 0; c < nch; ++c) {
+      uint32_t r[32];
+      tmem_ld32(taddr + c * 32, r);
+      tmem_ld_wait();
+#pragma unroll
+      for (int q = 0; q < 32; ++q)
+        if (c * 32 + q < E) sum += expf(nan_to_neginf(__uint_as_float(r[q])) - tk.mx);
+    }
+    if (!valid) return;
+    float ex[KMAX];
+    float sel = 0.f;
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      ex[j] = expf(tk.v[j] - tk.mx);
+      if (j < a.top_k) sel += ex[j];
+    }
+    const float denom = a.renorm ? sel : sum;
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      if (j < a.top_k) {
+        const size_t o = static_cast<size_t>(t) * a.top_k + j;
+        a.topk_idx[o] = tk.i[j];
+        a.topk_w[o] = ex[j] / denom;
+        if (a.counts) atomicAdd(&sched[tk.i[j]], 1);
+      }
+    }
+  }
+  static __device__ void finish(const Args& a, int* sched) {
+    if (!a.counts) return;
+    for (int e = threadIdx.x; e < a.E; e += blockDim.x)
+      if (sched[e]) atomicAdd(&a.counts[e], sched[e]);
+  }
+};
+
+// Grouped problems: schedule over expert segments.  sched layout:
+//   [0] total tiles  [1] n-tiles per m-tile row  [8 .. 8+E]  offsets
+//   [8+E+1 .. 8+2E+1] cumulative tile counts
+template <int BN_, int NUM_B_, int NCOLS_PER_TILE>
+struct GroupedSched {
+  static constexpr int BN = BN_;
+  static constexpr int NUM_B = NUM_B_;
+  static constexpr int SCHED_INTS = 8 + 2 * (kMaxExperts + 1);
+
+  static __device__ void prologue(const Args& a, int* sched) {
+    const int E = a.E;
+    int* off = sched + 8;
+    int* cum = off + E + 1;
+    for (int i = threadIdx.x; i <= E; i += blockDim.x) off[i] = a.offsets[i];
+    __syncthreads();
+    if (threadIdx.x < 32) {
+      const int lane = threadIdx.x;
+      const int nt = cdiv(a.n_out, NCOLS_PER_TILE);
+      const int per = cdiv(E, 32);
+      const int e0 = min(E, lane * per), e1 = min(E, e0 + per);
+      int local = 0;
+      int bad = 0;
+      for (int e = e0; e < e1; ++e) {
+        const int cnt = off[e + 1] - off[e];
+        bad |= cnt < 0;
+        local += cdiv(max(cnt, 0), BM) * nt;
+      }
+      int incl = local;
+#pragma unroll
+      for (int sh = 1; sh < 32; sh <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, sh);
+        if (lane >= sh) incl += v;
+      }
+      int run = incl - local;
+      for (int e = e0; e < e1; ++e) {
+        cum[e] = run;
+        run += cdiv(max(off[e + 1] - off[e], 0), BM) * nt;
+      }
+      bad = __any_sync(0xffffffffu, bad);
+      const int total = __shfl_sync(0xffffffffu, incl, 31);
+      if (lane == 0) {
+        bad |= (off[0] != 0) || (off[E] != a.M);
+        cum[E] = total;
+        sched[0] = bad ? 0 : total;
+        sched[1] = nt;
+        if (bad && blockIdx.x == 0) set_status(a.status, MOE_DEV_BAD_OFFSETS);
+      }
+    }
+  }
+  static __device__ int num_tiles(const Args&, const int* sched) { return sched[0]; }
+  // tile -> (expert e, n-tile, m-tile); m-tiles of one (e, n-tile) are adjacent.
+  static __device__ void locate(const Args& a, const int* sched, int tile, int& e, int& nt,
+                                int& mt, int& cnt, int& seg0) {
+    const int E = a.E;
+    const int* off = sched + 8;
+    const int* cum = off + E + 1;
+    int lo = 0, hi = E - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (cum[mid] <= tile) lo = mid; else hi = mid - 1;
+    }
+    e = lo;
+    seg0 = off[e];
+    cnt = off[e + 1] - seg0;
+    const int mtiles = cdiv(cnt, BM);
+    const int local = tile - cum[e];
+    nt = local / mtiles;
+    mt = local - nt * mtiles;
+  }
+};
+
+// GEMM1: B0 = w1 rows [e*h + n0, +128), B1 = w3 rows (same), accumulator
+// columns [0,128) = G, [128,256) = U.
+struct UpPolicy : GroupedSched<256, 2, 128> {
+  static __device__ TileInfo tile_info(const Args& a, const int* sched, int tile) {
+    int e, nt, mt, cnt, seg0;
+    locate(a, sched, tile, e, nt, mt, cnt, seg0);
+    TileInfo t;
+    t.a_row = seg0 + mt * BM;
+    t.m_valid = min(BM, cnt - mt * BM);
+    t.n0 = nt * 128;
+    t.b_row = e * a.n_out + t.n0;
+    return t;
+  }
+  static __device__ void epilogue(const Args& a, int*, const TileInfo& ti, uint32_t taddr,
+                                  int row) {
+    const bool valid = row < ti.m_valid;
+    __nv_bfloat16* dst_row = a.out + static_cast<size_t>(ti.a_row + row) * a.n_out + ti.n0;
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      uint32_t g[32], u[32];
+      tmem_ld32(taddr + c * 32, g);
+      tmem_ld32(taddr + 128 + c * 32, u);
+      tmem_ld_wait();
+      if (valid && ti.n0 + c * 32 < a.n_out) {
+        uint32_t p[16];
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          const float g0 = __uint_as_float(g[2 * q]), g1 = __uint_as_float(g[2 * q + 1]);
+          const float u0 = __uint_as_float(u[2 * q]), u1 = __uint_as_float(u[2 * q + 1]);
+          const float h0 = __fdividef(g0, 1.0f + __expf(-g0)) * u0;
+          const float h1 = __fdividef(g1, 1.0f + __expf(-g1)) * u1;
+          p[q] = pack_bf16x2(h0, h1);
+        }
+        uint4* d4 = reinterpret_cast<uint4*>(dst_row + c * 32);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) d4[q] = make_uint4(p[4 * q], p[4 * q + 1], p[4 * q + 2], p[4 * q + 3]);
+      }
+    }
+  }
+  static __device__ void finish(const Args&, int*) {}
+};
+
+// GEMM2: B = w2 rows [e*d + n0, +256).
+struct DownPolicy : GroupedSched<256, 1, 256> {
+  static __device__ TileInfo tile_info(const Args& a, const int* sched, int tile) {
+    int e, nt, mt, cnt, seg0;
+    locate(a, sched, tile, e, nt, mt, cnt, seg0);
+    TileInfo t;
+    t.a_row = seg0 + mt * BM;
+    t.m_valid = min(BM, cnt - mt * BM);
+    t.n0 = nt * 256;
+    t.b_row = e * a.n_out + t.n0;
+    return t;
+  }
+  static __device__ void epilogue(const Args& a, int*, const TileInfo& ti, uint32_t taddr,
+                                  int row) {
+    const bool valid = row < ti.m_valid;
+    const size_t grow = static_cast<size_t>(ti.a_row + row);
+    const float scale = (valid && a.row_scale) ? a.row_scale[grow] : 1.0f;
+    __nv_bfloat16* dst_row = a.out + grow * a.n_out + ti.n0;
+#pragma unroll 1
+    for (int c = 0; c < 8; ++c) {
+      uint32_t r[32];
+      tmem_ld32(taddr + c * 32, r);
+      tmem_ld_wait();
+      if (valid && ti.n0 + c * 32 < a.n_out) {
+        uint32_t p[16];
+#pragma unroll
+        for (int q = 0; q < 16; ++q)
+          p[q] = pack_bf16x2(__uint_as_float(r[2 * q]) * scale,
+                             __uint_as_float(r[2 * q + 1]) * scale);
+        uint4* d4 = reinterpret_cast<uint4*>(dst_row + c * 32);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) d4[q] = make_uint4(p[4 * q], p[4 * q + 1], p[4 * q + 2], p[4 * q + 3]);
+      }
+    }
+  }
+  static __device__ void finish(const Args&, int*) {}
+};
+
+// ------------------------------------------------------------- the kernel
+template <class P>
+struct Layout {
+  static constexpr int BN = P::BN;
+  static constexpr int kBTileBytes = BN * BK * 2;
+  static constexpr int kStageBytes = kATileBytes + kBTileBytes;
+  static constexpr int kStages = stages_for(BN);
+  static constexpr uint32_t kTmemCols = tmem_cols_for(BN);
+  static constexpr int kBarOff = kStages * kStageBytes;
+  static constexpr int kNumBars = 2 * kStages + 5;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kSchedOff = (kMiscOff + 16 + 15) / 16 * 16;
+  static constexpr int kBytes = kSchedOff + P::SCHED_INTS * 4;
+  static constexpr int kLaunchBytes = kBytes + 1024;   // slack for 1 KB alignment
+  static_assert(kLaunchBytes <= 227 * 1024, "shared memory budget");
+  static_assert(kStages >= 2, "pipeline depth");
+};
+
+template <class P>
+__global__ void __launch_bounds__(kThreads, 1)
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
+                   const __grid_constant__ CUtensorMap tmB1, const Args args) {
+  using L = Layout<P>;
+  constexpr int BN = P::BN;
+  constexpr int STAGES = L::kStages;
+  constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+  uint8_t* tiles = smem;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* mma_done = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+  int* sched = reinterpret_cast<int*>(smem + L::kSchedOff);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(empty + s, 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull + a, 1);
+      mbar_init(tempty + a, 4);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB0);
+    if (P::NUM_B == 2) tma_prefetch_desc(&tmB1);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, L::kTmemCols);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  P::prologue(args, sched);
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = P::num_tiles(args, sched);
+  const int KB = cdiv(args.K, BK);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------ TMA producer
+      const uint64_t pol_b = l2_policy_evict_last();
+      const uint64_t pol_a = l2_policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        const TileInfo ti = P::tile_info(args, sched, tile);
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(empty + stage, phase ^ 1u, abort_flag, args.status)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = tiles + stage * L::kStageBytes;
+          uint8_t* sb = sa + kATileBytes;
+          mbar_arrive_expect_tx(full + stage, L::kStageBytes);
+          tma_load_2d(sa, &tmA, full + stage, kb * BK, ti.a_row, pol_a);
+          if (P::NUM_B == 1) {
+            tma_load_2d(sb, &tmB0, full + stage, kb * BK, ti.b_row, pol_b);
+          } else {
+            tma_load_2d(sb, &tmB0, full + stage, kb * BK, ti.b_row, pol_b);
+            tma_load_2d(sb + L::kBTileBytes / 2, &tmB1, full + stage, kb * BK, ti.b_row, pol_b);
+          }
+          ++issued;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // Drain: the last loads land before the CTA may exit.
+      int s = stage;
+      uint32_t ph = phase;
+      for (int i = 0; i < min(issued, STAGES); ++i) {
+        if (s == 0) {
+          s = STAGES - 1;
+          ph ^= 1u;
+        } else {
+          --s;
+        }
+        mbar_wait(full + s, ph, nullptr, args.status);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------ MMA issuer
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++it) {
+        const int acc = it & 1;
+        const uint32_t aph = (it >> 1) & 1;
+        if (!mbar_wait(tempty + acc, aph ^ 1u, abort_flag, args.status)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(full + stage, phase, abort_flag, args.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint8_t* sa = tiles + stage * L::kStageBytes;
+          const uint64_t ad = sw128_kmajor_desc(sa);
+          const uint64_t bd = sw128_kmajor_desc(sa + kATileBytes);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            tc_mma_bf16(d_tmem, ad + 2u * kk, bd + 2u * kk, IDESC, (kb | kk) ? 1u : 0u);
+          tc_commit(empty + stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(tfull + acc);
+      }
+      tc_commit(mma_done);
+      mbar_wait(mma_done, 0, nullptr, args.status);
+    }
+  } else {
+    // -------------------------------------------------- epilogue warps
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
+      const int acc = it & 1;
+      const uint32_t aph = (it >> 1) & 1;
+      int ok = 1;
+      if (lane == 0) ok = mbar_wait(tfull + acc, aph, abort_flag, args.status) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      tc_fence_after();
+      const TileInfo ti = P::tile_info(args, sched, tile);
+      const uint32_t taddr =
+          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
+      P::epilogue(args, sched, ti, taddr, row);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty + acc);
+    }
+  }
+  __syncthreads();
+  P::finish(args, sched);
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, L::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor map over a row-major [rows, inner] array, box [box_rows, 64],
+// 128-byte swizzle, zero fill outside the array.
+bool make_tmap(CUtensorMap* tm, const void* ptr, uint64_t inner, uint64_t rows, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) {
+    set_last_error("cuTensorMapEncodeTiled is not available from the driver");
+    return false;
+  }
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(BK), box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    set_last_error("cuTensorMapEncodeTiled failed (%d) for rows=%llu inner=%llu", (int)r,
+                   (unsigned long long)rows, (unsigned long long)inner);
+    return false;
+  }
+  return true;
+}
+
+template <class P>
+cudaError_t launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
+                   const Args& args, int grid, cudaStream_t s) {
+  using L = Layout<P>;
+  static int configured[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !configured[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<P>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         L::kLaunchBytes);
+    if (e != cudaSuccess) return e;
+    configured[dev] = 1;
+  }
+  tc_gemm_kernel<P><<<grid, kThreads, L::kLaunchBytes, s>>>(a, b0, b1, args);
+  return cudaGetLastError();
+}
+
+template <int BN>
+cudaError_t launch_router_bn(const CUtensorMap& a, const CUtensorMap& b, const Args& args,
+                             int grid, cudaStream_t s) {
+  const int k = args.top_k;
+  if (k <= 1) return launch<RouterPolicy<BN, 1>>(a, b, b, args, grid, s);
+  if (k <= 2) return launch<RouterPolicy<BN, 2>>(a, b, b, args, grid, s);
+  if (k <= 4) return launch<RouterPolicy<BN, 4>>(a, b, b, args, grid, s);
+  if (k <= 8) return launch<RouterPolicy<BN, 8>>(a, b, b, args, grid, s);
+  return launch<RouterPolicy<BN, 16>>(a, b, b, args, grid, s);
+}
+
+}  // namespace tc
+
+cudaError_t launch_router_tc(const void* x, const void* w_router, int T, int d, int E,
+                             int top_k, int renorm, float* logits_out, int32_t* topk_idx,
+                             float* topk_w, int32_t* counts, int* status, cudaStream_t s) {
+  using namespace tc;
+  const int bn = E <= 32 ? 32 : E <= 64 ? 64 : E <= 128 ? 128 : 256;
+  CUtensorMap ta, tb;
+  if (!make_tmap(&ta, x, d, T, BM)) return cudaErrorInvalidValue;
+  if (!make_tmap(&tb, w_router, d, E, bn)) return cudaErrorInvalidValue;
+  Args a{};
+  a.M = T;
+  a.K = d;
+  a.E = E;
+  a.n_out = E;
+  a.status = status;
+  a.logits_out = logits_out;
+  a.topk_idx = topk_idx;
+  a.topk_w = topk_w;
+  a.counts = counts;
+  a.top_k = top_k;
+  a.renorm = renorm;
+  const int grid = std::min(num_sms(), cdiv(T, BM));
+  switch (bn) {
+    case 32: return launch_router_bn<32>(ta, tb, a, grid, s);
+    case 64: return launch_router_bn<64>(ta, tb, a, grid, s);
+    case 128: return launch_router_bn<128>(ta, tb, a, grid, s);
+    default: return launch_router_bn<256>(ta, tb, a, grid, s);
+  }
+}
+
+cudaError_t launch_swiglu_tc(const void* x_perm, const int32_t* offsets, const void* w1,
+                             const void* w3, const void* w2, const float* row_scale, int N,
+                             int d, int h, int E, void* y, void* H, int* status,
+                             cudaStream_t s) {
+  using namespace tc;
+  CUtensorMap tx, t1, t3, th, t2;
+  if (!make_tmap(&tx, x_perm, d, N, BM)) return cudaErrorInvalidValue;
+  if (!make_tmap(&t1, w1, d, static_cast<uint64_t>(E) * h, 128)) return cudaErrorInvalidValue;
+  if (!make_tmap(&t3, w3, d, static_cast<uint64_t>(E) * h, 128)) return cudaErrorInvalidValue;
+  if (!make_tmap(&th, H, h, N, BM)) return cudaErrorInvalidValue;
+  if (!make_tmap(&t2, w2, h, static_cast<uint64_t>(E) * d, 256)) return cudaErrorInvalidValue;
+  const int max_mt = cdiv(N, BM) + E;   // upper bound on m-tiles over all segments
+  Args a{};
+  a.M = N;
+  a.E = E;
+  a.offsets = offsets;
+  a.status = status;
+  // GEMM1: H = silu(x w1^T) * (x w3^T)
+  a.K = d;
+  a.n_out = h;
+  a.out = static_cast<__nv_bfloat16*>(H);
+  int grid = static_cast<int>(std::min<long long>(num_sms(), 1LL * max_mt * cdiv(h, 128)));
+  cudaError_t e = launch<UpPolicy>(tx, t1, t3, a, grid, s);
+  if (e != cudaSuccess) return e;
+  // GEMM2: y = H w2^T (* row_scale)
+  a.K = h;
+  a.n_out = d;
+  a.out = static_cast<__nv_bfloat16*>(y);
+  a.row_scale = row_scale;
+  grid = static_cast<int>(std::min<long long>(num_sms(), 1LL * max_mt * cdiv(d, 256)));
+  return launch<DownPolicy>(th, t2, t2, a, grid, s);
+}
+
+}  // namespace moe

@@ -1,0 +1,119 @@
+"""Host-only checks of the C ABI: the library loads, exports every function
+include/moe.h declares, and rejects bad arguments before touching the GPU.
+No kernel is launched here (these run without a GPU)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from routing_dispatch_grouped_topk_b200 import build
+    build.build()
+    import routing_dispatch_grouped_topk_b200 as m
+    return m.lib()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ["moe_router_topk", "moe_dispatch", "moe_ep_local_regroup", "moe_grouped_swiglu",
+              "moe_combine", "moe_forward"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    import routing_dispatch_grouped_topk_b200 as m
+    names = declared_functions()
+    for n in names:
+        assert hasattr(L, n), n
+    assert sorted(m.EXPORTED_SYMBOLS) == names
+    out = subprocess.run(["nm", "-D", "--defined-only", m.LIB_PATH], capture_output=True,
+                         text=True).stdout
+    exported = set(re.findall(r"\bT (moe_[a-z0-9_]+)", out))
+    assert set(names) <= exported
+    # plain C names: nothing C++-mangled with the moe_ prefix leaks out
+    assert not re.search(r"\bT _Z\S*moe_", out)
+
+
+def test_version_and_strings(L):
+    assert L.moe_version() == 10000
+    assert L.moe_status_string(0) == b"ok"
+    assert L.moe_status_string(1) == b"invalid argument"
+
+
+def test_workspace_sizes_are_host_only(L):
+    assert L.moe_dispatch_workspace_size(4096, 128, 8) >= 256
+    assert L.moe_forward_workspace_size(4096, 2048, 128, 8, 768, 1, 1) > 2 * 4096 * 8 * 2048 * 2
+    assert L.moe_forward_workspace_size(8192, 2880, 128, 4, 2880, 8, 1) > \
+        L.moe_forward_workspace_size(8192, 2880, 128, 4, 2880, 1, 1)
+    assert L.moe_regroup_workspace_size(8, 8, 16) >= 256
+    assert L.moe_grouped_swiglu_workspace_size(100, 64, 128, 4, 1) >= 256 + 100 * 128 * 2
+
+
+@pytest.mark.parametrize("case", [
+    dict(top_k=0), dict(top_k=17), dict(E=0), dict(E=513), dict(T=-1), dict(dt=7), dict(score=1),
+    dict(top_k=9, E=8),
+])
+def test_router_rejects_bad_arguments(L, case):
+    a = dict(T=4, d=64, E=8, top_k=2, score=0, dt=1)
+    a.update(case)
+    p = ctypes.c_void_p(16)
+    r = L.moe_router_topk(p, p, None, a["T"], a["d"], a["E"], a["top_k"], a["score"], 1, a["dt"],
+                          None, p, p, None, p, 1 << 20, None)
+    assert r == 1, L.moe_last_error()
+    assert L.moe_last_error() != b""
+
+
+def test_router_rejects_unaligned_and_null(L):
+    p = ctypes.c_void_p(16)
+    q = ctypes.c_void_p(18)
+    assert L.moe_router_topk(q, p, None, 4, 64, 8, 2, 0, 1, 1, None, p, p, None, p, 1 << 20,
+                             None) == 1
+    assert L.moe_router_topk(None, p, None, 4, 64, 8, 2, 0, 1, 1, None, p, p, None, p, 1 << 20,
+                             None) == 1
+    # d not a whole number of 16-byte vectors for bf16
+    assert L.moe_router_topk(p, p, None, 4, 60, 8, 2, 0, 1, 1, None, p, p, None, p, 1 << 20,
+                             None) == 1
+
+
+def test_grouped_swiglu_shape_rules(L):
+    p = ctypes.c_void_p(256)
+    # bf16 tensor-core path needs d, h multiples of 64
+    assert L.moe_grouped_swiglu(p, p, p, p, p, None, 10, 96, 128, 4, 1, p, p, 1 << 30, None) == 2
+    assert L.moe_grouped_swiglu(p, p, p, p, p, None, 10, 128, 96, 4, 1, p, p, 1 << 30, None) == 2
+    # workspace too small
+    assert L.moe_grouped_swiglu(p, p, p, p, p, None, 10, 128, 128, 4, 1, p, p, 16, None) == 4
+
+
+def test_dispatch_and_regroup_argument_rules(L):
+    p = ctypes.c_void_p(256)
+    # R must divide E
+    assert L.moe_ep_dispatch_rank_major(p, p, 8, 64, 10, 2, 3, 1, p, p, p, p, p, p, 1 << 20,
+                                        None) == 1
+    # E * R above the bin limit
+    assert L.moe_ep_dispatch_rank_major(p, p, 8, 64, 512, 2, 32, 1, p, p, p, p, p, p, 1 << 20,
+                                        None) == 1
+    assert L.moe_ep_local_regroup(p, p, 0, 2, 2, 10, 64, 1, p, p, p, p, None, p, 1 << 20,
+                                  None) == 1
+    assert L.moe_dispatch(p, p, 8, 64, 8, 2, 1, p, p, p, p, p, p, 8, None) == 4
+    assert L.moe_combine(p, p, None, None, 4, 64, 8, 0, 1, p, None) == 1
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    import routing_dispatch_grouped_topk_b200 as m
+    monkeypatch.setattr(m, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(m, "_lib", None)
+    with pytest.raises(m.MoEError, match="no CPU fallback"):
+        m.lib()
