@@ -363,13 +363,15 @@ def dense_moe(x, idx, w, w1, w3, w2) -> np.ndarray:
 def moe_tokens(x_rows, idx_rows, w_rows, w1, w3, w2) -> np.ndarray:
     """Token-by-token definition for a sample of tokens:
     ``out[t] = sum_j w[t, j] * FFN_{idx[t, j]}(x[t])``.  Used to check sampled
-    outputs of layers too large for the full oracle."""
+    outputs of layers too large for the full oracle.  Each expert's weights
+    are widened to fp64 once, for all sampled copies routed to it."""
     x_rows = as_f64(x_rows)
     idx_rows = _i64(idx_rows)
     w_rows = as_f64(w_rows)
     out = np.zeros((x_rows.shape[0], w2.shape[1]))
-    for t in range(x_rows.shape[0]):
-        for j in range(idx_rows.shape[1]):
-            e = int(idx_rows[t, j])
-            out[t] += w_rows[t, j] * swiglu_ffn(x_rows[t:t + 1], w1[e], w3[e], w2[e])[0]
+    for e in np.unique(idx_rows):
+        tt, jj = np.nonzero(idx_rows == e)
+        ye = swiglu_ffn(x_rows[tt], w1[int(e)], w3[int(e)], w2[int(e)])
+        for q in range(len(tt)):
+            out[tt[q]] += w_rows[tt[q], jj[q]] * ye[q]
     return out
