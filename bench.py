@@ -125,13 +125,26 @@ def barrier(ws):
         dist.barrier()
 
 
-def max_over_ranks(v, ws):
+def max_over_ranks(v, ws, device="cuda"):
+    """Max of a per-rank float over all ranks (the job's device time)."""
     if ws == 1:
         return v
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_workload(cfg, rank):
+    """Workload of one rank: the same experts, an independent token batch."""
+    if rank == 0:
+        return cfg
+    return W.MoEConfig(**{**cfg.__dict__, "seed": cfg.seed + 1000 * rank})
+
+
+def job_tokens_per_s(T, ws, steps, total_ms_max):
+    """Whole-job throughput: every rank processed T tokens per step."""
+    return T * ws * steps / (total_ms_max / 1e3)
 
 
 # --------------------------------------------------------------- CPU oracle
@@ -197,8 +210,7 @@ def run_ours(args, ws, rank, local):
     dev = torch.device("cuda", local)
     lay = W.make_layer(cfg, dev)
     if rank:   # independent token batch per rank
-        lay["x"] = W.make_layer(W.MoEConfig(**{**cfg.__dict__, "seed": cfg.seed + 1000 * rank}),
-                                dev, experts=False)["x"]
+        lay["x"] = W.make_layer(rank_workload(cfg, rank), dev, experts=False)["x"]
     x, wr, w1, w3, w2 = lay["x"], lay["w_router"], lay["w1"], lay["w3"], lay["w2"]
     dt = M.MOE_BF16 if cfg.dtype == "bf16" else M.MOE_F32
     stream = torch.cuda.current_stream()
@@ -258,14 +270,21 @@ def run_ours(args, ws, rank, local):
         mark(i + 2)
 
     nmarks = len(stages) + 1
-    for _ in range(args.warmup):
-        step()
-        flush.zero_()
-    torch.cuda.synchronize()
-
+    # The clock sampler runs from the start of the warm-up (which lasts at
+    # least ~1.5 s of back-to-back steps) to the end of the timed region, so
+    # nvidia-smi has samples under load even when the timed region is short.
     sampler = ClockSampler(local)
     if rank == 0:
         sampler.start()
+    t_warm = time.perf_counter()
+    n_warm = 0
+    while n_warm < args.warmup or time.perf_counter() - t_warm < 1.5:
+        step()
+        flush.zero_()
+        n_warm += 1
+        if n_warm % 16 == 0:
+            torch.cuda.synchronize()
+    torch.cuda.synchronize()
     events = [[torch.cuda.Event(enable_timing=True) for _ in range(nmarks)]
               for _ in range(args.steps)]
     barrier(ws)
@@ -290,7 +309,7 @@ def run_ours(args, ws, rank, local):
     total_ms = sum(step_ms)
     total_ms_max = max_over_ranks(total_ms, ws)
     ms_per_step = total_ms_max / args.steps
-    value = T * ws * args.steps / (total_ms_max / 1e3)
+    value = job_tokens_per_s(T, ws, args.steps, total_ms_max)
 
     # e2e: host buffers through the public moe_forward call, copies included
     x_host = x.cpu().pin_memory()
@@ -323,7 +342,7 @@ def run_ours(args, ws, rank, local):
     torch.cuda.synchronize()
     barrier(ws)
     e2e_total = max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ms), ws)
-    e2e_value = T * ws * args.steps / (e2e_total / 1e3)
+    e2e_value = job_tokens_per_s(T, ws, args.steps, e2e_total)
     # the e2e output equals the device-resident step's output
     e2e_match = bool(torch.equal(out_host.to(dev), out))
 

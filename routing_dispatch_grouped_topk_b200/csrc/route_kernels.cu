@@ -19,7 +19,8 @@ __device__ __forceinline__ int dispatch_key(int e, int t, int R, int L, int S) {
   return (g * R + r) * L + l;
 }
 
-// K1: histogram of the keys of each block of `tb` tokens.
+// K1: histogram of the keys of each block of `tb` tokens, stored bin-major
+// (blk[bin * nblk + block]) so that K2 scans contiguous columns.
 __global__ void dispatch_hist_kernel(const int32_t* __restrict__ idx, int T, int k, int E, int R,
                                      int L, int S, int tb, int nbins, int32_t* __restrict__ blk,
                                      int* status) {
@@ -38,8 +39,9 @@ __global__ void dispatch_hist_kernel(const int32_t* __restrict__ idx, int T, int
     atomicAdd(&hist[dispatch_key(e, static_cast<int>(f / k), R, L, S)], 1);
   }
   __syncthreads();
-  int32_t* out = blk + static_cast<size_t>(blockIdx.x) * nbins;
-  for (int i = threadIdx.x; i < nbins; i += blockDim.x) out[i] = hist[i];
+  const int nblk = gridDim.x;
+  for (int i = threadIdx.x; i < nbins; i += blockDim.x)
+    blk[static_cast<size_t>(i) * nblk + blockIdx.x] = hist[i];
 }
 
 // Block-wide exclusive scan of `n` ints held in shared memory `a` (in place);
@@ -83,54 +85,88 @@ __device__ int block_exclusive_scan(int* a, int n, int* warp_sums) {
   return total;
 }
 
-// K2 (one block): per-bin prefix over blocks, totals -> counts, exclusive scan
-// over bins -> offsets, and the absolute base of every (block, bin).
-__global__ void dispatch_scan_kernel(int32_t* __restrict__ blk, int nblk, int nbins, int N,
-                                     int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
-                                     int32_t* __restrict__ src_row) {
-  extern __shared__ int sm[];
-  int* tot = sm;                 // nbins
-  int* wsum = sm + nbins;        // 33
-  for (int b = threadIdx.x; b < nbins; b += blockDim.x) {
-    int run = 0;
-    for (int k = 0; k < nblk; ++k) {
-      int32_t* p = blk + static_cast<size_t>(k) * nbins + b;
-      const int v = *p;
-      *p = run;
-      run += v;
+// Exclusive block-wide scan of one value per thread; *total receives the sum.
+// Every thread of the block must call it.
+__device__ int block_scan_value(int v, int* warp_sums, int* total) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int sh = 1; sh < 32; sh <<= 1) {
+    const int u = __shfl_up_sync(0xffffffffu, incl, sh);
+    if (lane >= sh) incl += u;
+  }
+  if (lane == 31) warp_sums[w] = incl;
+  __syncthreads();
+  if (w == 0) {
+    const int nw = blockDim.x >> 5;
+    const int s = lane < nw ? warp_sums[lane] : 0;
+    int si = s;
+#pragma unroll
+    for (int sh = 1; sh < 32; sh <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, si, sh);
+      if (lane >= sh) si += u;
     }
-    tot[b] = run;
-    counts[b] = run;
+    if (lane < nw) warp_sums[lane] = si - s;
+    if (lane == 31) warp_sums[32] = si;
   }
   __syncthreads();
-  const int total = block_exclusive_scan(tot, nbins, wsum);
-  for (int b = threadIdx.x; b < nbins; b += blockDim.x) offsets[b] = tot[b];
-  if (threadIdx.x == 0) offsets[nbins] = total;
+  const int ex = warp_sums[w] + incl - v;
+  *total = warp_sums[32];
   __syncthreads();
-  for (int b = threadIdx.x; b < nbins; b += blockDim.x) {
-    const int base = tot[b];
-    for (int k = 0; k < nblk; ++k) blk[static_cast<size_t>(k) * nbins + b] += base;
+  return ex;
+}
+
+// K2: for every bin (one block per bin, grid-stride), the exclusive prefix of
+// its column over the token blocks, in place; the column total is counts[bin].
+__global__ void dispatch_colscan_kernel(int32_t* __restrict__ blk, int nblk, int nbins,
+                                        int32_t* __restrict__ counts) {
+  __shared__ int wsum[33];
+  for (int bin = blockIdx.x; bin < nbins; bin += gridDim.x) {
+    int32_t* col = blk + static_cast<size_t>(bin) * nblk;
+    int carry = 0;
+    for (int base = 0; base < nblk; base += blockDim.x) {
+      const int i = base + threadIdx.x;
+      const int v = i < nblk ? col[i] : 0;
+      int tot;
+      const int ex = block_scan_value(v, wsum, &tot);
+      if (i < nblk) col[i] = carry + ex;
+      carry += tot;
+    }
+    if (threadIdx.x == 0) counts[bin] = carry;
   }
-  // slots left empty by invalid expert ids
-  for (int s = total + threadIdx.x; s < N; s += blockDim.x) src_row[s] = -1;
 }
 
 // K3: stable slot of every copy (warp 0), then the row copies (all warps):
 // each token row is read once and written to its k slots with 16-byte stores.
+// Each block also turns the bin totals into bin offsets (a block scan of
+// nbins values) and adds its column prefix; block 0 publishes the offsets
+// and marks slots left empty by invalid expert ids.
 __global__ void dispatch_scatter_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ idx,
                                         int T, int k, int E, int R, int L, int S, int tb,
                                         int nbins, const int32_t* __restrict__ blk,
+                                        const int32_t* __restrict__ counts,
+                                        int32_t* __restrict__ offsets,
                                         int32_t* __restrict__ src_row,
                                         int32_t* __restrict__ dst_pos, uint4* __restrict__ x_perm,
                                         int row_vec) {
   extern __shared__ int sm[];
-  int* run = sm;              // nbins
-  int* slot = sm + nbins;     // tb * k
+  int* run = sm;                   // nbins
+  int* wsum = sm + nbins;          // 33
+  int* slot = wsum + 33;           // tb * k
+  const int nblk = gridDim.x;
   const int t0 = blockIdx.x * tb;
   const int t1 = min(T, t0 + tb);
   const int nf = (t1 - t0) * k;
-  const int32_t* base = blk + static_cast<size_t>(blockIdx.x) * nbins;
-  for (int i = threadIdx.x; i < nbins; i += blockDim.x) run[i] = base[i];
+  for (int i = threadIdx.x; i < nbins; i += blockDim.x) run[i] = counts[i];
+  __syncthreads();
+  const int total = block_exclusive_scan(run, nbins, wsum);
+  if (blockIdx.x == 0) {
+    for (int i = threadIdx.x; i < nbins; i += blockDim.x) offsets[i] = run[i];
+    if (threadIdx.x == 0) offsets[nbins] = total;
+    for (long long s = total + threadIdx.x; s < 1LL * T * k; s += blockDim.x) src_row[s] = -1;
+  }
+  for (int i = threadIdx.x; i < nbins; i += blockDim.x)
+    run[i] += blk[static_cast<size_t>(i) * nblk + blockIdx.x];
   __syncthreads();
   if (threadIdx.x < 32) {
     const int lane = threadIdx.x;
@@ -208,16 +244,17 @@ cudaError_t launch_dispatch(const DispatchPlan& p, const void* x, const int32_t*
     if (e == cudaSuccess) e = cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (p.nbins + 1), s);
     return e;
   }
+  (void)N;
   dispatch_hist_kernel<<<p.nblk, 256, p.nbins * sizeof(int), s>>>(
       topk_idx, p.T, p.k, p.E, p.R, p.L, p.S, p.tb, p.nbins, blk, status);
-  dispatch_scan_kernel<<<1, 1024, (p.nbins + 33) * sizeof(int), s>>>(blk, p.nblk, p.nbins, N,
-                                                                     counts, offsets, src_row);
+  dispatch_colscan_kernel<<<std::min(p.nbins, num_sms() * 8), 256, 0, s>>>(blk, p.nblk, p.nbins,
+                                                                           counts);
   const int elt = dt == MOE_BF16 ? 2 : 4;
   const int row_vec = d * elt / 16;
-  const size_t sm3 = (p.nbins + p.tb * p.k) * sizeof(int);
+  const size_t sm3 = (p.nbins + 33 + p.tb * p.k) * sizeof(int);
   dispatch_scatter_kernel<<<p.nblk, 256, sm3, s>>>(
       static_cast<const uint4*>(x), topk_idx, p.T, p.k, p.E, p.R, p.L, p.S, p.tb, p.nbins, blk,
-      src_row, dst_pos, static_cast<uint4*>(x_perm), row_vec);
+      counts, offsets, src_row, dst_pos, static_cast<uint4*>(x_perm), row_vec);
   return cudaGetLastError();
 }
 
