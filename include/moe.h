@@ -205,6 +205,23 @@ MOE_API moe_status_t moe_grouped_swiglu(const void* x_perm, const int32_t* offse
                                 void* ws, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * moe_grouped_swiglu_gather -- moe_grouped_swiglu without the expert-major
+ * copy of the tokens: the rows of expert segment s are read straight from
+ * x through src_row (the gather [HP] MoE.forward writes as
+ * routed_x = x_flat[token_indices], fused into the first GEMM's loads).
+ *   H[s] = silu(x[src_row[s]] . w1[e]^T) * (x[src_row[s]] . w3[e]^T), then
+ *   y[s] as moe_grouped_swiglu.
+ * x [T, d]; src_row [N] int32 (device; entries outside [0, T) read zeros);
+ * offsets [E+1]; weights, row_scale, y, ws and the shape rules as
+ * moe_grouped_swiglu (workspace: moe_grouped_swiglu_workspace_size).
+ * ---------------------------------------------------------------------- */
+MOE_API moe_status_t moe_grouped_swiglu_gather(const void* x, int T, const int32_t* src_row,
+                                       const int32_t* offsets, const void* w1, const void* w3,
+                                       const void* w2, const float* row_scale, int N, int d,
+                                       int h, int E, moe_dtype_t dt, void* y, void* ws,
+                                       size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * moe_combine -- [QO] SpeedupMoeExperts.forward training branch
  * (weighted index_add_); [HP] MoE.unpermutation (scatter_add).
  *

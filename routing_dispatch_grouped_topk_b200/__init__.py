@@ -29,7 +29,8 @@ __all__ = [
     "MOE_DEV_BAD_EXPERT", "MOE_DEV_BAD_COUNTS", "MOE_DEV_BAD_OFFSETS", "MOE_DEV_TIMEOUT",
     "EXPORTED_SYMBOLS",
     "moe_router_topk", "moe_dispatch", "moe_ep_dispatch_rank_major", "moe_ep_local_regroup",
-    "moe_grouped_swiglu", "moe_combine", "moe_forward", "moe_get_device_status",
+    "moe_grouped_swiglu", "moe_grouped_swiglu_gather", "moe_combine", "moe_forward",
+    "moe_get_device_status", "grouped_swiglu_gather",
     "router_workspace_size", "dispatch_workspace_size", "ep_dispatch_workspace_size",
     "regroup_workspace_size", "grouped_swiglu_workspace_size", "forward_workspace_size",
     "router_topk", "dispatch", "ep_dispatch_rank_major", "ep_local_regroup",
@@ -47,7 +48,7 @@ EXPORTED_SYMBOLS = [
     "moe_dispatch_workspace_size", "moe_dispatch",
     "moe_ep_dispatch_workspace_size", "moe_ep_dispatch_rank_major",
     "moe_regroup_workspace_size", "moe_ep_local_regroup",
-    "moe_grouped_swiglu_workspace_size", "moe_grouped_swiglu",
+    "moe_grouped_swiglu_workspace_size", "moe_grouped_swiglu", "moe_grouped_swiglu_gather",
     "moe_combine",
     "moe_forward_workspace_size", "moe_forward",
     "moe_get_device_status", "moe_status_string", "moe_last_error", "moe_version",
@@ -74,6 +75,8 @@ _SIGS = {
                                   _P]),
     "moe_grouped_swiglu_workspace_size": (_Z, [_I, _I, _I, _I, _I]),
     "moe_grouped_swiglu": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _Z, _P]),
+    "moe_grouped_swiglu_gather": (_I, [_P, _I, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P,
+                                       _P, _Z, _P]),
     "moe_combine": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P]),
     "moe_forward_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I, _I]),
     "moe_forward": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P,
@@ -219,6 +222,16 @@ def moe_grouped_swiglu(x_perm, offsets, w1, w3, w2, row_scale, N, d, h, E, dt, y
         "moe_grouped_swiglu")
 
 
+def moe_grouped_swiglu_gather(x, T, src_row, offsets, w1, w3, w2, row_scale, N, d, h, E, dt, y,
+                              ws, stream=None):
+    _check(lib().moe_grouped_swiglu_gather(
+        _ptr(x, name="x"), T, _ptr(src_row, torch.int32, "src_row"),
+        _ptr(offsets, torch.int32, "offsets"), _ptr(w1, name="w1"), _ptr(w3, name="w3"),
+        _ptr(w2, name="w2"), _ptr(row_scale, torch.float32, "row_scale"), N, d, h, E, dt,
+        _ptr(y, name="y"), _ptr(ws, name="ws"), _nbytes(ws), _stream(stream)),
+        "moe_grouped_swiglu_gather")
+
+
 def moe_combine(y, dst_pos, row_map, topk_w, T, d, N, top_k, dt, out, stream=None):
     _check(lib().moe_combine(
         _ptr(y, name="y"), _ptr(dst_pos, torch.int32, "dst_pos"),
@@ -330,6 +343,18 @@ def grouped_swiglu(x_perm, offsets, w1, w3, w2, row_scale=None):
     y = torch.empty(N, d, dtype=x_perm.dtype, device=x_perm.device)
     ws = _ws(grouped_swiglu_workspace_size(N, d, h, E, _dt(x_perm)), x_perm.device)
     moe_grouped_swiglu(x_perm, offsets, w1, w3, w2, row_scale, N, d, h, E, _dt(x_perm), y, ws)
+    return y, ws
+
+
+def grouped_swiglu_gather(x, src_row, offsets, w1, w3, w2, row_scale=None):
+    """Grouped SwiGLU reading the rows of x through src_row.  Returns (y, ws)."""
+    T, d = x.shape
+    N = src_row.numel()
+    E, h, _ = w1.shape
+    y = torch.empty(N, d, dtype=x.dtype, device=x.device)
+    ws = _ws(grouped_swiglu_workspace_size(N, d, h, E, _dt(x)), x.device)
+    moe_grouped_swiglu_gather(x, T, src_row, offsets, w1, w3, w2, row_scale, N, d, h, E, _dt(x),
+                              y, ws)
     return y, ws
 
 

@@ -73,10 +73,11 @@ moe_status_t check_rows(int d, moe_dtype_t dt, const char* name) {
 
 bool router_uses_tc(int E, moe_dtype_t dt) { return dt == MOE_BF16 && E <= 256; }
 
-size_t router_ws(int T, int E, moe_dtype_t dt) {
-  size_t b = kStatusBytes;
-  if (!router_uses_tc(E, dt)) b += align_up(static_cast<size_t>(T) * E * sizeof(float), 256);
-  return b;
+// Status word plus the fp32 logit scratch: [ksplit, T, E] partial logits of
+// the tensor-core GEMM, or [T, E] logits of the CUDA-core path.
+size_t router_ws(int T, int d, int E, moe_dtype_t dt) {
+  const size_t planes = router_uses_tc(E, dt) ? router_plan(T, d).ksplit : 1;
+  return kStatusBytes + align_up(planes * T * E * sizeof(float), 256);
 }
 
 moe_status_t check_router(const void* x, const void* w_router, const float* logits_in, int T,
@@ -106,14 +107,19 @@ cudaError_t run_router(const void* x, const void* w_router, const float* logits_
                        int* status, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
   if (logits_in)
-    return launch_topk_from_logits(logits_in, T, E, top_k, renorm, topk_idx, topk_w, counts, s);
-  if (router_uses_tc(E, dt))
-    return launch_router_tc(x, w_router, T, d, E, top_k, renorm, logits_out, topk_idx, topk_w,
-                            counts, status, s);
-  float* L = logits_out ? logits_out : static_cast<float*>(scratch);
+    return launch_router_topk(logits_in, 1, T, E, top_k, renorm, nullptr, topk_idx, topk_w,
+                              counts, s);
+  float* part = static_cast<float*>(scratch);
+  if (router_uses_tc(E, dt)) {
+    cudaError_t e = launch_router_tc(x, w_router, T, d, E, part, status, s);
+    if (e != cudaSuccess) return e;
+    return launch_router_topk(part, router_plan(T, d).ksplit, T, E, top_k, renorm, logits_out,
+                              topk_idx, topk_w, counts, s);
+  }
+  float* L = logits_out ? logits_out : part;
   cudaError_t e = launch_router_logits_simt(x, w_router, T, d, E, dt, L, s);
   if (e != cudaSuccess) return e;
-  return launch_topk_from_logits(L, T, E, top_k, renorm, topk_idx, topk_w, counts, s);
+  return launch_router_topk(L, 1, T, E, top_k, renorm, nullptr, topk_idx, topk_w, counts, s);
 }
 
 size_t swiglu_ws(int N, int h, moe_dtype_t dt) {
@@ -145,6 +151,21 @@ cudaError_t run_swiglu(const void* x_perm, const int32_t* offsets, const void* w
                                 static_cast<const float*>(w1), static_cast<const float*>(w3),
                                 static_cast<const float*>(w2), row_scale, N, d, h, E,
                                 static_cast<float*>(y), static_cast<float*>(H), status, s);
+}
+
+cudaError_t run_swiglu_gather(const void* x, int T, const int32_t* src_row,
+                              const int32_t* offsets, const void* w1, const void* w3,
+                              const void* w2, const float* row_scale, int N, int d, int h, int E,
+                              moe_dtype_t dt, void* y, void* H, int* status, cudaStream_t s) {
+  if (N == 0) return cudaSuccess;
+  if (dt == MOE_BF16)
+    return launch_swiglu_tc_gather(x, T, src_row, offsets, w1, w3, w2, row_scale, N, d, h, E, y,
+                                   H, status, s);
+  return launch_swiglu_simt_f32_gather(static_cast<const float*>(x), T, src_row, offsets,
+                                       static_cast<const float*>(w1),
+                                       static_cast<const float*>(w3),
+                                       static_cast<const float*>(w2), row_scale, N, d, h, E,
+                                       static_cast<float*>(y), static_cast<float*>(H), status, s);
 }
 
 struct Carve {
@@ -189,7 +210,7 @@ ForwardWs carve_forward(void* ws, int T, int d, int E, int k, int h, int R, moe_
   const size_t N = static_cast<size_t>(T) * k;
   const size_t row = static_cast<size_t>(d) * elt_bytes(dt);
   f.status = c.take<int>(kStatusBytes / sizeof(int));
-  f.router_scratch = c.take<char>(router_ws(T, E, dt) - kStatusBytes);
+  f.router_scratch = c.take<char>(router_ws(T, d, E, dt) - kStatusBytes);
   f.idx = c.take<int32_t>(N);
   f.w = c.take<float>(N);
   const DispatchPlan p = make_dispatch_plan(T, E, k, R);
@@ -198,7 +219,7 @@ ForwardWs carve_forward(void* ws, int T, int d, int E, int k, int h, int R, moe_
   f.src_row = c.take<int32_t>(N);
   f.dst_pos = c.take<int32_t>(N);
   f.disp_ws = c.take<char>(dispatch_ws_bytes(p));
-  f.x_a = c.take<char>(N * row);
+  f.x_a = c.take<char>(R > 1 ? N * row : 0);   // single device: GEMM1 gathers from x
   if (R > 1) {
     f.x_em = c.take<char>(N * row);
     f.counts_em = c.take<int32_t>(E);
@@ -254,7 +275,7 @@ moe_status_t moe_get_device_status(const void* ws, int* code, void* stream) {
 size_t moe_router_workspace_size(int T, int d, int E, moe_dtype_t dt) {
   (void)d;
   if (T < 0 || E < 1) return kStatusBytes;
-  return router_ws(T, E, dt);
+  return router_ws(T, d, E, dt);
 }
 
 moe_status_t moe_router_topk(const void* x, const void* w_router, const float* logits_in, int T,
@@ -265,8 +286,8 @@ moe_status_t moe_router_topk(const void* x, const void* w_router, const float* l
                                      topk_w))
     return st;
   MOE_CHECK_ARG(ws != nullptr, "ws is required");
-  if (ws_bytes < router_ws(T, E, dt)) {
-    set_last_error("router workspace %zu < %zu", ws_bytes, router_ws(T, E, dt));
+  if (ws_bytes < router_ws(T, d, E, dt)) {
+    set_last_error("router workspace %zu < %zu", ws_bytes, router_ws(T, d, E, dt));
     return MOE_ERR_WORKSPACE;
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -411,6 +432,35 @@ moe_status_t moe_grouped_swiglu(const void* x_perm, const int32_t* offsets, cons
   return cuda_status(e, "moe_grouped_swiglu");
 }
 
+moe_status_t moe_grouped_swiglu_gather(const void* x, int T, const int32_t* src_row,
+                                       const int32_t* offsets, const void* w1, const void* w3,
+                                       const void* w2, const float* row_scale, int N, int d,
+                                       int h, int E, moe_dtype_t dt, void* y, void* ws,
+                                       size_t ws_bytes, void* stream) {
+  if (moe_status_t st = check_swiglu_shape(N, d, h, E, dt)) return st;
+  MOE_CHECK_ARG(T >= 0, "T must be >= 0");
+  if (N > 0) {
+    MOE_CHECK_ARG(T > 0 && x && src_row && offsets && w1 && w3 && w2 && y,
+                  "x (T > 0), src_row, offsets, w1, w3, w2, y required");
+    MOE_CHECK_ARG(aligned16(x) && aligned16(w1) && aligned16(w3) && aligned16(w2) &&
+                      aligned16(y),
+                  "x, w1, w3, w2, y must be 16-byte aligned");
+  }
+  MOE_CHECK_ARG(ws != nullptr, "ws is required");
+  const size_t need = swiglu_ws(N, h, dt);
+  if (ws_bytes < need) {
+    set_last_error("grouped_swiglu workspace %zu < %zu", ws_bytes, need);
+    return MOE_ERR_WORKSPACE;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* status = static_cast<int*>(ws);
+  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), s);
+  if (e == cudaSuccess)
+    e = run_swiglu_gather(x, T, src_row, offsets, w1, w3, w2, row_scale, N, d, h, E, dt, y,
+                          static_cast<char*>(ws) + kStatusBytes, status, s);
+  return cuda_status(e, "moe_grouped_swiglu_gather");
+}
+
 // ------------------------------------------------------------------ combine
 moe_status_t moe_combine(const void* y, const int32_t* dst_pos, const int32_t* row_map,
                          const float* topk_w, int T, int d, int N, int top_k, moe_dtype_t dt,
@@ -476,13 +526,23 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* logit
   if (e != cudaSuccess) return cuda_status(e, "moe_forward/router");
   const DispatchPlan p = make_dispatch_plan(T, E, top_k, R);
   int32_t* cnt_a = (R == 1 && counts) ? counts : f.counts_a;
-  e = launch_dispatch(p, x, idx, d, dt, cnt_a, f.offsets_a, f.src_row, f.dst_pos, f.x_a,
-                      f.disp_ws, f.status, s);
+  // Single device: only the routing indices are dispatched; GEMM1 gathers
+  // the token rows itself.  Simulated EP: the rank-major rows are
+  // materialised (they are what an all-to-all would deliver) and regrouped.
+  e = launch_dispatch(p, x, idx, d, dt, cnt_a, f.offsets_a, f.src_row, f.dst_pos,
+                      R > 1 ? f.x_a : nullptr, f.disp_ws, f.status, s);
   if (e != cudaSuccess) return cuda_status(e, "moe_forward/dispatch");
   const void* xe = f.x_a;
   const int32_t* off = f.offsets_a;
   const int32_t* row_map = nullptr;
-  if (R > 1) {
+  if (R == 1) {
+    e = run_swiglu_gather(x, T, f.src_row, off, w1, w3, w2, nullptr, N, d, h, E, dt, f.y, f.H,
+                          f.status, s);
+    if (e != cudaSuccess) return cuda_status(e, "moe_forward/grouped_swiglu");
+    e = launch_combine(f.y, f.dst_pos, nullptr, w, T, d, N, top_k, dt, out, s);
+    return cuda_status(e, "moe_forward/combine");
+  }
+  {
     int32_t* cem = counts ? counts : f.counts_em;
     e = launch_regroup(f.x_a, f.counts_a, R, R, E / R, N, d, dt, f.x_em, cem, f.offsets_em,
                        f.perm, f.perm_inv, f.reg_ws, f.status, s);

@@ -15,17 +15,27 @@ int num_sms();                               // SM count of the current device
 void set_last_error(const char* fmt, ...);   // thread-local text for moe_last_error
 
 // ---- router -------------------------------------------------------------
-// tcgen05 router GEMM with the top-k/softmax epilogue (bf16, E <= 256).
+// The tcgen05 router GEMM splits the reduction over d so that the number of
+// (128-token, K-split) tiles is close to kRouterTargetTiles (the SM count of
+// a B200); the plan depends on the sizes only, so workspace sizes can be
+// computed on the host without a device.
+constexpr int kRouterTargetTiles = 148;
+struct RouterPlan {
+  int ksplit;         // number of K splits (partial logit buffers)
+  int kb_per_split;   // 64-wide K blocks per split
+};
+RouterPlan router_plan(int T, int d);
+// tcgen05 router GEMM (bf16, E <= 256): fp32 partial logits [ksplit, T, E].
 cudaError_t launch_router_tc(const void* x, const void* w_router, int T, int d, int E,
-                             int top_k, int renorm, float* logits_out, int32_t* topk_idx,
-                             float* topk_w, int32_t* counts, int* status, cudaStream_t s);
+                             float* logits_part, int* status, cudaStream_t s);
 // CUDA-core fp32 logits (x fp32 or bf16) into `logits` [T, E].
 cudaError_t launch_router_logits_simt(const void* x, const void* w_router, int T, int d, int E,
                                       moe_dtype_t dt, float* logits, cudaStream_t s);
-// top-k / softmax / renormalisation / counts from fp32 logits.
-cudaError_t launch_topk_from_logits(const float* logits, int T, int E, int top_k, int renorm,
-                                    int32_t* topk_idx, float* topk_w, int32_t* counts,
-                                    cudaStream_t s);
+// Sum of `nsplit` partial logit arrays [nsplit, T, E] (in split order), then
+// softmax / top-k / renormalisation / counts; writes the logits if asked.
+cudaError_t launch_router_topk(const float* parts, int nsplit, int T, int E, int top_k,
+                               int renorm, float* logits_out, int32_t* topk_idx, float* topk_w,
+                               int32_t* counts, cudaStream_t s);
 
 // ---- dispatch -------------------------------------------------------------
 struct DispatchPlan {
@@ -59,10 +69,20 @@ cudaError_t launch_swiglu_tc(const void* x_perm, const int32_t* offsets, const v
                              const void* w3, const void* w2, const float* row_scale, int N,
                              int d, int h, int E, void* y, void* H, int* status,
                              cudaStream_t s);
+// Same with GEMM1's rows read from x [T, d] through src_row [N] (TMA gather4).
+cudaError_t launch_swiglu_tc_gather(const void* x, int T, const int32_t* src_row,
+                                    const int32_t* offsets, const void* w1, const void* w3,
+                                    const void* w2, const float* row_scale, int N, int d, int h,
+                                    int E, void* y, void* H, int* status, cudaStream_t s);
 // fp32 CUDA-core path: H (fp32 [N, h]) is scratch.
 cudaError_t launch_swiglu_simt_f32(const float* x_perm, const int32_t* offsets,
                                    const float* w1, const float* w3, const float* w2,
                                    const float* row_scale, int N, int d, int h, int E, float* y,
                                    float* H, int* status, cudaStream_t s);
+cudaError_t launch_swiglu_simt_f32_gather(const float* x, int x_rows, const int32_t* src_row,
+                                          const int32_t* offsets, const float* w1,
+                                          const float* w3, const float* w2,
+                                          const float* row_scale, int N, int d, int h, int E,
+                                          float* y, float* H, int* status, cudaStream_t s);
 
 }  // namespace moe

@@ -472,79 +472,115 @@ cudaError_t launch_router_logits_simt(const void* x, const void* w_router, int T
   return cudaGetLastError();
 }
 
-// One thread per token: top-KMAX in registers (score desc, index asc; NaN as
-// -inf), softmax denominator over all E, weights, counts.
-template <int KMAX>
-__global__ void topk_from_logits_kernel(const float* __restrict__ logits, int T, int E, int k,
-                                        int renorm, int32_t* __restrict__ topk_idx,
-                                        float* __restrict__ topk_w, int32_t* __restrict__ counts) {
-  for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < T; t += gridDim.x * blockDim.x) {
-    const float* L = logits + static_cast<size_t>(t) * E;
-    float v[KMAX];
-    int id[KMAX];
+// One warp per token.  Lane l holds experts l, l+32, ... (EPL of them): the
+// logit is the sum of the nsplit partial values in split order.  The k
+// winners are found by k rounds of a warp arg-max on (score desc, expert
+// asc); lane j keeps winner j.  NaN scores count as -inf (indices stay valid).
+template <int EPL>
+__global__ void __launch_bounds__(256) router_topk_kernel(
+    const float* __restrict__ parts, int nsplit, int T, int E, int k, int renorm,
+    float* __restrict__ logits_out, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
+    int32_t* __restrict__ counts) {
+  __shared__ int hist[kMaxExperts];
+  if (counts)
+    for (int i = threadIdx.x; i < E; i += blockDim.x) hist[i] = 0;
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int nwarps = (gridDim.x * blockDim.x) >> 5;
+  const size_t plane = static_cast<size_t>(T) * E;
+  for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += nwarps) {
+    float sv[EPL];
+    bool avail[EPL];
 #pragma unroll
-    for (int j = 0; j < KMAX; ++j) {
-      v[j] = -INFINITY;
-      id[j] = E + j;
+    for (int i = 0; i < EPL; ++i) {
+      const int e = lane + 32 * i;
+      avail[i] = e < E;
+      float v = 0.f;
+      if (avail[i]) {
+        const float* p = parts + static_cast<size_t>(t) * E + e;
+        v = p[0];
+        for (int sp = 1; sp < nsplit; ++sp) v += p[sp * plane];
+        if (logits_out) logits_out[static_cast<size_t>(t) * E + e] = v;
+      }
+      sv[i] = (v != v) ? -INFINITY : v;
     }
     float mx = -INFINITY;
-    for (int e = 0; e < E; ++e) {
-      float s = L[e];
-      if (s != s) s = -INFINITY;
-      mx = fmaxf(mx, s);
-      float cv = s;
-      int ci = e;
+    float my_v = 0.f;
+    int my_e = 0;
+    for (int j = 0; j < k; ++j) {
+      float bv = -INFINITY;
+      int be = 0x7fffffff;
 #pragma unroll
-      for (int j = 0; j < KMAX; ++j) {
-        const bool sw = (cv > v[j]) || (cv == v[j] && ci < id[j]);
-        const float tv = v[j];
-        const int ti = id[j];
-        v[j] = sw ? cv : tv;
-        id[j] = sw ? ci : ti;
-        cv = sw ? tv : cv;
-        ci = sw ? ti : ci;
+      for (int i = 0; i < EPL; ++i) {
+        const int e = lane + 32 * i;
+        if (avail[i] && (sv[i] > bv || (sv[i] == bv && e < be))) {
+          bv = sv[i];
+          be = e;
+        }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+        const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+        if (ov > bv || (ov == bv && oe < be)) {
+          bv = ov;
+          be = oe;
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < EPL; ++i)
+        if (lane + 32 * i == be) avail[i] = false;
+      if (j == 0) mx = bv;
+      if (lane == j) {
+        my_v = bv;
+        my_e = be;
       }
     }
-    float sum = 0.f;
-    for (int e = 0; e < E; ++e) {
-      float s = L[e];
-      if (s != s) s = -INFINITY;
-      sum += expf(s - mx);
-    }
-    float ex[KMAX];
-    float sel = 0.f;
+    float se = 0.f;
 #pragma unroll
-    for (int j = 0; j < KMAX; ++j) {
-      ex[j] = expf(v[j] - mx);
-      if (j < k) sel += ex[j];
-    }
-    const float denom = renorm ? sel : sum;
+    for (int i = 0; i < EPL; ++i)
+      if (lane + 32 * i < E) se += expf(sv[i] - mx);
+    const float ex = lane < k ? expf(my_v - mx) : 0.f;
+    float sel = ex;
 #pragma unroll
-    for (int j = 0; j < KMAX; ++j) {
-      if (j < k) {
-        topk_idx[static_cast<size_t>(t) * k + j] = id[j];
-        topk_w[static_cast<size_t>(t) * k + j] = ex[j] / denom;
-        if (counts) atomicAdd(&counts[id[j]], 1);
-      }
+    for (int off = 16; off > 0; off >>= 1) {
+      se += __shfl_xor_sync(0xffffffffu, se, off);
+      sel += __shfl_xor_sync(0xffffffffu, sel, off);
     }
+    if (lane < k) {
+      const size_t o = static_cast<size_t>(t) * k + lane;
+      topk_idx[o] = my_e;
+      topk_w[o] = ex / (renorm ? sel : se);
+      if (counts) atomicAdd(&hist[my_e], 1);
+    }
+  }
+  if (counts) {
+    __syncthreads();
+    for (int i = threadIdx.x; i < E; i += blockDim.x)
+      if (hist[i]) atomicAdd(&counts[i], hist[i]);
   }
 }
 
-cudaError_t launch_topk_from_logits(const float* logits, int T, int E, int top_k, int renorm,
-                                    int32_t* topk_idx, float* topk_w, int32_t* counts,
-                                    cudaStream_t s) {
+cudaError_t launch_router_topk(const float* parts, int nsplit, int T, int E, int top_k,
+                               int renorm, float* logits_out, int32_t* topk_idx, float* topk_w,
+                               int32_t* counts, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
-  const int blocks = std::min(cdiv(T, 128), num_sms() * 8);
-  if (top_k <= 1)
-    topk_from_logits_kernel<1><<<blocks, 128, 0, s>>>(logits, T, E, top_k, renorm, topk_idx, topk_w, counts);
-  else if (top_k <= 2)
-    topk_from_logits_kernel<2><<<blocks, 128, 0, s>>>(logits, T, E, top_k, renorm, topk_idx, topk_w, counts);
-  else if (top_k <= 4)
-    topk_from_logits_kernel<4><<<blocks, 128, 0, s>>>(logits, T, E, top_k, renorm, topk_idx, topk_w, counts);
-  else if (top_k <= 8)
-    topk_from_logits_kernel<8><<<blocks, 128, 0, s>>>(logits, T, E, top_k, renorm, topk_idx, topk_w, counts);
+  const int blocks = std::min(cdiv(T, 8), num_sms() * 16);
+  if (E <= 32)
+    router_topk_kernel<1><<<blocks, 256, 0, s>>>(parts, nsplit, T, E, top_k, renorm, logits_out,
+                                                 topk_idx, topk_w, counts);
+  else if (E <= 64)
+    router_topk_kernel<2><<<blocks, 256, 0, s>>>(parts, nsplit, T, E, top_k, renorm, logits_out,
+                                                 topk_idx, topk_w, counts);
+  else if (E <= 128)
+    router_topk_kernel<4><<<blocks, 256, 0, s>>>(parts, nsplit, T, E, top_k, renorm, logits_out,
+                                                 topk_idx, topk_w, counts);
+  else if (E <= 256)
+    router_topk_kernel<8><<<blocks, 256, 0, s>>>(parts, nsplit, T, E, top_k, renorm, logits_out,
+                                                 topk_idx, topk_w, counts);
   else
-    topk_from_logits_kernel<16><<<blocks, 128, 0, s>>>(logits, T, E, top_k, renorm, topk_idx, topk_w, counts);
+    router_topk_kernel<16><<<blocks, 256, 0, s>>>(parts, nsplit, T, E, top_k, renorm, logits_out,
+                                                  topk_idx, topk_w, counts);
   return cudaGetLastError();
 }
 

@@ -50,11 +50,13 @@ __device__ void simt_locate(const int* off, const int* cum, int E, int tile, int
 
 // H[s, n] = silu(sum_i x[s,i] w1[e,n,i]) * (sum_i x[s,i] w3[e,n,i])
 __global__ void __launch_bounds__(256) swiglu_up_f32_kernel(
-    const float* __restrict__ x, const int32_t* __restrict__ offsets,
-    const float* __restrict__ w1, const float* __restrict__ w3, int N, int d, int h, int E,
-    float* __restrict__ H, int* status) {
+    const float* __restrict__ x, const int32_t* __restrict__ src_row, int x_rows,
+    const int32_t* __restrict__ offsets, const float* __restrict__ w1,
+    const float* __restrict__ w3, int N, int d, int h, int E, float* __restrict__ H,
+    int* status) {
   __shared__ int off[kMaxExperts + 1], cum[kMaxExperts + 1];
   __shared__ float xs[SB][SB + 1], as[SB][SB + 1], bs[SB][SB + 1];
+  __shared__ int xrow[SB];
   if (!simt_schedule(offsets, E, N, off, cum, status)) return;
   const int tile = blockIdx.x;
   if (tile >= cum[E]) return;
@@ -68,6 +70,17 @@ __global__ void __launch_bounds__(256) swiglu_up_f32_kernel(
   simt_locate(off, cum, E, tile, row0, valid);
   const int n0 = blockIdx.y * SB;
   const int ty = threadIdx.x >> 3, tx = threadIdx.x & 7;   // row ty, columns tx*4..+3
+  // source row of every tile row: the slot itself, or its token when gathering
+  if (threadIdx.x < SB) {
+    const int r = threadIdx.x;
+    int src = -1;
+    if (r < valid) {
+      src = src_row ? src_row[row0 + r] : row0 + r;
+      if (static_cast<unsigned>(src) >= static_cast<unsigned>(x_rows)) src = -1;
+    }
+    xrow[r] = src;
+  }
+  __syncthreads();
   const float* W1 = w1 + static_cast<size_t>(e) * h * d;
   const float* W3 = w3 + static_cast<size_t>(e) * h * d;
   float g[4] = {0, 0, 0, 0}, u[4] = {0, 0, 0, 0};
@@ -75,7 +88,7 @@ __global__ void __launch_bounds__(256) swiglu_up_f32_kernel(
     for (int i = threadIdx.x; i < SB * SB; i += blockDim.x) {
       const int r = i / SB, c = i % SB;
       const bool kin = k0 + c < d;
-      xs[r][c] = (r < valid && kin) ? x[static_cast<size_t>(row0 + r) * d + k0 + c] : 0.f;
+      xs[r][c] = (xrow[r] >= 0 && kin) ? x[static_cast<size_t>(xrow[r]) * d + k0 + c] : 0.f;
       const bool nin = n0 + r < h;
       as[r][c] = (nin && kin) ? W1[static_cast<size_t>(n0 + r) * d + k0 + c] : 0.f;
       bs[r][c] = (nin && kin) ? W3[static_cast<size_t>(n0 + r) * d + k0 + c] : 0.f;
@@ -155,9 +168,19 @@ cudaError_t launch_swiglu_simt_f32(const float* x_perm, const int32_t* offsets,
                                    const float* w1, const float* w3, const float* w2,
                                    const float* row_scale, int N, int d, int h, int E, float* y,
                                    float* H, int* status, cudaStream_t s) {
+  return launch_swiglu_simt_f32_gather(x_perm, N, nullptr, offsets, w1, w3, w2, row_scale, N, d,
+                                       h, E, y, H, status, s);
+}
+
+cudaError_t launch_swiglu_simt_f32_gather(const float* x, int x_rows, const int32_t* src_row,
+                                          const int32_t* offsets, const float* w1,
+                                          const float* w3, const float* w2,
+                                          const float* row_scale, int N, int d, int h, int E,
+                                          float* y, float* H, int* status, cudaStream_t s) {
   const int max_tiles = cdiv(N, SB) + E;   // upper bound over all segmentations
   dim3 g1(max_tiles, cdiv(h, SB));
-  swiglu_up_f32_kernel<<<g1, 256, 0, s>>>(x_perm, offsets, w1, w3, N, d, h, E, H, status);
+  swiglu_up_f32_kernel<<<g1, 256, 0, s>>>(x, src_row, x_rows, offsets, w1, w3, N, d, h, E, H,
+                                          status);
   dim3 g2(max_tiles, cdiv(d, SB));
   swiglu_down_f32_kernel<<<g2, 256, 0, s>>>(H, offsets, w2, row_scale, N, d, h, E, y, status);
   return cudaGetLastError();

@@ -45,7 +45,8 @@ struct TileInfo {
   int a_row;     // first A row (token or routed copy)
   int b_row;     // first B row in the [E * n, K] view of the weights
   int m_valid;   // rows of this tile that belong to the problem / expert
-  int n0;        // first output column
+  int n0;        // first output column (router: the K split)
+  int kb0, kb1;  // K blocks [kb0, kb1) of this tile
 };
 
 struct Args {
@@ -56,14 +57,13 @@ struct Args {
   const int32_t* offsets;    // [E+1] expert segments (grouped)
   int* status;
   // router
-  float* logits_out;
-  int32_t* topk_idx;
-  float* topk_w;
-  int32_t* counts;
-  int top_k;
-  int renorm;
+  float* logits_part;        // [ksplit, T, E] fp32 partial logits
+  int ksplit;                // number of K splits
+  int kb_per_split;          // K blocks per split
   // grouped
   __nv_bfloat16* out;        // H [N, h] (up) or y [N, d] (down)
+  const int32_t* src_row;    // gathered GEMM1: token of every expert-major slot
+  int src_rows;              // gathered GEMM1: rows of x (T); row T reads as zeros
   const float* row_scale;    // down only, may be null
 };
 
@@ -76,127 +76,60 @@ __host__ __device__ constexpr uint32_t tmem_cols_for(int bn) {
                                                      : (2 * bn <= 256) ? 256u : 512u;
 }
 
-// ---------------------------------------------------------------- top-k
-// Running top-KMAX of (score, expert) pairs ordered by score descending then
-// expert ascending; NaN scores count as -inf.  Sentinels carry indices E..
-// so that any real expert, even at -inf, displaces them.
-template <int KMAX>
-struct TopK {
-  float v[KMAX];
-  int i[KMAX];
-  float mx;
-  __device__ __forceinline__ void init(int E) {
-#pragma unroll
-    for (int j = 0; j < KMAX; ++j) {
-      v[j] = -INFINITY;
-      i[j] = E + j;
-    }
-    mx = -INFINITY;
-  }
-  __device__ __forceinline__ void push(float s, int e) {
-    if (s != s) s = -INFINITY;
-    mx = fmaxf(mx, s);
-    float cv = s;
-    int ci = e;
-#pragma unroll
-    for (int j = 0; j < KMAX; ++j) {
-      const bool sw = (cv > v[j]) || (cv == v[j] && ci < i[j]);
-      const float tv = v[j];
-      const int ti = i[j];
-      v[j] = sw ? cv : tv;
-      i[j] = sw ? ci : ti;
-      cv = sw ? tv : cv;
-      ci = sw ? ti : ci;
-    }
-  }
-};
-
-__device__ __forceinline__ float nan_to_neginf(float s) { return (s != s) ? -INFINITY : s; }
-
 // ---------------------------------------------------------------- policies
-// Router: A = x [T, d], B = w_router [E, d] (rows >= E are zero-filled by TMA).
-template <int BN_, int KMAX>
+// Router: A = x [T, d], B = w_router [E, d] (rows >= E are zero-filled by
+// TMA).  A tile is 128 tokens x one slice of the reduction: d is split into
+// `ksplit` ranges so that there are about as many tiles as SMs even for a
+// few hundred tokens, and each tile writes its fp32 partial logits to
+// logits_part[split][t][0..E).  router_topk_kernel adds the splits in a fixed
+// order and does softmax / top-k, one warp per token.
+template <int BN_>
 struct RouterPolicy {
   static constexpr int BN = BN_;
   static constexpr int NUM_B = 1;
-  static constexpr int SCHED_INTS = kMaxExperts + 8;   // per-CTA expert histogram
+  static constexpr bool GATHER_A = false;
+  static constexpr int SCHED_INTS = 8;
 
-  static __device__ void prologue(const Args& a, int* sched) {
-    for (int i = threadIdx.x; i < a.E; i += blockDim.x) sched[i] = 0;
-  }
-  static __device__ int num_tiles(const Args& a, const int*) { return cdiv(a.M, BM); }
+  static __device__ void prologue(const Args&, int*) {}
+  static __device__ int num_tiles(const Args& a, const int*) { return cdiv(a.M, BM) * a.ksplit; }
   static __device__ TileInfo tile_info(const Args& a, const int*, int tile) {
+    const int mt = tile / a.ksplit;
+    const int sp = tile - mt * a.ksplit;
     TileInfo t;
-    t.a_row = tile * BM;
+    t.a_row = mt * BM;
     t.b_row = 0;
     t.m_valid = min(BM, a.M - t.a_row);
-    t.n0 = 0;
+    t.n0 = sp;
+    t.kb0 = sp * a.kb_per_split;
+    t.kb1 = min(cdiv(a.K, BK), t.kb0 + a.kb_per_split);
     return t;
   }
-  static __device__ void epilogue(const Args& a, int* sched, const TileInfo& ti, uint32_t taddr,
+  static __device__ void epilogue(const Args& a, int*, const TileInfo& ti, uint32_t taddr,
                                   int row) {
     const int E = a.E;
     const bool valid = row < ti.m_valid;
-    const int t = ti.a_row + row;
-    TopK<KMAX> tk;
-    tk.init(E);
+    float* dst = a.logits_part + (static_cast<size_t>(ti.n0) * a.M + ti.a_row + row) * E;
+    const bool vec = (E % 4) == 0;
     const int nch = cdiv(E, 32);
-    // pass 1: logits out, running max, top-k
     for (int c = 0; c < nch; ++c) {
       uint32_t r[32];
       tmem_ld32(taddr + c * 32, r);
       tmem_ld_wait();
-      if (valid && a.logits_out) {
-        float* dst = a.logits_out + static_cast<size_t>(t) * E + c * 32;
-        const int ncol = min(32, E - c * 32);
-        if (ncol == 32 && (reinterpret_cast<uintptr_t>(dst) & 15u) == 0) {
+      if (!valid) continue;
+      if (vec && c * 32 + 32 <= E) {
 #pragma unroll
-          for (int q = 0; q < 8; ++q)
-            reinterpret_cast<float4*>(dst)[q] =
-                make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
-                            __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3]));
-        } else {
-          for (int q = 0; q < ncol; ++q) dst[q] = __uint_as_float(r[q]);
-        }
-      }
+        for (int q = 0; q < 8; ++q)
+          reinterpret_cast<float4*>(dst + c * 32)[q] =
+              make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
+                          __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3]));
+      } else {
 #pragma unroll
-      for (int q = 0; q < 32; ++q)
-        if (c * 32 + q < E) tk.push(__uint_as_float(r[q]), c * 32 + q);
-    }
-    // pass 2: softmax denominator over all E
-    float sum = 0.f;
-    for (int c = 0; c < nch; ++c) {
-      uint32_t r[32];
-      tmem_ld32(taddr + c * 32, r);
-      tmem_ld_wait();
-#pragma unroll
-      for (int q = 0; q < 32; ++q)
-        if (c * 32 + q < E) sum += expf(nan_to_neginf(__uint_as_float(r[q])) - tk.mx);
-    }
-    if (!valid) return;
-    float ex[KMAX];
-    float sel = 0.f;
-#pragma unroll
-    for (int j = 0; j < KMAX; ++j) {
-      ex[j] = expf(tk.v[j] - tk.mx);
-      if (j < a.top_k) sel += ex[j];
-    }
-    const float denom = a.renorm ? sel : sum;
-#pragma unroll
-    for (int j = 0; j < KMAX; ++j) {
-      if (j < a.top_k) {
-        const size_t o = static_cast<size_t>(t) * a.top_k + j;
-        a.topk_idx[o] = tk.i[j];
-        a.topk_w[o] = ex[j] / denom;
-        if (a.counts) atomicAdd(&sched[tk.i[j]], 1);
+        for (int q = 0; q < 32; ++q)
+          if (c * 32 + q < E) dst[c * 32 + q] = __uint_as_float(r[q]);
       }
     }
   }
-  static __device__ void finish(const Args& a, int* sched) {
-    if (!a.counts) return;
-    for (int e = threadIdx.x; e < a.E; e += blockDim.x)
-      if (sched[e]) atomicAdd(&a.counts[e], sched[e]);
-  }
+  static __device__ void finish(const Args&, int*) {}
 };
 
 // Grouped problems: schedule over expert segments.  sched layout:
@@ -206,6 +139,7 @@ template <int BN_, int NUM_B_, int NCOLS_PER_TILE>
 struct GroupedSched {
   static constexpr int BN = BN_;
   static constexpr int NUM_B = NUM_B_;
+  static constexpr bool GATHER_A = false;
   static constexpr int SCHED_INTS = 8 + 2 * (kMaxExperts + 1);
 
   static __device__ void prologue(const Args& a, int* sched) {
@@ -272,7 +206,12 @@ struct GroupedSched {
 
 // GEMM1: B0 = w1 rows [e*h + n0, +128), B1 = w3 rows (same), accumulator
 // columns [0,128) = G, [128,256) = U.
-struct UpPolicy : GroupedSched<256, 2, 128> {
+template <bool GATHER>
+struct UpPolicyT : GroupedSched<256, 2, 128> {
+  // With GATHER the A operand is not an expert-major copy of the tokens: the
+  // producer warp reads the 128 rows of a tile straight from x through
+  // src_row with TMA tile::gather4 (4 rows per instruction, one per lane).
+  static constexpr bool GATHER_A = GATHER;
   static __device__ TileInfo tile_info(const Args& a, const int* sched, int tile) {
     int e, nt, mt, cnt, seg0;
     locate(a, sched, tile, e, nt, mt, cnt, seg0);
@@ -281,6 +220,8 @@ struct UpPolicy : GroupedSched<256, 2, 128> {
     t.m_valid = min(BM, cnt - mt * BM);
     t.n0 = nt * 128;
     t.b_row = e * a.n_out + t.n0;
+    t.kb0 = 0;
+    t.kb1 = cdiv(a.K, BK);
     return t;
   }
   static __device__ void epilogue(const Args& a, int*, const TileInfo& ti, uint32_t taddr,
@@ -311,6 +252,8 @@ struct UpPolicy : GroupedSched<256, 2, 128> {
   }
   static __device__ void finish(const Args&, int*) {}
 };
+using UpPolicy = UpPolicyT<false>;
+using UpGatherPolicy = UpPolicyT<true>;
 
 // GEMM2: B = w2 rows [e*d + n0, +256).
 struct DownPolicy : GroupedSched<256, 1, 256> {
@@ -322,6 +265,8 @@ struct DownPolicy : GroupedSched<256, 1, 256> {
     t.m_valid = min(BM, cnt - mt * BM);
     t.n0 = nt * 256;
     t.b_row = e * a.n_out + t.n0;
+    t.kb0 = 0;
+    t.kb1 = cdiv(a.K, BK);
     return t;
   }
   static __device__ void epilogue(const Args& a, int*, const TileInfo& ti, uint32_t taddr,
@@ -421,9 +366,72 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int total = P::num_tiles(args, sched);
-  const int KB = cdiv(args.K, BK);
 
-  if (warp == 0) {
+  if (warp == 0 && P::GATHER_A) {
+    // ------------------------------------ TMA producer, gathered A rows
+    // Lane l fetches rows 4l..4l+3 of every A tile with one tile::gather4
+    // (token ids from src_row; rows outside the segment read row src_rows,
+    // which is past the end of x and comes back as zeros); lane 0 owns the
+    // barriers and the weight loads.
+    const uint64_t pol_b = l2_policy_evict_last();
+    const uint64_t pol_a = l2_policy_evict_last();
+    int stage = 0;
+    uint32_t phase = 0;
+    int issued = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      const TileInfo ti = P::tile_info(args, sched, tile);
+      int rows[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int r = 4 * lane + q;
+        int t = args.src_rows;
+        if (r < ti.m_valid) {
+          const int v = args.src_row[ti.a_row + r];
+          if (static_cast<unsigned>(v) < static_cast<unsigned>(args.src_rows)) t = v;
+        }
+        rows[q] = t;
+      }
+      for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
+        int go = 1;
+        if (lane == 0) go = mbar_wait(empty + stage, phase ^ 1u, abort_flag, args.status) ? 1 : 0;
+        go = __shfl_sync(0xffffffffu, go, 0);
+        if (!go) {
+          ok = false;
+          break;
+        }
+        uint8_t* sa = tiles + stage * L::kStageBytes;
+        uint8_t* sb = sa + kATileBytes;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(full + stage, L::kStageBytes);
+          tma_load_2d(sb, &tmB0, full + stage, kb * BK, ti.b_row, pol_b);
+          if (P::NUM_B == 2)
+            tma_load_2d(sb + L::kBTileBytes / 2, &tmB1, full + stage, kb * BK, ti.b_row, pol_b);
+        }
+        __syncwarp();
+        tma_gather4(sa + lane * 4 * (BK * 2), &tmA, full + stage, kb * BK, rows[0], rows[1],
+                    rows[2], rows[3], pol_a);
+        ++issued;
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    if (lane == 0) {
+      int s = stage;
+      uint32_t ph = phase;
+      for (int i = 0; i < min(issued, STAGES); ++i) {
+        if (s == 0) {
+          s = STAGES - 1;
+          ph ^= 1u;
+        } else {
+          --s;
+        }
+        mbar_wait(full + s, ph, nullptr, args.status);
+      }
+    }
+  } else if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------ TMA producer
       const uint64_t pol_b = l2_policy_evict_last();
@@ -434,7 +442,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         const TileInfo ti = P::tile_info(args, sched, tile);
-        for (int kb = 0; kb < KB; ++kb) {
+        for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
           if (!mbar_wait(empty + stage, phase ^ 1u, abort_flag, args.status)) {
             ok = false;
             break;
@@ -482,7 +490,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(tempty + acc, aph ^ 1u, abort_flag, args.status)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
-        for (int kb = 0; kb < KB; ++kb) {
+        const TileInfo ti = P::tile_info(args, sched, tile);
+        for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
           if (!mbar_wait(full + stage, phase, abort_flag, args.status)) {
             ok = false;
             break;
@@ -493,7 +502,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t bd = sw128_kmajor_desc(sa + kATileBytes);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
-            tc_mma_bf16(d_tmem, ad + 2u * kk, bd + 2u * kk, IDESC, (kb | kk) ? 1u : 0u);
+            tc_mma_bf16(d_tmem, ad + 2u * kk, bd + 2u * kk, IDESC,
+                        (kb != ti.kb0 || kk != 0) ? 1u : 0u);
           tc_commit(empty + stage);
           if (++stage == STAGES) {
             stage = 0;
@@ -592,55 +602,75 @@ cudaError_t launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMa
   return cudaGetLastError();
 }
 
-template <int BN>
-cudaError_t launch_router_bn(const CUtensorMap& a, const CUtensorMap& b, const Args& args,
-                             int grid, cudaStream_t s) {
-  const int k = args.top_k;
-  if (k <= 1) return launch<RouterPolicy<BN, 1>>(a, b, b, args, grid, s);
-  if (k <= 2) return launch<RouterPolicy<BN, 2>>(a, b, b, args, grid, s);
-  if (k <= 4) return launch<RouterPolicy<BN, 4>>(a, b, b, args, grid, s);
-  if (k <= 8) return launch<RouterPolicy<BN, 8>>(a, b, b, args, grid, s);
-  return launch<RouterPolicy<BN, 16>>(a, b, b, args, grid, s);
-}
-
 }  // namespace tc
 
+RouterPlan router_plan(int T, int d) {
+  RouterPlan p{};
+  const int mt = std::max(1, cdiv(T, tc::BM));
+  const int kb = std::max(1, cdiv(d, tc::BK));
+  int split = std::max(1, std::min(kb, cdiv(kRouterTargetTiles, mt)));
+  p.kb_per_split = cdiv(kb, split);
+  p.ksplit = cdiv(kb, p.kb_per_split);   // every split has at least one K block
+  return p;
+}
+
 cudaError_t launch_router_tc(const void* x, const void* w_router, int T, int d, int E,
-                             int top_k, int renorm, float* logits_out, int32_t* topk_idx,
-                             float* topk_w, int32_t* counts, int* status, cudaStream_t s) {
+                             float* logits_part, int* status, cudaStream_t s) {
   using namespace tc;
   const int bn = E <= 32 ? 32 : E <= 64 ? 64 : E <= 128 ? 128 : 256;
   CUtensorMap ta, tb;
   if (!make_tmap(&ta, x, d, T, BM)) return cudaErrorInvalidValue;
   if (!make_tmap(&tb, w_router, d, E, bn)) return cudaErrorInvalidValue;
+  const RouterPlan p = router_plan(T, d);
   Args a{};
   a.M = T;
   a.K = d;
   a.E = E;
   a.n_out = E;
   a.status = status;
-  a.logits_out = logits_out;
-  a.topk_idx = topk_idx;
-  a.topk_w = topk_w;
-  a.counts = counts;
-  a.top_k = top_k;
-  a.renorm = renorm;
-  const int grid = std::min(num_sms(), cdiv(T, BM));
+  a.logits_part = logits_part;
+  a.ksplit = p.ksplit;
+  a.kb_per_split = p.kb_per_split;
+  const int grid = std::min(num_sms(), cdiv(T, BM) * p.ksplit);
   switch (bn) {
-    case 32: return launch_router_bn<32>(ta, tb, a, grid, s);
-    case 64: return launch_router_bn<64>(ta, tb, a, grid, s);
-    case 128: return launch_router_bn<128>(ta, tb, a, grid, s);
-    default: return launch_router_bn<256>(ta, tb, a, grid, s);
+    case 32: return launch<RouterPolicy<32>>(ta, tb, tb, a, grid, s);
+    case 64: return launch<RouterPolicy<64>>(ta, tb, tb, a, grid, s);
+    case 128: return launch<RouterPolicy<128>>(ta, tb, tb, a, grid, s);
+    default: return launch<RouterPolicy<256>>(ta, tb, tb, a, grid, s);
   }
 }
+
+// Grouped SwiGLU with GEMM1's A operand gathered from x [T, d] through
+// src_row (no expert-major copy of the tokens in memory).
+static cudaError_t swiglu_tc_impl(const void* a_src, int a_rows, const int32_t* src_row,
+                                  const int32_t* offsets, const void* w1, const void* w3,
+                                  const void* w2, const float* row_scale, int N, int d, int h,
+                                  int E, void* y, void* H, int* status, cudaStream_t s);
 
 cudaError_t launch_swiglu_tc(const void* x_perm, const int32_t* offsets, const void* w1,
                              const void* w3, const void* w2, const float* row_scale, int N,
                              int d, int h, int E, void* y, void* H, int* status,
                              cudaStream_t s) {
+  return swiglu_tc_impl(x_perm, N, nullptr, offsets, w1, w3, w2, row_scale, N, d, h, E, y, H,
+                        status, s);
+}
+
+cudaError_t launch_swiglu_tc_gather(const void* x, int T, const int32_t* src_row,
+                                    const int32_t* offsets, const void* w1, const void* w3,
+                                    const void* w2, const float* row_scale, int N, int d, int h,
+                                    int E, void* y, void* H, int* status, cudaStream_t s) {
+  return swiglu_tc_impl(x, T, src_row, offsets, w1, w3, w2, row_scale, N, d, h, E, y, H, status,
+                        s);
+}
+
+static cudaError_t swiglu_tc_impl(const void* a_src, int a_rows, const int32_t* src_row,
+                                  const int32_t* offsets, const void* w1, const void* w3,
+                                  const void* w2, const float* row_scale, int N, int d, int h,
+                                  int E, void* y, void* H, int* status, cudaStream_t s) {
   using namespace tc;
   CUtensorMap tx, t1, t3, th, t2;
-  if (!make_tmap(&tx, x_perm, d, N, BM)) return cudaErrorInvalidValue;
+  const bool gather = src_row != nullptr;
+  if (!make_tmap(&tx, a_src, d, a_rows, gather ? 1 : BM)) return cudaErrorInvalidValue;
   if (!make_tmap(&t1, w1, d, static_cast<uint64_t>(E) * h, 128)) return cudaErrorInvalidValue;
   if (!make_tmap(&t3, w3, d, static_cast<uint64_t>(E) * h, 128)) return cudaErrorInvalidValue;
   if (!make_tmap(&th, H, h, N, BM)) return cudaErrorInvalidValue;
@@ -655,8 +685,11 @@ cudaError_t launch_swiglu_tc(const void* x_perm, const int32_t* offsets, const v
   a.K = d;
   a.n_out = h;
   a.out = static_cast<__nv_bfloat16*>(H);
+  a.src_row = src_row;
+  a.src_rows = a_rows;
   int grid = static_cast<int>(std::min<long long>(num_sms(), 1LL * max_mt * cdiv(h, 128)));
-  cudaError_t e = launch<UpPolicy>(tx, t1, t3, a, grid, s);
+  cudaError_t e = gather ? launch<UpGatherPolicy>(tx, t1, t3, a, grid, s)
+                         : launch<UpPolicy>(tx, t1, t3, a, grid, s);
   if (e != cudaSuccess) return e;
   // GEMM2: y = H w2^T (* row_scale)
   a.K = h;

@@ -282,15 +282,20 @@ def test_regroup_bad_counts_sets_status(M):
 
 
 # ----------------------------------------------------------- grouped SwiGLU
-def swiglu_case(M, T, d, E, k, h, seed, dtype, row_scale=False, logits=None, sample=None):
+def swiglu_case(M, T, d, E, k, h, seed, dtype, row_scale=False, logits=None, sample=None,
+                gather=False):
     x, wr, w1, w3, w2 = small_layer(T, d, E, k, h, seed, dtype, device="cpu")
     L = W.make_logits(T, E, k, seed=seed) if logits is None else logits
     idx, w, *_ = O.router_topk(k, True, logits=L)
     c, off, src, dst = O.dispatch(idx, E)
     xp = x[torch.from_numpy(src)].contiguous()
     rs = torch.rand(T * k, generator=torch.Generator().manual_seed(seed)) if row_scale else None
-    gy, ws = M.grouped_swiglu(xp.cuda(), i32(off), w1.cuda(), w3.cuda(), w2.cuda(),
-                              None if rs is None else rs.cuda())
+    if gather:
+        gy, ws = M.grouped_swiglu_gather(x.cuda(), i32(src), i32(off), w1.cuda(), w3.cuda(),
+                                         w2.cuda(), None if rs is None else rs.cuda())
+    else:
+        gy, ws = M.grouped_swiglu(xp.cuda(), i32(off), w1.cuda(), w3.cuda(), w2.cuda(),
+                                  None if rs is None else rs.cuda())
     assert M.device_status(ws) == 0
     if sample is None:
         ref = O.grouped_swiglu(xp, off, w1, w3, w2, None if rs is None else rs.numpy())
@@ -316,14 +321,28 @@ def swiglu_case(M, T, d, E, k, h, seed, dtype, row_scale=False, logits=None, sam
     (517, 192, 130, 4, 128),    # many experts, empty experts
 ])
 @pytest.mark.parametrize("row_scale", [False, True])
-def test_grouped_swiglu_bf16_shapes(M, T, d, E, k, h, row_scale):
-    swiglu_case(M, T, d, E, k, h, seed=T + d, dtype=torch.bfloat16, row_scale=row_scale)
+@pytest.mark.parametrize("gather", [False, True])
+def test_grouped_swiglu_bf16_shapes(M, T, d, E, k, h, row_scale, gather):
+    swiglu_case(M, T, d, E, k, h, seed=T + d, dtype=torch.bfloat16, row_scale=row_scale,
+                gather=gather)
 
 
 @pytest.mark.parametrize("row_scale", [False, True])
-def test_grouped_swiglu_f32(M, row_scale):
-    swiglu_case(M, 256, 128, 8, 2, 256, seed=0, dtype=torch.float32, row_scale=row_scale)
-    swiglu_case(M, 77, 36, 5, 3, 20, seed=1, dtype=torch.float32, row_scale=row_scale)
+@pytest.mark.parametrize("gather", [False, True])
+def test_grouped_swiglu_f32(M, row_scale, gather):
+    swiglu_case(M, 256, 128, 8, 2, 256, seed=0, dtype=torch.float32, row_scale=row_scale,
+                gather=gather)
+    swiglu_case(M, 77, 36, 5, 3, 20, seed=1, dtype=torch.float32, row_scale=row_scale,
+                gather=gather)
+
+
+@pytest.mark.parametrize("cfg", [1, 3, 4])
+def test_grouped_swiglu_gather_full_size_sampled(M, cfg):
+    """Workload sizes, the launch the forward uses (rows gathered from x),
+    checked on 256 sampled output rows."""
+    c = W.config(cfg)
+    swiglu_case(M, c.T, c.d, c.E, c.top_k, c.h, seed=c.seed, dtype=torch.bfloat16, sample=256,
+                gather=True)
 
 
 def test_grouped_swiglu_all_rows_one_expert(M):
