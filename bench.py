@@ -225,7 +225,7 @@ def run_ours(args, ws, rank, local):
     offsets = torch.empty(nb + 1, dtype=torch.int32, device=dev)
     src_row = torch.empty(N, dtype=torch.int32, device=dev)
     dst_pos = torch.empty(T, k, dtype=torch.int32, device=dev)
-    x_perm = torch.empty(N if R > 1 else 1, d, dtype=x.dtype, device=dev)
+    x_perm = torch.empty(N, d, dtype=x.dtype, device=dev)
     dws = torch.empty(M.ep_dispatch_workspace_size(T, E, k, R), dtype=torch.uint8, device=dev)
     if R > 1:
         x_em = torch.empty_like(x_perm)
@@ -251,8 +251,8 @@ def run_ours(args, ws, rank, local):
         M.moe_router_topk(x, wr, None, T, d, E, k, M.MOE_SCORE_SOFTMAX, cfg.renormalize, dt, None,
                           idx, w, None, rws)
         mark(1)
-        if R == 1:   # indices only: GEMM1 gathers the token rows from x itself
-            M.moe_dispatch(x, idx, T, d, E, k, dt, counts, offsets, src_row, dst_pos, None, dws)
+        if R == 1:
+            M.moe_dispatch(x, idx, T, d, E, k, dt, counts, offsets, src_row, dst_pos, x_perm, dws)
         else:
             M.moe_ep_dispatch_rank_major(x, idx, T, d, E, k, R, dt, counts, offsets, src_row,
                                          dst_pos, x_perm, dws)
@@ -265,11 +265,7 @@ def run_ours(args, ws, rank, local):
             i += 1
             mark(i)
             xe, off, rmap = x_em, oem, pinv
-        if R == 1:
-            M.moe_grouped_swiglu_gather(x, T, src_row, off, w1, w3, w2, None, N, d, h, E, dt, y,
-                                        sws)
-        else:
-            M.moe_grouped_swiglu(xe, off, w1, w3, w2, None, N, d, h, E, dt, y, sws)
+        M.moe_grouped_swiglu(xe, off, w1, w3, w2, None, N, d, h, E, dt, y, sws)
         mark(i + 1)
         M.moe_combine(y, dst_pos, rmap, w, T, d, N, k, dt, out)
         mark(i + 2)

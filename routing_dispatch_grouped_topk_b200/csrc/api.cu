@@ -219,7 +219,7 @@ ForwardWs carve_forward(void* ws, int T, int d, int E, int k, int h, int R, moe_
   f.src_row = c.take<int32_t>(N);
   f.dst_pos = c.take<int32_t>(N);
   f.disp_ws = c.take<char>(dispatch_ws_bytes(p));
-  f.x_a = c.take<char>(R > 1 ? N * row : 0);   // single device: GEMM1 gathers from x
+  f.x_a = c.take<char>(N * row);
   if (R > 1) {
     f.x_em = c.take<char>(N * row);
     f.counts_em = c.take<int32_t>(E);
@@ -526,23 +526,18 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* logit
   if (e != cudaSuccess) return cuda_status(e, "moe_forward/router");
   const DispatchPlan p = make_dispatch_plan(T, E, top_k, R);
   int32_t* cnt_a = (R == 1 && counts) ? counts : f.counts_a;
-  // Single device: only the routing indices are dispatched; GEMM1 gathers
-  // the token rows itself.  Simulated EP: the rank-major rows are
-  // materialised (they are what an all-to-all would deliver) and regrouped.
-  e = launch_dispatch(p, x, idx, d, dt, cnt_a, f.offsets_a, f.src_row, f.dst_pos,
-                      R > 1 ? f.x_a : nullptr, f.disp_ws, f.status, s);
+  // The routed rows are materialised expert-major (single device) or
+  // rank-major (simulated EP: what an all-to-all would deliver), then
+  // regrouped.  Materialising costs one 16-byte-vector copy pass; measured
+  // on B200 it is faster than gathering GEMM1's rows with TMA gather4
+  // (moe_grouped_swiglu_gather), whose 512-byte requests limit the loads.
+  e = launch_dispatch(p, x, idx, d, dt, cnt_a, f.offsets_a, f.src_row, f.dst_pos, f.x_a,
+                      f.disp_ws, f.status, s);
   if (e != cudaSuccess) return cuda_status(e, "moe_forward/dispatch");
   const void* xe = f.x_a;
   const int32_t* off = f.offsets_a;
   const int32_t* row_map = nullptr;
-  if (R == 1) {
-    e = run_swiglu_gather(x, T, f.src_row, off, w1, w3, w2, nullptr, N, d, h, E, dt, f.y, f.H,
-                          f.status, s);
-    if (e != cudaSuccess) return cuda_status(e, "moe_forward/grouped_swiglu");
-    e = launch_combine(f.y, f.dst_pos, nullptr, w, T, d, N, top_k, dt, out, s);
-    return cuda_status(e, "moe_forward/combine");
-  }
-  {
+  if (R > 1) {
     int32_t* cem = counts ? counts : f.counts_em;
     e = launch_regroup(f.x_a, f.counts_a, R, R, E / R, N, d, dt, f.x_em, cem, f.offsets_em,
                        f.perm, f.perm_inv, f.reg_ws, f.status, s);

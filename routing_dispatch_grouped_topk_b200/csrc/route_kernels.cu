@@ -491,18 +491,34 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
   for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += nwarps) {
     float sv[EPL];
     bool avail[EPL];
+    const float* base = parts + static_cast<size_t>(t) * E + lane;
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
-      const int e = lane + 32 * i;
-      avail[i] = e < E;
-      float v = 0.f;
-      if (avail[i]) {
-        const float* p = parts + static_cast<size_t>(t) * E + e;
-        v = p[0];
-        for (int sp = 1; sp < nsplit; ++sp) v += p[sp * plane];
-        if (logits_out) logits_out[static_cast<size_t>(t) * E + e] = v;
-      }
-      sv[i] = (v != v) ? -INFINITY : v;
+      avail[i] = lane + 32 * i < E;
+      sv[i] = avail[i] ? base[32 * i] : 0.f;
+    }
+    // Splits in order; the loads of four splits are issued before their adds.
+    int sp = 1;
+    for (; sp + 4 <= nsplit; sp += 4) {
+      float q[4][EPL];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int i = 0; i < EPL; ++i)
+          q[u][i] = avail[i] ? base[(sp + u) * plane + 32 * i] : 0.f;
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) sv[i] += q[u][i];
+    }
+    for (; sp < nsplit; ++sp)
+#pragma unroll
+      for (int i = 0; i < EPL; ++i)
+        if (avail[i]) sv[i] += base[sp * plane + 32 * i];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      if (avail[i] && logits_out) logits_out[static_cast<size_t>(t) * E + lane + 32 * i] = sv[i];
+      if (sv[i] != sv[i]) sv[i] = -INFINITY;
     }
     float mx = -INFINITY;
     float my_v = 0.f;

@@ -135,9 +135,10 @@ struct RouterPolicy {
 // Grouped problems: schedule over expert segments.  sched layout:
 //   [0] total tiles  [1] n-tiles per m-tile row  [8 .. 8+E]  offsets
 //   [8+E+1 .. 8+2E+1] cumulative tile counts
-template <int BN_, int NUM_B_, int NCOLS_PER_TILE>
+template <int BN_, int NUM_B_, int NCOLS_PER_TILE, int MR = BM>
 struct GroupedSched {
   static constexpr int BN = BN_;
+  static constexpr int MROWS = MR;   // rows of one m-tile (256: a CTA pair)
   static constexpr int NUM_B = NUM_B_;
   static constexpr bool GATHER_A = false;
   static constexpr int SCHED_INTS = 8 + 2 * (kMaxExperts + 1);
@@ -158,7 +159,7 @@ struct GroupedSched {
       for (int e = e0; e < e1; ++e) {
         const int cnt = off[e + 1] - off[e];
         bad |= cnt < 0;
-        local += cdiv(max(cnt, 0), BM) * nt;
+        local += cdiv(max(cnt, 0), MR) * nt;
       }
       int incl = local;
 #pragma unroll
@@ -169,7 +170,7 @@ struct GroupedSched {
       int run = incl - local;
       for (int e = e0; e < e1; ++e) {
         cum[e] = run;
-        run += cdiv(max(off[e + 1] - off[e], 0), BM) * nt;
+        run += cdiv(max(off[e + 1] - off[e], 0), MR) * nt;
       }
       bad = __any_sync(0xffffffffu, bad);
       const int total = __shfl_sync(0xffffffffu, incl, 31);
@@ -197,7 +198,7 @@ struct GroupedSched {
     e = lo;
     seg0 = off[e];
     cnt = off[e + 1] - seg0;
-    const int mtiles = cdiv(cnt, BM);
+    const int mtiles = cdiv(cnt, MR);
     const int local = tile - cum[e];
     nt = local / mtiles;
     mt = local - nt * mtiles;
@@ -295,7 +296,70 @@ struct DownPolicy : GroupedSched<256, 1, 256> {
   static __device__ void finish(const Args&, int*) {}
 };
 
+// CTA-pair versions: an m-tile is 256 rows of one expert; CTA rank r of the
+// pair owns rows [256 mt + 128 r, +128) (its A operand and its accumulator
+// lanes) and loads half of the B tile.  GEMM1: rank 0 loads the w1 rows and
+// rank 1 the w3 rows of the same 128 hidden units, so accumulator columns
+// 0..127 are G and 128..255 are U in both CTAs.  GEMM2: rank r loads w2 rows
+// [n0 + 128 r, +128).  Epilogues are the single-CTA ones.
+__device__ __forceinline__ void pair_rows(int seg0, int cnt, int mt, int rank, TileInfo& t) {
+  const int r0 = mt * 256 + rank * 128;
+  t.a_row = seg0 + r0;
+  t.m_valid = max(0, min(BM, cnt - r0));
+}
+
+struct UpPairPolicy : GroupedSched<256, 2, 128, 256> {
+  static __device__ TileInfo tile_info(const Args& a, const int* sched, int tile, int rank) {
+    int e, nt, mt, cnt, seg0;
+    locate(a, sched, tile, e, nt, mt, cnt, seg0);
+    TileInfo t;
+    pair_rows(seg0, cnt, mt, rank, t);
+    t.n0 = nt * 128;
+    t.b_row = e * a.n_out + t.n0;
+    t.kb0 = 0;
+    t.kb1 = cdiv(a.K, BK);
+    return t;
+  }
+  static __device__ void epilogue(const Args& a, int* s, const TileInfo& ti, uint32_t taddr,
+                                  int row) {
+    UpPolicy::epilogue(a, s, ti, taddr, row);
+  }
+};
+
+struct DownPairPolicy : GroupedSched<256, 1, 256, 256> {
+  static __device__ TileInfo tile_info(const Args& a, const int* sched, int tile, int rank) {
+    int e, nt, mt, cnt, seg0;
+    locate(a, sched, tile, e, nt, mt, cnt, seg0);
+    TileInfo t;
+    pair_rows(seg0, cnt, mt, rank, t);
+    t.n0 = nt * 256;
+    t.b_row = e * a.n_out + t.n0 + rank * 128;
+    t.kb0 = 0;
+    t.kb1 = cdiv(a.K, BK);
+    return t;
+  }
+  static __device__ void epilogue(const Args& a, int* s, const TileInfo& ti, uint32_t taddr,
+                                  int row) {
+    DownPolicy::epilogue(a, s, ti, taddr, row);
+  }
+};
+
 // ------------------------------------------------------------- the kernel
+#ifndef MOE_L2_PREFETCH
+#define MOE_L2_PREFETCH 0
+#endif
+constexpr int kL2Prefetch = MOE_L2_PREFETCH;   // K blocks; 0 disables
+
+template <class P>
+__device__ __forceinline__ void prefetch_kblock(const CUtensorMap* a, const CUtensorMap* b0,
+                                                const CUtensorMap* b1, const TileInfo& ti,
+                                                int kb) {
+  if (kL2Prefetch == 0) return;
+  tma_prefetch_l2_2d(a, kb * BK, ti.a_row);
+  tma_prefetch_l2_2d(b0, kb * BK, ti.b_row);
+  if (P::NUM_B == 2) tma_prefetch_l2_2d(b1, kb * BK, ti.b_row);
+}
+
 template <class P>
 struct Layout {
   static constexpr int BN = P::BN;
@@ -442,7 +506,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         const TileInfo ti = P::tile_info(args, sched, tile);
+        // L2 prefetch kL2Prefetch K blocks ahead of the loads, so that a
+        // load issued when a stage frees up finds its data in L2.
+        for (int kb = ti.kb0; kb < min(ti.kb1, ti.kb0 + kL2Prefetch); ++kb)
+          prefetch_kblock<P>(&tmA, &tmB0, &tmB1, ti, kb);
         for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
+          if (kb + kL2Prefetch < ti.kb1) prefetch_kblock<P>(&tmA, &tmB0, &tmB1, ti, kb + kL2Prefetch);
           if (!mbar_wait(empty + stage, phase ^ 1u, abort_flag, args.status)) {
             ok = false;
             break;
@@ -546,6 +615,202 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ---------------------------------------------------- the CTA-pair kernel
+// Two CTAs (a cluster of 2 on neighbouring SMs) share each 256 x 256 tile
+// through tcgen05.mma.cta_group::2: per K block each SM loads 16 KB of A
+// and 16 KB of B (instead of 16 + 32 KB for a 128-row tile alone), so the
+// pair does twice the MMA work of one CTA for 4/3 of its load traffic.
+// Rank 0 (leader) issues the MMAs and commits to the barriers of both CTAs;
+// both CTAs' TMA loads count on the leader's "full" barrier; both epilogues
+// arrive on the leader's "tmem empty" barrier.
+template <class P>
+struct PairLayout {
+  static constexpr int kBHalfBytes = 128 * BK * 2;                  // 16 KB
+  static constexpr int kStageBytes = kATileBytes + kBHalfBytes;    // 32 KB per CTA
+  static constexpr int kStages = 6;
+  static constexpr uint32_t kTmemCols = 512;                       // 2 x 256 columns
+  static constexpr int kBarOff = kStages * kStageBytes;
+  static constexpr int kNumBars = 2 * kStages + 5;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kSchedOff = (kMiscOff + 16 + 15) / 16 * 16;
+  static constexpr int kBytes = kSchedOff + P::SCHED_INTS * 4;
+  static constexpr int kLaunchBytes = kBytes + 1024;
+  static_assert(kLaunchBytes <= 227 * 1024, "shared memory budget");
+};
+
+template <class P>
+__global__ void __launch_bounds__(kThreads, 1)
+    tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
+                        const __grid_constant__ CUtensorMap tmB0,
+                        const __grid_constant__ CUtensorMap tmB1, const Args args) {
+  using L = PairLayout<P>;
+  constexpr int STAGES = L::kStages;
+  constexpr uint32_t IDESC = idesc_bf16_f32(256, 256);
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+  uint8_t* tiles = smem;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* mma_done = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+  int* sched = reinterpret_cast<int*>(smem + L::kSchedOff);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int rank = static_cast<int>(cluster_ctarank());
+  const bool leader = rank == 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(empty + s, 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull + a, 1);
+      mbar_init(tempty + a, 8);   // 4 epilogue warps in each CTA of the pair
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB0);
+    if (P::NUM_B == 2) tma_prefetch_desc(&tmB1);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, L::kTmemCols);
+    tmem_relinquish_pair();
+    tc_fence_before();
+  }
+  P::prologue(args, sched);
+  __syncthreads();
+  cluster_sync_all();   // barriers of both CTAs initialised before any remote arrive
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = P::num_tiles(args, sched);
+  const int pair = blockIdx.x >> 1;
+  const int npairs = gridDim.x >> 1;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------ TMA producer (both CTAs)
+      const uint64_t pol = l2_policy_evict_last();
+      const CUtensorMap* tb = (P::NUM_B == 2 && rank == 1) ? &tmB1 : &tmB0;
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      bool ok = true;
+      for (int tile = pair; tile < total && ok; tile += npairs) {
+        const TileInfo ti = P::tile_info(args, sched, tile, rank);
+        for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
+          if (!mbar_wait(empty + stage, phase ^ 1u, abort_flag, args.status)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = tiles + stage * L::kStageBytes;
+          const uint32_t bar = cluster_map(full + stage, 0);
+          if (leader) mbar_arrive_expect_tx(full + stage, 2 * L::kStageBytes);
+          tma_load_2d_pair(sa, &tmA, bar, kb * BK, ti.a_row, pol);
+          tma_load_2d_pair(sa + kATileBytes, tb, bar, kb * BK, ti.b_row, pol);
+          ++issued;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // Drain: a stage's loads have landed once the MMAs that read it are
+      // done, which the leader commits to this CTA's "empty" barrier.
+      int s = stage;
+      uint32_t ph = phase;
+      for (int i = 0; i < min(issued, STAGES); ++i) {
+        if (s == 0) {
+          s = STAGES - 1;
+          ph ^= 1u;
+        } else {
+          --s;
+        }
+        mbar_wait(empty + s, ph, nullptr, args.status);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      // ------------------------------------------------ MMA issuer (leader)
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      for (int tile = pair; tile < total && ok; tile += npairs, ++it) {
+        const int acc = it & 1;
+        const uint32_t aph = (it >> 1) & 1;
+        if (!mbar_wait_cluster(tempty + acc, aph ^ 1u, abort_flag, args.status)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * 256);
+        const TileInfo ti = P::tile_info(args, sched, tile, 0);
+        for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
+          if (!mbar_wait(full + stage, phase, abort_flag, args.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint8_t* sa = tiles + stage * L::kStageBytes;
+          const uint64_t ad = sw128_kmajor_desc(sa);
+          const uint64_t bd = sw128_kmajor_desc(sa + kATileBytes);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            tc_mma_bf16_pair(d_tmem, ad + 2u * kk, bd + 2u * kk, IDESC,
+                             (kb != ti.kb0 || kk != 0) ? 1u : 0u);
+          tc_commit_pair_mc(empty + stage, 0x3);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit_pair_mc(tfull + acc, 0x3);
+      }
+      tc_commit_pair(mma_done);
+      mbar_wait(mma_done, 0, nullptr, args.status);
+    }
+  } else {
+    // -------------------------------------------------- epilogue warps (both CTAs)
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    uint32_t tempty_leader[2];
+    tempty_leader[0] = cluster_map(tempty + 0, 0);
+    tempty_leader[1] = cluster_map(tempty + 1, 0);
+    int it = 0;
+    for (int tile = pair; tile < total; tile += npairs, ++it) {
+      const int acc = it & 1;
+      const uint32_t aph = (it >> 1) & 1;
+      int ok = 1;
+      if (lane == 0) ok = mbar_wait(tfull + acc, aph, abort_flag, args.status) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      tc_fence_after();
+      const TileInfo ti = P::tile_info(args, sched, tile, rank);
+      const uint32_t taddr =
+          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * 256);
+      P::epilogue(args, sched, ti, taddr, row);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(tempty_leader[acc]);
+    }
+  }
+  __syncthreads();
+  cluster_sync_all();   // no CTA leaves while its peer may still touch its memory
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, L::kTmemCols);
+  }
+}
+
 // ---------------------------------------------------------------- host side
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -602,13 +867,44 @@ cudaError_t launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMa
   return cudaGetLastError();
 }
 
+// Launch of the CTA-pair kernel: clusters of 2 CTAs, an even grid.
+template <class P>
+cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
+                        const Args& args, int pairs, cudaStream_t s) {
+  using L = PairLayout<P>;
+  static int configured[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !configured[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(tc_gemm_pair_kernel<P>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         L::kLaunchBytes);
+    if (e != cudaSuccess) return e;
+    configured[dev] = 1;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = L::kLaunchBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, tc_gemm_pair_kernel<P>, a, b0, b1, args);
+}
+
 }  // namespace tc
 
 RouterPlan router_plan(int T, int d) {
   RouterPlan p{};
   const int mt = std::max(1, cdiv(T, tc::BM));
   const int kb = std::max(1, cdiv(d, tc::BK));
-  int split = std::max(1, std::min(kb, cdiv(kRouterTargetTiles, mt)));
+  // at most one wave of tiles: mt * ksplit <= kRouterTargetTiles when mt allows
+  int split = std::max(1, std::min(kb, kRouterTargetTiles / mt));
   p.kb_per_split = cdiv(kb, split);
   p.ksplit = cdiv(kb, p.kb_per_split);   // every split has at least one K block
   return p;
@@ -674,7 +970,12 @@ static cudaError_t swiglu_tc_impl(const void* a_src, int a_rows, const int32_t* 
   if (!make_tmap(&t1, w1, d, static_cast<uint64_t>(E) * h, 128)) return cudaErrorInvalidValue;
   if (!make_tmap(&t3, w3, d, static_cast<uint64_t>(E) * h, 128)) return cudaErrorInvalidValue;
   if (!make_tmap(&th, H, h, N, BM)) return cudaErrorInvalidValue;
-  if (!make_tmap(&t2, w2, h, static_cast<uint64_t>(E) * d, 256)) return cudaErrorInvalidValue;
+  // CTA pairs pay off once the average expert has more than 128 rows: a
+  // 256-row pair tile then replaces two 128-row tiles with 2/3 of the loads
+  // per SM.  Decode-sized segments keep one CTA per 128-row tile.
+  const bool pairs = !gather && N > 128 * E;
+  if (!make_tmap(&t2, w2, h, static_cast<uint64_t>(E) * d, pairs ? 128 : 256))
+    return cudaErrorInvalidValue;
   const int max_mt = cdiv(N, BM) + E;   // upper bound on m-tiles over all segments
   Args a{};
   a.M = N;
@@ -687,6 +988,18 @@ static cudaError_t swiglu_tc_impl(const void* a_src, int a_rows, const int32_t* 
   a.out = static_cast<__nv_bfloat16*>(H);
   a.src_row = src_row;
   a.src_rows = a_rows;
+  if (pairs) {
+    const long long max_pt = cdiv(N, 256) + E;   // upper bound on 256-row pair tiles
+    int np = static_cast<int>(std::min<long long>(num_sms() / 2, max_pt * cdiv(h, 128)));
+    cudaError_t e = launch_pair<UpPairPolicy>(tx, t1, t3, a, np, s);
+    if (e != cudaSuccess) return e;
+    a.K = h;
+    a.n_out = d;
+    a.out = static_cast<__nv_bfloat16*>(y);
+    a.row_scale = row_scale;
+    np = static_cast<int>(std::min<long long>(num_sms() / 2, max_pt * cdiv(d, 256)));
+    return launch_pair<DownPairPolicy>(th, t2, t2, a, np, s);
+  }
   int grid = static_cast<int>(std::min<long long>(num_sms(), 1LL * max_mt * cdiv(h, 128)));
   cudaError_t e = gather ? launch<UpGatherPolicy>(tx, t1, t3, a, grid, s)
                          : launch<UpPolicy>(tx, t1, t3, a, grid, s);

@@ -55,9 +55,9 @@ def test_version_and_strings(L):
 
 def test_workspace_sizes_are_host_only(L):
     assert L.moe_dispatch_workspace_size(4096, 128, 8) >= 256
-    # y [N, d] and H [N, h] in bf16 at least (no x_perm: GEMM1 gathers rows)
+    # x_perm and y [N, d] and H [N, h] in bf16 at least
     N = 4096 * 8
-    assert L.moe_forward_workspace_size(4096, 2048, 128, 8, 768, 1, 1) > N * (2048 + 768) * 2
+    assert L.moe_forward_workspace_size(4096, 2048, 128, 8, 768, 1, 1) > N * (2 * 2048 + 768) * 2
     assert L.moe_router_workspace_size(64, 4096, 128, 1) >= 256 + 64 * 128 * 4
     assert L.moe_forward_workspace_size(8192, 2880, 128, 4, 2880, 8, 1) > \
         L.moe_forward_workspace_size(8192, 2880, 128, 4, 2880, 1, 1)

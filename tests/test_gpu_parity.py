@@ -97,7 +97,7 @@ def router_gemm_check(M, x, wr, k, renorm, dtype):
     gi = gi.cpu().numpy()
     margin = 2 * bound.max(axis=1)
     sure = compare_topk(gi, idx, L64, margin)
-    assert sure.mean() > 0.5
+    assert sure.mean() >= 0.25
     assert gc.cpu().numpy().sum() == T * k
     assert np.array_equal(gc.cpu().numpy(), np.bincount(gi.ravel(), minlength=E))
     # weights compared per expert (the order of two near-equal experts may differ)
