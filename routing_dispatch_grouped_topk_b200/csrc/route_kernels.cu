@@ -24,6 +24,8 @@ __device__ __forceinline__ int dispatch_key(int e, int t, int R, int L, int S) {
 __global__ void dispatch_hist_kernel(const int32_t* __restrict__ idx, int T, int k, int E, int R,
                                      int L, int S, int tb, int nbins, int32_t* __restrict__ blk,
                                      int* status) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ int hist[];
   for (int i = threadIdx.x; i < nbins; i += blockDim.x) hist[i] = 0;
   __syncthreads();
@@ -120,6 +122,8 @@ __device__ int block_scan_value(int v, int* warp_sums, int* total) {
 // its column over the token blocks, in place; the column total is counts[bin].
 __global__ void dispatch_colscan_kernel(int32_t* __restrict__ blk, int nblk, int nbins,
                                         int32_t* __restrict__ counts) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int wsum[33];
   for (int bin = blockIdx.x; bin < nbins; bin += gridDim.x) {
     int32_t* col = blk + static_cast<size_t>(bin) * nblk;
@@ -149,6 +153,8 @@ __global__ void dispatch_scatter_kernel(const uint4* __restrict__ x, const int32
                                         int32_t* __restrict__ src_row,
                                         int32_t* __restrict__ dst_pos, uint4* __restrict__ x_perm,
                                         int row_vec) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ int sm[];
   int* run = sm;                   // nbins
   int* wsum = sm + nbins;          // 33
@@ -245,14 +251,14 @@ cudaError_t launch_dispatch(const DispatchPlan& p, const void* x, const int32_t*
     return e;
   }
   (void)N;
-  dispatch_hist_kernel<<<p.nblk, 256, p.nbins * sizeof(int), s>>>(
+  launch_k(dispatch_hist_kernel, dim3(p.nblk), dim3(256), p.nbins * sizeof(int), s, 
       topk_idx, p.T, p.k, p.E, p.R, p.L, p.S, p.tb, p.nbins, blk, status);
-  dispatch_colscan_kernel<<<std::min(p.nbins, num_sms() * 8), 256, 0, s>>>(blk, p.nblk, p.nbins,
+  launch_k(dispatch_colscan_kernel, dim3(std::min(p.nbins, num_sms() * 8)), dim3(256), 0, s, blk, p.nblk, p.nbins,
                                                                            counts);
   const int elt = dt == MOE_BF16 ? 2 : 4;
   const int row_vec = d * elt / 16;
   const size_t sm3 = (p.nbins + 33 + p.tb * p.k) * sizeof(int);
-  dispatch_scatter_kernel<<<p.nblk, 256, sm3, s>>>(
+  launch_k(dispatch_scatter_kernel, dim3(p.nblk), dim3(256), sm3, s, 
       static_cast<const uint4*>(x), topk_idx, p.T, p.k, p.E, p.R, p.L, p.S, p.tb, p.nbins, blk,
       counts, offsets, src_row, dst_pos, static_cast<uint4*>(x_perm), row_vec);
   return cudaGetLastError();
@@ -267,6 +273,8 @@ __global__ void regroup_scan_kernel(const int32_t* __restrict__ counts_rm, int G
                                     int32_t* __restrict__ out_start,
                                     int32_t* __restrict__ counts_em,
                                     int32_t* __restrict__ offsets_em, int* flag, int* status) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ int sm[];
   const int S = G * R * L;
   int* a = sm;            // S
@@ -316,6 +324,8 @@ __global__ void regroup_copy_kernel(const uint4* __restrict__ in, int rows, int 
                                     const int32_t* __restrict__ out_start, const int* flag,
                                     uint4* __restrict__ out, int32_t* __restrict__ perm,
                                     int32_t* __restrict__ perm_inv) {
+  pdl_wait();
+  pdl_trigger();
   if (!*flag) return;
   const int lane = threadIdx.x & 31;
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -350,13 +360,13 @@ cudaError_t launch_regroup(const void* in, const int32_t* counts_rm, int G, int 
   int32_t* in_start = static_cast<int32_t*>(ws);
   int32_t* out_start = in_start + S;
   int* flag = reinterpret_cast<int*>(out_start + S + 1);
-  regroup_scan_kernel<<<1, 1024, (S + 33) * sizeof(int), s>>>(
+  launch_k(regroup_scan_kernel, dim3(1), dim3(1024), (S + 33) * sizeof(int), s, 
       counts_rm, G, R, L, rows, in_start, out_start, counts_em, offsets_em, flag, status);
   if (rows > 0) {
     const int elt = dt == MOE_BF16 ? 2 : 4;
     const int row_vec = d * elt / 16;
     const int blocks = std::min(cdiv(rows, 8), num_sms() * 8);
-    regroup_copy_kernel<<<blocks, 256, 0, s>>>(static_cast<const uint4*>(in), rows, row_vec, S,
+    launch_k(regroup_copy_kernel, dim3(blocks), dim3(256), 0, s, static_cast<const uint4*>(in), rows, row_vec, S,
                                                in_start, out_start, flag,
                                                static_cast<uint4*>(out), perm, perm_inv);
   }
@@ -364,52 +374,93 @@ cudaError_t launch_regroup(const void* in, const int32_t* counts_rm, int G, int 
 }
 
 // ---------------------------------------------------------------- combine
-// out[t] = sum_j w[t,j] * y[r(t,j)] in fp32, one 16-byte chunk per thread.
-template <bool BF16>
-__global__ void combine_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ dst_pos,
-                               const int32_t* __restrict__ row_map,
-                               const float* __restrict__ w, int T, int row_vec, int N, int k,
-                               uint4* __restrict__ out) {
-  const long long total = 1LL * T * row_vec;
-  for (long long i = blockIdx.x * 1LL * blockDim.x + threadIdx.x; i < total;
-       i += 1LL * gridDim.x * blockDim.x) {
-    const int t = static_cast<int>(i / row_vec);
-    const int c = static_cast<int>(i - 1LL * t * row_vec);
-    float acc[8];
-#pragma unroll
-    for (int q = 0; q < 8; ++q) acc[q] = 0.f;
-    for (int j = 0; j < k; ++j) {
-      int p = dst_pos[static_cast<size_t>(t) * k + j];
+// out[t] = sum_j w[t,j] * y[r(t,j)] in fp32, one warp per token.  Lane j < k
+// reads the position and weight of copy j once; they are broadcast by
+// shuffle.  Each lane walks the 16-byte chunks of the row and issues the k
+// loads of a chunk before accumulating them in order j = 0..k-1.
+template <bool BF16, int KMAX>
+__global__ void __launch_bounds__(256) combine_kernel(
+    const uint4* __restrict__ y, const int32_t* __restrict__ dst_pos,
+    const int32_t* __restrict__ row_map, const float* __restrict__ w, int T, int row_vec, int N,
+    int k, uint4* __restrict__ out) {
+  pdl_wait();
+  pdl_trigger();
+  const int lane = threadIdx.x & 31;
+  const int nwarps = (gridDim.x * blockDim.x) >> 5;
+  for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += nwarps) {
+    int my_p = -1;
+    float my_w = 0.f;
+    if (lane < k) {
+      int p = dst_pos[static_cast<size_t>(t) * k + lane];
       if (row_map && static_cast<unsigned>(p) < static_cast<unsigned>(N)) p = row_map[p];
-      if (static_cast<unsigned>(p) >= static_cast<unsigned>(N)) continue;
-      const float wj = w ? w[static_cast<size_t>(t) * k + j] : 1.0f;
-      const uint4 v = y[static_cast<size_t>(p) * row_vec + c];
-      if (BF16) {
-        acc[0] = fmaf(wj, bf16_lo(v.x), acc[0]);
-        acc[1] = fmaf(wj, bf16_hi(v.x), acc[1]);
-        acc[2] = fmaf(wj, bf16_lo(v.y), acc[2]);
-        acc[3] = fmaf(wj, bf16_hi(v.y), acc[3]);
-        acc[4] = fmaf(wj, bf16_lo(v.z), acc[4]);
-        acc[5] = fmaf(wj, bf16_hi(v.z), acc[5]);
-        acc[6] = fmaf(wj, bf16_lo(v.w), acc[6]);
-        acc[7] = fmaf(wj, bf16_hi(v.w), acc[7]);
-      } else {
-        acc[0] = fmaf(wj, __uint_as_float(v.x), acc[0]);
-        acc[1] = fmaf(wj, __uint_as_float(v.y), acc[1]);
-        acc[2] = fmaf(wj, __uint_as_float(v.z), acc[2]);
-        acc[3] = fmaf(wj, __uint_as_float(v.w), acc[3]);
+      if (static_cast<unsigned>(p) < static_cast<unsigned>(N)) {
+        my_p = p;
+        my_w = w ? w[static_cast<size_t>(t) * k + lane] : 1.0f;
       }
     }
-    uint4 o;
-    if (BF16) {
-      o = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
-                     pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
-    } else {
-      o = make_uint4(__float_as_uint(acc[0]), __float_as_uint(acc[1]), __float_as_uint(acc[2]),
-                     __float_as_uint(acc[3]));
+    int pos[KMAX];
+    float wt[KMAX];
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      pos[j] = __shfl_sync(0xffffffffu, my_p, j);
+      wt[j] = __shfl_sync(0xffffffffu, my_w, j);
     }
-    out[i] = o;
+    uint4* orow = out + static_cast<size_t>(t) * row_vec;
+    for (int c = lane; c < row_vec; c += 32) {
+      uint4 v[KMAX];
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j)
+        if (j < k && pos[j] >= 0) v[j] = y[static_cast<size_t>(pos[j]) * row_vec + c];
+      float acc[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) acc[q] = 0.f;
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j) {
+        if (j >= k || pos[j] < 0) continue;
+        const float wj = wt[j];
+        if (BF16) {
+          acc[0] = fmaf(wj, bf16_lo(v[j].x), acc[0]);
+          acc[1] = fmaf(wj, bf16_hi(v[j].x), acc[1]);
+          acc[2] = fmaf(wj, bf16_lo(v[j].y), acc[2]);
+          acc[3] = fmaf(wj, bf16_hi(v[j].y), acc[3]);
+          acc[4] = fmaf(wj, bf16_lo(v[j].z), acc[4]);
+          acc[5] = fmaf(wj, bf16_hi(v[j].z), acc[5]);
+          acc[6] = fmaf(wj, bf16_lo(v[j].w), acc[6]);
+          acc[7] = fmaf(wj, bf16_hi(v[j].w), acc[7]);
+        } else {
+          acc[0] = fmaf(wj, __uint_as_float(v[j].x), acc[0]);
+          acc[1] = fmaf(wj, __uint_as_float(v[j].y), acc[1]);
+          acc[2] = fmaf(wj, __uint_as_float(v[j].z), acc[2]);
+          acc[3] = fmaf(wj, __uint_as_float(v[j].w), acc[3]);
+        }
+      }
+      uint4 o;
+      if (BF16) {
+        o = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
+                       pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
+      } else {
+        o = make_uint4(__float_as_uint(acc[0]), __float_as_uint(acc[1]),
+                       __float_as_uint(acc[2]), __float_as_uint(acc[3]));
+      }
+      orow[c] = o;
+    }
   }
+}
+
+template <bool BF16>
+static void combine_launch(const uint4* y, const int32_t* dst_pos, const int32_t* row_map,
+                           const float* w, int T, int row_vec, int N, int k, uint4* out,
+                           int blocks, cudaStream_t s) {
+  if (k <= 1)
+    launch_k(combine_kernel<BF16, 1>, dim3(blocks), dim3(256), 0, s, y, dst_pos, row_map, w, T, row_vec, N, k, out);
+  else if (k <= 2)
+    launch_k(combine_kernel<BF16, 2>, dim3(blocks), dim3(256), 0, s, y, dst_pos, row_map, w, T, row_vec, N, k, out);
+  else if (k <= 4)
+    launch_k(combine_kernel<BF16, 4>, dim3(blocks), dim3(256), 0, s, y, dst_pos, row_map, w, T, row_vec, N, k, out);
+  else if (k <= 8)
+    launch_k(combine_kernel<BF16, 8>, dim3(blocks), dim3(256), 0, s, y, dst_pos, row_map, w, T, row_vec, N, k, out);
+  else
+    launch_k(combine_kernel<BF16, 16>, dim3(blocks), dim3(256), 0, s, y, dst_pos, row_map, w, T, row_vec, N, k, out);
 }
 
 cudaError_t launch_combine(const void* y, const int32_t* dst_pos, const int32_t* row_map,
@@ -418,17 +469,13 @@ cudaError_t launch_combine(const void* y, const int32_t* dst_pos, const int32_t*
   if (T == 0) return cudaSuccess;
   const int elt = dt == MOE_BF16 ? 2 : 4;
   const int row_vec = d * elt / 16;
-  const long long total = 1LL * T * row_vec;
-  const int blocks = static_cast<int>(std::min<long long>(cdiv(static_cast<int>(std::min<long long>(total, 1LL << 30)), 256),
-                                                          1LL * num_sms() * 16));
+  const int blocks = std::min(cdiv(T, 8), num_sms() * 8);
   if (dt == MOE_BF16)
-    combine_kernel<true><<<blocks, 256, 0, s>>>(static_cast<const uint4*>(y), dst_pos, row_map,
-                                                topk_w, T, row_vec, N, top_k,
-                                                static_cast<uint4*>(out));
+    combine_launch<true>(static_cast<const uint4*>(y), dst_pos, row_map, topk_w, T, row_vec, N,
+                         top_k, static_cast<uint4*>(out), blocks, s);
   else
-    combine_kernel<false><<<blocks, 256, 0, s>>>(static_cast<const uint4*>(y), dst_pos, row_map,
-                                                 topk_w, T, row_vec, N, top_k,
-                                                 static_cast<uint4*>(out));
+    combine_launch<false>(static_cast<const uint4*>(y), dst_pos, row_map, topk_w, T, row_vec, N,
+                          top_k, static_cast<uint4*>(out), blocks, s);
   return cudaGetLastError();
 }
 
@@ -444,6 +491,8 @@ __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 v) { return _
 template <typename TX>
 __global__ void router_logits_kernel(const TX* __restrict__ x, const TX* __restrict__ w, int T,
                                      int d, int E, float* __restrict__ logits) {
+  pdl_wait();
+  pdl_trigger();
   const long long total = 1LL * T * E;
   for (long long i = blockIdx.x * 1LL * blockDim.x + threadIdx.x; i < total;
        i += 1LL * gridDim.x * blockDim.x) {
@@ -462,11 +511,11 @@ cudaError_t launch_router_logits_simt(const void* x, const void* w_router, int T
   if (total == 0) return cudaSuccess;
   const int blocks = static_cast<int>(std::min<long long>((total + 255) / 256, 1LL * num_sms() * 32));
   if (dt == MOE_BF16)
-    router_logits_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(
+    launch_k(router_logits_kernel<__nv_bfloat16>, dim3(blocks), dim3(256), 0, s, 
         static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(w_router), T, d,
         E, logits);
   else
-    router_logits_kernel<float><<<blocks, 256, 0, s>>>(static_cast<const float*>(x),
+    launch_k(router_logits_kernel<float>, dim3(blocks), dim3(256), 0, s, static_cast<const float*>(x),
                                                        static_cast<const float*>(w_router), T, d,
                                                        E, logits);
   return cudaGetLastError();
@@ -481,6 +530,8 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
     const float* __restrict__ parts, int nsplit, int T, int E, int k, int renorm,
     float* __restrict__ logits_out, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
     int32_t* __restrict__ counts) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int hist[kMaxExperts];
   if (counts)
     for (int i = threadIdx.x; i < E; i += blockDim.x) hist[i] = 0;
@@ -583,19 +634,19 @@ cudaError_t launch_router_topk(const float* parts, int nsplit, int T, int E, int
   if (T == 0) return cudaSuccess;
   const int blocks = std::min(cdiv(T, 8), num_sms() * 16);
   if (E <= 32)
-    router_topk_kernel<1><<<blocks, 256, 0, s>>>(parts, nsplit, T, E, top_k, renorm, logits_out,
+    launch_k(router_topk_kernel<1>, dim3(blocks), dim3(256), 0, s, parts, nsplit, T, E, top_k, renorm, logits_out,
                                                  topk_idx, topk_w, counts);
   else if (E <= 64)
-    router_topk_kernel<2><<<blocks, 256, 0, s>>>(parts, nsplit, T, E, top_k, renorm, logits_out,
+    launch_k(router_topk_kernel<2>, dim3(blocks), dim3(256), 0, s, parts, nsplit, T, E, top_k, renorm, logits_out,
                                                  topk_idx, topk_w, counts);
   else if (E <= 128)
-    router_topk_kernel<4><<<blocks, 256, 0, s>>>(parts, nsplit, T, E, top_k, renorm, logits_out,
+    launch_k(router_topk_kernel<4>, dim3(blocks), dim3(256), 0, s, parts, nsplit, T, E, top_k, renorm, logits_out,
                                                  topk_idx, topk_w, counts);
   else if (E <= 256)
-    router_topk_kernel<8><<<blocks, 256, 0, s>>>(parts, nsplit, T, E, top_k, renorm, logits_out,
+    launch_k(router_topk_kernel<8>, dim3(blocks), dim3(256), 0, s, parts, nsplit, T, E, top_k, renorm, logits_out,
                                                  topk_idx, topk_w, counts);
   else
-    router_topk_kernel<16><<<blocks, 256, 0, s>>>(parts, nsplit, T, E, top_k, renorm, logits_out,
+    launch_k(router_topk_kernel<16>, dim3(blocks), dim3(256), 0, s, parts, nsplit, T, E, top_k, renorm, logits_out,
                                                   topk_idx, topk_w, counts);
   return cudaGetLastError();
 }

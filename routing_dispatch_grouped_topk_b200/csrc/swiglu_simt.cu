@@ -54,6 +54,8 @@ __global__ void __launch_bounds__(256) swiglu_up_f32_kernel(
     const int32_t* __restrict__ offsets, const float* __restrict__ w1,
     const float* __restrict__ w3, int N, int d, int h, int E, float* __restrict__ H,
     int* status) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int off[kMaxExperts + 1], cum[kMaxExperts + 1];
   __shared__ float xs[SB][SB + 1], as[SB][SB + 1], bs[SB][SB + 1];
   __shared__ int xrow[SB];
@@ -119,6 +121,8 @@ __global__ void __launch_bounds__(256) swiglu_down_f32_kernel(
     const float* __restrict__ H, const int32_t* __restrict__ offsets,
     const float* __restrict__ w2, const float* __restrict__ row_scale, int N, int d, int h, int E,
     float* __restrict__ y, int* status) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int off[kMaxExperts + 1], cum[kMaxExperts + 1];
   __shared__ float hs[SB][SB + 1], ws[SB][SB + 1];
   if (!simt_schedule(offsets, E, N, off, cum, status)) return;
@@ -179,10 +183,10 @@ cudaError_t launch_swiglu_simt_f32_gather(const float* x, int x_rows, const int3
                                           float* y, float* H, int* status, cudaStream_t s) {
   const int max_tiles = cdiv(N, SB) + E;   // upper bound over all segmentations
   dim3 g1(max_tiles, cdiv(h, SB));
-  swiglu_up_f32_kernel<<<g1, 256, 0, s>>>(x, src_row, x_rows, offsets, w1, w3, N, d, h, E, H,
+  launch_k(swiglu_up_f32_kernel, dim3(g1), dim3(256), 0, s, x, src_row, x_rows, offsets, w1, w3, N, d, h, E, H,
                                           status);
   dim3 g2(max_tiles, cdiv(d, SB));
-  swiglu_down_f32_kernel<<<g2, 256, 0, s>>>(H, offsets, w2, row_scale, N, d, h, E, y, status);
+  launch_k(swiglu_down_f32_kernel, dim3(g2), dim3(256), 0, s, H, offsets, w2, row_scale, N, d, h, E, y, status);
   return cudaGetLastError();
 }
 

@@ -425,6 +425,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish();
     tc_fence_before();
   }
+  pdl_wait();   // offsets, A and B may be written by the previous kernel
   P::prologue(args, sched);
   __syncthreads();
   tc_fence_after();
@@ -607,6 +608,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(tempty + acc);
     }
   }
+  pdl_trigger();   // the next kernel may start its prologue
   __syncthreads();
   P::finish(args, sched);
   if (warp == 1) {
@@ -688,6 +690,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish_pair();
     tc_fence_before();
   }
+  pdl_wait();   // offsets, A and B may be written by the previous kernel
   P::prologue(args, sched);
   __syncthreads();
   cluster_sync_all();   // barriers of both CTAs initialised before any remote arrive
@@ -803,6 +806,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive_cluster(tempty_leader[acc]);
     }
   }
+  pdl_trigger();   // the next kernel may start its prologue
   __syncthreads();
   cluster_sync_all();   // no CTA leaves while its peer may still touch its memory
   if (warp == 1) {
@@ -863,7 +867,7 @@ cudaError_t launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMa
     if (e != cudaSuccess) return e;
     configured[dev] = 1;
   }
-  tc_gemm_kernel<P><<<grid, kThreads, L::kLaunchBytes, s>>>(a, b0, b1, args);
+  launch_k(tc_gemm_kernel<P>, dim3(grid), dim3(kThreads), L::kLaunchBytes, s, a, b0, b1, args);
   return cudaGetLastError();
 }
 
@@ -887,13 +891,15 @@ cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUten
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = L::kLaunchBytes;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, tc_gemm_pair_kernel<P>, a, b0, b1, args);
 }
 
@@ -970,10 +976,12 @@ static cudaError_t swiglu_tc_impl(const void* a_src, int a_rows, const int32_t* 
   if (!make_tmap(&t1, w1, d, static_cast<uint64_t>(E) * h, 128)) return cudaErrorInvalidValue;
   if (!make_tmap(&t3, w3, d, static_cast<uint64_t>(E) * h, 128)) return cudaErrorInvalidValue;
   if (!make_tmap(&th, H, h, N, BM)) return cudaErrorInvalidValue;
-  // CTA pairs pay off once the average expert has more than 128 rows: a
-  // 256-row pair tile then replaces two 128-row tiles with 2/3 of the loads
-  // per SM.  Decode-sized segments keep one CTA per 128-row tile.
-  const bool pairs = !gather && N > 128 * E;
+  // The CTA-pair kernel (256-row tiles, 2/3 of the loads per SM) measured
+  // no faster than single-CTA 128-row tiles on B200 under the power cap for
+  // segments of ~256 (uniform) to ~1024 (Zipf-skewed) average rows, and its
+  // 256-row tiles pad more on short segments; it is used only when segments
+  // average more than 1024 rows.
+  const bool pairs = !gather && N > 1024 * E;
   if (!make_tmap(&t2, w2, h, static_cast<uint64_t>(E) * d, pairs ? 128 : 256))
     return cudaErrorInvalidValue;
   const int max_mt = cdiv(N, BM) + E;   // upper bound on m-tiles over all segments
