@@ -145,6 +145,36 @@ MOE_API moe_status_t moe_dispatch(const void* x, const int32_t* topk_idx, int T,
                           size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * moe_dispatch_noalloc -- moe_dispatch without a caller workspace.  The
+ * pages have no counterpart: it exists for callers that cannot allocate
+ * device memory where they dispatch, e.g. an engine or plugin whose enqueue
+ * path must not allocate, a server whose device memory is all reserved by
+ * another framework's pool, or a latency-critical path that must never wait
+ * on an allocator.
+ *
+ * Same arguments, outputs and error behaviour as moe_dispatch, minus ws.
+ * Its scratch (status word and per-block histogram table) is a fixed
+ * MOE_NOALLOC_SCRATCH_BYTES array inside the library, held by every GPU that
+ * loads it until the process exits.  Sizes for which
+ * moe_dispatch_workspace_size(T, E, top_k) exceeds MOE_NOALLOC_SCRATCH_BYTES
+ * (for E = 128 about a million tokens) return MOE_ERR_UNSUPPORTED with a
+ * message and launch nothing.  It allocates nothing: no cudaMalloc,
+ * cudaFree or allocating library call.
+ * The first call on a device looks the array's device address up
+ * (cudaGetSymbolAddress) and caches it; make that first call before any
+ * stream capture.  All calls share the array and it keeps the last call's
+ * contents (the status word is cleared at the start of each call), so calls
+ * that overlap on the GPU -- on different streams, or from several host
+ * threads -- race; serialise them.  The device status word is not exposed:
+ * ids outside [0, E) show up as dst_pos = -1 and offsets[E] < T*k.
+ * ---------------------------------------------------------------------- */
+#define MOE_NOALLOC_SCRATCH_BYTES (4 << 20)
+MOE_API moe_status_t moe_dispatch_noalloc(const void* x, const int32_t* topk_idx, int T, int d,
+                                          int E, int top_k, moe_dtype_t dt, int32_t* counts,
+                                          int32_t* offsets, int32_t* src_row, int32_t* dst_pos,
+                                          void* x_perm, void* stream);
+
+/* ------------------------------------------------------------------------
  * moe_ep_dispatch_rank_major -- the layout in which R expert-parallel ranks
  * receive the routed copies ([EP] Ep2DpParallel._token_dispatch): source
  * rank r owns tokens [r*S, min(T, (r+1)*S)), S = ceil(T/R), and destination

@@ -45,7 +45,7 @@ MOE_DEV_BAD_EXPERT, MOE_DEV_BAD_COUNTS, MOE_DEV_BAD_OFFSETS, MOE_DEV_TIMEOUT = 1
 
 EXPORTED_SYMBOLS = [
     "moe_router_workspace_size", "moe_router_topk",
-    "moe_dispatch_workspace_size", "moe_dispatch",
+    "moe_dispatch_workspace_size", "moe_dispatch", "moe_dispatch_noalloc",
     "moe_ep_dispatch_workspace_size", "moe_ep_dispatch_rank_major",
     "moe_regroup_workspace_size", "moe_ep_local_regroup",
     "moe_grouped_swiglu_workspace_size", "moe_grouped_swiglu", "moe_grouped_swiglu_gather",
@@ -67,6 +67,7 @@ _SIGS = {
     "moe_router_topk": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _Z, _P]),
     "moe_dispatch_workspace_size": (_Z, [_I, _I, _I]),
     "moe_dispatch": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _Z, _P]),
+    "moe_dispatch_noalloc": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
     "moe_ep_dispatch_workspace_size": (_Z, [_I, _I, _I, _I]),
     "moe_ep_dispatch_rank_major": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P,
                                         _Z, _P]),
