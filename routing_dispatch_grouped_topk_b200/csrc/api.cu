@@ -101,25 +101,28 @@ moe_status_t check_router(const void* x, const void* w_router, const float* logi
 }
 
 // Router launch sequence (status and counts already cleared by the caller).
+// With `plan` and `blk` the top-k kernel also writes the dispatch histogram.
 cudaError_t run_router(const void* x, const void* w_router, const float* logits_in, int T, int d,
                        int E, int top_k, int renorm, moe_dtype_t dt, float* logits_out,
                        int32_t* topk_idx, float* topk_w, int32_t* counts, void* scratch,
-                       int* status, cudaStream_t s) {
+                       int* status, cudaStream_t s, const DispatchPlan* plan = nullptr,
+                       int32_t* blk = nullptr) {
   if (T == 0) return cudaSuccess;
   if (logits_in)
     return launch_router_topk(logits_in, 1, T, E, top_k, renorm, nullptr, topk_idx, topk_w,
-                              counts, s);
+                              counts, plan, blk, s);
   float* part = static_cast<float*>(scratch);
   if (router_uses_tc(E, dt)) {
     cudaError_t e = launch_router_tc(x, w_router, T, d, E, part, status, s);
     if (e != cudaSuccess) return e;
     return launch_router_topk(part, router_plan(T, d).ksplit, T, E, top_k, renorm, logits_out,
-                              topk_idx, topk_w, counts, s);
+                              topk_idx, topk_w, counts, plan, blk, s);
   }
   float* L = logits_out ? logits_out : part;
   cudaError_t e = launch_router_logits_simt(x, w_router, T, d, E, dt, L, s);
   if (e != cudaSuccess) return e;
-  return launch_router_topk(L, 1, T, E, top_k, renorm, nullptr, topk_idx, topk_w, counts, s);
+  return launch_router_topk(L, 1, T, E, top_k, renorm, nullptr, topk_idx, topk_w, counts, plan,
+                            blk, s);
 }
 
 size_t swiglu_ws(int N, int h, moe_dtype_t dt) {
@@ -520,11 +523,13 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* logit
   float* w = topk_w ? topk_w : f.w;
   const int R = ep_ranks;
   cudaError_t e = cudaMemsetAsync(f.status, 0, sizeof(int), s);
+  const DispatchPlan p = make_dispatch_plan(T, E, top_k, R);
+  // The router's top-k kernel also writes the dispatch histogram table.
   if (e == cudaSuccess)
     e = run_router(x, w_router, logits_in, T, d, E, top_k, renormalize, dt, logits_out, idx, w,
-                   nullptr, f.router_scratch, f.status, s);
+                   nullptr, f.router_scratch, f.status, s, &p,
+                   static_cast<int32_t*>(f.disp_ws));
   if (e != cudaSuccess) return cuda_status(e, "moe_forward/router");
-  const DispatchPlan p = make_dispatch_plan(T, E, top_k, R);
   int32_t* cnt_a = (R == 1 && counts) ? counts : f.counts_a;
   // The routed rows are materialised expert-major (single device) or
   // rank-major (simulated EP: what an all-to-all would deliver), then
@@ -532,7 +537,7 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* logit
   // on B200 it is faster than gathering GEMM1's rows with TMA gather4
   // (moe_grouped_swiglu_gather), whose 512-byte requests limit the loads.
   e = launch_dispatch(p, x, idx, d, dt, cnt_a, f.offsets_a, f.src_row, f.dst_pos, f.x_a,
-                      f.disp_ws, f.status, s);
+                      f.disp_ws, f.status, s, /*hist_done=*/T > 0);
   if (e != cudaSuccess) return cuda_status(e, "moe_forward/dispatch");
   const void* xe = f.x_a;
   const int32_t* off = f.offsets_a;

@@ -31,13 +31,7 @@ cudaError_t launch_router_tc(const void* x, const void* w_router, int T, int d, 
 // CUDA-core fp32 logits (x fp32 or bf16) into `logits` [T, E].
 cudaError_t launch_router_logits_simt(const void* x, const void* w_router, int T, int d, int E,
                                       moe_dtype_t dt, float* logits, cudaStream_t s);
-// Sum of `nsplit` partial logit arrays [nsplit, T, E] (in split order), then
-// softmax / top-k / renormalisation / counts; writes the logits if asked.
-cudaError_t launch_router_topk(const float* parts, int nsplit, int T, int E, int top_k,
-                               int renorm, float* logits_out, int32_t* topk_idx, float* topk_w,
-                               int32_t* counts, cudaStream_t s);
-
-// ---- dispatch -------------------------------------------------------------
+// ---- dispatch plan ----------------------------------------------------------
 struct DispatchPlan {
   int T, k, E, R, L, S;   // R = 1: plain dispatch; R > 1: rank-major EP layout
   int nbins;              // E or E * R
@@ -46,10 +40,23 @@ struct DispatchPlan {
 };
 DispatchPlan make_dispatch_plan(int T, int E, int top_k, int R);
 size_t dispatch_ws_bytes(const DispatchPlan& p);
+
+// Sum of `nsplit` partial logit arrays [nsplit, T, E] (in split order), then
+// softmax / top-k / renormalisation; writes the logits if asked.  With
+// `plan` and `blk` it also writes the dispatch histogram table of `plan`
+// (so launch_dispatch can skip its histogram kernel); otherwise it adds the
+// expert histogram to `counts` when given.
+cudaError_t launch_router_topk(const float* parts, int nsplit, int T, int E, int top_k,
+                               int renorm, float* logits_out, int32_t* topk_idx, float* topk_w,
+                               int32_t* counts, const DispatchPlan* plan, int32_t* blk,
+                               cudaStream_t s);
+
+// ---- dispatch -------------------------------------------------------------
+// hist_done: the histogram table in `ws` was already written (by the router).
 cudaError_t launch_dispatch(const DispatchPlan& p, const void* x, const int32_t* topk_idx,
                             int d, moe_dtype_t dt, int32_t* counts, int32_t* offsets,
                             int32_t* src_row, int32_t* dst_pos, void* x_perm, void* ws,
-                            int* status, cudaStream_t s);
+                            int* status, cudaStream_t s, bool hist_done = false);
 
 // ---- regroup ----------------------------------------------------------------
 size_t regroup_ws_bytes(int G, int R, int L);

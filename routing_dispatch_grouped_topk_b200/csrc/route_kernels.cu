@@ -6,6 +6,7 @@
 // global atomics: per-block histograms, one scan over (block, bin), then a
 // warp-synchronous stable rank (match.any + popc) inside each block.
 #include <algorithm>
+#include <climits>
 
 #include "common.cuh"
 #include "internal.h"
@@ -242,25 +243,24 @@ size_t dispatch_ws_bytes(const DispatchPlan& p) {
 cudaError_t launch_dispatch(const DispatchPlan& p, const void* x, const int32_t* topk_idx,
                             int d, moe_dtype_t dt, int32_t* counts, int32_t* offsets,
                             int32_t* src_row, int32_t* dst_pos, void* x_perm, void* ws,
-                            int* status, cudaStream_t s) {
+                            int* status, cudaStream_t s, bool hist_done) {
   int32_t* blk = static_cast<int32_t*>(ws);
-  const int N = p.T * p.k;
   if (p.T == 0) {
     cudaError_t e = cudaMemsetAsync(counts, 0, sizeof(int32_t) * p.nbins, s);
     if (e == cudaSuccess) e = cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (p.nbins + 1), s);
     return e;
   }
-  (void)N;
-  launch_k(dispatch_hist_kernel, dim3(p.nblk), dim3(256), p.nbins * sizeof(int), s, 
-      topk_idx, p.T, p.k, p.E, p.R, p.L, p.S, p.tb, p.nbins, blk, status);
-  launch_k(dispatch_colscan_kernel, dim3(std::min(p.nbins, num_sms() * 8)), dim3(256), 0, s, blk, p.nblk, p.nbins,
-                                                                           counts);
+  if (!hist_done)
+    launch_k(dispatch_hist_kernel, dim3(p.nblk), dim3(256), p.nbins * sizeof(int), s, topk_idx,
+             p.T, p.k, p.E, p.R, p.L, p.S, p.tb, p.nbins, blk, status);
+  launch_k(dispatch_colscan_kernel, dim3(std::min(p.nbins, num_sms() * 8)), dim3(256), 0, s, blk,
+           p.nblk, p.nbins, counts);
   const int elt = dt == MOE_BF16 ? 2 : 4;
   const int row_vec = d * elt / 16;
   const size_t sm3 = (p.nbins + 33 + p.tb * p.k) * sizeof(int);
-  launch_k(dispatch_scatter_kernel, dim3(p.nblk), dim3(256), sm3, s, 
-      static_cast<const uint4*>(x), topk_idx, p.T, p.k, p.E, p.R, p.L, p.S, p.tb, p.nbins, blk,
-      counts, offsets, src_row, dst_pos, static_cast<uint4*>(x_perm), row_vec);
+  launch_k(dispatch_scatter_kernel, dim3(p.nblk), dim3(256), sm3, s,
+           static_cast<const uint4*>(x), topk_idx, p.T, p.k, p.E, p.R, p.L, p.S, p.tb, p.nbins,
+           blk, counts, offsets, src_row, dst_pos, static_cast<uint4*>(x_perm), row_vec);
   return cudaGetLastError();
 }
 
@@ -521,25 +521,42 @@ cudaError_t launch_router_logits_simt(const void* x, const void* w_router, int T
   return cudaGetLastError();
 }
 
-// One warp per token.  Lane l holds experts l, l+32, ... (EPL of them): the
-// logit is the sum of the nsplit partial values in split order.  The k
-// winners are found by k rounds of a warp arg-max on (score desc, expert
-// asc); lane j keeps winner j.  NaN scores count as -inf (indices stay valid).
+// Order-preserving map of a float score to int32 (NaN must be mapped to -inf
+// first; -0 and +0 compare equal, as floats do).
+__device__ __forceinline__ int score_key(float f) {
+  f += 0.0f;
+  const int i = __float_as_int(f);
+  return i ^ ((i >> 31) & 0x7fffffff);
+}
+__device__ __forceinline__ float key_score(int k) { return __int_as_float(k ^ ((k >> 31) & 0x7fffffff)); }
+
+// One warp per token; block b owns tokens [b*tpb, (b+1)*tpb).  Lane l holds
+// experts l, l+32, ... (EPL of them); the logit is the sum of the nsplit
+// partial values in split order.  The k winners come from k rounds of a warp
+// arg-max on (score desc, expert asc) done with two redux.sync reductions
+// (max of the score key, then min expert index among the lanes holding it);
+// lane j keeps winner j.  NaN scores count as -inf (indices stay valid).
+// With `blk` the block also writes its histogram of dispatch keys as column
+// b of the dispatch table blk[bin * gridDim.x + b]; with `counts` it adds its
+// expert histogram to counts.
 template <int EPL>
 __global__ void __launch_bounds__(256) router_topk_kernel(
-    const float* __restrict__ parts, int nsplit, int T, int E, int k, int renorm,
+    const float* __restrict__ parts, int nsplit, int T, int E, int k, int renorm, int tpb,
     float* __restrict__ logits_out, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
-    int32_t* __restrict__ counts) {
+    int32_t* __restrict__ counts, int32_t* __restrict__ blk, int nbins, int R, int L, int S) {
   pdl_wait();
   pdl_trigger();
-  __shared__ int hist[kMaxExperts];
-  if (counts)
-    for (int i = threadIdx.x; i < E; i += blockDim.x) hist[i] = 0;
+  extern __shared__ int bins[];   // nbins (dispatch keys) or E (counts)
+  const int nb = blk ? nbins : E;
+  const bool tally = blk != nullptr || counts != nullptr;
+  if (tally)
+    for (int i = threadIdx.x; i < nb; i += blockDim.x) bins[i] = 0;
   __syncthreads();
   const int lane = threadIdx.x & 31;
-  const int nwarps = (gridDim.x * blockDim.x) >> 5;
+  const int warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
   const size_t plane = static_cast<size_t>(T) * E;
-  for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += nwarps) {
+  const int t_end = min(T, (blockIdx.x + 1) * tpb);
+  for (int t = blockIdx.x * tpb + warp; t < t_end; t += nwarps) {
     float sv[EPL];
     bool avail[EPL];
     const float* base = parts + static_cast<size_t>(t) * E + lane;
@@ -566,48 +583,39 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
 #pragma unroll
       for (int i = 0; i < EPL; ++i)
         if (avail[i]) sv[i] += base[sp * plane + 32 * i];
+    int key[EPL];
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
       if (avail[i] && logits_out) logits_out[static_cast<size_t>(t) * E + lane + 32 * i] = sv[i];
       if (sv[i] != sv[i]) sv[i] = -INFINITY;
+      key[i] = score_key(sv[i]);
     }
-    float mx = -INFINITY;
-    float my_v = 0.f;
-    int my_e = 0;
+    int my_key = 0, my_e = 0, top_key = 0;
     for (int j = 0; j < k; ++j) {
-      float bv = -INFINITY;
-      int be = 0x7fffffff;
+      int lk = INT_MIN, li = 0x7fffffff;
 #pragma unroll
-      for (int i = 0; i < EPL; ++i) {
-        const int e = lane + 32 * i;
-        if (avail[i] && (sv[i] > bv || (sv[i] == bv && e < be))) {
-          bv = sv[i];
-          be = e;
+      for (int i = 0; i < EPL; ++i)
+        if (avail[i] && key[i] > lk) {   // experts of a lane ascend with i: first max wins
+          lk = key[i];
+          li = lane + 32 * i;
         }
-      }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-        const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-        if (ov > bv || (ov == bv && oe < be)) {
-          bv = ov;
-          be = oe;
-        }
-      }
+      const int mk = __reduce_max_sync(0xffffffffu, lk);
+      const int be = __reduce_min_sync(0xffffffffu, lk == mk ? li : 0x7fffffff);
 #pragma unroll
       for (int i = 0; i < EPL; ++i)
         if (lane + 32 * i == be) avail[i] = false;
-      if (j == 0) mx = bv;
+      if (j == 0) top_key = mk;
       if (lane == j) {
-        my_v = bv;
+        my_key = mk;
         my_e = be;
       }
     }
+    const float mx = key_score(top_key);
     float se = 0.f;
 #pragma unroll
     for (int i = 0; i < EPL; ++i)
       if (lane + 32 * i < E) se += expf(sv[i] - mx);
-    const float ex = lane < k ? expf(my_v - mx) : 0.f;
+    const float ex = lane < k ? expf(key_score(my_key) - mx) : 0.f;
     float sel = ex;
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) {
@@ -618,36 +626,49 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
       const size_t o = static_cast<size_t>(t) * k + lane;
       topk_idx[o] = my_e;
       topk_w[o] = ex / (renorm ? sel : se);
-      if (counts) atomicAdd(&hist[my_e], 1);
+      if (blk) atomicAdd(&bins[dispatch_key(my_e, t, R, L, S)], 1);
+      else if (counts) atomicAdd(&bins[my_e], 1);
     }
   }
-  if (counts) {
-    __syncthreads();
-    for (int i = threadIdx.x; i < E; i += blockDim.x)
-      if (hist[i]) atomicAdd(&counts[i], hist[i]);
+  if (!tally) return;
+  __syncthreads();
+  if (blk) {
+    for (int i = threadIdx.x; i < nb; i += blockDim.x)
+      blk[static_cast<size_t>(i) * gridDim.x + blockIdx.x] = bins[i];
+  } else {
+    for (int i = threadIdx.x; i < nb; i += blockDim.x)
+      if (bins[i]) atomicAdd(&counts[i], bins[i]);
   }
 }
 
 cudaError_t launch_router_topk(const float* parts, int nsplit, int T, int E, int top_k,
                                int renorm, float* logits_out, int32_t* topk_idx, float* topk_w,
-                               int32_t* counts, cudaStream_t s) {
+                               int32_t* counts, const DispatchPlan* plan, int32_t* blk,
+                               cudaStream_t s) {
   if (T == 0) return cudaSuccess;
-  const int blocks = std::min(cdiv(T, 8), num_sms() * 16);
+  const bool fuse = plan && blk;
+  const int tpb = fuse ? plan->tb : 16;
+  const int blocks = cdiv(T, tpb);
+  const int nbins = fuse ? plan->nbins : 0;
+  const size_t smem = sizeof(int) * (fuse ? nbins : (counts ? E : 0));
+  const int R = fuse ? plan->R : 1, L = fuse ? plan->L : E, S = fuse ? plan->S : T;
+  int32_t* b = fuse ? blk : nullptr;
+  int32_t* c = fuse ? nullptr : counts;
   if (E <= 32)
-    launch_k(router_topk_kernel<1>, dim3(blocks), dim3(256), 0, s, parts, nsplit, T, E, top_k, renorm, logits_out,
-                                                 topk_idx, topk_w, counts);
+    launch_k(router_topk_kernel<1>, dim3(blocks), dim3(256), smem, s, parts, nsplit, T, E, top_k,
+             renorm, tpb, logits_out, topk_idx, topk_w, c, b, nbins, R, L, S);
   else if (E <= 64)
-    launch_k(router_topk_kernel<2>, dim3(blocks), dim3(256), 0, s, parts, nsplit, T, E, top_k, renorm, logits_out,
-                                                 topk_idx, topk_w, counts);
+    launch_k(router_topk_kernel<2>, dim3(blocks), dim3(256), smem, s, parts, nsplit, T, E, top_k,
+             renorm, tpb, logits_out, topk_idx, topk_w, c, b, nbins, R, L, S);
   else if (E <= 128)
-    launch_k(router_topk_kernel<4>, dim3(blocks), dim3(256), 0, s, parts, nsplit, T, E, top_k, renorm, logits_out,
-                                                 topk_idx, topk_w, counts);
+    launch_k(router_topk_kernel<4>, dim3(blocks), dim3(256), smem, s, parts, nsplit, T, E, top_k,
+             renorm, tpb, logits_out, topk_idx, topk_w, c, b, nbins, R, L, S);
   else if (E <= 256)
-    launch_k(router_topk_kernel<8>, dim3(blocks), dim3(256), 0, s, parts, nsplit, T, E, top_k, renorm, logits_out,
-                                                 topk_idx, topk_w, counts);
+    launch_k(router_topk_kernel<8>, dim3(blocks), dim3(256), smem, s, parts, nsplit, T, E, top_k,
+             renorm, tpb, logits_out, topk_idx, topk_w, c, b, nbins, R, L, S);
   else
-    launch_k(router_topk_kernel<16>, dim3(blocks), dim3(256), 0, s, parts, nsplit, T, E, top_k, renorm, logits_out,
-                                                  topk_idx, topk_w, counts);
+    launch_k(router_topk_kernel<16>, dim3(blocks), dim3(256), smem, s, parts, nsplit, T, E,
+             top_k, renorm, tpb, logits_out, topk_idx, topk_w, c, b, nbins, R, L, S);
   return cudaGetLastError();
 }
 
