@@ -227,10 +227,10 @@ DispatchPlan make_dispatch_plan(int T, int E, int top_k, int R) {
   p.L = E / R;
   p.S = R > 1 ? std::max(1, cdiv(T, R)) : std::max(T, 1);
   p.nbins = E * R;
-  // Enough blocks to cover the SMs about twice; small blocks keep the
-  // warp-serial ranking short.
-  int tb = 16;
-  while (tb < 128 && cdiv(T, tb * 2) >= 2 * 148) tb *= 2;
+  // About four blocks per SM, so that the row copies balance across SMs;
+  // small blocks also keep the warp-serial ranking short.
+  int tb = 8;
+  while (tb < 128 && cdiv(T, tb * 2) >= 4 * 148) tb *= 2;
   p.tb = tb;
   p.nblk = std::max(1, cdiv(T, tb));
   return p;

@@ -47,7 +47,19 @@ struct TileInfo {
   int m_valid;   // rows of this tile that belong to the problem / expert
   int n0;        // first output column (router: the K split)
   int kb0, kb1;  // K blocks [kb0, kb1) of this tile
+  int swap_np;   // 0, or: swap-AB tile whose MMA N is this many token rows
 };
+
+// A grouped tile with few valid rows (an expert's last rows, or decode) is
+// computed with A and B swapped: the 128-row weight halves of the B stage
+// become the MMA's M = 128 operand and the tile's token rows (rounded up to
+// 16) its N, as two MMAs of N = np instead of one of N = 256.  The shared
+// memory stages are the same; only the MMA issue and the epilogue differ
+// (accumulator lanes are weight rows, columns are tokens).
+constexpr int kSwapMaxRows = 112;   // 2 * 112 < 256: a swap tile always costs less
+__device__ __forceinline__ void set_swap(TileInfo& t) {
+  t.swap_np = (t.m_valid <= kSwapMaxRows) ? ((max(t.m_valid, 1) + 15) & ~15) : 0;
+}
 
 struct Args {
   int M;                     // rows of A: T (router) or N (grouped)
@@ -102,6 +114,7 @@ struct RouterPolicy {
     t.n0 = sp;
     t.kb0 = sp * a.kb_per_split;
     t.kb1 = min(cdiv(a.K, BK), t.kb0 + a.kb_per_split);
+    t.swap_np = 0;
     return t;
   }
   static __device__ void epilogue(const Args& a, int*, const TileInfo& ti, uint32_t taddr,
@@ -223,10 +236,40 @@ struct UpPolicyT : GroupedSched<256, 2, 128> {
     t.b_row = e * a.n_out + t.n0;
     t.kb0 = 0;
     t.kb1 = cdiv(a.K, BK);
+    set_swap(t);
     return t;
+  }
+  // Swap-AB tile: lane = hidden unit n0 + row; columns [0, np) hold G and
+  // [np, 2 np) hold U for the tile's tokens.  A warp stores 64 contiguous
+  // bytes of H per token.
+  static __device__ void epilogue_swap(const Args& a, const TileInfo& ti, uint32_t taddr,
+                                       int row) {
+    const int n = ti.n0 + row;
+    const bool nvalid = n < a.n_out;
+    __nv_bfloat16* col = a.out + static_cast<size_t>(ti.a_row) * a.n_out + n;
+    for (int t0 = 0; t0 < ti.m_valid; t0 += 16) {
+      uint32_t g[16], u[16];
+      tmem_ld16(taddr + t0, g);
+      tmem_ld16(taddr + ti.swap_np + t0, u);
+      tmem_ld_wait();
+      if (nvalid) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          if (t0 + i < ti.m_valid) {
+            const float gv = __uint_as_float(g[i]), uv = __uint_as_float(u[i]);
+            col[static_cast<size_t>(t0 + i) * a.n_out] =
+                __float2bfloat16_rn(__fdividef(gv, 1.0f + __expf(-gv)) * uv);
+          }
+        }
+      }
+    }
   }
   static __device__ void epilogue(const Args& a, int*, const TileInfo& ti, uint32_t taddr,
                                   int row) {
+    if (ti.swap_np) {
+      epilogue_swap(a, ti, taddr, row);
+      return;
+    }
     const bool valid = row < ti.m_valid;
     __nv_bfloat16* dst_row = a.out + static_cast<size_t>(ti.a_row + row) * a.n_out + ti.n0;
 #pragma unroll 1
@@ -268,10 +311,38 @@ struct DownPolicy : GroupedSched<256, 1, 256> {
     t.b_row = e * a.n_out + t.n0;
     t.kb0 = 0;
     t.kb1 = cdiv(a.K, BK);
+    set_swap(t);
     return t;
+  }
+  // Swap-AB tile: lane = output column n0 + row (columns [0, np)) and
+  // n0 + 128 + row (columns [np, 2 np)); columns are the tile's tokens.
+  static __device__ void epilogue_swap(const Args& a, const TileInfo& ti, uint32_t taddr,
+                                       int row) {
+    const int c1 = ti.n0 + row, c2 = ti.n0 + 128 + row;
+    __nv_bfloat16* base = a.out + static_cast<size_t>(ti.a_row) * a.n_out;
+    for (int t0 = 0; t0 < ti.m_valid; t0 += 16) {
+      uint32_t v1[16], v2[16];
+      tmem_ld16(taddr + t0, v1);
+      tmem_ld16(taddr + ti.swap_np + t0, v2);
+      tmem_ld_wait();
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int t = t0 + i;
+        if (t < ti.m_valid) {
+          const float sc = a.row_scale ? a.row_scale[ti.a_row + t] : 1.0f;
+          __nv_bfloat16* r = base + static_cast<size_t>(t) * a.n_out;
+          if (c1 < a.n_out) r[c1] = __float2bfloat16_rn(__uint_as_float(v1[i]) * sc);
+          if (c2 < a.n_out) r[c2] = __float2bfloat16_rn(__uint_as_float(v2[i]) * sc);
+        }
+      }
+    }
   }
   static __device__ void epilogue(const Args& a, int*, const TileInfo& ti, uint32_t taddr,
                                   int row) {
+    if (ti.swap_np) {
+      epilogue_swap(a, ti, taddr, row);
+      return;
+    }
     const bool valid = row < ti.m_valid;
     const size_t grow = static_cast<size_t>(ti.a_row + row);
     const float scale = (valid && a.row_scale) ? a.row_scale[grow] : 1.0f;
@@ -306,6 +377,7 @@ __device__ __forceinline__ void pair_rows(int seg0, int cnt, int mt, int rank, T
   const int r0 = mt * 256 + rank * 128;
   t.a_row = seg0 + r0;
   t.m_valid = max(0, min(BM, cnt - r0));
+  t.swap_np = 0;
 }
 
 struct UpPairPolicy : GroupedSched<256, 2, 128, 256> {
@@ -570,10 +642,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint8_t* sa = tiles + stage * L::kStageBytes;
           const uint64_t ad = sw128_kmajor_desc(sa);
           const uint64_t bd = sw128_kmajor_desc(sa + kATileBytes);
+          if (BN == 256 && ti.swap_np) {
+            // D[:, 0:np) = B[0:128) A^T, D[:, np:2np) = B[128:256) A^T
+            const uint32_t idesc_s = idesc_bf16_f32(128, ti.swap_np);
+            const uint64_t bd_hi = bd + ((128u * 128u) >> 4);   // rows 128.. of the B stage
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk)
-            tc_mma_bf16(d_tmem, ad + 2u * kk, bd + 2u * kk, IDESC,
-                        (kb != ti.kb0 || kk != 0) ? 1u : 0u);
+            for (int kk = 0; kk < BK / 16; ++kk) {
+              const uint32_t accum = (kb != ti.kb0 || kk != 0) ? 1u : 0u;
+              tc_mma_bf16(d_tmem, bd + 2u * kk, ad + 2u * kk, idesc_s, accum);
+              tc_mma_bf16(d_tmem + static_cast<uint32_t>(ti.swap_np), bd_hi + 2u * kk,
+                          ad + 2u * kk, idesc_s, accum);
+            }
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk)
+              tc_mma_bf16(d_tmem, ad + 2u * kk, bd + 2u * kk, IDESC,
+                          (kb != ti.kb0 || kk != 0) ? 1u : 0u);
+          }
           tc_commit(empty + stage);
           if (++stage == STAGES) {
             stage = 0;
