@@ -75,7 +75,8 @@ struct Args {
   // grouped
   __nv_bfloat16* out;        // H [N, h] (up) or y [N, d] (down)
   const int32_t* src_row;    // gathered GEMM1: token of every expert-major slot
-  int src_rows;              // gathered GEMM1: rows of x (T); row T reads as zeros
+  int src_rows;              // gathered GEMM1: rows of x (T)
+  const void* gather_src;    // gathered GEMM1: x [T, K]
   const float* row_scale;    // down only, may be null
 };
 
@@ -100,6 +101,7 @@ struct RouterPolicy {
   static constexpr int BN = BN_;
   static constexpr int NUM_B = 1;
   static constexpr bool GATHER_A = false;
+  static constexpr int THREADS = kThreads;
   static constexpr int SCHED_INTS = 8;
 
   static __device__ void prologue(const Args&, int*) {}
@@ -154,6 +156,7 @@ struct GroupedSched {
   static constexpr int MROWS = MR;   // rows of one m-tile (256: a CTA pair)
   static constexpr int NUM_B = NUM_B_;
   static constexpr bool GATHER_A = false;
+  static constexpr int THREADS = kThreads;
   static constexpr int SCHED_INTS = 8 + 2 * (kMaxExperts + 1);
 
   static __device__ void prologue(const Args& a, int* sched) {
@@ -222,10 +225,11 @@ struct GroupedSched {
 // columns [0,128) = G, [128,256) = U.
 template <bool GATHER>
 struct UpPolicyT : GroupedSched<256, 2, 128> {
-  // With GATHER the A operand is not an expert-major copy of the tokens: the
-  // producer warp reads the 128 rows of a tile straight from x through
-  // src_row with TMA tile::gather4 (4 rows per instruction, one per lane).
+  // With GATHER the A operand is not an expert-major copy of the tokens: four
+  // extra warps copy the 128 rows of a tile straight from x through src_row
+  // (16-byte cp.async, one warp per pipeline stage).
   static constexpr bool GATHER_A = GATHER;
+  static constexpr int THREADS = GATHER ? kThreads + 128 : kThreads;
   static __device__ TileInfo tile_info(const Args& a, const int* sched, int tile) {
     int e, nt, mt, cnt, seg0;
     locate(a, sched, tile, e, nt, mt, cnt, seg0);
@@ -447,10 +451,11 @@ struct Layout {
   static constexpr int kLaunchBytes = kBytes + 1024;   // slack for 1 KB alignment
   static_assert(kLaunchBytes <= 227 * 1024, "shared memory budget");
   static_assert(kStages >= 2, "pipeline depth");
+  static_assert(!P::GATHER_A || kStages == 4, "one gather warp per stage (warps 6..9)");
 };
 
 template <class P>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(P::THREADS, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                    const __grid_constant__ CUtensorMap tmB1, const Args args) {
   using L = Layout<P>;
@@ -476,7 +481,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(full + s, 1);
+      mbar_init(full + s, P::GATHER_A ? 2 : 1);   // TMA producer (+ gather warp)
       mbar_init(empty + s, 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -505,57 +510,34 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int total = P::num_tiles(args, sched);
 
   if (warp == 0 && P::GATHER_A) {
-    // ------------------------------------ TMA producer, gathered A rows
-    // Lane l fetches rows 4l..4l+3 of every A tile with one tile::gather4
-    // (token ids from src_row; rows outside the segment read row src_rows,
-    // which is past the end of x and comes back as zeros); lane 0 owns the
-    // barriers and the weight loads.
-    const uint64_t pol_b = l2_policy_evict_last();
-    const uint64_t pol_a = l2_policy_evict_last();
-    int stage = 0;
-    uint32_t phase = 0;
-    int issued = 0;
-    bool ok = true;
-    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-      const TileInfo ti = P::tile_info(args, sched, tile);
-      int rows[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int r = 4 * lane + q;
-        int t = args.src_rows;
-        if (r < ti.m_valid) {
-          const int v = args.src_row[ti.a_row + r];
-          if (static_cast<unsigned>(v) < static_cast<unsigned>(args.src_rows)) t = v;
-        }
-        rows[q] = t;
-      }
-      for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
-        int go = 1;
-        if (lane == 0) go = mbar_wait(empty + stage, phase ^ 1u, abort_flag, args.status) ? 1 : 0;
-        go = __shfl_sync(0xffffffffu, go, 0);
-        if (!go) {
-          ok = false;
-          break;
-        }
-        uint8_t* sa = tiles + stage * L::kStageBytes;
-        uint8_t* sb = sa + kATileBytes;
-        if (lane == 0) {
-          mbar_arrive_expect_tx(full + stage, L::kStageBytes);
+    // ------------------------------ TMA producer of the weights (gathered A)
+    // The A rows of each stage are copied by the gather warps below; this
+    // thread loads the B tile and arms the barrier for its bytes only.
+    if (lane == 0) {
+      const uint64_t pol_b = l2_policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        const TileInfo ti = P::tile_info(args, sched, tile);
+        for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
+          if (!mbar_wait(empty + stage, phase ^ 1u, abort_flag, args.status)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sb = tiles + stage * L::kStageBytes + kATileBytes;
+          mbar_arrive_expect_tx(full + stage, L::kBTileBytes);
           tma_load_2d(sb, &tmB0, full + stage, kb * BK, ti.b_row, pol_b);
           if (P::NUM_B == 2)
             tma_load_2d(sb + L::kBTileBytes / 2, &tmB1, full + stage, kb * BK, ti.b_row, pol_b);
-        }
-        __syncwarp();
-        tma_gather4(sa + lane * 4 * (BK * 2), &tmA, full + stage, kb * BK, rows[0], rows[1],
-                    rows[2], rows[3], pol_a);
-        ++issued;
-        if (++stage == STAGES) {
-          stage = 0;
-          phase ^= 1u;
+          ++issued;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
         }
       }
-    }
-    if (lane == 0) {
       int s = stage;
       uint32_t ph = phase;
       for (int i = 0; i < min(issued, STAGES); ++i) {
@@ -567,6 +549,66 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_wait(full + s, ph, nullptr, args.status);
       }
+    }
+  } else if (P::GATHER_A && warp >= 6) {
+    // ------------------------------------ gather warps (A rows from x)
+    // Gather warp g owns stage g (STAGES gather warps): for every K block
+    // that lands in its stage it copies the tile's 128 rows x 64 columns
+    // from x[src_row[.]] with 16-byte cp.async into the 128-byte-swizzled
+    // K-major layout the MMA descriptor expects (chunk c of row r at
+    // (c ^ (r & 7)) * 16), waits for its copies, fences them into the async
+    // proxy and arrives on the stage's "full" barrier.  Rows outside the
+    // segment are zero-filled.
+    const int g = warp - 6;
+    int it = 0;
+    bool ok = true;
+    const __nv_bfloat16* xg = static_cast<const __nv_bfloat16*>(args.gather_src);
+    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      const TileInfo ti = P::tile_info(args, sched, tile);
+      const int nkb = ti.kb1 - ti.kb0;
+      // this warp's K blocks of the tile: global index it + j with (it + j) % STAGES == g
+      int j0 = (g - it % STAGES + STAGES) % STAGES;
+      if (j0 < nkb) {
+        int rows[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int r = 4 * lane + q;
+          int t = -1;
+          if (r < ti.m_valid) {
+            const int v = args.src_row[ti.a_row + r];
+            if (static_cast<unsigned>(v) < static_cast<unsigned>(args.src_rows)) t = v;
+          }
+          rows[q] = t;
+        }
+        for (int j = j0; j < nkb; j += STAGES) {
+          const int gi = it + j;                 // global K-block counter
+          const uint32_t phase = static_cast<uint32_t>(gi / STAGES) & 1u;
+          int go = 1;
+          if (lane == 0) go = mbar_wait(empty + g, phase ^ 1u, abort_flag, args.status) ? 1 : 0;
+          go = __shfl_sync(0xffffffffu, go, 0);
+          if (!go) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = tiles + g * L::kStageBytes;
+          const int col0 = (ti.kb0 + j) * BK;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int r = 4 * lane + q;
+            const __nv_bfloat16* src =
+                xg + static_cast<size_t>(rows[q] < 0 ? 0 : rows[q]) * args.K + col0;
+            const uint32_t nbytes = rows[q] < 0 ? 0u : 16u;
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              cp_async16(sa + r * 128 + ((c ^ (r & 7)) << 4), src + c * 8, nbytes);
+          }
+          cp_async_wait_all();
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(full + g);
+        }
+      }
+      it += nkb;
     }
   } else if (warp == 0) {
     if (lane == 0) {
@@ -671,7 +713,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_commit(mma_done);
       mbar_wait(mma_done, 0, nullptr, args.status);
     }
-  } else {
+  } else if (warp < 6) {
     // -------------------------------------------------- epilogue warps
     const int q = warp & 3;
     const int row = q * 32 + lane;
@@ -952,7 +994,7 @@ cudaError_t launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMa
     if (e != cudaSuccess) return e;
     configured[dev] = 1;
   }
-  launch_k(tc_gemm_kernel<P>, dim3(grid), dim3(kThreads), L::kLaunchBytes, s, a, b0, b1, args);
+  launch_k(tc_gemm_kernel<P>, dim3(grid), dim3(P::THREADS), L::kLaunchBytes, s, a, b0, b1, args);
   return cudaGetLastError();
 }
 
@@ -1081,6 +1123,7 @@ static cudaError_t swiglu_tc_impl(const void* a_src, int a_rows, const int32_t* 
   a.out = static_cast<__nv_bfloat16*>(H);
   a.src_row = src_row;
   a.src_rows = a_rows;
+  a.gather_src = a_src;
   if (pairs) {
     const long long max_pt = cdiv(N, 256) + E;   // upper bound on 256-row pair tiles
     int np = static_cast<int>(std::min<long long>(num_sms() / 2, max_pt * cdiv(h, 128)));
