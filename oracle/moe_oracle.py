@@ -45,7 +45,8 @@ from __future__ import annotations
 import numpy as np
 
 __all__ = [
-    "as_f64", "router_logits", "topk_select", "softmax", "router_topk",
+    "as_f64", "router_logits", "topk_select", "softmax", "router_topk", "sigmoid",
+    "node_limited_mask", "router_topk_general",
     "expert_counts", "dispatch", "permute_rows", "ep_dispatch_rank_major",
     "ep_local_regroup", "apply_row_perm", "silu", "swiglu_ffn",
     "grouped_swiglu", "combine", "moe_forward", "dense_moe", "moe_tokens",
@@ -124,6 +125,54 @@ def router_topk(top_k: int, renormalize: bool, x=None, w_router=None, logits=Non
         w = w / w.sum(axis=1, keepdims=True)
     counts = expert_counts(idx, L.shape[1])
     return idx, w, counts, L
+
+
+def sigmoid(L) -> np.ndarray:
+    """``1 / (1 + exp(-L))`` in fp64."""
+    L = as_f64(L)
+    with np.errstate(over="ignore"):
+        return 1.0 / (1.0 + np.exp(-L))
+
+
+def node_limited_mask(scores, num_groups: int, topk_groups: int) -> np.ndarray:
+    """Node-limited routing ([HP] ``_get_node_limited_routing_scores``): the
+    experts form ``num_groups`` equal consecutive groups; per token, the
+    ``topk_groups`` groups with the largest maximum score are kept (ties to
+    the lower group) and every expert of the other groups gets -inf."""
+    s = as_f64(scores)
+    T, E = s.shape
+    gs = E // num_groups
+    gmax = s.reshape(T, num_groups, gs).max(axis=2)
+    keep = topk_select(gmax, topk_groups)
+    mask = np.zeros((T, num_groups), dtype=bool)
+    mask[np.arange(T)[:, None], keep] = True
+    return np.where(np.repeat(mask, gs, axis=1), s, -np.inf)
+
+
+def router_topk_general(top_k: int, x=None, w_router=None, logits=None, score: str = "softmax",
+                        renormalize: bool = False, route_scale: float = 1.0, expert_bias=None,
+                        num_groups: int = 0, topk_groups: int = 0):
+    """Token-choice router with every option of [HP] ``TokenChoiceTopKRouter``,
+    in its order: gate logits -> ``score_func`` (softmax over the experts or
+    sigmoid) -> times ``route_scale`` -> node-limited group masking ->
+    plus ``expert_bias`` (selection only) -> top-k -> gather of the unbiased
+    scores as weights -> bincount.  With ``renormalize`` ([QO]
+    ``norm_topk_prob``) the gathered weights are divided by their sum; the
+    scale is applied after that division (so that it survives it; without
+    renormalisation this equals gathering the scaled scores).  Returns
+    ``(idx, w, counts, logits)`` like :func:`router_topk`."""
+    L = as_f64(logits) if logits is not None else router_logits(x, w_router)
+    E = L.shape[1]
+    s = softmax(L) if score == "softmax" else sigmoid(L)
+    scaled = s * route_scale
+    for_topk = node_limited_mask(scaled, num_groups, topk_groups) if num_groups else scaled
+    keys = for_topk + as_f64(expert_bias)[None, :] if expert_bias is not None else for_topk
+    idx = topk_select(keys, top_k)
+    w = np.take_along_axis(s, idx, axis=1)
+    if renormalize:
+        w = w / w.sum(axis=1, keepdims=True)
+    w = w * route_scale
+    return idx, w, expert_counts(idx, E), L
 
 
 def expert_counts(idx, E: int) -> np.ndarray:
@@ -309,24 +358,38 @@ def combine(y, dst_pos, topk_w=None) -> np.ndarray:
 # --------------------------------------------------------------------------
 
 def moe_forward(x, w_router, w1, w3, w2, top_k: int, renormalize: bool = True,
-                logits=None, ep_ranks: int = 1):
+                logits=None, ep_ranks: int = 1, router=None, score_before_experts=False):
     """Router -> dispatch -> (EP regroup) -> grouped SwiGLU -> combine.
 
     Returns a dict with every intermediate (fp64 / int64).  With
     ``ep_ranks > 1`` the routed rows are first laid out as received by
     ``ep_ranks`` simulated EP ranks and regrouped before the experts.
+    ``router`` (a dict of :func:`router_topk_general` options) selects the
+    general router.  With ``score_before_experts`` ([HP] ``MoE.forward``)
+    every routed row is multiplied by its routing weight before the experts
+    and the combine adds the expert outputs unweighted.
     """
     E = w1.shape[0]
-    idx, w, counts, L = router_topk(top_k, renormalize, x=x, w_router=w_router,
-                                    logits=logits)
+    if router is None:
+        idx, w, counts, L = router_topk(top_k, renormalize, x=x, w_router=w_router,
+                                        logits=logits)
+    else:
+        idx, w, counts, L = router_topk_general(top_k, x=x, w_router=w_router, logits=logits,
+                                                renormalize=renormalize, **router)
     res = {"logits": L, "topk_idx": idx, "topk_w": w}
     if ep_ranks == 1:
         c, off, src_row, dst_pos = dispatch(idx, E)
         res.update(counts=c, offsets=off, src_row=src_row, dst_pos=dst_pos)
         x_perm = permute_rows(x, src_row)
+        if score_before_experts:
+            slot_w = np.empty(len(src_row))
+            slot_w[_i64(dst_pos).ravel()] = w.ravel()
+            x_perm = x_perm * slot_w[:, None]
         y = grouped_swiglu(x_perm, off, w1, w3, w2)
-        res.update(x_perm=x_perm, y=y, out=combine(y, dst_pos, w))
+        out = combine(y, dst_pos, None if score_before_experts else w)
+        res.update(x_perm=x_perm, y=y, out=out)
         return res
+    assert not score_before_experts, "score_before_experts is defined on the single-device path"
     counts_rm, src_rm, dst_rm = ep_dispatch_rank_major(idx, E, ep_ranks)
     x_rm = permute_rows(x, src_rm)
     perm, counts_em, off_em = ep_local_regroup(counts_rm)
