@@ -161,27 +161,34 @@ def swiglu_algorithmic_bytes(cfg) -> int:
     return esz * (2 * cfg.N * cfg.d + 2 * cfg.N * cfg.h + 3 * cfg.E * cfg.h * cfg.d)
 
 
-def source_digest() -> str:
-    """Hash of the CUDA sources whose counters profiles/ records."""
+# Sources each profiled kernel is compiled from: a recorded DRAM traffic
+# figure is used only while these files are byte-identical to the capture.
+KERNEL_SOURCES = {
+    "grouped_swiglu": ["tc_gemm.cu", "common.cuh"],
+}
+
+
+def source_digest(kernel: str) -> str:
+    """Hash of the CUDA sources of `kernel` (KERNEL_SOURCES)."""
     import hashlib
     hsh = hashlib.sha256()
     csrc = os.path.join(ROOT, "routing_dispatch_grouped_topk_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh", ".h")):
-            hsh.update(open(os.path.join(csrc, f), "rb").read())
+    for f in KERNEL_SOURCES[kernel]:
+        hsh.update(f.encode())
+        hsh.update(open(os.path.join(csrc, f), "rb").read())
     return hsh.hexdigest()[:16]
 
 
 def profiled_traffic(kernel: str, workload: str):
     """DRAM bytes per launch measured by ncu (profiles/ncu_traffic.json), or
-    None when the kernels changed since the capture."""
+    None when the kernel's sources changed since the capture."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(p):
         return None
-    d = json.load(open(p))
-    if d.get("source_digest") != source_digest():
+    rec = json.load(open(p)).get("traffic", {}).get(workload, {}).get(kernel)
+    if not rec or rec.get("source_digest") != source_digest(kernel):
         return None
-    return d.get("traffic", {}).get(workload, {}).get(kernel)
+    return rec.get("dram_bytes_per_launch")
 
 
 # --------------------------------------------------------------- CPU oracle
