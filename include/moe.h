@@ -77,10 +77,10 @@ typedef enum {
 
 typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype_t;
 
-/* Score function of the router.  Only softmax is defined by the layers this
- * library targets ([HP] TokenChoiceTopKRouter with score_func="softmax",
- * [QO] SpeedupMoeSparseMoeBlock).  Other values return MOE_ERR_UNSUPPORTED. */
-typedef enum { MOE_SCORE_SOFTMAX = 0 } moe_score_t;
+/* Score function of the router ([HP] TokenChoiceTopKRouter, score_func):
+ * softmax over the E experts, or an element-wise sigmoid.  Other values
+ * return MOE_ERR_INVALID_ARG. */
+typedef enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID = 1 } moe_score_t;
 
 /* Bits of the device status word. */
 #define MOE_DEV_BAD_EXPERT 1   /* dispatch: expert id outside [0, E)            */
@@ -93,15 +93,16 @@ typedef enum { MOE_SCORE_SOFTMAX = 0 } moe_score_t;
 #define MOE_MAX_TOPK 16
 
 /* ------------------------------------------------------------------------
- * moe_router_topk -- [HP] TokenChoiceTopKRouter.forward, softmax branch;
- * [QO] SpeedupMoeSparseMoeBlock.forward (norm_topk_prob).
+ * moe_router_topk -- [HP] TokenChoiceTopKRouter.forward without bias,
+ * groups or scale; [QO] SpeedupMoeSparseMoeBlock.forward (norm_topk_prob).
  *
  *   scores  = logits_in            if logits_in != NULL
  *           = x @ w_router^T (fp32 accumulation, no rounding of the logits)
- *   p       = softmax(scores) over all E experts
+ *   p       = softmax(scores) over all E experts (score MOE_SCORE_SOFTMAX)
+ *           = sigmoid(scores)                    (score MOE_SCORE_SIGMOID)
  *   topk_idx[t, 0..k-1] = the k largest scores, largest first; equal scores
  *             go to the lower expert index (selection is made on the fp32
- *             scores; softmax is increasing so this is the top-k of p)
+ *             scores; p is increasing in them so this is the top-k of p)
  *   topk_w[t, j] = p[t, topk_idx[t, j]], divided by their sum over j when
  *             renormalize != 0
  *   counts[e] = number of (t, j) with topk_idx[t, j] == e
@@ -121,6 +122,65 @@ MOE_API moe_status_t moe_router_topk(const void* x, const void* w_router, const 
                              int renormalize, moe_dtype_t dt, float* logits_out,
                              int32_t* topk_idx, float* topk_w, int32_t* counts,
                              void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Router options -- the settings of [HP] TokenChoiceTopKRouter.__init__ and
+ * of the MoE module around it (expert_bias, tokens_per_expert,
+ * score_before_experts), taken by moe_router_topk_ex and moe_forward_ex.
+ *
+ * For token t with logits z (fp32) the router computes
+ *   s      = softmax(z) over the E experts, or sigmoid(z)      (score)
+ *   c      = s * route_scale
+ *   c'     = c with every expert outside the topk_groups groups of largest
+ *            max(c) set to -inf, when num_groups > 0 (node-limited routing;
+ *            groups are the num_groups equal runs of consecutive experts;
+ *            equal group maxima go to the lower group index)
+ *   key    = c' + expert_bias          (expert_bias may be NULL = 0)
+ *   topk_idx[t, :] = the k largest keys, largest first, ties to the lower
+ *            expert index
+ *   topk_w[t, j]   = s[topk_idx[t, j]] (the unbiased score, before the
+ *            scale), divided by the sum over j when renormalize != 0, then
+ *            times route_scale
+ *   tokens_per_expert[e] += number of (t, j) with topk_idx[t, j] == e
+ * Keys are compared in fp32.  Without expert_bias and with route_scale > 0
+ * the keys are increasing functions of z, and the selection (groups
+ * included) is made on z itself, so it is exact.
+ *
+ * score_before_experts (moe_forward_ex only; [HP] MoE.forward): the routed
+ * row of copy (t, j) is multiplied by topk_w[t, j] before the experts
+ * (fp32 product, rounded once to dt) and the combine is unweighted.
+ * moe_router_options_init sets the defaults: softmax, no renormalisation,
+ * route_scale 1, no bias, no groups, no histogram, and weights applied after
+ * the experts (score_before_experts = 0, the semantics of moe_forward).
+ *
+ * Rules: route_scale finite and != 0; num_groups = 0, or 1 <= num_groups
+ * <= 32 dividing E with 1 <= topk_groups <= num_groups and
+ * top_k <= topk_groups * (E / num_groups); expert_bias [E] fp32 device or
+ * NULL; tokens_per_expert [E] fp32 device or NULL (accumulated, never
+ * cleared by the library).
+ * ---------------------------------------------------------------------- */
+typedef struct moe_router_options {
+  moe_score_t score;
+  int renormalize;
+  float route_scale;
+  const float* expert_bias;
+  int num_groups;
+  int topk_groups;
+  float* tokens_per_expert;
+  int score_before_experts;
+} moe_router_options_t;
+
+MOE_API void moe_router_options_init(moe_router_options_t* opts);
+
+/* moe_router_topk_ex -- moe_router_topk with the options above (opts NULL =
+ * the defaults).  Same arguments, workspace, outputs and error rules as
+ * moe_router_topk otherwise; score_before_experts is ignored here. */
+MOE_API moe_status_t moe_router_topk_ex(const void* x, const void* w_router,
+                                        const float* logits_in, int T, int d, int E, int top_k,
+                                        const moe_router_options_t* opts, moe_dtype_t dt,
+                                        float* logits_out, int32_t* topk_idx, float* topk_w,
+                                        int32_t* counts, void* ws, size_t ws_bytes,
+                                        void* stream);
 
 /* ------------------------------------------------------------------------
  * moe_dispatch -- [HP] MoE.permutation (stable argsort of the flat expert
@@ -283,6 +343,18 @@ MOE_API moe_status_t moe_forward(const void* x, const void* w_router, const floa
                          moe_dtype_t dt, void* out, float* logits_out, int32_t* topk_idx,
                          float* topk_w, int32_t* counts, void* ws, size_t ws_bytes,
                          void* stream);
+
+/* moe_forward_ex -- [HP] MoE.forward with the router options above (opts
+ * NULL = the defaults, which make it moe_forward).  With
+ * score_before_experts the routed rows are scaled in the dispatch copy and
+ * the combine sums the expert outputs unweighted.  Same arguments,
+ * workspace (moe_forward_workspace_size) and error rules as moe_forward. */
+MOE_API moe_status_t moe_forward_ex(const void* x, const void* w_router, const float* logits_in,
+                                    const void* w1, const void* w3, const void* w2, int T, int d,
+                                    int E, int top_k, int h, const moe_router_options_t* opts,
+                                    int ep_ranks, moe_dtype_t dt, void* out, float* logits_out,
+                                    int32_t* topk_idx, float* topk_w, int32_t* counts, void* ws,
+                                    size_t ws_bytes, void* stream);
 
 /* Synchronises `stream`, then copies the status word at the start of `ws`
  * into *code (host).  Returns MOE_ERR_CUDA if the copy fails. */

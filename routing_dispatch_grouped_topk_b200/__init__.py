@@ -8,10 +8,13 @@ fallback: importing the binding without the built library raises.
 
 Two layers of API:
 
-* ``moe_router_topk``, ``moe_dispatch``, ``moe_ep_dispatch_rank_major``,
-  ``moe_ep_local_regroup``, ``moe_grouped_swiglu``, ``moe_combine``,
-  ``moe_forward`` -- same names and argument order as the C functions, with
-  torch tensors (or None) in place of pointers; outputs are caller-allocated.
+* ``moe_router_topk``, ``moe_router_topk_ex``, ``moe_dispatch``,
+  ``moe_ep_dispatch_rank_major``, ``moe_ep_local_regroup``,
+  ``moe_grouped_swiglu``, ``moe_combine``, ``moe_forward``,
+  ``moe_forward_ex`` -- same names and argument order as the C functions,
+  with torch tensors (or None) in place of pointers and a
+  ``RouterOptions`` structure for ``moe_router_options_t``; outputs are
+  caller-allocated.
 * ``router_topk``, ``dispatch``, ``ep_dispatch_rank_major``,
   ``ep_local_regroup``, ``grouped_swiglu``, ``combine``, ``forward`` --
   allocate their outputs and workspace with torch and return them.
@@ -26,6 +29,8 @@ import torch
 
 __all__ = [
     "MoEError", "lib", "LIB_PATH", "MOE_F32", "MOE_BF16", "MOE_SCORE_SOFTMAX",
+    "MOE_SCORE_SIGMOID", "RouterOptions", "router_options", "moe_router_options_init",
+    "moe_router_topk_ex", "moe_forward_ex",
     "MOE_DEV_BAD_EXPERT", "MOE_DEV_BAD_COUNTS", "MOE_DEV_BAD_OFFSETS", "MOE_DEV_TIMEOUT",
     "EXPORTED_SYMBOLS",
     "moe_router_topk", "moe_dispatch", "moe_ep_dispatch_rank_major", "moe_ep_local_regroup",
@@ -40,17 +45,18 @@ __all__ = [
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe.so")
 
 MOE_F32, MOE_BF16 = 0, 1
-MOE_SCORE_SOFTMAX = 0
+MOE_SCORE_SOFTMAX, MOE_SCORE_SIGMOID = 0, 1
 MOE_DEV_BAD_EXPERT, MOE_DEV_BAD_COUNTS, MOE_DEV_BAD_OFFSETS, MOE_DEV_TIMEOUT = 1, 2, 4, 8
 
 EXPORTED_SYMBOLS = [
-    "moe_router_workspace_size", "moe_router_topk",
+    "moe_router_workspace_size", "moe_router_topk", "moe_router_options_init",
+    "moe_router_topk_ex",
     "moe_dispatch_workspace_size", "moe_dispatch", "moe_dispatch_noalloc",
     "moe_ep_dispatch_workspace_size", "moe_ep_dispatch_rank_major",
     "moe_regroup_workspace_size", "moe_ep_local_regroup",
     "moe_grouped_swiglu_workspace_size", "moe_grouped_swiglu", "moe_grouped_swiglu_gather",
     "moe_combine",
-    "moe_forward_workspace_size", "moe_forward",
+    "moe_forward_workspace_size", "moe_forward", "moe_forward_ex",
     "moe_get_device_status", "moe_status_string", "moe_last_error", "moe_version",
 ]
 
@@ -59,12 +65,29 @@ class MoEError(RuntimeError):
     pass
 
 
+class RouterOptions(ctypes.Structure):
+    """``moe_router_options_t`` of include/moe.h (device pointers as ints)."""
+    _fields_ = [
+        ("score", ctypes.c_int),
+        ("renormalize", ctypes.c_int),
+        ("route_scale", ctypes.c_float),
+        ("expert_bias", ctypes.c_void_p),
+        ("num_groups", ctypes.c_int),
+        ("topk_groups", ctypes.c_int),
+        ("tokens_per_expert", ctypes.c_void_p),
+        ("score_before_experts", ctypes.c_int),
+    ]
+
+
 _P = ctypes.c_void_p
 _I = ctypes.c_int
 _Z = ctypes.c_size_t
 _SIGS = {
     "moe_router_workspace_size": (_Z, [_I, _I, _I, _I]),
     "moe_router_topk": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _Z, _P]),
+    "moe_router_options_init": (None, [ctypes.POINTER(RouterOptions)]),
+    "moe_router_topk_ex": (_I, [_P, _P, _P, _I, _I, _I, _I, ctypes.POINTER(RouterOptions), _I,
+                                _P, _P, _P, _P, _P, _Z, _P]),
     "moe_dispatch_workspace_size": (_Z, [_I, _I, _I]),
     "moe_dispatch": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _Z, _P]),
     "moe_dispatch_noalloc": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
@@ -82,6 +105,9 @@ _SIGS = {
     "moe_forward_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I, _I]),
     "moe_forward": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P,
                          _P, _P, _P, _Z, _P]),
+    "moe_forward_ex": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I,
+                            ctypes.POINTER(RouterOptions), _I, _I, _P, _P, _P, _P, _P, _P, _Z,
+                            _P]),
     "moe_get_device_status": (_I, [_P, ctypes.POINTER(_I), _P]),
     "moe_status_string": (ctypes.c_char_p, [_I]),
     "moe_last_error": (ctypes.c_char_p, []),
@@ -184,6 +210,44 @@ def moe_router_topk(x, w_router, logits_in, T, d, E, top_k, score, renormalize, 
         _ptr(ws, name="ws"), _nbytes(ws), _stream(stream)), "moe_router_topk")
 
 
+def moe_router_options_init() -> RouterOptions:
+    o = RouterOptions()
+    lib().moe_router_options_init(ctypes.byref(o))
+    return o
+
+
+def router_options(score="softmax", renormalize=False, route_scale=1.0, expert_bias=None,
+                   num_groups=0, topk_groups=0, tokens_per_expert=None,
+                   score_before_experts=False) -> RouterOptions:
+    """A RouterOptions from keyword values ([HP] TokenChoiceTopKRouter's
+    settings).  expert_bias / tokens_per_expert are fp32 CUDA tensors [E] or
+    None and must stay alive while the call that takes the options runs."""
+    o = moe_router_options_init()
+    o.score = {"softmax": MOE_SCORE_SOFTMAX, "sigmoid": MOE_SCORE_SIGMOID}[score]
+    o.renormalize = int(bool(renormalize))
+    o.route_scale = float(route_scale)
+    o.expert_bias = _ptr(expert_bias, torch.float32, "expert_bias")
+    o.num_groups = int(num_groups or 0)
+    o.topk_groups = int(topk_groups or 0)
+    o.tokens_per_expert = _ptr(tokens_per_expert, torch.float32, "tokens_per_expert")
+    o.score_before_experts = int(bool(score_before_experts))
+    return o
+
+
+def _opts(o: Optional[RouterOptions]):
+    return None if o is None else ctypes.byref(o)
+
+
+def moe_router_topk_ex(x, w_router, logits_in, T, d, E, top_k, opts, dt, logits_out, topk_idx,
+                       topk_w, counts, ws, stream=None):
+    _check(lib().moe_router_topk_ex(
+        _ptr(x, name="x"), _ptr(w_router, name="w_router"),
+        _ptr(logits_in, torch.float32, "logits_in"), T, d, E, top_k, _opts(opts), dt,
+        _ptr(logits_out, torch.float32, "logits_out"), _ptr(topk_idx, torch.int32, "topk_idx"),
+        _ptr(topk_w, torch.float32, "topk_w"), _ptr(counts, torch.int32, "counts"),
+        _ptr(ws, name="ws"), _nbytes(ws), _stream(stream)), "moe_router_topk_ex")
+
+
 def moe_dispatch(x, topk_idx, T, d, E, top_k, dt, counts, offsets, src_row, dst_pos, x_perm, ws,
                  stream=None):
     _check(lib().moe_dispatch(
@@ -252,6 +316,18 @@ def moe_forward(x, w_router, logits_in, w1, w3, w2, T, d, E, top_k, h, score, re
         "moe_forward")
 
 
+def moe_forward_ex(x, w_router, logits_in, w1, w3, w2, T, d, E, top_k, h, opts, ep_ranks, dt,
+                   out, logits_out, topk_idx, topk_w, counts, ws, stream=None):
+    _check(lib().moe_forward_ex(
+        _ptr(x, name="x"), _ptr(w_router, name="w_router"),
+        _ptr(logits_in, torch.float32, "logits_in"), _ptr(w1, name="w1"), _ptr(w3, name="w3"),
+        _ptr(w2, name="w2"), T, d, E, top_k, h, _opts(opts), ep_ranks, dt,
+        _ptr(out, name="out"), _ptr(logits_out, torch.float32, "logits_out"),
+        _ptr(topk_idx, torch.int32, "topk_idx"), _ptr(topk_w, torch.float32, "topk_w"),
+        _ptr(counts, torch.int32, "counts"), _ptr(ws, name="ws"), _nbytes(ws), _stream(stream)),
+        "moe_forward_ex")
+
+
 def moe_get_device_status(ws, stream=None) -> int:
     code = _I(0)
     _check(lib().moe_get_device_status(_ptr(ws, name="ws"), ctypes.byref(code), _stream(stream)),
@@ -264,9 +340,11 @@ device_status = moe_get_device_status
 
 # --------------------------------------------------- allocating wrappers
 def router_topk(x=None, w_router=None, top_k=1, renormalize=True, logits_in=None,
-                want_logits=False, E=None):
+                want_logits=False, E=None, **options):
     """Returns (topk_idx int32 [T,k], topk_w fp32 [T,k], counts int32 [E],
-    logits fp32 [T,E] or None, ws)."""
+    logits fp32 [T,E] or None, ws).  ``options`` are router_options()
+    keywords (score, route_scale, expert_bias, num_groups, topk_groups,
+    tokens_per_expert)."""
     src = logits_in if logits_in is not None else x
     dev = src.device
     if logits_in is not None:
@@ -283,8 +361,9 @@ def router_topk(x=None, w_router=None, top_k=1, renormalize=True, logits_in=None
     logits = torch.empty(T, E, dtype=torch.float32, device=dev) if (
         want_logits and logits_in is None) else None
     ws = _ws(router_workspace_size(T, d, E, dt), dev)
-    moe_router_topk(x, w_router, logits_in, T, d, E, top_k, MOE_SCORE_SOFTMAX, renormalize, dt,
-                    logits, idx, w, counts, ws)
+    opts = router_options(renormalize=renormalize, **options)
+    moe_router_topk_ex(x, w_router, logits_in, T, d, E, top_k, opts, dt, logits, idx, w, counts,
+                       ws)
     return idx, w, counts, logits, ws
 
 
@@ -368,9 +447,12 @@ def combine(y, dst_pos, topk_w=None, row_map=None):
 
 
 def forward(x, w_router, w1, w3, w2, top_k, renormalize=True, ep_ranks=1, logits_in=None,
-            want_router=False, ws=None, out=None):
+            want_router=False, ws=None, out=None, **options):
     """Whole layer.  Returns ``out`` ([T, d], x's dtype), or with
-    ``want_router`` a dict with out, topk_idx, topk_w, counts, logits, ws."""
+    ``want_router`` a dict with out, topk_idx, topk_w, counts, logits, ws.
+    ``options`` are router_options() keywords (score, route_scale,
+    expert_bias, num_groups, topk_groups, tokens_per_expert,
+    score_before_experts)."""
     T, d = x.shape
     E, h, _ = w1.shape
     dt = _dt(x)
@@ -386,8 +468,9 @@ def forward(x, w_router, w1, w3, w2, top_k, renormalize=True, ep_ranks=1, logits
         w = torch.empty(T, top_k, dtype=torch.float32, device=dev)
         counts = torch.empty(E, dtype=torch.int32, device=dev)
         logits = torch.empty(T, E, dtype=torch.float32, device=dev) if logits_in is None else None
-    moe_forward(x, w_router, logits_in, w1, w3, w2, T, d, E, top_k, h, MOE_SCORE_SOFTMAX,
-                renormalize, ep_ranks, dt, out, logits, idx, w, counts, ws)
+    opts = router_options(renormalize=renormalize, **options)
+    moe_forward_ex(x, w_router, logits_in, w1, w3, w2, T, d, E, top_k, h, opts, ep_ranks, dt, out,
+                   logits, idx, w, counts, ws)
     if want_router:
         return {"out": out, "topk_idx": idx, "topk_w": w, "counts": counts, "logits": logits,
                 "ws": ws}

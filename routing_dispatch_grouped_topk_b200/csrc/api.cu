@@ -5,6 +5,7 @@
 #include <stdio.h>
 
 #include <algorithm>
+#include <cmath>
 
 #include "common.cuh"
 #include "internal.h"
@@ -80,15 +81,39 @@ size_t router_ws(int T, int d, int E, moe_dtype_t dt) {
   return kStatusBytes + align_up(planes * T * E * sizeof(float), 256);
 }
 
+moe_router_options_t default_options() {
+  moe_router_options_t o;
+  o.score = MOE_SCORE_SOFTMAX;
+  o.renormalize = 0;
+  o.route_scale = 1.0f;
+  o.expert_bias = nullptr;
+  o.num_groups = 0;
+  o.topk_groups = 0;
+  o.tokens_per_expert = nullptr;
+  o.score_before_experts = 0;
+  return o;
+}
+
 moe_status_t check_router(const void* x, const void* w_router, const float* logits_in, int T,
-                          int d, int E, int top_k, moe_score_t score, moe_dtype_t dt,
+                          int d, int E, int top_k, const moe_router_options_t& o, moe_dtype_t dt,
                           const int32_t* topk_idx, const float* topk_w) {
   if (moe_status_t s = check_dtype(dt)) return s;
-  MOE_CHECK_ARG(score == MOE_SCORE_SOFTMAX, "score: only MOE_SCORE_SOFTMAX is defined");
+  MOE_CHECK_ARG(o.score == MOE_SCORE_SOFTMAX || o.score == MOE_SCORE_SIGMOID,
+                "score must be MOE_SCORE_SOFTMAX or MOE_SCORE_SIGMOID");
   MOE_CHECK_ARG(T >= 0, "T=%d must be >= 0", T);
   MOE_CHECK_ARG(E >= 1 && E <= kMaxExperts, "E=%d must be in [1, %d]", E, kMaxExperts);
   MOE_CHECK_ARG(top_k >= 1 && top_k <= std::min(E, kMaxTopK), "top_k=%d must be in [1, min(E, %d)]",
                 top_k, kMaxTopK);
+  MOE_CHECK_ARG(std::isfinite(o.route_scale) && o.route_scale != 0.0f,
+                "route_scale must be finite and non-zero");
+  if (o.num_groups != 0) {
+    MOE_CHECK_ARG(o.num_groups >= 1 && o.num_groups <= 32 && E % o.num_groups == 0,
+                  "num_groups=%d must be in [1, 32] and divide E=%d", o.num_groups, E);
+    MOE_CHECK_ARG(o.topk_groups >= 1 && o.topk_groups <= o.num_groups &&
+                      top_k <= o.topk_groups * (E / o.num_groups),
+                  "topk_groups=%d must be in [1, num_groups] and keep >= top_k experts",
+                  o.topk_groups);
+  }
   if (T > 0) {
     MOE_CHECK_ARG(topk_idx && topk_w, "topk_idx and topk_w are required");
     if (!logits_in) {
@@ -100,29 +125,42 @@ moe_status_t check_router(const void* x, const void* w_router, const float* logi
   return MOE_OK;
 }
 
+RouterOptions kernel_options(const moe_router_options_t& o) {
+  RouterOptions k;
+  k.sigmoid = o.score == MOE_SCORE_SIGMOID;
+  k.scale = o.route_scale;
+  k.bias = o.expert_bias;
+  k.groups = o.num_groups;
+  k.topk_groups = o.num_groups ? o.topk_groups : 0;
+  return k;
+}
+
 // Router launch sequence (status and counts already cleared by the caller).
 // With `plan` and `blk` the top-k kernel also writes the dispatch histogram.
 cudaError_t run_router(const void* x, const void* w_router, const float* logits_in, int T, int d,
-                       int E, int top_k, int renorm, moe_dtype_t dt, float* logits_out,
-                       int32_t* topk_idx, float* topk_w, int32_t* counts, void* scratch,
-                       int* status, cudaStream_t s, const DispatchPlan* plan = nullptr,
-                       int32_t* blk = nullptr) {
+                       int E, int top_k, const moe_router_options_t& o, moe_dtype_t dt,
+                       float* logits_out, int32_t* topk_idx, float* topk_w, int32_t* counts,
+                       void* scratch, int* status, cudaStream_t s,
+                       const DispatchPlan* plan = nullptr, int32_t* blk = nullptr) {
   if (T == 0) return cudaSuccess;
+  const RouterOptions ko = kernel_options(o);
+  const int renorm = o.renormalize;
+  float* tpe = o.tokens_per_expert;
   if (logits_in)
-    return launch_router_topk(logits_in, 1, T, E, top_k, renorm, nullptr, topk_idx, topk_w,
-                              counts, plan, blk, s);
+    return launch_router_topk(logits_in, 1, T, E, top_k, renorm, ko, nullptr, topk_idx, topk_w,
+                              counts, tpe, plan, blk, s);
   float* part = static_cast<float*>(scratch);
   if (router_uses_tc(E, dt)) {
     cudaError_t e = launch_router_tc(x, w_router, T, d, E, part, status, s);
     if (e != cudaSuccess) return e;
-    return launch_router_topk(part, router_plan(T, d).ksplit, T, E, top_k, renorm, logits_out,
-                              topk_idx, topk_w, counts, plan, blk, s);
+    return launch_router_topk(part, router_plan(T, d).ksplit, T, E, top_k, renorm, ko,
+                              logits_out, topk_idx, topk_w, counts, tpe, plan, blk, s);
   }
   float* L = logits_out ? logits_out : part;
   cudaError_t e = launch_router_logits_simt(x, w_router, T, d, E, dt, L, s);
   if (e != cudaSuccess) return e;
-  return launch_router_topk(L, 1, T, E, top_k, renorm, nullptr, topk_idx, topk_w, counts, plan,
-                            blk, s);
+  return launch_router_topk(L, 1, T, E, top_k, renorm, ko, nullptr, topk_idx, topk_w, counts, tpe,
+                            plan, blk, s);
 }
 
 size_t swiglu_ws(int N, int h, moe_dtype_t dt) {
@@ -281,11 +319,17 @@ size_t moe_router_workspace_size(int T, int d, int E, moe_dtype_t dt) {
   return router_ws(T, d, E, dt);
 }
 
-moe_status_t moe_router_topk(const void* x, const void* w_router, const float* logits_in, int T,
-                             int d, int E, int top_k, moe_score_t score, int renormalize,
-                             moe_dtype_t dt, float* logits_out, int32_t* topk_idx, float* topk_w,
-                             int32_t* counts, void* ws, size_t ws_bytes, void* stream) {
-  if (moe_status_t st = check_router(x, w_router, logits_in, T, d, E, top_k, score, dt, topk_idx,
+void moe_router_options_init(moe_router_options_t* opts) {
+  if (opts) *opts = default_options();
+}
+
+moe_status_t moe_router_topk_ex(const void* x, const void* w_router, const float* logits_in,
+                                int T, int d, int E, int top_k, const moe_router_options_t* opts,
+                                moe_dtype_t dt, float* logits_out, int32_t* topk_idx,
+                                float* topk_w, int32_t* counts, void* ws, size_t ws_bytes,
+                                void* stream) {
+  const moe_router_options_t o = opts ? *opts : default_options();
+  if (moe_status_t st = check_router(x, w_router, logits_in, T, d, E, top_k, o, dt, topk_idx,
                                      topk_w))
     return st;
   MOE_CHECK_ARG(ws != nullptr, "ws is required");
@@ -298,9 +342,20 @@ moe_status_t moe_router_topk(const void* x, const void* w_router, const float* l
   cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), s);
   if (e == cudaSuccess && counts) e = cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, s);
   if (e == cudaSuccess)
-    e = run_router(x, w_router, logits_in, T, d, E, top_k, renormalize, dt, logits_out, topk_idx,
-                   topk_w, counts, static_cast<char*>(ws) + kStatusBytes, status, s);
+    e = run_router(x, w_router, logits_in, T, d, E, top_k, o, dt, logits_out, topk_idx, topk_w,
+                   counts, static_cast<char*>(ws) + kStatusBytes, status, s);
   return cuda_status(e, "moe_router_topk");
+}
+
+moe_status_t moe_router_topk(const void* x, const void* w_router, const float* logits_in, int T,
+                             int d, int E, int top_k, moe_score_t score, int renormalize,
+                             moe_dtype_t dt, float* logits_out, int32_t* topk_idx, float* topk_w,
+                             int32_t* counts, void* ws, size_t ws_bytes, void* stream) {
+  moe_router_options_t o = default_options();
+  o.score = score;
+  o.renormalize = renormalize;
+  return moe_router_topk_ex(x, w_router, logits_in, T, d, E, top_k, &o, dt, logits_out, topk_idx,
+                            topk_w, counts, ws, ws_bytes, stream);
 }
 
 // ----------------------------------------------------------------- dispatch
@@ -490,13 +545,14 @@ size_t moe_forward_workspace_size(int T, int d, int E, int top_k, int h, int ep_
   return carve_forward(nullptr, T, d, E, top_k, h, ep_ranks, dt).bytes;
 }
 
-moe_status_t moe_forward(const void* x, const void* w_router, const float* logits_in,
-                         const void* w1, const void* w3, const void* w2, int T, int d, int E,
-                         int top_k, int h, moe_score_t score, int renormalize, int ep_ranks,
-                         moe_dtype_t dt, void* out, float* logits_out, int32_t* topk_idx,
-                         float* topk_w, int32_t* counts, void* ws, size_t ws_bytes,
-                         void* stream) {
-  if (moe_status_t st = check_router(x, w_router, logits_in, T, d, E, top_k, score, dt,
+moe_status_t moe_forward_ex(const void* x, const void* w_router, const float* logits_in,
+                            const void* w1, const void* w3, const void* w2, int T, int d, int E,
+                            int top_k, int h, const moe_router_options_t* opts, int ep_ranks,
+                            moe_dtype_t dt, void* out, float* logits_out, int32_t* topk_idx,
+                            float* topk_w, int32_t* counts, void* ws, size_t ws_bytes,
+                            void* stream) {
+  const moe_router_options_t o = opts ? *opts : default_options();
+  if (moe_status_t st = check_router(x, w_router, logits_in, T, d, E, top_k, o, dt,
                                      reinterpret_cast<int32_t*>(1), reinterpret_cast<float*>(1)))
     return st;
   const int N = T * top_k;
@@ -526,9 +582,8 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* logit
   const DispatchPlan p = make_dispatch_plan(T, E, top_k, R);
   // The router's top-k kernel also writes the dispatch histogram table.
   if (e == cudaSuccess)
-    e = run_router(x, w_router, logits_in, T, d, E, top_k, renormalize, dt, logits_out, idx, w,
-                   nullptr, f.router_scratch, f.status, s, &p,
-                   static_cast<int32_t*>(f.disp_ws));
+    e = run_router(x, w_router, logits_in, T, d, E, top_k, o, dt, logits_out, idx, w, nullptr,
+                   f.router_scratch, f.status, s, &p, static_cast<int32_t*>(f.disp_ws));
   if (e != cudaSuccess) return cuda_status(e, "moe_forward/router");
   int32_t* cnt_a = (R == 1 && counts) ? counts : f.counts_a;
   // The routed rows are materialised expert-major (single device) or
@@ -536,8 +591,11 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* logit
   // regrouped.  Materialising costs one 16-byte-vector copy pass; measured
   // on B200 it is faster than gathering GEMM1's rows with TMA gather4
   // (moe_grouped_swiglu_gather), whose 512-byte requests limit the loads.
+  // With score_before_experts the copy also scales each routed row by its
+  // weight and the combine below is unweighted.
+  const bool before = o.score_before_experts != 0;
   e = launch_dispatch(p, x, idx, d, dt, cnt_a, f.offsets_a, f.src_row, f.dst_pos, f.x_a,
-                      f.disp_ws, f.status, s, /*hist_done=*/T > 0);
+                      f.disp_ws, f.status, s, /*hist_done=*/T > 0, before ? w : nullptr);
   if (e != cudaSuccess) return cuda_status(e, "moe_forward/dispatch");
   const void* xe = f.x_a;
   const int32_t* off = f.offsets_a;
@@ -553,8 +611,21 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* logit
   }
   e = run_swiglu(xe, off, w1, w3, w2, nullptr, N, d, h, E, dt, f.y, f.H, f.status, s);
   if (e != cudaSuccess) return cuda_status(e, "moe_forward/grouped_swiglu");
-  e = launch_combine(f.y, f.dst_pos, row_map, w, T, d, N, top_k, dt, out, s);
+  e = launch_combine(f.y, f.dst_pos, row_map, before ? nullptr : w, T, d, N, top_k, dt, out, s);
   return cuda_status(e, "moe_forward/combine");
+}
+
+moe_status_t moe_forward(const void* x, const void* w_router, const float* logits_in,
+                         const void* w1, const void* w3, const void* w2, int T, int d, int E,
+                         int top_k, int h, moe_score_t score, int renormalize, int ep_ranks,
+                         moe_dtype_t dt, void* out, float* logits_out, int32_t* topk_idx,
+                         float* topk_w, int32_t* counts, void* ws, size_t ws_bytes,
+                         void* stream) {
+  moe_router_options_t o = default_options();
+  o.score = score;
+  o.renormalize = renormalize;
+  return moe_forward_ex(x, w_router, logits_in, w1, w3, w2, T, d, E, top_k, h, &o, ep_ranks, dt,
+                        out, logits_out, topk_idx, topk_w, counts, ws, ws_bytes, stream);
 }
 
 }  // extern "C"

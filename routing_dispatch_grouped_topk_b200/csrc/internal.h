@@ -41,22 +41,38 @@ struct DispatchPlan {
 DispatchPlan make_dispatch_plan(int T, int E, int top_k, int R);
 size_t dispatch_ws_bytes(const DispatchPlan& p);
 
+// Scoring options of the top-k kernel (moe_router_options_t without the
+// host-only fields).  sigmoid: score function; scale: route_scale; bias:
+// expert_bias [E] or null; groups / topk_groups: node-limited routing (0 =
+// off).
+struct RouterOptions {
+  int sigmoid = 0;
+  float scale = 1.0f;
+  const float* bias = nullptr;
+  int groups = 0;
+  int topk_groups = 0;
+};
+
 // Sum of `nsplit` partial logit arrays [nsplit, T, E] (in split order), then
-// softmax / top-k / renormalisation; writes the logits if asked.  With
+// scores / top-k / weights as `o` says; writes the logits if asked.  With
 // `plan` and `blk` it also writes the dispatch histogram table of `plan`
-// (so launch_dispatch can skip its histogram kernel); otherwise it adds the
-// expert histogram to `counts` when given.
+// (so launch_dispatch can skip its histogram kernel).  The expert histogram
+// is added to `counts` (int) and to `tokens_per_expert` (fp32) when given.
 cudaError_t launch_router_topk(const float* parts, int nsplit, int T, int E, int top_k,
-                               int renorm, float* logits_out, int32_t* topk_idx, float* topk_w,
-                               int32_t* counts, const DispatchPlan* plan, int32_t* blk,
-                               cudaStream_t s);
+                               int renorm, const RouterOptions& o, float* logits_out,
+                               int32_t* topk_idx, float* topk_w, int32_t* counts,
+                               float* tokens_per_expert, const DispatchPlan* plan,
+                               int32_t* blk, cudaStream_t s);
 
 // ---- dispatch -------------------------------------------------------------
 // hist_done: the histogram table in `ws` was already written (by the router).
+// row_w [T*k] (or null): copy f = t*k + j of row t is multiplied by row_w[f]
+// (fp32 product, one rounding to dt) as it is written to x_perm.
 cudaError_t launch_dispatch(const DispatchPlan& p, const void* x, const int32_t* topk_idx,
                             int d, moe_dtype_t dt, int32_t* counts, int32_t* offsets,
                             int32_t* src_row, int32_t* dst_pos, void* x_perm, void* ws,
-                            int* status, cudaStream_t s, bool hist_done = false);
+                            int* status, cudaStream_t s, bool hist_done = false,
+                            const float* row_w = nullptr);
 
 // ---- regroup ----------------------------------------------------------------
 size_t regroup_ws_bytes(int G, int R, int L);

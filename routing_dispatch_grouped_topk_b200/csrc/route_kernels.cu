@@ -141,6 +141,19 @@ __global__ void dispatch_colscan_kernel(int32_t* __restrict__ blk, int nblk, int
   }
 }
 
+// Eight bf16 or four fp32 values times w (fp32 product, rounded once).
+__device__ __forceinline__ uint4 scale_vec(uint4 v, float w, int bf16) {
+  uint32_t u[4] = {v.x, v.y, v.z, v.w};
+  if (bf16) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) u[i] = pack_bf16x2(bf16_lo(u[i]) * w, bf16_hi(u[i]) * w);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * w);
+  }
+  return make_uint4(u[0], u[1], u[2], u[3]);
+}
+
 // K3: stable slot of every copy (warp 0), then the row copies (all warps):
 // each token row is read once and written to its k slots with 16-byte stores.
 // Each block also turns the bin totals into bin offsets (a block scan of
@@ -153,7 +166,7 @@ __global__ void dispatch_scatter_kernel(const uint4* __restrict__ x, const int32
                                         int32_t* __restrict__ offsets,
                                         int32_t* __restrict__ src_row,
                                         int32_t* __restrict__ dst_pos, uint4* __restrict__ x_perm,
-                                        int row_vec) {
+                                        int row_vec, const float* __restrict__ row_w, int bf16) {
   pdl_wait();
   pdl_trigger();
   extern __shared__ int sm[];
@@ -205,6 +218,23 @@ __global__ void dispatch_scatter_kernel(const uint4* __restrict__ x, const int32
   __syncthreads();
   if (!x_perm) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  if (row_w) {
+    // [HP] MoE.forward with score_before_experts: routed row times its weight
+    for (int t = t0 + warp; t < t1; t += nw) {
+      const uint4* src = x + static_cast<size_t>(t) * row_vec;
+      const int* sl = slot + (t - t0) * k;
+      for (int c = lane; c < row_vec; c += 32) {
+        const uint4 v = src[c];
+        for (int j = 0; j < k; ++j) {
+          const int s = sl[j];
+          if (s >= 0)
+            x_perm[static_cast<size_t>(s) * row_vec + c] =
+                scale_vec(v, row_w[static_cast<size_t>(t) * k + j], bf16);
+        }
+      }
+    }
+    return;
+  }
   for (int t = t0 + warp; t < t1; t += nw) {
     const uint4* src = x + static_cast<size_t>(t) * row_vec;
     const int* sl = slot + (t - t0) * k;
@@ -243,7 +273,7 @@ size_t dispatch_ws_bytes(const DispatchPlan& p) {
 cudaError_t launch_dispatch(const DispatchPlan& p, const void* x, const int32_t* topk_idx,
                             int d, moe_dtype_t dt, int32_t* counts, int32_t* offsets,
                             int32_t* src_row, int32_t* dst_pos, void* x_perm, void* ws,
-                            int* status, cudaStream_t s, bool hist_done) {
+                            int* status, cudaStream_t s, bool hist_done, const float* row_w) {
   int32_t* blk = static_cast<int32_t*>(ws);
   if (p.T == 0) {
     cudaError_t e = cudaMemsetAsync(counts, 0, sizeof(int32_t) * p.nbins, s);
@@ -260,7 +290,8 @@ cudaError_t launch_dispatch(const DispatchPlan& p, const void* x, const int32_t*
   const size_t sm3 = (p.nbins + 33 + p.tb * p.k) * sizeof(int);
   launch_k(dispatch_scatter_kernel, dim3(p.nblk), dim3(256), sm3, s,
            static_cast<const uint4*>(x), topk_idx, p.T, p.k, p.E, p.R, p.L, p.S, p.tb, p.nbins,
-           blk, counts, offsets, src_row, dst_pos, static_cast<uint4*>(x_perm), row_vec);
+           blk, counts, offsets, src_row, dst_pos, static_cast<uint4*>(x_perm), row_vec, row_w,
+           dt == MOE_BF16 ? 1 : 0);
   return cudaGetLastError();
 }
 
@@ -533,28 +564,49 @@ __device__ __forceinline__ float key_score(int k) { return __int_as_float(k ^ ((
 // One warp per token; block b owns tokens [b*tpb, (b+1)*tpb).  Lane l holds
 // experts l, l+32, ... (EPL of them); the logit is the sum of the nsplit
 // partial values in split order.  The k winners come from k rounds of a warp
-// arg-max on (score desc, expert asc) done with two redux.sync reductions
-// (max of the score key, then min expert index among the lanes holding it);
-// lane j keeps winner j.  NaN scores count as -inf (indices stay valid).
+// arg-max on (key desc, expert asc) done with two redux.sync reductions
+// (max of the order-preserving key, then min expert index among the lanes
+// holding it); lane j keeps winner j.  NaN scores count as -inf.
+//
+// Selection keys ([HP] TokenChoiceTopKRouter.forward): the scores are
+// s = softmax or sigmoid of the logits; the keys are c = s * route_scale,
+// with the experts of groups outside the top `topk_groups` (by the group's
+// maximum c) masked, plus expert_bias.  Without a bias and with a positive
+// scale c is increasing in the logit, so the keys are the logits themselves
+// (no rounding of s can merge or swap them).  Weights are the unbiased s of
+// the winners, divided by their sum when renormalising, times route_scale;
+// for softmax the division by the softmax denominator and the
+// renormalisation are one division of the exponentials.
+//
 // With `blk` the block also writes its histogram of dispatch keys as column
-// b of the dispatch table blk[bin * gridDim.x + b]; with `counts` it adds its
-// expert histogram to counts.
+// b of the dispatch table blk[bin * gridDim.x + b]; `counts` (int) and
+// `tokens_per_expert` (float, accumulated with +=) get the expert histogram.
+constexpr int kMaskedKey = INT_MIN + 1;   // below score_key(-inf), above "none"
+
 template <int EPL>
 __global__ void __launch_bounds__(256) router_topk_kernel(
     const float* __restrict__ parts, int nsplit, int T, int E, int k, int renorm, int tpb,
-    float* __restrict__ logits_out, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
-    int32_t* __restrict__ counts, int32_t* __restrict__ blk, int nbins, int R, int L, int S) {
+    RouterOptions opt, float* __restrict__ logits_out, int32_t* __restrict__ topk_idx,
+    float* __restrict__ topk_w, int32_t* __restrict__ counts,
+    float* __restrict__ tokens_per_expert, int32_t* __restrict__ blk, int nbins, int R, int L,
+    int S) {
   pdl_wait();
   pdl_trigger();
-  extern __shared__ int bins[];   // nbins (dispatch keys) or E (counts)
-  const int nb = blk ? nbins : E;
-  const bool tally = blk != nullptr || counts != nullptr;
-  if (tally)
-    for (int i = threadIdx.x; i < nb; i += blockDim.x) bins[i] = 0;
+  extern __shared__ int sm_bins[];   // [nbins] dispatch keys (blk), then [E] experts
+  __shared__ int gkey[8][32];        // per-warp group maxima (node-limited routing)
+  int* dbins = sm_bins;
+  int* ebins = sm_bins + (blk ? nbins : 0);
+  const bool tally_e = counts != nullptr || tokens_per_expert != nullptr;
+  if (blk)
+    for (int i = threadIdx.x; i < nbins; i += blockDim.x) dbins[i] = 0;
+  if (tally_e)
+    for (int i = threadIdx.x; i < E; i += blockDim.x) ebins[i] = 0;
   __syncthreads();
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
   const size_t plane = static_cast<size_t>(T) * E;
+  const bool on_logits = opt.bias == nullptr && opt.scale > 0.f;
+  const int gsize = opt.groups ? E / opt.groups : 1;
   const int t_end = min(T, (blockIdx.x + 1) * tpb);
   for (int t = blockIdx.x * tpb + warp; t < t_end; t += nwarps) {
     float sv[EPL];
@@ -583,92 +635,155 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
 #pragma unroll
       for (int i = 0; i < EPL; ++i)
         if (avail[i]) sv[i] += base[sp * plane + 32 * i];
-    int key[EPL];
+    float mx = -INFINITY;
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
       if (avail[i] && logits_out) logits_out[static_cast<size_t>(t) * E + lane + 32 * i] = sv[i];
       if (sv[i] != sv[i]) sv[i] = -INFINITY;
-      key[i] = score_key(sv[i]);
+      if (avail[i]) mx = fmaxf(mx, sv[i]);
     }
-    int my_key = 0, my_e = 0, top_key = 0;
+    // ex = exp(z - max z) (softmax numerators) or sigmoid(z); s = ex / den
+    float ex[EPL];
+    float den = 1.f;
+    if (opt.sigmoid) {
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) ex[i] = avail[i] ? 1.0f / (1.0f + expf(-sv[i])) : 0.f;
+    } else {
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1)
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+      den = 0.f;
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) {
+        ex[i] = avail[i] ? expf(sv[i] - mx) : 0.f;
+        den += ex[i];
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
+    }
+    int key[EPL];
+    float kv[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      kv[i] = on_logits ? sv[i] : ex[i] / den * opt.scale;
+      key[i] = score_key(kv[i]);
+    }
+    if (opt.groups) {
+      // group maxima of the keys in shared memory, then the kept groups by
+      // redux rounds (largest maximum first, ties to the lower group)
+      gkey[warp][lane] = INT_MIN;
+      __syncwarp();
+#pragma unroll
+      for (int i = 0; i < EPL; ++i)
+        if (avail[i]) atomicMax(&gkey[warp][(lane + 32 * i) / gsize], key[i]);
+      __syncwarp();
+      const int gk = gkey[warp][lane];
+      unsigned kept = 0u;
+      bool gavail = lane < opt.groups;
+      for (int j = 0; j < opt.topk_groups; ++j) {
+        const int mk = __reduce_max_sync(0xffffffffu, gavail ? gk : INT_MIN);
+        const int bg = __reduce_min_sync(0xffffffffu, (gavail && gk == mk) ? lane : 31);
+        kept |= 1u << bg;
+        if (lane == bg) gavail = false;
+      }
+      __syncwarp();
+#pragma unroll
+      for (int i = 0; i < EPL; ++i)
+        if (!((kept >> min((lane + 32 * i) / gsize, 31)) & 1u)) key[i] = kMaskedKey;
+    }
+    if (opt.bias) {
+#pragma unroll
+      for (int i = 0; i < EPL; ++i)
+        if (avail[i] && key[i] != kMaskedKey) {
+          const float b = kv[i] + opt.bias[lane + 32 * i];
+          key[i] = score_key(b != b ? -INFINITY : b);
+        }
+    }
+    int my_e = 0;
+    float my_x = 0.f;
     for (int j = 0; j < k; ++j) {
       int lk = INT_MIN, li = 0x7fffffff;
+      float lx = 0.f;
 #pragma unroll
       for (int i = 0; i < EPL; ++i)
         if (avail[i] && key[i] > lk) {   // experts of a lane ascend with i: first max wins
           lk = key[i];
           li = lane + 32 * i;
+          lx = ex[i];
         }
       const int mk = __reduce_max_sync(0xffffffffu, lk);
       const int be = __reduce_min_sync(0xffffffffu, lk == mk ? li : 0x7fffffff);
+      const float bx = __shfl_sync(0xffffffffu, lx, be & 31);
 #pragma unroll
       for (int i = 0; i < EPL; ++i)
         if (lane + 32 * i == be) avail[i] = false;
-      if (j == 0) top_key = mk;
       if (lane == j) {
-        my_key = mk;
         my_e = be;
+        my_x = bx;
       }
     }
-    const float mx = key_score(top_key);
-    float se = 0.f;
+    // weights: the unbiased score of each winner (renormalised), times the scale
+    const float wx = lane < k ? my_x : 0.f;
+    float sel = wx;
 #pragma unroll
-    for (int i = 0; i < EPL; ++i)
-      if (lane + 32 * i < E) se += expf(sv[i] - mx);
-    const float ex = lane < k ? expf(key_score(my_key) - mx) : 0.f;
-    float sel = ex;
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      se += __shfl_xor_sync(0xffffffffu, se, off);
-      sel += __shfl_xor_sync(0xffffffffu, sel, off);
-    }
+    for (int off = 16; off > 0; off >>= 1) sel += __shfl_xor_sync(0xffffffffu, sel, off);
     if (lane < k) {
       const size_t o = static_cast<size_t>(t) * k + lane;
       topk_idx[o] = my_e;
-      topk_w[o] = ex / (renorm ? sel : se);
-      if (blk) atomicAdd(&bins[dispatch_key(my_e, t, R, L, S)], 1);
-      else if (counts) atomicAdd(&bins[my_e], 1);
+      topk_w[o] = wx / (renorm ? sel : den) * opt.scale;
+      if (blk) atomicAdd(&dbins[dispatch_key(my_e, t, R, L, S)], 1);
+      if (tally_e) atomicAdd(&ebins[my_e], 1);
     }
   }
-  if (!tally) return;
   __syncthreads();
-  if (blk) {
-    for (int i = threadIdx.x; i < nb; i += blockDim.x)
-      blk[static_cast<size_t>(i) * gridDim.x + blockIdx.x] = bins[i];
-  } else {
-    for (int i = threadIdx.x; i < nb; i += blockDim.x)
-      if (bins[i]) atomicAdd(&counts[i], bins[i]);
+  if (blk)
+    for (int i = threadIdx.x; i < nbins; i += blockDim.x)
+      blk[static_cast<size_t>(i) * gridDim.x + blockIdx.x] = dbins[i];
+  if (tally_e) {
+    for (int i = threadIdx.x; i < E; i += blockDim.x) {
+      const int c = ebins[i];
+      if (!c) continue;
+      if (counts) atomicAdd(&counts[i], c);
+      if (tokens_per_expert) atomicAdd(&tokens_per_expert[i], static_cast<float>(c));
+    }
   }
 }
 
 cudaError_t launch_router_topk(const float* parts, int nsplit, int T, int E, int top_k,
-                               int renorm, float* logits_out, int32_t* topk_idx, float* topk_w,
-                               int32_t* counts, const DispatchPlan* plan, int32_t* blk,
-                               cudaStream_t s) {
+                               int renorm, const RouterOptions& o, float* logits_out,
+                               int32_t* topk_idx, float* topk_w, int32_t* counts,
+                               float* tokens_per_expert, const DispatchPlan* plan,
+                               int32_t* blk, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
   const bool fuse = plan && blk;
   const int tpb = fuse ? plan->tb : 16;
   const int blocks = cdiv(T, tpb);
   const int nbins = fuse ? plan->nbins : 0;
-  const size_t smem = sizeof(int) * (fuse ? nbins : (counts ? E : 0));
+  const bool tally_e = counts || tokens_per_expert;
+  const size_t smem = sizeof(int) * ((fuse ? nbins : 0) + (tally_e ? E : 0));
   const int R = fuse ? plan->R : 1, L = fuse ? plan->L : E, S = fuse ? plan->S : T;
   int32_t* b = fuse ? blk : nullptr;
-  int32_t* c = fuse ? nullptr : counts;
+  const RouterOptions opt = o;
   if (E <= 32)
     launch_k(router_topk_kernel<1>, dim3(blocks), dim3(256), smem, s, parts, nsplit, T, E, top_k,
-             renorm, tpb, logits_out, topk_idx, topk_w, c, b, nbins, R, L, S);
+             renorm, tpb, opt, logits_out, topk_idx, topk_w, counts, tokens_per_expert, b,
+             nbins, R, L, S);
   else if (E <= 64)
     launch_k(router_topk_kernel<2>, dim3(blocks), dim3(256), smem, s, parts, nsplit, T, E, top_k,
-             renorm, tpb, logits_out, topk_idx, topk_w, c, b, nbins, R, L, S);
+             renorm, tpb, opt, logits_out, topk_idx, topk_w, counts, tokens_per_expert, b,
+             nbins, R, L, S);
   else if (E <= 128)
     launch_k(router_topk_kernel<4>, dim3(blocks), dim3(256), smem, s, parts, nsplit, T, E, top_k,
-             renorm, tpb, logits_out, topk_idx, topk_w, c, b, nbins, R, L, S);
+             renorm, tpb, opt, logits_out, topk_idx, topk_w, counts, tokens_per_expert, b,
+             nbins, R, L, S);
   else if (E <= 256)
     launch_k(router_topk_kernel<8>, dim3(blocks), dim3(256), smem, s, parts, nsplit, T, E, top_k,
-             renorm, tpb, logits_out, topk_idx, topk_w, c, b, nbins, R, L, S);
+             renorm, tpb, opt, logits_out, topk_idx, topk_w, counts, tokens_per_expert, b,
+             nbins, R, L, S);
   else
     launch_k(router_topk_kernel<16>, dim3(blocks), dim3(256), smem, s, parts, nsplit, T, E,
-             top_k, renorm, tpb, logits_out, topk_idx, topk_w, c, b, nbins, R, L, S);
+             top_k, renorm, tpb, opt, logits_out, topk_idx, topk_w, counts, tokens_per_expert,
+             b, nbins, R, L, S);
   return cudaGetLastError();
 }
 

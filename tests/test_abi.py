@@ -66,7 +66,7 @@ def test_workspace_sizes_are_host_only(L):
 
 
 @pytest.mark.parametrize("case", [
-    dict(top_k=0), dict(top_k=17), dict(E=0), dict(E=513), dict(T=-1), dict(dt=7), dict(score=1),
+    dict(top_k=0), dict(top_k=17), dict(E=0), dict(E=513), dict(T=-1), dict(dt=7), dict(score=2),
     dict(top_k=9, E=8),
 ])
 def test_router_rejects_bad_arguments(L, case):
@@ -120,3 +120,38 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(m, "_lib", None)
     with pytest.raises(m.MoEError, match="no CPU fallback"):
         m.lib()
+
+
+@pytest.mark.parametrize("case", [
+    dict(score=2), dict(route_scale=0.0), dict(route_scale=float("nan")),
+    dict(route_scale=float("inf")), dict(num_groups=3), dict(num_groups=64, E=128),
+    dict(num_groups=4, topk_groups=0), dict(num_groups=4, topk_groups=5),
+    dict(num_groups=4, topk_groups=1, top_k=3), dict(num_groups=-1),
+])
+def test_router_options_are_checked(L, case):
+    """Options the router cannot honour (include/moe.h, moe_router_options_t
+    rules) are rejected on the host before anything is launched."""
+    import routing_dispatch_grouped_topk_b200 as m
+    E = case.pop("E", 8)
+    top_k = case.pop("top_k", 2)
+    o = m.RouterOptions()
+    L.moe_router_options_init(ctypes.byref(o))
+    for k, v in case.items():
+        setattr(o, k, v)
+    p = ctypes.c_void_p(16)
+    r = L.moe_router_topk_ex(p, p, None, 4, 64, E, top_k, ctypes.byref(o), 1, None, p, p, None, p,
+                             1 << 20, None)
+    assert r == 1, L.moe_last_error()
+    r = L.moe_forward_ex(p, p, None, p, p, p, 4, 64, E, top_k, 64, ctypes.byref(o), 1, 1, p, None,
+                         None, None, None, p, 1 << 30, None)
+    assert r == 1, L.moe_last_error()
+
+
+def test_router_options_defaults(L):
+    import routing_dispatch_grouped_topk_b200 as m
+    o = m.RouterOptions()
+    o.route_scale = 7.0
+    o.num_groups = 3
+    L.moe_router_options_init(ctypes.byref(o))
+    assert (o.score, o.renormalize, o.route_scale, o.expert_bias, o.num_groups, o.topk_groups,
+            o.tokens_per_expert, o.score_before_experts) == (0, 0, 1.0, None, 0, 0, None, 0)
