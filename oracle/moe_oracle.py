@@ -358,7 +358,8 @@ def combine(y, dst_pos, topk_w=None) -> np.ndarray:
 # --------------------------------------------------------------------------
 
 def moe_forward(x, w_router, w1, w3, w2, top_k: int, renormalize: bool = True,
-                logits=None, ep_ranks: int = 1, router=None, score_before_experts=False):
+                logits=None, ep_ranks: int = 1, router=None, score_before_experts=False,
+                shared=None):
     """Router -> dispatch -> (EP regroup) -> grouped SwiGLU -> combine.
 
     Returns a dict with every intermediate (fp64 / int64).  With
@@ -367,8 +368,21 @@ def moe_forward(x, w_router, w1, w3, w2, top_k: int, renormalize: bool = True,
     ``router`` (a dict of :func:`router_topk_general` options) selects the
     general router.  With ``score_before_experts`` ([HP] ``MoE.forward``)
     every routed row is multiplied by its routing weight before the experts
-    and the combine adds the expert outputs unweighted.
+    and the combine adds the expert outputs unweighted.  ``shared`` =
+    ``(ws1 [hs, d], ws3 [hs, d], ws2 [d, hs])`` adds the shared expert, a
+    dense SwiGLU ``FeedForward`` on every token ([HP] ``MoE.forward``:
+    ``out = unpermutation(...) + shared_expert(x_flat)``).
     """
+    res = _moe_routed(x, w_router, w1, w3, w2, top_k, renormalize, logits, ep_ranks, router,
+                      score_before_experts)
+    if shared is not None:
+        res["shared_out"] = swiglu_ffn(x, *shared)
+        res["out"] = res["out"] + res["shared_out"]
+    return res
+
+
+def _moe_routed(x, w_router, w1, w3, w2, top_k, renormalize, logits, ep_ranks, router,
+                score_before_experts):
     E = w1.shape[0]
     if router is None:
         idx, w, counts, L = router_topk(top_k, renormalize, x=x, w_router=w_router,
