@@ -344,15 +344,35 @@ MOE_API moe_status_t moe_forward(const void* x, const void* w_router, const floa
                          float* topk_w, int32_t* counts, void* ws, size_t ws_bytes,
                          void* stream);
 
+/* Shared expert of [HP] MoE.forward (shared_expert = FeedForward(dim,
+ * hidden)): a dense SwiGLU on every token whose output is added to the routed
+ * output,  out[t] += (silu(x[t] w1^T) * (x[t] w3^T)) w2^T.
+ * w1, w3 [h, d] and w2 [d, h] in dt (device, 16-byte aligned); bf16 needs
+ * h % 64 == 0, fp32 h % 4 == 0. */
+typedef struct moe_shared_expert {
+  const void* w1;
+  const void* w3;
+  const void* w2;
+  int h;
+} moe_shared_expert_t;
+
 /* moe_forward_ex -- [HP] MoE.forward with the router options above (opts
- * NULL = the defaults, which make it moe_forward).  With
- * score_before_experts the routed rows are scaled in the dispatch copy and
- * the combine sums the expert outputs unweighted.  Same arguments,
- * workspace (moe_forward_workspace_size) and error rules as moe_forward. */
+ * NULL = the defaults) and an optional shared expert (shared NULL = none;
+ * both NULL make it moe_forward).  With score_before_experts the routed rows
+ * are scaled in the dispatch copy and the combine sums the expert outputs
+ * unweighted.  The shared expert runs as a one-segment grouped SwiGLU over
+ * x; the combine adds its row to each token's routed sum in fp32 before the
+ * single rounding to dt.  Workspace: moe_forward_ex_workspace_size with
+ * h_shared = shared->h (0 without a shared expert, which equals
+ * moe_forward_workspace_size).  Other arguments and error rules as
+ * moe_forward. */
+MOE_API size_t moe_forward_ex_workspace_size(int T, int d, int E, int top_k, int h, int ep_ranks,
+                                             moe_dtype_t dt, int h_shared);
 MOE_API moe_status_t moe_forward_ex(const void* x, const void* w_router, const float* logits_in,
                                     const void* w1, const void* w3, const void* w2, int T, int d,
                                     int E, int top_k, int h, const moe_router_options_t* opts,
-                                    int ep_ranks, moe_dtype_t dt, void* out, float* logits_out,
+                                    const moe_shared_expert_t* shared, int ep_ranks,
+                                    moe_dtype_t dt, void* out, float* logits_out,
                                     int32_t* topk_idx, float* topk_w, int32_t* counts, void* ws,
                                     size_t ws_bytes, void* stream);
 

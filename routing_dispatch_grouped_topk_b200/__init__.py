@@ -30,6 +30,7 @@ import torch
 __all__ = [
     "MoEError", "lib", "LIB_PATH", "MOE_F32", "MOE_BF16", "MOE_SCORE_SOFTMAX",
     "MOE_SCORE_SIGMOID", "RouterOptions", "router_options", "moe_router_options_init",
+    "SharedExpert", "shared_expert", "forward_ex_workspace_size",
     "moe_router_topk_ex", "moe_forward_ex",
     "MOE_DEV_BAD_EXPERT", "MOE_DEV_BAD_COUNTS", "MOE_DEV_BAD_OFFSETS", "MOE_DEV_TIMEOUT",
     "EXPORTED_SYMBOLS",
@@ -56,8 +57,8 @@ EXPORTED_SYMBOLS = [
     "moe_regroup_workspace_size", "moe_ep_local_regroup",
     "moe_grouped_swiglu_workspace_size", "moe_grouped_swiglu", "moe_grouped_swiglu_gather",
     "moe_combine",
-    "moe_forward_workspace_size", "moe_forward", "moe_forward_ex",
-    "moe_get_device_status", "moe_status_string", "moe_last_error", "moe_version",
+    "moe_forward_workspace_size", "moe_forward", "moe_forward_ex_workspace_size",
+    "moe_forward_ex", "moe_get_device_status", "moe_status_string", "moe_last_error", "moe_version",
 ]
 
 
@@ -76,6 +77,16 @@ class RouterOptions(ctypes.Structure):
         ("topk_groups", ctypes.c_int),
         ("tokens_per_expert", ctypes.c_void_p),
         ("score_before_experts", ctypes.c_int),
+    ]
+
+
+class SharedExpert(ctypes.Structure):
+    """``moe_shared_expert_t`` of include/moe.h (device pointers as ints)."""
+    _fields_ = [
+        ("w1", ctypes.c_void_p),
+        ("w3", ctypes.c_void_p),
+        ("w2", ctypes.c_void_p),
+        ("h", ctypes.c_int),
     ]
 
 
@@ -105,9 +116,10 @@ _SIGS = {
     "moe_forward_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I, _I]),
     "moe_forward": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P,
                          _P, _P, _P, _Z, _P]),
+    "moe_forward_ex_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I, _I, _I]),
     "moe_forward_ex": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I,
-                            ctypes.POINTER(RouterOptions), _I, _I, _P, _P, _P, _P, _P, _P, _Z,
-                            _P]),
+                            ctypes.POINTER(RouterOptions), ctypes.POINTER(SharedExpert), _I, _I,
+                            _P, _P, _P, _P, _P, _P, _Z, _P]),
     "moe_get_device_status": (_I, [_P, ctypes.POINTER(_I), _P]),
     "moe_status_string": (ctypes.c_char_p, [_I]),
     "moe_last_error": (ctypes.c_char_p, []),
@@ -198,6 +210,10 @@ def grouped_swiglu_workspace_size(N, d, h, E, dt) -> int:
 
 def forward_workspace_size(T, d, E, top_k, h, ep_ranks, dt) -> int:
     return lib().moe_forward_workspace_size(T, d, E, top_k, h, ep_ranks, dt)
+
+
+def forward_ex_workspace_size(T, d, E, top_k, h, ep_ranks, dt, h_shared=0) -> int:
+    return lib().moe_forward_ex_workspace_size(T, d, E, top_k, h, ep_ranks, dt, h_shared)
 
 
 def moe_router_topk(x, w_router, logits_in, T, d, E, top_k, score, renormalize, dt, logits_out,
@@ -316,12 +332,20 @@ def moe_forward(x, w_router, logits_in, w1, w3, w2, T, d, E, top_k, h, score, re
         "moe_forward")
 
 
-def moe_forward_ex(x, w_router, logits_in, w1, w3, w2, T, d, E, top_k, h, opts, ep_ranks, dt,
-                   out, logits_out, topk_idx, topk_w, counts, ws, stream=None):
+def shared_expert(w1, w3, w2) -> SharedExpert:
+    """A SharedExpert for weights w1, w3 [hs, d] and w2 [d, hs] (CUDA
+    tensors that must stay alive while the call that takes it runs)."""
+    return SharedExpert(_ptr(w1, name="shared w1"), _ptr(w3, name="shared w3"),
+                        _ptr(w2, name="shared w2"), int(w1.shape[0]))
+
+
+def moe_forward_ex(x, w_router, logits_in, w1, w3, w2, T, d, E, top_k, h, opts, shared,
+                   ep_ranks, dt, out, logits_out, topk_idx, topk_w, counts, ws, stream=None):
     _check(lib().moe_forward_ex(
         _ptr(x, name="x"), _ptr(w_router, name="w_router"),
         _ptr(logits_in, torch.float32, "logits_in"), _ptr(w1, name="w1"), _ptr(w3, name="w3"),
-        _ptr(w2, name="w2"), T, d, E, top_k, h, _opts(opts), ep_ranks, dt,
+        _ptr(w2, name="w2"), T, d, E, top_k, h, _opts(opts),
+        None if shared is None else ctypes.byref(shared), ep_ranks, dt,
         _ptr(out, name="out"), _ptr(logits_out, torch.float32, "logits_out"),
         _ptr(topk_idx, torch.int32, "topk_idx"), _ptr(topk_w, torch.float32, "topk_w"),
         _ptr(counts, torch.int32, "counts"), _ptr(ws, name="ws"), _nbytes(ws), _stream(stream)),
@@ -447,17 +471,19 @@ def combine(y, dst_pos, topk_w=None, row_map=None):
 
 
 def forward(x, w_router, w1, w3, w2, top_k, renormalize=True, ep_ranks=1, logits_in=None,
-            want_router=False, ws=None, out=None, **options):
+            want_router=False, ws=None, out=None, shared=None, **options):
     """Whole layer.  Returns ``out`` ([T, d], x's dtype), or with
     ``want_router`` a dict with out, topk_idx, topk_w, counts, logits, ws.
-    ``options`` are router_options() keywords (score, route_scale,
+    ``shared`` = (ws1 [hs, d], ws3 [hs, d], ws2 [d, hs]) adds a shared
+    expert.  ``options`` are router_options() keywords (score, route_scale,
     expert_bias, num_groups, topk_groups, tokens_per_expert,
     score_before_experts)."""
     T, d = x.shape
     E, h, _ = w1.shape
     dt = _dt(x)
     dev = x.device
-    need = forward_workspace_size(T, d, E, top_k, h, ep_ranks, dt)
+    sh = None if shared is None else shared_expert(*shared)
+    need = forward_ex_workspace_size(T, d, E, top_k, h, ep_ranks, dt, 0 if sh is None else sh.h)
     if ws is None or _nbytes(ws) < need:
         ws = _ws(need, dev)
     if out is None:
@@ -469,8 +495,8 @@ def forward(x, w_router, w1, w3, w2, top_k, renormalize=True, ep_ranks=1, logits
         counts = torch.empty(E, dtype=torch.int32, device=dev)
         logits = torch.empty(T, E, dtype=torch.float32, device=dev) if logits_in is None else None
     opts = router_options(renormalize=renormalize, **options)
-    moe_forward_ex(x, w_router, logits_in, w1, w3, w2, T, d, E, top_k, h, opts, ep_ranks, dt, out,
-                   logits, idx, w, counts, ws)
+    moe_forward_ex(x, w_router, logits_in, w1, w3, w2, T, d, E, top_k, h, opts, sh, ep_ranks, dt,
+                   out, logits, idx, w, counts, ws)
     if want_router:
         return {"out": out, "topk_idx": idx, "topk_w": w, "counts": counts, "logits": logits,
                 "ws": ws}

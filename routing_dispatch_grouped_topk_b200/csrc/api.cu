@@ -242,10 +242,14 @@ struct ForwardWs {
   void* reg_ws;
   void* y;
   void* H;
+  int32_t* offsets_s;   // shared expert (hs > 0): its one-segment offsets,
+  void* H_s;            // hidden activation [T, hs]
+  void* y_s;            // and output [T, d]
   size_t bytes;
 };
 
-ForwardWs carve_forward(void* ws, int T, int d, int E, int k, int h, int R, moe_dtype_t dt) {
+ForwardWs carve_forward(void* ws, int T, int d, int E, int k, int h, int R, moe_dtype_t dt,
+                        int hs = 0) {
   ForwardWs f{};
   Carve c(ws);
   const size_t N = static_cast<size_t>(T) * k;
@@ -271,6 +275,11 @@ ForwardWs carve_forward(void* ws, int T, int d, int E, int k, int h, int R, moe_
   }
   f.y = c.take<char>(N * row);
   f.H = c.take<char>(N * static_cast<size_t>(h) * elt_bytes(dt));
+  if (hs > 0) {
+    f.offsets_s = c.take<int32_t>(2);
+    f.H_s = c.take<char>(static_cast<size_t>(T) * hs * elt_bytes(dt));
+    f.y_s = c.take<char>(static_cast<size_t>(T) * row);
+  }
   f.bytes = c.off;
   return f;
 }
@@ -538,6 +547,14 @@ moe_status_t moe_combine(const void* y, const int32_t* dst_pos, const int32_t* r
 }
 
 // ------------------------------------------------------------------ forward
+size_t moe_forward_ex_workspace_size(int T, int d, int E, int top_k, int h, int ep_ranks,
+                                     moe_dtype_t dt, int h_shared) {
+  if (T < 0 || d < 1 || E < 1 || top_k < 1 || h < 1 || ep_ranks < 1 || E % ep_ranks ||
+      h_shared < 0)
+    return kStatusBytes;
+  return carve_forward(nullptr, T, d, E, top_k, h, ep_ranks, dt, h_shared).bytes;
+}
+
 size_t moe_forward_workspace_size(int T, int d, int E, int top_k, int h, int ep_ranks,
                                   moe_dtype_t dt) {
   if (T < 0 || d < 1 || E < 1 || top_k < 1 || h < 1 || ep_ranks < 1 || E % ep_ranks)
@@ -547,11 +564,22 @@ size_t moe_forward_workspace_size(int T, int d, int E, int top_k, int h, int ep_
 
 moe_status_t moe_forward_ex(const void* x, const void* w_router, const float* logits_in,
                             const void* w1, const void* w3, const void* w2, int T, int d, int E,
-                            int top_k, int h, const moe_router_options_t* opts, int ep_ranks,
-                            moe_dtype_t dt, void* out, float* logits_out, int32_t* topk_idx,
-                            float* topk_w, int32_t* counts, void* ws, size_t ws_bytes,
-                            void* stream) {
+                            int top_k, int h, const moe_router_options_t* opts,
+                            const moe_shared_expert_t* shared, int ep_ranks, moe_dtype_t dt,
+                            void* out, float* logits_out, int32_t* topk_idx, float* topk_w,
+                            int32_t* counts, void* ws, size_t ws_bytes, void* stream) {
   const moe_router_options_t o = opts ? *opts : default_options();
+  const int hs = shared ? shared->h : 0;
+  if (shared) {
+    MOE_CHECK_ARG(hs >= 1, "shared->h=%d must be >= 1", hs);
+    if (moe_status_t st = check_swiglu_shape(T, d, hs, 1, dt)) return st;
+    if (T > 0) {
+      MOE_CHECK_ARG(shared->w1 && shared->w3 && shared->w2,
+                    "shared expert w1, w3, w2 are required");
+      MOE_CHECK_ARG(aligned16(shared->w1) && aligned16(shared->w3) && aligned16(shared->w2),
+                    "shared expert weights must be 16-byte aligned");
+    }
+  }
   if (moe_status_t st = check_router(x, w_router, logits_in, T, d, E, top_k, o, dt,
                                      reinterpret_cast<int32_t*>(1), reinterpret_cast<float*>(1)))
     return st;
@@ -568,12 +596,12 @@ moe_status_t moe_forward_ex(const void* x, const void* w_router, const float* lo
     if (moe_status_t st = check_rows(d, dt, "forward")) return st;
   }
   MOE_CHECK_ARG(ws != nullptr, "ws is required");
-  const ForwardWs need = carve_forward(nullptr, T, d, E, top_k, h, ep_ranks, dt);
+  const ForwardWs need = carve_forward(nullptr, T, d, E, top_k, h, ep_ranks, dt, hs);
   if (ws_bytes < need.bytes) {
     set_last_error("forward workspace %zu < %zu", ws_bytes, need.bytes);
     return MOE_ERR_WORKSPACE;
   }
-  const ForwardWs f = carve_forward(ws, T, d, E, top_k, h, ep_ranks, dt);
+  const ForwardWs f = carve_forward(ws, T, d, E, top_k, h, ep_ranks, dt, hs);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int32_t* idx = topk_idx ? topk_idx : f.idx;
   float* w = topk_w ? topk_w : f.w;
@@ -611,7 +639,17 @@ moe_status_t moe_forward_ex(const void* x, const void* w_router, const float* lo
   }
   e = run_swiglu(xe, off, w1, w3, w2, nullptr, N, d, h, E, dt, f.y, f.H, f.status, s);
   if (e != cudaSuccess) return cuda_status(e, "moe_forward/grouped_swiglu");
-  e = launch_combine(f.y, f.dst_pos, row_map, before ? nullptr : w, T, d, N, top_k, dt, out, s);
+  // [HP] MoE.forward: shared_expert(x_flat), added to the routed output in
+  // the combine.
+  if (hs > 0 && T > 0) {
+    e = launch_single_segment(f.offsets_s, T, s);
+    if (e == cudaSuccess)
+      e = run_swiglu(x, f.offsets_s, shared->w1, shared->w3, shared->w2, nullptr, T, d, hs, 1,
+                     dt, f.y_s, f.H_s, f.status, s);
+    if (e != cudaSuccess) return cuda_status(e, "moe_forward/shared_expert");
+  }
+  e = launch_combine(f.y, f.dst_pos, row_map, before ? nullptr : w, T, d, N, top_k, dt, out, s,
+                     hs > 0 ? f.y_s : nullptr);
   return cuda_status(e, "moe_forward/combine");
 }
 
@@ -624,8 +662,9 @@ moe_status_t moe_forward(const void* x, const void* w_router, const float* logit
   moe_router_options_t o = default_options();
   o.score = score;
   o.renormalize = renormalize;
-  return moe_forward_ex(x, w_router, logits_in, w1, w3, w2, T, d, E, top_k, h, &o, ep_ranks, dt,
-                        out, logits_out, topk_idx, topk_w, counts, ws, ws_bytes, stream);
+  return moe_forward_ex(x, w_router, logits_in, w1, w3, w2, T, d, E, top_k, h, &o, nullptr,
+                        ep_ranks, dt, out, logits_out, topk_idx, topk_w, counts, ws, ws_bytes,
+                        stream);
 }
 
 }  // extern "C"

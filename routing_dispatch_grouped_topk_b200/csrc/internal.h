@@ -82,9 +82,13 @@ cudaError_t launch_regroup(const void* in, const int32_t* counts_rm, int G, int 
                            int* status, cudaStream_t s);
 
 // ---- combine ----------------------------------------------------------------
+// shared [T, d] (or null): a row added to each token's weighted sum in fp32
+// before the rounding (the shared expert's output).
 cudaError_t launch_combine(const void* y, const int32_t* dst_pos, const int32_t* row_map,
                            const float* topk_w, int T, int d, int N, int top_k, moe_dtype_t dt,
-                           void* out, cudaStream_t s);
+                           void* out, cudaStream_t s, const void* shared = nullptr);
+// offsets[0] = 0, offsets[1] = n: the segmentation of a single expert.
+cudaError_t launch_single_segment(int32_t* offsets, int n, cudaStream_t s);
 
 // ---- grouped SwiGLU -----------------------------------------------------
 // bf16 tcgen05 path: H (bf16 [N, h]) is scratch.

@@ -413,7 +413,7 @@ template <bool BF16, int KMAX>
 __global__ void __launch_bounds__(256) combine_kernel(
     const uint4* __restrict__ y, const int32_t* __restrict__ dst_pos,
     const int32_t* __restrict__ row_map, const float* __restrict__ w, int T, int row_vec, int N,
-    int k, uint4* __restrict__ out) {
+    int k, const uint4* __restrict__ shared, uint4* __restrict__ out) {
   pdl_wait();
   pdl_trigger();
   const int lane = threadIdx.x & 31;
@@ -465,6 +465,24 @@ __global__ void __launch_bounds__(256) combine_kernel(
           acc[3] = fmaf(wj, __uint_as_float(v[j].w), acc[3]);
         }
       }
+      if (shared) {   // [HP] MoE.forward: out + shared_expert(x)
+        const uint4 sv = shared[static_cast<size_t>(t) * row_vec + c];
+        if (BF16) {
+          acc[0] += bf16_lo(sv.x);
+          acc[1] += bf16_hi(sv.x);
+          acc[2] += bf16_lo(sv.y);
+          acc[3] += bf16_hi(sv.y);
+          acc[4] += bf16_lo(sv.z);
+          acc[5] += bf16_hi(sv.z);
+          acc[6] += bf16_lo(sv.w);
+          acc[7] += bf16_hi(sv.w);
+        } else {
+          acc[0] += __uint_as_float(sv.x);
+          acc[1] += __uint_as_float(sv.y);
+          acc[2] += __uint_as_float(sv.z);
+          acc[3] += __uint_as_float(sv.w);
+        }
+      }
       uint4 o;
       if (BF16) {
         o = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
@@ -480,33 +498,46 @@ __global__ void __launch_bounds__(256) combine_kernel(
 
 template <bool BF16>
 static void combine_launch(const uint4* y, const int32_t* dst_pos, const int32_t* row_map,
-                           const float* w, int T, int row_vec, int N, int k, uint4* out,
-                           int blocks, cudaStream_t s) {
+                           const float* w, int T, int row_vec, int N, int k,
+                           const uint4* shared, uint4* out, int blocks, cudaStream_t s) {
   if (k <= 1)
-    launch_k(combine_kernel<BF16, 1>, dim3(blocks), dim3(256), 0, s, y, dst_pos, row_map, w, T, row_vec, N, k, out);
+    launch_k(combine_kernel<BF16, 1>, dim3(blocks), dim3(256), 0, s, y, dst_pos, row_map, w, T, row_vec, N, k, shared, out);
   else if (k <= 2)
-    launch_k(combine_kernel<BF16, 2>, dim3(blocks), dim3(256), 0, s, y, dst_pos, row_map, w, T, row_vec, N, k, out);
+    launch_k(combine_kernel<BF16, 2>, dim3(blocks), dim3(256), 0, s, y, dst_pos, row_map, w, T, row_vec, N, k, shared, out);
   else if (k <= 4)
-    launch_k(combine_kernel<BF16, 4>, dim3(blocks), dim3(256), 0, s, y, dst_pos, row_map, w, T, row_vec, N, k, out);
+    launch_k(combine_kernel<BF16, 4>, dim3(blocks), dim3(256), 0, s, y, dst_pos, row_map, w, T, row_vec, N, k, shared, out);
   else if (k <= 8)
-    launch_k(combine_kernel<BF16, 8>, dim3(blocks), dim3(256), 0, s, y, dst_pos, row_map, w, T, row_vec, N, k, out);
+    launch_k(combine_kernel<BF16, 8>, dim3(blocks), dim3(256), 0, s, y, dst_pos, row_map, w, T, row_vec, N, k, shared, out);
   else
-    launch_k(combine_kernel<BF16, 16>, dim3(blocks), dim3(256), 0, s, y, dst_pos, row_map, w, T, row_vec, N, k, out);
+    launch_k(combine_kernel<BF16, 16>, dim3(blocks), dim3(256), 0, s, y, dst_pos, row_map, w, T, row_vec, N, k, shared, out);
 }
 
 cudaError_t launch_combine(const void* y, const int32_t* dst_pos, const int32_t* row_map,
                            const float* topk_w, int T, int d, int N, int top_k, moe_dtype_t dt,
-                           void* out, cudaStream_t s) {
+                           void* out, cudaStream_t s, const void* shared) {
   if (T == 0) return cudaSuccess;
   const int elt = dt == MOE_BF16 ? 2 : 4;
   const int row_vec = d * elt / 16;
   const int blocks = std::min(cdiv(T, 8), num_sms() * 8);
+  const uint4* sh = static_cast<const uint4*>(shared);
   if (dt == MOE_BF16)
     combine_launch<true>(static_cast<const uint4*>(y), dst_pos, row_map, topk_w, T, row_vec, N,
-                         top_k, static_cast<uint4*>(out), blocks, s);
+                         top_k, sh, static_cast<uint4*>(out), blocks, s);
   else
     combine_launch<false>(static_cast<const uint4*>(y), dst_pos, row_map, topk_w, T, row_vec, N,
-                          top_k, static_cast<uint4*>(out), blocks, s);
+                          top_k, sh, static_cast<uint4*>(out), blocks, s);
+  return cudaGetLastError();
+}
+
+__global__ void single_segment_kernel(int32_t* offsets, int n) {
+  pdl_wait();
+  pdl_trigger();
+  offsets[0] = 0;
+  offsets[1] = n;
+}
+
+cudaError_t launch_single_segment(int32_t* offsets, int n, cudaStream_t s) {
+  launch_k(single_segment_kernel, dim3(1), dim3(1), 0, s, offsets, n);
   return cudaGetLastError();
 }
 

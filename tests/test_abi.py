@@ -142,7 +142,7 @@ def test_router_options_are_checked(L, case):
     r = L.moe_router_topk_ex(p, p, None, 4, 64, E, top_k, ctypes.byref(o), 1, None, p, p, None, p,
                              1 << 20, None)
     assert r == 1, L.moe_last_error()
-    r = L.moe_forward_ex(p, p, None, p, p, p, 4, 64, E, top_k, 64, ctypes.byref(o), 1, 1, p, None,
+    r = L.moe_forward_ex(p, p, None, p, p, p, 4, 64, E, top_k, 64, ctypes.byref(o), None, 1, 1, p, None,
                          None, None, None, p, 1 << 30, None)
     assert r == 1, L.moe_last_error()
 
@@ -155,3 +155,20 @@ def test_router_options_defaults(L):
     L.moe_router_options_init(ctypes.byref(o))
     assert (o.score, o.renormalize, o.route_scale, o.expert_bias, o.num_groups, o.topk_groups,
             o.tokens_per_expert, o.score_before_experts) == (0, 0, 1.0, None, 0, 0, None, 0)
+
+
+def test_shared_expert_workspace_and_checks(L):
+    """moe_forward_ex_workspace_size with h_shared = 0 is moe_forward's;
+    a shared expert adds its [T, hs] hidden and [T, d] output; bad shared
+    experts are rejected before any launch."""
+    import routing_dispatch_grouped_topk_b200 as m
+    base = L.moe_forward_workspace_size(4096, 2048, 128, 8, 768, 1, 1)
+    assert L.moe_forward_ex_workspace_size(4096, 2048, 128, 8, 768, 1, 1, 0) == base
+    assert L.moe_forward_ex_workspace_size(4096, 2048, 128, 8, 768, 1, 1, 1024) >= \
+        base + 4096 * (1024 + 2048) * 2
+    p = ctypes.c_void_p(256)
+    for sh, code in [(m.SharedExpert(256, 256, 256, 0), 1), (m.SharedExpert(256, 256, 256, 96), 2),
+                     (m.SharedExpert(None, 256, 256, 128), 1), (m.SharedExpert(264, 256, 256, 128), 1)]:
+        r = L.moe_forward_ex(p, p, None, p, p, p, 4, 64, 8, 2, 64, None, ctypes.byref(sh), 1, 1, p,
+                             None, None, None, None, p, 1 << 30, None)
+        assert r == code, (sh.h, r, L.moe_last_error())
