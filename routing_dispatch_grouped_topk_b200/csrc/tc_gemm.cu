@@ -1,10 +1,10 @@
 // tcgen05 (5th-generation tensor core) GEMMs of the MoE layer on sm_100a.
 //
 // One warp-specialised, persistent kernel skeleton serves three problems:
-//   * the router        logits[T, E] = x[T, d] . w_router[E, d]^T, with the
-//                       softmax / top-k / renormalisation / histogram done in
-//                       the epilogue straight out of TMEM
-//                       ([HP] TokenChoiceTopKRouter.forward);
+//   * the router        fp32 partial logits of x[T, d] . w_router[E, d]^T,
+//                       split over d so that the (token tile, K split) tiles
+//                       fill the SMs; router_topk_kernel adds the splits
+//                       ([HP] TokenChoiceTopKRouter.forward, the gate);
 //   * GEMM1 (up)        for every expert segment, one 128 x 256 accumulator
 //                       holds x . w1^T (columns 0..127) and x . w3^T
 //                       (columns 128..255) for the same 128 hidden units; the
@@ -14,14 +14,19 @@
 //
 // Roles (192 threads): warp 0 issues TMA loads into a STAGES-deep ring of
 // shared-memory stages, warp 1 allocates TMEM and issues tcgen05.mma from one
-// thread, warps 2..5 drain the accumulator (tcgen05.ld) and write results.
-// Two TMEM accumulators let the epilogue of tile i overlap the MMAs of tile
-// i + 1.  Tiles are 128 rows (BM) x BN columns, K in steps of 64 bf16 (one
-// 128-byte swizzle row).  The expert tile schedule is built on the device
-// from the offsets array: no host synchronisation, no per-expert launches.
-// Tiles of one expert that share a weight tile are adjacent in the schedule,
-// so the CTAs that read the same weight tile run at the same time and the
-// second read hits L2.
+// thread, warps 2..5 drain the accumulator (tcgen05.ld) and write results
+// (the gathered GEMM1 adds four cp.async gather warps).  Two TMEM
+// accumulators let the epilogue of tile i overlap the MMAs of tile i + 1.
+// Tiles are 128 rows (BM) x BN columns, K in steps of 64 bf16 (one 128-byte
+// swizzle row).  The expert tile schedule is built on the device from the
+// offsets array: no host synchronisation, no per-expert launches.  Tiles of
+// one expert that share a weight tile are adjacent in the schedule, so the
+// CTAs that read the same weight tile run at the same time and the second
+// read hits L2.
+//
+// On B200 these kernels are bound by the delivery of operand tiles from L2
+// to shared memory (about 100 GB/s per SM), not by DRAM or the tensor pipe:
+// each 64-wide K block of a 128 x 256 tile moves 48 KB for 512 MMA cycles.
 //
 // Every mbarrier wait is bounded (2 s), sets MOE_DEV_TIMEOUT and unwinds;
 // the kernel then waits (bounded) for its own loads and MMAs and frees TMEM.
@@ -421,20 +426,6 @@ struct DownPairPolicy : GroupedSched<256, 1, 256, 256> {
 };
 
 // ------------------------------------------------------------- the kernel
-#ifndef MOE_L2_PREFETCH
-#define MOE_L2_PREFETCH 0
-#endif
-constexpr int kL2Prefetch = MOE_L2_PREFETCH;   // K blocks; 0 disables
-
-template <class P>
-__device__ __forceinline__ void prefetch_kblock(const CUtensorMap* a, const CUtensorMap* b0,
-                                                const CUtensorMap* b1, const TileInfo& ti,
-                                                int kb) {
-  if (kL2Prefetch == 0) return;
-  tma_prefetch_l2_2d(a, kb * BK, ti.a_row);
-  tma_prefetch_l2_2d(b0, kb * BK, ti.b_row);
-  if (P::NUM_B == 2) tma_prefetch_l2_2d(b1, kb * BK, ti.b_row);
-}
 
 template <class P>
 struct Layout {
@@ -621,12 +612,7 @@ __global__ void __launch_bounds__(P::THREADS, 1)
       bool ok = true;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         const TileInfo ti = P::tile_info(args, sched, tile);
-        // L2 prefetch kL2Prefetch K blocks ahead of the loads, so that a
-        // load issued when a stage frees up finds its data in L2.
-        for (int kb = ti.kb0; kb < min(ti.kb1, ti.kb0 + kL2Prefetch); ++kb)
-          prefetch_kblock<P>(&tmA, &tmB0, &tmB1, ti, kb);
         for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
-          if (kb + kL2Prefetch < ti.kb1) prefetch_kblock<P>(&tmA, &tmB0, &tmB1, ti, kb + kL2Prefetch);
           if (!mbar_wait(empty + stage, phase ^ 1u, abort_flag, args.status)) {
             ok = false;
             break;
