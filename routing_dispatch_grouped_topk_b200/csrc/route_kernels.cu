@@ -217,32 +217,30 @@ __global__ void dispatch_scatter_kernel(const uint4* __restrict__ x, const int32
   }
   __syncthreads();
   if (!x_perm) return;
+  // Row copies: a warp per token; each lane issues up to four 16-byte loads
+  // of the row before storing them to the token's k slots.
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-  if (row_w) {
-    // [HP] MoE.forward with score_before_experts: routed row times its weight
-    for (int t = t0 + warp; t < t1; t += nw) {
-      const uint4* src = x + static_cast<size_t>(t) * row_vec;
-      const int* sl = slot + (t - t0) * k;
-      for (int c = lane; c < row_vec; c += 32) {
-        const uint4 v = src[c];
-        for (int j = 0; j < k; ++j) {
-          const int s = sl[j];
-          if (s >= 0)
-            x_perm[static_cast<size_t>(s) * row_vec + c] =
-                scale_vec(v, row_w[static_cast<size_t>(t) * k + j], bf16);
-        }
-      }
-    }
-    return;
-  }
   for (int t = t0 + warp; t < t1; t += nw) {
     const uint4* src = x + static_cast<size_t>(t) * row_vec;
     const int* sl = slot + (t - t0) * k;
-    for (int c = lane; c < row_vec; c += 32) {
-      const uint4 v = src[c];
+    for (int c0 = 0; c0 < row_vec; c0 += 128) {
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int c = c0 + u * 32 + lane;
+        if (c < row_vec) v[u] = src[c];
+      }
       for (int j = 0; j < k; ++j) {
         const int s = sl[j];
-        if (s >= 0) x_perm[static_cast<size_t>(s) * row_vec + c] = v;
+        if (s < 0) continue;
+        uint4* dst = x_perm + static_cast<size_t>(s) * row_vec;
+        // [HP] MoE.forward with score_before_experts: routed row times its weight
+        const float wj = row_w ? row_w[static_cast<size_t>(t) * k + j] : 1.0f;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int c = c0 + u * 32 + lane;
+          if (c < row_vec) dst[c] = row_w ? scale_vec(v[u], wj, bf16) : v[u];
+        }
       }
     }
   }
@@ -391,15 +389,15 @@ cudaError_t launch_regroup(const void* in, const int32_t* counts_rm, int G, int 
   int32_t* in_start = static_cast<int32_t*>(ws);
   int32_t* out_start = in_start + S;
   int* flag = reinterpret_cast<int*>(out_start + S + 1);
-  launch_k(regroup_scan_kernel, dim3(1), dim3(1024), (S + 33) * sizeof(int), s, 
-      counts_rm, G, R, L, rows, in_start, out_start, counts_em, offsets_em, flag, status);
+  launch_k(regroup_scan_kernel, dim3(1), dim3(1024), (S + 33) * sizeof(int), s, counts_rm, G, R,
+           L, rows, in_start, out_start, counts_em, offsets_em, flag, status);
   if (rows > 0) {
     const int elt = dt == MOE_BF16 ? 2 : 4;
     const int row_vec = d * elt / 16;
     const int blocks = std::min(cdiv(rows, 8), num_sms() * 8);
-    launch_k(regroup_copy_kernel, dim3(blocks), dim3(256), 0, s, static_cast<const uint4*>(in), rows, row_vec, S,
-                                               in_start, out_start, flag,
-                                               static_cast<uint4*>(out), perm, perm_inv);
+    launch_k(regroup_copy_kernel, dim3(blocks), dim3(256), 0, s, static_cast<const uint4*>(in),
+             rows, row_vec, S, in_start, out_start, flag, static_cast<uint4*>(out), perm,
+             perm_inv);
   }
   return cudaGetLastError();
 }
