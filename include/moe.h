@@ -376,6 +376,16 @@ MOE_API moe_status_t moe_forward_ex(const void* x, const void* w_router, const f
                                     int32_t* topk_idx, float* topk_w, int32_t* counts, void* ws,
                                     size_t ws_bytes, void* stream);
 
+/* moe_selftest_timeout -- test of the failure path every pipeline of the
+ * library shares (no counterpart on the pages).  Launches one thread that
+ * waits, through the library's bounded mbarrier wait, on a shared-memory
+ * barrier that nothing arrives at.  After the wait limit (2 s of
+ * %globaltimer) the wait gives up, the kernel ORs MOE_DEV_TIMEOUT into the
+ * status word at the start of ws (cleared first) and returns; nothing
+ * faults or traps, and the context stays usable.  ws: device, >= 256 bytes.
+ * Asynchronous on `stream` like every entry point. */
+MOE_API moe_status_t moe_selftest_timeout(void* ws, size_t ws_bytes, void* stream);
+
 /* Synchronises `stream`, then copies the status word at the start of `ws`
  * into *code (host).  Returns MOE_ERR_CUDA if the copy fails. */
 MOE_API moe_status_t moe_get_device_status(const void* ws, int* code, void* stream);

@@ -58,7 +58,8 @@ EXPORTED_SYMBOLS = [
     "moe_grouped_swiglu_workspace_size", "moe_grouped_swiglu", "moe_grouped_swiglu_gather",
     "moe_combine",
     "moe_forward_workspace_size", "moe_forward", "moe_forward_ex_workspace_size",
-    "moe_forward_ex", "moe_get_device_status", "moe_status_string", "moe_last_error", "moe_version",
+    "moe_forward_ex", "moe_get_device_status", "moe_selftest_timeout", "moe_status_string",
+    "moe_last_error", "moe_version",
 ]
 
 
@@ -120,6 +121,7 @@ _SIGS = {
     "moe_forward_ex": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I,
                             ctypes.POINTER(RouterOptions), ctypes.POINTER(SharedExpert), _I, _I,
                             _P, _P, _P, _P, _P, _P, _Z, _P]),
+    "moe_selftest_timeout": (_I, [_P, _Z, _P]),
     "moe_get_device_status": (_I, [_P, ctypes.POINTER(_I), _P]),
     "moe_status_string": (ctypes.c_char_p, [_I]),
     "moe_last_error": (ctypes.c_char_p, []),
@@ -350,6 +352,11 @@ def moe_forward_ex(x, w_router, logits_in, w1, w3, w2, T, d, E, top_k, h, opts, 
         _ptr(topk_idx, torch.int32, "topk_idx"), _ptr(topk_w, torch.float32, "topk_w"),
         _ptr(counts, torch.int32, "counts"), _ptr(ws, name="ws"), _nbytes(ws), _stream(stream)),
         "moe_forward_ex")
+
+
+def moe_selftest_timeout(ws, stream=None):
+    _check(lib().moe_selftest_timeout(_ptr(ws, name="ws"), _nbytes(ws), _stream(stream)),
+           "moe_selftest_timeout")
 
 
 def moe_get_device_status(ws, stream=None) -> int:

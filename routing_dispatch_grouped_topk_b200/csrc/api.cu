@@ -307,6 +307,16 @@ const char* moe_status_string(moe_status_t s) {
   return "unknown status";
 }
 
+moe_status_t moe_selftest_timeout(void* ws, size_t ws_bytes, void* stream) {
+  MOE_CHECK_ARG(ws != nullptr && ws_bytes >= kStatusBytes, "ws of at least %zu bytes is required",
+                kStatusBytes);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* status = static_cast<int*>(ws);
+  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), s);
+  if (e == cudaSuccess) e = launch_selftest_timeout(status, s);
+  return cuda_status(e, "moe_selftest_timeout");
+}
+
 moe_status_t moe_get_device_status(const void* ws, int* code, void* stream) {
   if (!ws || !code) {
     set_last_error("ws and code are required");

@@ -87,6 +87,8 @@ cudaError_t launch_regroup(const void* in, const int32_t* counts_rm, int G, int 
 cudaError_t launch_combine(const void* y, const int32_t* dst_pos, const int32_t* row_map,
                            const float* topk_w, int T, int d, int N, int top_k, moe_dtype_t dt,
                            void* out, cudaStream_t s, const void* shared = nullptr);
+// Self-test of the bounded wait: sets MOE_DEV_TIMEOUT after kWaitLimitNs.
+cudaError_t launch_selftest_timeout(int* status, cudaStream_t s);
 // offsets[0] = 0, offsets[1] = n: the segmentation of a single expert.
 cudaError_t launch_single_segment(int32_t* offsets, int n, cudaStream_t s);
 

@@ -527,6 +527,22 @@ cudaError_t launch_combine(const void* y, const int32_t* dst_pos, const int32_t*
   return cudaGetLastError();
 }
 
+// One thread waits on a barrier that nothing arrives at; the bounded wait
+// gives up after kWaitLimitNs and records MOE_DEV_TIMEOUT.
+__global__ void selftest_timeout_kernel(int* status) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    mbar_wait(&bar, 0, nullptr, status);
+  }
+}
+
+cudaError_t launch_selftest_timeout(int* status, cudaStream_t s) {
+  selftest_timeout_kernel<<<1, 32, 0, s>>>(status);
+  return cudaGetLastError();
+}
+
 __global__ void single_segment_kernel(int32_t* offsets, int n) {
   pdl_wait();
   pdl_trigger();

@@ -172,3 +172,8 @@ def test_shared_expert_workspace_and_checks(L):
         r = L.moe_forward_ex(p, p, None, p, p, p, 4, 64, 8, 2, 64, None, ctypes.byref(sh), 1, 1, p,
                              None, None, None, None, p, 1 << 30, None)
         assert r == code, (sh.h, r, L.moe_last_error())
+
+
+def test_selftest_timeout_checks_its_workspace(L):
+    assert L.moe_selftest_timeout(None, 1 << 10, None) == 1
+    assert L.moe_selftest_timeout(ctypes.c_void_p(256), 16, None) == 1

@@ -53,3 +53,40 @@ def test_two_ranks_gloo():
     assert differ                       # independent token batches
     assert mx == 150.0                  # slowest rank sets the job time
     assert abs(val - 4096 * 2 * 10 / 0.150) < 1e-6
+
+
+def _failing_worker(rank, ws, port, q):
+    import datetime
+    import time
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=ws,
+                            timeout=datetime.timedelta(seconds=10))
+    import bench
+    dist.barrier()
+    if rank == 1:
+        raise SystemExit(3)             # a rank that leaves between steps
+    t0 = time.time()
+    try:
+        bench.max_over_ranks(1.0, ws, device="cpu")
+        q.put(("no error", time.time() - t0))
+    except Exception as e:              # the survivor's next collective fails
+        q.put((type(e).__name__, time.time() - t0))
+
+
+def test_a_rank_that_leaves_ends_the_others_collective():
+    """A rank that exits between steps: the surviving rank's next collective
+    (the max-over-ranks timing reduction) ends with an error within the
+    process group's timeout instead of waiting for ever."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_failing_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+    assert procs[1].exitcode == 3
+    assert procs[0].exitcode == 0
+    what, secs = q.get(timeout=10)
+    assert what != "no error"
+    assert secs < 60
