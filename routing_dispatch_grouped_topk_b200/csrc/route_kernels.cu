@@ -407,6 +407,60 @@ cudaError_t launch_regroup(const void* in, const int32_t* counts_rm, int G, int 
 // reads the position and weight of copy j once; they are broadcast by
 // shuffle.  Each lane walks the 16-byte chunks of the row and issues the k
 // loads of a chunk before accumulating them in order j = 0..k-1.
+// Weighted sum over the k copies of one 16-byte chunk (fp32, j in order),
+// plus the shared expert's chunk, rounded once.
+template <bool BF16, int KMAX>
+__device__ __forceinline__ uint4 combine_chunk(const uint4 (&v)[KMAX], const float (&wt)[KMAX],
+                                               const int (&pos)[KMAX], int k,
+                                               const uint4* shared) {
+  float acc[8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) acc[q] = 0.f;
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j) {
+    if (j >= k || pos[j] < 0) continue;
+    const float wj = wt[j];
+    if (BF16) {
+      acc[0] = fmaf(wj, bf16_lo(v[j].x), acc[0]);
+      acc[1] = fmaf(wj, bf16_hi(v[j].x), acc[1]);
+      acc[2] = fmaf(wj, bf16_lo(v[j].y), acc[2]);
+      acc[3] = fmaf(wj, bf16_hi(v[j].y), acc[3]);
+      acc[4] = fmaf(wj, bf16_lo(v[j].z), acc[4]);
+      acc[5] = fmaf(wj, bf16_hi(v[j].z), acc[5]);
+      acc[6] = fmaf(wj, bf16_lo(v[j].w), acc[6]);
+      acc[7] = fmaf(wj, bf16_hi(v[j].w), acc[7]);
+    } else {
+      acc[0] = fmaf(wj, __uint_as_float(v[j].x), acc[0]);
+      acc[1] = fmaf(wj, __uint_as_float(v[j].y), acc[1]);
+      acc[2] = fmaf(wj, __uint_as_float(v[j].z), acc[2]);
+      acc[3] = fmaf(wj, __uint_as_float(v[j].w), acc[3]);
+    }
+  }
+  if (shared) {   // [HP] MoE.forward: out + shared_expert(x)
+    const uint4 sv = *shared;
+    if (BF16) {
+      acc[0] += bf16_lo(sv.x);
+      acc[1] += bf16_hi(sv.x);
+      acc[2] += bf16_lo(sv.y);
+      acc[3] += bf16_hi(sv.y);
+      acc[4] += bf16_lo(sv.z);
+      acc[5] += bf16_hi(sv.z);
+      acc[6] += bf16_lo(sv.w);
+      acc[7] += bf16_hi(sv.w);
+    } else {
+      acc[0] += __uint_as_float(sv.x);
+      acc[1] += __uint_as_float(sv.y);
+      acc[2] += __uint_as_float(sv.z);
+      acc[3] += __uint_as_float(sv.w);
+    }
+  }
+  if (BF16)
+    return make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
+                      pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
+  return make_uint4(__float_as_uint(acc[0]), __float_as_uint(acc[1]), __float_as_uint(acc[2]),
+                    __float_as_uint(acc[3]));
+}
+
 template <bool BF16, int KMAX>
 __global__ void __launch_bounds__(256) combine_kernel(
     const uint4* __restrict__ y, const int32_t* __restrict__ dst_pos,
@@ -435,61 +489,25 @@ __global__ void __launch_bounds__(256) combine_kernel(
       wt[j] = __shfl_sync(0xffffffffu, my_w, j);
     }
     uint4* orow = out + static_cast<size_t>(t) * row_vec;
-    for (int c = lane; c < row_vec; c += 32) {
-      uint4 v[KMAX];
+    // Two 16-byte chunks per lane per iteration: 2k row loads in flight.
+    for (int c0 = lane; c0 < row_vec; c0 += 64) {
+      uint4 v[2][KMAX];
 #pragma unroll
-      for (int j = 0; j < KMAX; ++j)
-        if (j < k && pos[j] >= 0) v[j] = y[static_cast<size_t>(pos[j]) * row_vec + c];
-      float acc[8];
+      for (int h = 0; h < 2; ++h) {
+        const int c = c0 + 32 * h;
 #pragma unroll
-      for (int q = 0; q < 8; ++q) acc[q] = 0.f;
+        for (int j = 0; j < KMAX; ++j)
+          if (c < row_vec && j < k && pos[j] >= 0)
+            v[h][j] = y[static_cast<size_t>(pos[j]) * row_vec + c];
+      }
 #pragma unroll
-      for (int j = 0; j < KMAX; ++j) {
-        if (j >= k || pos[j] < 0) continue;
-        const float wj = wt[j];
-        if (BF16) {
-          acc[0] = fmaf(wj, bf16_lo(v[j].x), acc[0]);
-          acc[1] = fmaf(wj, bf16_hi(v[j].x), acc[1]);
-          acc[2] = fmaf(wj, bf16_lo(v[j].y), acc[2]);
-          acc[3] = fmaf(wj, bf16_hi(v[j].y), acc[3]);
-          acc[4] = fmaf(wj, bf16_lo(v[j].z), acc[4]);
-          acc[5] = fmaf(wj, bf16_hi(v[j].z), acc[5]);
-          acc[6] = fmaf(wj, bf16_lo(v[j].w), acc[6]);
-          acc[7] = fmaf(wj, bf16_hi(v[j].w), acc[7]);
-        } else {
-          acc[0] = fmaf(wj, __uint_as_float(v[j].x), acc[0]);
-          acc[1] = fmaf(wj, __uint_as_float(v[j].y), acc[1]);
-          acc[2] = fmaf(wj, __uint_as_float(v[j].z), acc[2]);
-          acc[3] = fmaf(wj, __uint_as_float(v[j].w), acc[3]);
-        }
+      for (int h = 0; h < 2; ++h) {
+        const int c = c0 + 32 * h;
+        if (c >= row_vec) break;
+        orow[c] = combine_chunk<BF16, KMAX>(v[h], wt, pos, k,
+                                            shared ? shared + static_cast<size_t>(t) * row_vec + c
+                                                   : nullptr);
       }
-      if (shared) {   // [HP] MoE.forward: out + shared_expert(x)
-        const uint4 sv = shared[static_cast<size_t>(t) * row_vec + c];
-        if (BF16) {
-          acc[0] += bf16_lo(sv.x);
-          acc[1] += bf16_hi(sv.x);
-          acc[2] += bf16_lo(sv.y);
-          acc[3] += bf16_hi(sv.y);
-          acc[4] += bf16_lo(sv.z);
-          acc[5] += bf16_hi(sv.z);
-          acc[6] += bf16_lo(sv.w);
-          acc[7] += bf16_hi(sv.w);
-        } else {
-          acc[0] += __uint_as_float(sv.x);
-          acc[1] += __uint_as_float(sv.y);
-          acc[2] += __uint_as_float(sv.z);
-          acc[3] += __uint_as_float(sv.w);
-        }
-      }
-      uint4 o;
-      if (BF16) {
-        o = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
-                       pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
-      } else {
-        o = make_uint4(__float_as_uint(acc[0]), __float_as_uint(acc[1]),
-                       __float_as_uint(acc[2]), __float_as_uint(acc[3]));
-      }
-      orow[c] = o;
     }
   }
 }
