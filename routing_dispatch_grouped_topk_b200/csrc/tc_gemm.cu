@@ -1090,11 +1090,10 @@ static cudaError_t swiglu_tc_impl(const void* a_src, int a_rows, const int32_t* 
   if (!make_tmap(&t3, w3, d, static_cast<uint64_t>(E) * h, 128)) return cudaErrorInvalidValue;
   if (!make_tmap(&th, H, h, N, BM)) return cudaErrorInvalidValue;
   // The CTA-pair kernel (256-row tiles, 2/3 of the loads per SM) measured
-  // no faster than single-CTA 128-row tiles on B200 under the power cap for
-  // segments of ~256 (uniform) to ~1024 (Zipf-skewed) average rows, and its
-  // 256-row tiles pad more on short segments; it is used only when segments
-  // average more than 1024 rows.
-  const bool pairs = !gather && N > 1024 * E;
+  // 5-10% slower than single-CTA 128-row tiles on B200 for segments of ~256
+  // average rows (its 256-row tiles pad to 1.5 tiles per expert) and ~2%
+  // faster at 1024 average rows (Zipf-skewed); it is used from 1024 up.
+  const bool pairs = !gather && N >= 1024 * E;
   if (!make_tmap(&t2, w2, h, static_cast<uint64_t>(E) * d, pairs ? 128 : 256))
     return cudaErrorInvalidValue;
   const int max_mt = cdiv(N, BM) + E;   // upper bound on m-tiles over all segments
