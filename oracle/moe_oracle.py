@@ -46,7 +46,7 @@ import numpy as np
 
 __all__ = [
     "as_f64", "router_logits", "topk_select", "softmax", "router_topk", "sigmoid",
-    "node_limited_mask", "router_topk_general",
+    "node_limited_mask", "router_topk_general", "load_balance_loss",
     "expert_counts", "dispatch", "permute_rows", "ep_dispatch_rank_major",
     "ep_local_regroup", "apply_row_perm", "silu", "swiglu_ffn",
     "grouped_swiglu", "combine", "moe_forward", "dense_moe", "moe_tokens",
@@ -173,6 +173,29 @@ def router_topk_general(top_k: int, x=None, w_router=None, logits=None, score: s
         w = w / w.sum(axis=1, keepdims=True)
     w = w * route_scale
     return idx, w, expert_counts(idx, E), L
+
+
+def load_balance_loss(top_scores, selected_experts, E: int) -> float:
+    """Auxiliary load-balance loss of one router call ([HP]
+    ``_compute_load_balance_loss``, without the sequence-partition
+    all-reduce): with ``f_e`` the fraction of the ``T*k`` routed copies that
+    go to expert e and ``P_e`` the sum of those copies' routing weights
+    divided by T, the loss is ``E * sum_e f_e * P_e``; 0 for no tokens.
+    The caller multiplies it by its coefficient."""
+    w = as_f64(top_scores)
+    idx = _i64(selected_experts)
+    T, k = idx.shape
+    if T == 0:
+        return 0.0
+    frac = np.zeros(E)
+    prob = np.zeros(E)
+    for t in range(T):
+        for j in range(k):
+            frac[idx[t, j]] += 1.0
+            prob[idx[t, j]] += w[t, j]
+    frac /= T * k
+    prob /= T
+    return float(E * np.sum(frac * prob))
 
 
 def expert_counts(idx, E: int) -> np.ndarray:
