@@ -142,6 +142,11 @@ MOE_API moe_status_t moe_router_topk(const void* x, const void* w_router, const 
  *            scale), divided by the sum over j when renormalize != 0, then
  *            times route_scale
  *   tokens_per_expert[e] += number of (t, j) with topk_idx[t, j] == e
+ *   *aux_loss = E * sum_e f_e * P_e, f_e = #{(t, j): topk_idx = e} / (T k),
+ *            P_e = sum of those copies' topk_w / T: the load-balance loss of
+ *            this call ([HP] _compute_load_balance_loss without the
+ *            sequence-partition reduction; 0 for T = 0; P_e is summed with
+ *            fp32 atomics, so its last bits depend on the order of blocks)
  * Keys are compared in fp32.  Without expert_bias and with route_scale > 0
  * the keys are increasing functions of z, and the selection (groups
  * included) is made on z itself, so it is exact.
@@ -157,7 +162,7 @@ MOE_API moe_status_t moe_router_topk(const void* x, const void* w_router, const 
  * <= 32 dividing E with 1 <= topk_groups <= num_groups and
  * top_k <= topk_groups * (E / num_groups); expert_bias [E] fp32 device or
  * NULL; tokens_per_expert [E] fp32 device or NULL (accumulated, never
- * cleared by the library).
+ * cleared by the library); aux_loss one fp32 device scalar or NULL (written).
  * ---------------------------------------------------------------------- */
 typedef struct moe_router_options {
   moe_score_t score;
@@ -168,6 +173,7 @@ typedef struct moe_router_options {
   int topk_groups;
   float* tokens_per_expert;
   int score_before_experts;
+  float* aux_loss;
 } moe_router_options_t;
 
 MOE_API void moe_router_options_init(moe_router_options_t* opts);

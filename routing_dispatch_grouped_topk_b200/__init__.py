@@ -78,6 +78,7 @@ class RouterOptions(ctypes.Structure):
         ("topk_groups", ctypes.c_int),
         ("tokens_per_expert", ctypes.c_void_p),
         ("score_before_experts", ctypes.c_int),
+        ("aux_loss", ctypes.c_void_p),
     ]
 
 
@@ -236,10 +237,11 @@ def moe_router_options_init() -> RouterOptions:
 
 def router_options(score="softmax", renormalize=False, route_scale=1.0, expert_bias=None,
                    num_groups=0, topk_groups=0, tokens_per_expert=None,
-                   score_before_experts=False) -> RouterOptions:
+                   score_before_experts=False, aux_loss=None) -> RouterOptions:
     """A RouterOptions from keyword values ([HP] TokenChoiceTopKRouter's
-    settings).  expert_bias / tokens_per_expert are fp32 CUDA tensors [E] or
-    None and must stay alive while the call that takes the options runs."""
+    settings).  expert_bias / tokens_per_expert are fp32 CUDA tensors [E],
+    aux_loss an fp32 CUDA tensor of one element, or None; they must stay
+    alive while the call that takes the options runs."""
     o = moe_router_options_init()
     o.score = {"softmax": MOE_SCORE_SOFTMAX, "sigmoid": MOE_SCORE_SIGMOID}[score]
     o.renormalize = int(bool(renormalize))
@@ -249,6 +251,7 @@ def router_options(score="softmax", renormalize=False, route_scale=1.0, expert_b
     o.topk_groups = int(topk_groups or 0)
     o.tokens_per_expert = _ptr(tokens_per_expert, torch.float32, "tokens_per_expert")
     o.score_before_experts = int(bool(score_before_experts))
+    o.aux_loss = _ptr(aux_loss, torch.float32, "aux_loss")
     return o
 
 

@@ -74,11 +74,15 @@ moe_status_t check_rows(int d, moe_dtype_t dt, const char* name) {
 
 bool router_uses_tc(int E, moe_dtype_t dt) { return dt == MOE_BF16 && E <= 256; }
 
-// Status word plus the fp32 logit scratch: [ksplit, T, E] partial logits of
-// the tensor-core GEMM, or [T, E] logits of the CUDA-core path.
+// Load-balance statistics (copies and weight sums per expert, 2E floats).
+size_t lb_bytes(int E) { return align_up(2 * static_cast<size_t>(E) * sizeof(float), 256); }
+
+// Status word, the load-balance statistics, then the fp32 logit scratch:
+// [ksplit, T, E] partial logits of the tensor-core GEMM, or [T, E] logits of
+// the CUDA-core path.
 size_t router_ws(int T, int d, int E, moe_dtype_t dt) {
   const size_t planes = router_uses_tc(E, dt) ? router_plan(T, d).ksplit : 1;
-  return kStatusBytes + align_up(planes * T * E * sizeof(float), 256);
+  return kStatusBytes + lb_bytes(E) + align_up(planes * T * E * sizeof(float), 256);
 }
 
 moe_router_options_t default_options() {
@@ -91,6 +95,7 @@ moe_router_options_t default_options() {
   o.topk_groups = 0;
   o.tokens_per_expert = nullptr;
   o.score_before_experts = 0;
+  o.aux_loss = nullptr;
   return o;
 }
 
@@ -142,25 +147,33 @@ cudaError_t run_router(const void* x, const void* w_router, const float* logits_
                        float* logits_out, int32_t* topk_idx, float* topk_w, int32_t* counts,
                        void* scratch, int* status, cudaStream_t s,
                        const DispatchPlan* plan = nullptr, int32_t* blk = nullptr) {
-  if (T == 0) return cudaSuccess;
   const RouterOptions ko = kernel_options(o);
   const int renorm = o.renormalize;
   float* tpe = o.tokens_per_expert;
-  if (logits_in)
-    return launch_router_topk(logits_in, 1, T, E, top_k, renorm, ko, nullptr, topk_idx, topk_w,
-                              counts, tpe, plan, blk, s);
-  float* part = static_cast<float*>(scratch);
-  if (router_uses_tc(E, dt)) {
-    cudaError_t e = launch_router_tc(x, w_router, T, d, E, part, status, s);
-    if (e != cudaSuccess) return e;
-    return launch_router_topk(part, router_plan(T, d).ksplit, T, E, top_k, renorm, ko,
-                              logits_out, topk_idx, topk_w, counts, tpe, plan, blk, s);
+  float* lb = o.aux_loss ? static_cast<float*>(scratch) : nullptr;
+  float* part = reinterpret_cast<float*>(static_cast<char*>(scratch) + lb_bytes(E));
+  cudaError_t e = cudaSuccess;
+  if (lb) e = cudaMemsetAsync(lb, 0, 2 * sizeof(float) * E, s);
+  if (e == cudaSuccess && T > 0) {
+    if (logits_in) {
+      e = launch_router_topk(logits_in, 1, T, E, top_k, renorm, ko, nullptr, topk_idx, topk_w,
+                             counts, tpe, plan, blk, s, lb);
+    } else if (router_uses_tc(E, dt)) {
+      e = launch_router_tc(x, w_router, T, d, E, part, status, s);
+      if (e == cudaSuccess)
+        e = launch_router_topk(part, router_plan(T, d).ksplit, T, E, top_k, renorm, ko,
+                               logits_out, topk_idx, topk_w, counts, tpe, plan, blk, s, lb);
+    } else {
+      float* L = logits_out ? logits_out : part;
+      e = launch_router_logits_simt(x, w_router, T, d, E, dt, L, s);
+      if (e == cudaSuccess)
+        e = launch_router_topk(L, 1, T, E, top_k, renorm, ko, nullptr, topk_idx, topk_w, counts,
+                               tpe, plan, blk, s, lb);
+    }
   }
-  float* L = logits_out ? logits_out : part;
-  cudaError_t e = launch_router_logits_simt(x, w_router, T, d, E, dt, L, s);
-  if (e != cudaSuccess) return e;
-  return launch_router_topk(L, 1, T, E, top_k, renorm, ko, nullptr, topk_idx, topk_w, counts, tpe,
-                            plan, blk, s);
+  // [HP] _compute_load_balance_loss of this call (0 for no tokens)
+  if (e == cudaSuccess && lb) e = launch_lb_loss(lb, E, T, top_k, o.aux_loss, s);
+  return e;
 }
 
 size_t swiglu_ws(int N, int h, moe_dtype_t dt) {

@@ -57,12 +57,16 @@ struct RouterOptions {
 // scores / top-k / weights as `o` says; writes the logits if asked.  With
 // `plan` and `blk` it also writes the dispatch histogram table of `plan`
 // (so launch_dispatch can skip its histogram kernel).  The expert histogram
-// is added to `counts` (int) and to `tokens_per_expert` (fp32) when given.
+// is added to `counts` (int) and to `tokens_per_expert` (fp32) when given;
+// with `lb` (2E zeroed floats) it adds the copies per expert to lb[0..E)
+// and their routing weights to lb[E..2E).
 cudaError_t launch_router_topk(const float* parts, int nsplit, int T, int E, int top_k,
                                int renorm, const RouterOptions& o, float* logits_out,
                                int32_t* topk_idx, float* topk_w, int32_t* counts,
                                float* tokens_per_expert, const DispatchPlan* plan,
-                               int32_t* blk, cudaStream_t s);
+                               int32_t* blk, cudaStream_t s, float* lb = nullptr);
+// *loss = E * sum_e (lb[e] / (T k)) * (lb[E + e] / T), or 0 for T = 0.
+cudaError_t launch_lb_loss(const float* lb, int E, int T, int top_k, float* loss, cudaStream_t s);
 
 // ---- dispatch -------------------------------------------------------------
 // hist_done: the histogram table in `ws` was already written (by the router).

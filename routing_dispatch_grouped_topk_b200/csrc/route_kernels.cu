@@ -652,18 +652,22 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
     RouterOptions opt, float* __restrict__ logits_out, int32_t* __restrict__ topk_idx,
     float* __restrict__ topk_w, int32_t* __restrict__ counts,
     float* __restrict__ tokens_per_expert, int32_t* __restrict__ blk, int nbins, int R, int L,
-    int S) {
+    int S, float* __restrict__ lb) {
   pdl_wait();
   pdl_trigger();
-  extern __shared__ int sm_bins[];   // [nbins] dispatch keys (blk), then [E] experts
+  // [nbins] dispatch keys (blk), then [E] experts, then [E] weight sums (lb)
+  extern __shared__ int sm_bins[];
   __shared__ int gkey[8][32];        // per-warp group maxima (node-limited routing)
   int* dbins = sm_bins;
   int* ebins = sm_bins + (blk ? nbins : 0);
-  const bool tally_e = counts != nullptr || tokens_per_expert != nullptr;
+  float* wsum = reinterpret_cast<float*>(ebins + E);
+  const bool tally_e = counts != nullptr || tokens_per_expert != nullptr || lb != nullptr;
   if (blk)
     for (int i = threadIdx.x; i < nbins; i += blockDim.x) dbins[i] = 0;
   if (tally_e)
     for (int i = threadIdx.x; i < E; i += blockDim.x) ebins[i] = 0;
+  if (lb)
+    for (int i = threadIdx.x; i < E; i += blockDim.x) wsum[i] = 0.f;
   __syncthreads();
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
@@ -793,9 +797,11 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
     if (lane < k) {
       const size_t o = static_cast<size_t>(t) * k + lane;
       topk_idx[o] = my_e;
-      topk_w[o] = wx / (renorm ? sel : den) * opt.scale;
+      const float wout = wx / (renorm ? sel : den) * opt.scale;
+      topk_w[o] = wout;
       if (blk) atomicAdd(&dbins[dispatch_key(my_e, t, R, L, S)], 1);
       if (tally_e) atomicAdd(&ebins[my_e], 1);
+      if (lb) atomicAdd(&wsum[my_e], wout);
     }
   }
   __syncthreads();
@@ -808,45 +814,75 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
       if (!c) continue;
       if (counts) atomicAdd(&counts[i], c);
       if (tokens_per_expert) atomicAdd(&tokens_per_expert[i], static_cast<float>(c));
+      if (lb) {
+        atomicAdd(&lb[i], static_cast<float>(c));
+        atomicAdd(&lb[E + i], wsum[i]);
+      }
     }
   }
+}
+
+// [HP] _compute_load_balance_loss from the per-expert copy counts and
+// weight sums: E * sum_e (count_e / (T k)) * (wsum_e / T).
+__global__ void lb_loss_kernel(const float* __restrict__ lb, int E, int T, int k,
+                               float* __restrict__ loss) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ float part[32];
+  float acc = 0.f;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) acc += lb[e] * lb[E + e];
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float tot = 0.f;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) tot += part[w];
+    *loss = T > 0 ? static_cast<float>(E) * tot / (static_cast<float>(T) * k * T) : 0.f;
+  }
+}
+
+cudaError_t launch_lb_loss(const float* lb, int E, int T, int top_k, float* loss, cudaStream_t s) {
+  launch_k(lb_loss_kernel, dim3(1), dim3(256), 0, s, lb, E, T, top_k, loss);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_router_topk(const float* parts, int nsplit, int T, int E, int top_k,
                                int renorm, const RouterOptions& o, float* logits_out,
                                int32_t* topk_idx, float* topk_w, int32_t* counts,
                                float* tokens_per_expert, const DispatchPlan* plan,
-                               int32_t* blk, cudaStream_t s) {
+                               int32_t* blk, cudaStream_t s, float* lb) {
   if (T == 0) return cudaSuccess;
   const bool fuse = plan && blk;
   const int tpb = fuse ? plan->tb : 16;
   const int blocks = cdiv(T, tpb);
   const int nbins = fuse ? plan->nbins : 0;
-  const bool tally_e = counts || tokens_per_expert;
-  const size_t smem = sizeof(int) * ((fuse ? nbins : 0) + (tally_e ? E : 0));
+  const bool tally_e = counts || tokens_per_expert || lb;
+  const size_t smem =
+      sizeof(int) * ((fuse ? nbins : 0) + (tally_e ? E : 0)) + (lb ? sizeof(float) * E : 0);
   const int R = fuse ? plan->R : 1, L = fuse ? plan->L : E, S = fuse ? plan->S : T;
   int32_t* b = fuse ? blk : nullptr;
   const RouterOptions opt = o;
   if (E <= 32)
     launch_k(router_topk_kernel<1>, dim3(blocks), dim3(256), smem, s, parts, nsplit, T, E, top_k,
              renorm, tpb, opt, logits_out, topk_idx, topk_w, counts, tokens_per_expert, b,
-             nbins, R, L, S);
+             nbins, R, L, S, lb);
   else if (E <= 64)
     launch_k(router_topk_kernel<2>, dim3(blocks), dim3(256), smem, s, parts, nsplit, T, E, top_k,
              renorm, tpb, opt, logits_out, topk_idx, topk_w, counts, tokens_per_expert, b,
-             nbins, R, L, S);
+             nbins, R, L, S, lb);
   else if (E <= 128)
     launch_k(router_topk_kernel<4>, dim3(blocks), dim3(256), smem, s, parts, nsplit, T, E, top_k,
              renorm, tpb, opt, logits_out, topk_idx, topk_w, counts, tokens_per_expert, b,
-             nbins, R, L, S);
+             nbins, R, L, S, lb);
   else if (E <= 256)
     launch_k(router_topk_kernel<8>, dim3(blocks), dim3(256), smem, s, parts, nsplit, T, E, top_k,
              renorm, tpb, opt, logits_out, topk_idx, topk_w, counts, tokens_per_expert, b,
-             nbins, R, L, S);
+             nbins, R, L, S, lb);
   else
     launch_k(router_topk_kernel<16>, dim3(blocks), dim3(256), smem, s, parts, nsplit, T, E,
              top_k, renorm, tpb, opt, logits_out, topk_idx, topk_w, counts, tokens_per_expert,
-             b, nbins, R, L, S);
+             b, nbins, R, L, S, lb);
   return cudaGetLastError();
 }
 

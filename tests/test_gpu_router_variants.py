@@ -286,3 +286,34 @@ def test_forward_before_experts_ep_equals_single_device_bitwise(M):
     a = M.forward(*args, ep_ranks=8, score_before_experts=True, score="sigmoid")
     b = M.forward(*args, ep_ranks=1, score_before_experts=True, score="sigmoid")
     assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("vi", [0, 5])
+def test_load_balance_loss(M, vi):
+    """aux_loss = E sum_e f_e P_e of the call ([HP] _compute_load_balance_loss)
+    against the oracle on the GPU's own routing (fp32 atomics: 1e-5)."""
+    T, E, k = 1000, 128, 8
+    o, g = materialize(dict(VARIANTS[vi]), E, seed=vi)
+    L = W.make_logits(T, E, k, seed=vi + 31)
+    aux = torch.full((1,), -1.0, device="cuda")
+    gi, gw, _, _, ws = M.router_topk(logits_in=torch.from_numpy(L).cuda(), top_k=k,
+                                     renormalize=True, aux_loss=aux, **g)
+    assert M.device_status(ws) == 0
+    ref = O.load_balance_loss(gw.cpu().numpy(), gi.cpu().numpy(), E)
+    assert abs(aux.item() - ref) <= 1e-5 * abs(ref), (aux.item(), ref)
+
+
+def test_load_balance_loss_in_forward_and_empty(M):
+    c = W.config(1)
+    lay = W.make_layer(c, "cuda")
+    aux = torch.full((1,), -1.0, device="cuda")
+    res = M.forward(lay["x"], lay["w_router"], lay["w1"], lay["w3"], lay["w2"], c.top_k, True,
+                    want_router=True, aux_loss=aux)
+    assert M.device_status(res["ws"]) == 0
+    ref = O.load_balance_loss(res["topk_w"].cpu().numpy(), res["topk_idx"].cpu().numpy(), c.E)
+    assert abs(aux.item() - ref) <= 1e-5 * abs(ref), (aux.item(), ref)
+    assert 0.9 < ref < 1.1            # a near-uniform router is near the balanced value 1
+    aux.fill_(-1.0)
+    L0 = torch.zeros(0, 16, device="cuda")
+    M.router_topk(logits_in=L0, top_k=2, aux_loss=aux)
+    assert aux.item() == 0.0
