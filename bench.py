@@ -152,6 +152,23 @@ def job_tokens_per_s(T, ws, steps, total_ms_max):
     return T * ws * steps / (total_ms_max / 1e3)
 
 
+def stage_algorithmic_bytes(cfg) -> dict:
+    """Unique HBM bytes each staged entry point must move (read + write):
+    router: x and w_router read, indices and weights written (the fp32
+    partial logits stay on chip / in L2 and are not counted); dispatch: x
+    read, the routed rows written, the four int32 index arrays; regroup:
+    the routed rows read and written; combine: the expert outputs read,
+    the output written, indices and weights read."""
+    esz = 2 if cfg.dtype == "bf16" else 4
+    T, d, E, k, N = cfg.T, cfg.d, cfg.E, cfg.top_k, cfg.N
+    out = {"router": esz * (T * d + E * d) + 8 * N,
+           "dispatch": esz * (T * d + N * d) + 4 * (2 * N + N + N),
+           "combine": esz * (N * d + T * d) + 8 * N}
+    if cfg.ep_ranks > 1:
+        out["regroup"] = esz * 2 * N * d + 4 * 2 * N
+    return out
+
+
 def swiglu_algorithmic_bytes(cfg) -> int:
     """Unique HBM bytes of one grouped SwiGLU launch: the routed rows read
     (N x d) and the output written (N x d), the hidden activation written and
@@ -514,6 +531,10 @@ def run_ours(args, ws, rank, local):
         "grouped_gemm_tflops": tflops,
         "grouped_gemm_frac_of_tensor_peak": tflops / pk["bf16_tflops_sustained"],
         "stage_ms": stage_ms,
+        "stage_hbm": {n: {"GBps": b / (stage_ms[n] * 1e-3) / 1e9,
+                          "frac": b / (stage_ms[n] * 1e-3) / 1e9 / pk["hbm_gbs"],
+                          "algorithmic_bytes": b}
+                      for n, b in stage_algorithmic_bytes(cfg).items() if n in stage_ms},
         "staged_ms_per_step": staged_ms_per_step,
         "forward_matches_staged": forward_matches_staged,
         "copies_per_s": value * k,
