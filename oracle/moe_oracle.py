@@ -50,6 +50,8 @@ __all__ = [
     "expert_counts", "dispatch", "permute_rows", "ep_dispatch_rank_major",
     "ep_local_regroup", "apply_row_perm", "silu", "swiglu_ffn",
     "grouped_swiglu", "combine", "moe_forward", "dense_moe", "moe_tokens",
+    "silu_grad", "grouped_preactivations", "combine_backward", "grouped_swiglu_backward",
+    "dispatch_backward",
 ]
 
 
@@ -440,6 +442,103 @@ def _moe_routed(x, w_router, w1, w3, w2, top_k, renormalize, logits, ep_ranks, r
                src_row=src_rm[perm], x_perm=x_em, y=y,
                out=combine(y, dst_em, w))
     return res
+
+
+# --------------------------------------------------------------------------
+# Backward (the training path: [HP] MoE.forward and _run_experts_for_loop
+# differentiated by the chain rule; [QO] training branch)
+# --------------------------------------------------------------------------
+
+def silu_grad(z) -> np.ndarray:
+    """``d silu(z) / dz = s(z) (1 + z (1 - s(z)))`` with ``s`` the logistic
+    sigmoid (derivative of ``z s(z)`` by the product rule, ``s' = s(1-s)``)."""
+    s = sigmoid(z)
+    z = as_f64(z)
+    return s * (1.0 + z * (1.0 - s))
+
+
+def grouped_preactivations(x_perm, offsets, w1, w3):
+    """The two first-layer products of every expert segment, ``G = S w1^T``
+    and ``U = S w3^T`` ([HP] ``FeedForward.forward`` before the SiLU), as
+    ``[N, h]`` fp64 arrays (what a training forward keeps for the
+    backward)."""
+    xp = as_f64(x_perm)
+    off = _i64(offsets)
+    h = w1.shape[1]
+    G = np.zeros((xp.shape[0], h))
+    U = np.zeros((xp.shape[0], h))
+    for e in range(len(off) - 1):
+        lo, hi = int(off[e]), int(off[e + 1])
+        if hi > lo:
+            G[lo:hi] = xp[lo:hi] @ as_f64(w1[e]).T
+            U[lo:hi] = xp[lo:hi] @ as_f64(w3[e]).T
+    return G, U
+
+
+def combine_backward(dout, y, dst_pos, topk_w=None):
+    """Gradients of ``out[t] = sum_j w[t, j] y[dst_pos[t, j]]``.
+
+    Returns ``(dy, dw)``: ``dy[dst_pos[t, j]] = w[t, j] dout[t]`` (every slot
+    is the copy of exactly one ``(t, j)``) and ``dw[t, j] = <dout[t],
+    y[dst_pos[t, j]]>`` (``dw`` is None when the combine is unweighted).
+    """
+    dout = as_f64(dout)
+    y = as_f64(y)
+    dp = _i64(dst_pos)
+    T, k = dp.shape
+    w = np.ones((T, k)) if topk_w is None else as_f64(topk_w)
+    dy = np.zeros_like(y)
+    dw = np.zeros((T, k))
+    for t in range(T):
+        for j in range(k):
+            dy[dp[t, j]] = w[t, j] * dout[t]
+            dw[t, j] = float(dout[t] @ y[dp[t, j]])
+    return dy, (None if topk_w is None else dw)
+
+
+def grouped_swiglu_backward(x_perm, offsets, w1, w3, w2, dy):
+    """Gradients of :func:`grouped_swiglu` (no row scale) for an upstream
+    gradient ``dy [N, d]``, one expert segment at a time.
+
+    With ``S`` the expert's rows, ``G = S w1^T``, ``U = S w3^T``,
+    ``A = silu(G) * U`` and ``Y = A w2^T``:
+    ``dA = dY w2``, ``dU = dA * silu(G)``, ``dG = dA * U * silu'(G)``,
+    ``dw2 = dY^T A``, ``dw1 = dG^T S``, ``dw3 = dU^T S``,
+    ``dS = dG w1 + dU w3``.  Experts with no rows get zero weight gradients.
+    Returns ``(dx_perm, dw1, dw3, dw2)`` in fp64.
+    """
+    xp = as_f64(x_perm)
+    g = as_f64(dy)
+    off = _i64(offsets)
+    E = len(off) - 1
+    h, d = w1.shape[1], w1.shape[2]
+    dxp = np.zeros_like(xp)
+    dw1 = np.zeros((E, h, d))
+    dw3 = np.zeros((E, h, d))
+    dw2 = np.zeros((E, d, h))
+    for e in range(E):
+        lo, hi = int(off[e]), int(off[e + 1])
+        if hi == lo:
+            continue
+        S, dY = xp[lo:hi], g[lo:hi]
+        W1, W3, W2 = as_f64(w1[e]), as_f64(w3[e]), as_f64(w2[e])
+        G, U = S @ W1.T, S @ W3.T
+        A = silu(G) * U
+        dA = dY @ W2
+        dU = dA * silu(G)
+        dG = dA * U * silu_grad(G)
+        dw2[e] = dY.T @ A
+        dw1[e] = dG.T @ S
+        dw3[e] = dU.T @ S
+        dxp[lo:hi] = dG @ W1 + dU @ W3
+    return dxp, dw1, dw3, dw2
+
+
+def dispatch_backward(dx_perm, dst_pos) -> np.ndarray:
+    """Gradient of ``x_perm = x[src_row]`` with respect to ``x``: every token
+    collects the gradients of its copies, ``dx[t] = sum_j dx_perm[dst_pos[t,
+    j]]`` (the adjoint of the row gather is the scatter-add)."""
+    return combine(dx_perm, dst_pos, None)
 
 
 def dense_moe(x, idx, w, w1, w3, w2) -> np.ndarray:
