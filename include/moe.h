@@ -333,6 +333,69 @@ MOE_API moe_status_t moe_combine(const void* y, const int32_t* dst_pos, const in
                          moe_dtype_t dt, void* out, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Training path: the backward of the experts, the combine and the dispatch.
+ * The pages train these layers ([HP] MoE.forward under autograd, [QO]
+ * SpeedupMoeExperts training branch); the gradients below are the
+ * derivatives of the forward definitions above, by the chain rule.
+ *
+ * moe_grouped_swiglu_train -- moe_grouped_swiglu (no row_scale) that also
+ * returns what the backward needs:
+ *   H [N, h]   = silu(G) * U, rounded to bf16 (the GEMM2 operand)
+ *   gu [N, 2h] = G | U with G = x_perm[s] . w1[e]^T in columns [0, h) and
+ *                U = x_perm[s] . w3[e]^T in [h, 2h), each rounded once to
+ *                bf16 from the fp32 accumulator.
+ * bf16 only (MOE_ERR_UNSUPPORTED otherwise); shapes and alignment as
+ * moe_grouped_swiglu; rows of empty experts are not written.  No workspace
+ * beyond a 256-byte device status word (ws, ws_bytes >= 256).
+ *
+ * moe_grouped_swiglu_backward -- for every expert e with rows S (the
+ * segment of x_perm), G, U from gu and upstream gradient dY = dy[seg]:
+ *   dA = dY . w2[e];  dU = dA * silu(G);  dG = dA * U * silu'(G)
+ *   dx_perm[seg] = dG . w1[e] + dU . w3[e]                    [N, d]
+ *   dw1[e] = dG^T . S,  dw3[e] = dU^T . S                      [E, h, d]
+ *   dw2[e] = dY^T . H[seg]                                    [E, d, h]
+ * silu'(g) = s(g) (1 + g (1 - s(g))), s the logistic sigmoid.  fp32
+ * accumulation on tcgen05 tensor cores; dG and dU are rounded to bf16 once
+ * (they are operands of the next products), every output once.  Experts
+ * with no rows get zero weight gradients.  bf16 only; d % 64 == 0 and
+ * h % 64 == 0; all pointers 16-byte aligned; workspace
+ * moe_grouped_swiglu_backward_workspace_size (dG | dU [N, 2h] bf16 plus
+ * the status word).  Bad offsets set MOE_DEV_BAD_OFFSETS in the status
+ * word (moe_get_device_status) and the outputs are not written.
+ *
+ * moe_combine_backward -- gradient of moe_combine (row_map NULL):
+ *   dy[dst_pos[t, j]] = w[t, j] * dout[t]      (one rounding to dt)
+ *   d_topk_w[t, j]    = <dout[t], y[dst_pos[t, j]]>   (fp32 accumulation)
+ * w = topk_w or 1 when topk_w == NULL; d_topk_w may be NULL (not computed).
+ * dout [T, d]; y, dy [N, d]; dst_pos [T, k].  Slots outside [0, N) are
+ * skipped (their d_topk_w is 0).  bf16 or fp32; d a whole number of
+ * 16-byte vectors.
+ *
+ * moe_dispatch_backward -- gradient of x_perm = x[src_row] with respect to
+ * x: dx[t] = sum_j dx_perm[dst_pos[t, j]] (fp32 sum over j in order, one
+ * rounding): the unweighted combine.  Rules as moe_combine.
+ * ---------------------------------------------------------------------- */
+MOE_API moe_status_t moe_grouped_swiglu_train(const void* x_perm, const int32_t* offsets,
+                                      const void* w1, const void* w3, const void* w2, int N,
+                                      int d, int h, int E, moe_dtype_t dt, void* y, void* h_act,
+                                      void* gu, void* ws, size_t ws_bytes, void* stream);
+MOE_API size_t moe_grouped_swiglu_backward_workspace_size(int N, int d, int h, int E,
+                                                  moe_dtype_t dt);
+MOE_API moe_status_t moe_grouped_swiglu_backward(const void* x_perm, const int32_t* offsets,
+                                         const void* w1, const void* w3, const void* w2,
+                                         const void* h_act, const void* gu, const void* dy,
+                                         int N, int d, int h, int E, moe_dtype_t dt,
+                                         void* dx_perm, void* dw1, void* dw3, void* dw2,
+                                         void* ws, size_t ws_bytes, void* stream);
+MOE_API moe_status_t moe_combine_backward(const void* dout, const void* y,
+                                  const int32_t* dst_pos, const float* topk_w, int T, int d,
+                                  int N, int top_k, moe_dtype_t dt, void* dy, float* d_topk_w,
+                                  void* stream);
+MOE_API moe_status_t moe_dispatch_backward(const void* dx_perm, const int32_t* dst_pos, int T,
+                                   int d, int N, int top_k, moe_dtype_t dt, void* dx,
+                                   void* stream);
+
+/* ------------------------------------------------------------------------
  * moe_forward -- [HP] MoE.forward with score_before_experts=False and no
  * shared expert: router -> dispatch -> grouped SwiGLU -> combine.
  * With ep_ranks R > 1 the routed rows are laid out as R simulated EP ranks

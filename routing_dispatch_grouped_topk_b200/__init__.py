@@ -41,6 +41,9 @@ __all__ = [
     "regroup_workspace_size", "grouped_swiglu_workspace_size", "forward_workspace_size",
     "router_topk", "dispatch", "ep_dispatch_rank_major", "ep_local_regroup",
     "grouped_swiglu", "combine", "forward", "device_status",
+    "moe_grouped_swiglu_train", "moe_grouped_swiglu_backward", "moe_combine_backward",
+    "moe_dispatch_backward", "grouped_swiglu_backward_workspace_size",
+    "grouped_swiglu_train", "grouped_swiglu_backward", "combine_backward", "dispatch_backward",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe.so")
@@ -57,6 +60,8 @@ EXPORTED_SYMBOLS = [
     "moe_regroup_workspace_size", "moe_ep_local_regroup",
     "moe_grouped_swiglu_workspace_size", "moe_grouped_swiglu", "moe_grouped_swiglu_gather",
     "moe_combine",
+    "moe_grouped_swiglu_train", "moe_grouped_swiglu_backward_workspace_size",
+    "moe_grouped_swiglu_backward", "moe_combine_backward", "moe_dispatch_backward",
     "moe_forward_workspace_size", "moe_forward", "moe_forward_ex_workspace_size",
     "moe_forward_ex", "moe_get_device_status", "moe_selftest_timeout", "moe_status_string",
     "moe_last_error", "moe_version",
@@ -115,6 +120,13 @@ _SIGS = {
     "moe_grouped_swiglu_gather": (_I, [_P, _I, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P,
                                        _P, _Z, _P]),
     "moe_combine": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P]),
+    "moe_grouped_swiglu_train": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _Z,
+                                      _P]),
+    "moe_grouped_swiglu_backward_workspace_size": (_Z, [_I, _I, _I, _I, _I]),
+    "moe_grouped_swiglu_backward": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P,
+                                         _P, _P, _P, _P, _Z, _P]),
+    "moe_combine_backward": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P]),
+    "moe_dispatch_backward": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P]),
     "moe_forward_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I, _I]),
     "moe_forward": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P,
                          _P, _P, _P, _Z, _P]),
@@ -325,6 +337,39 @@ def moe_combine(y, dst_pos, row_map, topk_w, T, d, N, top_k, dt, out, stream=Non
         top_k, dt, _ptr(out, name="out"), _stream(stream)), "moe_combine")
 
 
+def moe_grouped_swiglu_train(x_perm, offsets, w1, w3, w2, N, d, h, E, dt, y, h_act, gu, ws,
+                             stream=None):
+    _check(lib().moe_grouped_swiglu_train(
+        _ptr(x_perm, name="x_perm"), _ptr(offsets, torch.int32, "offsets"), _ptr(w1, name="w1"),
+        _ptr(w3, name="w3"), _ptr(w2, name="w2"), N, d, h, E, dt, _ptr(y, name="y"),
+        _ptr(h_act, name="h_act"), _ptr(gu, name="gu"), _ptr(ws, name="ws"), _nbytes(ws),
+        _stream(stream)), "moe_grouped_swiglu_train")
+
+
+def moe_grouped_swiglu_backward(x_perm, offsets, w1, w3, w2, h_act, gu, dy, N, d, h, E, dt,
+                                dx_perm, dw1, dw3, dw2, ws, stream=None):
+    _check(lib().moe_grouped_swiglu_backward(
+        _ptr(x_perm, name="x_perm"), _ptr(offsets, torch.int32, "offsets"), _ptr(w1, name="w1"),
+        _ptr(w3, name="w3"), _ptr(w2, name="w2"), _ptr(h_act, name="h_act"), _ptr(gu, name="gu"),
+        _ptr(dy, name="dy"), N, d, h, E, dt, _ptr(dx_perm, name="dx_perm"),
+        _ptr(dw1, name="dw1"), _ptr(dw3, name="dw3"), _ptr(dw2, name="dw2"),
+        _ptr(ws, name="ws"), _nbytes(ws), _stream(stream)), "moe_grouped_swiglu_backward")
+
+
+def moe_combine_backward(dout, y, dst_pos, topk_w, T, d, N, top_k, dt, dy, d_topk_w,
+                         stream=None):
+    _check(lib().moe_combine_backward(
+        _ptr(dout, name="dout"), _ptr(y, name="y"), _ptr(dst_pos, torch.int32, "dst_pos"),
+        _ptr(topk_w, torch.float32, "topk_w"), T, d, N, top_k, dt, _ptr(dy, name="dy"),
+        _ptr(d_topk_w, torch.float32, "d_topk_w"), _stream(stream)), "moe_combine_backward")
+
+
+def moe_dispatch_backward(dx_perm, dst_pos, T, d, N, top_k, dt, dx, stream=None):
+    _check(lib().moe_dispatch_backward(
+        _ptr(dx_perm, name="dx_perm"), _ptr(dst_pos, torch.int32, "dst_pos"), T, d, N, top_k,
+        dt, _ptr(dx, name="dx"), _stream(stream)), "moe_dispatch_backward")
+
+
 def moe_forward(x, w_router, logits_in, w1, w3, w2, T, d, E, top_k, h, score, renormalize,
                 ep_ranks, dt, out, logits_out, topk_idx, topk_w, counts, ws, stream=None):
     _check(lib().moe_forward(
@@ -478,6 +523,59 @@ def combine(y, dst_pos, topk_w=None, row_map=None):
     out = torch.empty(T, d, dtype=y.dtype, device=y.device)
     moe_combine(y, dst_pos, row_map, topk_w, T, d, N, k, _dt(y), out)
     return out
+
+
+def grouped_swiglu_backward_workspace_size(N, d, h, E, dt) -> int:
+    return lib().moe_grouped_swiglu_backward_workspace_size(N, d, h, E, dt)
+
+
+def grouped_swiglu_train(x_perm, offsets, w1, w3, w2):
+    """Training forward of the experts.  Returns (y [N, d], h_act [N, h],
+    gu [N, 2h], ws)."""
+    N, d = x_perm.shape
+    E, h, _ = w1.shape
+    dev = x_perm.device
+    y = torch.empty(N, d, dtype=x_perm.dtype, device=dev)
+    h_act = torch.empty(N, h, dtype=x_perm.dtype, device=dev)
+    gu = torch.empty(N, 2 * h, dtype=x_perm.dtype, device=dev)
+    ws = _ws(256, dev)
+    moe_grouped_swiglu_train(x_perm, offsets, w1, w3, w2, N, d, h, E, _dt(x_perm), y, h_act, gu,
+                             ws)
+    return y, h_act, gu, ws
+
+
+def grouped_swiglu_backward(x_perm, offsets, w1, w3, w2, h_act, gu, dy):
+    """Backward of the experts.  Returns (dx_perm, dw1, dw3, dw2, ws)."""
+    N, d = x_perm.shape
+    E, h, _ = w1.shape
+    dev = x_perm.device
+    dx_perm = torch.empty(N, d, dtype=x_perm.dtype, device=dev)
+    dw1 = torch.empty_like(w1)
+    dw3 = torch.empty_like(w3)
+    dw2 = torch.empty_like(w2)
+    ws = _ws(grouped_swiglu_backward_workspace_size(N, d, h, E, _dt(x_perm)), dev)
+    moe_grouped_swiglu_backward(x_perm, offsets, w1, w3, w2, h_act, gu, dy, N, d, h, E,
+                                _dt(x_perm), dx_perm, dw1, dw3, dw2, ws)
+    return dx_perm, dw1, dw3, dw2, ws
+
+
+def combine_backward(dout, y, dst_pos, topk_w=None, want_dw=True):
+    """Backward of combine.  Returns (dy [N, d], d_topk_w [T, k] fp32 or None)."""
+    T, k = dst_pos.shape
+    N, d = y.shape
+    dy = torch.empty(N, d, dtype=y.dtype, device=y.device)
+    dw = torch.empty(T, k, dtype=torch.float32, device=y.device) if want_dw else None
+    moe_combine_backward(dout, y, dst_pos, topk_w, T, d, N, k, _dt(y), dy, dw)
+    return dy, dw
+
+
+def dispatch_backward(dx_perm, dst_pos):
+    """dx [T, d]: every token's sum of its copies' gradients."""
+    T, k = dst_pos.shape
+    N, d = dx_perm.shape
+    dx = torch.empty(T, d, dtype=dx_perm.dtype, device=dx_perm.device)
+    moe_dispatch_backward(dx_perm, dst_pos, T, d, N, k, _dt(dx_perm), dx)
+    return dx
 
 
 def forward(x, w_router, w1, w3, w2, top_k, renormalize=True, ep_ranks=1, logits_in=None,

@@ -569,6 +569,113 @@ moe_status_t moe_combine(const void* y, const int32_t* dst_pos, const int32_t* r
                      "moe_combine");
 }
 
+// ------------------------------------------------------------ training path
+moe_status_t moe_grouped_swiglu_train(const void* x_perm, const int32_t* offsets, const void* w1,
+                                      const void* w3, const void* w2, int N, int d, int h, int E,
+                                      moe_dtype_t dt, void* y, void* h_act, void* gu, void* ws,
+                                      size_t ws_bytes, void* stream) {
+  if (moe_status_t st = check_swiglu_shape(N, d, h, E, dt)) return st;
+  if (dt != MOE_BF16) {
+    set_last_error("moe_grouped_swiglu_train: bf16 only");
+    return MOE_ERR_UNSUPPORTED;
+  }
+  if (N > 0) {
+    MOE_CHECK_ARG(x_perm && offsets && w1 && w3 && w2 && y && h_act && gu,
+                  "x_perm, offsets, w1, w3, w2, y, h_act, gu required");
+    MOE_CHECK_ARG(aligned16(x_perm) && aligned16(w1) && aligned16(w3) && aligned16(w2) &&
+                      aligned16(y) && aligned16(h_act) && aligned16(gu),
+                  "x_perm, w1, w3, w2, y, h_act, gu must be 16-byte aligned");
+  }
+  MOE_CHECK_ARG(ws != nullptr, "ws is required");
+  if (ws_bytes < kStatusBytes) {
+    set_last_error("grouped_swiglu_train workspace %zu < %zu", ws_bytes, kStatusBytes);
+    return MOE_ERR_WORKSPACE;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* status = static_cast<int*>(ws);
+  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), s);
+  if (e == cudaSuccess && N > 0)
+    e = launch_swiglu_tc_train(x_perm, offsets, w1, w3, w2, N, d, h, E, y, h_act, gu, status, s);
+  return cuda_status(e, "moe_grouped_swiglu_train");
+}
+
+size_t moe_grouped_swiglu_backward_workspace_size(int N, int d, int h, int E, moe_dtype_t dt) {
+  (void)d;
+  (void)E;
+  (void)dt;
+  if (N < 0 || h < 1) return kStatusBytes;
+  return kStatusBytes + align_up(static_cast<size_t>(N) * 2 * h * 2, 256);
+}
+
+moe_status_t moe_grouped_swiglu_backward(const void* x_perm, const int32_t* offsets,
+                                         const void* w1, const void* w3, const void* w2,
+                                         const void* h_act, const void* gu, const void* dy, int N,
+                                         int d, int h, int E, moe_dtype_t dt, void* dx_perm,
+                                         void* dw1, void* dw3, void* dw2, void* ws,
+                                         size_t ws_bytes, void* stream) {
+  if (moe_status_t st = check_swiglu_shape(N, d, h, E, dt)) return st;
+  if (dt != MOE_BF16) {
+    set_last_error("moe_grouped_swiglu_backward: bf16 only");
+    return MOE_ERR_UNSUPPORTED;
+  }
+  MOE_CHECK_ARG(offsets && w1 && w3 && w2 && dw1 && dw3 && dw2,
+                "offsets, w1, w3, w2, dw1, dw3, dw2 required");
+  if (N > 0) {
+    MOE_CHECK_ARG(x_perm && h_act && gu && dy && dx_perm,
+                  "x_perm, h_act, gu, dy, dx_perm required");
+    MOE_CHECK_ARG(aligned16(x_perm) && aligned16(h_act) && aligned16(gu) && aligned16(dy) &&
+                      aligned16(dx_perm),
+                  "x_perm, h_act, gu, dy, dx_perm must be 16-byte aligned");
+  }
+  MOE_CHECK_ARG(aligned16(w1) && aligned16(w3) && aligned16(w2) && aligned16(dw1) &&
+                    aligned16(dw3) && aligned16(dw2),
+                "w1, w3, w2, dw1, dw3, dw2 must be 16-byte aligned");
+  MOE_CHECK_ARG(ws != nullptr, "ws is required");
+  const size_t need = moe_grouped_swiglu_backward_workspace_size(N, d, h, E, dt);
+  if (ws_bytes < need) {
+    set_last_error("grouped_swiglu_backward workspace %zu < %zu", ws_bytes, need);
+    return MOE_ERR_WORKSPACE;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* status = static_cast<int*>(ws);
+  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), s);
+  if (e == cudaSuccess && N == 0) {
+    // no rows: every weight gradient is zero
+    const size_t wbytes = static_cast<size_t>(E) * h * d * 2;
+    e = cudaMemsetAsync(dw1, 0, wbytes, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dw3, 0, wbytes, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dw2, 0, wbytes, s);
+  } else if (e == cudaSuccess) {
+    e = launch_swiglu_bwd_tc(x_perm, offsets, w1, w3, w2, h_act, gu, dy, N, d, h, E, dx_perm, dw1,
+                             dw3, dw2, static_cast<char*>(ws) + kStatusBytes, status, s);
+  }
+  return cuda_status(e, "moe_grouped_swiglu_backward");
+}
+
+moe_status_t moe_combine_backward(const void* dout, const void* y, const int32_t* dst_pos,
+                                  const float* topk_w, int T, int d, int N, int top_k,
+                                  moe_dtype_t dt, void* dy, float* d_topk_w, void* stream) {
+  if (moe_status_t st = check_dtype(dt)) return st;
+  MOE_CHECK_ARG(T >= 0 && N >= 0, "T, N must be >= 0");
+  MOE_CHECK_ARG(top_k >= 1 && top_k <= kMaxTopK, "top_k=%d out of range", top_k);
+  if (T > 0) {
+    MOE_CHECK_ARG(dout && dst_pos && dy, "dout, dst_pos and dy are required");
+    MOE_CHECK_ARG(!d_topk_w || y, "y is required for d_topk_w");
+    MOE_CHECK_ARG(aligned16(dout) && aligned16(dy) && aligned16(y),
+                  "dout / dy / y must be 16-byte aligned");
+    if (moe_status_t st = check_rows(d, dt, "combine_backward")) return st;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return cuda_status(launch_combine_backward(dout, y, dst_pos, topk_w, T, d, N, top_k, dt, dy,
+                                             d_topk_w, s),
+                     "moe_combine_backward");
+}
+
+moe_status_t moe_dispatch_backward(const void* dx_perm, const int32_t* dst_pos, int T, int d,
+                                   int N, int top_k, moe_dtype_t dt, void* dx, void* stream) {
+  return moe_combine(dx_perm, dst_pos, nullptr, nullptr, T, d, N, top_k, dt, dx, stream);
+}
+
 // ------------------------------------------------------------------ forward
 size_t moe_forward_ex_workspace_size(int T, int d, int E, int top_k, int h, int ep_ranks,
                                      moe_dtype_t dt, int h_shared) {

@@ -255,6 +255,22 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(const void* tile) {
   return desc;
 }
 
+// Shared-memory descriptor of an MN-major bf16 operand in the 128-byte
+// swizzle layout: the tile is stored as chunks of 64 MN elements (one
+// 128-byte line per K row, 8 K rows per 1 KB swizzle atom); consecutive
+// 64-element MN chunks are `chunk_bytes` apart (leading byte offset) and
+// consecutive groups of 8 K rows 1 KB apart (stride byte offset).
+__device__ __forceinline__ uint64_t sw128_mnmajor_desc(const void* tile, uint32_t chunk_bytes) {
+  const uint32_t addr = smem_u32(tile);
+  uint64_t desc = 0;
+  desc |= static_cast<uint64_t>((addr >> 4) & 0x3FFFu);                 // start address
+  desc |= static_cast<uint64_t>((chunk_bytes >> 4) & 0x3FFFu) << 16;     // leading byte offset
+  desc |= static_cast<uint64_t>((1024u >> 4) & 0x3FFFu) << 32;           // stride byte offset
+  desc |= static_cast<uint64_t>(1u) << 46;                                // version (sm_100)
+  desc |= static_cast<uint64_t>(2u) << 61;                                // 128-byte swizzle
+  return desc;
+}
+
 // Instruction descriptor of tcgen05.mma kind::f16: bf16 A and B (both
 // K-major), fp32 accumulator, dense, shape M x N.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
@@ -263,6 +279,10 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
          | (1u << 10)                                // B format: bf16
          | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
          | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
+}
+// Same with the operands' majorness: a_mn / b_mn set "A (B) is MN-major".
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_major(int M, int N, bool a_mn, bool b_mn) {
+  return idesc_bf16_f32(M, N) | (a_mn ? (1u << 15) : 0u) | (b_mn ? (1u << 16) : 0u);
 }
 
 // D[tmem] (+)= A[smem] * B[smem]^T, one 128 x N x 16 step, issued by one thread.

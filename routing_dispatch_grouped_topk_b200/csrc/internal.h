@@ -91,6 +91,12 @@ cudaError_t launch_regroup(const void* in, const int32_t* counts_rm, int G, int 
 cudaError_t launch_combine(const void* y, const int32_t* dst_pos, const int32_t* row_map,
                            const float* topk_w, int T, int d, int N, int top_k, moe_dtype_t dt,
                            void* out, cudaStream_t s, const void* shared = nullptr);
+// Backward of the combine: dy [N, d] (every slot p(t, j) = w[t, j] dout[t];
+// w = 1 when topk_w is null) and, if d_topk_w is given, the fp32 dot products
+// <dout[t], y[p(t, j)]> ([T, k]).
+cudaError_t launch_combine_backward(const void* dout, const void* y, const int32_t* dst_pos,
+                                    const float* topk_w, int T, int d, int N, int top_k,
+                                    moe_dtype_t dt, void* dy, float* d_topk_w, cudaStream_t s);
 // Self-test of the bounded wait: sets MOE_DEV_TIMEOUT after kWaitLimitNs.
 cudaError_t launch_selftest_timeout(int* status, cudaStream_t s);
 // offsets[0] = 0, offsets[1] = n: the segmentation of a single expert.
@@ -107,6 +113,17 @@ cudaError_t launch_swiglu_tc_gather(const void* x, int T, const int32_t* src_row
                                     const int32_t* offsets, const void* w1, const void* w3,
                                     const void* w2, const float* row_scale, int N, int d, int h,
                                     int E, void* y, void* H, int* status, cudaStream_t s);
+// Training forward: also writes GU [N, 2h] bf16 (G = x w1^T | U = x w3^T),
+// and H [N, h] is an output the backward reads.
+cudaError_t launch_swiglu_tc_train(const void* x_perm, const int32_t* offsets, const void* w1,
+                                   const void* w3, const void* w2, int N, int d, int h, int E,
+                                   void* y, void* H, void* GU, int* status, cudaStream_t s);
+// Backward of the grouped SwiGLU (bf16, tcgen05): dX [N, d], dW1/dW3 [E, h, d],
+// dW2 [E, d, h]; dGU [N, 2h] bf16 is scratch.
+cudaError_t launch_swiglu_bwd_tc(const void* x_perm, const int32_t* offsets, const void* w1,
+                                 const void* w3, const void* w2, const void* H, const void* GU,
+                                 const void* dY, int N, int d, int h, int E, void* dX, void* dW1,
+                                 void* dW3, void* dW2, void* dGU, int* status, cudaStream_t s);
 // fp32 CUDA-core path: H (fp32 [N, h]) is scratch.
 cudaError_t launch_swiglu_simt_f32(const float* x_perm, const int32_t* offsets,
                                    const float* w1, const float* w3, const float* w2,

@@ -545,6 +545,112 @@ cudaError_t launch_combine(const void* y, const int32_t* dst_pos, const int32_t*
   return cudaGetLastError();
 }
 
+// ------------------------------------------------------- combine backward
+// Gradient of out[t] = sum_j w[t, j] y[p(t, j)] for an upstream dout [T, d]:
+// dy[p(t, j)] = w[t, j] dout[t] (one rounding of the fp32 product) and, when
+// dw is given, dw[t, j] = <dout[t], y[p(t, j)]> accumulated in fp32.  One warp
+// per token; each 16-byte chunk of dout is read once and its k products and
+// k dot-product terms are formed from registers (k + 1 loads in flight).
+__device__ __forceinline__ float dot_chunk(uint4 a, uint4 b, int bf16) {
+  if (bf16)
+    return bf16_lo(a.x) * bf16_lo(b.x) + bf16_hi(a.x) * bf16_hi(b.x) +
+           bf16_lo(a.y) * bf16_lo(b.y) + bf16_hi(a.y) * bf16_hi(b.y) +
+           bf16_lo(a.z) * bf16_lo(b.z) + bf16_hi(a.z) * bf16_hi(b.z) +
+           bf16_lo(a.w) * bf16_lo(b.w) + bf16_hi(a.w) * bf16_hi(b.w);
+  return __uint_as_float(a.x) * __uint_as_float(b.x) + __uint_as_float(a.y) * __uint_as_float(b.y) +
+         __uint_as_float(a.z) * __uint_as_float(b.z) + __uint_as_float(a.w) * __uint_as_float(b.w);
+}
+
+template <bool BF16, int KMAX>
+__global__ void __launch_bounds__(256) combine_backward_kernel(
+    const uint4* __restrict__ dout, const uint4* __restrict__ y,
+    const int32_t* __restrict__ dst_pos, const float* __restrict__ w, int T, int row_vec, int N,
+    int k, uint4* __restrict__ dy, float* __restrict__ dw) {
+  pdl_wait();
+  pdl_trigger();
+  const int lane = threadIdx.x & 31;
+  const int nwarps = (gridDim.x * blockDim.x) >> 5;
+  for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += nwarps) {
+    int my_p = -1;
+    float my_w = 0.f;
+    if (lane < k) {
+      const int p = dst_pos[static_cast<size_t>(t) * k + lane];
+      if (static_cast<unsigned>(p) < static_cast<unsigned>(N)) {
+        my_p = p;
+        my_w = w ? w[static_cast<size_t>(t) * k + lane] : 1.0f;
+      }
+    }
+    int pos[KMAX];
+    float wt[KMAX], dot[KMAX];
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      pos[j] = __shfl_sync(0xffffffffu, my_p, j);
+      wt[j] = __shfl_sync(0xffffffffu, my_w, j);
+      dot[j] = 0.f;
+    }
+    const uint4* grow = dout + static_cast<size_t>(t) * row_vec;
+    for (int c = lane; c < row_vec; c += 32) {
+      const uint4 g = grow[c];
+      uint4 v[KMAX];
+      if (dw) {
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j)
+          if (j < k && pos[j] >= 0) v[j] = y[static_cast<size_t>(pos[j]) * row_vec + c];
+      }
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j) {
+        if (j >= k || pos[j] < 0) continue;
+        dy[static_cast<size_t>(pos[j]) * row_vec + c] = scale_vec(g, wt[j], BF16);
+        if (dw) dot[j] += dot_chunk(g, v[j], BF16);
+      }
+    }
+    if (dw) {
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j) {
+        if (j >= k) break;
+        float sdot = dot[j];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) sdot += __shfl_xor_sync(0xffffffffu, sdot, off);
+        if (lane == 0) dw[static_cast<size_t>(t) * k + j] = pos[j] >= 0 ? sdot : 0.f;
+      }
+    }
+  }
+}
+
+template <bool BF16>
+static void combine_backward_launch(const uint4* dout, const uint4* y, const int32_t* dst_pos,
+                                    const float* w, int T, int row_vec, int N, int k, uint4* dy,
+                                    float* dw, int blocks, cudaStream_t s) {
+  if (k <= 1)
+    launch_k(combine_backward_kernel<BF16, 1>, dim3(blocks), dim3(256), 0, s, dout, y, dst_pos, w, T, row_vec, N, k, dy, dw);
+  else if (k <= 2)
+    launch_k(combine_backward_kernel<BF16, 2>, dim3(blocks), dim3(256), 0, s, dout, y, dst_pos, w, T, row_vec, N, k, dy, dw);
+  else if (k <= 4)
+    launch_k(combine_backward_kernel<BF16, 4>, dim3(blocks), dim3(256), 0, s, dout, y, dst_pos, w, T, row_vec, N, k, dy, dw);
+  else if (k <= 8)
+    launch_k(combine_backward_kernel<BF16, 8>, dim3(blocks), dim3(256), 0, s, dout, y, dst_pos, w, T, row_vec, N, k, dy, dw);
+  else
+    launch_k(combine_backward_kernel<BF16, 16>, dim3(blocks), dim3(256), 0, s, dout, y, dst_pos, w, T, row_vec, N, k, dy, dw);
+}
+
+cudaError_t launch_combine_backward(const void* dout, const void* y, const int32_t* dst_pos,
+                                    const float* topk_w, int T, int d, int N, int top_k,
+                                    moe_dtype_t dt, void* dy, float* d_topk_w, cudaStream_t s) {
+  if (T == 0) return cudaSuccess;
+  const int elt = dt == MOE_BF16 ? 2 : 4;
+  const int row_vec = d * elt / 16;
+  const int blocks = std::min(cdiv(T, 8), num_sms() * 8);
+  if (dt == MOE_BF16)
+    combine_backward_launch<true>(static_cast<const uint4*>(dout), static_cast<const uint4*>(y),
+                                  dst_pos, topk_w, T, row_vec, N, top_k, static_cast<uint4*>(dy),
+                                  d_topk_w, blocks, s);
+  else
+    combine_backward_launch<false>(static_cast<const uint4*>(dout), static_cast<const uint4*>(y),
+                                   dst_pos, topk_w, T, row_vec, N, top_k, static_cast<uint4*>(dy),
+                                   d_topk_w, blocks, s);
+  return cudaGetLastError();
+}
+
 // One thread waits on a barrier that nothing arrives at; the bounded wait
 // gives up after kWaitLimitNs and records MOE_DEV_TIMEOUT.
 __global__ void selftest_timeout_kernel(int* status) {

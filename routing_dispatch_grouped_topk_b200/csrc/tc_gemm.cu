@@ -53,6 +53,7 @@ struct TileInfo {
   int n0;        // first output column (router: the K split)
   int kb0, kb1;  // K blocks [kb0, kb1) of this tile
   int swap_np;   // 0, or: swap-AB tile whose MMA N is this many token rows
+  int m0;        // weight-gradient tiles: first output row (A column)
 };
 
 // A grouped tile with few valid rows (an expert's last rows, or decode) is
@@ -83,6 +84,13 @@ struct Args {
   int src_rows;              // gathered GEMM1: rows of x (T)
   const void* gather_src;    // gathered GEMM1: x [T, K]
   const float* row_scale;    // down only, may be null
+  // training forward: GEMM1 also keeps its two products for the backward
+  __nv_bfloat16* gu_out;     // [N, 2h]: G = x w1^T in columns [0, h), U = x w3^T in [h, 2h)
+  // backward
+  const __nv_bfloat16* gu_in;  // [N, 2h] the saved G | U (data gradient of GEMM2)
+  __nv_bfloat16* out1;       // weight gradient: output rows >= split of each expert
+  int split;                 // weight gradient: rows of each expert that go to `out`
+  int Ma;                    // weight gradient: output rows per expert
 };
 
 __host__ __device__ constexpr int stages_for(int bn) {
@@ -106,6 +114,8 @@ struct RouterPolicy {
   static constexpr int BN = BN_;
   static constexpr int NUM_B = 1;
   static constexpr bool GATHER_A = false;
+  static constexpr bool A_MN = false, B_MN = false, MASK_K = false, CUSTOM_LOADS = false;
+  static __device__ int k_rows(const TileInfo&, int) { return BK; }
   static constexpr int THREADS = kThreads;
   static constexpr int SCHED_INTS = 8;
 
@@ -161,6 +171,8 @@ struct GroupedSched {
   static constexpr int MROWS = MR;   // rows of one m-tile (256: a CTA pair)
   static constexpr int NUM_B = NUM_B_;
   static constexpr bool GATHER_A = false;
+  static constexpr bool A_MN = false, B_MN = false, MASK_K = false, CUSTOM_LOADS = false;
+  static __device__ int k_rows(const TileInfo&, int) { return BK; }
   static constexpr int THREADS = kThreads;
   static constexpr int SCHED_INTS = 8 + 2 * (kMaxExperts + 1);
 
@@ -268,6 +280,12 @@ struct UpPolicyT : GroupedSched<256, 2, 128> {
             const float gv = __uint_as_float(g[i]), uv = __uint_as_float(u[i]);
             col[static_cast<size_t>(t0 + i) * a.n_out] =
                 __float2bfloat16_rn(__fdividef(gv, 1.0f + __expf(-gv)) * uv);
+            if (a.gu_out) {
+              __nv_bfloat16* gu =
+                  a.gu_out + static_cast<size_t>(ti.a_row + t0 + i) * (2 * a.n_out) + n;
+              gu[0] = __float2bfloat16_rn(gv);
+              gu[a.n_out] = __float2bfloat16_rn(uv);
+            }
           }
         }
       }
@@ -300,6 +318,23 @@ struct UpPolicyT : GroupedSched<256, 2, 128> {
         uint4* d4 = reinterpret_cast<uint4*>(dst_row + c * 32);
 #pragma unroll
         for (int q = 0; q < 4; ++q) d4[q] = make_uint4(p[4 * q], p[4 * q + 1], p[4 * q + 2], p[4 * q + 3]);
+        if (a.gu_out) {
+          // the bf16 G and U of these 32 hidden units, for the backward
+          uint4* g4 = reinterpret_cast<uint4*>(
+              a.gu_out + static_cast<size_t>(ti.a_row + row) * (2 * a.n_out) + ti.n0 + c * 32);
+          uint4* u4 = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(g4) + a.n_out);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            g4[q] = make_uint4(pack_bf16x2(__uint_as_float(g[8 * q]), __uint_as_float(g[8 * q + 1])),
+                               pack_bf16x2(__uint_as_float(g[8 * q + 2]), __uint_as_float(g[8 * q + 3])),
+                               pack_bf16x2(__uint_as_float(g[8 * q + 4]), __uint_as_float(g[8 * q + 5])),
+                               pack_bf16x2(__uint_as_float(g[8 * q + 6]), __uint_as_float(g[8 * q + 7])));
+            u4[q] = make_uint4(pack_bf16x2(__uint_as_float(u[8 * q]), __uint_as_float(u[8 * q + 1])),
+                               pack_bf16x2(__uint_as_float(u[8 * q + 2]), __uint_as_float(u[8 * q + 3])),
+                               pack_bf16x2(__uint_as_float(u[8 * q + 4]), __uint_as_float(u[8 * q + 5])),
+                               pack_bf16x2(__uint_as_float(u[8 * q + 6]), __uint_as_float(u[8 * q + 7])));
+          }
+        }
       }
     }
   }
@@ -425,6 +460,237 @@ struct DownPairPolicy : GroupedSched<256, 1, 256, 256> {
   }
 };
 
+// ------------------------------------------------------- backward policies
+// The backward of the grouped SwiGLU (the derivative of the forward above,
+// one expert segment at a time; G = S w1^T, U = S w3^T, A = silu(G) * U,
+// Y = A w2^T):
+//   dA = dY w2,  dU = dA * silu(G),  dG = dA * U * silu'(G)   (DownBwdPolicy)
+//   dS = dG w1 + dU w3                                          (UpBwdPolicy)
+//   dw2 = dY^T A,  dw1 = dG^T S,  dw3 = dU^T S                  (WgradPolicy)
+// The weights enter the data gradients untransposed, so their tiles are
+// MN-major: a stage holds BN/64 TMA boxes of 64 K rows x 64 columns (one
+// 128-byte swizzled line per K row), 8 KB apart.  The weight gradients
+// reduce over an expert's rows: both operands are MN-major and the K loop
+// runs over the segment, 64 rows per stage; rows of the last stage that
+// belong to the next segment are zeroed in shared memory before the MMA.
+constexpr int kMnBoxBytes = 64 * BK * 2;   // one 64 x 64 MN-major box: 8 KB
+
+__device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
+
+// Data gradient of GEMM2 with the SwiGLU backward in the epilogue:
+// A = dY [N, d] (K-major, K = d), B = w2[e] [d, h] as K rows x h columns.
+// The accumulator holds dA for 256 hidden units; the epilogue reads G and U
+// from gu_in and writes dG | dU into `out` ([N, 2h], the layout of gu).
+struct DownBwdPolicy : GroupedSched<256, 1, 256> {
+  static constexpr bool B_MN = true, CUSTOM_LOADS = true;
+  static __device__ TileInfo tile_info(const Args& a, const int* sched, int tile) {
+    int e, nt, mt, cnt, seg0;
+    locate(a, sched, tile, e, nt, mt, cnt, seg0);
+    TileInfo t;
+    t.a_row = seg0 + mt * BM;
+    t.m_valid = min(BM, cnt - mt * BM);
+    t.n0 = nt * 256;
+    t.b_row = e * a.K;
+    t.kb0 = 0;
+    t.kb1 = cdiv(a.K, BK);
+    t.swap_np = 0;
+    t.m0 = 0;
+    return t;
+  }
+  static __device__ void issue_loads(const Args&, const CUtensorMap* tmA, const CUtensorMap* tmB0,
+                                     const CUtensorMap*, const TileInfo& ti, int kb, uint8_t* sa,
+                                     uint8_t* sb, uint64_t* bar, uint64_t pa, uint64_t pb) {
+    tma_load_2d(sa, tmA, bar, kb * BK, ti.a_row, pa);
+#pragma unroll
+    for (int c = 0; c < BN / 64; ++c)
+      tma_load_2d(sb + c * kMnBoxBytes, tmB0, bar, ti.n0 + 64 * c, ti.b_row + kb * BK, pb);
+  }
+  static __device__ void epilogue(const Args& a, int*, const TileInfo& ti, uint32_t taddr,
+                                  int row) {
+    const int h = a.n_out;
+    const bool valid = row < ti.m_valid;
+    const size_t base = static_cast<size_t>(ti.a_row + row) * (2 * h) + ti.n0;
+#pragma unroll 1
+    for (int c = 0; c < 8; ++c) {
+      const bool live = valid && ti.n0 + c * 32 < h;
+      uint4 gq[4], uq[4];
+      if (live) {
+        const uint4* g4 = reinterpret_cast<const uint4*>(a.gu_in + base + c * 32);
+        const uint4* u4 = reinterpret_cast<const uint4*>(a.gu_in + base + h + c * 32);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          gq[q] = g4[q];
+          uq[q] = u4[q];
+        }
+      }
+      uint32_t r[32];
+      tmem_ld32(taddr + c * 32, r);
+      tmem_ld_wait();
+      if (!live) continue;
+      const uint32_t* gw = reinterpret_cast<const uint32_t*>(gq);
+      const uint32_t* uw = reinterpret_cast<const uint32_t*>(uq);
+      uint32_t pg[16], pu[16];
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        float dg[2], du[2];
+#pragma unroll
+        for (int hlf = 0; hlf < 2; ++hlf) {
+          const uint32_t gbits = hlf ? (gw[q] & 0xffff0000u) : (gw[q] << 16);
+          const uint32_t ubits = hlf ? (uw[q] & 0xffff0000u) : (uw[q] << 16);
+          const float g = __uint_as_float(gbits), u = __uint_as_float(ubits);
+          const float da = __uint_as_float(r[2 * q + hlf]);
+          const float sg = 1.0f / (1.0f + __expf(-g));
+          du[hlf] = da * (g * sg);
+          dg[hlf] = da * u * (sg * (1.0f + g * (1.0f - sg)));
+        }
+        pg[q] = pack_bf16x2(dg[0], dg[1]);
+        pu[q] = pack_bf16x2(du[0], du[1]);
+      }
+      uint4* dg4 = reinterpret_cast<uint4*>(a.out + base + c * 32);
+      uint4* du4 = reinterpret_cast<uint4*>(a.out + base + h + c * 32);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        dg4[q] = make_uint4(pg[4 * q], pg[4 * q + 1], pg[4 * q + 2], pg[4 * q + 3]);
+        du4[q] = make_uint4(pu[4 * q], pu[4 * q + 1], pu[4 * q + 2], pu[4 * q + 3]);
+      }
+    }
+  }
+  static __device__ void finish(const Args&, int*) {}
+};
+
+// Data gradient of GEMM1: A = dG | dU [N, 2h] (K-major, K = 2h), B = the
+// K rows of w1[e] (K blocks [0, h/64)) then of w3[e] ([h/64, 2h/64)), each
+// [h, d] as K rows x d columns.  Output dS [N, d].
+struct UpBwdPolicy : GroupedSched<256, 2, 256> {
+  static constexpr bool B_MN = true, CUSTOM_LOADS = true;
+  static __device__ TileInfo tile_info(const Args& a, const int* sched, int tile) {
+    int e, nt, mt, cnt, seg0;
+    locate(a, sched, tile, e, nt, mt, cnt, seg0);
+    TileInfo t;
+    t.a_row = seg0 + mt * BM;
+    t.m_valid = min(BM, cnt - mt * BM);
+    t.n0 = nt * 256;
+    t.b_row = e * (a.K / 2);
+    t.kb0 = 0;
+    t.kb1 = cdiv(a.K, BK);
+    t.swap_np = 0;
+    t.m0 = 0;
+    return t;
+  }
+  static __device__ void issue_loads(const Args& a, const CUtensorMap* tmA,
+                                     const CUtensorMap* tmB0, const CUtensorMap* tmB1,
+                                     const TileInfo& ti, int kb, uint8_t* sa, uint8_t* sb,
+                                     uint64_t* bar, uint64_t pa, uint64_t pb) {
+    tma_load_2d(sa, tmA, bar, kb * BK, ti.a_row, pa);
+    const int hb = (a.K / 2) / BK;   // K blocks of w1
+    const CUtensorMap* m = kb < hb ? tmB0 : tmB1;
+    const int y = ti.b_row + (kb < hb ? kb : kb - hb) * BK;
+#pragma unroll
+    for (int c = 0; c < BN / 64; ++c) tma_load_2d(sb + c * kMnBoxBytes, m, bar, ti.n0 + 64 * c, y, pb);
+  }
+  static __device__ void epilogue(const Args& a, int* s, const TileInfo& ti, uint32_t taddr,
+                                  int row) {
+    DownPolicy::epilogue(a, s, ti, taddr, row);   // plain bf16 rows (row_scale is null)
+  }
+  static __device__ void finish(const Args&, int*) {}
+};
+
+// Weight gradients: out[e] = A_e^T B_e over the rows of segment e, with
+// A [N, Ma] and B [N, n_out] both MN-major (their columns are the output's
+// rows and columns).  Tiles are (expert, 128 output rows, 256 output
+// columns), expert-major; an expert with no rows gets zeros.  Output rows
+// [0, split) of expert e go to out[e], rows [split, Ma) to out1[e].
+struct WgradPolicy {
+  static constexpr int BN = 256;
+  static constexpr int NUM_B = 1;
+  static constexpr bool GATHER_A = false;
+  static constexpr bool A_MN = true, B_MN = true, MASK_K = true, CUSTOM_LOADS = true;
+  static constexpr int THREADS = kThreads;
+  static constexpr int SCHED_INTS = 8 + kMaxExperts + 1;   // [0] tiles [1] m-tiles [2] n-tiles, offsets
+
+  static __device__ void prologue(const Args& a, int* sched) {
+    const int E = a.E;
+    int* off = sched + 8;
+    for (int i = threadIdx.x; i <= E; i += blockDim.x) off[i] = a.offsets[i];
+    __syncthreads();
+    if (threadIdx.x < 32) {
+      int bad = 0;
+      for (int e = threadIdx.x; e < E; e += 32) bad |= off[e + 1] < off[e];
+      bad = __any_sync(0xffffffffu, bad);
+      if (threadIdx.x == 0) {
+        bad |= (off[0] != 0) || (off[E] != a.M);
+        const int mt = cdiv(a.Ma, BM), nt = cdiv(a.n_out, BN);
+        sched[0] = bad ? 0 : E * mt * nt;
+        sched[1] = mt;
+        sched[2] = nt;
+        if (bad && blockIdx.x == 0) set_status(a.status, MOE_DEV_BAD_OFFSETS);
+      }
+    }
+  }
+  static __device__ int num_tiles(const Args&, const int* sched) { return sched[0]; }
+  static __device__ TileInfo tile_info(const Args&, const int* sched, int tile) {
+    const int mt = sched[1], nt = sched[2];
+    const int per = mt * nt;
+    const int e = tile / per;
+    const int r = tile - e * per;
+    const int m = r / nt;
+    const int* off = sched + 8;
+    TileInfo t;
+    t.a_row = off[e];
+    t.m_valid = off[e + 1] - off[e];
+    t.b_row = e;
+    t.m0 = m * BM;
+    t.n0 = (r - m * nt) * BN;
+    t.kb0 = 0;
+    t.kb1 = cdiv(t.m_valid, BK);
+    t.swap_np = 0;
+    return t;
+  }
+  // rows of K block kb that belong to the segment (the rest are zeroed)
+  static __device__ int k_rows(const TileInfo& ti, int kb) { return min(BK, ti.m_valid - kb * BK); }
+  static __device__ void issue_loads(const Args&, const CUtensorMap* tmA, const CUtensorMap* tmB0,
+                                     const CUtensorMap*, const TileInfo& ti, int kb, uint8_t* sa,
+                                     uint8_t* sb, uint64_t* bar, uint64_t pa, uint64_t pb) {
+    const int y = ti.a_row + kb * BK;
+#pragma unroll
+    for (int c = 0; c < BM / 64; ++c) tma_load_2d(sa + c * kMnBoxBytes, tmA, bar, ti.m0 + 64 * c, y, pa);
+#pragma unroll
+    for (int c = 0; c < BN / 64; ++c) tma_load_2d(sb + c * kMnBoxBytes, tmB0, bar, ti.n0 + 64 * c, y, pb);
+  }
+  static __device__ void epilogue(const Args& a, int*, const TileInfo& ti, uint32_t taddr,
+                                  int row) {
+    const int m = ti.m0 + row;
+    const bool valid = m < a.Ma;
+    const int Nb = a.n_out;
+    const int e = ti.b_row;
+    __nv_bfloat16* dst =
+        m < a.split ? a.out + (static_cast<size_t>(e) * a.split + m) * Nb + ti.n0
+                    : a.out1 + (static_cast<size_t>(e) * (a.Ma - a.split) + (m - a.split)) * Nb + ti.n0;
+    const bool empty = ti.kb1 == ti.kb0;
+#pragma unroll 1
+    for (int c = 0; c < 8; ++c) {
+      uint32_t r[32];
+      if (!empty) {
+        tmem_ld32(taddr + c * 32, r);
+        tmem_ld_wait();
+      } else {
+#pragma unroll
+        for (int q = 0; q < 32; ++q) r[q] = 0u;
+      }
+      if (valid && ti.n0 + c * 32 < Nb) {
+        uint32_t p[16];
+#pragma unroll
+        for (int q = 0; q < 16; ++q)
+          p[q] = pack_bf16x2(__uint_as_float(r[2 * q]), __uint_as_float(r[2 * q + 1]));
+        uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) d4[q] = make_uint4(p[4 * q], p[4 * q + 1], p[4 * q + 2], p[4 * q + 3]);
+      }
+    }
+  }
+  static __device__ void finish(const Args&, int*) {}
+};
+
 // ------------------------------------------------------------- the kernel
 
 template <class P>
@@ -452,7 +718,11 @@ __global__ void __launch_bounds__(P::THREADS, 1)
   using L = Layout<P>;
   constexpr int BN = P::BN;
   constexpr int STAGES = L::kStages;
-  constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
+  constexpr uint32_t IDESC = idesc_bf16_f32_major(BM, BN, P::A_MN, P::B_MN);
+  // descriptor advance per 16-wide K step, in 16-byte units: 32 bytes along
+  // a K-major line, or two 128-byte K rows of an MN-major box
+  constexpr uint32_t A_KSTEP = P::A_MN ? 128u : 2u;
+  constexpr uint32_t B_KSTEP = P::B_MN ? 128u : 2u;
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -620,12 +890,16 @@ __global__ void __launch_bounds__(P::THREADS, 1)
           uint8_t* sa = tiles + stage * L::kStageBytes;
           uint8_t* sb = sa + kATileBytes;
           mbar_arrive_expect_tx(full + stage, L::kStageBytes);
-          tma_load_2d(sa, &tmA, full + stage, kb * BK, ti.a_row, pol_a);
-          if (P::NUM_B == 1) {
-            tma_load_2d(sb, &tmB0, full + stage, kb * BK, ti.b_row, pol_b);
+          if constexpr (P::CUSTOM_LOADS) {
+            P::issue_loads(args, &tmA, &tmB0, &tmB1, ti, kb, sa, sb, full + stage, pol_a, pol_b);
           } else {
-            tma_load_2d(sb, &tmB0, full + stage, kb * BK, ti.b_row, pol_b);
-            tma_load_2d(sb + L::kBTileBytes / 2, &tmB1, full + stage, kb * BK, ti.b_row, pol_b);
+            tma_load_2d(sa, &tmA, full + stage, kb * BK, ti.a_row, pol_a);
+            if (P::NUM_B == 1) {
+              tma_load_2d(sb, &tmB0, full + stage, kb * BK, ti.b_row, pol_b);
+            } else {
+              tma_load_2d(sb, &tmB0, full + stage, kb * BK, ti.b_row, pol_b);
+              tma_load_2d(sb + L::kBTileBytes / 2, &tmB1, full + stage, kb * BK, ti.b_row, pol_b);
+            }
           }
           ++issued;
           if (++stage == STAGES) {
@@ -646,6 +920,78 @@ __global__ void __launch_bounds__(P::THREADS, 1)
         }
         mbar_wait(full + s, ph, nullptr, args.status);
       }
+    }
+  } else if (warp == 1 && P::MASK_K) {
+    // ------------------------------------- MMA issuer, K tails zeroed
+    // The whole warp walks the schedule; lane 0 waits on the barriers and
+    // issues the MMAs.  In the last K block of a segment the rows past its
+    // end (the next segment's, loaded by the same box) are zeroed in both
+    // operands by the 32 lanes first: each K row is one 128-byte line of
+    // every 8 KB box of the stage, whatever the swizzle.
+    int stage = 0;
+    uint32_t phase = 0;
+    int it = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++it) {
+      const int acc = it & 1;
+      const uint32_t aph = (it >> 1) & 1;
+      int go = 1;
+      if (lane == 0) go = mbar_wait(tempty + acc, aph ^ 1u, abort_flag, args.status) ? 1 : 0;
+      go = __shfl_sync(0xffffffffu, go, 0);
+      if (!go) break;
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+      const TileInfo ti = P::tile_info(args, sched, tile);
+      for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
+        if (lane == 0) go = mbar_wait(full + stage, phase, abort_flag, args.status) ? 1 : 0;
+        go = __shfl_sync(0xffffffffu, go, 0);
+        if (!go) {
+          ok = false;
+          break;
+        }
+        uint8_t* sa = tiles + stage * L::kStageBytes;
+        const int rows = P::k_rows(ti, kb);
+        if (rows < BK) {
+          // every lane observes the landed stage before overwriting it
+          if (!mbar_wait(full + stage, phase, abort_flag, args.status)) go = 0;
+          if (!__all_sync(0xffffffffu, go)) {
+            ok = false;
+            break;
+          }
+          const int per_box = (BK - rows) * 8;   // 16-byte chunks to clear per box
+          constexpr int kBoxes = L::kStageBytes / kMnBoxBytes;
+          for (int i = lane; i < kBoxes * per_box; i += 32) {
+            const int bx = i / per_box;
+            const int j = i - bx * per_box;
+            *reinterpret_cast<uint4*>(sa + bx * kMnBoxBytes + rows * 128 + j * 16) =
+                make_uint4(0u, 0u, 0u, 0u);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+        }
+        if (lane == 0) {
+          tc_fence_after();
+          const uint64_t ad = sw128_mnmajor_desc(sa, kMnBoxBytes);
+          const uint64_t bd = sw128_mnmajor_desc(sa + kATileBytes, kMnBoxBytes);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            tc_mma_bf16(d_tmem, ad + A_KSTEP * kk, bd + B_KSTEP * kk, IDESC,
+                        (kb != ti.kb0 || kk != 0) ? 1u : 0u);
+          tc_commit(empty + stage);
+        }
+        __syncwarp();
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) break;
+      if (lane == 0) tc_commit(tfull + acc);
+      __syncwarp();
+    }
+    if (lane == 0) {
+      tc_commit(mma_done);
+      mbar_wait(mma_done, 0, nullptr, args.status);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -668,9 +1014,11 @@ __global__ void __launch_bounds__(P::THREADS, 1)
           }
           tc_fence_after();
           const uint8_t* sa = tiles + stage * L::kStageBytes;
-          const uint64_t ad = sw128_kmajor_desc(sa);
-          const uint64_t bd = sw128_kmajor_desc(sa + kATileBytes);
-          if (BN == 256 && ti.swap_np) {
+          const uint64_t ad =
+              P::A_MN ? sw128_mnmajor_desc(sa, kMnBoxBytes) : sw128_kmajor_desc(sa);
+          const uint64_t bd = P::B_MN ? sw128_mnmajor_desc(sa + kATileBytes, kMnBoxBytes)
+                                      : sw128_kmajor_desc(sa + kATileBytes);
+          if (BN == 256 && !P::A_MN && !P::B_MN && ti.swap_np) {
             // D[:, 0:np) = B[0:128) A^T, D[:, np:2np) = B[128:256) A^T
             const uint32_t idesc_s = idesc_bf16_f32(128, ti.swap_np);
             const uint64_t bd_hi = bd + ((128u * 128u) >> 4);   // rows 128.. of the B stage
@@ -684,7 +1032,7 @@ __global__ void __launch_bounds__(P::THREADS, 1)
           } else {
 #pragma unroll
             for (int kk = 0; kk < BK / 16; ++kk)
-              tc_mma_bf16(d_tmem, ad + 2u * kk, bd + 2u * kk, IDESC,
+              tc_mma_bf16(d_tmem, ad + A_KSTEP * kk, bd + B_KSTEP * kk, IDESC,
                           (kb != ti.kb0 || kk != 0) ? 1u : 0u);
           }
           tc_commit(empty + stage);
@@ -1060,7 +1408,8 @@ cudaError_t launch_router_tc(const void* x, const void* w_router, int T, int d, 
 static cudaError_t swiglu_tc_impl(const void* a_src, int a_rows, const int32_t* src_row,
                                   const int32_t* offsets, const void* w1, const void* w3,
                                   const void* w2, const float* row_scale, int N, int d, int h,
-                                  int E, void* y, void* H, int* status, cudaStream_t s);
+                                  int E, void* y, void* H, int* status, cudaStream_t s,
+                                  void* gu = nullptr);
 
 cudaError_t launch_swiglu_tc(const void* x_perm, const int32_t* offsets, const void* w1,
                              const void* w3, const void* w2, const float* row_scale, int N,
@@ -1081,7 +1430,8 @@ cudaError_t launch_swiglu_tc_gather(const void* x, int T, const int32_t* src_row
 static cudaError_t swiglu_tc_impl(const void* a_src, int a_rows, const int32_t* src_row,
                                   const int32_t* offsets, const void* w1, const void* w3,
                                   const void* w2, const float* row_scale, int N, int d, int h,
-                                  int E, void* y, void* H, int* status, cudaStream_t s) {
+                                  int E, void* y, void* H, int* status, cudaStream_t s,
+                                  void* gu) {
   using namespace tc;
   CUtensorMap tx, t1, t3, th, t2;
   const bool gather = src_row != nullptr;
@@ -1109,6 +1459,7 @@ static cudaError_t swiglu_tc_impl(const void* a_src, int a_rows, const int32_t* 
   a.src_row = src_row;
   a.src_rows = a_rows;
   a.gather_src = a_src;
+  a.gu_out = static_cast<__nv_bfloat16*>(gu);
   if (pairs) {
     const long long max_pt = cdiv(N, 256) + E;   // upper bound on 256-row pair tiles
     int np = static_cast<int>(std::min<long long>(num_sms() / 2, max_pt * cdiv(h, 128)));
@@ -1132,6 +1483,77 @@ static cudaError_t swiglu_tc_impl(const void* a_src, int a_rows, const int32_t* 
   a.row_scale = row_scale;
   grid = static_cast<int>(std::min<long long>(num_sms(), 1LL * max_mt * cdiv(d, 256)));
   return launch<DownPolicy>(th, t2, t2, a, grid, s);
+}
+
+cudaError_t launch_swiglu_tc_train(const void* x_perm, const int32_t* offsets, const void* w1,
+                                   const void* w3, const void* w2, int N, int d, int h, int E,
+                                   void* y, void* H, void* GU, int* status, cudaStream_t s) {
+  return swiglu_tc_impl(x_perm, N, nullptr, offsets, w1, w3, w2, nullptr, N, d, h, E, y, H,
+                        status, s, GU);
+}
+
+// Backward of the grouped SwiGLU: four launches on `s`.
+//   1. dG | dU = SwiGLU'(G, U) applied to dY w2     (DownBwdPolicy, into dGU)
+//   2. dx_perm = dG w1 + dU w3                       (UpBwdPolicy)
+//   3. dw2 = dY^T H per expert                       (WgradPolicy)
+//   4. dw1 | dw3 = (dG | dU)^T x_perm per expert     (WgradPolicy, rows split at h)
+cudaError_t launch_swiglu_bwd_tc(const void* x_perm, const int32_t* offsets, const void* w1,
+                                 const void* w3, const void* w2, const void* H, const void* GU,
+                                 const void* dY, int N, int d, int h, int E, void* dX, void* dW1,
+                                 void* dW3, void* dW2, void* dGU, int* status, cudaStream_t s) {
+  using namespace tc;
+  const uint64_t Eh = static_cast<uint64_t>(E) * h, Ed = static_cast<uint64_t>(E) * d;
+  const int max_mt = cdiv(N, BM) + E;
+  CUtensorMap t_dy, t_w2, t_dgu, t_w1, t_w3;
+  if (!make_tmap(&t_dy, dY, d, N, BM)) return cudaErrorInvalidValue;
+  if (!make_tmap(&t_w2, w2, h, Ed, 64)) return cudaErrorInvalidValue;
+  if (!make_tmap(&t_dgu, dGU, 2 * static_cast<uint64_t>(h), N, BM)) return cudaErrorInvalidValue;
+  if (!make_tmap(&t_w1, w1, d, Eh, 64)) return cudaErrorInvalidValue;
+  if (!make_tmap(&t_w3, w3, d, Eh, 64)) return cudaErrorInvalidValue;
+  Args a{};
+  a.M = N;
+  a.E = E;
+  a.offsets = offsets;
+  a.status = status;
+  // 1. data gradient of GEMM2 and the SwiGLU backward
+  a.K = d;
+  a.n_out = h;
+  a.out = static_cast<__nv_bfloat16*>(dGU);
+  a.gu_in = static_cast<const __nv_bfloat16*>(GU);
+  int grid = static_cast<int>(std::min<long long>(num_sms(), 1LL * max_mt * cdiv(h, 256)));
+  cudaError_t e = launch<DownBwdPolicy>(t_dy, t_w2, t_w2, a, grid, s);
+  if (e != cudaSuccess) return e;
+  // 2. data gradient of GEMM1
+  a.K = 2 * h;
+  a.n_out = d;
+  a.out = static_cast<__nv_bfloat16*>(dX);
+  a.gu_in = nullptr;
+  grid = static_cast<int>(std::min<long long>(num_sms(), 1LL * max_mt * cdiv(d, 256)));
+  e = launch<UpBwdPolicy>(t_dgu, t_w1, t_w3, a, grid, s);
+  if (e != cudaSuccess) return e;
+  // 3. dw2[e] = dY_e^T H_e: output rows d (A = dY columns), columns h
+  CUtensorMap m_dy, m_h, m_dgu, m_x;
+  if (!make_tmap(&m_dy, dY, d, N, 64)) return cudaErrorInvalidValue;
+  if (!make_tmap(&m_h, H, h, N, 64)) return cudaErrorInvalidValue;
+  if (!make_tmap(&m_dgu, dGU, 2 * static_cast<uint64_t>(h), N, 64)) return cudaErrorInvalidValue;
+  if (!make_tmap(&m_x, x_perm, d, N, 64)) return cudaErrorInvalidValue;
+  a.K = 0;
+  a.Ma = d;
+  a.split = d;
+  a.n_out = h;
+  a.out = static_cast<__nv_bfloat16*>(dW2);
+  a.out1 = nullptr;
+  grid = static_cast<int>(std::min<long long>(num_sms(), 1LL * E * cdiv(d, BM) * cdiv(h, 256)));
+  e = launch<WgradPolicy>(m_dy, m_h, m_h, a, grid, s);
+  if (e != cudaSuccess) return e;
+  // 4. dw1[e] = dG_e^T x_e, dw3[e] = dU_e^T x_e: output rows 2h, columns d
+  a.Ma = 2 * h;
+  a.split = h;
+  a.n_out = d;
+  a.out = static_cast<__nv_bfloat16*>(dW1);
+  a.out1 = static_cast<__nv_bfloat16*>(dW3);
+  grid = static_cast<int>(std::min<long long>(num_sms(), 1LL * E * cdiv(2 * h, BM) * cdiv(d, 256)));
+  return launch<WgradPolicy>(m_dgu, m_x, m_x, a, grid, s);
 }
 
 }  // namespace moe

@@ -1,0 +1,257 @@
+"""GPU parity of the training path: the training forward of the experts
+(moe_grouped_swiglu_train), the backward of the grouped SwiGLU, of the
+combine and of the dispatch, against the fp64 oracle's derivatives.
+
+Tolerances (bf16 operands, fp32 accumulation; the backward reads the
+bf16-rounded G, U, H and rounds dG, dU once to bf16 before the next
+products, so each output carries at most a few bf16 roundings):
+
+* bf16 outputs: max|err| <= 3e-2 (1 + |ref|) and ||err||_F <= 1e-2 ||ref||_F
+* fp32 routing-weight gradients (dot products of bf16 rows): |err| <=
+  1.01 d 2^-24 sum_i |dout_i y_i| + 1e-30, the worst-case bound of an fp32
+  sum of d exact products.
+
+Integer layouts come from the oracle's dispatch; experts with no rows must
+get weight gradients that are exactly zero.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def M(cuda_ok):
+    from routing_dispatch_grouped_topk_b200 import build
+    build.build()
+    import routing_dispatch_grouped_topk_b200 as m
+    m.lib()
+    return m
+
+
+def f64(t):
+    return O.as_f64(t)
+
+
+def close(got, ref, tol_max=3e-2, tol_fro=1e-2):
+    g = f64(got)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert g.shape == ref.shape, (g.shape, ref.shape)
+    err = np.abs(g - ref)
+    bad = err > tol_max * (1 + np.abs(ref))
+    assert not bad.any(), f"{bad.sum()} elements off, worst {err.max()}"
+    den = np.linalg.norm(ref)
+    if den > 0:
+        assert np.linalg.norm(g - ref) <= tol_fro * den, np.linalg.norm(g - ref) / den
+
+
+def i32(a):
+    return torch.as_tensor(np.asarray(a), dtype=torch.int32, device="cuda")
+
+
+def expert_problem(counts, d, h, seed):
+    """x_perm [N, d], w1/w3 [E, h, d], w2 [E, d, h], dy [N, d] in bf16 with
+    the layer's scales (x, dy ~ N(0, 1), weights ~ N(0, 1/fan_in))."""
+    g = torch.Generator().manual_seed(seed)
+    E, N = len(counts), int(sum(counts))
+    bf = torch.bfloat16
+    xp = torch.randn(N, d, generator=g).to(bf)
+    w1 = (torch.randn(E, h, d, generator=g) / math.sqrt(d)).to(bf)
+    w3 = (torch.randn(E, h, d, generator=g) / math.sqrt(d)).to(bf)
+    w2 = (torch.randn(E, d, h, generator=g) / math.sqrt(h)).to(bf)
+    dy = torch.randn(N, d, generator=g).to(bf)
+    off = np.concatenate([[0], np.cumsum(counts)]).astype(np.int64)
+    return xp, w1, w3, w2, dy, off
+
+
+# Segment mixes: empty experts, single rows, 64 / 128 boundaries, ragged
+# tails, several 128-row tiles; d and h that leave partial 256-column and
+# 128-row tiles; the smallest d = h = 64.
+CASES = [
+    ([64, 0, 1, 129, 300, 17, 128], 256, 192),
+    ([5, 250, 0, 77], 320, 128),
+    ([130], 64, 64),
+    ([0, 0, 63, 65, 0], 128, 320),
+]
+
+
+@pytest.mark.parametrize("counts,d,h", CASES)
+def test_train_forward_keeps_g_u_h(M, counts, d, h):
+    xp, w1, w3, w2, _, off = expert_problem(counts, d, h, seed=sum(counts) + d)
+    c = [t.cuda() for t in (xp, w1, w3, w2)]
+    y, h_act, gu, ws = M.grouped_swiglu_train(c[0], i32(off), *c[1:])
+    torch.cuda.synchronize()
+    assert M.device_status(ws) == 0
+    G, U = O.grouped_preactivations(xp, off, w1, w3)
+    close(gu[:, :h], G)
+    close(gu[:, h:], U)
+    close(h_act, O.silu(G) * U)
+    close(y, O.grouped_swiglu(xp, off, w1, w3, w2))
+    # the same kernels as the inference forward: y is bit-identical
+    y_inf, _ = M.grouped_swiglu(c[0], i32(off), *c[1:])
+    assert torch.equal(y, y_inf)
+
+
+@pytest.mark.parametrize("counts,d,h", CASES)
+def test_grouped_swiglu_backward_matches_oracle(M, counts, d, h):
+    xp, w1, w3, w2, dy, off = expert_problem(counts, d, h, seed=7 * sum(counts) + h)
+    c = [t.cuda() for t in (xp, w1, w3, w2)]
+    o = i32(off)
+    _, h_act, gu, _ = M.grouped_swiglu_train(c[0], o, *c[1:])
+    dxp, dw1, dw3, dw2, ws = M.grouped_swiglu_backward(c[0], o, *c[1:], h_act, gu, dy.cuda())
+    torch.cuda.synchronize()
+    assert M.device_status(ws) == 0
+    rdx, rw1, rw3, rw2 = O.grouped_swiglu_backward(xp, off, w1, w3, w2, dy)
+    close(dxp, rdx)
+    close(dw1, rw1)
+    close(dw3, rw3)
+    close(dw2, rw2)
+    for e, n in enumerate(counts):
+        if n == 0:
+            assert not dw1[e].any() and not dw3[e].any() and not dw2[e].any()
+
+
+def test_backward_with_no_rows_zeroes_weight_gradients(M):
+    xp, w1, w3, w2, dy, off = expert_problem([0, 0, 0], 128, 64, seed=1)
+    c = [t.cuda() for t in (w1, w3, w2)]
+    empty = torch.empty(0, 128, dtype=torch.bfloat16, device="cuda")
+    dw = [torch.full_like(t, 5.0) for t in c]
+    ws = torch.empty(M.grouped_swiglu_backward_workspace_size(0, 128, 64, 3, M.MOE_BF16),
+                     dtype=torch.uint8, device="cuda")
+    M.moe_grouped_swiglu_backward(empty, i32(off), *c, empty, empty, empty, 0, 128, 64, 3,
+                                  M.MOE_BF16, empty, *dw, ws)
+    torch.cuda.synchronize()
+    assert all(not t.any() for t in dw)
+
+
+def test_backward_rejects_bad_offsets_without_writing(M):
+    xp, w1, w3, w2, dy, off = expert_problem([10, 6], 64, 64, seed=2)
+    c = [t.cuda() for t in (xp, w1, w3, w2)]
+    _, h_act, gu, _ = M.grouped_swiglu_train(c[0], i32(off), *c[1:])
+    dx = torch.full((16, 64), 3.0, dtype=torch.bfloat16, device="cuda")
+    dw = [torch.full_like(t, 3.0) for t in c[1:]]
+    ws = torch.empty(M.grouped_swiglu_backward_workspace_size(16, 64, 64, 2, M.MOE_BF16),
+                     dtype=torch.uint8, device="cuda")
+    for bad in ([0, 12, 10], [1, 6, 16], [0, 6, 15]):
+        M.moe_grouped_swiglu_backward(c[0], i32(bad), *c[1:], h_act, gu, dy.cuda(), 16, 64, 64,
+                                      2, M.MOE_BF16, dx, *dw, ws)
+        assert M.device_status(ws) & M.MOE_DEV_BAD_OFFSETS
+    assert torch.all(dx == 3.0) and all(torch.all(t == 3.0) for t in dw)
+
+
+def _routing(T, E, k, seed):
+    L = W.make_logits(T, E, k, seed=seed)
+    idx, w, _, _ = O.router_topk(k, True, logits=L)
+    _, off, src, dst = O.dispatch(idx, E)
+    return idx, w, off, src, dst
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("k", [1, 2, 8, 16])
+def test_combine_backward_matches_oracle(M, dtype, k):
+    T, E, d = 300, 32, 256
+    idx, w, off, src, dst = _routing(T, E, k, seed=k)
+    g = torch.Generator().manual_seed(k)
+    N = T * k
+    y = torch.randn(N, d, generator=g).to(dtype)
+    dout = torch.randn(T, d, generator=g).to(dtype)
+    wt = torch.from_numpy(w).float()
+    dy, dw = M.combine_backward(dout.cuda(), y.cuda(), i32(dst), wt.cuda())
+    rdy, rdw = O.combine_backward(dout, y, dst, wt)
+    if dtype == torch.bfloat16:
+        close(dy, rdy)
+    else:
+        close(dy, rdy, 1e-6, 1e-6)
+    # fp32 dot products of d exact products: worst-case recursive-sum bound
+    yy, gg = f64(y), f64(dout)
+    mag = np.array([[np.abs(gg[t]) @ np.abs(yy[dst[t, j]]) for j in range(k)] for t in range(T)])
+    err = np.abs(f64(dw) - rdw)
+    assert np.all(err <= 1.01 * d * 2.0 ** -24 * mag + 1e-30), err.max()
+    # unweighted, no weight gradient
+    dy1, dw1 = M.combine_backward(dout.cuda(), y.cuda(), i32(dst), None, want_dw=False)
+    assert dw1 is None
+    assert torch.equal(dy1.cpu()[torch.from_numpy(dst[:, 0]).long()], dout)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_dispatch_backward_matches_oracle(M, dtype):
+    T, E, k, d = 257, 16, 4, 128
+    idx, w, off, src, dst = _routing(T, E, k, seed=5)
+    g = torch.Generator().manual_seed(9)
+    dxp = torch.randn(T * k, d, generator=g).to(dtype)
+    dx = M.dispatch_backward(dxp.cuda(), i32(dst))
+    ref = O.dispatch_backward(dxp, dst)
+    if dtype == torch.bfloat16:
+        close(dx, ref)
+    else:
+        close(dx, ref, 1e-6, 1e-6)
+
+
+@pytest.mark.parametrize("cfg_index", [1, 2])
+def test_training_chain_full_size_sampled(M, cfg_index):
+    """The whole training chain at the Qwen3-30B-A3B layer sizes (T=4096
+    near-uniform, T=16384 Zipf-skewed): router and dispatch on the GPU,
+    training forward, combine backward of a random dout, experts backward,
+    dispatch backward.  The weight gradients of three experts (the first,
+    the largest, one in the middle) and the input gradients of 16 sampled
+    tokens are checked against the oracle, one expert's rows at a time."""
+    cfg = W.config(cfg_index)
+    lay = W.make_layer(cfg, device="cuda")
+    x, wr, w1, w3, w2 = (lay[n] for n in ("x", "w_router", "w1", "w3", "w2"))
+    T, d, E, k, h = cfg.T, cfg.d, cfg.E, cfg.top_k, cfg.h
+    idx, tw, counts, _, _ = M.router_topk(x, wr, k, True)
+    cnt, off, src, dst, xp, _ = M.dispatch(x, idx, E)
+    y, h_act, gu, _ = M.grouped_swiglu_train(xp, off, w1, w3, w2)
+    g = torch.Generator(device="cuda").manual_seed(cfg.seed)
+    dout = torch.randn(T, d, generator=g, device="cuda").to(torch.bfloat16)
+    dy, dtw = M.combine_backward(dout, y, dst, tw)
+    dxp, dw1, dw3, dw2, ws = M.grouped_swiglu_backward(xp, off, w1, w3, w2, h_act, gu, dy)
+    dx = M.dispatch_backward(dxp, dst)
+    torch.cuda.synchronize()
+    assert M.device_status(ws) == 0
+    offs = off.cpu().numpy().astype(np.int64)
+    cnt_h = np.diff(offs)
+    # weight gradients of three experts, from their whole segments
+    for e in sorted({0, int(np.argmax(cnt_h)), E // 2}):
+        lo, hi = int(offs[e]), int(offs[e + 1])
+        sub = np.array([0, hi - lo])
+        _, rw1, rw3, rw2 = O.grouped_swiglu_backward(
+            xp[lo:hi].cpu(), sub, w1[e:e + 1].cpu(), w3[e:e + 1].cpu(), w2[e:e + 1].cpu(),
+            dy[lo:hi].cpu())
+        close(dw1[e], rw1[0])
+        close(dw3[e], rw3[0])
+        close(dw2[e], rw2[0])
+    # input gradients of sampled tokens: dx_perm rows are row-local, so each
+    # expert's sampled rows form their own segment
+    rng = np.random.default_rng(cfg.seed)
+    toks = rng.choice(T, 16, replace=False)
+    dst_h = dst.cpu().numpy()
+    idx_h = idx.cpu().numpy()
+    rows = {}
+    for t in toks:
+        for j in range(k):
+            rows.setdefault(int(idx_h[t, j]), []).append(int(dst_h[t, j]))
+    ref_dxp = {}
+    for e, rs in rows.items():
+        rs_t = torch.as_tensor(rs, device="cuda").long()
+        rdx, _, _, _ = O.grouped_swiglu_backward(
+            xp[rs_t].cpu(), np.array([0, len(rs)]), w1[e:e + 1].cpu(), w3[e:e + 1].cpu(),
+            w2[e:e + 1].cpu(), dy[rs_t].cpu())
+        close(dxp[rs_t], rdx)
+        for r, v in zip(rs, rdx):
+            ref_dxp[r] = v
+    ref_dx = np.stack([sum(ref_dxp[int(dst_h[t, j])] for j in range(k)) for t in toks])
+    close(dx[torch.as_tensor(toks, device="cuda").long()], ref_dx)
+    # routing-weight gradients of the sampled tokens
+    yy = f64(y[torch.as_tensor(dst_h[toks].ravel(), device="cuda").long()]).reshape(16, k, d)
+    gg = f64(dout[torch.as_tensor(toks, device="cuda").long()])
+    ref_dtw = np.einsum("td,tjd->tj", gg, yy)
+    mag = np.einsum("td,tjd->tj", np.abs(gg), np.abs(yy))
+    assert np.all(np.abs(f64(dtw[torch.as_tensor(toks, device="cuda").long()]) - ref_dtw)
+                  <= 1.01 * d * 2.0 ** -24 * mag + 1e-30)
