@@ -7,6 +7,15 @@ bf16-rounded G, U, H and rounds dG, dU once to bf16 before the next
 products, so each output carries at most a few bf16 roundings):
 
 * bf16 outputs: max|err| <= 3e-2 (1 + |ref|) and ||err||_F <= 1e-2 ||ref||_F
+* weight gradients (sums over an expert's rows): per expert,
+  max|err| <= 6e-2 (|ref| + rms(ref)) and ||err||_F <= 1e-2 ||ref||_F.
+  Every term of the sum carries the relative rounding of the saved bf16 G
+  and U (about 2^-8, larger near the zero of silu' where it is |G| silu''
+  times 2^-9 in absolute terms); the terms have random signs, so the error
+  of the sum scales with the size of a typical entry (the RMS), not with
+  the entry itself, which can cancel to near zero.  An fp64 emulation of
+  exactly these roundings gives max err / (|ref| + rms) = 0.026 on the cases
+  below and a Frobenius error of 0.3%.
 * fp32 routing-weight gradients (dot products of bf16 rows): |err| <=
   1.01 d 2^-24 sum_i |dout_i y_i| + 1e-30, the worst-case bound of an fp32
   sum of d exact products.
@@ -49,6 +58,21 @@ def close(got, ref, tol_max=3e-2, tol_fro=1e-2):
     den = np.linalg.norm(ref)
     if den > 0:
         assert np.linalg.norm(g - ref) <= tol_fro * den, np.linalg.norm(g - ref) / den
+
+
+def close_wgrad(got, ref):
+    """Weight gradient of one expert: RMS-relative elementwise bound and a
+    Frobenius bound (see the module docstring)."""
+    g = f64(got)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert g.shape == ref.shape, (g.shape, ref.shape)
+    rms = np.sqrt(np.mean(ref ** 2))
+    err = np.abs(g - ref)
+    bad = err > 6e-2 * (np.abs(ref) + rms)
+    assert not bad.any(), f"{bad.sum()} elements off, worst {(err / (np.abs(ref) + rms)).max()}"
+    den = np.linalg.norm(ref)
+    if den > 0:
+        assert np.linalg.norm(g - ref) <= 1e-2 * den, np.linalg.norm(g - ref) / den
 
 
 def i32(a):
@@ -109,12 +133,13 @@ def test_grouped_swiglu_backward_matches_oracle(M, counts, d, h):
     assert M.device_status(ws) == 0
     rdx, rw1, rw3, rw2 = O.grouped_swiglu_backward(xp, off, w1, w3, w2, dy)
     close(dxp, rdx)
-    close(dw1, rw1)
-    close(dw3, rw3)
-    close(dw2, rw2)
     for e, n in enumerate(counts):
         if n == 0:
             assert not dw1[e].any() and not dw3[e].any() and not dw2[e].any()
+            continue
+        close_wgrad(dw1[e], rw1[e])
+        close_wgrad(dw3[e], rw3[e])
+        close_wgrad(dw2[e], rw2[e])
 
 
 def test_backward_with_no_rows_zeroes_weight_gradients(M):
@@ -224,9 +249,9 @@ def test_training_chain_full_size_sampled(M, cfg_index):
         _, rw1, rw3, rw2 = O.grouped_swiglu_backward(
             xp[lo:hi].cpu(), sub, w1[e:e + 1].cpu(), w3[e:e + 1].cpu(), w2[e:e + 1].cpu(),
             dy[lo:hi].cpu())
-        close(dw1[e], rw1[0])
-        close(dw3[e], rw3[0])
-        close(dw2[e], rw2[0])
+        close_wgrad(dw1[e], rw1[0])
+        close_wgrad(dw3[e], rw3[0])
+        close_wgrad(dw2[e], rw2[0])
     # input gradients of sampled tokens: dx_perm rows are row-local, so each
     # expert's sampled rows form their own segment
     rng = np.random.default_rng(cfg.seed)
