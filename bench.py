@@ -13,6 +13,11 @@ weak scaling, no data-path collective).
 
 ``--impl reference`` times the fp64 CPU oracle on the host cores instead
 (a bounded token sample per step) and prints the same metric.
+
+``--training`` times the training step instead (its own JSON line): the
+forward with the experts' training variant (which keeps G | U), then the
+backward of the combine, of the grouped SwiGLU (data and weight gradients)
+and of the dispatch, each stage bracketed by CUDA events.
 """
 from __future__ import annotations
 
@@ -553,6 +558,142 @@ def run_ours(args, ws, rank, local):
     print(json.dumps(line), flush=True)
 
 
+TRAIN_STAGES = ["router", "dispatch", "grouped_swiglu_train", "combine", "combine_backward",
+                "grouped_swiglu_backward", "dispatch_backward"]
+# kernels of ours per training step: router 2, dispatch 3 (histogram, scan,
+# scatter), training GEMMs 2, combine 1, combine backward 1, backward GEMMs 4,
+# dispatch backward 1
+TRAIN_LAUNCHES = 14
+
+
+def run_training(args, ws, rank, local):
+    import routing_dispatch_grouped_topk_b200 as M
+    M.lib()
+    cfg = W.config(args.config)
+    if cfg.dtype != "bf16" or cfg.ep_ranks != 1:
+        raise SystemExit("--training runs the bf16 single-device layouts (configs 1-3)")
+    T, d, E, k, h = cfg.T, cfg.d, cfg.E, cfg.top_k, cfg.h
+    N = T * k
+    dev = torch.device("cuda", local)
+    lay = W.make_layer(cfg, dev)
+    if rank:
+        lay["x"] = W.make_layer(rank_workload(cfg, rank), dev, experts=False)["x"]
+    x, wr, w1, w3, w2 = lay["x"], lay["w_router"], lay["w1"], lay["w3"], lay["w2"]
+    dt = M.MOE_BF16
+    stream = torch.cuda.current_stream()
+    bf = torch.bfloat16
+    g = torch.Generator(device=dev).manual_seed(cfg.seed * 7 + rank)
+    dout = torch.randn(T, d, generator=g, device=dev).to(bf)
+    idx = torch.empty(T, k, dtype=torch.int32, device=dev)
+    w = torch.empty(T, k, dtype=torch.float32, device=dev)
+    rws = torch.empty(M.router_workspace_size(T, d, E, dt), dtype=torch.uint8, device=dev)
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    src_row = torch.empty(N, dtype=torch.int32, device=dev)
+    dst_pos = torch.empty(T, k, dtype=torch.int32, device=dev)
+    x_perm = torch.empty(N, d, dtype=bf, device=dev)
+    dws = torch.empty(M.dispatch_workspace_size(T, E, k), dtype=torch.uint8, device=dev)
+    y = torch.empty(N, d, dtype=bf, device=dev)
+    h_act = torch.empty(N, h, dtype=bf, device=dev)
+    gu = torch.empty(N, 2 * h, dtype=bf, device=dev)
+    tws = torch.empty(256, dtype=torch.uint8, device=dev)
+    out = torch.empty(T, d, dtype=bf, device=dev)
+    dy = torch.empty(N, d, dtype=bf, device=dev)
+    dtw = torch.empty(T, k, dtype=torch.float32, device=dev)
+    dxp = torch.empty(N, d, dtype=bf, device=dev)
+    dw1, dw3, dw2 = torch.empty_like(w1), torch.empty_like(w3), torch.empty_like(w2)
+    bws = torch.empty(M.grouped_swiglu_backward_workspace_size(N, d, h, E, dt),
+                      dtype=torch.uint8, device=dev)
+    dx = torch.empty(T, d, dtype=bf, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step(ev=None):
+        def mark(i):
+            if ev is not None:
+                ev[i].record(stream)
+        mark(0)
+        M.moe_router_topk(x, wr, None, T, d, E, k, M.MOE_SCORE_SOFTMAX, cfg.renormalize, dt, None,
+                          idx, w, None, rws)
+        mark(1)
+        M.moe_dispatch(x, idx, T, d, E, k, dt, counts, offsets, src_row, dst_pos, x_perm, dws)
+        mark(2)
+        M.moe_grouped_swiglu_train(x_perm, offsets, w1, w3, w2, N, d, h, E, dt, y, h_act, gu, tws)
+        mark(3)
+        M.moe_combine(y, dst_pos, None, w, T, d, N, k, dt, out)
+        mark(4)
+        M.moe_combine_backward(dout, y, dst_pos, w, T, d, N, k, dt, dy, dtw)
+        mark(5)
+        M.moe_grouped_swiglu_backward(x_perm, offsets, w1, w3, w2, h_act, gu, dy, N, d, h, E, dt,
+                                      dxp, dw1, dw3, dw2, bws)
+        mark(6)
+        M.moe_dispatch_backward(dxp, dst_pos, T, d, N, k, dt, dx)
+        mark(7)
+
+    if args.profile:
+        for _ in range(2):
+            step()
+        torch.cuda.synchronize()
+        return
+    sampler = ClockSampler(local)
+    if rank == 0:
+        sampler.start()
+    t_warm = time.perf_counter()
+    n_warm = 0
+    while n_warm < args.warmup or time.perf_counter() - t_warm < 1.5:
+        step()
+        flush.zero_()
+        n_warm += 1
+        if n_warm % 8 == 0:
+            torch.cuda.synchronize()
+    torch.cuda.synchronize()
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(len(TRAIN_STAGES) + 1)]
+              for _ in range(args.steps)]
+    barrier(ws)
+    torch.cuda.synchronize()
+    for s_ in range(args.steps):
+        step(events[s_])
+        flush.zero_()          # L2 flush between steps, outside the step's events
+    torch.cuda.synchronize()
+    barrier(ws)
+    clocks = sampler.stop() if rank == 0 else None
+    total_ms = sum(ev[0].elapsed_time(ev[-1]) for ev in events)
+    total_ms_max = max_over_ranks(total_ms, ws)
+    status = int(bws[:4].view(torch.int32)[0].item())
+    if rank != 0:
+        return
+    pk = peaks()
+    stage_ms = {n: statistics.mean(ev[i].elapsed_time(ev[i + 1]) for ev in events)
+                for i, n in enumerate(TRAIN_STAGES)}
+    bwd_flops = 2 * cfg.gemm_flops()   # dgrad 2Ndh + 4Ndh, wgrad 2Ndh + 4Ndh
+    fwd_flops = cfg.gemm_flops()
+    bwd_ms = stage_ms["grouped_swiglu_backward"]
+    tflops = bwd_flops / (bwd_ms / 1e3) / 1e12
+    line = {
+        "metric": "MoE-layer training step (forward + backward) routed tokens/s (bf16)",
+        "value": job_tokens_per_s(T, ws, args.steps, total_ms_max), "unit": UNIT,
+        "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": total_ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": cfg.name, "T": T, "d": d, "E": E, "top_k": k, "h": h,
+                   "global_batch": T * ws, "parallelism": f"dp{ws}",
+                   "l2": "flushed between steps (256 MB write, outside step events)",
+                   "inputs": "seeded synthetic, resident in HBM; dout ~ N(0,1)"},
+        "roofline": {"kernel": "moe_grouped_swiglu_backward (4 tcgen05 GEMMs: dgrad w2 + "
+                               "SwiGLU', dgrad w1|w3, wgrad w2, wgrad w1|w3)",
+                     "bound": "tensor", "achieved": tflops,
+                     "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                     "frac": tflops / pk["bf16_tflops_sustained"], "traffic": None,
+                     "launch_ms": bwd_ms, "algorithmic_flops_per_launch": bwd_flops,
+                     "peak_kind": f"bf16 sustained, {pk['source']}"},
+        "forward_experts_tflops": fwd_flops / (stage_ms["grouped_swiglu_train"] / 1e3) / 1e12,
+        "stage_ms": stage_ms,
+        "device_status": status,
+        "gpu_launches": args.steps * TRAIN_LAUNCHES,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -564,6 +705,8 @@ def main():
     ap.add_argument("--cpu-tokens", type=int, default=256)
     ap.add_argument("--ref-tokens", type=int, default=128)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--training", action="store_true",
+                    help="time the training step (forward + backward) instead")
     ap.add_argument("--profile", action="store_true",
                     help="for ncu captures: run the staged step twice, then moe_forward "
                          "once, and exit (no timing, no JSON)")
@@ -577,7 +720,10 @@ def main():
         return
     ws, rank, local = dist_setup(args.gpus)
     try:
-        run_ours(args, ws, rank, local)
+        if args.training:
+            run_training(args, ws, rank, local)
+        else:
+            run_ours(args, ws, rank, local)
     finally:
         if ws > 1:
             import torch.distributed as dist

@@ -115,6 +115,8 @@ struct RouterPolicy {
   static constexpr int NUM_B = 1;
   static constexpr bool GATHER_A = false;
   static constexpr bool A_MN = false, B_MN = false, MASK_K = false, CUSTOM_LOADS = false;
+  static constexpr int EPI_STAGE_BYTES = 0;   // shared staging of the epilogue warps
+  static constexpr int EPI_WARPS = 4;         // one per TMEM lane quadrant
   static __device__ int k_rows(const TileInfo&, int) { return BK; }
   static constexpr int THREADS = kThreads;
   static constexpr int SCHED_INTS = 8;
@@ -172,6 +174,8 @@ struct GroupedSched {
   static constexpr int NUM_B = NUM_B_;
   static constexpr bool GATHER_A = false;
   static constexpr bool A_MN = false, B_MN = false, MASK_K = false, CUSTOM_LOADS = false;
+  static constexpr int EPI_STAGE_BYTES = 0;   // shared staging of the epilogue warps
+  static constexpr int EPI_WARPS = 4;         // one per TMEM lane quadrant
   static __device__ int k_rows(const TileInfo&, int) { return BK; }
   static constexpr int THREADS = kThreads;
   static constexpr int SCHED_INTS = 8 + 2 * (kMaxExperts + 1);
@@ -477,12 +481,24 @@ constexpr int kMnBoxBytes = 64 * BK * 2;   // one 64 x 64 MN-major box: 8 KB
 
 __device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
+// Epilogue staging: a warp's 32 rows x 32 bf16 columns (64 bytes per row)
+// pass through 2 KB of shared memory so that global loads and stores move
+// whole 64-byte row segments (4 lanes per row, 8 rows per instruction)
+// instead of one 16-byte piece of 32 different rows.  The 16-byte part j of
+// row r sits at r * 64 + (j ^ ((r >> 1) & 3)) * 16: conflict-free both for
+// "one row per lane" and for "four lanes per row".
+__device__ __forceinline__ uint32_t stg_off(int r, int j) {
+  return static_cast<uint32_t>(r * 64 + ((j ^ ((r >> 1) & 3)) << 4));
+}
+
 // Data gradient of GEMM2 with the SwiGLU backward in the epilogue:
 // A = dY [N, d] (K-major, K = d), B = w2[e] [d, h] as K rows x h columns.
 // The accumulator holds dA for 256 hidden units; the epilogue reads G and U
 // from gu_in and writes dG | dU into `out` ([N, 2h], the layout of gu).
 struct DownBwdPolicy : GroupedSched<256, 1, 256> {
   static constexpr bool B_MN = true, CUSTOM_LOADS = true;
+  static constexpr int EPI_WARPS = 8;   // two per lane quadrant, 128 columns each
+  static constexpr int THREADS = kThreads + 128;
   static __device__ TileInfo tile_info(const Args& a, const int* sched, int tile) {
     int e, nt, mt, cnt, seg0;
     locate(a, sched, tile, e, nt, mt, cnt, seg0);
@@ -505,54 +521,101 @@ struct DownBwdPolicy : GroupedSched<256, 1, 256> {
     for (int c = 0; c < BN / 64; ++c)
       tma_load_2d(sb + c * kMnBoxBytes, tmB0, bar, ti.n0 + 64 * c, ti.b_row + kb * BK, pb);
   }
-  static __device__ void epilogue(const Args& a, int*, const TileInfo& ti, uint32_t taddr,
-                                  int row) {
+  static constexpr int EPI_STAGE_BYTES = 8 * 2048;   // per warp: 32 rows x 64 bytes
+  static __device__ void epilogue(const Args&, int*, const TileInfo&, uint32_t, int) {}
+  // Per 32-column chunk in [c0, c1): the warp loads G and U of its 32 rows
+  // (coalesced; the next chunk's loads are in flight while this one is
+  // computed), each lane takes its own row through shared memory, forms dG
+  // and dU with the accumulator's dA, and the warp stores them coalesced.
+  static __device__ void epilogue_staged(const Args& a, int*, const TileInfo& ti, uint32_t taddr,
+                                         int row, uint8_t* stg, int c0, int c1) {
     const int h = a.n_out;
-    const bool valid = row < ti.m_valid;
-    const size_t base = static_cast<size_t>(ti.a_row + row) * (2 * h) + ti.n0;
-#pragma unroll 1
-    for (int c = 0; c < 8; ++c) {
-      const bool live = valid && ti.n0 + c * 32 < h;
-      uint4 gq[4], uq[4];
-      if (live) {
-        const uint4* g4 = reinterpret_cast<const uint4*>(a.gu_in + base + c * 32);
-        const uint4* u4 = reinterpret_cast<const uint4*>(a.gu_in + base + h + c * 32);
+    const int lane = threadIdx.x & 31;
+    const int wrow0 = row - lane;
+    const int j = lane & 3;
+    auto load_chunk = [&](int c, uint4 (&buf)[8]) {
+      const bool live = ti.n0 + c * 32 < h;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          gq[q] = g4[q];
-          uq[q] = u4[q];
+      for (int q = 0; q < 4; ++q) {
+        const int rr = 8 * q + (lane >> 2);
+        if (live && wrow0 + rr < ti.m_valid) {
+          const __nv_bfloat16* src =
+              a.gu_in + static_cast<size_t>(ti.a_row + wrow0 + rr) * (2 * h) + ti.n0 + c * 32 + j * 8;
+          buf[q] = *reinterpret_cast<const uint4*>(src);
+          buf[4 + q] = *reinterpret_cast<const uint4*>(src + h);
+        } else {
+          buf[q] = make_uint4(0u, 0u, 0u, 0u);
+          buf[4 + q] = make_uint4(0u, 0u, 0u, 0u);
         }
       }
+    };
+    // coalesced rows -> staging -> this lane's row (16 words)
+    auto to_row = [&](const uint4* part, uint32_t (&w)[16]) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        *reinterpret_cast<uint4*>(stg + stg_off(8 * q + (lane >> 2), j)) = part[q];
+      __syncwarp();
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        const uint4 v = *reinterpret_cast<const uint4*>(stg + stg_off(lane, p));
+        w[4 * p] = v.x;
+        w[4 * p + 1] = v.y;
+        w[4 * p + 2] = v.z;
+        w[4 * p + 3] = v.w;
+      }
+      __syncwarp();
+    };
+    // this lane's row (16 words) -> staging -> coalesced stores at column offset
+    auto from_row = [&](const uint32_t (&w)[16], int c, int col_off) {
+#pragma unroll
+      for (int p = 0; p < 4; ++p)
+        *reinterpret_cast<uint4*>(stg + stg_off(lane, p)) =
+            make_uint4(w[4 * p], w[4 * p + 1], w[4 * p + 2], w[4 * p + 3]);
+      __syncwarp();
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int rr = 8 * q + (lane >> 2);
+        if (wrow0 + rr < ti.m_valid)
+          *reinterpret_cast<uint4*>(a.out + static_cast<size_t>(ti.a_row + wrow0 + rr) * (2 * h) +
+                                    col_off + ti.n0 + c * 32 + j * 8) =
+              *reinterpret_cast<const uint4*>(stg + stg_off(rr, j));
+      }
+      __syncwarp();
+    };
+    uint4 cur[8], nxt[8];
+    load_chunk(c0, cur);
+#pragma unroll 1
+    for (int c = c0; c < c1; ++c) {
+      const bool live = ti.n0 + c * 32 < h;
+      if (c + 1 < c1) load_chunk(c + 1, nxt);
       uint32_t r[32];
       tmem_ld32(taddr + c * 32, r);
       tmem_ld_wait();
-      if (!live) continue;
-      const uint32_t* gw = reinterpret_cast<const uint32_t*>(gq);
-      const uint32_t* uw = reinterpret_cast<const uint32_t*>(uq);
-      uint32_t pg[16], pu[16];
+      if (live) {
+        uint32_t gw[16], uw[16];
+        to_row(cur, gw);
+        to_row(cur + 4, uw);
+        uint32_t pg[16], pu[16];
 #pragma unroll
-      for (int q = 0; q < 16; ++q) {
-        float dg[2], du[2];
+        for (int q = 0; q < 16; ++q) {
+          float dg[2], du[2];
 #pragma unroll
-        for (int hlf = 0; hlf < 2; ++hlf) {
-          const uint32_t gbits = hlf ? (gw[q] & 0xffff0000u) : (gw[q] << 16);
-          const uint32_t ubits = hlf ? (uw[q] & 0xffff0000u) : (uw[q] << 16);
-          const float g = __uint_as_float(gbits), u = __uint_as_float(ubits);
-          const float da = __uint_as_float(r[2 * q + hlf]);
-          const float sg = 1.0f / (1.0f + __expf(-g));
-          du[hlf] = da * (g * sg);
-          dg[hlf] = da * u * (sg * (1.0f + g * (1.0f - sg)));
+          for (int hlf = 0; hlf < 2; ++hlf) {
+            const float g = hlf ? bf16_hi(gw[q]) : bf16_lo(gw[q]);
+            const float u = hlf ? bf16_hi(uw[q]) : bf16_lo(uw[q]);
+            const float da = __uint_as_float(r[2 * q + hlf]);
+            const float sgm = 1.0f / (1.0f + __expf(-g));
+            du[hlf] = da * (g * sgm);
+            dg[hlf] = da * u * (sgm * (1.0f + g * (1.0f - sgm)));
+          }
+          pg[q] = pack_bf16x2(dg[0], dg[1]);
+          pu[q] = pack_bf16x2(du[0], du[1]);
         }
-        pg[q] = pack_bf16x2(dg[0], dg[1]);
-        pu[q] = pack_bf16x2(du[0], du[1]);
+        from_row(pg, c, 0);
+        from_row(pu, c, h);
       }
-      uint4* dg4 = reinterpret_cast<uint4*>(a.out + base + c * 32);
-      uint4* du4 = reinterpret_cast<uint4*>(a.out + base + h + c * 32);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        dg4[q] = make_uint4(pg[4 * q], pg[4 * q + 1], pg[4 * q + 2], pg[4 * q + 3]);
-        du4[q] = make_uint4(pu[4 * q], pu[4 * q + 1], pu[4 * q + 2], pu[4 * q + 3]);
-      }
+      for (int q = 0; q < 8; ++q) cur[q] = nxt[q];
     }
   }
   static __device__ void finish(const Args&, int*) {}
@@ -605,7 +668,8 @@ struct WgradPolicy {
   static constexpr int NUM_B = 1;
   static constexpr bool GATHER_A = false;
   static constexpr bool A_MN = true, B_MN = true, MASK_K = true, CUSTOM_LOADS = true;
-  static constexpr int THREADS = kThreads;
+  static constexpr int EPI_WARPS = 8;   // two per lane quadrant, 128 columns each
+  static constexpr int THREADS = kThreads + 128;
   static constexpr int SCHED_INTS = 8 + kMaxExperts + 1;   // [0] tiles [1] m-tiles [2] n-tiles, offsets
 
   static __device__ void prologue(const Args& a, int* sched) {
@@ -657,18 +721,33 @@ struct WgradPolicy {
 #pragma unroll
     for (int c = 0; c < BN / 64; ++c) tma_load_2d(sb + c * kMnBoxBytes, tmB0, bar, ti.n0 + 64 * c, y, pb);
   }
-  static __device__ void epilogue(const Args& a, int*, const TileInfo& ti, uint32_t taddr,
-                                  int row) {
-    const int m = ti.m0 + row;
-    const bool valid = m < a.Ma;
+  static constexpr int EPI_STAGE_BYTES = 8 * 2048;   // per warp: 32 rows x 64 bytes
+  static __device__ void epilogue(const Args&, int*, const TileInfo&, uint32_t, int) {}
+  // Each lane converts its row's 32 accumulator columns of a chunk to bf16
+  // into the warp's staging rows; the warp then stores 8 rows x 64 bytes per
+  // instruction.
+  static __device__ void epilogue_staged(const Args& a, int*, const TileInfo& ti, uint32_t taddr,
+                                         int row, uint8_t* stg, int c0, int c1) {
+    const int lane = threadIdx.x & 31;
+    const int wrow0 = row - lane;
     const int Nb = a.n_out;
     const int e = ti.b_row;
-    __nv_bfloat16* dst =
-        m < a.split ? a.out + (static_cast<size_t>(e) * a.split + m) * Nb + ti.n0
-                    : a.out1 + (static_cast<size_t>(e) * (a.Ma - a.split) + (m - a.split)) * Nb + ti.n0;
+    const int j = lane & 3;
     const bool empty = ti.kb1 == ti.kb0;
+    __nv_bfloat16* dst[4];
+    bool rvalid[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int m = ti.m0 + wrow0 + 8 * q + (lane >> 2);
+      rvalid[q] = m < a.Ma;
+      dst[q] = m < a.split
+                   ? a.out + (static_cast<size_t>(e) * a.split + m) * Nb + ti.n0 + j * 8
+                   : a.out1 + (static_cast<size_t>(e) * (a.Ma - a.split) + (m - a.split)) * Nb +
+                         ti.n0 + j * 8;
+    }
 #pragma unroll 1
-    for (int c = 0; c < 8; ++c) {
+    for (int c = c0; c < c1; ++c) {
+      if (ti.n0 + c * 32 >= Nb) break;   // warp-uniform
       uint32_t r[32];
       if (!empty) {
         tmem_ld32(taddr + c * 32, r);
@@ -677,15 +756,20 @@ struct WgradPolicy {
 #pragma unroll
         for (int q = 0; q < 32; ++q) r[q] = 0u;
       }
-      if (valid && ti.n0 + c * 32 < Nb) {
-        uint32_t p[16];
 #pragma unroll
-        for (int q = 0; q < 16; ++q)
-          p[q] = pack_bf16x2(__uint_as_float(r[2 * q]), __uint_as_float(r[2 * q + 1]));
-        uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+      for (int p = 0; p < 4; ++p)
+        *reinterpret_cast<uint4*>(stg + stg_off(lane, p)) =
+            make_uint4(pack_bf16x2(__uint_as_float(r[8 * p]), __uint_as_float(r[8 * p + 1])),
+                       pack_bf16x2(__uint_as_float(r[8 * p + 2]), __uint_as_float(r[8 * p + 3])),
+                       pack_bf16x2(__uint_as_float(r[8 * p + 4]), __uint_as_float(r[8 * p + 5])),
+                       pack_bf16x2(__uint_as_float(r[8 * p + 6]), __uint_as_float(r[8 * p + 7])));
+      __syncwarp();
 #pragma unroll
-        for (int q = 0; q < 4; ++q) d4[q] = make_uint4(p[4 * q], p[4 * q + 1], p[4 * q + 2], p[4 * q + 3]);
-      }
+      for (int q = 0; q < 4; ++q)
+        if (rvalid[q])
+          *reinterpret_cast<uint4*>(dst[q] + c * 32) =
+              *reinterpret_cast<const uint4*>(stg + stg_off(8 * q + (lane >> 2), j));
+      __syncwarp();
     }
   }
   static __device__ void finish(const Args&, int*) {}
@@ -704,11 +788,14 @@ struct Layout {
   static constexpr int kNumBars = 2 * kStages + 5;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSchedOff = (kMiscOff + 16 + 15) / 16 * 16;
-  static constexpr int kBytes = kSchedOff + P::SCHED_INTS * 4;
+  static constexpr int kEpiOff = (kSchedOff + P::SCHED_INTS * 4 + 15) / 16 * 16;
+  static constexpr int kBytes = kEpiOff + P::EPI_STAGE_BYTES;
   static constexpr int kLaunchBytes = kBytes + 1024;   // slack for 1 KB alignment
   static_assert(kLaunchBytes <= 227 * 1024, "shared memory budget");
   static_assert(kStages >= 2, "pipeline depth");
   static_assert(!P::GATHER_A || kStages == 4, "one gather warp per stage (warps 6..9)");
+  static_assert(!P::GATHER_A || P::EPI_WARPS == 4, "warps 6..9 are either gather or epilogue");
+  static_assert(P::THREADS == 64 + 32 * P::EPI_WARPS + (P::GATHER_A ? 128 : 0), "warp roles");
 };
 
 template <class P>
@@ -747,7 +834,7 @@ __global__ void __launch_bounds__(P::THREADS, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull + a, 1);
-      mbar_init(tempty + a, 4);
+      mbar_init(tempty + a, P::EPI_WARPS);
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -1047,10 +1134,15 @@ __global__ void __launch_bounds__(P::THREADS, 1)
       tc_commit(mma_done);
       mbar_wait(mma_done, 0, nullptr, args.status);
     }
-  } else if (warp < 6) {
+  } else if (warp < 2 + P::EPI_WARPS) {
     // -------------------------------------------------- epilogue warps
+    // Warp w reads TMEM lanes 32 (w % 4) .. +32 (its quadrant); with 8
+    // epilogue warps the two warps of a quadrant split the 8 column chunks.
     const int q = warp & 3;
     const int row = q * 32 + lane;
+    const int half = (warp - 2) >> 2;
+    const int c0 = P::EPI_WARPS == 8 ? 4 * half : 0;
+    const int c1 = P::EPI_WARPS == 8 ? c0 + 4 : 8;
     int it = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
       const int acc = it & 1;
@@ -1063,7 +1155,12 @@ __global__ void __launch_bounds__(P::THREADS, 1)
       const TileInfo ti = P::tile_info(args, sched, tile);
       const uint32_t taddr =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
-      P::epilogue(args, sched, ti, taddr, row);
+      if constexpr (P::EPI_STAGE_BYTES > 0)
+        P::epilogue_staged(args, sched, ti, taddr, row,
+                           smem + L::kEpiOff + (warp - 2) * (P::EPI_STAGE_BYTES / P::EPI_WARPS),
+                           c0, c1);
+      else
+        P::epilogue(args, sched, ti, taddr, row);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty + acc);
