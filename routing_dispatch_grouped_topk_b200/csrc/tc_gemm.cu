@@ -1009,12 +1009,14 @@ __global__ void __launch_bounds__(P::THREADS, 1)
       }
     }
   } else if (warp == 1 && P::MASK_K) {
-    // ------------------------------------- MMA issuer, K tails zeroed
+    // ------------------------------------- MMA issuer, K tails masked
     // The whole warp walks the schedule; lane 0 waits on the barriers and
-    // issues the MMAs.  In the last K block of a segment the rows past its
-    // end (the next segment's, loaded by the same box) are zeroed in both
-    // operands by the 32 lanes first: each K row is one 128-byte line of
-    // every 8 KB box of the stage, whatever the swizzle.
+    // issues the MMAs.  In the last K block of a segment only the 16-row MMA
+    // steps that hold segment rows are issued, and the rows of the last of
+    // them past the segment's end (the next segment's, loaded by the same
+    // box; fewer than 16) are zeroed in both operands by the 32 lanes
+    // first: each K row is one 128-byte line of every 8 KB box of the stage,
+    // whatever the swizzle.
     int stage = 0;
     uint32_t phase = 0;
     int it = 0;
@@ -1038,21 +1040,22 @@ __global__ void __launch_bounds__(P::THREADS, 1)
         }
         uint8_t* sa = tiles + stage * L::kStageBytes;
         const int rows = P::k_rows(ti, kb);
-        if (rows < BK) {
+        const int ksteps = (rows + 15) >> 4;   // 16-row MMA steps holding segment rows
+        const int zr = ksteps * 16 - rows;      // rows [rows, 16 ksteps) to clear
+        if (zr > 0) {
           // every lane observes the landed stage before overwriting it
           if (!mbar_wait(full + stage, phase, abort_flag, args.status)) go = 0;
           if (!__all_sync(0xffffffffu, go)) {
             ok = false;
             break;
           }
-          const int per_box = (BK - rows) * 8;   // 16-byte chunks to clear per box
+          const int per_box = zr * 8;   // 16-byte chunks to clear per box (< 128)
           constexpr int kBoxes = L::kStageBytes / kMnBoxBytes;
-          for (int i = lane; i < kBoxes * per_box; i += 32) {
-            const int bx = i / per_box;
-            const int j = i - bx * per_box;
-            *reinterpret_cast<uint4*>(sa + bx * kMnBoxBytes + rows * 128 + j * 16) =
-                make_uint4(0u, 0u, 0u, 0u);
-          }
+#pragma unroll
+          for (int bx = 0; bx < kBoxes; ++bx)
+            for (int i = lane; i < per_box; i += 32)
+              *reinterpret_cast<uint4*>(sa + bx * kMnBoxBytes + rows * 128 + i * 16) =
+                  make_uint4(0u, 0u, 0u, 0u);
           fence_proxy_async_smem();
           __syncwarp();
         }
@@ -1060,8 +1063,7 @@ __global__ void __launch_bounds__(P::THREADS, 1)
           tc_fence_after();
           const uint64_t ad = sw128_mnmajor_desc(sa, kMnBoxBytes);
           const uint64_t bd = sw128_mnmajor_desc(sa + kATileBytes, kMnBoxBytes);
-#pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk)
+          for (int kk = 0; kk < ksteps; ++kk)
             tc_mma_bf16(d_tmem, ad + A_KSTEP * kk, bd + B_KSTEP * kk, IDESC,
                         (kb != ti.kb0 || kk != 0) ? 1u : 0u);
           tc_commit(empty + stage);
