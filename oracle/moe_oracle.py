@@ -51,7 +51,7 @@ __all__ = [
     "ep_local_regroup", "apply_row_perm", "silu", "swiglu_ffn",
     "grouped_swiglu", "combine", "moe_forward", "dense_moe", "moe_tokens",
     "silu_grad", "grouped_preactivations", "combine_backward", "grouped_swiglu_backward",
-    "dispatch_backward",
+    "dispatch_backward", "router_backward",
 ]
 
 
@@ -539,6 +539,44 @@ def dispatch_backward(dx_perm, dst_pos) -> np.ndarray:
     collects the gradients of its copies, ``dx[t] = sum_j dx_perm[dst_pos[t,
     j]]`` (the adjoint of the row gather is the scatter-add)."""
     return combine(dx_perm, dst_pos, None)
+
+
+def router_backward(logits, topk_idx, d_topk_w, score: str = "softmax",
+                    renormalize: bool = False, route_scale: float = 1.0, x=None, w_router=None):
+    """Gradient of the routing weights of :func:`router_topk_general` with
+    respect to the gate logits, for upstream gradients ``d_topk_w [T, k]``
+    and the experts it selected (selection itself has no gradient; the
+    expert bias and the group masking only select).
+
+    Per token, with ``s`` the scores (softmax or sigmoid of the logits), ``S``
+    the selected set and ``c`` the route scale: ``w_j = c s_j / sum_S s``
+    (renormalised) or ``w_j = c s_j``, so ``ds_j = c (g_j - sum_S g s /
+    sum_S s) / sum_S s`` or ``ds_j = c g_j`` on ``S`` and 0 elsewhere; then
+    ``dz = s * (ds - <s, ds>)`` (softmax) or ``dz = ds * s (1 - s)``
+    (sigmoid).  Returns ``dz [T, E]``; with ``x`` and ``w_router`` also the
+    gate's gradients ``(dz, dw_router = dz^T x, dx = dz w_router)``.
+    """
+    L = as_f64(logits)
+    idx = _i64(topk_idx)
+    g = as_f64(d_topk_w)
+    T, E = L.shape
+    s = softmax(L) if score == "softmax" else sigmoid(L)
+    dz = np.zeros((T, E))
+    for t in range(T):
+        sel = s[t, idx[t]]
+        ds = np.zeros(E)
+        if renormalize:
+            tot = sel.sum()
+            ds[idx[t]] = route_scale * (g[t] - float(g[t] @ sel) / tot) / tot
+        else:
+            ds[idx[t]] = route_scale * g[t]
+        if score == "softmax":
+            dz[t] = s[t] * (ds - float(s[t] @ ds))
+        else:
+            dz[t] = ds * s[t] * (1.0 - s[t])
+    if x is None:
+        return dz
+    return dz, dz.T @ as_f64(x), dz @ as_f64(w_router)
 
 
 def dense_moe(x, idx, w, w1, w3, w2) -> np.ndarray:

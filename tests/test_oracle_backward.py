@@ -14,6 +14,7 @@ import torch
 import torch.nn.functional as F
 
 import oracle as O
+import workloads as W
 
 
 def _problem(seed=0, N=9, d=5, h=4, E=3, empty=1):
@@ -178,3 +179,60 @@ def test_pins_catch_planted_mistakes(mistake):
     errs = [np.max(np.abs(g - _fd(loss, a))) for g, a in zip((dxp, dw1, dw3, dw2),
                                                              (xp, w1, w3, w2))]
     assert max(errs) > 1e-3
+
+
+@pytest.mark.parametrize("score,renorm,scale", [("softmax", True, 1.0), ("softmax", False, 2.5),
+                                                ("sigmoid", True, 1.0), ("sigmoid", False, 0.7)])
+def test_router_backward_matches_finite_differences(score, renorm, scale):
+    """d(sum g * w)/d logits by central differences of the general router
+    (logits with gaps >= 1e-3 so the selection stays fixed under the
+    perturbation), one token at a time."""
+    T, E, k = 5, 9, 3
+    L = W.make_logits(T, E, k, seed=3)
+    rng = np.random.default_rng(4)
+    g = rng.standard_normal((T, k))
+    idx, w, _, _ = O.router_topk_general(k, logits=L, score=score, renormalize=renorm,
+                                         route_scale=scale)
+    dz = O.router_backward(L, idx, g, score=score, renormalize=renorm, route_scale=scale)
+    Lw = L.astype(np.float64).copy()
+
+    def loss():
+        i2, w2, _, _ = O.router_topk_general(k, logits=Lw, score=score, renormalize=renorm,
+                                             route_scale=scale)
+        assert np.array_equal(i2, idx)
+        return float(np.sum(g * w2))
+
+    np.testing.assert_allclose(dz, _fd(loss, Lw), atol=1e-8)
+
+
+def test_router_backward_gate_gradients_match_torch_autograd():
+    """dz, dw_router = dz^T x and dx = dz w_router against autograd of
+    softmax -> gather -> renormalise -> scale in fp64."""
+    T, E, k, d = 7, 6, 2, 5
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((T, d))
+    wr = rng.standard_normal((E, d))
+    g = rng.standard_normal((T, k))
+    idx, _, _, L = O.router_topk_general(k, x=x, w_router=wr, renormalize=True,
+                                         route_scale=1.5)
+    dz, dwr, dx = O.router_backward(L, idx, g, renormalize=True, route_scale=1.5, x=x,
+                                    w_router=wr)
+    tx = torch.tensor(x, requires_grad=True)
+    tw = torch.tensor(wr, requires_grad=True)
+    p = torch.softmax(tx @ tw.T, dim=1).gather(1, torch.tensor(idx))
+    (torch.sum(torch.tensor(g) * 1.5 * p / p.sum(1, keepdim=True))).backward()
+    np.testing.assert_allclose(dwr, tw.grad.numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dx, tx.grad.numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_router_backward_closed_forms():
+    """k = E with renormalisation: the weights are the softmax itself, whose
+    gradient sums to zero per token; top-1 renormalised: w = 1, no gradient."""
+    rng = np.random.default_rng(6)
+    L = rng.standard_normal((4, 5))
+    g = rng.standard_normal((4, 5))
+    idx = np.argsort(-L, axis=1)
+    dz = O.router_backward(L, idx, g, renormalize=True)
+    np.testing.assert_allclose(dz.sum(axis=1), 0.0, atol=1e-14)
+    dz1 = O.router_backward(L, idx[:, :1], g[:, :1], renormalize=True)
+    np.testing.assert_allclose(dz1, 0.0, atol=1e-15)
