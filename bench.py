@@ -15,9 +15,10 @@ weak scaling, no data-path collective).
 (a bounded token sample per step) and prints the same metric.
 
 ``--training`` times the training step instead (its own JSON line): the
-forward with the experts' training variant (which keeps G | U), then the
-backward of the combine, of the grouped SwiGLU (data and weight gradients)
-and of the dispatch, each stage bracketed by CUDA events.
+forward with the experts' training variant (which keeps G | U) and the
+router's logits, then the backward of the combine, of the grouped SwiGLU
+(data and weight gradients), of the router (logits, gate weight, its share
+of dx) and of the dispatch, each stage bracketed by CUDA events.
 """
 from __future__ import annotations
 
@@ -559,11 +560,11 @@ def run_ours(args, ws, rank, local):
 
 
 TRAIN_STAGES = ["router", "dispatch", "grouped_swiglu_train", "combine", "combine_backward",
-                "grouped_swiglu_backward", "dispatch_backward"]
+                "grouped_swiglu_backward", "router_backward", "dispatch_backward"]
 # kernels of ours per training step: router 2, dispatch 3 (histogram, scan,
 # scatter), training GEMMs 2, combine 1, combine backward 1, backward GEMMs 4,
-# dispatch backward 1
-TRAIN_LAUNCHES = 14
+# router backward 4 (scores, segment, two gate GEMMs), dispatch backward 1
+TRAIN_LAUNCHES = 18
 
 
 def run_training(args, ws, rank, local):
@@ -605,6 +606,11 @@ def run_training(args, ws, rank, local):
     bws = torch.empty(M.grouped_swiglu_backward_workspace_size(N, d, h, E, dt),
                       dtype=torch.uint8, device=dev)
     dx = torch.empty(T, d, dtype=bf, device=dev)
+    logits = torch.empty(T, E, dtype=torch.float32, device=dev)
+    dwr = torch.empty_like(wr)
+    dxr = torch.empty(T, d, dtype=bf, device=dev)
+    rbws = torch.empty(M.router_backward_workspace_size(T, d, E), dtype=torch.uint8, device=dev)
+    ropts = M.router_options(renormalize=cfg.renormalize)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
     def step(ev=None):
@@ -612,8 +618,8 @@ def run_training(args, ws, rank, local):
             if ev is not None:
                 ev[i].record(stream)
         mark(0)
-        M.moe_router_topk(x, wr, None, T, d, E, k, M.MOE_SCORE_SOFTMAX, cfg.renormalize, dt, None,
-                          idx, w, None, rws)
+        M.moe_router_topk(x, wr, None, T, d, E, k, M.MOE_SCORE_SOFTMAX, cfg.renormalize, dt,
+                          logits, idx, w, None, rws)
         mark(1)
         M.moe_dispatch(x, idx, T, d, E, k, dt, counts, offsets, src_row, dst_pos, x_perm, dws)
         mark(2)
@@ -626,8 +632,10 @@ def run_training(args, ws, rank, local):
         M.moe_grouped_swiglu_backward(x_perm, offsets, w1, w3, w2, h_act, gu, dy, N, d, h, E, dt,
                                       dxp, dw1, dw3, dw2, bws)
         mark(6)
-        M.moe_dispatch_backward(dxp, dst_pos, T, d, N, k, dt, dx)
+        M.moe_router_backward(logits, idx, dtw, x, wr, T, d, E, k, ropts, dt, None, dwr, dxr, rbws)
         mark(7)
+        M.moe_dispatch_backward(dxp, dst_pos, dxr, T, d, N, k, dt, dx)
+        mark(8)
 
     if args.profile:
         for _ in range(2):

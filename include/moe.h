@@ -372,8 +372,28 @@ MOE_API moe_status_t moe_combine(const void* y, const int32_t* dst_pos, const in
  * 16-byte vectors.
  *
  * moe_dispatch_backward -- gradient of x_perm = x[src_row] with respect to
- * x: dx[t] = sum_j dx_perm[dst_pos[t, j]] (fp32 sum over j in order, one
- * rounding): the unweighted combine.  Rules as moe_combine.
+ * x: dx[t] = dx_add[t] + sum_j dx_perm[dst_pos[t, j]] (fp32 sum over j in
+ * order, one rounding): the unweighted combine.  dx_add [T, d] or NULL (the
+ * router's share of dx, from moe_router_backward).  Rules as moe_combine.
+ *
+ * moe_router_backward -- gradient of the routing weights of
+ * moe_router_topk_ex with respect to the gate logits and the gate's inputs,
+ * for upstream gradients d_topk_w [T, k] and the experts the forward
+ * selected (topk_idx).  Selection has no gradient: the expert bias and the
+ * group masking only choose experts.  Per token, with s the scores
+ * (softmax or sigmoid of the saved fp32 logits [T, E], as opts->score), S
+ * the selected experts and c = opts->route_scale:
+ *   w_j = c s_j / sum_S s   (opts->renormalize)   or   w_j = c s_j
+ *   ds_j = c (g_j - sum_S g s / sum_S s) / sum_S s   or   ds_j = c g_j
+ *   (0 for experts outside S)
+ *   dz = s * (ds - <s, ds>)   (softmax)   or   dz = ds * s * (1 - s)  (sigmoid)
+ *   d_logits = dz (fp32, optional), dw_router = dz^T x [E, d] (optional),
+ *   dx = dz w_router [T, d] (optional)
+ * The gate products run on tcgen05 from dz rounded once to bf16, with fp32
+ * accumulation (bf16 x and w_router; dw_router and dx need dt = MOE_BF16
+ * and E % 8 == 0).  opts NULL = defaults (softmax, no renormalisation, scale
+ * 1).  E <= 512.  Workspace moe_router_backward_workspace_size (dz in bf16
+ * plus the status word).  Entries of topk_idx outside [0, E) are skipped.
  * ---------------------------------------------------------------------- */
 MOE_API moe_status_t moe_grouped_swiglu_train(const void* x_perm, const int32_t* offsets,
                                       const void* w1, const void* w3, const void* w2, int N,
@@ -391,9 +411,16 @@ MOE_API moe_status_t moe_combine_backward(const void* dout, const void* y,
                                   const int32_t* dst_pos, const float* topk_w, int T, int d,
                                   int N, int top_k, moe_dtype_t dt, void* dy, float* d_topk_w,
                                   void* stream);
-MOE_API moe_status_t moe_dispatch_backward(const void* dx_perm, const int32_t* dst_pos, int T,
-                                   int d, int N, int top_k, moe_dtype_t dt, void* dx,
-                                   void* stream);
+MOE_API moe_status_t moe_dispatch_backward(const void* dx_perm, const int32_t* dst_pos,
+                                   const void* dx_add, int T, int d, int N, int top_k,
+                                   moe_dtype_t dt, void* dx, void* stream);
+MOE_API size_t moe_router_backward_workspace_size(int T, int d, int E);
+MOE_API moe_status_t moe_router_backward(const float* logits, const int32_t* topk_idx,
+                                 const float* d_topk_w, const void* x, const void* w_router,
+                                 int T, int d, int E, int top_k,
+                                 const moe_router_options_t* opts, moe_dtype_t dt,
+                                 float* d_logits, void* dw_router, void* dx, void* ws,
+                                 size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
  * moe_forward -- [HP] MoE.forward with score_before_experts=False and no

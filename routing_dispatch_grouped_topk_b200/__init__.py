@@ -44,6 +44,7 @@ __all__ = [
     "moe_grouped_swiglu_train", "moe_grouped_swiglu_backward", "moe_combine_backward",
     "moe_dispatch_backward", "grouped_swiglu_backward_workspace_size",
     "grouped_swiglu_train", "grouped_swiglu_backward", "combine_backward", "dispatch_backward",
+    "moe_router_backward", "router_backward_workspace_size", "router_backward",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe.so")
@@ -62,6 +63,7 @@ EXPORTED_SYMBOLS = [
     "moe_combine",
     "moe_grouped_swiglu_train", "moe_grouped_swiglu_backward_workspace_size",
     "moe_grouped_swiglu_backward", "moe_combine_backward", "moe_dispatch_backward",
+    "moe_router_backward_workspace_size", "moe_router_backward",
     "moe_forward_workspace_size", "moe_forward", "moe_forward_ex_workspace_size",
     "moe_forward_ex", "moe_get_device_status", "moe_selftest_timeout", "moe_status_string",
     "moe_last_error", "moe_version",
@@ -126,7 +128,10 @@ _SIGS = {
     "moe_grouped_swiglu_backward": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P,
                                          _P, _P, _P, _P, _Z, _P]),
     "moe_combine_backward": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P]),
-    "moe_dispatch_backward": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P]),
+    "moe_dispatch_backward": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P]),
+    "moe_router_backward_workspace_size": (_Z, [_I, _I, _I]),
+    "moe_router_backward": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _I, _P, _P, _P, _P, _Z,
+                                 _P]),
     "moe_forward_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I, _I]),
     "moe_forward": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P,
                          _P, _P, _P, _Z, _P]),
@@ -364,10 +369,22 @@ def moe_combine_backward(dout, y, dst_pos, topk_w, T, d, N, top_k, dt, dy, d_top
         _ptr(d_topk_w, torch.float32, "d_topk_w"), _stream(stream)), "moe_combine_backward")
 
 
-def moe_dispatch_backward(dx_perm, dst_pos, T, d, N, top_k, dt, dx, stream=None):
+def moe_dispatch_backward(dx_perm, dst_pos, dx_add, T, d, N, top_k, dt, dx, stream=None):
     _check(lib().moe_dispatch_backward(
-        _ptr(dx_perm, name="dx_perm"), _ptr(dst_pos, torch.int32, "dst_pos"), T, d, N, top_k,
-        dt, _ptr(dx, name="dx"), _stream(stream)), "moe_dispatch_backward")
+        _ptr(dx_perm, name="dx_perm"), _ptr(dst_pos, torch.int32, "dst_pos"),
+        _ptr(dx_add, name="dx_add"), T, d, N, top_k, dt, _ptr(dx, name="dx"), _stream(stream)),
+        "moe_dispatch_backward")
+
+
+def moe_router_backward(logits, topk_idx, d_topk_w, x, w_router, T, d, E, top_k, opts, dt,
+                        d_logits, dw_router, dx, ws, stream=None):
+    _check(lib().moe_router_backward(
+        _ptr(logits, torch.float32, "logits"), _ptr(topk_idx, torch.int32, "topk_idx"),
+        _ptr(d_topk_w, torch.float32, "d_topk_w"), _ptr(x, name="x"),
+        _ptr(w_router, name="w_router"), T, d, E, top_k, _opts(opts), dt,
+        _ptr(d_logits, torch.float32, "d_logits"), _ptr(dw_router, name="dw_router"),
+        _ptr(dx, name="dx"), _ptr(ws, name="ws"), _nbytes(ws), _stream(stream)),
+        "moe_router_backward")
 
 
 def moe_forward(x, w_router, logits_in, w1, w3, w2, T, d, E, top_k, h, score, renormalize,
@@ -569,13 +586,38 @@ def combine_backward(dout, y, dst_pos, topk_w=None, want_dw=True):
     return dy, dw
 
 
-def dispatch_backward(dx_perm, dst_pos):
-    """dx [T, d]: every token's sum of its copies' gradients."""
+def dispatch_backward(dx_perm, dst_pos, dx_add=None):
+    """dx [T, d]: every token's sum of its copies' gradients (plus dx_add)."""
     T, k = dst_pos.shape
     N, d = dx_perm.shape
     dx = torch.empty(T, d, dtype=dx_perm.dtype, device=dx_perm.device)
-    moe_dispatch_backward(dx_perm, dst_pos, T, d, N, k, _dt(dx_perm), dx)
+    moe_dispatch_backward(dx_perm, dst_pos, dx_add, T, d, N, k, _dt(dx_perm), dx)
     return dx
+
+
+def router_backward_workspace_size(T, d, E) -> int:
+    return lib().moe_router_backward_workspace_size(T, d, E)
+
+
+def router_backward(logits, topk_idx, d_topk_w, x=None, w_router=None, want_d_logits=True,
+                    **options):
+    """Router backward.  Returns (d_logits fp32 [T, E] or None, dw_router
+    [E, d] or None, dx [T, d] or None, ws); the gate gradients are computed
+    when x / w_router are given.  ``options`` are router_options() keywords
+    (score, renormalize, route_scale)."""
+    T, E = logits.shape
+    k = topk_idx.shape[1]
+    dev = logits.device
+    d = x.shape[1] if x is not None else (w_router.shape[1] if w_router is not None else 8)
+    dt = _dt(x) if x is not None else (_dt(w_router) if w_router is not None else MOE_BF16)
+    dl = torch.empty(T, E, dtype=torch.float32, device=dev) if want_d_logits else None
+    dwr = torch.empty(E, d, dtype=x.dtype, device=dev) if x is not None else None
+    dx = torch.empty(T, d, dtype=w_router.dtype, device=dev) if w_router is not None else None
+    ws = _ws(router_backward_workspace_size(T, d, E), dev)
+    opts = router_options(**options)
+    moe_router_backward(logits, topk_idx, d_topk_w, x, w_router, T, d, E, k, opts, dt, dl, dwr,
+                        dx, ws)
+    return dl, dwr, dx, ws
 
 
 def forward(x, w_router, w1, w3, w2, top_k, renormalize=True, ep_ranks=1, logits_in=None,

@@ -671,9 +671,78 @@ moe_status_t moe_combine_backward(const void* dout, const void* y, const int32_t
                      "moe_combine_backward");
 }
 
-moe_status_t moe_dispatch_backward(const void* dx_perm, const int32_t* dst_pos, int T, int d,
-                                   int N, int top_k, moe_dtype_t dt, void* dx, void* stream) {
-  return moe_combine(dx_perm, dst_pos, nullptr, nullptr, T, d, N, top_k, dt, dx, stream);
+moe_status_t moe_dispatch_backward(const void* dx_perm, const int32_t* dst_pos,
+                                   const void* dx_add, int T, int d, int N, int top_k,
+                                   moe_dtype_t dt, void* dx, void* stream) {
+  if (moe_status_t st = check_dtype(dt)) return st;
+  MOE_CHECK_ARG(T >= 0 && N >= 0, "T, N must be >= 0");
+  MOE_CHECK_ARG(top_k >= 1 && top_k <= kMaxTopK, "top_k=%d out of range", top_k);
+  if (T > 0) {
+    MOE_CHECK_ARG(dx && dst_pos, "dx and dst_pos are required");
+    MOE_CHECK_ARG(N == 0 || dx_perm, "dx_perm is required");
+    MOE_CHECK_ARG(aligned16(dx) && aligned16(dx_perm) && aligned16(dx_add),
+                  "dx_perm / dx_add / dx must be 16-byte aligned");
+    if (moe_status_t st = check_rows(d, dt, "dispatch_backward")) return st;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return cuda_status(launch_combine(dx_perm, dst_pos, nullptr, nullptr, T, d, N, top_k, dt, dx, s,
+                                    dx_add),
+                     "moe_dispatch_backward");
+}
+
+size_t moe_router_backward_workspace_size(int T, int d, int E) {
+  (void)d;
+  if (T < 0 || E < 1) return kStatusBytes;
+  return kStatusBytes + 256 + align_up(static_cast<size_t>(T) * E * 2, 256);
+}
+
+moe_status_t moe_router_backward(const float* logits, const int32_t* topk_idx,
+                                 const float* d_topk_w, const void* x, const void* w_router,
+                                 int T, int d, int E, int top_k,
+                                 const moe_router_options_t* opts, moe_dtype_t dt,
+                                 float* d_logits, void* dw_router, void* dx, void* ws,
+                                 size_t ws_bytes, void* stream) {
+  const moe_router_options_t o = opts ? *opts : default_options();
+  if (moe_status_t st = check_dtype(dt)) return st;
+  MOE_CHECK_ARG(T >= 0 && d >= 1 && E >= 1 && E <= kMaxExperts, "bad sizes T=%d d=%d E=%d", T,
+                d, E);
+  MOE_CHECK_ARG(top_k >= 1 && top_k <= kMaxTopK && top_k <= E, "top_k=%d out of range", top_k);
+  MOE_CHECK_ARG(o.score == MOE_SCORE_SOFTMAX || o.score == MOE_SCORE_SIGMOID, "bad score");
+  MOE_CHECK_ARG(std::isfinite(o.route_scale) && o.route_scale != 0.0f, "bad route_scale");
+  const bool gemm = dw_router || dx;
+  if (gemm) {
+    if (dt != MOE_BF16 || E % 8 != 0 || d % 8 != 0) {
+      set_last_error("router backward gate gradients need bf16, E %% 8 == 0 and d %% 8 == 0");
+      return MOE_ERR_UNSUPPORTED;
+    }
+  }
+  if (T > 0) {
+    MOE_CHECK_ARG(logits && topk_idx && d_topk_w, "logits, topk_idx, d_topk_w required");
+    MOE_CHECK_ARG(!dw_router || x, "x is required for dw_router");
+    MOE_CHECK_ARG(!dx || w_router, "w_router is required for dx");
+    MOE_CHECK_ARG(aligned16(x) && aligned16(w_router) && aligned16(dw_router) && aligned16(dx),
+                  "x, w_router, dw_router, dx must be 16-byte aligned");
+  }
+  MOE_CHECK_ARG(ws != nullptr, "ws is required");
+  const size_t need = moe_router_backward_workspace_size(T, d, E);
+  if (ws_bytes < need) {
+    set_last_error("router_backward workspace %zu < %zu", ws_bytes, need);
+    return MOE_ERR_WORKSPACE;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* status = static_cast<int*>(ws);
+  int32_t* off2 = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + kStatusBytes);
+  void* dz16 = static_cast<char*>(ws) + kStatusBytes + 256;
+  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), s);
+  if (e == cudaSuccess && T == 0 && dw_router)
+    e = cudaMemsetAsync(dw_router, 0, static_cast<size_t>(E) * d * 2, s);
+  if (e == cudaSuccess && T > 0)
+    e = launch_router_backward(logits, topk_idx, d_topk_w, T, E, top_k,
+                               o.score == MOE_SCORE_SIGMOID, o.renormalize, o.route_scale,
+                               d_logits, gemm ? dz16 : nullptr, s);
+  if (e == cudaSuccess && T > 0 && gemm)
+    e = launch_gate_backward_tc(dz16, x, w_router, T, d, E, dw_router, dx, off2, status, s);
+  return cuda_status(e, "moe_router_backward");
 }
 
 // ------------------------------------------------------------------ forward

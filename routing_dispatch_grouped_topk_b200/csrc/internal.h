@@ -97,6 +97,19 @@ cudaError_t launch_combine(const void* y, const int32_t* dst_pos, const int32_t*
 cudaError_t launch_combine_backward(const void* dout, const void* y, const int32_t* dst_pos,
                                     const float* topk_w, int T, int d, int N, int top_k,
                                     moe_dtype_t dt, void* dy, float* d_topk_w, cudaStream_t s);
+// Router backward: dz = d(routing weights)/d(logits) applied to d_topk_w,
+// per token from the saved fp32 logits; dz32 [T, E] fp32 and dz16 [T, E]
+// bf16 are each optional.
+cudaError_t launch_router_backward(const float* logits, const int32_t* topk_idx,
+                                   const float* d_topk_w, int T, int E, int top_k, int sigmoid,
+                                   int renorm, float scale, float* dz32, void* dz16,
+                                   cudaStream_t s);
+// Gradients of the gate x . w_router^T for dz16 [T, E] bf16: dw_router =
+// dz^T x [E, d] and dx = dz w_router [T, d] (bf16, each optional); offsets2 is
+// device scratch for two ints.
+cudaError_t launch_gate_backward_tc(const void* dz16, const void* x, const void* w_router, int T,
+                                    int d, int E, void* dw_router, void* dx, int32_t* offsets2,
+                                    int* status, cudaStream_t s);
 // Self-test of the bounded wait: sets MOE_DEV_TIMEOUT after kWaitLimitNs.
 cudaError_t launch_selftest_timeout(int* status, cudaStream_t s);
 // offsets[0] = 0, offsets[1] = n: the segmentation of a single expert.

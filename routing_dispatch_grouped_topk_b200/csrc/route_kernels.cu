@@ -545,6 +545,126 @@ cudaError_t launch_combine(const void* y, const int32_t* dst_pos, const int32_t*
   return cudaGetLastError();
 }
 
+// -------------------------------------------------------- router backward
+// Gradient of the routing weights with respect to the gate logits, one warp
+// per token (expert i lives in lane i % 32, register slot i / 32).  With s
+// the scores (softmax or sigmoid of the saved fp32 logits), S the selected
+// experts and c the route scale: w_j = c s_j / sum_S s (renormalised) or
+// c s_j, so ds_j = c (g_j - sum_S g s / sum_S s) / sum_S s or c g_j on S,
+// 0 elsewhere; dz = s (ds - <s, ds>) (softmax) or ds s (1 - s) (sigmoid).
+// Writes dz in fp32 (dz32, optional) and bf16 (dz16, optional; the operand
+// of the gate's gradient GEMMs).
+template <int EPL>
+__global__ void __launch_bounds__(256) router_backward_kernel(
+    const float* __restrict__ logits, const int32_t* __restrict__ topk_idx,
+    const float* __restrict__ g_w, int T, int E, int k, int sigmoid, int renorm, float scale,
+    float* __restrict__ dz32, __nv_bfloat16* __restrict__ dz16) {
+  pdl_wait();
+  pdl_trigger();
+  const int lane = threadIdx.x & 31;
+  const int nwarps = (gridDim.x * blockDim.x) >> 5;
+  for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += nwarps) {
+    const float* row = logits + static_cast<size_t>(t) * E;
+    float sv[EPL];
+    bool avail[EPL];
+    float mx = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      avail[i] = lane + 32 * i < E;
+      sv[i] = avail[i] ? row[lane + 32 * i] : -INFINITY;
+      mx = fmaxf(mx, sv[i]);
+    }
+    if (sigmoid) {
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) sv[i] = avail[i] ? 1.0f / (1.0f + expf(-sv[i])) : 0.f;
+    } else {
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+      float den = 0.f;
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) {
+        sv[i] = avail[i] ? expf(sv[i] - mx) : 0.f;
+        den += sv[i];
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) sv[i] /= den;
+    }
+    // lane j < k: the j-th selected expert, its upstream gradient and score
+    int my_e = -1;
+    float my_g = 0.f;
+    if (lane < k) {
+      const int e = topk_idx[static_cast<size_t>(t) * k + lane];
+      if (static_cast<unsigned>(e) < static_cast<unsigned>(E)) {
+        my_e = e;
+        my_g = g_w[static_cast<size_t>(t) * k + lane];
+      }
+    }
+    float my_s = 0.f;
+    for (int j = 0; j < k; ++j) {
+      const int ej = __shfl_sync(0xffffffffu, my_e, j);
+      float v = 0.f;
+#pragma unroll
+      for (int i = 0; i < EPL; ++i)
+        if (i == (ej >> 5)) v = sv[i];
+      v = __shfl_sync(0xffffffffu, v, ej & 31);
+      if (lane == j) my_s = ej >= 0 ? v : 0.f;
+    }
+    float tot = my_s, gs = my_g * my_s;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      tot += __shfl_xor_sync(0xffffffffu, tot, off);
+      gs += __shfl_xor_sync(0xffffffffu, gs, off);
+    }
+    const float my_ds = my_e < 0 ? 0.f : (renorm ? scale * (my_g - gs / tot) / tot : scale * my_g);
+    float ds[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) ds[i] = 0.f;
+    for (int j = 0; j < k; ++j) {
+      const int ej = __shfl_sync(0xffffffffu, my_e, j);
+      const float dj = __shfl_sync(0xffffffffu, my_ds, j);
+#pragma unroll
+      for (int i = 0; i < EPL; ++i)
+        if (lane + 32 * i == ej) ds[i] = dj;
+    }
+    float c = 0.f;
+    if (!sigmoid) {
+      c = my_s * my_ds;   // <s, ds> over the selected experts
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) c += __shfl_xor_sync(0xffffffffu, c, off);
+    }
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      if (!avail[i]) continue;
+      const float dz = sigmoid ? ds[i] * sv[i] * (1.0f - sv[i]) : sv[i] * (ds[i] - c);
+      const size_t o = static_cast<size_t>(t) * E + lane + 32 * i;
+      if (dz32) dz32[o] = dz;
+      if (dz16) dz16[o] = __float2bfloat16_rn(dz);
+    }
+  }
+}
+
+cudaError_t launch_router_backward(const float* logits, const int32_t* topk_idx,
+                                   const float* d_topk_w, int T, int E, int top_k, int sigmoid,
+                                   int renorm, float scale, float* dz32, void* dz16,
+                                   cudaStream_t s) {
+  if (T == 0) return cudaSuccess;
+  const int blocks = std::min(cdiv(T, 8), num_sms() * 8);
+  __nv_bfloat16* d16 = static_cast<__nv_bfloat16*>(dz16);
+  if (E <= 32)
+    launch_k(router_backward_kernel<1>, dim3(blocks), dim3(256), 0, s, logits, topk_idx, d_topk_w, T, E, top_k, sigmoid, renorm, scale, dz32, d16);
+  else if (E <= 64)
+    launch_k(router_backward_kernel<2>, dim3(blocks), dim3(256), 0, s, logits, topk_idx, d_topk_w, T, E, top_k, sigmoid, renorm, scale, dz32, d16);
+  else if (E <= 128)
+    launch_k(router_backward_kernel<4>, dim3(blocks), dim3(256), 0, s, logits, topk_idx, d_topk_w, T, E, top_k, sigmoid, renorm, scale, dz32, d16);
+  else if (E <= 256)
+    launch_k(router_backward_kernel<8>, dim3(blocks), dim3(256), 0, s, logits, topk_idx, d_topk_w, T, E, top_k, sigmoid, renorm, scale, dz32, d16);
+  else
+    launch_k(router_backward_kernel<16>, dim3(blocks), dim3(256), 0, s, logits, topk_idx, d_topk_w, T, E, top_k, sigmoid, renorm, scale, dz32, d16);
+  return cudaGetLastError();
+}
+
 // ------------------------------------------------------- combine backward
 // Gradient of out[t] = sum_j w[t, j] y[p(t, j)] for an upstream dout [T, d]:
 // dy[p(t, j)] = w[t, j] dout[t] (one rounding of the fp32 product) and, when

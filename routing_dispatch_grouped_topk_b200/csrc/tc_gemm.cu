@@ -658,6 +658,38 @@ struct UpBwdPolicy : GroupedSched<256, 2, 256> {
   static __device__ void finish(const Args&, int*) {}
 };
 
+// Data gradient through one untransposed weight: out [M, n_out] = A B with
+// A [M, K] K-major and B [K, n_out] (K rows, MN-major), one segment.  Used
+// for the gate: dx = dz . w_router (K = E).
+struct DgradPolicy : GroupedSched<256, 1, 256> {
+  static constexpr bool B_MN = true, CUSTOM_LOADS = true;
+  static __device__ TileInfo tile_info(const Args& a, const int* sched, int tile) {
+    int e, nt, mt, cnt, seg0;
+    locate(a, sched, tile, e, nt, mt, cnt, seg0);
+    TileInfo t;
+    t.a_row = seg0 + mt * BM;
+    t.m_valid = min(BM, cnt - mt * BM);
+    t.n0 = nt * 256;
+    t.b_row = e * a.K;
+    t.kb0 = 0;
+    t.kb1 = cdiv(a.K, BK);
+    t.swap_np = 0;
+    t.m0 = 0;
+    return t;
+  }
+  static __device__ void issue_loads(const Args& a, const CUtensorMap* tmA,
+                                     const CUtensorMap* tmB0, const CUtensorMap* tmB1,
+                                     const TileInfo& ti, int kb, uint8_t* sa, uint8_t* sb,
+                                     uint64_t* bar, uint64_t pa, uint64_t pb) {
+    DownBwdPolicy::issue_loads(a, tmA, tmB0, tmB1, ti, kb, sa, sb, bar, pa, pb);
+  }
+  static __device__ void epilogue(const Args& a, int* s, const TileInfo& ti, uint32_t taddr,
+                                  int row) {
+    DownPolicy::epilogue(a, s, ti, taddr, row);   // plain bf16 rows (row_scale is null)
+  }
+  static __device__ void finish(const Args&, int*) {}
+};
+
 // Weight gradients: out[e] = A_e^T B_e over the rows of segment e, with
 // A [N, Ma] and B [N, n_out] both MN-major (their columns are the output's
 // rows and columns).  Tiles are (expert, 128 output rows, 256 output
@@ -1653,6 +1685,49 @@ cudaError_t launch_swiglu_bwd_tc(const void* x_perm, const int32_t* offsets, con
   a.out1 = static_cast<__nv_bfloat16*>(dW3);
   grid = static_cast<int>(std::min<long long>(num_sms(), 1LL * E * cdiv(2 * h, BM) * cdiv(d, 256)));
   return launch<WgradPolicy>(m_dgu, m_x, m_x, a, grid, s);
+}
+
+// Gradients of the gate logits = x . w_router^T for dz16 [T, E] (bf16):
+//   dw_router = dz^T x   (WgradPolicy over one segment of T rows)
+//   dx        = dz w_router (DgradPolicy, K = E)
+cudaError_t launch_gate_backward_tc(const void* dz16, const void* x, const void* w_router, int T,
+                                    int d, int E, void* dw_router, void* dx, int32_t* offsets2,
+                                    int* status, cudaStream_t s) {
+  using namespace tc;
+  if (T == 0) return cudaSuccess;
+  cudaError_t e = launch_single_segment(offsets2, T, s);
+  if (e != cudaSuccess) return e;
+  Args a{};
+  a.M = T;
+  a.E = 1;
+  a.offsets = offsets2;
+  a.status = status;
+  if (dw_router) {
+    CUtensorMap m_dz, m_x;
+    if (!make_tmap(&m_dz, dz16, E, T, 64)) return cudaErrorInvalidValue;
+    if (!make_tmap(&m_x, x, d, T, 64)) return cudaErrorInvalidValue;
+    a.Ma = E;
+    a.split = E;
+    a.n_out = d;
+    a.out = static_cast<__nv_bfloat16*>(dw_router);
+    a.out1 = nullptr;
+    const int grid = std::min(num_sms(), cdiv(E, BM) * cdiv(d, 256));
+    e = launch<WgradPolicy>(m_dz, m_x, m_x, a, grid, s);
+    if (e != cudaSuccess) return e;
+  }
+  if (dx) {
+    CUtensorMap t_dz, t_wr;
+    if (!make_tmap(&t_dz, dz16, E, T, BM)) return cudaErrorInvalidValue;
+    if (!make_tmap(&t_wr, w_router, d, E, 64)) return cudaErrorInvalidValue;
+    a.K = E;
+    a.n_out = d;
+    a.out = static_cast<__nv_bfloat16*>(dx);
+    a.out1 = nullptr;
+    a.row_scale = nullptr;
+    const int grid = std::min(num_sms(), cdiv(T, BM) * cdiv(d, 256));
+    e = launch<DgradPolicy>(t_dz, t_wr, t_wr, a, grid, s);
+  }
+  return e;
 }
 
 }  // namespace moe

@@ -280,3 +280,91 @@ def test_training_chain_full_size_sampled(M, cfg_index):
     mag = np.einsum("td,tjd->tj", np.abs(gg), np.abs(yy))
     assert np.all(np.abs(f64(dtw[torch.as_tensor(toks, device="cuda").long()]) - ref_dtw)
                   <= 1.01 * d * 2.0 ** -24 * mag + 1e-30)
+
+
+# ----------------------------------------------------------- router backward
+ROUTER_BWD = [("softmax", True, 1.0), ("softmax", False, 2.5), ("sigmoid", True, 1.0),
+              ("sigmoid", False, 0.7)]
+
+
+@pytest.mark.parametrize("score,renorm,scale", ROUTER_BWD)
+@pytest.mark.parametrize("T,E,k,d", [(300, 128, 8, 256), (77, 72, 4, 192), (33, 8, 2, 64)])
+def test_router_backward_matches_oracle(M, score, renorm, scale, T, E, k, d):
+    """d_logits (fp32) within 2e-5 of the row's largest entry; dw_router and
+    the router's dx (bf16, from dz rounded once to bf16) within the
+    RMS-relative bound of sums over mixed-sign terms."""
+    L = W.make_logits(T, E, k, seed=T + E)
+    idx, w, _, _ = O.router_topk_general(k, logits=L, score=score, renormalize=renorm,
+                                         route_scale=scale)
+    g = torch.Generator().manual_seed(E)
+    gw = torch.randn(T, k, generator=g)
+    x = torch.randn(T, d, generator=g).to(torch.bfloat16)
+    wr = (torch.randn(E, d, generator=g) * 0.05).to(torch.bfloat16)
+    dl, dwr, dx, ws = M.router_backward(torch.from_numpy(L).float().cuda(), i32(idx), gw.cuda(),
+                                        x.cuda(), wr.cuda(), score=score, renormalize=renorm,
+                                        route_scale=scale)
+    torch.cuda.synchronize()
+    assert M.device_status(ws) == 0
+    rdz, rdwr, rdx = O.router_backward(L.astype(np.float32), idx, gw, score=score,
+                                       renormalize=renorm, route_scale=scale, x=x, w_router=wr)
+    err = np.abs(f64(dl) - rdz)
+    rowmax = np.abs(rdz).max(axis=1, keepdims=True)
+    assert np.all(err <= 2e-5 * (np.abs(rdz) + rowmax) + 1e-30), err.max()
+    close_wgrad(dwr, rdwr)
+    close_wgrad(dx, rdx)
+
+
+def test_router_backward_without_gate_gradients(M):
+    T, E, k = 50, 16, 2
+    L = W.make_logits(T, E, k, seed=1)
+    idx, _, _, _ = O.router_topk(k, True, logits=L)
+    gw = torch.randn(T, k)
+    dl, dwr, dx, ws = M.router_backward(torch.from_numpy(L).float().cuda(), i32(idx), gw.cuda(),
+                                        renormalize=True)
+    assert dwr is None and dx is None
+    rdz = O.router_backward(L.astype(np.float32), idx, gw, renormalize=True)
+    assert np.allclose(f64(dl), rdz, atol=2e-6)
+
+
+def test_layer_backward_full_size_sampled_tokens(M):
+    """The whole layer's input gradient at the Qwen3-30B-A3B sizes (T=4096):
+    router (logits kept) -> dispatch -> training forward -> combine, then
+    combine backward -> experts backward -> router backward -> dispatch
+    backward with the router's dx added.  Sampled tokens' dx against the
+    oracle (experts' share row by row, router's share from the oracle's
+    router backward on the GPU's logits)."""
+    cfg = W.config(1)
+    lay = W.make_layer(cfg, device="cuda")
+    x, wr, w1, w3, w2 = (lay[n] for n in ("x", "w_router", "w1", "w3", "w2"))
+    T, d, E, k, h = cfg.T, cfg.d, cfg.E, cfg.top_k, cfg.h
+    idx, tw, counts, logits, _ = M.router_topk(x, wr, k, True, want_logits=True)
+    cnt, off, src, dst, xp, _ = M.dispatch(x, idx, E)
+    y, h_act, gu, _ = M.grouped_swiglu_train(xp, off, w1, w3, w2)
+    g = torch.Generator(device="cuda").manual_seed(3)
+    dout = torch.randn(T, d, generator=g, device="cuda").to(torch.bfloat16)
+    dy, dtw = M.combine_backward(dout, y, dst, tw)
+    dxp, _, _, _, ws = M.grouped_swiglu_backward(xp, off, w1, w3, w2, h_act, gu, dy)
+    dl, dwr, dxr, rws = M.router_backward(logits, idx, dtw, x, wr, renormalize=True)
+    dx = M.dispatch_backward(dxp, dst, dxr)
+    torch.cuda.synchronize()
+    assert M.device_status(ws) == 0 and M.device_status(rws) == 0
+    rng = np.random.default_rng(11)
+    toks = np.sort(rng.choice(T, 8, replace=False))
+    tt = torch.as_tensor(toks, device="cuda").long()
+    # router share for the sampled tokens, from the GPU's logits and dtw
+    rdz, _, rdxr = O.router_backward(logits[tt].cpu(), idx[tt].cpu(), dtw[tt].cpu(),
+                                     renormalize=True, x=x[tt].cpu(), w_router=wr.cpu())
+    # experts' share: dx_perm rows are row-local
+    dst_h = dst.cpu().numpy()
+    idx_h = idx.cpu().numpy()
+    ref = rdxr.copy()
+    for a, t in enumerate(toks):
+        for j in range(k):
+            r = int(dst_h[t, j])
+            e = int(idx_h[t, j])
+            rr = torch.tensor([r], device="cuda")
+            rdx1, _, _, _ = O.grouped_swiglu_backward(
+                xp[rr].cpu(), np.array([0, 1]), w1[e:e + 1].cpu(), w3[e:e + 1].cpu(),
+                w2[e:e + 1].cpu(), dy[rr].cpu())
+            ref[a] += rdx1[0]
+    close(dx[tt], ref)
