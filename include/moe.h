@@ -423,6 +423,47 @@ MOE_API moe_status_t moe_router_backward(const float* logits, const int32_t* top
                                  size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * moe_forward_train / moe_backward -- the whole layer's training step in two
+ * calls ([HP] MoE.forward trained under autograd).
+ *
+ * moe_forward_train computes `out` exactly as moe_forward (ep_ranks = 1, no
+ * shared expert) and keeps in `state` (caller-owned, opaque, sized by
+ * moe_train_state_size) what the backward needs: the router's fp32 logits,
+ * the routing, the dispatch layout, x_perm, the experts' outputs, H and G | U.
+ * The state must stay untouched until moe_backward has run on the stream.
+ * logits_in (as moe_forward) replaces the gate; the state then keeps a copy.
+ *
+ * moe_backward, for an upstream gradient dout [T, d] of `out`, runs the
+ * chain rule through every step (the entry points of the training path
+ * above, in order: combine, experts, router, dispatch) and writes
+ *   dw1, dw3 [E, h, d], dw2 [E, d, h]         the expert weight gradients
+ *   dw_router [E, d] (NULL: not computed)      the gate's weight gradient
+ *   dx [T, d]                                  the input gradient: the sum of
+ *      each token's copies' gradients, plus the router's share dz w_router
+ *      when dw_router is computed (a gate driven by logits_in has neither)
+ *   d_logits [T, E] fp32 (NULL: not written)   the logits' gradient dz
+ * `opts` must be the options of the forward (score, renormalize, route_scale
+ * enter the router's derivative; bias and groups only selected).  bf16 only;
+ * d % 64 == 0, h % 64 == 0, E % 8 == 0; score_before_experts is rejected
+ * (MOE_ERR_UNSUPPORTED).  Workspace: moe_backward_workspace_size.  Device
+ * errors: the status word of `state` (forward) and of `ws` (backward).
+ * ---------------------------------------------------------------------- */
+MOE_API size_t moe_train_state_size(int T, int d, int E, int top_k, int h);
+MOE_API moe_status_t moe_forward_train(const void* x, const void* w_router,
+                                       const float* logits_in, const void* w1, const void* w3,
+                                       const void* w2, int T, int d, int E, int top_k, int h,
+                                       const moe_router_options_t* opts, moe_dtype_t dt,
+                                       void* out, void* state, size_t state_bytes,
+                                       void* stream);
+MOE_API size_t moe_backward_workspace_size(int T, int d, int E, int top_k, int h);
+MOE_API moe_status_t moe_backward(const void* dout, const void* x, const void* w_router,
+                                  const void* w1, const void* w3, const void* w2, int T, int d,
+                                  int E, int top_k, int h, const moe_router_options_t* opts,
+                                  moe_dtype_t dt, const void* state, void* dx, float* d_logits,
+                                  void* dw_router, void* dw1, void* dw3, void* dw2, void* ws,
+                                  size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * moe_forward -- [HP] MoE.forward with score_before_experts=False and no
  * shared expert: router -> dispatch -> grouped SwiGLU -> combine.
  * With ep_ranks R > 1 the routed rows are laid out as R simulated EP ranks

@@ -45,6 +45,8 @@ __all__ = [
     "moe_dispatch_backward", "grouped_swiglu_backward_workspace_size",
     "grouped_swiglu_train", "grouped_swiglu_backward", "combine_backward", "dispatch_backward",
     "moe_router_backward", "router_backward_workspace_size", "router_backward",
+    "moe_train_state_size", "moe_forward_train", "moe_backward_workspace_size", "moe_backward",
+    "forward_train", "backward",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe.so")
@@ -64,6 +66,7 @@ EXPORTED_SYMBOLS = [
     "moe_grouped_swiglu_train", "moe_grouped_swiglu_backward_workspace_size",
     "moe_grouped_swiglu_backward", "moe_combine_backward", "moe_dispatch_backward",
     "moe_router_backward_workspace_size", "moe_router_backward",
+    "moe_train_state_size", "moe_forward_train", "moe_backward_workspace_size", "moe_backward",
     "moe_forward_workspace_size", "moe_forward", "moe_forward_ex_workspace_size",
     "moe_forward_ex", "moe_get_device_status", "moe_selftest_timeout", "moe_status_string",
     "moe_last_error", "moe_version",
@@ -130,6 +133,12 @@ _SIGS = {
     "moe_combine_backward": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P]),
     "moe_dispatch_backward": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P]),
     "moe_router_backward_workspace_size": (_Z, [_I, _I, _I]),
+    "moe_train_state_size": (_Z, [_I, _I, _I, _I, _I]),
+    "moe_forward_train": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _I, _P, _P, _Z,
+                               _P]),
+    "moe_backward_workspace_size": (_Z, [_I, _I, _I, _I, _I]),
+    "moe_backward": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _I, _P, _P, _P, _P, _P,
+                          _P, _P, _P, _Z, _P]),
     "moe_router_backward": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _I, _P, _P, _P, _P, _Z,
                                  _P]),
     "moe_forward_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I, _I]),
@@ -387,6 +396,26 @@ def moe_router_backward(logits, topk_idx, d_topk_w, x, w_router, T, d, E, top_k,
         "moe_router_backward")
 
 
+def moe_forward_train(x, w_router, logits_in, w1, w3, w2, T, d, E, top_k, h, opts, dt, out,
+                      state, stream=None):
+    _check(lib().moe_forward_train(
+        _ptr(x, name="x"), _ptr(w_router, name="w_router"),
+        _ptr(logits_in, torch.float32, "logits_in"), _ptr(w1, name="w1"), _ptr(w3, name="w3"),
+        _ptr(w2, name="w2"), T, d, E, top_k, h, _opts(opts), dt, _ptr(out, name="out"),
+        _ptr(state, name="state"), _nbytes(state), _stream(stream)), "moe_forward_train")
+
+
+def moe_backward(dout, x, w_router, w1, w3, w2, T, d, E, top_k, h, opts, dt, state, dx,
+                 d_logits, dw_router, dw1, dw3, dw2, ws, stream=None):
+    _check(lib().moe_backward(
+        _ptr(dout, name="dout"), _ptr(x, name="x"), _ptr(w_router, name="w_router"),
+        _ptr(w1, name="w1"), _ptr(w3, name="w3"), _ptr(w2, name="w2"), T, d, E, top_k, h,
+        _opts(opts), dt, _ptr(state, name="state"), _ptr(dx, name="dx"),
+        _ptr(d_logits, torch.float32, "d_logits"), _ptr(dw_router, name="dw_router"),
+        _ptr(dw1, name="dw1"), _ptr(dw3, name="dw3"), _ptr(dw2, name="dw2"),
+        _ptr(ws, name="ws"), _nbytes(ws), _stream(stream)), "moe_backward")
+
+
 def moe_forward(x, w_router, logits_in, w1, w3, w2, T, d, E, top_k, h, score, renormalize,
                 ep_ranks, dt, out, logits_out, topk_idx, topk_w, counts, ws, stream=None):
     _check(lib().moe_forward(
@@ -618,6 +647,39 @@ def router_backward(logits, topk_idx, d_topk_w, x=None, w_router=None, want_d_lo
     moe_router_backward(logits, topk_idx, d_topk_w, x, w_router, T, d, E, k, opts, dt, dl, dwr,
                         dx, ws)
     return dl, dwr, dx, ws
+
+
+def forward_train(x, w_router, w1, w3, w2, top_k, renormalize=True, logits_in=None, **options):
+    """Training forward of the whole layer.  Returns (out [T, d], state), the
+    state to hand to :func:`backward` (it records the sizes and options)."""
+    T, d = x.shape
+    E, h, _ = w1.shape
+    st = _ws(lib().moe_train_state_size(T, d, E, top_k, h), x.device)
+    out = torch.empty(T, d, dtype=x.dtype, device=x.device)
+    opts = router_options(renormalize=renormalize, **options)
+    moe_forward_train(x, w_router, logits_in, w1, w3, w2, T, d, E, top_k, h, opts, _dt(x), out,
+                      st)
+    state = {"state": st, "T": T, "d": d, "E": E, "k": top_k, "h": h,
+             "options": dict(options, renormalize=renormalize)}
+    return out, state
+
+
+def backward(state, dout, x, w_router, w1, w3, w2, router_grads=True, want_d_logits=False):
+    """Backward of the whole layer for dout [T, d].  Returns a dict with dx,
+    dw1, dw3, dw2, dw_router (None unless router_grads), d_logits (None
+    unless asked) and ws."""
+    T, d, E, k, h = (state[n] for n in ("T", "d", "E", "k", "h"))
+    dev = dout.device
+    dx = torch.empty(T, d, dtype=dout.dtype, device=dev)
+    dw1, dw3, dw2 = torch.empty_like(w1), torch.empty_like(w3), torch.empty_like(w2)
+    dwr = torch.empty_like(w_router) if router_grads else None
+    dl = torch.empty(T, E, dtype=torch.float32, device=dev) if want_d_logits else None
+    ws = _ws(lib().moe_backward_workspace_size(T, d, E, k, h), dev)
+    opts = router_options(**state["options"])
+    moe_backward(dout, x, w_router, w1, w3, w2, T, d, E, k, h, opts, _dt(dout), state["state"],
+                 dx, dl, dwr, dw1, dw3, dw2, ws)
+    return {"dx": dx, "dw1": dw1, "dw3": dw3, "dw2": dw2, "dw_router": dwr, "d_logits": dl,
+            "ws": ws}
 
 
 def forward(x, w_router, w1, w3, w2, top_k, renormalize=True, ep_ranks=1, logits_in=None,

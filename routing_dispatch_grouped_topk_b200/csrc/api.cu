@@ -297,6 +297,99 @@ ForwardWs carve_forward(void* ws, int T, int d, int E, int k, int h, int R, moe_
   return f;
 }
 
+// State a training forward keeps for its backward (caller-owned, opaque).
+struct TrainState {
+  int* status;
+  float* logits;       // [T, E] fp32
+  int32_t* idx;        // [T, k]
+  float* w;            // [T, k]
+  int32_t* counts;     // [E]
+  int32_t* offsets;    // [E + 1]
+  int32_t* src_row;    // [N]
+  int32_t* dst_pos;    // [T, k]
+  void* router_scratch;
+  void* disp_ws;
+  void* x_perm;        // [N, d]
+  void* y;             // [N, d]
+  void* H;             // [N, h]
+  void* GU;            // [N, 2h]
+  size_t bytes;
+};
+
+TrainState carve_train(void* base, int T, int d, int E, int k, int h) {
+  TrainState t{};
+  Carve c(base);
+  const size_t N = static_cast<size_t>(T) * k;
+  t.status = c.take<int>(kStatusBytes / sizeof(int));
+  t.logits = c.take<float>(static_cast<size_t>(T) * E);
+  t.idx = c.take<int32_t>(N);
+  t.w = c.take<float>(N);
+  const DispatchPlan p = make_dispatch_plan(T, E, k, 1);
+  t.counts = c.take<int32_t>(E);
+  t.offsets = c.take<int32_t>(static_cast<size_t>(E) + 1);
+  t.src_row = c.take<int32_t>(N);
+  t.dst_pos = c.take<int32_t>(N);
+  t.router_scratch = c.take<char>(router_ws(T, d, E, MOE_BF16) - kStatusBytes);
+  t.disp_ws = c.take<char>(dispatch_ws_bytes(p));
+  t.x_perm = c.take<char>(N * d * 2);
+  t.y = c.take<char>(N * d * 2);
+  t.H = c.take<char>(N * h * 2);
+  t.GU = c.take<char>(N * 2 * h * 2);
+  t.bytes = c.off;
+  return t;
+}
+
+// Backward workspace of moe_backward.
+struct BackwardWs {
+  int* status;
+  int32_t* off2;       // one-segment offsets of the gate's weight gradient
+  void* dY;            // [N, d]
+  float* dtw;          // [T, k]
+  void* dXp;           // [N, d]
+  void* dGU;           // [N, 2h]
+  void* dz16;          // [T, E]
+  void* dxr;           // [T, d] the router's share of dx
+  size_t bytes;
+};
+
+BackwardWs carve_backward(void* base, int T, int d, int E, int k, int h) {
+  BackwardWs b{};
+  Carve c(base);
+  const size_t N = static_cast<size_t>(T) * k;
+  b.status = c.take<int>(kStatusBytes / sizeof(int));
+  b.off2 = c.take<int32_t>(2);
+  b.dY = c.take<char>(N * d * 2);
+  b.dtw = c.take<float>(N);
+  b.dXp = c.take<char>(N * d * 2);
+  b.dGU = c.take<char>(N * 2 * h * 2);
+  b.dz16 = c.take<char>(static_cast<size_t>(T) * E * 2);
+  b.dxr = c.take<char>(static_cast<size_t>(T) * d * 2);
+  b.bytes = c.off;
+  return b;
+}
+
+// Shape and option rules of the whole-layer training entry points.
+moe_status_t check_train(int T, int d, int E, int top_k, int h, const moe_router_options_t& o,
+                         moe_dtype_t dt) {
+  if (dt != MOE_BF16) {
+    set_last_error("training entry points: bf16 only");
+    return MOE_ERR_UNSUPPORTED;
+  }
+  MOE_CHECK_ARG(T >= 0 && E >= 1 && E <= kMaxExperts && top_k >= 1 && top_k <= kMaxTopK &&
+                    top_k <= E,
+                "bad sizes T=%d E=%d top_k=%d", T, E, top_k);
+  if (moe_status_t st = check_swiglu_shape(T * top_k, d, h, E, dt)) return st;
+  if (E % 8 != 0) {
+    set_last_error("training entry points need E %% 8 == 0 (E=%d)", E);
+    return MOE_ERR_UNSUPPORTED;
+  }
+  if (o.score_before_experts) {
+    set_last_error("training entry points: score_before_experts has no backward here");
+    return MOE_ERR_UNSUPPORTED;
+  }
+  return MOE_OK;
+}
+
 }  // namespace
 }  // namespace moe
 
@@ -743,6 +836,118 @@ moe_status_t moe_router_backward(const float* logits, const int32_t* topk_idx,
   if (e == cudaSuccess && T > 0 && gemm)
     e = launch_gate_backward_tc(dz16, x, w_router, T, d, E, dw_router, dx, off2, status, s);
   return cuda_status(e, "moe_router_backward");
+}
+
+// ---------------------------------------------------- whole-layer training
+size_t moe_train_state_size(int T, int d, int E, int top_k, int h) {
+  if (T < 0 || d < 1 || E < 1 || top_k < 1 || h < 1) return kStatusBytes;
+  return carve_train(nullptr, T, d, E, top_k, h).bytes;
+}
+
+size_t moe_backward_workspace_size(int T, int d, int E, int top_k, int h) {
+  if (T < 0 || d < 1 || E < 1 || top_k < 1 || h < 1) return kStatusBytes;
+  return carve_backward(nullptr, T, d, E, top_k, h).bytes;
+}
+
+moe_status_t moe_forward_train(const void* x, const void* w_router, const float* logits_in,
+                               const void* w1, const void* w3, const void* w2, int T, int d,
+                               int E, int top_k, int h, const moe_router_options_t* opts,
+                               moe_dtype_t dt, void* out, void* state, size_t state_bytes,
+                               void* stream) {
+  const moe_router_options_t o = opts ? *opts : default_options();
+  if (moe_status_t st = check_train(T, d, E, top_k, h, o, dt)) return st;
+  if (moe_status_t st = check_router(x, w_router, logits_in, T, d, E, top_k, o, dt,
+                                     reinterpret_cast<int32_t*>(1), reinterpret_cast<float*>(1)))
+    return st;
+  if (T > 0) {
+    MOE_CHECK_ARG(x && w1 && w3 && w2 && out, "x, w1, w3, w2, out are required");
+    MOE_CHECK_ARG(aligned16(x) && aligned16(w1) && aligned16(w3) && aligned16(w2) &&
+                      aligned16(out),
+                  "x, w1, w3, w2, out must be 16-byte aligned");
+  }
+  MOE_CHECK_ARG(state != nullptr, "state is required");
+  const TrainState need = carve_train(nullptr, T, d, E, top_k, h);
+  if (state_bytes < need.bytes) {
+    set_last_error("training state %zu < %zu", state_bytes, need.bytes);
+    return MOE_ERR_WORKSPACE;
+  }
+  const TrainState t = carve_train(state, T, d, E, top_k, h);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int N = T * top_k;
+  const DispatchPlan p = make_dispatch_plan(T, E, top_k, 1);
+  cudaError_t e = cudaMemsetAsync(t.status, 0, sizeof(int), s);
+  if (e == cudaSuccess)
+    e = run_router(x, w_router, logits_in, T, d, E, top_k, o, dt, t.logits, t.idx, t.w, nullptr,
+                   t.router_scratch, t.status, s, &p, static_cast<int32_t*>(t.disp_ws));
+  if (e == cudaSuccess && logits_in && T > 0)   // the backward reads the logits from the state
+    e = cudaMemcpyAsync(t.logits, logits_in, static_cast<size_t>(T) * E * sizeof(float),
+                        cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess)
+    e = launch_dispatch(p, x, t.idx, d, dt, t.counts, t.offsets, t.src_row, t.dst_pos, t.x_perm,
+                        t.disp_ws, t.status, s, /*hist_done=*/T > 0);
+  if (e == cudaSuccess && N > 0)
+    e = launch_swiglu_tc_train(t.x_perm, t.offsets, w1, w3, w2, N, d, h, E, t.y, t.H, t.GU,
+                               t.status, s);
+  if (e == cudaSuccess)
+    e = launch_combine(t.y, t.dst_pos, nullptr, t.w, T, d, N, top_k, dt, out, s);
+  return cuda_status(e, "moe_forward_train");
+}
+
+moe_status_t moe_backward(const void* dout, const void* x, const void* w_router, const void* w1,
+                          const void* w3, const void* w2, int T, int d, int E, int top_k, int h,
+                          const moe_router_options_t* opts, moe_dtype_t dt, const void* state,
+                          void* dx, float* d_logits, void* dw_router, void* dw1, void* dw3,
+                          void* dw2, void* ws, size_t ws_bytes, void* stream) {
+  const moe_router_options_t o = opts ? *opts : default_options();
+  if (moe_status_t st = check_train(T, d, E, top_k, h, o, dt)) return st;
+  MOE_CHECK_ARG(std::isfinite(o.route_scale) && o.route_scale != 0.0f, "bad route_scale");
+  MOE_CHECK_ARG(w1 && w3 && w2 && dw1 && dw3 && dw2, "w1, w3, w2, dw1, dw3, dw2 are required");
+  MOE_CHECK_ARG(!dw_router || (x && w_router), "dw_router needs x and w_router");
+  MOE_CHECK_ARG(aligned16(w1) && aligned16(w3) && aligned16(w2) && aligned16(dw1) &&
+                    aligned16(dw3) && aligned16(dw2) && aligned16(dw_router) &&
+                    aligned16(x) && aligned16(w_router),
+                "weights, gradients and x must be 16-byte aligned");
+  if (T > 0) {
+    MOE_CHECK_ARG(dout && dx, "dout and dx are required");
+    MOE_CHECK_ARG(aligned16(dout) && aligned16(dx), "dout, dx must be 16-byte aligned");
+  }
+  MOE_CHECK_ARG(state != nullptr && ws != nullptr, "state and ws are required");
+  const BackwardWs need = carve_backward(nullptr, T, d, E, top_k, h);
+  if (ws_bytes < need.bytes) {
+    set_last_error("backward workspace %zu < %zu", ws_bytes, need.bytes);
+    return MOE_ERR_WORKSPACE;
+  }
+  const TrainState t = carve_train(const_cast<void*>(state), T, d, E, top_k, h);
+  const BackwardWs b = carve_backward(ws, T, d, E, top_k, h);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int N = T * top_k;
+  const bool gate = dw_router != nullptr;
+  cudaError_t e = cudaMemsetAsync(b.status, 0, sizeof(int), s);
+  if (N == 0) {
+    const size_t wbytes = static_cast<size_t>(E) * h * d * 2;
+    if (e == cudaSuccess) e = cudaMemsetAsync(dw1, 0, wbytes, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dw3, 0, wbytes, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dw2, 0, wbytes, s);
+    if (e == cudaSuccess && gate) e = cudaMemsetAsync(dw_router, 0, static_cast<size_t>(E) * d * 2, s);
+    return cuda_status(e, "moe_backward");
+  }
+  // combine -> experts -> router -> dispatch, all on `s`
+  if (e == cudaSuccess)
+    e = launch_combine_backward(dout, t.y, t.dst_pos, t.w, T, d, N, top_k, dt, b.dY, b.dtw, s);
+  if (e == cudaSuccess)
+    e = launch_swiglu_bwd_tc(t.x_perm, t.offsets, w1, w3, w2, t.H, t.GU, b.dY, N, d, h, E, b.dXp,
+                             dw1, dw3, dw2, b.dGU, b.status, s);
+  if (e == cudaSuccess)
+    e = launch_router_backward(t.logits, t.idx, b.dtw, T, E, top_k,
+                               o.score == MOE_SCORE_SIGMOID, o.renormalize, o.route_scale,
+                               d_logits, gate ? b.dz16 : nullptr, s);
+  if (e == cudaSuccess && gate)
+    e = launch_gate_backward_tc(b.dz16, x, w_router, T, d, E, dw_router, b.dxr, b.off2, b.status,
+                                s);
+  if (e == cudaSuccess)
+    e = launch_combine(b.dXp, t.dst_pos, nullptr, nullptr, T, d, N, top_k, dt, dx, s,
+                       gate ? b.dxr : nullptr);
+  return cuda_status(e, "moe_backward");
 }
 
 // ------------------------------------------------------------------ forward

@@ -177,3 +177,34 @@ def test_shared_expert_workspace_and_checks(L):
 def test_selftest_timeout_checks_its_workspace(L):
     assert L.moe_selftest_timeout(None, 1 << 10, None) == 1
     assert L.moe_selftest_timeout(ctypes.c_void_p(256), 16, None) == 1
+
+
+def test_training_entry_points_check_their_arguments(L):
+    """Whole-layer training: host-only sizes, and the rules of include/moe.h
+    (bf16 only, E % 8 == 0, no score_before_experts) enforced before any
+    launch."""
+    import routing_dispatch_grouped_topk_b200 as m
+    T, d, E, k, h = 4096, 2048, 128, 8, 768
+    N = T * k
+    assert L.moe_train_state_size(T, d, E, k, h) >= N * (2 * d + 3 * h) * 2 + T * E * 4
+    assert L.moe_backward_workspace_size(T, d, E, k, h) >= N * (2 * d + 2 * h) * 2
+    p = ctypes.c_void_p(256)
+    big = 1 << 40
+    # fp32 is not supported
+    assert L.moe_forward_train(p, p, None, p, p, p, 4, 64, 8, 2, 64, None, 0, p, p, big,
+                               None) == 2
+    # E not a multiple of 8
+    assert L.moe_forward_train(p, p, None, p, p, p, 4, 64, 12, 2, 64, None, 1, p, p, big,
+                               None) == 2
+    o = m.RouterOptions()
+    L.moe_router_options_init(ctypes.byref(o))
+    o.score_before_experts = 1
+    assert L.moe_forward_train(p, p, None, p, p, p, 4, 64, 8, 2, 64, ctypes.byref(o), 1, p, p,
+                               big, None) == 2
+    assert L.moe_backward(p, p, p, p, p, p, 4, 64, 8, 2, 64, ctypes.byref(o), 1, p, p, None, p,
+                          p, p, p, p, big, None) == 2
+    # state / workspace too small
+    assert L.moe_forward_train(p, p, None, p, p, p, 4, 64, 8, 2, 64, None, 1, p, p, 16,
+                               None) == 4
+    assert L.moe_backward(p, p, p, p, p, p, 4, 64, 8, 2, 64, None, 1, p, p, None, p, p, p, p, p,
+                          16, None) == 4

@@ -368,3 +368,87 @@ def test_layer_backward_full_size_sampled_tokens(M):
                 w2[e:e + 1].cpu(), dy[rr].cpu())
             ref[a] += rdx1[0]
     close(dx[tt], ref)
+
+
+# --------------------------------------------- whole-layer training entry points
+def _staged_training(M, x, wr, w1, w3, w2, k, dout, **opts):
+    """The layer's training step through the per-step entry points."""
+    E = w1.shape[0]
+    idx, tw, counts, logits, _ = M.router_topk(x, wr, k, want_logits=True, **opts)
+    cnt, off, src, dst, xp, _ = M.dispatch(x, idx, E)
+    y, h_act, gu, _ = M.grouped_swiglu_train(xp, off, w1, w3, w2)
+    out = M.combine(y, dst, tw)
+    dy, dtw = M.combine_backward(dout, y, dst, tw)
+    dxp, dw1, dw3, dw2, _ = M.grouped_swiglu_backward(xp, off, w1, w3, w2, h_act, gu, dy)
+    ropts = {n: v for n, v in opts.items() if n in ("score", "renormalize", "route_scale")}
+    dl, dwr, dxr, _ = M.router_backward(logits, idx, dtw, x, wr, **ropts)
+    dx = M.dispatch_backward(dxp, dst, dxr)
+    return dict(out=out, dx=dx, dw1=dw1, dw3=dw3, dw2=dw2, dw_router=dwr, d_logits=dl)
+
+
+@pytest.mark.parametrize("cfg_index", [1, 2])
+def test_forward_train_and_backward_equal_the_staged_calls(M, cfg_index):
+    """moe_forward_train / moe_backward run the same kernels in the same
+    order as the per-step entry points: every output is bit-identical, and
+    the forward's output equals moe_forward's."""
+    cfg = W.config(cfg_index)
+    lay = W.make_layer(cfg, device="cuda")
+    x, wr, w1, w3, w2 = (lay[n] for n in ("x", "w_router", "w1", "w3", "w2"))
+    g = torch.Generator(device="cuda").manual_seed(5)
+    dout = torch.randn(cfg.T, cfg.d, generator=g, device="cuda").to(torch.bfloat16)
+    ref = _staged_training(M, x, wr, w1, w3, w2, cfg.top_k, dout, renormalize=True)
+    out, state = M.forward_train(x, wr, w1, w3, w2, cfg.top_k, renormalize=True)
+    grads = M.backward(state, dout, x, wr, w1, w3, w2, want_d_logits=True)
+    torch.cuda.synchronize()
+    assert M.device_status(state["state"]) == 0 and M.device_status(grads["ws"]) == 0
+    assert torch.equal(out, ref["out"])
+    assert torch.equal(out, M.forward(x, wr, w1, w3, w2, cfg.top_k, True))
+    for n in ("dx", "dw1", "dw3", "dw2", "dw_router", "d_logits"):
+        assert torch.equal(grads[n], ref[n]), n
+
+
+@pytest.mark.parametrize("opts", [dict(), dict(score="sigmoid", route_scale=2.5),
+                                  dict(num_groups=4, topk_groups=2)])
+def test_layer_backward_matches_oracle(M, opts):
+    """Every gradient of the whole layer (x, w_router, w1, w3, w2, logits)
+    on a small layer against the oracle's chain rule, with router options."""
+    T, d, E, k, h = 200, 256, 16, 4, 192
+    g = torch.Generator().manual_seed(len(opts))
+    bf = torch.bfloat16
+    x = torch.randn(T, d, generator=g).to(bf)
+    # logits of std ~8: the fp32 gate and the fp64 oracle select the same experts
+    wr = (torch.randn(E, d, generator=g) * 0.5).to(bf)
+    w1 = (torch.randn(E, h, d, generator=g) / math.sqrt(d)).to(bf)
+    w3 = (torch.randn(E, h, d, generator=g) / math.sqrt(d)).to(bf)
+    w2 = (torch.randn(E, d, h, generator=g) / math.sqrt(h)).to(bf)
+    dout = torch.randn(T, d, generator=g).to(bf)
+    c = [t.cuda() for t in (x, wr, w1, w3, w2)]
+    out, state = M.forward_train(*c, k, renormalize=True, **opts)
+    grads = M.backward(state, dout.cuda(), *c, want_d_logits=True)
+    torch.cuda.synchronize()
+    assert M.device_status(state["state"]) == 0 and M.device_status(grads["ws"]) == 0
+    # the oracle: forward, then the chain rule step by step
+    ro = dict(score=opts.get("score", "softmax"), route_scale=opts.get("route_scale", 1.0),
+              num_groups=opts.get("num_groups", 0), topk_groups=opts.get("topk_groups", 0))
+    ref = O.moe_forward(x, wr, w1, w3, w2, k, True, router=ro)
+    gi = M.router_topk(c[0], c[1], k, True, **opts)[0]
+    assert np.array_equal(gi.cpu().numpy(), ref["topk_idx"])
+    close(out, ref["out"])
+    rdy, rdtw = O.combine_backward(dout, ref["y"], ref["dst_pos"], ref["topk_w"])
+    rdxp, rw1, rw3, rw2 = O.grouped_swiglu_backward(ref["x_perm"], ref["offsets"], w1, w3, w2,
+                                                    rdy)
+    rdz, rdwr, rdxr = O.router_backward(ref["logits"], ref["topk_idx"], rdtw,
+                                        score=ro["score"], renormalize=True,
+                                        route_scale=ro["route_scale"], x=x, w_router=wr)
+    rdx = O.dispatch_backward(rdxp, ref["dst_pos"]) + rdxr
+    close(grads["dx"], rdx)
+    for e in range(E):
+        if int(ref["counts"][e]) == 0:
+            assert not grads["dw1"][e].any()
+            continue
+        close_wgrad(grads["dw1"][e], rw1[e])
+        close_wgrad(grads["dw3"][e], rw3[e])
+        close_wgrad(grads["dw2"][e], rw2[e])
+    close_wgrad(grads["dw_router"], rdwr)
+    rowmax = np.abs(rdz).max(axis=1, keepdims=True)
+    assert np.all(np.abs(f64(grads["d_logits"]) - rdz) <= 5e-3 * (np.abs(rdz) + rowmax) + 1e-12)
