@@ -561,10 +561,11 @@ def run_ours(args, ws, rank, local):
 
 TRAIN_STAGES = ["router", "dispatch", "grouped_swiglu_train", "combine", "combine_backward",
                 "grouped_swiglu_backward", "router_backward", "dispatch_backward"]
-# kernels of ours per training step: router 2, dispatch 3 (histogram, scan,
-# scatter), training GEMMs 2, combine 1, combine backward 1, backward GEMMs 4,
-# router backward 4 (scores, segment, two gate GEMMs), dispatch backward 1
-TRAIN_LAUNCHES = 18
+# kernels of ours per two-call training step: router 2 (its top-k kernel also
+# writes the dispatch histogram), dispatch 2, training GEMMs 2, combine 1,
+# combine backward 1, backward GEMMs 4, router backward 4 (scores, segment,
+# two gate GEMMs), dispatch backward 1
+TRAIN_LAUNCHES = 17
 
 
 def run_training(args, ws, rank, local):
@@ -612,6 +613,20 @@ def run_training(args, ws, rank, local):
     rbws = torch.empty(M.router_backward_workspace_size(T, d, E), dtype=torch.uint8, device=dev)
     ropts = M.router_options(renormalize=cfg.renormalize)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    # the public two-call training step: moe_forward_train + moe_backward
+    tstate = torch.empty(M.lib().moe_train_state_size(T, d, E, k, h), dtype=torch.uint8,
+                         device=dev)
+    tws = torch.empty(M.lib().moe_backward_workspace_size(T, d, E, k, h), dtype=torch.uint8,
+                      device=dev)
+    tout = torch.empty(T, d, dtype=bf, device=dev)
+    tdx = torch.empty(T, d, dtype=bf, device=dev)
+    tdw1, tdw3, tdw2 = torch.empty_like(w1), torch.empty_like(w3), torch.empty_like(w2)
+    tdwr = torch.empty_like(wr)
+
+    def train_step():
+        M.moe_forward_train(x, wr, None, w1, w3, w2, T, d, E, k, h, ropts, dt, tout, tstate)
+        M.moe_backward(dout, x, wr, w1, w3, w2, T, d, E, k, h, ropts, dt, tstate, tdx, None,
+                       tdwr, tdw1, tdw3, tdw2, tws)
 
     def step(ev=None):
         def mark(i):
@@ -648,12 +663,29 @@ def run_training(args, ws, rank, local):
     t_warm = time.perf_counter()
     n_warm = 0
     while n_warm < args.warmup or time.perf_counter() - t_warm < 1.5:
+        train_step()
+        flush.zero_()
         step()
         flush.zero_()
         n_warm += 1
         if n_warm % 8 == 0:
             torch.cuda.synchronize()
     torch.cuda.synchronize()
+    # Timed region 1 (the value): the two public calls per step.
+    tev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    barrier(ws)
+    torch.cuda.synchronize()
+    for a_ev, b_ev in tev:
+        a_ev.record(stream)
+        train_step()
+        b_ev.record(stream)
+        flush.zero_()
+    torch.cuda.synchronize()
+    barrier(ws)
+    two_call_ms = sum(a.elapsed_time(b) for a, b in tev)
+    two_call_ms_max = max_over_ranks(two_call_ms, ws)
+    # Timed region 2 (breakdown): the per-step entry points, each bracketed.
     events = [[torch.cuda.Event(enable_timing=True) for _ in range(len(TRAIN_STAGES) + 1)]
               for _ in range(args.steps)]
     barrier(ws)
@@ -666,7 +698,8 @@ def run_training(args, ws, rank, local):
     clocks = sampler.stop() if rank == 0 else None
     total_ms = sum(ev[0].elapsed_time(ev[-1]) for ev in events)
     total_ms_max = max_over_ranks(total_ms, ws)
-    status = int(bws[:4].view(torch.int32)[0].item())
+    status = int(bws[:4].view(torch.int32)[0].item()) | int(tws[:4].view(torch.int32)[0].item())
+    matches = bool(torch.equal(tdx, dx) and torch.equal(tdw1, dw1) and torch.equal(tdwr, dwr))
     if rank != 0:
         return
     pk = peaks()
@@ -678,9 +711,9 @@ def run_training(args, ws, rank, local):
     tflops = bwd_flops / (bwd_ms / 1e3) / 1e12
     line = {
         "metric": "MoE-layer training step (forward + backward) routed tokens/s (bf16)",
-        "value": job_tokens_per_s(T, ws, args.steps, total_ms_max), "unit": UNIT,
+        "value": job_tokens_per_s(T, ws, args.steps, two_call_ms_max), "unit": UNIT,
         "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": total_ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
+        "ms_per_step": two_call_ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": cfg.name, "T": T, "d": d, "E": E, "top_k": k, "h": h,
                    "global_batch": T * ws, "parallelism": f"dp{ws}",
@@ -695,8 +728,14 @@ def run_training(args, ws, rank, local):
                      "peak_kind": f"bf16 sustained, {pk['source']}"},
         "forward_experts_tflops": fwd_flops / (stage_ms["grouped_swiglu_train"] / 1e3) / 1e12,
         "stage_ms": stage_ms,
+        "staged_ms_per_step": total_ms_max / args.steps,
+        "two_call_matches_staged": matches,
         "device_status": status,
         "gpu_launches": args.steps * TRAIN_LAUNCHES,
+        "gpu_launches_note": "kernels of libmoe per moe_forward_train + moe_backward step: "
+                             "router 2, dispatch 2, experts forward 2, combine 1, combine "
+                             "backward 1, experts backward 4, router backward 4, dispatch "
+                             "backward 1",
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)
