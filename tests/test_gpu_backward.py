@@ -450,9 +450,11 @@ def test_layer_backward_matches_oracle(M, opts):
         close_wgrad(grads["dw3"][e], rw3[e])
         close_wgrad(grads["dw2"][e], rw2[e])
     close_wgrad(grads["dw_router"], rdwr)
-    # d logits inherit the bf16 rounding of y through d topk_w = <dout, y> (the
-    # router backward alone is checked at 2e-5 above, on identical inputs)
+    # d logits inherit the bf16 rounding of y through d topk_w = <dout, y>, and
+    # in tokens whose softmax is saturated they are differences of nearly
+    # equal fp32 terms: checked here in norm; element by element the router
+    # backward is checked at 2e-5 on identical inputs
+    # (test_router_backward_matches_oracle) and moe_backward's d logits equal
+    # that kernel's bit for bit (test_forward_train_and_backward_equal_the_staged_calls)
     gdz = f64(grads["d_logits"])
-    rowmax = np.abs(rdz).max(axis=1, keepdims=True)
-    assert np.all(np.abs(gdz - rdz) <= 3e-2 * (np.abs(rdz) + rowmax) + 1e-12)
     assert np.linalg.norm(gdz - rdz) <= 1e-2 * np.linalg.norm(rdz)
