@@ -701,7 +701,7 @@ struct WgradPolicy {
   static constexpr bool GATHER_A = false;
   static constexpr bool A_MN = true, B_MN = true, MASK_K = true, CUSTOM_LOADS = true;
   static constexpr int EPI_WARPS = 8;   // two per lane quadrant, 128 columns each
-  static constexpr int THREADS = kThreads + 128;
+  static constexpr int THREADS = kThreads + 128 + 32;   // + the tail-clearing warp
   static constexpr int SCHED_INTS = 8 + kMaxExperts + 1;   // [0] tiles [1] m-tiles [2] n-tiles, offsets
 
   static __device__ void prologue(const Args& a, int* sched) {
@@ -817,7 +817,7 @@ struct Layout {
   static constexpr int kStages = stages_for(BN);
   static constexpr uint32_t kTmemCols = tmem_cols_for(BN);
   static constexpr int kBarOff = kStages * kStageBytes;
-  static constexpr int kNumBars = 2 * kStages + 5;
+  static constexpr int kNumBars = 3 * kStages + 5;   // full, empty, tail-cleared; 5 more
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSchedOff = (kMiscOff + 16 + 15) / 16 * 16;
   static constexpr int kEpiOff = (kSchedOff + P::SCHED_INTS * 4 + 15) / 16 * 16;
@@ -827,7 +827,9 @@ struct Layout {
   static_assert(kStages >= 2, "pipeline depth");
   static_assert(!P::GATHER_A || kStages == 4, "one gather warp per stage (warps 6..9)");
   static_assert(!P::GATHER_A || P::EPI_WARPS == 4, "warps 6..9 are either gather or epilogue");
-  static_assert(P::THREADS == 64 + 32 * P::EPI_WARPS + (P::GATHER_A ? 128 : 0), "warp roles");
+  static_assert(P::THREADS == 64 + 32 * P::EPI_WARPS + (P::GATHER_A ? 128 : 0) +
+                                  (P::MASK_K ? 32 : 0),
+                "warp roles");
 };
 
 template <class P>
@@ -852,6 +854,7 @@ __global__ void __launch_bounds__(P::THREADS, 1)
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* mma_done = tempty + 2;
+  uint64_t* cleared = mma_done + 1;   // [STAGES] MASK_K: tail rows of the stage zeroed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
   int* sched = reinterpret_cast<int*>(smem + L::kSchedOff);
@@ -869,6 +872,8 @@ __global__ void __launch_bounds__(P::THREADS, 1)
       mbar_init(tempty + a, P::EPI_WARPS);
     }
     mbar_init(mma_done, 1);
+    if (P::MASK_K)
+      for (int st = 0; st < STAGES; ++st) mbar_init(cleared + st, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -1040,48 +1045,35 @@ __global__ void __launch_bounds__(P::THREADS, 1)
         mbar_wait(full + s, ph, nullptr, args.status);
       }
     }
-  } else if (warp == 1 && P::MASK_K) {
-    // ------------------------------------- MMA issuer, K tails masked
-    // The whole warp walks the schedule; lane 0 waits on the barriers and
-    // issues the MMAs.  In the last K block of a segment only the 16-row MMA
-    // steps that hold segment rows are issued, and the rows of the last of
-    // them past the segment's end (the next segment's, loaded by the same
-    // box; fewer than 16) are zeroed in both operands by the 32 lanes
-    // first: each K row is one 128-byte line of every 8 KB box of the stage,
-    // whatever the swizzle.
+  } else if (P::MASK_K && warp == 2 + P::EPI_WARPS) {
+    // ------------------------------------------ tail-clearing warp
+    // The last K block of a segment also holds rows of the next segment.
+    // Only the 16-row MMA steps that hold segment rows are issued; the rows
+    // of the last of them past the segment's end (fewer than 16) are zeroed
+    // here in both operands as soon as the stage lands (a K row is one
+    // 128-byte line of every 8 KB box, whatever the swizzle).  The warp is a
+    // stage of the pipeline: it waits for every fill in order and hands every
+    // stage to the MMA thread through its "cleared" barrier, so it can
+    // neither run a ring cycle ahead of the fills nor fall behind them (a
+    // parity wait cannot tell phases two apart).  Off the MMA thread's path:
+    // the pipeline runs ahead, so a stage is usually cleared before the MMAs
+    // reach it.
     int stage = 0;
     uint32_t phase = 0;
-    int it = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++it) {
-      const int acc = it & 1;
-      const uint32_t aph = (it >> 1) & 1;
-      int go = 1;
-      if (lane == 0) go = mbar_wait(tempty + acc, aph ^ 1u, abort_flag, args.status) ? 1 : 0;
-      go = __shfl_sync(0xffffffffu, go, 0);
-      if (!go) break;
-      tc_fence_after();
-      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
       const TileInfo ti = P::tile_info(args, sched, tile);
       for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
-        if (lane == 0) go = mbar_wait(full + stage, phase, abort_flag, args.status) ? 1 : 0;
-        go = __shfl_sync(0xffffffffu, go, 0);
-        if (!go) {
+        const int rows = P::k_rows(ti, kb);
+        const int zr = ((rows + 15) & ~15) - rows;   // rows [rows, ceil16(rows)) to clear
+        const bool landed = mbar_wait(full + stage, phase, abort_flag, args.status);
+        if (!__all_sync(0xffffffffu, landed)) {
           ok = false;
           break;
         }
-        uint8_t* sa = tiles + stage * L::kStageBytes;
-        const int rows = P::k_rows(ti, kb);
-        const int ksteps = (rows + 15) >> 4;   // 16-row MMA steps holding segment rows
-        const int zr = ksteps * 16 - rows;      // rows [rows, 16 ksteps) to clear
         if (zr > 0) {
-          // every lane observes the landed stage before overwriting it
-          if (!mbar_wait(full + stage, phase, abort_flag, args.status)) go = 0;
-          if (!__all_sync(0xffffffffu, go)) {
-            ok = false;
-            break;
-          }
-          const int per_box = zr * 8;   // 16-byte chunks to clear per box (< 128)
+          uint8_t* sa = tiles + stage * L::kStageBytes;
+          const int per_box = zr * 8;   // 16-byte chunks per box (< 128)
           constexpr int kBoxes = L::kStageBytes / kMnBoxBytes;
 #pragma unroll
           for (int bx = 0; bx < kBoxes; ++bx)
@@ -1089,28 +1081,53 @@ __global__ void __launch_bounds__(P::THREADS, 1)
               *reinterpret_cast<uint4*>(sa + bx * kMnBoxBytes + rows * 128 + i * 16) =
                   make_uint4(0u, 0u, 0u, 0u);
           fence_proxy_async_smem();
-          __syncwarp();
         }
-        if (lane == 0) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(cleared + stage);
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+  } else if (warp == 1 && P::MASK_K) {
+    if (lane == 0) {
+      // ------------------------------------- MMA issuer, K tails masked
+      // Every stage comes through the tail-clearing warp; a segment's last K
+      // block issues only the 16-row steps holding its rows.
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++it) {
+        const int acc = it & 1;
+        const uint32_t aph = (it >> 1) & 1;
+        if (!mbar_wait(tempty + acc, aph ^ 1u, abort_flag, args.status)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        const TileInfo ti = P::tile_info(args, sched, tile);
+        for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
+          const int ksteps = (P::k_rows(ti, kb) + 15) >> 4;
+          if (!mbar_wait(cleared + stage, phase, abort_flag, args.status)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
+          const uint8_t* sa = tiles + stage * L::kStageBytes;
           const uint64_t ad = sw128_mnmajor_desc(sa, kMnBoxBytes);
           const uint64_t bd = sw128_mnmajor_desc(sa + kATileBytes, kMnBoxBytes);
           for (int kk = 0; kk < ksteps; ++kk)
             tc_mma_bf16(d_tmem, ad + A_KSTEP * kk, bd + B_KSTEP * kk, IDESC,
                         (kb != ti.kb0 || kk != 0) ? 1u : 0u);
           tc_commit(empty + stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
         }
-        __syncwarp();
-        if (++stage == STAGES) {
-          stage = 0;
-          phase ^= 1u;
-        }
+        if (!ok) break;
+        tc_commit(tfull + acc);
       }
-      if (!ok) break;
-      if (lane == 0) tc_commit(tfull + acc);
-      __syncwarp();
-    }
-    if (lane == 0) {
       tc_commit(mma_done);
       mbar_wait(mma_done, 0, nullptr, args.status);
     }
