@@ -390,10 +390,12 @@ MOE_API moe_status_t moe_combine(const void* y, const int32_t* dst_pos, const in
  *   d_logits = dz (fp32, optional), dw_router = dz^T x [E, d] (optional),
  *   dx = dz w_router [T, d] (optional)
  * The gate products run on tcgen05 from dz rounded once to bf16, with fp32
- * accumulation (bf16 x and w_router; dw_router and dx need dt = MOE_BF16
- * and E % 8 == 0).  opts NULL = defaults (softmax, no renormalisation, scale
- * 1).  E <= 512.  Workspace moe_router_backward_workspace_size (dz in bf16
- * plus the status word).  Entries of topk_idx outside [0, E) are skipped.
+ * accumulation (bf16 x and w_router; dw_router and dx need dt = MOE_BF16,
+ * E % 8 == 0 and d % 64 == 0).  dw_router is reduced over token segments
+ * into fp32 partials summed in segment order (deterministic).  opts NULL =
+ * defaults (softmax, no renormalisation, scale 1).  E <= 512.  Workspace
+ * moe_router_backward_workspace_size (dz in bf16, the partials and the
+ * status word).  Entries of topk_idx outside [0, E) are skipped.
  * ---------------------------------------------------------------------- */
 MOE_API moe_status_t moe_grouped_swiglu_train(const void* x_perm, const int32_t* offsets,
                                       const void* w1, const void* w3, const void* w2, int N,

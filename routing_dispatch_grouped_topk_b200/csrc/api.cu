@@ -342,13 +342,14 @@ TrainState carve_train(void* base, int T, int d, int E, int k, int h) {
 // Backward workspace of moe_backward.
 struct BackwardWs {
   int* status;
-  int32_t* off2;       // one-segment offsets of the gate's weight gradient
+  int32_t* off2;       // segment offsets of the gate's products (256 B)
   void* dY;            // [N, d]
   float* dtw;          // [T, k]
   void* dXp;           // [N, d]
   void* dGU;           // [N, 2h]
   void* dz16;          // [T, E]
   void* dxr;           // [T, d] the router's share of dx
+  float* gpart;        // [splits, E, d] fp32 partials of dw_router
   size_t bytes;
 };
 
@@ -357,13 +358,14 @@ BackwardWs carve_backward(void* base, int T, int d, int E, int k, int h) {
   Carve c(base);
   const size_t N = static_cast<size_t>(T) * k;
   b.status = c.take<int>(kStatusBytes / sizeof(int));
-  b.off2 = c.take<int32_t>(2);
+  b.off2 = c.take<int32_t>(64);
   b.dY = c.take<char>(N * d * 2);
   b.dtw = c.take<float>(N);
   b.dXp = c.take<char>(N * d * 2);
   b.dGU = c.take<char>(N * 2 * h * 2);
   b.dz16 = c.take<char>(static_cast<size_t>(T) * E * 2);
   b.dxr = c.take<char>(static_cast<size_t>(T) * d * 2);
+  b.gpart = c.take<float>(static_cast<size_t>(gate_splits(T, d, E)) * E * d);
   b.bytes = c.off;
   return b;
 }
@@ -783,10 +785,12 @@ moe_status_t moe_dispatch_backward(const void* dx_perm, const int32_t* dst_pos,
                      "moe_dispatch_backward");
 }
 
+// status, segment offsets (256 B), dz in bf16 [T, E], fp32 partials of
+// dw_router [splits, E, d]
 size_t moe_router_backward_workspace_size(int T, int d, int E) {
-  (void)d;
-  if (T < 0 || E < 1) return kStatusBytes;
-  return kStatusBytes + 256 + align_up(static_cast<size_t>(T) * E * 2, 256);
+  if (T < 0 || E < 1 || d < 1) return kStatusBytes;
+  return kStatusBytes + 256 + align_up(static_cast<size_t>(T) * E * 2, 256) +
+         align_up(static_cast<size_t>(gate_splits(T, d, E)) * E * d * 4, 256);
 }
 
 moe_status_t moe_router_backward(const float* logits, const int32_t* topk_idx,
@@ -804,8 +808,8 @@ moe_status_t moe_router_backward(const float* logits, const int32_t* topk_idx,
   MOE_CHECK_ARG(std::isfinite(o.route_scale) && o.route_scale != 0.0f, "bad route_scale");
   const bool gemm = dw_router || dx;
   if (gemm) {
-    if (dt != MOE_BF16 || E % 8 != 0 || d % 8 != 0) {
-      set_last_error("router backward gate gradients need bf16, E %% 8 == 0 and d %% 8 == 0");
+    if (dt != MOE_BF16 || E % 8 != 0 || d % 64 != 0) {
+      set_last_error("router backward gate gradients need bf16, E %% 8 == 0 and d %% 64 == 0");
       return MOE_ERR_UNSUPPORTED;
     }
   }
@@ -826,6 +830,8 @@ moe_status_t moe_router_backward(const float* logits, const int32_t* topk_idx,
   int* status = static_cast<int*>(ws);
   int32_t* off2 = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + kStatusBytes);
   void* dz16 = static_cast<char*>(ws) + kStatusBytes + 256;
+  float* gpart = reinterpret_cast<float*>(static_cast<char*>(dz16) +
+                                          align_up(static_cast<size_t>(T) * E * 2, 256));
   cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), s);
   if (e == cudaSuccess && T == 0 && dw_router)
     e = cudaMemsetAsync(dw_router, 0, static_cast<size_t>(E) * d * 2, s);
@@ -834,7 +840,8 @@ moe_status_t moe_router_backward(const float* logits, const int32_t* topk_idx,
                                o.score == MOE_SCORE_SIGMOID, o.renormalize, o.route_scale,
                                d_logits, gemm ? dz16 : nullptr, s);
   if (e == cudaSuccess && T > 0 && gemm)
-    e = launch_gate_backward_tc(dz16, x, w_router, T, d, E, dw_router, dx, off2, status, s);
+    e = launch_gate_backward_tc(dz16, x, w_router, T, d, E, dw_router, dx, off2, gpart, status,
+                                s);
   return cuda_status(e, "moe_router_backward");
 }
 
@@ -942,8 +949,8 @@ moe_status_t moe_backward(const void* dout, const void* x, const void* w_router,
                                o.score == MOE_SCORE_SIGMOID, o.renormalize, o.route_scale,
                                d_logits, gate ? b.dz16 : nullptr, s);
   if (e == cudaSuccess && gate)
-    e = launch_gate_backward_tc(b.dz16, x, w_router, T, d, E, dw_router, b.dxr, b.off2, b.status,
-                                s);
+    e = launch_gate_backward_tc(b.dz16, x, w_router, T, d, E, dw_router, b.dxr, b.off2, b.gpart,
+                                b.status, s);
   if (e == cudaSuccess)
     e = launch_combine(b.dXp, t.dst_pos, nullptr, nullptr, T, d, N, top_k, dt, dx, s,
                        gate ? b.dxr : nullptr);

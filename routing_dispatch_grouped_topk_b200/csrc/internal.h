@@ -107,9 +107,18 @@ cudaError_t launch_router_backward(const float* logits, const int32_t* topk_idx,
 // Gradients of the gate x . w_router^T for dz16 [T, E] bf16: dw_router =
 // dz^T x [E, d] and dx = dz w_router [T, d] (bf16, each optional); offsets2 is
 // device scratch for two ints.
+// dw_router is reduced over gate_splits(T, d, E) token segments into fp32
+// partials [splits, E, d] (gpart), then summed in order; offsets holds
+// splits + 1 ints (at most 64).
+int gate_splits(int T, int d, int E);
 cudaError_t launch_gate_backward_tc(const void* dz16, const void* x, const void* w_router, int T,
-                                    int d, int E, void* dw_router, void* dx, int32_t* offsets2,
-                                    int* status, cudaStream_t s);
+                                    int d, int E, void* dw_router, void* dx, int32_t* offsets,
+                                    float* gpart, int* status, cudaStream_t s);
+// offsets[i] = floor(i n / S), i = 0..S.
+cudaError_t launch_uniform_segments(int32_t* offsets, int S, int n, cudaStream_t s);
+// out [n] bf16 = sum over S fp32 partial arrays [S, n] (n a multiple of 4).
+cudaError_t launch_sum_partials_bf16(const float* part, int S, size_t n, void* out,
+                                     cudaStream_t s);
 // Self-test of the bounded wait: sets MOE_DEV_TIMEOUT after kWaitLimitNs.
 cudaError_t launch_selftest_timeout(int* status, cudaStream_t s);
 // offsets[0] = 0, offsets[1] = n: the segmentation of a single expert.

@@ -799,6 +799,48 @@ cudaError_t launch_single_segment(int32_t* offsets, int n, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+// offsets[i] = floor(i n / S), i = 0..S: S near-equal segments of n rows.
+__global__ void uniform_segments_kernel(int32_t* offsets, int S, int n) {
+  pdl_wait();
+  pdl_trigger();
+  for (int i = threadIdx.x; i <= S; i += blockDim.x)
+    offsets[i] = static_cast<int32_t>((static_cast<long long>(i) * n) / S);
+}
+
+cudaError_t launch_uniform_segments(int32_t* offsets, int S, int n, cudaStream_t s) {
+  launch_k(uniform_segments_kernel, dim3(1), dim3(128), 0, s, offsets, S, n);
+  return cudaGetLastError();
+}
+
+// out[i] = bf16(sum_{p < S} part[p][i]), fp32 sum in partial order (4 per thread).
+__global__ void __launch_bounds__(256) sum_partials_bf16_kernel(const float4* __restrict__ part,
+                                                                int S, size_t n4,
+                                                                uint2* __restrict__ out) {
+  pdl_wait();
+  pdl_trigger();
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n4;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    float4 a = part[i];
+    for (int p = 1; p < S; ++p) {
+      const float4 b = part[static_cast<size_t>(p) * n4 + i];
+      a.x += b.x;
+      a.y += b.y;
+      a.z += b.z;
+      a.w += b.w;
+    }
+    out[i] = make_uint2(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w));
+  }
+}
+
+cudaError_t launch_sum_partials_bf16(const float* part, int S, size_t n, void* out,
+                                     cudaStream_t s) {
+  const size_t n4 = n / 4;
+  const int blocks = static_cast<int>(std::min<size_t>((n4 + 255) / 256, 8 * num_sms()));
+  launch_k(sum_partials_bf16_kernel, dim3(std::max(blocks, 1)), dim3(256), 0, s,
+           reinterpret_cast<const float4*>(part), S, n4, static_cast<uint2*>(out));
+  return cudaGetLastError();
+}
+
 // ------------------------------------------------------- fp32 / SIMT router
 template <typename TX>
 __device__ __forceinline__ float to_f(TX v);

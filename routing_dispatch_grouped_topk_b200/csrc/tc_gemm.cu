@@ -91,6 +91,7 @@ struct Args {
   __nv_bfloat16* out1;       // weight gradient: output rows >= split of each expert
   int split;                 // weight gradient: rows of each expert that go to `out`
   int Ma;                    // weight gradient: output rows per expert
+  float* out_f32;            // weight gradient: fp32 output [E, Ma, n_out] instead of bf16
 };
 
 __host__ __device__ constexpr int stages_for(int bn) {
@@ -766,6 +767,30 @@ struct WgradPolicy {
     const int e = ti.b_row;
     const int j = lane & 3;
     const bool empty = ti.kb1 == ti.kb0;
+    if (a.out_f32) {
+      // fp32 partials (split reductions): each lane stores its own row
+      const int m = ti.m0 + row;
+      float* drow = a.out_f32 + (static_cast<size_t>(e) * a.Ma + m) * Nb + ti.n0;
+#pragma unroll 1
+      for (int c = c0; c < c1; ++c) {
+        if (ti.n0 + c * 32 >= Nb) break;   // warp-uniform
+        uint32_t r[32];
+        if (!empty) {
+          tmem_ld32(taddr + c * 32, r);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int q = 0; q < 32; ++q) r[q] = 0u;
+        }
+        if (m < a.Ma) {
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            reinterpret_cast<uint4*>(drow + c * 32)[q] =
+                make_uint4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
+        }
+      }
+      return;
+    }
     __nv_bfloat16* dst[4];
     bool rvalid[4];
 #pragma unroll
@@ -1704,35 +1729,54 @@ cudaError_t launch_swiglu_bwd_tc(const void* x_perm, const int32_t* offsets, con
   return launch<WgradPolicy>(m_dgu, m_x, m_x, a, grid, s);
 }
 
+// Token segments of the gate's weight gradient: enough (E, d) tiles x
+// segments to fill about kRouterTargetTiles SMs, segments of >= 256 tokens,
+// at most 63 (the offsets fit in 256 bytes).  Sizes only: workspace sizes
+// are computed on the host without a device.
+int gate_splits(int T, int d, int E) {
+  const int tiles = cdiv(E, tc::BM) * cdiv(d, 256);
+  return std::max(1, std::min(std::min(kRouterTargetTiles / tiles, T / 256), 63));
+}
+
 // Gradients of the gate logits = x . w_router^T for dz16 [T, E] (bf16):
-//   dw_router = dz^T x   (WgradPolicy over one segment of T rows)
-//   dx        = dz w_router (DgradPolicy, K = E)
+//   dw_router = dz^T x   (WgradPolicy over S token segments into fp32
+//                         partials, then summed in segment order)
+//   dx        = dz w_router (DgradPolicy, K = E, one segment)
 cudaError_t launch_gate_backward_tc(const void* dz16, const void* x, const void* w_router, int T,
-                                    int d, int E, void* dw_router, void* dx, int32_t* offsets2,
-                                    int* status, cudaStream_t s) {
+                                    int d, int E, void* dw_router, void* dx, int32_t* offsets,
+                                    float* gpart, int* status, cudaStream_t s) {
   using namespace tc;
   if (T == 0) return cudaSuccess;
-  cudaError_t e = launch_single_segment(offsets2, T, s);
-  if (e != cudaSuccess) return e;
+  cudaError_t e = cudaSuccess;
   Args a{};
   a.M = T;
-  a.E = 1;
-  a.offsets = offsets2;
   a.status = status;
+  a.offsets = offsets;
   if (dw_router) {
+    const int S = gate_splits(T, d, E);
+    e = launch_uniform_segments(offsets, S, T, s);
+    if (e != cudaSuccess) return e;
     CUtensorMap m_dz, m_x;
     if (!make_tmap(&m_dz, dz16, E, T, 64)) return cudaErrorInvalidValue;
     if (!make_tmap(&m_x, x, d, T, 64)) return cudaErrorInvalidValue;
+    a.E = S;
     a.Ma = E;
     a.split = E;
     a.n_out = d;
-    a.out = static_cast<__nv_bfloat16*>(dw_router);
+    a.out = nullptr;
     a.out1 = nullptr;
-    const int grid = std::min(num_sms(), cdiv(E, BM) * cdiv(d, 256));
+    a.out_f32 = gpart;
+    const int grid = std::min(num_sms(), S * cdiv(E, BM) * cdiv(d, 256));
     e = launch<WgradPolicy>(m_dz, m_x, m_x, a, grid, s);
+    if (e == cudaSuccess)
+      e = launch_sum_partials_bf16(gpart, S, static_cast<size_t>(E) * d, dw_router, s);
     if (e != cudaSuccess) return e;
+    a.out_f32 = nullptr;
   }
   if (dx) {
+    e = launch_single_segment(offsets, T, s);
+    if (e != cudaSuccess) return e;
+    a.E = 1;
     CUtensorMap t_dz, t_wr;
     if (!make_tmap(&t_dz, dz16, E, T, BM)) return cudaErrorInvalidValue;
     if (!make_tmap(&t_wr, w_router, d, E, 64)) return cudaErrorInvalidValue;

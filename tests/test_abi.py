@@ -208,3 +208,18 @@ def test_training_entry_points_check_their_arguments(L):
                                None) == 4
     assert L.moe_backward(p, p, p, p, p, p, 4, 64, 8, 2, 64, None, 1, p, p, None, p, p, p, p, p,
                           16, None) == 4
+
+
+def test_router_backward_gate_rules(L):
+    """The gate's gradients need bf16, E % 8 == 0 and d % 64 == 0 (the
+    epilogue writes 32-column chunks); d logits alone have no such rule."""
+    p = ctypes.c_void_p(256)
+    big = 1 << 30
+    assert L.moe_router_backward(p, p, p, p, p, 4, 96, 8, 2, None, 1, None, p, None, p, big,
+                                 None) == 2
+    assert L.moe_router_backward(p, p, p, p, p, 4, 64, 12, 2, None, 1, None, p, None, p, big,
+                                 None) == 2
+    assert L.moe_router_backward(p, p, p, p, p, 4, 64, 8, 2, None, 0, None, p, None, p, big,
+                                 None) == 2
+    assert L.moe_router_backward(p, p, p, p, p, 4, 96, 12, 2, None, 0, p, None, None, p, 16,
+                                 None) == 4

@@ -288,11 +288,13 @@ ROUTER_BWD = [("softmax", True, 1.0), ("softmax", False, 2.5), ("sigmoid", True,
 
 
 @pytest.mark.parametrize("score,renorm,scale", ROUTER_BWD)
-@pytest.mark.parametrize("T,E,k,d", [(300, 128, 8, 256), (77, 72, 4, 192), (33, 8, 2, 64)])
+@pytest.mark.parametrize("T,E,k,d", [(300, 128, 8, 256), (77, 72, 4, 192), (33, 8, 2, 64),
+                                     (2100, 64, 8, 256)])
 def test_router_backward_matches_oracle(M, score, renorm, scale, T, E, k, d):
     """d_logits (fp32) within 2e-5 of the row's largest entry; dw_router and
     the router's dx (bf16, from dz rounded once to bf16) within the
-    RMS-relative bound of sums over mixed-sign terms."""
+    RMS-relative bound of sums over mixed-sign terms.  T = 2100 splits
+    dw_router over 8 token segments (fp32 partials, a ragged last one)."""
     L = W.make_logits(T, E, k, seed=T + E)
     idx, w, _, _ = O.router_topk_general(k, logits=L, score=score, renormalize=renorm,
                                          route_scale=scale)
