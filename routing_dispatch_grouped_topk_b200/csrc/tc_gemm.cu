@@ -659,6 +659,69 @@ struct UpBwdPolicy : GroupedSched<256, 2, 256> {
   static __device__ void finish(const Args&, int*) {}
 };
 
+// GEMM1 of the training forward: H, G and U of 32 hidden units per chunk,
+// 8 epilogue warps (two per lane quadrant, two chunks each), every store
+// staged through shared memory so that a warp writes whole 64-byte row
+// segments (the per-row stores of the inference epilogue write 16 bytes of
+// 32 rows per instruction; with G and U added they cost ~15 % of GEMM1).
+struct UpTrainPolicy : UpPolicyT<false> {
+  static constexpr int EPI_WARPS = 8;
+  static constexpr int THREADS = kThreads + 128;
+  static constexpr int EPI_STAGE_BYTES = 8 * 2048;
+  static __device__ void epilogue_staged(const Args& a, int* s, const TileInfo& ti,
+                                         uint32_t taddr, int row, uint8_t* stg, int c0, int c1) {
+    if (ti.swap_np) {
+      // swap-AB tile: one lane per hidden unit; the first warp of each
+      // quadrant writes (the per-row epilogue, as inference)
+      if (c0 == 0) UpPolicyT<false>::epilogue(a, s, ti, taddr, row);
+      return;
+    }
+    const int lane = threadIdx.x & 31;
+    const int wrow0 = row - lane;
+    const int h = a.n_out;
+    const int j = lane & 3;
+    // chunk range over the 4 chunks of 32 hidden units (c0, c1 index 8 halves)
+    const int q0 = c0 / 2, q1 = c1 / 2;
+    auto store = [&](const uint32_t (&w)[16], __nv_bfloat16* base, size_t stride, int col) {
+#pragma unroll
+      for (int p = 0; p < 4; ++p)
+        *reinterpret_cast<uint4*>(stg + stg_off(lane, p)) =
+            make_uint4(w[4 * p], w[4 * p + 1], w[4 * p + 2], w[4 * p + 3]);
+      __syncwarp();
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int rr = 8 * q + (lane >> 2);
+        if (wrow0 + rr < ti.m_valid)
+          *reinterpret_cast<uint4*>(base + static_cast<size_t>(ti.a_row + wrow0 + rr) * stride +
+                                    col + j * 8) =
+              *reinterpret_cast<const uint4*>(stg + stg_off(rr, j));
+      }
+      __syncwarp();
+    };
+#pragma unroll 1
+    for (int c = q0; c < q1; ++c) {
+      uint32_t g[32], u[32];
+      tmem_ld32(taddr + c * 32, g);
+      tmem_ld32(taddr + 128 + c * 32, u);
+      tmem_ld_wait();
+      if (ti.n0 + c * 32 >= h) continue;   // warp-uniform
+      uint32_t ph[16], pg[16], pu[16];
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        const float g0 = __uint_as_float(g[2 * q]), g1 = __uint_as_float(g[2 * q + 1]);
+        const float u0 = __uint_as_float(u[2 * q]), u1 = __uint_as_float(u[2 * q + 1]);
+        ph[q] = pack_bf16x2(silu_f(g0) * u0, silu_f(g1) * u1);
+        pg[q] = pack_bf16x2(g0, g1);
+        pu[q] = pack_bf16x2(u0, u1);
+      }
+      const int col = ti.n0 + c * 32;
+      store(ph, a.out, static_cast<size_t>(h), col);
+      store(pg, a.gu_out, 2 * static_cast<size_t>(h), col);
+      store(pu, a.gu_out, 2 * static_cast<size_t>(h), h + col);
+    }
+  }
+};
+
 // Data gradient through one untransposed weight: out [M, n_out] = A B with
 // A [M, K] K-major and B [K, n_out] (K rows, MN-major), one segment.  Used
 // for the gate: dx = dz . w_router (K = E).
@@ -1647,6 +1710,7 @@ static cudaError_t swiglu_tc_impl(const void* a_src, int a_rows, const int32_t* 
   }
   int grid = static_cast<int>(std::min<long long>(num_sms(), 1LL * max_mt * cdiv(h, 128)));
   cudaError_t e = gather ? launch<UpGatherPolicy>(tx, t1, t3, a, grid, s)
+                  : gu   ? launch<UpTrainPolicy>(tx, t1, t3, a, grid, s)
                          : launch<UpPolicy>(tx, t1, t3, a, grid, s);
   if (e != cudaSuccess) return e;
   // GEMM2: y = H w2^T (* row_scale)
