@@ -722,6 +722,55 @@ struct UpTrainPolicy : UpPolicyT<false> {
   }
 };
 
+// GEMM2 with the staged epilogue: 8 warps (two per lane quadrant, four
+// 32-column chunks each), each chunk scaled per row, converted, staged and
+// stored as whole 64-byte row segments.  Swap-AB tiles keep the per-row
+// epilogue (the first warp of each quadrant).
+struct DownStagedPolicy : DownPolicy {
+  static constexpr int EPI_WARPS = 8;
+  static constexpr int THREADS = kThreads + 128;
+  static constexpr int EPI_STAGE_BYTES = 8 * 2048;
+  static __device__ void epilogue_staged(const Args& a, int* s, const TileInfo& ti,
+                                         uint32_t taddr, int row, uint8_t* stg, int c0, int c1) {
+    if (ti.swap_np) {
+      if (c0 == 0) DownPolicy::epilogue(a, s, ti, taddr, row);
+      return;
+    }
+    const int lane = threadIdx.x & 31;
+    const int wrow0 = row - lane;
+    const int j = lane & 3;
+    const bool valid = row < ti.m_valid;
+    const float scale = (valid && a.row_scale) ? a.row_scale[ti.a_row + row] : 1.0f;
+#pragma unroll 1
+    for (int c = c0; c < c1; ++c) {
+      uint32_t r[32];
+      tmem_ld32(taddr + c * 32, r);
+      tmem_ld_wait();
+      if (ti.n0 + c * 32 >= a.n_out) continue;   // warp-uniform
+#pragma unroll
+      for (int p = 0; p < 4; ++p)
+        *reinterpret_cast<uint4*>(stg + stg_off(lane, p)) = make_uint4(
+            pack_bf16x2(__uint_as_float(r[8 * p]) * scale, __uint_as_float(r[8 * p + 1]) * scale),
+            pack_bf16x2(__uint_as_float(r[8 * p + 2]) * scale,
+                        __uint_as_float(r[8 * p + 3]) * scale),
+            pack_bf16x2(__uint_as_float(r[8 * p + 4]) * scale,
+                        __uint_as_float(r[8 * p + 5]) * scale),
+            pack_bf16x2(__uint_as_float(r[8 * p + 6]) * scale,
+                        __uint_as_float(r[8 * p + 7]) * scale));
+      __syncwarp();
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int rr = 8 * q + (lane >> 2);
+        if (wrow0 + rr < ti.m_valid)
+          *reinterpret_cast<uint4*>(a.out + static_cast<size_t>(ti.a_row + wrow0 + rr) * a.n_out +
+                                    ti.n0 + c * 32 + j * 8) =
+              *reinterpret_cast<const uint4*>(stg + stg_off(rr, j));
+      }
+      __syncwarp();
+    }
+  }
+};
+
 // Data gradient through one untransposed weight: out [M, n_out] = A B with
 // A [M, K] K-major and B [K, n_out] (K rows, MN-major), one segment.  Used
 // for the gate: dx = dz . w_router (K = E).
@@ -1719,7 +1768,7 @@ static cudaError_t swiglu_tc_impl(const void* a_src, int a_rows, const int32_t* 
   a.out = static_cast<__nv_bfloat16*>(y);
   a.row_scale = row_scale;
   grid = static_cast<int>(std::min<long long>(num_sms(), 1LL * max_mt * cdiv(d, 256)));
-  return launch<DownPolicy>(th, t2, t2, a, grid, s);
+  return launch<DownStagedPolicy>(th, t2, t2, a, grid, s);
 }
 
 cudaError_t launch_swiglu_tc_train(const void* x_perm, const int32_t* offsets, const void* w1,
