@@ -236,3 +236,36 @@ def test_router_backward_closed_forms():
     np.testing.assert_allclose(dz.sum(axis=1), 0.0, atol=1e-14)
     dz1 = O.router_backward(L, idx[:, :1], g[:, :1], renormalize=True)
     np.testing.assert_allclose(dz1, 0.0, atol=1e-15)
+
+
+def test_whole_layer_gradients_compose_to_finite_differences():
+    """The layer's gradients assembled from the oracle's pieces (combine,
+    experts, router with its gate, dispatch) equal central differences of
+    the whole oracle layer L = <dout, moe_forward(x, w_router, ...)> with
+    respect to x and w_router (selection fixed: the gate's logits are well
+    separated), and with respect to one expert weight."""
+    rng = np.random.default_rng(21)
+    T, d, E, k, h = 6, 5, 4, 2, 3
+    x = rng.standard_normal((T, d))
+    wr = rng.standard_normal((E, d)) * 2.0
+    w1 = rng.standard_normal((E, h, d)) * 0.6
+    w3 = rng.standard_normal((E, h, d)) * 0.6
+    w2 = rng.standard_normal((E, d, h)) * 0.6
+    dout = rng.standard_normal((T, d))
+    ref = O.moe_forward(x, wr, w1, w3, w2, k, True)
+    L = ref["logits"]
+    srt = np.sort(L, axis=1)
+    assert np.min(srt[:, -k] - srt[:, -k - 1]) > 1e-3   # selection is stable under 1e-6 steps
+    dy, dtw = O.combine_backward(dout, ref["y"], ref["dst_pos"], ref["topk_w"])
+    dxp, dw1, dw3, dw2 = O.grouped_swiglu_backward(ref["x_perm"], ref["offsets"], w1, w3, w2, dy)
+    _, dwr, dxr = O.router_backward(L, ref["topk_idx"], dtw, renormalize=True, x=x, w_router=wr)
+    dx = O.dispatch_backward(dxp, ref["dst_pos"]) + dxr
+
+    def loss():
+        r = O.moe_forward(x, wr, w1, w3, w2, k, True)
+        assert np.array_equal(r["topk_idx"], ref["topk_idx"])
+        return float(np.sum(dout * r["out"]))
+
+    np.testing.assert_allclose(dx, _fd(loss, x), atol=2e-7)
+    np.testing.assert_allclose(dwr, _fd(loss, wr), atol=2e-7)
+    np.testing.assert_allclose(dw2, _fd(loss, w2), atol=2e-7)
