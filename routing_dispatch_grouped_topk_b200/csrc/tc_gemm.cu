@@ -659,12 +659,12 @@ struct UpBwdPolicy : GroupedSched<256, 2, 256> {
   static __device__ void finish(const Args&, int*) {}
 };
 
-// GEMM1 of the training forward: H, G and U of 32 hidden units per chunk,
-// 8 epilogue warps (two per lane quadrant, two chunks each), every store
-// staged through shared memory so that a warp writes whole 64-byte row
-// segments (the per-row stores of the inference epilogue write 16 bytes of
-// 32 rows per instruction; with G and U added they cost ~15 % of GEMM1).
-struct UpTrainPolicy : UpPolicyT<false> {
+// GEMM1 with the staged epilogue: H (and, in the training forward, G and U)
+// of 32 hidden units per chunk, 8 epilogue warps (two per lane quadrant, two
+// chunks each), every store staged through shared memory so that a warp
+// writes whole 64-byte row segments (per-row stores write 16 bytes of 32
+// rows per instruction; with G and U added they cost ~15 % of GEMM1).
+struct UpStagedPolicy : UpPolicyT<false> {
   static constexpr int EPI_WARPS = 8;
   static constexpr int THREADS = kThreads + 128;
   static constexpr int EPI_STAGE_BYTES = 8 * 2048;
@@ -716,8 +716,10 @@ struct UpTrainPolicy : UpPolicyT<false> {
       }
       const int col = ti.n0 + c * 32;
       store(ph, a.out, static_cast<size_t>(h), col);
-      store(pg, a.gu_out, 2 * static_cast<size_t>(h), col);
-      store(pu, a.gu_out, 2 * static_cast<size_t>(h), h + col);
+      if (a.gu_out) {
+        store(pg, a.gu_out, 2 * static_cast<size_t>(h), col);
+        store(pu, a.gu_out, 2 * static_cast<size_t>(h), h + col);
+      }
     }
   }
 };
@@ -1759,8 +1761,7 @@ static cudaError_t swiglu_tc_impl(const void* a_src, int a_rows, const int32_t* 
   }
   int grid = static_cast<int>(std::min<long long>(num_sms(), 1LL * max_mt * cdiv(h, 128)));
   cudaError_t e = gather ? launch<UpGatherPolicy>(tx, t1, t3, a, grid, s)
-                  : gu   ? launch<UpTrainPolicy>(tx, t1, t3, a, grid, s)
-                         : launch<UpPolicy>(tx, t1, t3, a, grid, s);
+                         : launch<UpStagedPolicy>(tx, t1, t3, a, grid, s);
   if (e != cudaSuccess) return e;
   // GEMM2: y = H w2^T (* row_scale)
   a.K = h;
