@@ -563,9 +563,10 @@ TRAIN_STAGES = ["router", "dispatch", "grouped_swiglu_train", "combine", "combin
                 "grouped_swiglu_backward", "router_backward", "dispatch_backward"]
 # kernels of ours per two-call training step: router 2 (its top-k kernel also
 # writes the dispatch histogram), dispatch 2, training GEMMs 2, combine 1,
-# combine backward 1, backward GEMMs 4, router backward 4 (scores, segment,
-# two gate GEMMs), dispatch backward 1
-TRAIN_LAUNCHES = 17
+# combine backward 1, backward GEMMs 4, router backward 6 (scores, token
+# segments, gate weight-gradient partials, their sum, one segment, gate data
+# gradient), dispatch backward 1
+TRAIN_LAUNCHES = 19
 
 
 def run_training(args, ws, rank, local):
@@ -734,7 +735,7 @@ def run_training(args, ws, rank, local):
         "gpu_launches": args.steps * TRAIN_LAUNCHES,
         "gpu_launches_note": "kernels of libmoe per moe_forward_train + moe_backward step: "
                              "router 2, dispatch 2, experts forward 2, combine 1, combine "
-                             "backward 1, experts backward 4, router backward 4, dispatch "
+                             "backward 1, experts backward 4, router backward 6, dispatch "
                              "backward 1",
         "clocks": clocks,
     }
