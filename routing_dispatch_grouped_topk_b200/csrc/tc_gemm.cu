@@ -605,7 +605,7 @@ struct DownBwdPolicy : GroupedSched<256, 1, 256> {
             const float g = hlf ? bf16_hi(gw[q]) : bf16_lo(gw[q]);
             const float u = hlf ? bf16_hi(uw[q]) : bf16_lo(uw[q]);
             const float da = __uint_as_float(r[2 * q + hlf]);
-            const float sgm = 1.0f / (1.0f + __expf(-g));
+            const float sgm = __fdividef(1.0f, 1.0f + __expf(-g));
             du[hlf] = da * (g * sgm);
             dg[hlf] = da * u * (sgm * (1.0f + g * (1.0f - sgm)));
           }
