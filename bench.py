@@ -1,15 +1,21 @@
 """Benchmark of the MoE layer forward on B200 (one JSON line on rank 0).
 
 A step is one pass of the whole hot path over one batch of synthetic tokens
-resident in HBM: router top-k -> dispatch -> grouped SwiGLU -> combine.
-Timed region 1 (the headline ``value``) calls the public moe_forward once
-per step.  Timed region 2 runs the same layer as the sequence of entry
-points (moe_router_topk, moe_dispatch, moe_grouped_swiglu, moe_combine),
-each bracketed by CUDA events on the launching stream, for the per-stage
-breakdown and the grouped-GEMM duration of the roofline.  L2 is flushed
-(256 MB write) between timed steps, outside the step's events.  ``value`` is
-tokens/s of the whole job (all ranks; ranks run independent token batches,
-weak scaling, no data-path collective).
+resident in HBM: router top-k -> dispatch -> (EP regroup) -> grouped SwiGLU
+-> combine.  The headline workload is the gpt-oss-120b-shaped layer with
+8 simulated EP ranks (T=8192, d=2880, E=128, k=4, h=2880), the largest
+single-GPU one and the one that runs the regroup.  Timed region 1 (the
+headline ``value``) calls the public moe_forward once per step.  Timed
+region 2 runs the same layer as the sequence of entry points
+(moe_router_topk, moe_ep_dispatch_rank_major, moe_ep_local_regroup,
+moe_grouped_swiglu, moe_combine), each bracketed by CUDA events on the
+launching stream, for the per-stage breakdown and the grouped-GEMM duration
+of the roofline.  L2 is flushed (256 MB write) between timed steps, outside
+the step's events.  ``value`` is tokens/s of the whole job (all ranks; ranks
+run independent token batches, weak scaling, no data-path collective).
+On one GPU the same run then measures every other workload (moe_forward
+and the staged entry points) into ``other_configs``, with the grouped
+SwiGLU against HBM and against the burst and sustained bf16 peaks.
 
 ``--impl reference`` times the fp64 CPU oracle on the host cores instead
 (a bounded token sample per step) and prints the same metric.
@@ -43,9 +49,6 @@ import workloads as W  # noqa: E402
 METRIC = "MoE-layer routed tokens/s (bf16); grouped-GEMM TFLOP/s as % of tensor peak"
 UNIT = "tokens/s"
 FLUSH_BYTES = 256 << 20
-# kernels of ours per moe_forward step (the router's top-k kernel also writes
-# the dispatch histogram; memsets of the status word are not kernels of ours)
-LAUNCHES_PER_STEP = {"router": 2, "dispatch": 2, "grouped_swiglu": 2, "combine": 1}
 
 
 def peaks():
@@ -268,89 +271,204 @@ def run_reference(args, ws, rank):
 
 
 # ------------------------------------------------------------------- GPU arm
+# kernels of libmoe that one moe_forward step launches: router (GEMM, top-k
+# with the dispatch histogram), dispatch (column scan, scatter), regroup on
+# the EP layout (scan, copy), grouped SwiGLU (GEMM1, GEMM2), combine
+def forward_launches(cfg) -> int:
+    return 2 + 2 + (2 if cfg.ep_ranks > 1 else 0) + 2 + 1
+
+
+class Layer:
+    """Device buffers of one workload and its two step functions: the public
+    moe_forward call, and the same layer as the sequence of entry points
+    (moe_router_topk, moe_dispatch / moe_ep_dispatch_rank_major,
+    moe_ep_local_regroup, moe_grouped_swiglu, moe_combine)."""
+
+    def __init__(self, M, cfg, dev, rank=0):
+        self.M, self.cfg, self.dev = M, cfg, dev
+        T, d, E, k, h, R = cfg.T, cfg.d, cfg.E, cfg.top_k, cfg.h, cfg.ep_ranks
+        N = T * k
+        lay = W.make_layer(cfg, dev)
+        if rank:   # independent token batch per rank
+            lay["x"] = W.make_layer(rank_workload(cfg, rank), dev, experts=False)["x"]
+        self.x, self.wr, self.w1, self.w3, self.w2 = (lay["x"], lay["w_router"], lay["w1"],
+                                                      lay["w3"], lay["w2"])
+        self.dt = M.MOE_BF16 if cfg.dtype == "bf16" else M.MOE_F32
+        x = self.x
+        self.idx = torch.empty(T, k, dtype=torch.int32, device=dev)
+        self.w = torch.empty(T, k, dtype=torch.float32, device=dev)
+        self.rws = torch.empty(M.router_workspace_size(T, d, E, self.dt), dtype=torch.uint8,
+                               device=dev)
+        nb = E * R
+        self.counts = torch.empty(nb, dtype=torch.int32, device=dev)
+        self.offsets = torch.empty(nb + 1, dtype=torch.int32, device=dev)
+        self.src_row = torch.empty(N, dtype=torch.int32, device=dev)
+        self.dst_pos = torch.empty(T, k, dtype=torch.int32, device=dev)
+        self.x_perm = torch.empty(N, d, dtype=x.dtype, device=dev)
+        self.dws = torch.empty(M.ep_dispatch_workspace_size(T, E, k, R), dtype=torch.uint8,
+                               device=dev)
+        if R > 1:
+            self.x_em = torch.empty_like(self.x_perm)
+            self.cem = torch.empty(E, dtype=torch.int32, device=dev)
+            self.oem = torch.empty(E + 1, dtype=torch.int32, device=dev)
+            self.perm = torch.empty(N, dtype=torch.int32, device=dev)
+            self.pinv = torch.empty(N, dtype=torch.int32, device=dev)
+            self.gws = torch.empty(M.regroup_workspace_size(R, R, E // R), dtype=torch.uint8,
+                                   device=dev)
+        self.y = torch.empty(N, d, dtype=x.dtype, device=dev)
+        self.sws = torch.empty(M.grouped_swiglu_workspace_size(N, d, h, E, self.dt),
+                               dtype=torch.uint8, device=dev)
+        self.out = torch.empty(T, d, dtype=x.dtype, device=dev)
+        self.fws = torch.empty(M.forward_workspace_size(T, d, E, k, h, R, self.dt),
+                               dtype=torch.uint8, device=dev)
+        self.fout = torch.empty_like(self.out)
+        self.stages = (["router", "dispatch"] + (["regroup"] if R > 1 else [])
+                       + ["grouped_swiglu", "combine"])
+
+    def forward(self, x=None, out=None):
+        c, M = self.cfg, self.M
+        M.moe_forward(self.x if x is None else x, self.wr, None, self.w1, self.w3, self.w2, c.T,
+                      c.d, c.E, c.top_k, c.h, M.MOE_SCORE_SOFTMAX, c.renormalize, c.ep_ranks,
+                      self.dt, self.fout if out is None else out, None, None, None, None,
+                      self.fws)
+
+    def staged(self, stream, ev=None):
+        c, M = self.cfg, self.M
+        T, d, E, k, h, R, N, dt = c.T, c.d, c.E, c.top_k, c.h, c.ep_ranks, c.N, self.dt
+
+        def mark(i):
+            if ev is not None:
+                ev[i].record(stream)
+        mark(0)
+        M.moe_router_topk(self.x, self.wr, None, T, d, E, k, M.MOE_SCORE_SOFTMAX,
+                          c.renormalize, dt, None, self.idx, self.w, None, self.rws)
+        mark(1)
+        if R == 1:
+            M.moe_dispatch(self.x, self.idx, T, d, E, k, dt, self.counts, self.offsets,
+                           self.src_row, self.dst_pos, self.x_perm, self.dws)
+        else:
+            M.moe_ep_dispatch_rank_major(self.x, self.idx, T, d, E, k, R, dt, self.counts,
+                                         self.offsets, self.src_row, self.dst_pos, self.x_perm,
+                                         self.dws)
+        mark(2)
+        i = 2
+        xe, off, rmap = self.x_perm, self.offsets, None
+        if R > 1:
+            M.moe_ep_local_regroup(self.x_perm, self.counts, R, R, E // R, N, d, dt, self.x_em,
+                                   self.cem, self.oem, self.perm, self.pinv, self.gws)
+            i += 1
+            mark(i)
+            xe, off, rmap = self.x_em, self.oem, self.pinv
+        M.moe_grouped_swiglu(xe, off, self.w1, self.w3, self.w2, None, N, d, h, E, dt, self.y,
+                             self.sws)
+        mark(i + 1)
+        M.moe_combine(self.y, self.dst_pos, rmap, self.w, T, d, N, k, dt, self.out)
+        mark(i + 2)
+
+
+def timed_forward(layer, stream, flush, steps):
+    """CUDA-event time (ms) of each moe_forward step; L2 flushed between
+    steps, outside the events."""
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    torch.cuda.synchronize()
+    for a_ev, b_ev in ev:
+        a_ev.record(stream)
+        layer.forward()
+        b_ev.record(stream)
+        flush.zero_()
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in ev]
+
+
+def timed_staged(layer, stream, flush, steps):
+    """Per-stage CUDA-event times (ms lists) of the entry-point sequence and
+    the whole staged step; L2 flushed between steps."""
+    n = len(layer.stages) + 1
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(n)] for _ in range(steps)]
+    torch.cuda.synchronize()
+    for s in range(steps):
+        layer.staged(stream, events[s])
+        flush.zero_()
+    torch.cuda.synchronize()
+    per_stage = {nm: [ev[i].elapsed_time(ev[i + 1]) for ev in events]
+                 for i, nm in enumerate(layer.stages)}
+    whole = [ev[0].elapsed_time(ev[-1]) for ev in events]
+    return per_stage, whole
+
+
+def gemm_views(cfg, sw_ms, pk):
+    """The grouped SwiGLU against HBM (its algorithmic bytes) and against the
+    bf16 tensor peak, burst and sustained."""
+    flops = cfg.gemm_flops()
+    alg_bytes = swiglu_algorithmic_bytes(cfg)
+    tflops = flops / (sw_ms / 1e3) / 1e12
+    gbs = alg_bytes / (sw_ms / 1e3) / 1e9
+    return {"launch_us": 1e3 * sw_ms, "algorithmic_bytes_per_launch": alg_bytes,
+            "algorithmic_flops_per_launch": flops,
+            "hbm": {"achieved_GBps": gbs, "frac": gbs / pk["hbm_gbs"]},
+            "tensor_burst": {"achieved_TFLOPs": tflops, "frac": tflops / pk["bf16_tflops"]},
+            "tensor_sustained": {"achieved_TFLOPs": tflops,
+                                 "frac": tflops / pk["bf16_tflops_sustained"]}}
+
+
+def stage_report(cfg, stage_ms, pk):
+    return {n: {"us": 1e3 * stage_ms[n], "algorithmic_bytes": b,
+                "GBps": b / (stage_ms[n] * 1e-3) / 1e9,
+                "frac": b / (stage_ms[n] * 1e-3) / 1e9 / pk["hbm_gbs"]}
+            for n, b in stage_algorithmic_bytes(cfg).items() if n in stage_ms}
+
+
+def other_config(M, idx, dev, stream, flush, pk, steps=10, warmup=3):
+    """One other workload: moe_forward and the staged entry points, timed
+    like the headline (L2 flushed between steps)."""
+    cfg = W.config(idx)
+    layer = Layer(M, cfg, dev)
+    for _ in range(warmup):
+        layer.forward()
+        flush.zero_()
+        layer.staged(stream)
+        flush.zero_()
+    fwd = timed_forward(layer, stream, flush, steps)
+    per_stage, _ = timed_staged(layer, stream, flush, steps)
+    fwd_ms = statistics.median(fwd)
+    stage_ms = {n: statistics.median(v) for n, v in per_stage.items()}
+    rec = {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "E": cfg.E, "top_k": cfg.top_k,
+           "h": cfg.h, "dtype": cfg.dtype, "moe_forward_us": 1e3 * fwd_ms,
+           "tokens_per_s": cfg.T / (fwd_ms / 1e3),
+           "forward_matches_staged": bool(torch.equal(layer.fout, layer.out)),
+           "grouped_swiglu": gemm_views(cfg, stage_ms["grouped_swiglu"], pk),
+           "stages": stage_report(cfg, stage_ms, pk)}
+    if cfg.T < 1024:
+        # weight-bandwidth view: every touched expert's three matrices once
+        touched = int((layer.counts.view(cfg.ep_ranks, -1).sum(0) > 0).sum().item()
+                      if cfg.ep_ranks > 1 else (layer.counts > 0).sum().item())
+        wbytes = touched * 3 * cfg.d * cfg.h * (2 if cfg.dtype == "bf16" else 4)
+        rec["touched_weight_bytes"] = wbytes
+        rec["weights_GBps"] = wbytes / (stage_ms["grouped_swiglu"] * 1e-3) / 1e9
+        rec["weights_frac_of_hbm"] = rec["weights_GBps"] / pk["hbm_gbs"]
+    del layer
+    torch.cuda.empty_cache()
+    return rec
+
+
 def run_ours(args, ws, rank, local):
     import routing_dispatch_grouped_topk_b200 as M
     M.lib()  # fails loudly if the CUDA library is missing
     cfg = W.config(args.config)
     T, d, E, k, h, R = cfg.T, cfg.d, cfg.E, cfg.top_k, cfg.h, cfg.ep_ranks
-    N = T * k
     dev = torch.device("cuda", local)
-    lay = W.make_layer(cfg, dev)
-    if rank:   # independent token batch per rank
-        lay["x"] = W.make_layer(rank_workload(cfg, rank), dev, experts=False)["x"]
-    x, wr, w1, w3, w2 = lay["x"], lay["w_router"], lay["w1"], lay["w3"], lay["w2"]
-    dt = M.MOE_BF16 if cfg.dtype == "bf16" else M.MOE_F32
     stream = torch.cuda.current_stream()
-
-    # buffers of the four stages (the same sequence moe_forward runs)
-    idx = torch.empty(T, k, dtype=torch.int32, device=dev)
-    w = torch.empty(T, k, dtype=torch.float32, device=dev)
-    rws = torch.empty(M.router_workspace_size(T, d, E, dt), dtype=torch.uint8, device=dev)
-    nb = E * R
-    counts = torch.empty(nb, dtype=torch.int32, device=dev)
-    offsets = torch.empty(nb + 1, dtype=torch.int32, device=dev)
-    src_row = torch.empty(N, dtype=torch.int32, device=dev)
-    dst_pos = torch.empty(T, k, dtype=torch.int32, device=dev)
-    x_perm = torch.empty(N, d, dtype=x.dtype, device=dev)
-    dws = torch.empty(M.ep_dispatch_workspace_size(T, E, k, R), dtype=torch.uint8, device=dev)
-    if R > 1:
-        x_em = torch.empty_like(x_perm)
-        cem = torch.empty(E, dtype=torch.int32, device=dev)
-        oem = torch.empty(E + 1, dtype=torch.int32, device=dev)
-        perm = torch.empty(N, dtype=torch.int32, device=dev)
-        pinv = torch.empty(N, dtype=torch.int32, device=dev)
-        gws = torch.empty(M.regroup_workspace_size(R, R, E // R), dtype=torch.uint8, device=dev)
-    y = torch.empty(N, d, dtype=x.dtype, device=dev)
-    sws = torch.empty(M.grouped_swiglu_workspace_size(N, d, h, E, dt), dtype=torch.uint8,
-                      device=dev)
-    out = torch.empty(T, d, dtype=x.dtype, device=dev)
+    layer = Layer(M, cfg, dev, rank)
+    x, out = layer.x, layer.out
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
-
-    stages = ["router", "dispatch"] + (["regroup"] if R > 1 else []) + ["grouped_swiglu",
-                                                                        "combine"]
-
-    def step(ev=None):
-        def mark(i):
-            if ev is not None:
-                ev[i].record(stream)
-        mark(0)
-        M.moe_router_topk(x, wr, None, T, d, E, k, M.MOE_SCORE_SOFTMAX, cfg.renormalize, dt, None,
-                          idx, w, None, rws)
-        mark(1)
-        if R == 1:
-            M.moe_dispatch(x, idx, T, d, E, k, dt, counts, offsets, src_row, dst_pos, x_perm, dws)
-        else:
-            M.moe_ep_dispatch_rank_major(x, idx, T, d, E, k, R, dt, counts, offsets, src_row,
-                                         dst_pos, x_perm, dws)
-        mark(2)
-        i = 2
-        xe, off, rmap = x_perm, offsets, None
-        if R > 1:
-            M.moe_ep_local_regroup(x_perm, counts, R, R, E // R, N, d, dt, x_em, cem, oem, perm,
-                                   pinv, gws)
-            i += 1
-            mark(i)
-            xe, off, rmap = x_em, oem, pinv
-        M.moe_grouped_swiglu(xe, off, w1, w3, w2, None, N, d, h, E, dt, y, sws)
-        mark(i + 1)
-        M.moe_combine(y, dst_pos, rmap, w, T, d, N, k, dt, out)
-        mark(i + 2)
-
-    nmarks = len(stages) + 1
-    fws = torch.empty(M.forward_workspace_size(T, d, E, k, h, R, dt), dtype=torch.uint8,
-                      device=dev)
-    fout = torch.empty_like(out)
-
-    def forward_step():
-        M.moe_forward(x, wr, None, w1, w3, w2, T, d, E, k, h, M.MOE_SCORE_SOFTMAX,
-                      cfg.renormalize, R, dt, fout, None, None, None, None, fws)
 
     if args.profile:
         # Kernel order per staged step (R = 1): router GEMM, router top-k,
         # dispatch histogram, column scan, scatter, GEMM1, GEMM2, combine.
         for _ in range(2):
-            step()
-        forward_step()
+            layer.staged(stream)
+        layer.forward()
         torch.cuda.synchronize()
         return
 
@@ -363,9 +481,9 @@ def run_ours(args, ws, rank, local):
     t_warm = time.perf_counter()
     n_warm = 0
     while n_warm < args.warmup or time.perf_counter() - t_warm < 1.5:
-        forward_step()
+        layer.forward()
         flush.zero_()
-        step()
+        layer.staged(stream)
         flush.zero_()
         n_warm += 1
         if n_warm % 16 == 0:
@@ -373,42 +491,25 @@ def run_ours(args, ws, rank, local):
     torch.cuda.synchronize()
 
     # Timed region 1 (headline): the public moe_forward, one call per step.
-    fwd_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(args.steps)]
     barrier(ws)
-    torch.cuda.synchronize()
-    for a_ev, b_ev in fwd_ev:
-        a_ev.record(stream)
-        forward_step()
-        b_ev.record(stream)
-        flush.zero_()          # L2 flush between steps, outside the step's events
-    torch.cuda.synchronize()
+    fwd_ms = timed_forward(layer, stream, flush, args.steps)
     barrier(ws)
-    total_ms = sum(a_ev.elapsed_time(b_ev) for a_ev, b_ev in fwd_ev)
-    total_ms_max = max_over_ranks(total_ms, ws)
+    total_ms_max = max_over_ranks(sum(fwd_ms), ws)
     ms_per_step = total_ms_max / args.steps
     value = job_tokens_per_s(T, ws, args.steps, total_ms_max)
 
     # Timed region 2 (breakdown): the same layer as the sequence of entry
     # points, each bracketed by events; gives the grouped-GEMM duration.
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(nmarks)]
-              for _ in range(args.steps)]
     barrier(ws)
-    torch.cuda.synchronize()
-    for s in range(args.steps):
-        step(events[s])
-        flush.zero_()
-    torch.cuda.synchronize()
+    per_stage, staged_whole = timed_staged(layer, stream, flush, args.steps)
     barrier(ws)
-    clocks = sampler.stop() if rank == 0 else None
-    per_stage = {n: [] for n in stages}
-    for ev in events:
-        for i, n in enumerate(stages):
-            per_stage[n].append(ev[i].elapsed_time(ev[i + 1]))
-    staged_ms_per_step = sum(ev[0].elapsed_time(ev[-1]) for ev in events) / args.steps
-    forward_matches_staged = bool(torch.equal(fout, out))
+    staged_ms_per_step = statistics.mean(staged_whole)
+    forward_matches_staged = bool(torch.equal(layer.fout, out))
 
-    # e2e: host buffers through the public moe_forward call, copies included
+    # e2e through the public moe_forward with host buffers: every step copies
+    # its input from pinned host memory, runs the layer and copies the output
+    # back, in sequence on one stream; L2 flushed between steps (outside the
+    # events).  This per-call cost is the headline e2e value.
     x_host = x.cpu().pin_memory()
     out_host = torch.empty(T, d, dtype=x.dtype).pin_memory()
     x_dev = torch.empty_like(x)
@@ -416,15 +517,14 @@ def run_ours(args, ws, rank, local):
 
     def e2e_step():
         x_dev.copy_(x_host, non_blocking=True)
-        M.moe_forward(x_dev, wr, None, w1, w3, w2, T, d, E, k, h, M.MOE_SCORE_SOFTMAX,
-                      cfg.renormalize, R, dt, out_dev, None, None, None, None, fws)
+        layer.forward(x_dev, out_dev)
         out_host.copy_(out_dev, non_blocking=True)
 
     for _ in range(args.warmup):
         e2e_step()
         flush.zero_()
     torch.cuda.synchronize()
-    e2e_ms = []
+    e2e_ev = []
     barrier(ws)
     for _ in range(args.steps):
         a = torch.cuda.Event(enable_timing=True)
@@ -433,10 +533,10 @@ def run_ours(args, ws, rank, local):
         e2e_step()
         b.record(stream)
         flush.zero_()
-        e2e_ms.append((a, b))
+        e2e_ev.append((a, b))
     torch.cuda.synchronize()
     barrier(ws)
-    e2e_seq_total = max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ms), ws)
+    e2e_seq_total = max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ev), ws)
     e2e_seq_value = job_tokens_per_s(T, ws, args.steps, e2e_seq_total)
     # the e2e output equals the device-resident step's output
     e2e_match = bool(torch.equal(out_host.to(dev), out))
@@ -444,8 +544,9 @@ def run_ours(args, ws, rank, local):
     # Pipelined e2e (a stream of batches): the H2D copy of step i+1 and the
     # D2H copy of step i-1 run on copy streams while step i's forward runs;
     # every step still copies its input in and its output out.  Double
-    # buffers on the device, events order the reuse.  The working set (the
-    # expert weights) is larger than L2, so no flush is inserted.
+    # buffers on the device, events order the reuse.  No L2 flush between
+    # steps here (the copies run concurrently with the forward), so this is
+    # a sub-key, not the e2e value.
     xb = [torch.empty_like(x) for _ in range(2)]
     ob = [torch.empty_like(out) for _ in range(2)]
     oh = [torch.empty(T, d, dtype=x.dtype).pin_memory() for _ in range(2)]
@@ -470,9 +571,7 @@ def run_ours(args, ws, rank, local):
                 stream.wait_event(h2d[j])
                 if j >= 2:
                     stream.wait_event(d2h[j - 2])     # out buffer j%2 copied out
-                M.moe_forward(xb[j % 2], wr, None, w1, w3, w2, T, d, E, k, h,
-                              M.MOE_SCORE_SOFTMAX, cfg.renormalize, R, dt, ob[j % 2], None, None,
-                              None, None, fws)
+                layer.forward(xb[j % 2], ob[j % 2])
                 fwd[j].record(stream)
                 with torch.cuda.stream(s_out):       # output of step j
                     s_out.wait_event(fwd[j])
@@ -490,41 +589,39 @@ def run_ours(args, ws, rank, local):
     pipelined(args.steps, t0e, t1e)
     torch.cuda.synchronize()
     barrier(ws)
-    e2e_total = max_over_ranks(t0e.elapsed_time(t1e), ws)
-    e2e_value = job_tokens_per_s(T, ws, args.steps, e2e_total)
+    e2e_pipe_total = max_over_ranks(t0e.elapsed_time(t1e), ws)
+    e2e_pipe_value = job_tokens_per_s(T, ws, args.steps, e2e_pipe_total)
     e2e_match = e2e_match and bool(torch.equal(oh[(args.steps - 1) % 2].to(dev), out))
+    clocks = sampler.stop() if rank == 0 else None
 
     if rank != 0:
         return
     pk = peaks()
-    sw_ms = statistics.mean(per_stage["grouped_swiglu"])
-    flops = cfg.gemm_flops()
-    alg_bytes = swiglu_algorithmic_bytes(cfg)
-    tflops = flops / (sw_ms / 1e3) / 1e12
-    gbs = alg_bytes / (sw_ms / 1e3) / 1e9
-    # The grouped SwiGLU sits near the ridge; report the binding roofline
-    # (the larger lower bound on time) and the other one beside it.
+    stage_ms = {n: statistics.mean(v) for n, v in per_stage.items()}
+    sw_ms = stage_ms["grouped_swiglu"]
+    views = gemm_views(cfg, sw_ms, pk)
+    flops, alg_bytes = views["algorithmic_flops_per_launch"], views["algorithmic_bytes_per_launch"]
+    # The grouped SwiGLU is timed as one launch pair inside a ~ms step (not
+    # a seconds-long loop): the burst peaks apply.  Its binding roofline is
+    # the larger lower bound on its time; the other views stand beside it.
     t_mem = alg_bytes / (pk["hbm_gbs"] * 1e9)
-    t_flop = flops / (pk["bf16_tflops_sustained"] * 1e12)
+    t_flop = flops / (pk["bf16_tflops"] * 1e12)
     traffic = profiled_traffic("grouped_swiglu", cfg.name)
-    tensor_view = {"achieved": tflops, "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                   "frac": tflops / pk["bf16_tflops_sustained"],
-                   "peak_kind": f"bf16 sustained, {pk['source']}",
-                   "algorithmic_flops_per_launch": flops}
-    hbm_view = {"achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "frac": gbs / pk["hbm_gbs"], "peak_kind": f"HBM copy, {pk['source']}",
-                "algorithmic_bytes_per_launch": alg_bytes}
-    main_view, other = (hbm_view, tensor_view) if t_mem >= t_flop else (tensor_view, hbm_view)
-    roofline = {"kernel": "moe_grouped_swiglu (GEMM1 w1|w3 + SiLU*up, GEMM2 w2)",
-                "bound": "hbm" if t_mem >= t_flop else "tensor",
-                "achieved": main_view["achieved"], "peak": main_view["peak"],
-                "unit": main_view["unit"], "frac": main_view["frac"],
+    if t_mem >= t_flop:
+        main = {"bound": "hbm", "achieved": views["hbm"]["achieved_GBps"],
+                "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": views["hbm"]["frac"],
+                "peak_kind": f"HBM copy, {pk['source']}"}
+    else:
+        main = {"bound": "tensor", "achieved": views["tensor_burst"]["achieved_TFLOPs"],
+                "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": views["tensor_burst"]["frac"],
+                "peak_kind": f"bf16 dense burst, {pk['source']}"}
+    roofline = {"kernel": "moe_grouped_swiglu (GEMM1 w1|w3 + SiLU*up, GEMM2 w2)", **main,
                 "traffic": traffic, "launch_ms": sw_ms,
                 "algorithmic_bytes_per_launch": alg_bytes,
                 "algorithmic_flops_per_launch": flops,
-                "peak_kind": main_view["peak_kind"],
-                "other_bound": other}
-    stage_ms = {n: statistics.mean(v) for n, v in per_stage.items()}
+                "views": {"hbm": views["hbm"], "tensor_burst": views["tensor_burst"],
+                          "tensor_sustained": views["tensor_sustained"]}}
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
@@ -534,26 +631,35 @@ def run_ours(args, ws, rank, local):
                    "l2": "flushed between steps (256 MB write, outside step events)",
                    "inputs": "seeded synthetic, resident in HBM"},
         "roofline": roofline,
-        "grouped_gemm_tflops": tflops,
-        "grouped_gemm_frac_of_tensor_peak": tflops / pk["bf16_tflops_sustained"],
+        "grouped_gemm_tflops": views["tensor_burst"]["achieved_TFLOPs"],
+        "grouped_gemm_frac_of_tensor_peak": views["tensor_burst"]["frac"],
+        "grouped_gemm_frac_of_tensor_peak_sustained": views["tensor_sustained"]["frac"],
         "stage_ms": stage_ms,
-        "stage_hbm": {n: {"GBps": b / (stage_ms[n] * 1e-3) / 1e9,
-                          "frac": b / (stage_ms[n] * 1e-3) / 1e9 / pk["hbm_gbs"],
-                          "algorithmic_bytes": b}
-                      for n, b in stage_algorithmic_bytes(cfg).items() if n in stage_ms},
+        "stage_hbm": stage_report(cfg, stage_ms, pk),
         "staged_ms_per_step": staged_ms_per_step,
         "forward_matches_staged": forward_matches_staged,
         "copies_per_s": value * k,
-        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": x.numel() * x.element_size(),
+        "e2e": {"value": e2e_seq_value, "unit": UNIT,
+                "h2d_bytes_per_step": x.numel() * x.element_size(),
                 "d2h_bytes_per_step": out.numel() * out.element_size(),
-                "mode": "pipelined: step i+1's H2D and step i-1's D2H overlap step i's "
-                        "moe_forward (pinned host buffers, two device buffers)",
-                "sequential_value": e2e_seq_value,
+                "mode": "sequential: every step copies x from pinned host memory, runs "
+                        "moe_forward and copies out back, on one stream; L2 flushed between "
+                        "steps",
+                "pipelined_value": e2e_pipe_value,
+                "pipelined_mode": "step i+1's H2D and step i-1's D2H overlap step i's "
+                                  "moe_forward on copy streams (two device buffers); no L2 "
+                                  "flush between steps",
                 "output_matches_device_step": e2e_match},
-        "gpu_launches": args.steps * (sum(LAUNCHES_PER_STEP.values()) + (2 if R > 1 else 0)),
+        "gpu_launches": args.steps * forward_launches(cfg),
         "gpu_launches_note": "kernels of libmoe in timed region 1 (moe_forward per step)",
         "clocks": clocks,
+        "peaks": pk,
     }
+    if ws == 1 and not args.no_other_configs:
+        del layer
+        torch.cuda.empty_cache()
+        line["other_configs"] = [other_config(M, i, dev, stream, flush, pk)
+                                 for i in range(len(W.CONFIGS)) if i != args.config]
     if not args.no_cpu_baseline and ws == 1:
         line["cpu_baseline"] = cpu_baseline(cfg, tokens=args.cpu_tokens)
     print(json.dumps(line), flush=True)
@@ -748,11 +854,15 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--config", type=int, default=1, help="workload index (default: the "
-                    "Qwen3-30B-A3B-shaped layer, T=4096)")
-    ap.add_argument("--cpu-tokens", type=int, default=256)
-    ap.add_argument("--ref-tokens", type=int, default=128)
+    ap.add_argument("--config", type=int, default=4, help="headline workload index (default: "
+                    "the gpt-oss-120b-shaped EP8 layer, T=8192, the largest single-GPU one)")
+    ap.add_argument("--cpu-tokens", type=int, default=64,
+                    help="tokens of the fp64 oracle's CPU-baseline sample")
+    ap.add_argument("--ref-tokens", type=int, default=8,
+                    help="tokens of the oracle per step of the reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-other-configs", action="store_true",
+                    help="skip the per-workload measurements of the other configs")
     ap.add_argument("--training", action="store_true",
                     help="time the training step (forward + backward) instead")
     ap.add_argument("--profile", action="store_true",

@@ -226,9 +226,11 @@ MOE_API moe_status_t moe_dispatch(const void* x, const int32_t* topk_idx, int T,
  * (for E = 128 about a million tokens) return MOE_ERR_UNSUPPORTED with a
  * message and launch nothing.  It allocates nothing: no cudaMalloc,
  * cudaFree or allocating library call.
- * The first call on a device looks the array's device address up
- * (cudaGetSymbolAddress) and caches it; make that first call before any
- * stream capture.  All calls share the array and it keeps the last call's
+ * Each call made outside stream capture looks the array's device address
+ * up (cudaGetSymbolAddress, with the device current), so a device reset or a
+ * re-created context is followed; a call on a capturing stream uses the
+ * address of the last lookup on that device, so make one call on the device
+ * before any capture.  All calls share the array and it keeps the last call's
  * contents (the status word is cleared at the start of each call), so calls
  * that overlap on the GPU -- on different streams, or from several host
  * threads -- race; serialise them.  The device status word is not exposed:

@@ -130,6 +130,35 @@ moe_status_t check_router(const void* x, const void* w_router, const float* logi
   return MOE_OK;
 }
 
+}  // namespace
+
+// Argument rules of the dispatch entry points (moe_dispatch,
+// moe_ep_dispatch_rank_major, moe_dispatch_noalloc): one copy, so that every
+// entry point rejects the same arguments with the same status and text.
+moe_status_t check_dispatch_args(const void* x, const int32_t* topk_idx, int T, int d, int E,
+                                 int top_k, int R, moe_dtype_t dt, const int32_t* counts,
+                                 const int32_t* offsets, const int32_t* src_row,
+                                 const int32_t* dst_pos, const void* x_perm) {
+  if (moe_status_t st = check_dtype(dt)) return st;
+  MOE_CHECK_ARG(T >= 0, "T must be >= 0");
+  MOE_CHECK_ARG(E >= 1 && E <= kMaxExperts, "E=%d must be in [1, %d]", E, kMaxExperts);
+  MOE_CHECK_ARG(top_k >= 1 && top_k <= std::min(E, kMaxTopK), "top_k=%d out of range", top_k);
+  MOE_CHECK_ARG(R >= 1 && E % R == 0 && E * R <= kMaxBins, "R=%d must divide E and E*R <= %d", R,
+                kMaxBins);
+  MOE_CHECK_ARG(counts && offsets, "counts and offsets are required");
+  if (T > 0) {
+    MOE_CHECK_ARG(topk_idx && src_row && dst_pos, "topk_idx, src_row, dst_pos are required");
+    if (x_perm) {
+      MOE_CHECK_ARG(x != nullptr, "x is required when x_perm is given");
+      MOE_CHECK_ARG(aligned16(x) && aligned16(x_perm), "x / x_perm must be 16-byte aligned");
+      if (moe_status_t st = check_rows(d, dt, "dispatch")) return st;
+    }
+  }
+  return MOE_OK;
+}
+
+namespace {
+
 RouterOptions kernel_options(const moe_router_options_t& o) {
   RouterOptions k;
   k.sigmoid = o.score == MOE_SCORE_SIGMOID;
@@ -490,21 +519,9 @@ static moe_status_t dispatch_common(const void* x, const int32_t* topk_idx, int 
                                     int top_k, int R, moe_dtype_t dt, int32_t* counts,
                                     int32_t* offsets, int32_t* src_row, int32_t* dst_pos,
                                     void* x_perm, void* ws, size_t ws_bytes, void* stream) {
-  if (moe_status_t st = check_dtype(dt)) return st;
-  MOE_CHECK_ARG(T >= 0, "T must be >= 0");
-  MOE_CHECK_ARG(E >= 1 && E <= kMaxExperts, "E=%d must be in [1, %d]", E, kMaxExperts);
-  MOE_CHECK_ARG(top_k >= 1 && top_k <= std::min(E, kMaxTopK), "top_k=%d out of range", top_k);
-  MOE_CHECK_ARG(R >= 1 && E % R == 0 && E * R <= kMaxBins, "R=%d must divide E and E*R <= %d", R,
-                kMaxBins);
-  MOE_CHECK_ARG(counts && offsets, "counts and offsets are required");
-  if (T > 0) {
-    MOE_CHECK_ARG(topk_idx && src_row && dst_pos, "topk_idx, src_row, dst_pos are required");
-    if (x_perm) {
-      MOE_CHECK_ARG(x != nullptr, "x is required when x_perm is given");
-      MOE_CHECK_ARG(aligned16(x) && aligned16(x_perm), "x / x_perm must be 16-byte aligned");
-      if (moe_status_t st = check_rows(d, dt, "dispatch")) return st;
-    }
-  }
+  if (moe_status_t st = check_dispatch_args(x, topk_idx, T, d, E, top_k, R, dt, counts, offsets,
+                                            src_row, dst_pos, x_perm))
+    return st;
   MOE_CHECK_ARG(ws != nullptr, "ws is required");
   const DispatchPlan p = make_dispatch_plan(T, E, top_k, R);
   const size_t need = kStatusBytes + dispatch_ws_bytes(p);

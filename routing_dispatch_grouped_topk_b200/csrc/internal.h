@@ -40,6 +40,12 @@ struct DispatchPlan {
 };
 DispatchPlan make_dispatch_plan(int T, int E, int top_k, int R);
 size_t dispatch_ws_bytes(const DispatchPlan& p);
+// Host-side argument rules shared by every dispatch entry point (returns
+// MOE_OK or MOE_ERR_INVALID_ARG with the text for moe_last_error set).
+moe_status_t check_dispatch_args(const void* x, const int32_t* topk_idx, int T, int d, int E,
+                                 int top_k, int R, moe_dtype_t dt, const int32_t* counts,
+                                 const int32_t* offsets, const int32_t* src_row,
+                                 const int32_t* dst_pos, const void* x_perm);
 
 // Scoring options of the top-k kernel (moe_router_options_t without the
 // host-only fields).  sigmoid: score function; scale: route_scale; bias:

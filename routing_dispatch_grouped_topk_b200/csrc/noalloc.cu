@@ -26,14 +26,21 @@ void* g_scratch_addr[64] = {nullptr};
 
 // Device address of g_dispatch_scratch on the current device.  In host code
 // the symbol itself is only a host-side handle, so the address is looked up
-// once per device with that device current.
-cudaError_t scratch_address(void** out) {
+// with that device current.  Outside stream capture it is looked up on every
+// call (a device reset or a re-created primary context moves the array);
+// while `s` is being captured no lookup is made and the address of the last
+// lookup on this device is used (the first call on a device must therefore
+// come before any capture).
+cudaError_t scratch_address(cudaStream_t s, void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  e = cudaStreamIsCapturing(s, &cap);
+  if (e != cudaSuccess) return e;
   std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (!g_scratch_addr[dev]) {
+  if (cap == cudaStreamCaptureStatusNone || !g_scratch_addr[dev]) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_dispatch_scratch);
     if (e != cudaSuccess) return e;
@@ -52,26 +59,10 @@ extern "C" moe_status_t moe_dispatch_noalloc(const void* x, const int32_t* topk_
                                              int E, int top_k, moe_dtype_t dt, int32_t* counts,
                                              int32_t* offsets, int32_t* src_row,
                                              int32_t* dst_pos, void* x_perm, void* stream) {
-  if (dt != MOE_F32 && dt != MOE_BF16) {
-    set_last_error("dt must be MOE_F32 or MOE_BF16");
-    return MOE_ERR_INVALID_ARG;
-  }
-  if (T < 0 || E < 1 || E > kMaxExperts || top_k < 1 || top_k > std::min(E, kMaxTopK)) {
-    set_last_error("bad sizes T=%d E=%d top_k=%d", T, E, top_k);
-    return MOE_ERR_INVALID_ARG;
-  }
-  if (!counts || !offsets || (T > 0 && (!topk_idx || !src_row || !dst_pos))) {
-    set_last_error("counts, offsets, topk_idx, src_row, dst_pos are required");
-    return MOE_ERR_INVALID_ARG;
-  }
-  const size_t esz = dt == MOE_BF16 ? 2 : 4;
-  if (T > 0 && x_perm) {
-    if (!x || d < 1 || (static_cast<size_t>(d) * esz) % 16 != 0 ||
-        (reinterpret_cast<uintptr_t>(x) & 15u) || (reinterpret_cast<uintptr_t>(x_perm) & 15u)) {
-      set_last_error("x / x_perm: 16-byte aligned rows of a whole number of 16-byte vectors");
-      return MOE_ERR_INVALID_ARG;
-    }
-  }
+  // the same argument rules, status codes and texts as moe_dispatch
+  if (moe_status_t st = check_dispatch_args(x, topk_idx, T, d, E, top_k, 1, dt, counts, offsets,
+                                            src_row, dst_pos, x_perm))
+    return st;
   const DispatchPlan p = make_dispatch_plan(T, E, top_k, 1);
   const size_t need = kNoAllocStatusBytes + dispatch_ws_bytes(p);
   if (need > MOE_NOALLOC_SCRATCH_BYTES) {
@@ -80,13 +71,13 @@ extern "C" moe_status_t moe_dispatch_noalloc(const void* x, const int32_t* topk_
                    T, E, need, MOE_NOALLOC_SCRATCH_BYTES);
     return MOE_ERR_UNSUPPORTED;
   }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
   void* base = nullptr;
-  cudaError_t e = scratch_address(&base);
+  cudaError_t e = scratch_address(s, &base);
   if (e != cudaSuccess) {
     set_last_error("moe_dispatch_noalloc: cudaGetSymbolAddress failed: %s", cudaGetErrorString(e));
     return MOE_ERR_CUDA;
   }
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   int* status = static_cast<int*>(base);
   e = cudaMemsetAsync(status, 0, sizeof(int), s);   // the array keeps the last call's bytes
   if (e == cudaSuccess)

@@ -1,10 +1,18 @@
 """Host-only checks of the C ABI: the library loads, exports every function
 include/moe.h declares, and rejects bad arguments before touching the GPU.
-No kernel is launched here (these run without a GPU)."""
+No kernel is launched here.
+
+The argument checks pass made-up device addresses: every call must be
+rejected on the host.  So that a regressed check cannot turn into a launch
+on those addresses, the checks only run in a process that sees no CUDA
+device; where this process sees one, the module re-runs itself in a child
+process with CUDA_VISIBLE_DEVICES="" (a launch there fails with "no
+device" instead of touching memory)."""
 import ctypes
 import os
 import re
 import subprocess
+import sys
 
 import pytest
 
@@ -12,12 +20,35 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "moe.h")
 
 
+def _device_visible() -> bool:
+    if os.environ.get("CUDA_VISIBLE_DEVICES") == "":
+        return False
+    try:
+        import torch
+        return torch.cuda.is_available()
+    except Exception:
+        return False
+
+
 @pytest.fixture(scope="module")
 def L():
+    if _device_visible():
+        pytest.skip("argument checks with made-up addresses run in a child process without a "
+                    "CUDA device (test_checks_in_a_process_without_a_device)")
     from routing_dispatch_grouped_topk_b200 import build
     build.build()
     import routing_dispatch_grouped_topk_b200 as m
     return m.lib()
+
+
+def test_checks_in_a_process_without_a_device():
+    if not _device_visible():
+        pytest.skip("this process sees no CUDA device: the checks run here directly")
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    r = subprocess.run([sys.executable, "-m", "pytest", os.path.abspath(__file__), "-q", "-x",
+                        "-p", "no:cacheprovider", "-m", "not gpu"], cwd=ROOT, env=env,
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stdout[-4000:] + r.stderr[-2000:]
 
 
 def declared_functions():
@@ -223,3 +254,45 @@ def test_router_backward_gate_rules(L):
                                  None) == 2
     assert L.moe_router_backward(p, p, p, p, p, 4, 96, 12, 2, None, 0, p, None, None, p, 16,
                                  None) == 4
+
+
+DISPATCH_BAD = [
+    dict(dt=7), dict(T=-1), dict(E=0), dict(E=513), dict(top_k=0), dict(top_k=9, E=8),
+    dict(top_k=17, E=64), dict(counts=None), dict(offsets=None), dict(idx=None),
+    dict(src_row=None), dict(dst_pos=None), dict(x=None), dict(x=18), dict(x_perm=24),
+    dict(d=60), dict(d=0),
+]
+
+
+@pytest.mark.parametrize("case", DISPATCH_BAD)
+def test_dispatch_entry_points_share_their_argument_rules(L, case):
+    """moe_dispatch and moe_dispatch_noalloc reject the same arguments with
+    the same status and the same text (one copy of the rules)."""
+    a = dict(x=256, idx=256, T=8, d=64, E=8, top_k=2, dt=1, counts=256, offsets=256,
+             src_row=256, dst_pos=256, x_perm=512)
+    a.update(case)
+
+    def p(v):
+        return None if v is None else ctypes.c_void_p(v)
+    r1 = L.moe_dispatch(p(a["x"]), p(a["idx"]), a["T"], a["d"], a["E"], a["top_k"], a["dt"],
+                        p(a["counts"]), p(a["offsets"]), p(a["src_row"]), p(a["dst_pos"]),
+                        p(a["x_perm"]), ctypes.c_void_p(256), 1 << 30, None)
+    m1 = L.moe_last_error()
+    r2 = L.moe_dispatch_noalloc(p(a["x"]), p(a["idx"]), a["T"], a["d"], a["E"], a["top_k"],
+                                a["dt"], p(a["counts"]), p(a["offsets"]), p(a["src_row"]),
+                                p(a["dst_pos"]), p(a["x_perm"]), None)
+    m2 = L.moe_last_error()
+    assert r1 == 1 and r2 == 1, (r1, r2, m1, m2)
+    assert m1 == m2
+
+
+def test_noalloc_rejects_sizes_beyond_its_array(L):
+    """Sizes whose scratch exceeds the fixed array are refused on the host
+    with MOE_ERR_UNSUPPORTED before anything is launched."""
+    T, E, k = 1 << 22, 512, 16
+    need = L.moe_dispatch_workspace_size(T, E, k)
+    assert need > (4 << 20)
+    p = ctypes.c_void_p(256)
+    rc = L.moe_dispatch_noalloc(p, p, T, 64, E, k, 1, p, p, p, p, None, None)
+    assert rc == 2
+    assert b"fixed array" in L.moe_last_error()
