@@ -51,7 +51,7 @@ __all__ = [
     "ep_local_regroup", "apply_row_perm", "silu", "swiglu_ffn",
     "grouped_swiglu", "combine", "moe_forward", "dense_moe", "moe_tokens",
     "silu_grad", "grouped_preactivations", "combine_backward", "grouped_swiglu_backward",
-    "dispatch_backward", "router_backward",
+    "dispatch_backward", "router_backward", "load_balance_loss_grad",
 ]
 
 
@@ -198,6 +198,30 @@ def load_balance_loss(top_scores, selected_experts, E: int) -> float:
     frac /= T * k
     prob /= T
     return float(E * np.sum(frac * prob))
+
+
+def load_balance_loss_grad(selected_experts, E: int) -> np.ndarray:
+    """Gradient of :func:`load_balance_loss` with respect to the routing
+    weights ``top_scores`` [T, k]: the loss is linear in them through
+    ``P_e`` and the fractions ``f_e`` are counts (no gradient), so the entry
+    for a copy routed to expert e is ``E * f_e / T``.  A trainer that adds
+    ``coef * loss`` to its objective ([HP] adds the auxiliary loss to the
+    training loss) adds ``coef`` times this to the upstream gradient of the
+    routing weights."""
+    idx = _i64(selected_experts)
+    T, k = idx.shape
+    g = np.zeros((T, k))
+    if T == 0:
+        return g
+    frac = np.zeros(E)
+    for t in range(T):
+        for j in range(k):
+            frac[idx[t, j]] += 1.0
+    frac /= T * k
+    for t in range(T):
+        for j in range(k):
+            g[t, j] = E * frac[idx[t, j]] / T
+    return g
 
 
 def expert_counts(idx, E: int) -> np.ndarray:

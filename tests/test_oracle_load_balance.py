@@ -2,7 +2,10 @@
 _compute_load_balance_loss: E * sum_e f_e P_e).  Closed forms: a perfectly
 balanced router gives exactly 1 (the page's own statement of the balanced
 value), a router that sends every copy to one expert with weight 1 gives E;
-a vectorised restatement with numpy bincount; the empty input gives 0."""
+a vectorised restatement with numpy bincount; the empty input gives 0.
+The gradient with respect to the routing weights is pinned by central finite
+differences of the loss itself (it is linear in the weights) and by the
+balanced closed form."""
 import numpy as np
 
 import oracle as O
@@ -32,3 +35,23 @@ def test_matches_bincount_formulation():
 
 def test_empty_input():
     assert O.load_balance_loss(np.zeros((0, 2)), np.zeros((0, 2), dtype=np.int64), 4) == 0.0
+
+
+def test_gradient_matches_finite_differences():
+    L = W.make_logits(40, 8, 3, seed=4)
+    idx, w, _, _ = O.router_topk(3, True, logits=L)
+    g = O.load_balance_loss_grad(idx, 8)
+    h = 1e-3
+    for t, j in [(0, 0), (5, 2), (17, 1), (39, 0)]:
+        wp, wm = w.copy(), w.copy()
+        wp[t, j] += h
+        wm[t, j] -= h
+        fd = (O.load_balance_loss(wp, idx, 8) - O.load_balance_loss(wm, idx, 8)) / (2 * h)
+        assert abs(fd - g[t, j]) < 1e-10
+
+
+def test_gradient_of_the_balanced_router():
+    # balanced: f_e = 1/E for every expert, so every entry is 1/T
+    idx = np.array([[t % 4, (t + 1) % 4] for t in range(8)])
+    g = O.load_balance_loss_grad(idx, 4)
+    assert np.allclose(g, 1.0 / 8, rtol=0, atol=1e-15)
