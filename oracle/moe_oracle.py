@@ -52,6 +52,7 @@ __all__ = [
     "grouped_swiglu", "combine", "moe_forward", "dense_moe", "moe_tokens",
     "silu_grad", "grouped_preactivations", "combine_backward", "grouped_swiglu_backward",
     "dispatch_backward", "router_backward", "load_balance_loss_grad",
+    "scaled_dispatch_backward",
 ]
 
 
@@ -563,6 +564,26 @@ def dispatch_backward(dx_perm, dst_pos) -> np.ndarray:
     collects the gradients of its copies, ``dx[t] = sum_j dx_perm[dst_pos[t,
     j]]`` (the adjoint of the row gather is the scatter-add)."""
     return combine(dx_perm, dst_pos, None)
+
+
+def scaled_dispatch_backward(dx_perm, dst_pos, topk_w, x):
+    """Gradients of the scaled row gather of ``score_before_experts`` ([HP]
+    ``MoE.forward``): the copy in slot ``p = dst_pos[t, j]`` is
+    ``x_perm[p] = topk_w[t, j] * x[t]``, so ``dx[t] = sum_j topk_w[t, j] *
+    dx_perm[p]`` and ``d_topk_w[t, j] = <dx_perm[p], x[t]>``.  Returns
+    ``(dx [T, d], d_topk_w [T, k])`` in fp64."""
+    g = as_f64(dx_perm)
+    xx = as_f64(x)
+    dp = _i64(dst_pos)
+    w = as_f64(topk_w)
+    T, k = dp.shape
+    dx = np.zeros_like(xx)
+    dw = np.zeros((T, k))
+    for t in range(T):
+        for j in range(k):
+            dx[t] += w[t, j] * g[dp[t, j]]
+            dw[t, j] = float(g[dp[t, j]] @ xx[t])
+    return dx, dw
 
 
 def router_backward(logits, topk_idx, d_topk_w, score: str = "softmax",

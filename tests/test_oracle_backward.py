@@ -269,3 +269,96 @@ def test_whole_layer_gradients_compose_to_finite_differences():
     np.testing.assert_allclose(dx, _fd(loss, x), atol=2e-7)
     np.testing.assert_allclose(dwr, _fd(loss, wr), atol=2e-7)
     np.testing.assert_allclose(dw2, _fd(loss, w2), atol=2e-7)
+
+
+def test_scaled_dispatch_backward_matches_finite_differences():
+    """score_before_experts: x_perm[p(t, j)] = w[t, j] x[t].  The gradients of
+    <G, x_perm> with respect to x and w against central differences."""
+    rng = np.random.default_rng(5)
+    T, d, E, k = 7, 4, 3, 2
+    L = rng.standard_normal((T, E))
+    idx, w, _, _ = O.router_topk(k, True, logits=L)
+    _, _, src, dst = O.dispatch(idx, E)
+    x = rng.standard_normal((T, d))
+    G = rng.standard_normal((T * k, d))
+
+    def f():
+        xp = np.empty((T * k, d))
+        for t in range(T):
+            for j in range(k):
+                xp[dst[t, j]] = w[t, j] * x[t]
+        return float(np.sum(G * xp))
+
+    dx, dw = O.scaled_dispatch_backward(G, dst, w, x)
+    np.testing.assert_allclose(dx, _fd(f, x), atol=1e-8)
+    np.testing.assert_allclose(dw, _fd(f, w), atol=1e-8)
+
+
+def test_score_before_experts_layer_gradients_compose_to_finite_differences():
+    """The layer with score_before_experts ([HP] MoE.forward: routed rows
+    scaled by their weights, unweighted combine): the chain combine (w = 1)
+    -> experts -> scaled dispatch -> router equals central differences of
+    the oracle layer with respect to x and w_router."""
+    rng = np.random.default_rng(22)
+    T, d, E, k, h = 6, 5, 4, 2, 3
+    x = rng.standard_normal((T, d))
+    wr = rng.standard_normal((E, d)) * 2.0
+    w1 = rng.standard_normal((E, h, d)) * 0.6
+    w3 = rng.standard_normal((E, h, d)) * 0.6
+    w2 = rng.standard_normal((E, d, h)) * 0.6
+    dout = rng.standard_normal((T, d))
+    ref = O.moe_forward(x, wr, w1, w3, w2, k, True, score_before_experts=True)
+    srt = np.sort(ref["logits"], axis=1)
+    assert np.min(srt[:, -k] - srt[:, -k - 1]) > 1e-3
+    dy, _ = O.combine_backward(dout, ref["y"], ref["dst_pos"], None)
+    dxp, dw1, dw3, dw2 = O.grouped_swiglu_backward(ref["x_perm"], ref["offsets"], w1, w3, w2, dy)
+    dxs, dtw = O.scaled_dispatch_backward(dxp, ref["dst_pos"], ref["topk_w"], x)
+    _, dwr, dxr = O.router_backward(ref["logits"], ref["topk_idx"], dtw, renormalize=True, x=x,
+                                    w_router=wr)
+
+    def loss():
+        r = O.moe_forward(x, wr, w1, w3, w2, k, True, score_before_experts=True)
+        assert np.array_equal(r["topk_idx"], ref["topk_idx"])
+        return float(np.sum(dout * r["out"]))
+
+    np.testing.assert_allclose(dxs + dxr, _fd(loss, x), atol=2e-7)
+    np.testing.assert_allclose(dwr, _fd(loss, wr), atol=2e-7)
+    np.testing.assert_allclose(dw1, _fd(loss, w1), atol=2e-7)
+
+
+def test_shared_expert_gradients_compose_to_finite_differences():
+    """A shared expert ([HP] MoE.forward: out = routed + shared_expert(x))
+    is a one-segment grouped SwiGLU over every token: its backward with the
+    upstream dout gives its share of dx and its weight gradients, against
+    central differences of the oracle layer with the shared expert."""
+    rng = np.random.default_rng(23)
+    T, d, E, k, h, hs = 5, 4, 3, 2, 3, 6
+    x = rng.standard_normal((T, d))
+    wr = rng.standard_normal((E, d)) * 2.0
+    w1 = rng.standard_normal((E, h, d)) * 0.6
+    w3 = rng.standard_normal((E, h, d)) * 0.6
+    w2 = rng.standard_normal((E, d, h)) * 0.6
+    s1 = rng.standard_normal((hs, d)) * 0.6
+    s3 = rng.standard_normal((hs, d)) * 0.6
+    s2 = rng.standard_normal((d, hs)) * 0.6
+    dout = rng.standard_normal((T, d))
+    ref = O.moe_forward(x, wr, w1, w3, w2, k, True, shared=(s1, s3, s2))
+    srt = np.sort(ref["logits"], axis=1)
+    assert np.min(srt[:, -k] - srt[:, -k - 1]) > 1e-3
+    dy, dtw = O.combine_backward(dout, ref["y"], ref["dst_pos"], ref["topk_w"])
+    dxp, _, _, _ = O.grouped_swiglu_backward(ref["x_perm"], ref["offsets"], w1, w3, w2, dy)
+    _, _, dxr = O.router_backward(ref["logits"], ref["topk_idx"], dtw, renormalize=True, x=x,
+                                  w_router=wr)
+    dxsh, ds1, ds3, ds2 = O.grouped_swiglu_backward(x, np.array([0, T]), s1[None], s3[None],
+                                                    s2[None], dout)
+
+    def loss():
+        r = O.moe_forward(x, wr, w1, w3, w2, k, True, shared=(s1, s3, s2))
+        assert np.array_equal(r["topk_idx"], ref["topk_idx"])
+        return float(np.sum(dout * r["out"]))
+
+    dx = O.dispatch_backward(dxp, ref["dst_pos"]) + dxr + dxsh
+    np.testing.assert_allclose(dx, _fd(loss, x), atol=2e-7)
+    np.testing.assert_allclose(ds1[0], _fd(loss, s1), atol=2e-7)
+    np.testing.assert_allclose(ds3[0], _fd(loss, s3), atol=2e-7)
+    np.testing.assert_allclose(ds2[0], _fd(loss, s2), atol=2e-7)
