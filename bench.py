@@ -271,11 +271,12 @@ def run_reference(args, ws, rank):
 
 
 # ------------------------------------------------------------------- GPU arm
-# kernels of libmoe that one moe_forward step launches: router (GEMM, top-k
-# with the dispatch histogram), dispatch (column scan, scatter), regroup on
-# the EP layout (scan, copy), grouped SwiGLU (GEMM1, GEMM2), combine
+# kernels of libmoe that one moe_forward step launches: router (one fused
+# kernel: gate GEMM, top-k, dispatch histogram), dispatch (column scan,
+# scatter), regroup on the EP layout (one kernel), grouped SwiGLU (GEMM1,
+# GEMM2), combine
 def forward_launches(cfg) -> int:
-    return 2 + 2 + (2 if cfg.ep_ranks > 1 else 0) + 2 + 1
+    return 1 + 2 + (1 if cfg.ep_ranks > 1 else 0) + 2 + 1
 
 
 class Layer:
@@ -464,8 +465,8 @@ def run_ours(args, ws, rank, local):
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
     if args.profile:
-        # Kernel order per staged step (R = 1): router GEMM, router top-k,
-        # dispatch histogram, column scan, scatter, GEMM1, GEMM2, combine.
+        # Kernel order per staged step: router (fused), dispatch histogram,
+        # column scan, scatter, [regroup], GEMM1, GEMM2, combine.
         for _ in range(2):
             layer.staged(stream)
         layer.forward()

@@ -163,6 +163,13 @@ MOE_API moe_status_t moe_router_topk(const void* x, const void* w_router, const 
  * top_k <= topk_groups * (E / num_groups); expert_bias [E] fp32 device or
  * NULL; tokens_per_expert [E] fp32 device or NULL (accumulated, never
  * cleared by the library); aux_loss one fp32 device scalar or NULL (written).
+ *
+ * aux_loss_coef (backward only: moe_router_backward, moe_backward): a trainer
+ * that adds aux_loss_coef * aux_loss to its objective ([HP] adds the
+ * auxiliary loss to the training loss) gets its gradient here: the routing
+ * weight of a copy routed to expert e receives aux_loss_coef * E * f_e / T
+ * (f_e as above; the counts carry no gradient), added to d_topk_w before the
+ * router's backward.  0 (the default) adds nothing.
  * ---------------------------------------------------------------------- */
 typedef struct moe_router_options {
   moe_score_t score;
@@ -174,6 +181,7 @@ typedef struct moe_router_options {
   float* tokens_per_expert;
   int score_before_experts;
   float* aux_loss;
+  float aux_loss_coef;
 } moe_router_options_t;
 
 MOE_API void moe_router_options_init(moe_router_options_t* opts);
@@ -447,10 +455,16 @@ MOE_API moe_status_t moe_router_backward(const float* logits, const int32_t* top
  *      when dw_router is computed (a gate driven by logits_in has neither)
  *   d_logits [T, E] fp32 (NULL: not written)   the logits' gradient dz
  * `opts` must be the options of the forward (score, renormalize, route_scale
- * enter the router's derivative; bias and groups only selected).  bf16 only;
- * d % 64 == 0, h % 64 == 0, E % 8 == 0; score_before_experts is rejected
- * (MOE_ERR_UNSUPPORTED).  Workspace: moe_backward_workspace_size.  Device
- * errors: the status word of `state` (forward) and of `ws` (backward).
+ * enter the router's derivative; bias and groups only selected;
+ * aux_loss_coef adds the load-balance loss's gradient).  With
+ * score_before_experts ([HP] MoE.forward) the forward scales the routed rows
+ * by their weights and combines unweighted, and the backward takes the
+ * weights' gradient from the scaled rows, d topk_w[t, j] =
+ * <dx_perm[p(t, j)], x[t]>, and weights each copy's share of dx by topk_w
+ * (x is then required).  bf16 only; d % 64 == 0, h % 64 == 0, E % 8 == 0.
+ * Workspace: moe_backward_workspace_size.  Device errors: the status word of
+ * `state` (forward) and of `ws` (backward).  A shared expert: the _ex forms
+ * below.
  * ---------------------------------------------------------------------- */
 MOE_API size_t moe_train_state_size(int T, int d, int E, int top_k, int h);
 MOE_API moe_status_t moe_forward_train(const void* x, const void* w_router,
@@ -516,6 +530,37 @@ MOE_API moe_status_t moe_forward_ex(const void* x, const void* w_router, const f
                                     moe_dtype_t dt, void* out, float* logits_out,
                                     int32_t* topk_idx, float* topk_w, int32_t* counts, void* ws,
                                     size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * moe_forward_train_ex / moe_backward_ex -- moe_forward_train / moe_backward
+ * with a shared expert ([HP] MoE.forward: out = routed + shared_expert(x),
+ * a dense SwiGLU FFN on every token; `shared` as moe_forward_ex, NULL =
+ * none).  The forward keeps the shared expert's H [T, hs] and G | U
+ * [T, 2hs] in the state (moe_train_state_size_ex); the backward runs its
+ * backward as a one-segment grouped SwiGLU backward over all T tokens with
+ * the layer's upstream gradient dout, writes dws1, dws3 [hs, d] and dws2
+ * [d, hs] (required when `shared` is given) and adds its share of dx.
+ * Workspace: moe_backward_workspace_size_ex.  h_shared = 0 gives the sizes
+ * of the plain forms, which are these calls with shared = NULL.
+ * ---------------------------------------------------------------------- */
+MOE_API size_t moe_train_state_size_ex(int T, int d, int E, int top_k, int h, int h_shared);
+MOE_API moe_status_t moe_forward_train_ex(const void* x, const void* w_router,
+                                          const float* logits_in, const void* w1,
+                                          const void* w3, const void* w2, int T, int d, int E,
+                                          int top_k, int h, const moe_router_options_t* opts,
+                                          const moe_shared_expert_t* shared, moe_dtype_t dt,
+                                          void* out, void* state, size_t state_bytes,
+                                          void* stream);
+MOE_API size_t moe_backward_workspace_size_ex(int T, int d, int E, int top_k, int h,
+                                              int h_shared);
+MOE_API moe_status_t moe_backward_ex(const void* dout, const void* x, const void* w_router,
+                                     const void* w1, const void* w3, const void* w2, int T, int d,
+                                     int E, int top_k, int h, const moe_router_options_t* opts,
+                                     const moe_shared_expert_t* shared, moe_dtype_t dt,
+                                     const void* state, void* dx, float* d_logits,
+                                     void* dw_router, void* dw1, void* dw3, void* dw2,
+                                     void* dws1, void* dws3, void* dws2, void* ws,
+                                     size_t ws_bytes, void* stream);
 
 /* moe_selftest_timeout -- test of the failure path every pipeline of the
  * library shares (no counterpart on the pages).  Launches one thread that

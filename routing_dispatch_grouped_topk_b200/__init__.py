@@ -46,7 +46,8 @@ __all__ = [
     "grouped_swiglu_train", "grouped_swiglu_backward", "combine_backward", "dispatch_backward",
     "moe_router_backward", "router_backward_workspace_size", "router_backward",
     "moe_train_state_size", "moe_forward_train", "moe_backward_workspace_size", "moe_backward",
-    "forward_train", "backward",
+    "moe_train_state_size_ex", "moe_forward_train_ex", "moe_backward_workspace_size_ex",
+    "moe_backward_ex", "forward_train", "backward",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe.so")
@@ -67,6 +68,8 @@ EXPORTED_SYMBOLS = [
     "moe_grouped_swiglu_backward", "moe_combine_backward", "moe_dispatch_backward",
     "moe_router_backward_workspace_size", "moe_router_backward",
     "moe_train_state_size", "moe_forward_train", "moe_backward_workspace_size", "moe_backward",
+    "moe_train_state_size_ex", "moe_forward_train_ex", "moe_backward_workspace_size_ex",
+    "moe_backward_ex",
     "moe_forward_workspace_size", "moe_forward", "moe_forward_ex_workspace_size",
     "moe_forward_ex", "moe_get_device_status", "moe_selftest_timeout", "moe_status_string",
     "moe_last_error", "moe_version",
@@ -89,6 +92,7 @@ class RouterOptions(ctypes.Structure):
         ("tokens_per_expert", ctypes.c_void_p),
         ("score_before_experts", ctypes.c_int),
         ("aux_loss", ctypes.c_void_p),
+        ("aux_loss_coef", ctypes.c_float),
     ]
 
 
@@ -141,6 +145,13 @@ _SIGS = {
                           _P, _P, _P, _Z, _P]),
     "moe_router_backward": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _I, _P, _P, _P, _P, _Z,
                                  _P]),
+    "moe_train_state_size_ex": (_Z, [_I, _I, _I, _I, _I, _I]),
+    "moe_forward_train_ex": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P,
+                                  ctypes.POINTER(SharedExpert), _I, _P, _P, _Z, _P]),
+    "moe_backward_workspace_size_ex": (_Z, [_I, _I, _I, _I, _I, _I]),
+    "moe_backward_ex": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P,
+                             ctypes.POINTER(SharedExpert), _I, _P, _P, _P, _P, _P, _P, _P, _P,
+                             _P, _P, _P, _Z, _P]),
     "moe_forward_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I, _I]),
     "moe_forward": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P,
                          _P, _P, _P, _Z, _P]),
@@ -263,11 +274,14 @@ def moe_router_options_init() -> RouterOptions:
 
 def router_options(score="softmax", renormalize=False, route_scale=1.0, expert_bias=None,
                    num_groups=0, topk_groups=0, tokens_per_expert=None,
-                   score_before_experts=False, aux_loss=None) -> RouterOptions:
+                   score_before_experts=False, aux_loss=None,
+                   aux_loss_coef=0.0) -> RouterOptions:
     """A RouterOptions from keyword values ([HP] TokenChoiceTopKRouter's
     settings).  expert_bias / tokens_per_expert are fp32 CUDA tensors [E],
     aux_loss an fp32 CUDA tensor of one element, or None; they must stay
-    alive while the call that takes the options runs."""
+    alive while the call that takes the options runs.  aux_loss_coef (the
+    backward entry points) adds the gradient of aux_loss_coef times the
+    load-balance loss to the routing weights' gradient."""
     o = moe_router_options_init()
     o.score = {"softmax": MOE_SCORE_SOFTMAX, "sigmoid": MOE_SCORE_SIGMOID}[score]
     o.renormalize = int(bool(renormalize))
@@ -278,6 +292,7 @@ def router_options(score="softmax", renormalize=False, route_scale=1.0, expert_b
     o.tokens_per_expert = _ptr(tokens_per_expert, torch.float32, "tokens_per_expert")
     o.score_before_experts = int(bool(score_before_experts))
     o.aux_loss = _ptr(aux_loss, torch.float32, "aux_loss")
+    o.aux_loss_coef = float(aux_loss_coef)
     return o
 
 
@@ -414,6 +429,29 @@ def moe_backward(dout, x, w_router, w1, w3, w2, T, d, E, top_k, h, opts, dt, sta
         _ptr(d_logits, torch.float32, "d_logits"), _ptr(dw_router, name="dw_router"),
         _ptr(dw1, name="dw1"), _ptr(dw3, name="dw3"), _ptr(dw2, name="dw2"),
         _ptr(ws, name="ws"), _nbytes(ws), _stream(stream)), "moe_backward")
+
+
+def moe_forward_train_ex(x, w_router, logits_in, w1, w3, w2, T, d, E, top_k, h, opts, shared,
+                         dt, out, state, stream=None):
+    _check(lib().moe_forward_train_ex(
+        _ptr(x, name="x"), _ptr(w_router, name="w_router"),
+        _ptr(logits_in, torch.float32, "logits_in"), _ptr(w1, name="w1"), _ptr(w3, name="w3"),
+        _ptr(w2, name="w2"), T, d, E, top_k, h, _opts(opts),
+        None if shared is None else ctypes.byref(shared), dt, _ptr(out, name="out"),
+        _ptr(state, name="state"), _nbytes(state), _stream(stream)), "moe_forward_train_ex")
+
+
+def moe_backward_ex(dout, x, w_router, w1, w3, w2, T, d, E, top_k, h, opts, shared, dt, state,
+                    dx, d_logits, dw_router, dw1, dw3, dw2, dws1, dws3, dws2, ws, stream=None):
+    _check(lib().moe_backward_ex(
+        _ptr(dout, name="dout"), _ptr(x, name="x"), _ptr(w_router, name="w_router"),
+        _ptr(w1, name="w1"), _ptr(w3, name="w3"), _ptr(w2, name="w2"), T, d, E, top_k, h,
+        _opts(opts), None if shared is None else ctypes.byref(shared), dt,
+        _ptr(state, name="state"), _ptr(dx, name="dx"),
+        _ptr(d_logits, torch.float32, "d_logits"), _ptr(dw_router, name="dw_router"),
+        _ptr(dw1, name="dw1"), _ptr(dw3, name="dw3"), _ptr(dw2, name="dw2"),
+        _ptr(dws1, name="dws1"), _ptr(dws3, name="dws3"), _ptr(dws2, name="dws2"),
+        _ptr(ws, name="ws"), _nbytes(ws), _stream(stream)), "moe_backward_ex")
 
 
 def moe_forward(x, w_router, logits_in, w1, w3, w2, T, d, E, top_k, h, score, renormalize,
@@ -649,37 +687,47 @@ def router_backward(logits, topk_idx, d_topk_w, x=None, w_router=None, want_d_lo
     return dl, dwr, dx, ws
 
 
-def forward_train(x, w_router, w1, w3, w2, top_k, renormalize=True, logits_in=None, **options):
+def forward_train(x, w_router, w1, w3, w2, top_k, renormalize=True, logits_in=None,
+                  shared=None, **options):
     """Training forward of the whole layer.  Returns (out [T, d], state), the
-    state to hand to :func:`backward` (it records the sizes and options)."""
+    state to hand to :func:`backward` (it records the sizes and options).
+    ``shared`` = (ws1 [hs, d], ws3 [hs, d], ws2 [d, hs]) adds a shared
+    expert; ``options`` are router_options() keywords."""
     T, d = x.shape
     E, h, _ = w1.shape
-    st = _ws(lib().moe_train_state_size(T, d, E, top_k, h), x.device)
+    sh = None if shared is None else shared_expert(*shared)
+    hs = 0 if sh is None else sh.h
+    st = _ws(lib().moe_train_state_size_ex(T, d, E, top_k, h, hs), x.device)
     out = torch.empty(T, d, dtype=x.dtype, device=x.device)
     opts = router_options(renormalize=renormalize, **options)
-    moe_forward_train(x, w_router, logits_in, w1, w3, w2, T, d, E, top_k, h, opts, _dt(x), out,
-                      st)
-    state = {"state": st, "T": T, "d": d, "E": E, "k": top_k, "h": h,
+    moe_forward_train_ex(x, w_router, logits_in, w1, w3, w2, T, d, E, top_k, h, opts, sh, _dt(x),
+                         out, st)
+    state = {"state": st, "T": T, "d": d, "E": E, "k": top_k, "h": h, "hs": hs,
              "options": dict(options, renormalize=renormalize)}
     return out, state
 
 
-def backward(state, dout, x, w_router, w1, w3, w2, router_grads=True, want_d_logits=False):
+def backward(state, dout, x, w_router, w1, w3, w2, router_grads=True, want_d_logits=False,
+             shared=None):
     """Backward of the whole layer for dout [T, d].  Returns a dict with dx,
     dw1, dw3, dw2, dw_router (None unless router_grads), d_logits (None
-    unless asked) and ws."""
+    unless asked), the shared expert's dws1, dws3, dws2 (None without one)
+    and ws.  ``shared`` must be the forward's."""
     T, d, E, k, h = (state[n] for n in ("T", "d", "E", "k", "h"))
     dev = dout.device
+    sh = None if shared is None else shared_expert(*shared)
+    hs = 0 if sh is None else sh.h
     dx = torch.empty(T, d, dtype=dout.dtype, device=dev)
     dw1, dw3, dw2 = torch.empty_like(w1), torch.empty_like(w3), torch.empty_like(w2)
     dwr = torch.empty_like(w_router) if router_grads else None
     dl = torch.empty(T, E, dtype=torch.float32, device=dev) if want_d_logits else None
-    ws = _ws(lib().moe_backward_workspace_size(T, d, E, k, h), dev)
+    ds = [torch.empty_like(t) for t in shared] if shared is not None else [None] * 3
+    ws = _ws(lib().moe_backward_workspace_size_ex(T, d, E, k, h, hs), dev)
     opts = router_options(**state["options"])
-    moe_backward(dout, x, w_router, w1, w3, w2, T, d, E, k, h, opts, _dt(dout), state["state"],
-                 dx, dl, dwr, dw1, dw3, dw2, ws)
+    moe_backward_ex(dout, x, w_router, w1, w3, w2, T, d, E, k, h, opts, sh, _dt(dout),
+                    state["state"], dx, dl, dwr, dw1, dw3, dw2, ds[0], ds[1], ds[2], ws)
     return {"dx": dx, "dw1": dw1, "dw3": dw3, "dw2": dw2, "dw_router": dwr, "d_logits": dl,
-            "ws": ws}
+            "dws1": ds[0], "dws3": ds[1], "dws2": ds[2], "ws": ws}
 
 
 def forward(x, w_router, w1, w3, w2, top_k, renormalize=True, ep_ranks=1, logits_in=None,

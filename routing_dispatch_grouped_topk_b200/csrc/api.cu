@@ -77,6 +77,14 @@ bool router_uses_tc(int E, moe_dtype_t dt) { return dt == MOE_BF16 && E <= 256; 
 // Load-balance statistics (copies and weight sums per expert, 2E floats).
 size_t lb_bytes(int E) { return align_up(2 * static_cast<size_t>(E) * sizeof(float), 256); }
 
+// Per-count factor of the load-balance loss's gradient: a copy routed to
+// expert e gets coef * E * f_e / T with f_e = counts_e / (T k).
+float lb_grad_scale(float coef, int E, int T, int k) {
+  return T > 0 ? static_cast<float>(static_cast<double>(coef) * E /
+                                    (static_cast<double>(T) * T * k))
+               : 0.f;
+}
+
 // Status word, the load-balance statistics, then the fp32 logit scratch:
 // [ksplit, T, E] partial logits of the tensor-core GEMM, or [T, E] logits of
 // the CUDA-core path.
@@ -96,6 +104,7 @@ moe_router_options_t default_options() {
   o.tokens_per_expert = nullptr;
   o.score_before_experts = 0;
   o.aux_loss = nullptr;
+  o.aux_loss_coef = 0.0f;
   return o;
 }
 
@@ -169,13 +178,25 @@ RouterOptions kernel_options(const moe_router_options_t& o) {
   return k;
 }
 
-// Router launch sequence (status and counts already cleared by the caller).
-// With `plan` and `blk` the top-k kernel also writes the dispatch histogram.
+// The fused tcgen05 router (bf16, E <= 256, no group limit, logits from
+// the gate) serves this call.
+bool router_is_fused(const float* logits_in, int T, int d, int E, const moe_router_options_t& o,
+                     moe_dtype_t dt, const DispatchPlan* plan) {
+  return T > 0 && !logits_in && router_uses_tc(E, dt) && o.num_groups == 0 &&
+         router_fused_plan(T, d, E, plan).ok;
+}
+
+// Router launch sequence.  With `plan` and `blk` the top-k step also writes
+// the dispatch histogram.  The fused router writes `counts` without atomics
+// (a per-CTA table and a summing kernel) and, with own_status, clears the
+// status word itself; on the other paths the caller has cleared the status
+// word and `counts` is cleared here (they add into it with atomics).
 cudaError_t run_router(const void* x, const void* w_router, const float* logits_in, int T, int d,
                        int E, int top_k, const moe_router_options_t& o, moe_dtype_t dt,
                        float* logits_out, int32_t* topk_idx, float* topk_w, int32_t* counts,
                        void* scratch, int* status, cudaStream_t s,
-                       const DispatchPlan* plan = nullptr, int32_t* blk = nullptr) {
+                       const DispatchPlan* plan = nullptr, int32_t* blk = nullptr,
+                       bool own_status = false) {
   const RouterOptions ko = kernel_options(o);
   const int renorm = o.renormalize;
   float* tpe = o.tokens_per_expert;
@@ -183,10 +204,17 @@ cudaError_t run_router(const void* x, const void* w_router, const float* logits_
   float* part = reinterpret_cast<float*>(static_cast<char*>(scratch) + lb_bytes(E));
   cudaError_t e = cudaSuccess;
   if (lb) e = cudaMemsetAsync(lb, 0, 2 * sizeof(float) * E, s);
+  const bool fused = router_is_fused(logits_in, T, d, E, o, dt, plan);
+  if (e == cudaSuccess && counts && !fused)
+    e = cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, s);
   if (e == cudaSuccess && T > 0) {
     if (logits_in) {
       e = launch_router_topk(logits_in, 1, T, E, top_k, renorm, ko, nullptr, topk_idx, topk_w,
                              counts, tpe, plan, blk, s, lb);
+    } else if (fused) {
+      e = launch_router_fused(x, w_router, T, d, E, top_k, renorm, ko, logits_out, topk_idx,
+                              topk_w, counts, reinterpret_cast<int32_t*>(part), tpe, lb, plan,
+                              blk, status, own_status, s);
     } else if (router_uses_tc(E, dt)) {
       e = launch_router_tc(x, w_router, T, d, E, part, status, s);
       if (e == cudaSuccess)
@@ -300,7 +328,7 @@ ForwardWs carve_forward(void* ws, int T, int d, int E, int k, int h, int R, moe_
   f.router_scratch = c.take<char>(router_ws(T, d, E, dt) - kStatusBytes);
   f.idx = c.take<int32_t>(N);
   f.w = c.take<float>(N);
-  const DispatchPlan p = make_dispatch_plan(T, E, k, R);
+  const DispatchPlan p = layer_dispatch_plan(T, d, E, k, R, dt);
   f.counts_a = c.take<int32_t>(static_cast<size_t>(p.nbins));
   f.offsets_a = c.take<int32_t>(static_cast<size_t>(p.nbins) + 1);
   f.src_row = c.take<int32_t>(N);
@@ -342,10 +370,16 @@ struct TrainState {
   void* y;             // [N, d]
   void* H;             // [N, h]
   void* GU;            // [N, 2h]
+  // shared expert (h_shared > 0): its one-segment offsets, output and the
+  // training forward's H and G | U over every token
+  int32_t* offsets_s;  // [2]
+  void* ys;            // [T, d]
+  void* Hs;            // [T, hs]
+  void* GUs;           // [T, 2hs]
   size_t bytes;
 };
 
-TrainState carve_train(void* base, int T, int d, int E, int k, int h) {
+TrainState carve_train(void* base, int T, int d, int E, int k, int h, int hs = 0) {
   TrainState t{};
   Carve c(base);
   const size_t N = static_cast<size_t>(T) * k;
@@ -353,7 +387,7 @@ TrainState carve_train(void* base, int T, int d, int E, int k, int h) {
   t.logits = c.take<float>(static_cast<size_t>(T) * E);
   t.idx = c.take<int32_t>(N);
   t.w = c.take<float>(N);
-  const DispatchPlan p = make_dispatch_plan(T, E, k, 1);
+  const DispatchPlan p = layer_dispatch_plan(T, d, E, k, 1, MOE_BF16);
   t.counts = c.take<int32_t>(E);
   t.offsets = c.take<int32_t>(static_cast<size_t>(E) + 1);
   t.src_row = c.take<int32_t>(N);
@@ -364,6 +398,12 @@ TrainState carve_train(void* base, int T, int d, int E, int k, int h) {
   t.y = c.take<char>(N * d * 2);
   t.H = c.take<char>(N * h * 2);
   t.GU = c.take<char>(N * 2 * h * 2);
+  if (hs > 0) {
+    t.offsets_s = c.take<int32_t>(2);
+    t.ys = c.take<char>(static_cast<size_t>(T) * d * 2);
+    t.Hs = c.take<char>(static_cast<size_t>(T) * hs * 2);
+    t.GUs = c.take<char>(static_cast<size_t>(T) * 2 * hs * 2);
+  }
   t.bytes = c.off;
   return t;
 }
@@ -379,10 +419,12 @@ struct BackwardWs {
   void* dz16;          // [T, E]
   void* dxr;           // [T, d] the router's share of dx
   float* gpart;        // [splits, E, d] fp32 partials of dw_router
+  void* dXs;           // [T, d] the shared expert's share of dx
+  void* dGUs;          // [T, 2hs]
   size_t bytes;
 };
 
-BackwardWs carve_backward(void* base, int T, int d, int E, int k, int h) {
+BackwardWs carve_backward(void* base, int T, int d, int E, int k, int h, int hs = 0) {
   BackwardWs b{};
   Carve c(base);
   const size_t N = static_cast<size_t>(T) * k;
@@ -395,6 +437,10 @@ BackwardWs carve_backward(void* base, int T, int d, int E, int k, int h) {
   b.dz16 = c.take<char>(static_cast<size_t>(T) * E * 2);
   b.dxr = c.take<char>(static_cast<size_t>(T) * d * 2);
   b.gpart = c.take<float>(static_cast<size_t>(gate_splits(T, d, E)) * E * d);
+  if (hs > 0) {
+    b.dXs = c.take<char>(static_cast<size_t>(T) * d * 2);
+    b.dGUs = c.take<char>(static_cast<size_t>(T) * 2 * hs * 2);
+  }
   b.bytes = c.off;
   return b;
 }
@@ -414,10 +460,18 @@ moe_status_t check_train(int T, int d, int E, int top_k, int h, const moe_router
     set_last_error("training entry points need E %% 8 == 0 (E=%d)", E);
     return MOE_ERR_UNSUPPORTED;
   }
-  if (o.score_before_experts) {
-    set_last_error("training entry points: score_before_experts has no backward here");
-    return MOE_ERR_UNSUPPORTED;
-  }
+  return MOE_OK;
+}
+
+// Shared expert of the training entry points: a dense SwiGLU FFN on every
+// token, with the tensor-core rules of the grouped SwiGLU.
+moe_status_t check_shared(const moe_shared_expert_t* sh, int T, int d, moe_dtype_t dt) {
+  if (!sh) return MOE_OK;
+  MOE_CHECK_ARG(sh->h >= 1, "shared->h=%d must be >= 1", sh->h);
+  if (moe_status_t st = check_swiglu_shape(T, d, sh->h, 1, dt)) return st;
+  MOE_CHECK_ARG(sh->w1 && sh->w3 && sh->w2, "shared expert w1, w3, w2 are required");
+  MOE_CHECK_ARG(aligned16(sh->w1) && aligned16(sh->w3) && aligned16(sh->w2),
+                "shared expert weights must be 16-byte aligned");
   return MOE_OK;
 }
 
@@ -495,11 +549,14 @@ moe_status_t moe_router_topk_ex(const void* x, const void* w_router, const float
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int* status = static_cast<int*>(ws);
-  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), s);
-  if (e == cudaSuccess && counts) e = cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, s);
+  // the fused router clears the status word itself (it is the only kernel
+  // that can write it); the other paths start from a cleared word
+  const bool fused = router_is_fused(logits_in, T, d, E, o, dt, nullptr);
+  cudaError_t e = fused ? cudaSuccess : cudaMemsetAsync(status, 0, sizeof(int), s);
   if (e == cudaSuccess)
     e = run_router(x, w_router, logits_in, T, d, E, top_k, o, dt, logits_out, topk_idx, topk_w,
-                   counts, static_cast<char*>(ws) + kStatusBytes, status, s);
+                   counts, static_cast<char*>(ws) + kStatusBytes, status, s, nullptr, nullptr,
+                   fused);
   return cuda_status(e, "moe_router_topk");
 }
 
@@ -593,10 +650,10 @@ moe_status_t moe_ep_local_regroup(const void* in, const int32_t* counts_rm, int 
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int* status = static_cast<int*>(ws);
-  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), s);
-  if (e == cudaSuccess)
-    e = launch_regroup(in, counts_rm, G, R, L, rows, d, dt, out, counts_em, offsets_em, perm,
-                       perm_inv, static_cast<char*>(ws) + kStatusBytes, status, s);
+  // one kernel, which writes the whole status word itself
+  cudaError_t e = launch_regroup(in, counts_rm, G, R, L, rows, d, dt, out, counts_em, offsets_em,
+                                 perm, perm_inv, static_cast<char*>(ws) + kStatusBytes, status, s,
+                                 /*own_status=*/true);
   return cuda_status(e, "moe_ep_local_regroup");
 }
 
@@ -806,8 +863,11 @@ moe_status_t moe_dispatch_backward(const void* dx_perm, const int32_t* dst_pos,
 // dw_router [splits, E, d]
 size_t moe_router_backward_workspace_size(int T, int d, int E) {
   if (T < 0 || E < 1 || d < 1) return kStatusBytes;
+  // status, gate segment offsets, dz in bf16, the gate's fp32 partials,
+  // then the expert counts of the load-balance gradient
   return kStatusBytes + 256 + align_up(static_cast<size_t>(T) * E * 2, 256) +
-         align_up(static_cast<size_t>(gate_splits(T, d, E)) * E * d * 4, 256);
+         align_up(static_cast<size_t>(gate_splits(T, d, E)) * E * d * 4, 256) +
+         align_up(static_cast<size_t>(E) * 4, 256);
 }
 
 moe_status_t moe_router_backward(const float* logits, const int32_t* topk_idx,
@@ -849,13 +909,23 @@ moe_status_t moe_router_backward(const float* logits, const int32_t* topk_idx,
   void* dz16 = static_cast<char*>(ws) + kStatusBytes + 256;
   float* gpart = reinterpret_cast<float*>(static_cast<char*>(dz16) +
                                           align_up(static_cast<size_t>(T) * E * 2, 256));
+  int32_t* lbc = reinterpret_cast<int32_t*>(
+      reinterpret_cast<char*>(gpart) +
+      align_up(static_cast<size_t>(gate_splits(T, d, E)) * E * d * 4, 256));
+  const bool lb = o.aux_loss_coef != 0.0f && T > 0;
+  MOE_CHECK_ARG(std::isfinite(o.aux_loss_coef), "aux_loss_coef must be finite");
   cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), s);
   if (e == cudaSuccess && T == 0 && dw_router)
     e = cudaMemsetAsync(dw_router, 0, static_cast<size_t>(E) * d * 2, s);
+  // the load-balance gradient needs the forward's expert counts: recounted
+  // from topk_idx
+  if (e == cudaSuccess && lb) e = cudaMemsetAsync(lbc, 0, static_cast<size_t>(E) * 4, s);
+  if (e == cudaSuccess && lb) e = launch_expert_hist(topk_idx, 1LL * T * top_k, E, lbc, s);
   if (e == cudaSuccess && T > 0)
     e = launch_router_backward(logits, topk_idx, d_topk_w, T, E, top_k,
                                o.score == MOE_SCORE_SIGMOID, o.renormalize, o.route_scale,
-                               d_logits, gemm ? dz16 : nullptr, s);
+                               d_logits, gemm ? dz16 : nullptr, s, lb ? lbc : nullptr,
+                               lb ? lb_grad_scale(o.aux_loss_coef, E, T, top_k) : 0.f);
   if (e == cudaSuccess && T > 0 && gemm)
     e = launch_gate_backward_tc(dz16, x, w_router, T, d, E, dw_router, dx, off2, gpart, status,
                                 s);
@@ -864,25 +934,35 @@ moe_status_t moe_router_backward(const float* logits, const int32_t* topk_idx,
 
 // ---------------------------------------------------- whole-layer training
 size_t moe_train_state_size(int T, int d, int E, int top_k, int h) {
-  if (T < 0 || d < 1 || E < 1 || top_k < 1 || h < 1) return kStatusBytes;
-  return carve_train(nullptr, T, d, E, top_k, h).bytes;
+  return moe_train_state_size_ex(T, d, E, top_k, h, 0);
+}
+
+size_t moe_train_state_size_ex(int T, int d, int E, int top_k, int h, int h_shared) {
+  if (T < 0 || d < 1 || E < 1 || top_k < 1 || h < 1 || h_shared < 0) return kStatusBytes;
+  return carve_train(nullptr, T, d, E, top_k, h, h_shared).bytes;
 }
 
 size_t moe_backward_workspace_size(int T, int d, int E, int top_k, int h) {
-  if (T < 0 || d < 1 || E < 1 || top_k < 1 || h < 1) return kStatusBytes;
-  return carve_backward(nullptr, T, d, E, top_k, h).bytes;
+  return moe_backward_workspace_size_ex(T, d, E, top_k, h, 0);
 }
 
-moe_status_t moe_forward_train(const void* x, const void* w_router, const float* logits_in,
-                               const void* w1, const void* w3, const void* w2, int T, int d,
-                               int E, int top_k, int h, const moe_router_options_t* opts,
-                               moe_dtype_t dt, void* out, void* state, size_t state_bytes,
-                               void* stream) {
+size_t moe_backward_workspace_size_ex(int T, int d, int E, int top_k, int h, int h_shared) {
+  if (T < 0 || d < 1 || E < 1 || top_k < 1 || h < 1 || h_shared < 0) return kStatusBytes;
+  return carve_backward(nullptr, T, d, E, top_k, h, h_shared).bytes;
+}
+
+moe_status_t moe_forward_train_ex(const void* x, const void* w_router, const float* logits_in,
+                                  const void* w1, const void* w3, const void* w2, int T, int d,
+                                  int E, int top_k, int h, const moe_router_options_t* opts,
+                                  const moe_shared_expert_t* shared, moe_dtype_t dt, void* out,
+                                  void* state, size_t state_bytes, void* stream) {
   const moe_router_options_t o = opts ? *opts : default_options();
   if (moe_status_t st = check_train(T, d, E, top_k, h, o, dt)) return st;
   if (moe_status_t st = check_router(x, w_router, logits_in, T, d, E, top_k, o, dt,
                                      reinterpret_cast<int32_t*>(1), reinterpret_cast<float*>(1)))
     return st;
+  if (moe_status_t st = check_shared(shared, T, d, dt)) return st;
+  const int hs = shared ? shared->h : 0;
   if (T > 0) {
     MOE_CHECK_ARG(x && w1 && w3 && w2 && out, "x, w1, w3, w2, out are required");
     MOE_CHECK_ARG(aligned16(x) && aligned16(w1) && aligned16(w3) && aligned16(w2) &&
@@ -890,15 +970,16 @@ moe_status_t moe_forward_train(const void* x, const void* w_router, const float*
                   "x, w1, w3, w2, out must be 16-byte aligned");
   }
   MOE_CHECK_ARG(state != nullptr, "state is required");
-  const TrainState need = carve_train(nullptr, T, d, E, top_k, h);
+  const TrainState need = carve_train(nullptr, T, d, E, top_k, h, hs);
   if (state_bytes < need.bytes) {
     set_last_error("training state %zu < %zu", state_bytes, need.bytes);
     return MOE_ERR_WORKSPACE;
   }
-  const TrainState t = carve_train(state, T, d, E, top_k, h);
+  const TrainState t = carve_train(state, T, d, E, top_k, h, hs);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int N = T * top_k;
-  const DispatchPlan p = make_dispatch_plan(T, E, top_k, 1);
+  const bool before = o.score_before_experts != 0;
+  const DispatchPlan p = layer_dispatch_plan(T, d, E, top_k, 1, dt);
   cudaError_t e = cudaMemsetAsync(t.status, 0, sizeof(int), s);
   if (e == cudaSuccess)
     e = run_router(x, w_router, logits_in, T, d, E, top_k, o, dt, t.logits, t.idx, t.w, nullptr,
@@ -906,43 +987,71 @@ moe_status_t moe_forward_train(const void* x, const void* w_router, const float*
   if (e == cudaSuccess && logits_in && T > 0)   // the backward reads the logits from the state
     e = cudaMemcpyAsync(t.logits, logits_in, static_cast<size_t>(T) * E * sizeof(float),
                         cudaMemcpyDeviceToDevice, s);
+  // [HP] MoE.forward with score_before_experts: the routed rows are scaled by
+  // their weights (the state's x_perm holds the scaled rows)
   if (e == cudaSuccess)
     e = launch_dispatch(p, x, t.idx, d, dt, t.counts, t.offsets, t.src_row, t.dst_pos, t.x_perm,
-                        t.disp_ws, t.status, s, /*hist_done=*/T > 0);
+                        t.disp_ws, t.status, s, /*hist_done=*/T > 0, before ? t.w : nullptr);
   if (e == cudaSuccess && N > 0)
     e = launch_swiglu_tc_train(t.x_perm, t.offsets, w1, w3, w2, N, d, h, E, t.y, t.H, t.GU,
                                t.status, s);
+  // [HP] MoE.forward: shared_expert(x_flat), kept for its backward
+  if (e == cudaSuccess && hs > 0 && T > 0) {
+    e = launch_single_segment(t.offsets_s, T, s);
+    if (e == cudaSuccess)
+      e = launch_swiglu_tc_train(x, t.offsets_s, shared->w1, shared->w3, shared->w2, T, d, hs, 1,
+                                 t.ys, t.Hs, t.GUs, t.status, s);
+  }
   if (e == cudaSuccess)
-    e = launch_combine(t.y, t.dst_pos, nullptr, t.w, T, d, N, top_k, dt, out, s);
+    e = launch_combine(t.y, t.dst_pos, nullptr, before ? nullptr : t.w, T, d, N, top_k, dt, out,
+                       s, hs > 0 ? t.ys : nullptr);
   return cuda_status(e, "moe_forward_train");
 }
 
-moe_status_t moe_backward(const void* dout, const void* x, const void* w_router, const void* w1,
-                          const void* w3, const void* w2, int T, int d, int E, int top_k, int h,
-                          const moe_router_options_t* opts, moe_dtype_t dt, const void* state,
-                          void* dx, float* d_logits, void* dw_router, void* dw1, void* dw3,
-                          void* dw2, void* ws, size_t ws_bytes, void* stream) {
+moe_status_t moe_forward_train(const void* x, const void* w_router, const float* logits_in,
+                               const void* w1, const void* w3, const void* w2, int T, int d,
+                               int E, int top_k, int h, const moe_router_options_t* opts,
+                               moe_dtype_t dt, void* out, void* state, size_t state_bytes,
+                               void* stream) {
+  return moe_forward_train_ex(x, w_router, logits_in, w1, w3, w2, T, d, E, top_k, h, opts,
+                              nullptr, dt, out, state, state_bytes, stream);
+}
+
+moe_status_t moe_backward_ex(const void* dout, const void* x, const void* w_router,
+                             const void* w1, const void* w3, const void* w2, int T, int d, int E,
+                             int top_k, int h, const moe_router_options_t* opts,
+                             const moe_shared_expert_t* shared, moe_dtype_t dt,
+                             const void* state, void* dx, float* d_logits, void* dw_router,
+                             void* dw1, void* dw3, void* dw2, void* dws1, void* dws3, void* dws2,
+                             void* ws, size_t ws_bytes, void* stream) {
   const moe_router_options_t o = opts ? *opts : default_options();
   if (moe_status_t st = check_train(T, d, E, top_k, h, o, dt)) return st;
   MOE_CHECK_ARG(std::isfinite(o.route_scale) && o.route_scale != 0.0f, "bad route_scale");
+  MOE_CHECK_ARG(std::isfinite(o.aux_loss_coef), "aux_loss_coef must be finite");
+  if (moe_status_t st = check_shared(shared, T, d, dt)) return st;
+  const int hs = shared ? shared->h : 0;
+  const bool before = o.score_before_experts != 0;
   MOE_CHECK_ARG(w1 && w3 && w2 && dw1 && dw3 && dw2, "w1, w3, w2, dw1, dw3, dw2 are required");
   MOE_CHECK_ARG(!dw_router || (x && w_router), "dw_router needs x and w_router");
+  MOE_CHECK_ARG(!shared || (dws1 && dws3 && dws2 && x), "a shared expert needs x, dws1, dws3, dws2");
+  MOE_CHECK_ARG(!before || x, "score_before_experts needs x");
   MOE_CHECK_ARG(aligned16(w1) && aligned16(w3) && aligned16(w2) && aligned16(dw1) &&
                     aligned16(dw3) && aligned16(dw2) && aligned16(dw_router) &&
-                    aligned16(x) && aligned16(w_router),
+                    aligned16(x) && aligned16(w_router) && aligned16(dws1) && aligned16(dws3) &&
+                    aligned16(dws2),
                 "weights, gradients and x must be 16-byte aligned");
   if (T > 0) {
     MOE_CHECK_ARG(dout && dx, "dout and dx are required");
     MOE_CHECK_ARG(aligned16(dout) && aligned16(dx), "dout, dx must be 16-byte aligned");
   }
   MOE_CHECK_ARG(state != nullptr && ws != nullptr, "state and ws are required");
-  const BackwardWs need = carve_backward(nullptr, T, d, E, top_k, h);
+  const BackwardWs need = carve_backward(nullptr, T, d, E, top_k, h, hs);
   if (ws_bytes < need.bytes) {
     set_last_error("backward workspace %zu < %zu", ws_bytes, need.bytes);
     return MOE_ERR_WORKSPACE;
   }
-  const TrainState t = carve_train(const_cast<void*>(state), T, d, E, top_k, h);
-  const BackwardWs b = carve_backward(ws, T, d, E, top_k, h);
+  const TrainState t = carve_train(const_cast<void*>(state), T, d, E, top_k, h, hs);
+  const BackwardWs b = carve_backward(ws, T, d, E, top_k, h, hs);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int N = T * top_k;
   const bool gate = dw_router != nullptr;
@@ -953,25 +1062,59 @@ moe_status_t moe_backward(const void* dout, const void* x, const void* w_router,
     if (e == cudaSuccess) e = cudaMemsetAsync(dw3, 0, wbytes, s);
     if (e == cudaSuccess) e = cudaMemsetAsync(dw2, 0, wbytes, s);
     if (e == cudaSuccess && gate) e = cudaMemsetAsync(dw_router, 0, static_cast<size_t>(E) * d * 2, s);
+    if (shared) {
+      const size_t sbytes = static_cast<size_t>(hs) * d * 2;
+      if (e == cudaSuccess) e = cudaMemsetAsync(dws1, 0, sbytes, s);
+      if (e == cudaSuccess) e = cudaMemsetAsync(dws3, 0, sbytes, s);
+      if (e == cudaSuccess) e = cudaMemsetAsync(dws2, 0, sbytes, s);
+    }
     return cuda_status(e, "moe_backward");
   }
-  // combine -> experts -> router -> dispatch, all on `s`
+  // combine -> experts -> (scaled dispatch) -> router -> shared expert ->
+  // dispatch, all on `s`.  With score_before_experts the combine was
+  // unweighted (its backward has no weight gradient) and the weights' gradient
+  // comes from the scaled rows: d topk_w[t, j] = <dx_perm[p(t, j)], x[t]>.
   if (e == cudaSuccess)
-    e = launch_combine_backward(dout, t.y, t.dst_pos, t.w, T, d, N, top_k, dt, b.dY, b.dtw, s);
+    e = launch_combine_backward(dout, t.y, t.dst_pos, before ? nullptr : t.w, T, d, N, top_k, dt,
+                                b.dY, before ? nullptr : b.dtw, s);
   if (e == cudaSuccess)
     e = launch_swiglu_bwd_tc(t.x_perm, t.offsets, w1, w3, w2, t.H, t.GU, b.dY, N, d, h, E, b.dXp,
                              dw1, dw3, dw2, b.dGU, b.status, s);
+  if (e == cudaSuccess && before)
+    e = launch_combine_backward(x, b.dXp, t.dst_pos, nullptr, T, d, N, top_k, dt, nullptr, b.dtw,
+                                s);
   if (e == cudaSuccess)
     e = launch_router_backward(t.logits, t.idx, b.dtw, T, E, top_k,
                                o.score == MOE_SCORE_SIGMOID, o.renormalize, o.route_scale,
-                               d_logits, gate ? b.dz16 : nullptr, s);
+                               d_logits, gate ? b.dz16 : nullptr, s,
+                               o.aux_loss_coef != 0.0f ? t.counts : nullptr,
+                               lb_grad_scale(o.aux_loss_coef, E, T, top_k));
   if (e == cudaSuccess && gate)
     e = launch_gate_backward_tc(b.dz16, x, w_router, T, d, E, dw_router, b.dxr, b.off2, b.gpart,
                                 b.status, s);
+  // the shared expert: a one-segment grouped SwiGLU backward over every token
+  // with the layer's upstream gradient
+  if (e == cudaSuccess && hs > 0)
+    e = launch_swiglu_bwd_tc(x, t.offsets_s, shared->w1, shared->w3, shared->w2, t.Hs, t.GUs,
+                             dout, T, d, hs, 1, b.dXs, dws1, dws3, dws2, b.dGUs, b.status, s);
+  // dx[t] = sum_j (w[t, j] with score_before_experts) dx_perm[p(t, j)] + the
+  // router's share + the shared expert's share
+  const void* add1 = gate ? b.dxr : (hs > 0 ? b.dXs : nullptr);
+  const void* add2 = (gate && hs > 0) ? b.dXs : nullptr;
   if (e == cudaSuccess)
-    e = launch_combine(b.dXp, t.dst_pos, nullptr, nullptr, T, d, N, top_k, dt, dx, s,
-                       gate ? b.dxr : nullptr);
+    e = launch_combine(b.dXp, t.dst_pos, nullptr, before ? t.w : nullptr, T, d, N, top_k, dt, dx,
+                       s, add1, add2);
   return cuda_status(e, "moe_backward");
+}
+
+moe_status_t moe_backward(const void* dout, const void* x, const void* w_router, const void* w1,
+                          const void* w3, const void* w2, int T, int d, int E, int top_k, int h,
+                          const moe_router_options_t* opts, moe_dtype_t dt, const void* state,
+                          void* dx, float* d_logits, void* dw_router, void* dw1, void* dw3,
+                          void* dw2, void* ws, size_t ws_bytes, void* stream) {
+  return moe_backward_ex(dout, x, w_router, w1, w3, w2, T, d, E, top_k, h, opts, nullptr, dt,
+                         state, dx, d_logits, dw_router, dw1, dw3, dw2, nullptr, nullptr, nullptr,
+                         ws, ws_bytes, stream);
 }
 
 // ------------------------------------------------------------------ forward
@@ -1035,7 +1178,7 @@ moe_status_t moe_forward_ex(const void* x, const void* w_router, const float* lo
   float* w = topk_w ? topk_w : f.w;
   const int R = ep_ranks;
   cudaError_t e = cudaMemsetAsync(f.status, 0, sizeof(int), s);
-  const DispatchPlan p = make_dispatch_plan(T, E, top_k, R);
+  const DispatchPlan p = layer_dispatch_plan(T, d, E, top_k, R, dt);
   // The router's top-k kernel also writes the dispatch histogram table.
   if (e == cudaSuccess)
     e = run_router(x, w_router, logits_in, T, d, E, top_k, o, dt, logits_out, idx, w, nullptr,

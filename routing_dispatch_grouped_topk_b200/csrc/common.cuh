@@ -64,6 +64,25 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
 
+// ----------------------------------------------------------- routing keys
+// Order-preserving map of a float score to int32 (NaN must be mapped to -inf
+// first; -0 and +0 compare equal, as floats do).
+__device__ __forceinline__ int score_key(float f) {
+  f += 0.0f;
+  const int i = __float_as_int(f);
+  return i ^ ((i >> 31) & 0x7fffffff);
+}
+__device__ __forceinline__ float key_score(int k) { return __int_as_float(k ^ ((k >> 31) & 0x7fffffff)); }
+
+// Bin of a routed copy in the dispatch: the expert (R = 1), or on the
+// rank-major EP layout (destination rank g, source rank r = t / S, local
+// expert l) numbered (g * R + r) * L + l.
+__device__ __forceinline__ int dispatch_key(int e, int t, int R, int L, int S) {
+  if (R == 1) return e;
+  const int g = e / L, l = e - g * L, r = t / S;
+  return (g * R + r) * L + l;
+}
+
 // ------------------------------------------------------------------- timers
 __device__ __forceinline__ unsigned long long global_ns() {
   unsigned long long t;

@@ -3,6 +3,7 @@
 // cudaError_t of its launches.  `status` points at the device status word.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -10,6 +11,12 @@
 #include "../../include/moe.h"
 
 namespace moe {
+
+namespace tc {
+// 2-D bf16 tensor map over a row-major [rows, inner] array, box [box_rows, 64],
+// 128-byte swizzle, zero fill outside the array.
+bool make_tmap(CUtensorMap* tm, const void* ptr, uint64_t inner, uint64_t rows, uint32_t box_rows);
+}  // namespace tc
 
 int num_sms();                               // SM count of the current device
 void set_last_error(const char* fmt, ...);   // thread-local text for moe_last_error
@@ -28,6 +35,37 @@ RouterPlan router_plan(int T, int d);
 // tcgen05 router GEMM (bf16, E <= 256): fp32 partial logits [ksplit, T, E].
 cudaError_t launch_router_tc(const void* x, const void* w_router, int T, int d, int E,
                              float* logits_part, int* status, cudaStream_t s);
+// Fused tcgen05 router (bf16, E <= 256, no node-limited groups): the gate
+// contraction on clusters of C CTAs per 128-token tile, the partial logits
+// reduced through distributed shared memory, then scores, top-k and weights
+// by one thread per token -- one kernel.  `plan`/`blk` as launch_router_topk
+// (the dispatch histogram); `counts` (or null) is written through the
+// per-CTA table `counts_part` ([grid, E] ints) by a second kernel;
+// tokens_per_expert and lb (2E floats) are added to.  With clear_status the
+// kernel clears the status word itself (it is the call's only writer).
+struct RouterFusedPlan {
+  int bn;           // accumulator columns (E rounded up to 32, 64, 128 or 256)
+  int tiles;        // 128-token tiles
+  int C;            // CTAs per tile (cluster size)
+  int kb_total, kb_per_cta;
+  int pitch;        // fp32 row pitch of the partial logits in shared memory
+  int region;       // shared bytes before the barriers (stages / exchange)
+  int smem;         // dynamic shared memory of a CTA
+  int grid;
+  bool ok;          // the plan fits the kernel's shared memory
+};
+struct DispatchPlan;
+RouterFusedPlan router_fused_plan(int T, int d, int E, const DispatchPlan* plan);
+// The dispatch plan of a whole-layer call: token blocks small enough that
+// every CTA of the fused router owns whole blocks.
+DispatchPlan layer_dispatch_plan(int T, int d, int E, int top_k, int R, moe_dtype_t dt);
+struct RouterOptions;
+cudaError_t launch_router_fused(const void* x, const void* w_router, int T, int d, int E,
+                                int top_k, int renorm, const RouterOptions& o, float* logits_out,
+                                int32_t* topk_idx, float* topk_w, int32_t* counts,
+                                int32_t* counts_part, float* tokens_per_expert, float* lb,
+                                const DispatchPlan* plan, int32_t* blk, int* status,
+                                bool clear_status, cudaStream_t s);
 // CUDA-core fp32 logits (x fp32 or bf16) into `logits` [T, E].
 cudaError_t launch_router_logits_simt(const void* x, const void* w_router, int T, int d, int E,
                                       moe_dtype_t dt, float* logits, cudaStream_t s);
@@ -38,7 +76,10 @@ struct DispatchPlan {
   int tb;                 // tokens per block
   int nblk;
 };
-DispatchPlan make_dispatch_plan(int T, int E, int top_k, int R);
+// max_tb caps the tokens per block (a power of two >= 8): inside the layer
+// the fused router writes the histogram table, and each of its CTAs owns
+// 128 / C tokens (layer_dispatch_plan).
+DispatchPlan make_dispatch_plan(int T, int E, int top_k, int R, int max_tb = 128);
 size_t dispatch_ws_bytes(const DispatchPlan& p);
 // Host-side argument rules shared by every dispatch entry point (returns
 // MOE_OK or MOE_ERR_INVALID_ARG with the text for moe_last_error set).
@@ -85,18 +126,23 @@ cudaError_t launch_dispatch(const DispatchPlan& p, const void* x, const int32_t*
                             const float* row_w = nullptr);
 
 // ---- regroup ----------------------------------------------------------------
+// One kernel (the segment tables are rebuilt in every block's shared
+// memory).  own_status: the call's only kernel, which writes the whole status
+// word (no clearing before it); otherwise it only adds MOE_DEV_BAD_COUNTS.
 size_t regroup_ws_bytes(int G, int R, int L);
 cudaError_t launch_regroup(const void* in, const int32_t* counts_rm, int G, int R, int L,
                            int rows, int d, moe_dtype_t dt, void* out, int32_t* counts_em,
                            int32_t* offsets_em, int32_t* perm, int32_t* perm_inv, void* ws,
-                           int* status, cudaStream_t s);
+                           int* status, cudaStream_t s, bool own_status = false);
 
 // ---- combine ----------------------------------------------------------------
-// shared [T, d] (or null): a row added to each token's weighted sum in fp32
-// before the rounding (the shared expert's output).
+// shared, shared2 [T, d] (or null): rows added to each token's weighted sum
+// in fp32 before the rounding (the shared expert's output; in the backward
+// the router's and the shared expert's shares of dx).
 cudaError_t launch_combine(const void* y, const int32_t* dst_pos, const int32_t* row_map,
                            const float* topk_w, int T, int d, int N, int top_k, moe_dtype_t dt,
-                           void* out, cudaStream_t s, const void* shared = nullptr);
+                           void* out, cudaStream_t s, const void* shared = nullptr,
+                           const void* shared2 = nullptr);
 // Backward of the combine: dy [N, d] (every slot p(t, j) = w[t, j] dout[t];
 // w = 1 when topk_w is null) and, if d_topk_w is given, the fp32 dot products
 // <dout[t], y[p(t, j)]> ([T, k]).
@@ -106,10 +152,17 @@ cudaError_t launch_combine_backward(const void* dout, const void* y, const int32
 // Router backward: dz = d(routing weights)/d(logits) applied to d_topk_w,
 // per token from the saved fp32 logits; dz32 [T, E] fp32 and dz16 [T, E]
 // bf16 are each optional.
+// With lb_counts (the expert counts of the forward, [E]) every selected
+// expert e's upstream gradient gets lb_scale * lb_counts[e] added (the
+// load-balance loss's gradient: lb_scale = coef * E / (T * T k)).
 cudaError_t launch_router_backward(const float* logits, const int32_t* topk_idx,
                                    const float* d_topk_w, int T, int E, int top_k, int sigmoid,
                                    int renorm, float scale, float* dz32, void* dz16,
-                                   cudaStream_t s);
+                                   cudaStream_t s, const int32_t* lb_counts = nullptr,
+                                   float lb_scale = 0.f);
+// counts [E] += histogram of idx [n] (counts cleared by the caller).
+cudaError_t launch_expert_hist(const int32_t* idx, long long n, int E, int32_t* counts,
+                               cudaStream_t s);
 // Gradients of the gate x . w_router^T for dz16 [T, E] bf16: dw_router =
 // dz^T x [E, d] and dx = dz w_router [T, d] (bf16, each optional); offsets2 is
 // device scratch for two ints.

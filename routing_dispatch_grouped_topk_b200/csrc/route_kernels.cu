@@ -14,11 +14,6 @@
 namespace moe {
 
 // --------------------------------------------------------------- dispatch
-__device__ __forceinline__ int dispatch_key(int e, int t, int R, int L, int S) {
-  if (R == 1) return e;
-  const int g = e / L, l = e - g * L, r = t / S;
-  return (g * R + r) * L + l;
-}
 
 // K1: histogram of the keys of each block of `tb` tokens, stored bin-major
 // (blk[bin * nblk + block]) so that K2 scans contiguous columns.
@@ -28,6 +23,9 @@ __global__ void dispatch_hist_kernel(const int32_t* __restrict__ idx, int T, int
   pdl_wait();
   pdl_trigger();
   extern __shared__ int hist[];
+  // the column scan's completion ticket sits after the table
+  if (blockIdx.x == 0 && threadIdx.x == 0)
+    blk[static_cast<size_t>(nbins) * gridDim.x] = 0;
   for (int i = threadIdx.x; i < nbins; i += blockDim.x) hist[i] = 0;
   __syncthreads();
   const int t0 = blockIdx.x * tb;
@@ -121,11 +119,19 @@ __device__ int block_scan_value(int v, int* warp_sums, int* total) {
 
 // K2: for every bin (one block per bin, grid-stride), the exclusive prefix of
 // its column over the token blocks, in place; the column total is counts[bin].
+// The last block to finish (a ticket counter after the table, zeroed by the
+// kernel that wrote the table) scans the totals into offsets[0..nbins] and
+// marks the slots that invalid expert ids left empty (src_row = -1): every
+// scatter block then reads only the entries of the bins it touches.
 __global__ void dispatch_colscan_kernel(int32_t* __restrict__ blk, int nblk, int nbins,
-                                        int32_t* __restrict__ counts) {
+                                        int32_t* __restrict__ counts,
+                                        int32_t* __restrict__ offsets,
+                                        int32_t* __restrict__ src_row, long long n_slots) {
   pdl_wait();
   pdl_trigger();
+  extern __shared__ int osm[];      // nbins (last block only)
   __shared__ int wsum[33];
+  __shared__ int last;
   for (int bin = blockIdx.x; bin < nbins; bin += gridDim.x) {
     int32_t* col = blk + static_cast<size_t>(bin) * nblk;
     int carry = 0;
@@ -139,6 +145,22 @@ __global__ void dispatch_colscan_kernel(int32_t* __restrict__ blk, int nblk, int
     }
     if (threadIdx.x == 0) counts[bin] = carry;
   }
+  // completion ticket: the block that takes the last one sees every count
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int* ticket = blk + static_cast<size_t>(nbins) * nblk;
+    last = atomicAdd(ticket, 1) == static_cast<int>(gridDim.x) - 1;
+  }
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  for (int i = threadIdx.x; i < nbins; i += blockDim.x) osm[i] = __ldcg(counts + i);
+  __syncthreads();
+  const int total = block_exclusive_scan(osm, nbins, wsum);
+  for (int i = threadIdx.x; i < nbins; i += blockDim.x) offsets[i] = osm[i];
+  if (threadIdx.x == 0) offsets[nbins] = total;
+  for (long long sl = total + threadIdx.x; sl < n_slots; sl += blockDim.x) src_row[sl] = -1;
 }
 
 // Eight bf16 or four fp32 values times w (fp32 product, rounded once).
@@ -154,64 +176,58 @@ __device__ __forceinline__ uint4 scale_vec(uint4 v, float w, int bf16) {
   return make_uint4(u[0], u[1], u[2], u[3]);
 }
 
-// K3: stable slot of every copy (warp 0), then the row copies (all warps):
-// each token row is read once and written to its k slots with 16-byte stores.
-// Each block also turns the bin totals into bin offsets (a block scan of
-// nbins values) and adds its column prefix; block 0 publishes the offsets
-// and marks slots left empty by invalid expert ids.
-__global__ void dispatch_scatter_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ idx,
+// K3: stable slot of every copy, then the row copies (all warps): each token
+// row is read once and written to its k slots with 16-byte stores.  A block
+// reads only what its own copies need: for every key it touches, the bin's
+// offset plus the block's column prefix; warp 0 then ranks the copies in
+// flat order (match.any + popc), so equal keys keep their flat order.
+__global__ void __launch_bounds__(1024) dispatch_scatter_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ idx,
                                         int T, int k, int E, int R, int L, int S, int tb,
                                         int nbins, const int32_t* __restrict__ blk,
-                                        const int32_t* __restrict__ counts,
-                                        int32_t* __restrict__ offsets,
+                                        const int32_t* __restrict__ offsets,
                                         int32_t* __restrict__ src_row,
                                         int32_t* __restrict__ dst_pos, uint4* __restrict__ x_perm,
                                         int row_vec, const float* __restrict__ row_w, int bf16) {
   pdl_wait();
   pdl_trigger();
   extern __shared__ int sm[];
-  int* run = sm;                   // nbins
-  int* wsum = sm + nbins;          // 33
-  int* slot = wsum + 33;           // tb * k
+  int* run = sm;                   // nbins (only the touched keys are set)
+  int* slot = sm + nbins;          // tb * k: the key, then the slot of each copy
   const int nblk = gridDim.x;
   const int t0 = blockIdx.x * tb;
   const int t1 = min(T, t0 + tb);
   const int nf = (t1 - t0) * k;
-  for (int i = threadIdx.x; i < nbins; i += blockDim.x) run[i] = counts[i];
-  __syncthreads();
-  const int total = block_exclusive_scan(run, nbins, wsum);
-  if (blockIdx.x == 0) {
-    for (int i = threadIdx.x; i < nbins; i += blockDim.x) offsets[i] = run[i];
-    if (threadIdx.x == 0) offsets[nbins] = total;
-    for (long long s = total + threadIdx.x; s < 1LL * T * k; s += blockDim.x) src_row[s] = -1;
+  const long long f0 = 1LL * t0 * k;
+  for (int i = threadIdx.x; i < nf; i += blockDim.x) {
+    const int e = idx[f0 + i];
+    int key = -1;
+    if (static_cast<unsigned>(e) < static_cast<unsigned>(E)) {
+      key = dispatch_key(e, static_cast<int>((f0 + i) / k), R, L, S);
+      // every copy with this key writes the same base (benign)
+      run[key] = offsets[key] + blk[static_cast<size_t>(key) * nblk + blockIdx.x];
+    }
+    slot[i] = key;
   }
-  for (int i = threadIdx.x; i < nbins; i += blockDim.x)
-    run[i] += blk[static_cast<size_t>(i) * nblk + blockIdx.x];
   __syncthreads();
   if (threadIdx.x < 32) {
     const int lane = threadIdx.x;
     const unsigned lt = (1u << lane) - 1u;
     for (int c0 = 0; c0 < nf; c0 += 32) {
       const int i = c0 + lane;
-      const long long f = 1LL * t0 * k + i;
-      int key = -1 - lane;                       // unique: never matches
-      if (i < nf) {
-        const int e = idx[f];
-        if (static_cast<unsigned>(e) < static_cast<unsigned>(E))
-          key = dispatch_key(e, static_cast<int>(f / k), R, L, S);
-      }
-      const unsigned peers = __match_any_sync(0xffffffffu, key);
+      const int key = i < nf ? slot[i] : -1;
+      const unsigned peers = __match_any_sync(0xffffffffu, key >= 0 ? key : -1 - lane);
       const int rank = __popc(peers & lt);
       const int leader = __ffs(peers) - 1;
-      int s = -1;
-      if (key >= 0) s = run[key] + rank;
+      int sl = -1;
+      if (key >= 0) sl = run[key] + rank;
       __syncwarp();
       if (key >= 0 && lane == leader) run[key] += __popc(peers);
       __syncwarp();
       if (i < nf) {
-        dst_pos[f] = s;
-        slot[i] = s;
-        if (s >= 0) src_row[s] = static_cast<int>(f / k);
+        const long long f = f0 + i;
+        dst_pos[f] = sl;
+        slot[i] = sl;
+        if (sl >= 0) src_row[sl] = static_cast<int>(f / k);
       }
     }
   }
@@ -246,7 +262,7 @@ __global__ void dispatch_scatter_kernel(const uint4* __restrict__ x, const int32
   }
 }
 
-DispatchPlan make_dispatch_plan(int T, int E, int top_k, int R) {
+DispatchPlan make_dispatch_plan(int T, int E, int top_k, int R, int max_tb) {
   DispatchPlan p{};
   p.T = T;
   p.k = top_k;
@@ -255,17 +271,24 @@ DispatchPlan make_dispatch_plan(int T, int E, int top_k, int R) {
   p.L = E / R;
   p.S = R > 1 ? std::max(1, cdiv(T, R)) : std::max(T, 1);
   p.nbins = E * R;
-  // About four blocks per SM, so that the row copies balance across SMs;
-  // small blocks also keep the warp-serial ranking short.
+  // About four blocks per SM, so that the row copies balance across SMs
+  // (small blocks also keep the warp-serial ranking short), and at most
+  // 2^17 entries in the histogram table: its write and its column scan cost
+  // nblk * nbins, which with the E * R bins of the rank-major layout would
+  // otherwise outweigh the copies.
   int tb = 8;
-  while (tb < 128 && cdiv(T, tb * 2) >= 4 * 148) tb *= 2;
+  while (tb < std::min(128, max_tb) &&
+         (cdiv(T, tb * 2) >= 4 * 148 ||
+          static_cast<long long>(cdiv(T, tb)) * p.nbins > (1LL << 17)))
+    tb *= 2;
   p.tb = tb;
   p.nblk = std::max(1, cdiv(T, tb));
   return p;
 }
 
 size_t dispatch_ws_bytes(const DispatchPlan& p) {
-  return align_up(static_cast<size_t>(p.nblk) * p.nbins * sizeof(int32_t), 256);
+  // the histogram table [nbins, nblk], then the column scan's ticket
+  return align_up((static_cast<size_t>(p.nblk) * p.nbins + 1) * sizeof(int32_t), 256);
 }
 
 cudaError_t launch_dispatch(const DispatchPlan& p, const void* x, const int32_t* topk_idx,
@@ -281,81 +304,85 @@ cudaError_t launch_dispatch(const DispatchPlan& p, const void* x, const int32_t*
   if (!hist_done)
     launch_k(dispatch_hist_kernel, dim3(p.nblk), dim3(256), p.nbins * sizeof(int), s, topk_idx,
              p.T, p.k, p.E, p.R, p.L, p.S, p.tb, p.nbins, blk, status);
-  launch_k(dispatch_colscan_kernel, dim3(std::min(p.nbins, num_sms() * 8)), dim3(256), 0, s, blk,
-           p.nblk, p.nbins, counts);
+  launch_k(dispatch_colscan_kernel, dim3(std::min(p.nbins, num_sms() * 8)), dim3(256),
+           p.nbins * sizeof(int), s, blk, p.nblk, p.nbins, counts, offsets, src_row,
+           1LL * p.T * p.k);
   const int elt = dt == MOE_BF16 ? 2 : 4;
   const int row_vec = d * elt / 16;
-  const size_t sm3 = (p.nbins + 33 + p.tb * p.k) * sizeof(int);
-  launch_k(dispatch_scatter_kernel, dim3(p.nblk), dim3(256), sm3, s,
+  const size_t sm3 = (p.nbins + p.tb * p.k) * sizeof(int);
+  // a warp per token row at a time: more warps for larger blocks
+  const int threads = std::min(1024, std::max(256, 16 * p.tb));
+  launch_k(dispatch_scatter_kernel, dim3(p.nblk), dim3(threads), sm3, s,
            static_cast<const uint4*>(x), topk_idx, p.T, p.k, p.E, p.R, p.L, p.S, p.tb, p.nbins,
-           blk, counts, offsets, src_row, dst_pos, static_cast<uint4*>(x_perm), row_vec, row_w,
+           blk, offsets, src_row, dst_pos, static_cast<uint4*>(x_perm), row_vec, row_w,
            dt == MOE_BF16 ? 1 : 0);
   return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------- regroup
-// Segment tables (one block): segments are numbered in OUTPUT order
-// o = (g*L + l)*R + r; in_start[o] is where segment (g, r, l) starts in the
-// rank-major input, out_start[o] (o = 0..S) where it starts in the output.
-__global__ void regroup_scan_kernel(const int32_t* __restrict__ counts_rm, int G, int R, int L,
-                                    int rows, int32_t* __restrict__ in_start,
-                                    int32_t* __restrict__ out_start,
-                                    int32_t* __restrict__ counts_em,
-                                    int32_t* __restrict__ offsets_em, int* flag, int* status) {
+// One kernel: every block builds the segment tables in shared memory from
+// counts_rm (two block scans of S = G*R*L counts), then its warps copy rows
+// grid-stride.  Segments are numbered in OUTPUT order o = (g*L + l)*R + r;
+// in_start[o] is where segment (g, r, l) starts in the rank-major input,
+// out_start[o] (o = 0..S) where it starts in the output; a row's segment is
+// found by binary search over out_start in shared memory.  Block 0 writes
+// counts_em / offsets_em and the status; if the counts are negative or do
+// not add up to `rows`, nothing is copied.
+__global__ void __launch_bounds__(256) regroup_kernel(
+    const uint4* __restrict__ in, const int32_t* __restrict__ counts_rm, int G, int R, int L,
+    int rows, int row_vec, uint4* __restrict__ out, int32_t* __restrict__ counts_em,
+    int32_t* __restrict__ offsets_em, int32_t* __restrict__ perm, int32_t* __restrict__ perm_inv,
+    int* status, int own_status) {
   pdl_wait();
   pdl_trigger();
   extern __shared__ int sm[];
   const int S = G * R * L;
-  int* a = sm;            // S
-  int* wsum = sm + S;     // 33
+  int* a = sm;                 // S: scan scratch
+  int* in_start = sm + S;      // S (output numbering)
+  int* out_start = sm + 2 * S; // S + 1
+  __shared__ int wsum[33];
   __shared__ int bad;
   if (threadIdx.x == 0) bad = 0;
   __syncthreads();
   // input order (g, r, l): exclusive scan of the counts as given
   for (int i = threadIdx.x; i < S; i += blockDim.x) {
     const int c = counts_rm[i];
-    if (c < 0) atomicOr(&bad, 1);
+    if (c < 0) bad = 1;
     a[i] = max(c, 0);
   }
   __syncthreads();
   const int total = block_exclusive_scan(a, S, wsum);
-  // scatter the input starts into output numbering
   for (int i = threadIdx.x; i < S; i += blockDim.x) {
     const int g = i / (R * L), r = (i / L) % R, l = i % L;
     in_start[(g * L + l) * R + r] = a[i];
   }
-  __syncthreads();
   for (int o = threadIdx.x; o < S; o += blockDim.x) {
     const int g = o / (L * R), l = (o / R) % L, r = o % R;
-    a[o] = max(counts_rm[(g * R + r) * L + l], 0);
+    out_start[o] = max(counts_rm[(g * R + r) * L + l], 0);
   }
   __syncthreads();
-  block_exclusive_scan(a, S, wsum);
-  for (int o = threadIdx.x; o < S; o += blockDim.x) out_start[o] = a[o];
-  if (threadIdx.x == 0) {
-    out_start[S] = total;
-    const int ok = (bad == 0) && (total == rows);
-    *flag = ok;
-    if (!ok) set_status(status, MOE_DEV_BAD_COUNTS);
+  block_exclusive_scan(out_start, S, wsum);
+  if (threadIdx.x == 0) out_start[S] = total;
+  __syncthreads();
+  const bool ok = (bad == 0) && (total == rows);
+  if (blockIdx.x == 0) {
+    // block 0 is the only writer: as the call's only kernel it writes the
+    // whole status word, inside a longer sequence it adds its bit
+    if (threadIdx.x == 0) {
+      if (own_status)
+        *status = ok ? 0 : MOE_DEV_BAD_COUNTS;
+      else if (!ok)
+        set_status(status, MOE_DEV_BAD_COUNTS);
+    }
+    // expert-major counts / offsets: sum over r
+    for (int gl = threadIdx.x; gl < G * L; gl += blockDim.x) {
+      const int o0 = gl * R;
+      counts_em[gl] = out_start[o0 + R] - out_start[o0];
+      offsets_em[gl] = out_start[o0];
+    }
+    if (threadIdx.x == 0) offsets_em[G * L] = total;
   }
-  // expert-major counts / offsets: sum over r
-  for (int gl = threadIdx.x; gl < G * L; gl += blockDim.x) {
-    int c = 0;
-    for (int r = 0; r < R; ++r) c += max(counts_rm[((gl / L) * R + r) * L + gl % L], 0);
-    counts_em[gl] = c;
-    offsets_em[gl] = a[gl * R];
-  }
-  if (threadIdx.x == 0) offsets_em[G * L] = total;
-}
-
-__global__ void regroup_copy_kernel(const uint4* __restrict__ in, int rows, int row_vec, int S,
-                                    const int32_t* __restrict__ in_start,
-                                    const int32_t* __restrict__ out_start, const int* flag,
-                                    uint4* __restrict__ out, int32_t* __restrict__ perm,
-                                    int32_t* __restrict__ perm_inv) {
-  pdl_wait();
-  pdl_trigger();
-  if (!*flag) return;
+  if (!ok) return;
   const int lane = threadIdx.x & 31;
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int nw = (gridDim.x * blockDim.x) >> 5;
@@ -370,35 +397,56 @@ __global__ void regroup_copy_kernel(const uint4* __restrict__ in, int rows, int 
       perm[o] = src;
       if (perm_inv) perm_inv[src] = o;
     }
-    const uint4* s = in + static_cast<size_t>(src) * row_vec;
-    uint4* dst = out + static_cast<size_t>(o) * row_vec;
-    for (int c = lane; c < row_vec; c += 32) dst[c] = s[c];
+    const uint4* sp = in + static_cast<size_t>(src) * row_vec;
+    uint4* dp = out + static_cast<size_t>(o) * row_vec;
+    // up to four 16-byte loads per lane in flight before the stores
+    for (int c0 = 0; c0 < row_vec; c0 += 128) {
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int c = c0 + u * 32 + lane;
+        if (c < row_vec) v[u] = sp[c];
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int c = c0 + u * 32 + lane;
+        if (c < row_vec) dp[c] = v[u];
+      }
+    }
   }
 }
 
 size_t regroup_ws_bytes(int G, int R, int L) {
-  const size_t S = static_cast<size_t>(G) * R * L;
-  return align_up((2 * S + 1) * sizeof(int32_t) + 16, 256);
+  (void)G;
+  (void)R;
+  (void)L;
+  return 0;
 }
 
 cudaError_t launch_regroup(const void* in, const int32_t* counts_rm, int G, int R, int L,
                            int rows, int d, moe_dtype_t dt, void* out, int32_t* counts_em,
                            int32_t* offsets_em, int32_t* perm, int32_t* perm_inv, void* ws,
-                           int* status, cudaStream_t s) {
+                           int* status, cudaStream_t s, bool own_status) {
+  (void)ws;
   const int S = G * R * L;
-  int32_t* in_start = static_cast<int32_t*>(ws);
-  int32_t* out_start = in_start + S;
-  int* flag = reinterpret_cast<int*>(out_start + S + 1);
-  launch_k(regroup_scan_kernel, dim3(1), dim3(1024), (S + 33) * sizeof(int), s, counts_rm, G, R,
-           L, rows, in_start, out_start, counts_em, offsets_em, flag, status);
-  if (rows > 0) {
-    const int elt = dt == MOE_BF16 ? 2 : 4;
-    const int row_vec = d * elt / 16;
-    const int blocks = std::min(cdiv(rows, 8), num_sms() * 8);
-    launch_k(regroup_copy_kernel, dim3(blocks), dim3(256), 0, s, static_cast<const uint4*>(in),
-             rows, row_vec, S, in_start, out_start, flag, static_cast<uint4*>(out), perm,
-             perm_inv);
+  const size_t smem = (3 * static_cast<size_t>(S) + 1) * sizeof(int);
+  static int configured[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (smem > 48 * 1024 && dev < 64 && !configured[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(regroup_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         3 * kMaxSegments * 4 + 16);
+    if (e != cudaSuccess) return e;
+    configured[dev] = 1;
   }
+  const int elt = dt == MOE_BF16 ? 2 : 4;
+  const int row_vec = rows > 0 ? d * elt / 16 : 0;
+  // one block when there is nothing to copy (the tables are still written)
+  const int blocks = rows > 0 ? std::min(cdiv(rows, 8), num_sms() * 4) : 1;
+  launch_k(regroup_kernel, dim3(blocks), dim3(256), smem, s, static_cast<const uint4*>(in),
+           counts_rm, G, R, L, rows, row_vec, static_cast<uint4*>(out), counts_em, offsets_em,
+           perm, perm_inv, status, own_status ? 1 : 0);
   return cudaGetLastError();
 }
 
@@ -412,7 +460,7 @@ cudaError_t launch_regroup(const void* in, const int32_t* counts_rm, int G, int 
 template <bool BF16, int KMAX>
 __device__ __forceinline__ uint4 combine_chunk(const uint4 (&v)[KMAX], const float (&wt)[KMAX],
                                                const int (&pos)[KMAX], int k,
-                                               const uint4* shared) {
+                                               const uint4* shared, const uint4* shared2) {
   float acc[8];
 #pragma unroll
   for (int q = 0; q < 8; ++q) acc[q] = 0.f;
@@ -436,8 +484,13 @@ __device__ __forceinline__ uint4 combine_chunk(const uint4 (&v)[KMAX], const flo
       acc[3] = fmaf(wj, __uint_as_float(v[j].w), acc[3]);
     }
   }
-  if (shared) {   // [HP] MoE.forward: out + shared_expert(x)
-    const uint4 sv = *shared;
+  // [HP] MoE.forward: out + shared_expert(x); in the backward, the router's
+  // and the shared expert's shares of dx
+  const uint4* adds[2] = {shared, shared2};
+#pragma unroll
+  for (int a = 0; a < 2; ++a) {
+    if (!adds[a]) continue;
+    const uint4 sv = *adds[a];
     if (BF16) {
       acc[0] += bf16_lo(sv.x);
       acc[1] += bf16_hi(sv.x);
@@ -465,7 +518,8 @@ template <bool BF16, int KMAX>
 __global__ void __launch_bounds__(256) combine_kernel(
     const uint4* __restrict__ y, const int32_t* __restrict__ dst_pos,
     const int32_t* __restrict__ row_map, const float* __restrict__ w, int T, int row_vec, int N,
-    int k, const uint4* __restrict__ shared, uint4* __restrict__ out) {
+    int k, const uint4* __restrict__ shared, const uint4* __restrict__ shared2,
+    uint4* __restrict__ out) {
   pdl_wait();
   pdl_trigger();
   const int lane = threadIdx.x & 31;
@@ -504,9 +558,9 @@ __global__ void __launch_bounds__(256) combine_kernel(
       for (int h = 0; h < 2; ++h) {
         const int c = c0 + 32 * h;
         if (c >= row_vec) break;
-        orow[c] = combine_chunk<BF16, KMAX>(v[h], wt, pos, k,
-                                            shared ? shared + static_cast<size_t>(t) * row_vec + c
-                                                   : nullptr);
+        const size_t o = static_cast<size_t>(t) * row_vec + c;
+        orow[c] = combine_chunk<BF16, KMAX>(v[h], wt, pos, k, shared ? shared + o : nullptr,
+                                            shared2 ? shared2 + o : nullptr);
       }
     }
   }
@@ -515,33 +569,36 @@ __global__ void __launch_bounds__(256) combine_kernel(
 template <bool BF16>
 static void combine_launch(const uint4* y, const int32_t* dst_pos, const int32_t* row_map,
                            const float* w, int T, int row_vec, int N, int k,
-                           const uint4* shared, uint4* out, int blocks, cudaStream_t s) {
+                           const uint4* shared, const uint4* shared2, uint4* out, int blocks,
+                           cudaStream_t s) {
   if (k <= 1)
-    launch_k(combine_kernel<BF16, 1>, dim3(blocks), dim3(256), 0, s, y, dst_pos, row_map, w, T, row_vec, N, k, shared, out);
+    launch_k(combine_kernel<BF16, 1>, dim3(blocks), dim3(256), 0, s, y, dst_pos, row_map, w, T, row_vec, N, k, shared, shared2, out);
   else if (k <= 2)
-    launch_k(combine_kernel<BF16, 2>, dim3(blocks), dim3(256), 0, s, y, dst_pos, row_map, w, T, row_vec, N, k, shared, out);
+    launch_k(combine_kernel<BF16, 2>, dim3(blocks), dim3(256), 0, s, y, dst_pos, row_map, w, T, row_vec, N, k, shared, shared2, out);
   else if (k <= 4)
-    launch_k(combine_kernel<BF16, 4>, dim3(blocks), dim3(256), 0, s, y, dst_pos, row_map, w, T, row_vec, N, k, shared, out);
+    launch_k(combine_kernel<BF16, 4>, dim3(blocks), dim3(256), 0, s, y, dst_pos, row_map, w, T, row_vec, N, k, shared, shared2, out);
   else if (k <= 8)
-    launch_k(combine_kernel<BF16, 8>, dim3(blocks), dim3(256), 0, s, y, dst_pos, row_map, w, T, row_vec, N, k, shared, out);
+    launch_k(combine_kernel<BF16, 8>, dim3(blocks), dim3(256), 0, s, y, dst_pos, row_map, w, T, row_vec, N, k, shared, shared2, out);
   else
-    launch_k(combine_kernel<BF16, 16>, dim3(blocks), dim3(256), 0, s, y, dst_pos, row_map, w, T, row_vec, N, k, shared, out);
+    launch_k(combine_kernel<BF16, 16>, dim3(blocks), dim3(256), 0, s, y, dst_pos, row_map, w, T, row_vec, N, k, shared, shared2, out);
 }
 
 cudaError_t launch_combine(const void* y, const int32_t* dst_pos, const int32_t* row_map,
                            const float* topk_w, int T, int d, int N, int top_k, moe_dtype_t dt,
-                           void* out, cudaStream_t s, const void* shared) {
+                           void* out, cudaStream_t s, const void* shared,
+                           const void* shared2) {
   if (T == 0) return cudaSuccess;
   const int elt = dt == MOE_BF16 ? 2 : 4;
   const int row_vec = d * elt / 16;
   const int blocks = std::min(cdiv(T, 8), num_sms() * 8);
   const uint4* sh = static_cast<const uint4*>(shared);
+  const uint4* sh2 = static_cast<const uint4*>(shared2);
   if (dt == MOE_BF16)
     combine_launch<true>(static_cast<const uint4*>(y), dst_pos, row_map, topk_w, T, row_vec, N,
-                         top_k, sh, static_cast<uint4*>(out), blocks, s);
+                         top_k, sh, sh2, static_cast<uint4*>(out), blocks, s);
   else
     combine_launch<false>(static_cast<const uint4*>(y), dst_pos, row_map, topk_w, T, row_vec, N,
-                          top_k, sh, static_cast<uint4*>(out), blocks, s);
+                          top_k, sh, sh2, static_cast<uint4*>(out), blocks, s);
   return cudaGetLastError();
 }
 
@@ -558,7 +615,8 @@ template <int EPL>
 __global__ void __launch_bounds__(256) router_backward_kernel(
     const float* __restrict__ logits, const int32_t* __restrict__ topk_idx,
     const float* __restrict__ g_w, int T, int E, int k, int sigmoid, int renorm, float scale,
-    float* __restrict__ dz32, __nv_bfloat16* __restrict__ dz16) {
+    float* __restrict__ dz32, __nv_bfloat16* __restrict__ dz16,
+    const int32_t* __restrict__ lb_counts, float lb_scale) {
   pdl_wait();
   pdl_trigger();
   const int lane = threadIdx.x & 31;
@@ -599,6 +657,8 @@ __global__ void __launch_bounds__(256) router_backward_kernel(
       if (static_cast<unsigned>(e) < static_cast<unsigned>(E)) {
         my_e = e;
         my_g = g_w[static_cast<size_t>(t) * k + lane];
+        // [HP] _compute_load_balance_loss: coef * E * f_e / T, f_e = c_e / (T k)
+        if (lb_counts) my_g += lb_scale * static_cast<float>(lb_counts[e]);
       }
     }
     float my_s = 0.f;
@@ -648,20 +708,47 @@ __global__ void __launch_bounds__(256) router_backward_kernel(
 cudaError_t launch_router_backward(const float* logits, const int32_t* topk_idx,
                                    const float* d_topk_w, int T, int E, int top_k, int sigmoid,
                                    int renorm, float scale, float* dz32, void* dz16,
-                                   cudaStream_t s) {
+                                   cudaStream_t s, const int32_t* lb_counts, float lb_scale) {
   if (T == 0) return cudaSuccess;
   const int blocks = std::min(cdiv(T, 8), num_sms() * 8);
   __nv_bfloat16* d16 = static_cast<__nv_bfloat16*>(dz16);
   if (E <= 32)
-    launch_k(router_backward_kernel<1>, dim3(blocks), dim3(256), 0, s, logits, topk_idx, d_topk_w, T, E, top_k, sigmoid, renorm, scale, dz32, d16);
+    launch_k(router_backward_kernel<1>, dim3(blocks), dim3(256), 0, s, logits, topk_idx, d_topk_w, T, E, top_k, sigmoid, renorm, scale, dz32, d16, lb_counts, lb_scale);
   else if (E <= 64)
-    launch_k(router_backward_kernel<2>, dim3(blocks), dim3(256), 0, s, logits, topk_idx, d_topk_w, T, E, top_k, sigmoid, renorm, scale, dz32, d16);
+    launch_k(router_backward_kernel<2>, dim3(blocks), dim3(256), 0, s, logits, topk_idx, d_topk_w, T, E, top_k, sigmoid, renorm, scale, dz32, d16, lb_counts, lb_scale);
   else if (E <= 128)
-    launch_k(router_backward_kernel<4>, dim3(blocks), dim3(256), 0, s, logits, topk_idx, d_topk_w, T, E, top_k, sigmoid, renorm, scale, dz32, d16);
+    launch_k(router_backward_kernel<4>, dim3(blocks), dim3(256), 0, s, logits, topk_idx, d_topk_w, T, E, top_k, sigmoid, renorm, scale, dz32, d16, lb_counts, lb_scale);
   else if (E <= 256)
-    launch_k(router_backward_kernel<8>, dim3(blocks), dim3(256), 0, s, logits, topk_idx, d_topk_w, T, E, top_k, sigmoid, renorm, scale, dz32, d16);
+    launch_k(router_backward_kernel<8>, dim3(blocks), dim3(256), 0, s, logits, topk_idx, d_topk_w, T, E, top_k, sigmoid, renorm, scale, dz32, d16, lb_counts, lb_scale);
   else
-    launch_k(router_backward_kernel<16>, dim3(blocks), dim3(256), 0, s, logits, topk_idx, d_topk_w, T, E, top_k, sigmoid, renorm, scale, dz32, d16);
+    launch_k(router_backward_kernel<16>, dim3(blocks), dim3(256), 0, s, logits, topk_idx, d_topk_w, T, E, top_k, sigmoid, renorm, scale, dz32, d16, lb_counts, lb_scale);
+  return cudaGetLastError();
+}
+
+// counts[e] += number of entries of idx [n] equal to e (entries outside
+// [0, E) skipped); counts cleared by the caller.
+__global__ void expert_hist_kernel(const int32_t* __restrict__ idx, long long n, int E,
+                                   int32_t* __restrict__ counts) {
+  pdl_wait();
+  pdl_trigger();
+  extern __shared__ int eh[];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) eh[e] = 0;
+  __syncthreads();
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int e = idx[i];
+    if (static_cast<unsigned>(e) < static_cast<unsigned>(E)) atomicAdd(&eh[e], 1);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x)
+    if (eh[e]) atomicAdd(&counts[e], eh[e]);
+}
+
+cudaError_t launch_expert_hist(const int32_t* idx, long long n, int E, int32_t* counts,
+                               cudaStream_t s) {
+  const int blocks = static_cast<int>(std::min<long long>(num_sms(), (n + 1023) / 1024));
+  if (blocks > 0)
+    launch_k(expert_hist_kernel, dim3(blocks), dim3(256), E * sizeof(int), s, idx, n, E, counts);
   return cudaGetLastError();
 }
 
@@ -720,7 +807,7 @@ __global__ void __launch_bounds__(256) combine_backward_kernel(
 #pragma unroll
       for (int j = 0; j < KMAX; ++j) {
         if (j >= k || pos[j] < 0) continue;
-        dy[static_cast<size_t>(pos[j]) * row_vec + c] = scale_vec(g, wt[j], BF16);
+        if (dy) dy[static_cast<size_t>(pos[j]) * row_vec + c] = scale_vec(g, wt[j], BF16);
         if (dw) dot[j] += dot_chunk(g, v[j], BF16);
       }
     }
@@ -883,14 +970,6 @@ cudaError_t launch_router_logits_simt(const void* x, const void* w_router, int T
   return cudaGetLastError();
 }
 
-// Order-preserving map of a float score to int32 (NaN must be mapped to -inf
-// first; -0 and +0 compare equal, as floats do).
-__device__ __forceinline__ int score_key(float f) {
-  f += 0.0f;
-  const int i = __float_as_int(f);
-  return i ^ ((i >> 31) & 0x7fffffff);
-}
-__device__ __forceinline__ float key_score(int k) { return __int_as_float(k ^ ((k >> 31) & 0x7fffffff)); }
 
 // One warp per token; block b owns tokens [b*tpb, (b+1)*tpb).  Lane l holds
 // experts l, l+32, ... (EPL of them); the logit is the sum of the nsplit
@@ -930,8 +1009,11 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
   int* ebins = sm_bins + (blk ? nbins : 0);
   float* wsum = reinterpret_cast<float*>(ebins + E);
   const bool tally_e = counts != nullptr || tokens_per_expert != nullptr || lb != nullptr;
-  if (blk)
+  if (blk) {
+    // the dispatch column scan's completion ticket sits after the table
+    if (blockIdx.x == 0 && threadIdx.x == 0) blk[static_cast<size_t>(nbins) * gridDim.x] = 0;
     for (int i = threadIdx.x; i < nbins; i += blockDim.x) dbins[i] = 0;
+  }
   if (tally_e)
     for (int i = threadIdx.x; i < E; i += blockDim.x) ebins[i] = 0;
   if (lb)

@@ -1,0 +1,583 @@
+// Fused tcgen05 router of libmoe: the gate contraction, the scores, the top-k
+// selection and the routing weights in one kernel ([HP]
+// TokenChoiceTopKRouter.forward: the gate in fp32, softmax or sigmoid,
+// topk, gather, optional renormalisation, route_scale, expert_bias).
+//
+// A tile of 128 tokens is computed by a cluster of C CTAs (C = 1, 2, 4 or 8,
+// chosen so that tiles x C come close to the SM count): CTA r of the cluster
+// accumulates the r-th K range of d into TMEM (tcgen05.mma, operands staged
+// by TMA).  The C partial logit tiles are reduced through distributed shared
+// memory, not HBM: CTA r owns token rows [r 128 / C, (r + 1) 128 / C) of the
+// tile, every CTA stores its partial rows into their owner's shared memory
+// (st.shared::cluster), and the owner adds the C partials in rank order (a
+// fixed order: the logits do not depend on timing or on the grid).  The C
+// threads of each owned token then split its E experts (thread j takes
+// experts j, j + C, ...), each keeps the top-k of its slice in registers,
+// and k rounds of a shuffle arg-max over the C threads merge the slices
+// (descending key, ties to the lower expert index); the first thread of the
+// token writes the indices and weights, and in the layer forward the
+// dispatch histogram of its token block.  The expert counts of the entry
+// point go through a per-CTA table that a second small kernel sums.  The
+// stage memory is sized so that two CTAs fit on an SM (for E <= 128): the
+// scores and top-k of one CTA overlap the loads of the other.
+//
+// Every mbarrier wait is bounded (2 s) and unwinds by setting
+// MOE_DEV_TIMEOUT; the control flow after the K loop is the same in every
+// CTA (no early exit), so the cluster and named barriers are always met.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <climits>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+namespace rtc {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int kThreads = 192;          // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+// Pipeline stages: 96 KB for E <= 128 (two CTAs per SM), 192 KB for the
+// 256-column accumulator (whose exchange buffer needs 133 KB).  After the K
+// loop the same memory (at least `region` bytes, see Args) holds the partial
+// logits of the cluster, the dispatch bins and the expert bins.
+template <int BN>
+struct Layout {
+  static constexpr int kStageBytes = BM * BK * 2 + BN * BK * 2;
+  static constexpr int kStages = BN <= 64 ? 4 : BN == 128 ? 3 : 4;
+  static constexpr int kStageRegion = kStages * kStageBytes;
+  static constexpr uint32_t kTmemCols = BN < 32 ? 32u : static_cast<uint32_t>(BN);
+  static constexpr int kNumBars = 2 * kStages + 1;
+  static constexpr int kTailBytes = kNumBars * 8 + 16;   // barriers, TMEM slot, abort flag
+};
+
+struct Args {
+  int T, d, E, k, renorm;
+  int C;                 // CTAs per tile (cluster size)
+  int kb_total;          // 64-wide K blocks of d
+  int kb_per_cta;        // K blocks of each CTA of a cluster
+  int pitch;             // fp32 pitch of a row of partial logits in shared memory
+  int region;            // bytes before the barriers: max(stages, exchange + bins)
+  RouterOptions opt;
+  float* logits_out;     // [T, E] or null
+  int32_t* topk_idx;     // [T, k]
+  float* topk_w;         // [T, k]
+  int32_t* counts_part;  // [grid, E] per-CTA expert histograms, or null
+  int clear_status;      // the kernel is its call's only status writer: clear it
+  float* tpe;            // tokens_per_expert [E] (+=) or null
+  float* lb;             // [2E] copies and weight sums per expert (+=) or null
+  int32_t* blk;          // dispatch histogram table [nbins, nblk] or null
+  int nbins, tb, nblk, R, L, S;
+  int* status;
+};
+
+__device__ __forceinline__ void st_cluster_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                              uint32_t d) {
+  asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b),
+               "r"(c), "r"(d)
+               : "memory");
+}
+__device__ __forceinline__ void bar_epi() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+template <int BN, int KMAX>
+__global__ void __launch_bounds__(kThreads, 1)
+    router_tc_kernel(const __grid_constant__ CUtensorMap tmX,
+                     const __grid_constant__ CUtensorMap tmW, const Args a) {
+  using Lay = Layout<BN>;
+  constexpr int STAGES = Lay::kStages;
+  constexpr int kABytes = BM * BK * 2;
+  constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + a.region);
+  uint64_t* empty = full + STAGES;
+  uint64_t* mma_done = empty + STAGES;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int C = a.C;
+  const int rank = static_cast<int>(cluster_ctarank());
+  const int tile = blockIdx.x / C;
+  const int own = BM / C;                       // token rows this CTA owns
+  const int kb0 = rank * a.kb_per_cta;
+  const int kb1 = min(a.kb_total, kb0 + a.kb_per_cta);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(empty + s, 1);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmX);
+    tma_prefetch_desc(&tmW);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, Lay::kTmemCols);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  pdl_wait();   // x may be written by the previous kernel
+  // When this kernel is its call's only writer of the status word, CTA 0
+  // clears it here (a wait can give up only 2 s after its CTA started).
+  if (a.clear_status && blockIdx.x == 0 && threadIdx.x == 0) *a.status = 0;
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  // ------------------------------------------------------------ K loop
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint64_t pol = l2_policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      for (int kb = kb0; kb < kb1; ++kb) {
+        if (!mbar_wait(empty + stage, phase ^ 1u, abort_flag, a.status)) break;
+        uint8_t* sa = smem + stage * Lay::kStageBytes;
+        mbar_arrive_expect_tx(full + stage, Lay::kStageBytes);
+        tma_load_2d(sa, &tmX, full + stage, kb * BK, tile * BM, pol);
+        tma_load_2d(sa + kABytes, &tmW, full + stage, kb * BK, 0, pol);
+        ++issued;
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      // drain: every issued load has landed before the stage memory is reused
+      int s = stage;
+      uint32_t ph = phase;
+      for (int i = 0; i < min(issued, STAGES); ++i) {
+        if (s == 0) {
+          s = STAGES - 1;
+          ph ^= 1u;
+        } else {
+          --s;
+        }
+        mbar_wait(full + s, ph, nullptr, a.status);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int kb = kb0; kb < kb1; ++kb) {
+        if (!mbar_wait(full + stage, phase, abort_flag, a.status)) break;
+        tc_fence_after();
+        const uint8_t* sa = smem + stage * Lay::kStageBytes;
+        const uint64_t ad = sw128_kmajor_desc(sa);
+        const uint64_t bd = sw128_kmajor_desc(sa + kABytes);
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk)
+          tc_mma_bf16(tmem_base, ad + 2u * kk, bd + 2u * kk, IDESC, (kb != kb0 || kk != 0) ? 1u : 0u);
+        tc_commit(empty + stage);
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      tc_commit(mma_done);
+      mbar_wait(mma_done, 0, nullptr, a.status);
+    }
+  } else {
+    if (lane == 0) mbar_wait(mma_done, 0, nullptr, a.status);
+    __syncwarp();
+    tc_fence_after();
+  }
+  __syncwarp();
+  pdl_trigger();
+  // #1: every CTA of the cluster is done with its MMAs and loads, so the
+  // stage memory may now receive the partial logits of the peers.
+  cluster_sync_all();
+
+  // ------------------------------------------------- partial-logit exchange
+  float* recv = reinterpret_cast<float*>(smem);   // [C][own][pitch]
+  const int pitch = a.pitch;
+  if (warp >= 2) {
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    const int o = row / own, lr = row - o * own;
+    const uint32_t dst =
+        cluster_map(recv, static_cast<uint32_t>(o)) +
+        static_cast<uint32_t>((rank * own + lr) * pitch) * 4u;
+    const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+    for (int c = 0; c * 32 < a.E; ++c) {
+      uint32_t v[32];
+      tmem_ld32(taddr + c * 32, v);
+      tmem_ld_wait();
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        st_cluster_v4(dst + static_cast<uint32_t>((c * 32 + 4 * j) * 4), v[4 * j], v[4 * j + 1],
+                      v[4 * j + 2], v[4 * j + 3]);
+    }
+    tc_fence_before();
+  }
+  __syncwarp();
+  // #2: the partials of every CTA are in their owners' shared memory
+  cluster_sync_all();
+
+  // --------------------------------------------------- scores and top-k
+  if (warp >= 2) {
+    const int i = threadIdx.x - 64;               // 0..127
+    const int E = a.E, k = a.k;
+    const RouterOptions& opt = a.opt;
+    const int tpt = C;                            // threads per owned token
+    const int it = i / tpt;                       // owned token
+    const int jsl = i - it * tpt;                 // expert slice: e = jsl + tpt m
+    const bool lead = jsl == 0;
+    int* dbins = reinterpret_cast<int*>(smem + align_up(static_cast<size_t>(BM) * pitch * 4, 16));
+    int* ebins = dbins + (a.blk ? a.nbins : 0);
+    float* wsum = reinterpret_cast<float*>(ebins + E);
+    for (int e = i; e < E; e += 128) {
+      ebins[e] = 0;
+      wsum[e] = 0.f;
+    }
+    bar_epi();
+    const int t_own0 = tile * BM + rank * own;
+    const int t = t_own0 + it;
+    const bool active = t < a.T;
+    const float* rp = recv + static_cast<size_t>(it) * pitch;
+    const size_t sstride = static_cast<size_t>(own) * pitch;
+    auto zval = [&](int e) {
+      float z = rp[e];
+      for (int s = 1; s < C; ++s) z += rp[s * sstride + e];   // ranks in order
+      return z;
+    };
+    // group reductions over the tpt threads of the token (aligned lanes)
+    auto gmax = [&](float v) {
+      for (int off = 1; off < tpt; off <<= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+      return v;
+    };
+    auto gsum = [&](float v) {
+      for (int off = 1; off < tpt; off <<= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+      return v;
+    };
+    const bool on_logits = opt.bias == nullptr && opt.scale > 0.f;
+    // softmax statistics where the keys or the weights need them
+    float mx = -INFINITY, den = 1.f;
+    const bool need_den = !opt.sigmoid && !(on_logits && a.renorm);
+    if (!on_logits || need_den) {
+      for (int e = jsl; e < E; e += tpt) {
+        float z = zval(e);
+        if (z != z) z = -INFINITY;
+        mx = fmaxf(mx, z);
+      }
+      mx = gmax(mx);
+      if (!opt.sigmoid) {
+        den = 0.f;
+        for (int e = jsl; e < E; e += tpt) {
+          float z = zval(e);
+          if (z != z) z = -INFINITY;
+          den += expf(z - mx);
+        }
+        den = gsum(den);
+      }
+    }
+    // the top-KMAX of this thread's slice (experts ascend within it, so an
+    // equal key never displaces an earlier expert)
+    int keyt[KMAX], idxt[KMAX];
+#pragma unroll
+    for (int q = 0; q < KMAX; ++q) {
+      keyt[q] = INT_MIN;
+      idxt[q] = -1;
+    }
+    for (int e = jsl; e < E; e += tpt) {
+      float z = zval(e);
+      if (a.logits_out && active) a.logits_out[static_cast<size_t>(t) * E + e] = z;
+      if (z != z) z = -INFINITY;
+      float kv = z;
+      if (!on_logits) {
+        const float ex = opt.sigmoid ? 1.0f / (1.0f + expf(-z)) : expf(z - mx);
+        kv = ex / den * opt.scale;
+        if (opt.bias) {
+          kv += opt.bias[e];
+          if (kv != kv) kv = -INFINITY;
+        }
+      }
+      const int key = score_key(kv);
+      if (key > keyt[KMAX - 1]) {
+#pragma unroll
+        for (int q = KMAX - 1; q > 0; --q) {
+          const bool shift = keyt[q - 1] < key;
+          const bool place = !shift && keyt[q] < key;
+          const int nk = shift ? keyt[q - 1] : (place ? key : keyt[q]);
+          const int ni = shift ? idxt[q - 1] : (place ? e : idxt[q]);
+          keyt[q] = nk;
+          idxt[q] = ni;
+        }
+        if (keyt[0] < key) {
+          keyt[0] = key;
+          idxt[0] = e;
+        }
+      }
+    }
+    // merge the slices: k rounds of an arg-max over the token's threads on
+    // (key descending, expert ascending); the winner pops its head
+    int sel[KMAX];
+#pragma unroll
+    for (int r = 0; r < KMAX; ++r) {
+      sel[r] = -1;
+      if (r < k) {
+        unsigned long long v =
+            (static_cast<unsigned long long>(static_cast<uint32_t>(keyt[0]) ^ 0x80000000u) << 32) |
+            static_cast<unsigned long long>(0xffffffffu - static_cast<uint32_t>(idxt[0]));
+        for (int off = 1; off < tpt; off <<= 1) {
+          const unsigned long long o = __shfl_xor_sync(0xffffffffu, v, off);
+          v = o > v ? o : v;
+        }
+        const int we = static_cast<int>(0xffffffffu - static_cast<uint32_t>(v & 0xffffffffu));
+        sel[r] = we;
+        if (idxt[0] == we) {
+#pragma unroll
+          for (int q = 0; q < KMAX - 1; ++q) {
+            keyt[q] = keyt[q + 1];
+            idxt[q] = idxt[q + 1];
+          }
+          keyt[KMAX - 1] = INT_MIN;
+          idxt[KMAX - 1] = -1;
+        }
+      }
+    }
+    // weights: the unbiased score of each winner, renormalised when asked,
+    // times the scale (softmax: exp(z - max) over the denominator)
+    if (lead && active) {
+      if (on_logits && !opt.sigmoid && a.renorm) {
+        mx = zval(sel[0]);          // the largest logit
+        if (mx != mx) mx = -INFINITY;
+      }
+      float exs[KMAX];
+      float ssum = 0.f;
+#pragma unroll
+      for (int r = 0; r < KMAX; ++r) {
+        exs[r] = 0.f;
+        if (r < k) {
+          float z = zval(sel[r]);
+          if (z != z) z = -INFINITY;
+          exs[r] = opt.sigmoid ? 1.0f / (1.0f + expf(-z)) : expf(z - mx);
+          ssum += exs[r];
+        }
+      }
+      const float dv = a.renorm ? ssum : den;
+#pragma unroll
+      for (int r = 0; r < KMAX; ++r) {
+        if (r < k) {
+          const float wv = exs[r] / dv * opt.scale;
+          const size_t o = static_cast<size_t>(t) * k + r;
+          a.topk_idx[o] = sel[r];
+          a.topk_w[o] = wv;
+          atomicAdd(&ebins[sel[r]], 1);
+          if (a.lb) atomicAdd(&wsum[sel[r]], wv);
+        }
+      }
+    }
+    // dispatch histogram of every token block of tb rows this CTA owns
+    if (a.blk) {
+      if (blockIdx.x == 0 && i == 0)   // the dispatch column scan's ticket
+        a.blk[static_cast<size_t>(a.nbins) * a.nblk] = 0;
+      const int nb = own / a.tb;
+      for (int jb = 0; jb < nb; ++jb) {
+        const int b = t_own0 / a.tb + jb;
+        for (int x = i; x < a.nbins; x += 128) dbins[x] = 0;
+        bar_epi();
+        if (lead && active && it / a.tb == jb) {
+#pragma unroll
+          for (int r = 0; r < KMAX; ++r)
+            if (r < k) atomicAdd(&dbins[dispatch_key(sel[r], t, a.R, a.L, a.S)], 1);
+        }
+        bar_epi();
+        if (b < a.nblk)
+          for (int x = i; x < a.nbins; x += 128)
+            a.blk[static_cast<size_t>(x) * a.nblk + b] = dbins[x];
+        bar_epi();
+      }
+    }
+    bar_epi();
+    for (int e = i; e < E; e += 128) {
+      const int c = ebins[e];
+      if (a.counts_part) a.counts_part[static_cast<size_t>(blockIdx.x) * E + e] = c;
+      if (c) {
+        if (a.tpe) atomicAdd(&a.tpe[e], static_cast<float>(c));
+        if (a.lb) {
+          atomicAdd(&a.lb[e], static_cast<float>(c));
+          atomicAdd(&a.lb[E + e], wsum[e]);
+        }
+      }
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, Lay::kTmemCols);
+  }
+}
+
+// counts[e] = sum over the CTAs of the fused router of their histograms
+// (plain stores: counts needs no clearing).
+__global__ void router_counts_kernel(const int32_t* __restrict__ part, int G, int E,
+                                     int32_t* __restrict__ counts) {
+  pdl_wait();
+  pdl_trigger();
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < E; e += gridDim.x * blockDim.x) {
+    int c = 0;
+    for (int g = 0; g < G; ++g) c += part[static_cast<size_t>(g) * E + e];
+    counts[e] = c;
+  }
+}
+
+template <int BN, int KMAX>
+cudaError_t launch_bn(const CUtensorMap& tx, const CUtensorMap& tw, const Args& a, int grid,
+                      size_t smem, cudaStream_t s) {
+  static int configured[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !configured[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(router_tc_kernel<BN, KMAX>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+    if (e != cudaSuccess) return e;
+    configured[dev] = 1;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = a.C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, router_tc_kernel<BN, KMAX>, tx, tw, a);
+}
+
+template <int BN>
+cudaError_t launch_k_of(const CUtensorMap& tx, const CUtensorMap& tw, const Args& a, int grid,
+                        size_t smem, cudaStream_t s) {
+  if (a.k <= 4) return launch_bn<BN, 4>(tx, tw, a, grid, smem, s);
+  if (a.k <= 8) return launch_bn<BN, 8>(tx, tw, a, grid, smem, s);
+  return launch_bn<BN, 16>(tx, tw, a, grid, smem, s);
+}
+
+}  // namespace rtc
+
+RouterFusedPlan router_fused_plan(int T, int d, int E, const DispatchPlan* plan) {
+  // (the plan only adds its bins to the shared memory; C does not depend on it)
+  RouterFusedPlan p{};
+  p.bn = E <= 32 ? 32 : E <= 64 ? 64 : E <= 128 ? 128 : 256;
+  p.tiles = std::max(1, cdiv(T, rtc::BM));
+  p.kb_total = std::max(1, cdiv(d, rtc::BK));
+  p.pitch = (E + 31) / 32 * 32 + 4;
+  // shared memory: the stages, or after the K loop the partial logits of the
+  // cluster, the dispatch bins and the expert bins, whichever is larger
+  int stages = 0, tail = 0;
+  switch (p.bn) {
+    case 32: stages = rtc::Layout<32>::kStageRegion; tail = rtc::Layout<32>::kTailBytes; break;
+    case 64: stages = rtc::Layout<64>::kStageRegion; tail = rtc::Layout<64>::kTailBytes; break;
+    case 128: stages = rtc::Layout<128>::kStageRegion; tail = rtc::Layout<128>::kTailBytes; break;
+    default: stages = rtc::Layout<256>::kStageRegion; tail = rtc::Layout<256>::kTailBytes; break;
+  }
+  const size_t exch = align_up(static_cast<size_t>(rtc::BM) * p.pitch * 4, 16) +
+                      (plan ? static_cast<size_t>(plan->nbins) * 4 : 0) + 8 * static_cast<size_t>(E);
+  p.region = static_cast<int>(align_up(std::max<size_t>(stages, exch), 1024));
+  p.smem = p.region + tail + 1024;   // + slack for the 1 KB alignment
+  // two CTAs per SM when they fit (228 KB per SM, 1 KB reserved per CTA)
+  const int per_sm = p.smem + 1024 <= 114 * 1024 ? 2 : 1;
+  // clusters of C CTAs per tile: tiles x C close to what the SMs hold at
+  // once and every CTA with at least one K block.  C depends on the sizes
+  // only, so the logits (summed over the C partials in rank order) are the
+  // same with and without the EP layout; the layer's dispatch plan is made
+  // with blocks of at most 128 / C tokens (layer_dispatch_plan).
+  int C = 1;
+  while (C < 8 && p.tiles * C * 2 <= per_sm * kRouterTargetTiles && 2 * C <= p.kb_total) C *= 2;
+  while (C > 1 && (C - 1) * cdiv(p.kb_total, C) >= p.kb_total) C /= 2;
+  p.C = C;
+  p.kb_per_cta = cdiv(p.kb_total, C);
+  p.grid = p.tiles * C;
+  p.ok = p.smem <= 227 * 1024 && (!plan || rtc::BM / C >= plan->tb);
+  return p;
+}
+
+cudaError_t launch_router_fused(const void* x, const void* w_router, int T, int d, int E,
+                                int top_k, int renorm, const RouterOptions& o, float* logits_out,
+                                int32_t* topk_idx, float* topk_w, int32_t* counts,
+                                int32_t* counts_part, float* tokens_per_expert, float* lb,
+                                const DispatchPlan* plan, int32_t* blk, int* status,
+                                bool clear_status, cudaStream_t s) {
+  const RouterFusedPlan p = router_fused_plan(T, d, E, plan);
+  if (!p.ok) return cudaErrorInvalidValue;
+  CUtensorMap tx, tw;
+  if (!tc::make_tmap(&tx, x, d, T, rtc::BM)) return cudaErrorInvalidValue;
+  if (!tc::make_tmap(&tw, w_router, d, E, p.bn)) return cudaErrorInvalidValue;
+  rtc::Args a{};
+  a.T = T;
+  a.d = d;
+  a.E = E;
+  a.k = top_k;
+  a.renorm = renorm;
+  a.C = p.C;
+  a.kb_total = p.kb_total;
+  a.kb_per_cta = p.kb_per_cta;
+  a.pitch = p.pitch;
+  a.region = p.region;
+  a.opt = o;
+  a.logits_out = logits_out;
+  a.topk_idx = topk_idx;
+  a.topk_w = topk_w;
+  a.counts_part = counts ? counts_part : nullptr;
+  a.clear_status = clear_status ? 1 : 0;
+  a.tpe = tokens_per_expert;
+  a.lb = lb;
+  a.blk = plan ? blk : nullptr;
+  if (plan) {
+    a.nbins = plan->nbins;
+    a.tb = plan->tb;
+    a.nblk = plan->nblk;
+    a.R = plan->R;
+    a.L = plan->L;
+    a.S = plan->S;
+  } else {
+    a.nbins = 0;
+    a.tb = 1;
+    a.nblk = 0;
+    a.R = 1;
+    a.L = E;
+    a.S = T;
+  }
+  a.status = status;
+  cudaError_t e;
+  switch (p.bn) {
+    case 32: e = rtc::launch_k_of<32>(tx, tw, a, p.grid, p.smem, s); break;
+    case 64: e = rtc::launch_k_of<64>(tx, tw, a, p.grid, p.smem, s); break;
+    case 128: e = rtc::launch_k_of<128>(tx, tw, a, p.grid, p.smem, s); break;
+    default: e = rtc::launch_k_of<256>(tx, tw, a, p.grid, p.smem, s); break;
+  }
+  if (e == cudaSuccess && counts) {
+    launch_k(rtc::router_counts_kernel, dim3(cdiv(E, 256)), dim3(256), 0, s, counts_part, p.grid,
+             E, counts);
+    e = cudaGetLastError();
+  }
+  return e;
+}
+
+}  // namespace moe
+
+namespace moe {
+
+DispatchPlan layer_dispatch_plan(int T, int d, int E, int top_k, int R, moe_dtype_t dt) {
+  int max_tb = 128;
+  if (dt == MOE_BF16 && E <= 256 && T > 0) max_tb = rtc::BM / router_fused_plan(T, d, E, nullptr).C;
+  return make_dispatch_plan(T, E, top_k, R, max_tb);
+}
+
+}  // namespace moe

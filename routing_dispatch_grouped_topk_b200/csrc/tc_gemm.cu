@@ -416,55 +416,6 @@ struct DownPolicy : GroupedSched<256, 1, 256> {
   static __device__ void finish(const Args&, int*) {}
 };
 
-// CTA-pair versions: an m-tile is 256 rows of one expert; CTA rank r of the
-// pair owns rows [256 mt + 128 r, +128) (its A operand and its accumulator
-// lanes) and loads half of the B tile.  GEMM1: rank 0 loads the w1 rows and
-// rank 1 the w3 rows of the same 128 hidden units, so accumulator columns
-// 0..127 are G and 128..255 are U in both CTAs.  GEMM2: rank r loads w2 rows
-// [n0 + 128 r, +128).  Epilogues are the single-CTA ones.
-__device__ __forceinline__ void pair_rows(int seg0, int cnt, int mt, int rank, TileInfo& t) {
-  const int r0 = mt * 256 + rank * 128;
-  t.a_row = seg0 + r0;
-  t.m_valid = max(0, min(BM, cnt - r0));
-  t.swap_np = 0;
-}
-
-struct UpPairPolicy : GroupedSched<256, 2, 128, 256> {
-  static __device__ TileInfo tile_info(const Args& a, const int* sched, int tile, int rank) {
-    int e, nt, mt, cnt, seg0;
-    locate(a, sched, tile, e, nt, mt, cnt, seg0);
-    TileInfo t;
-    pair_rows(seg0, cnt, mt, rank, t);
-    t.n0 = nt * 128;
-    t.b_row = e * a.n_out + t.n0;
-    t.kb0 = 0;
-    t.kb1 = cdiv(a.K, BK);
-    return t;
-  }
-  static __device__ void epilogue(const Args& a, int* s, const TileInfo& ti, uint32_t taddr,
-                                  int row) {
-    UpPolicy::epilogue(a, s, ti, taddr, row);
-  }
-};
-
-struct DownPairPolicy : GroupedSched<256, 1, 256, 256> {
-  static __device__ TileInfo tile_info(const Args& a, const int* sched, int tile, int rank) {
-    int e, nt, mt, cnt, seg0;
-    locate(a, sched, tile, e, nt, mt, cnt, seg0);
-    TileInfo t;
-    pair_rows(seg0, cnt, mt, rank, t);
-    t.n0 = nt * 256;
-    t.b_row = e * a.n_out + t.n0 + rank * 128;
-    t.kb0 = 0;
-    t.kb1 = cdiv(a.K, BK);
-    return t;
-  }
-  static __device__ void epilogue(const Args& a, int* s, const TileInfo& ti, uint32_t taddr,
-                                  int row) {
-    DownPolicy::epilogue(a, s, ti, taddr, row);
-  }
-};
-
 // ------------------------------------------------------- backward policies
 // The backward of the grouped SwiGLU (the derivative of the forward above,
 // one expert segment at a time; G = S w1^T, U = S w3^T, A = silu(G) * U,
@@ -770,6 +721,165 @@ struct DownStagedPolicy : DownPolicy {
       }
       __syncwarp();
     }
+  }
+};
+
+// ------------------------------------------- hybrid CTA-pair tile schedule
+// The forward GEMMs on CTA pairs (cta_group::2).  Every expert segment is
+// covered by 256-row pair tiles: CTA rank r owns rows [256 mt + 128 r, +128)
+// (its A operand and its accumulator lanes) and loads half of the B tile,
+// so a pair moves 64 KB per K block for the work that two single-CTA
+// 128 x 256 tiles do with 96 KB (the kernels are bound by this L2 -> shared
+// memory traffic).  The last m-tile of a segment, when it holds at most 128
+// rows, is a swap-AB pair tile instead: the weights are the M = 256 operand
+// (128 weight rows per SM) and the tile's tokens the N operand (the rows
+// rounded up to 32; each SM loads its N/2 token rows in 16-row boxes), so a
+// short tail costs in proportion to its rows instead of a full tile.
+//   GEMM1 normal tile: rank 0 loads w1 rows [e h + n0, +128), rank 1 the w3
+//     rows of the same hidden units; accumulator columns 0..127 hold G and
+//     128..255 hold U in both CTAs.
+//   GEMM1 swap tile: rank r loads w1 rows [e h + n0 + 64 r, +64) and the w3
+//     rows of the same units (two 64-row boxes): lanes 0..63 hold G and
+//     lanes 64..127 hold U of those 64 hidden units, one column per token.
+//   GEMM2: rank r loads w2 rows [e d + n0 + 128 r, +128), as the B half of a
+//     normal tile or as the A operand of a swap tile.
+constexpr int kPairSwapMaxRows = 128;
+constexpr int kTokBoxRows = 16;          // token rows per TMA box of a swap tile
+constexpr int kXchgPitch = 129;          // fp32 pitch of the swap tile's U exchange
+
+template <int NCOLS, int NUM_B_, bool UP_>
+struct HybridPolicy : GroupedSched<256, NUM_B_, NCOLS, 256> {
+  using Base = GroupedSched<256, NUM_B_, NCOLS, 256>;
+  static constexpr bool UP = UP_;
+  static __device__ TileInfo tile_info(const Args& a, const int* sched, int tile, int rank) {
+    int e, nt, mt, cnt, seg0;
+    Base::locate(a, sched, tile, e, nt, mt, cnt, seg0);
+    TileInfo t;
+    const int rows = cnt - mt * 256;        // rows from this m-tile to the segment's end
+    t.n0 = nt * NCOLS;
+    t.kb0 = 0;
+    t.kb1 = cdiv(a.K, BK);
+    t.m0 = 0;
+    if (rows <= kPairSwapMaxRows) {
+      t.a_row = seg0 + mt * 256;            // the tile's first token
+      t.m_valid = rows;                     // its tokens
+      t.swap_np = (rows + 31) & ~31;        // MMA N of the pair
+      t.b_row = UP ? e * a.n_out + t.n0 + 64 * rank : e * a.n_out + t.n0 + 128 * rank;
+    } else {
+      const int r0 = mt * 256 + rank * 128;
+      t.a_row = seg0 + r0;
+      t.m_valid = max(0, min(BM, cnt - r0));
+      t.swap_np = 0;
+      t.b_row = UP ? e * a.n_out + t.n0 : e * a.n_out + t.n0 + 128 * rank;
+    }
+    return t;
+  }
+};
+
+struct UpHybridPolicy : HybridPolicy<128, 2, true> {
+  // Swap tile: lanes 0..63 (quadrants 0, 1) hold G, lanes 64..127 (quadrants
+  // 2, 3) hold U of hidden units n0 + 64 rank + (lane mod 64), one column per
+  // token.  The U warps pass U through shared memory (fp32, 64 units x N
+  // tokens, odd pitch: conflict-free); the G warps then write H = silu(G) U
+  // (and, in the training forward, G and U) for 32 units per warp and
+  // instruction: 64 contiguous bytes of one token row.  `half` splits the
+  // tokens in chunks of 16 between the two warps of a quadrant.  The hand-off
+  // uses two mbarriers with bounded waits (xfull: the 4 U warps arrive after
+  // writing; xempty: the 4 G warps arrive after reading); `nswap` counts the
+  // swap tiles this warp has handled.  Returns false if a wait gave up.
+  static __device__ bool epilogue_swap_pair(const Args& a, const TileInfo& ti, uint32_t taddr,
+                                            int q, int half, float* xchg, int rank,
+                                            uint64_t* xfull, uint64_t* xempty, int nswap,
+                                            volatile int* abort_flag) {
+    const int lane = threadIdx.x & 31;
+    const int ntok = ti.m_valid;
+    const int h = a.n_out;
+    const uint32_t par = static_cast<uint32_t>(nswap) & 1u;
+    int ok = 1;
+    if (q >= 2) {
+      if (lane == 0) ok = mbar_wait(xempty, par ^ 1u, abort_flag, a.status) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) return false;
+      float* dst = xchg + ((q - 2) * 32 + lane) * kXchgPitch;
+      for (int t0 = 16 * half; t0 < ntok; t0 += 32) {
+        uint32_t u[16];
+        tmem_ld16(taddr + t0, u);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) dst[t0 + i] = __uint_as_float(u[i]);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(xfull);
+      return true;
+    }
+    if (lane == 0) ok = mbar_wait(xfull, par, abort_flag, a.status) ? 1 : 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (!ok) return false;
+    const int ul = q * 32 + lane;
+    const int unit = ti.n0 + 64 * rank + ul;
+    const bool uvalid = unit < h;
+    const float* src = xchg + ul * kXchgPitch;
+    for (int t0 = 16 * half; t0 < ntok; t0 += 32) {
+      uint32_t g[16];
+      tmem_ld16(taddr + t0, g);
+      tmem_ld_wait();
+      if (!uvalid) continue;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int t = t0 + i;
+        if (t < ntok) {
+          const float gv = __uint_as_float(g[i]), uv = src[t];
+          const size_t r = static_cast<size_t>(ti.a_row + t);
+          a.out[r * h + unit] = __float2bfloat16_rn(silu_f(gv) * uv);
+          if (a.gu_out) {
+            a.gu_out[r * (2 * h) + unit] = __float2bfloat16_rn(gv);
+            a.gu_out[r * (2 * h) + h + unit] = __float2bfloat16_rn(uv);
+          }
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(xempty);
+    return true;
+  }
+  static __device__ void epilogue_staged(const Args& a, int* s, const TileInfo& ti,
+                                         uint32_t taddr, int row, uint8_t* stg, int c0, int c1) {
+    UpStagedPolicy::epilogue_staged(a, s, ti, taddr, row, stg, c0, c1);
+  }
+};
+
+struct DownHybridPolicy : HybridPolicy<256, 1, false> {
+  // Swap tile: lane = output feature n0 + 128 rank + row, one column per
+  // token; a warp writes 32 features (64 contiguous bytes) of one token row
+  // per instruction.  Tokens in chunks of 16, split between the two warps of
+  // a quadrant by `half`.
+  static __device__ bool epilogue_swap_pair(const Args& a, const TileInfo& ti, uint32_t taddr,
+                                            int q, int half, float*, int rank, uint64_t*,
+                                            uint64_t*, int, volatile int*) {
+    const int lane = threadIdx.x & 31;
+    const int f = ti.n0 + 128 * rank + q * 32 + lane;
+    const bool fvalid = f < a.n_out;
+    const int ntok = ti.m_valid;
+    for (int t0 = 16 * half; t0 < ntok; t0 += 32) {
+      uint32_t v[16];
+      tmem_ld16(taddr + t0, v);
+      tmem_ld_wait();
+      if (!fvalid) continue;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int t = t0 + i;
+        if (t < ntok) {
+          const size_t r = static_cast<size_t>(ti.a_row + t);
+          const float sc = a.row_scale ? a.row_scale[r] : 1.0f;
+          a.out[r * a.n_out + f] = __float2bfloat16_rn(__uint_as_float(v[i]) * sc);
+        }
+      }
+    }
+    return true;
+  }
+  static __device__ void epilogue_staged(const Args& a, int* s, const TileInfo& ti,
+                                         uint32_t taddr, int row, uint8_t* stg, int c0, int c1) {
+    DownStagedPolicy::epilogue_staged(a, s, ti, taddr, row, stg, c0, c1);
   }
 };
 
@@ -1366,33 +1476,47 @@ __global__ void __launch_bounds__(P::THREADS, 1)
 }
 
 // ---------------------------------------------------- the CTA-pair kernel
-// Two CTAs (a cluster of 2 on neighbouring SMs) share each 256 x 256 tile
-// through tcgen05.mma.cta_group::2: per K block each SM loads 16 KB of A
-// and 16 KB of B (instead of 16 + 32 KB for a 128-row tile alone), so the
-// pair does twice the MMA work of one CTA for 4/3 of its load traffic.
-// Rank 0 (leader) issues the MMAs and commits to the barriers of both CTAs;
-// both CTAs' TMA loads count on the leader's "full" barrier; both epilogues
-// arrive on the leader's "tmem empty" barrier.
+// Two CTAs (a cluster of 2 on neighbouring SMs) share each tile of the
+// hybrid schedule through tcgen05.mma.cta_group::2.  Rank 0 (leader) issues
+// the MMAs and commits to the barriers of both CTAs; both CTAs' TMA loads
+// count on the leader's "full" barrier; both CTAs' epilogue warps arrive on
+// the leader's "tmem empty" barrier.  Roles per CTA (320 threads): warp 0
+// TMA producer, warp 1 TMEM owner and (leader) MMA issuer, warps 2..9 the
+// epilogue (two per TMEM lane quadrant, each taking half of the columns).
+// Maps: tmA / tmB0 / tmB1 the normal tiles' operands (128-row boxes; tmB1
+// only for GEMM1), tmT the tokens in 16-row boxes, tmW0 / tmW1 the GEMM1
+// weights in 64-row boxes (swap tiles).
 template <class P>
 struct PairLayout {
   static constexpr int kBHalfBytes = 128 * BK * 2;                  // 16 KB
   static constexpr int kStageBytes = kATileBytes + kBHalfBytes;    // 32 KB per CTA
-  static constexpr int kStages = 6;
+  static constexpr int kStages = 5;
   static constexpr uint32_t kTmemCols = 512;                       // 2 x 256 columns
+  static constexpr int kEpiWarps = 8;
+  static constexpr int kThreads = 64 + 32 * kEpiWarps;
   static constexpr int kBarOff = kStages * kStageBytes;
-  static constexpr int kNumBars = 2 * kStages + 5;
+  static constexpr int kNumBars = 2 * kStages + 7;   // + tfull[2], tempty[2], mma_done, xfull, xempty
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSchedOff = (kMiscOff + 16 + 15) / 16 * 16;
-  static constexpr int kBytes = kSchedOff + P::SCHED_INTS * 4;
+  static constexpr int kEpiOff = (kSchedOff + P::SCHED_INTS * 4 + 15) / 16 * 16;
+  // the staged epilogue (2 KB per warp), then a swap tile's U exchange (its
+  // own memory: warps of the next tile may still stage while it is written)
+  static constexpr int kStgBytes = kEpiWarps * 2048;
+  static constexpr int kXchgOff = kEpiOff + kStgBytes;
+  static constexpr int kBytes = kXchgOff + 64 * kXchgPitch * 4;
   static constexpr int kLaunchBytes = kBytes + 1024;
   static_assert(kLaunchBytes <= 227 * 1024, "shared memory budget");
+  static_assert((64 * kXchgPitch * 4) % 16 == 0, "exchange buffer size");
 };
 
 template <class P>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(PairLayout<P>::kThreads, 1)
     tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB0,
-                        const __grid_constant__ CUtensorMap tmB1, const Args args) {
+                        const __grid_constant__ CUtensorMap tmB1,
+                        const __grid_constant__ CUtensorMap tmT,
+                        const __grid_constant__ CUtensorMap tmW0,
+                        const __grid_constant__ CUtensorMap tmW1, const Args args) {
   using L = PairLayout<P>;
   constexpr int STAGES = L::kStages;
   constexpr uint32_t IDESC = idesc_bf16_f32(256, 256);
@@ -1406,9 +1530,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* mma_done = tempty + 2;
+  uint64_t* xfull = mma_done + 1;
+  uint64_t* xempty = xfull + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
   int* sched = reinterpret_cast<int*>(smem + L::kSchedOff);
+  uint8_t* epi = smem + L::kEpiOff;
+  float* xchg = reinterpret_cast<float*>(smem + L::kXchgOff);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -1422,16 +1550,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull + a, 1);
-      mbar_init(tempty + a, 8);   // 4 epilogue warps in each CTA of the pair
+      mbar_init(tempty + a, 2 * L::kEpiWarps);   // every epilogue warp of both CTAs
     }
     mbar_init(mma_done, 1);
+    mbar_init(xfull, 4);    // the four U warps (quadrants 2, 3; both halves)
+    mbar_init(xempty, 4);   // the four G warps (quadrants 0, 1; both halves)
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB0);
-    if (P::NUM_B == 2) tma_prefetch_desc(&tmB1);
+    tma_prefetch_desc(&tmT);
+    if (P::UP) {
+      tma_prefetch_desc(&tmB1);
+      tma_prefetch_desc(&tmW0);
+      tma_prefetch_desc(&tmW1);
+    }
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, L::kTmemCols);
@@ -1459,16 +1594,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int tile = pair; tile < total && ok; tile += npairs) {
         const TileInfo ti = P::tile_info(args, sched, tile, rank);
+        const int half_n = ti.swap_np / 2;                    // token rows of this CTA
+        const int nbox = (half_n + kTokBoxRows - 1) / kTokBoxRows;
+        const uint32_t cta_bytes =
+            ti.swap_np ? kATileBytes + nbox * kTokBoxRows * BK * 2 : L::kStageBytes;
         for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
           if (!mbar_wait(empty + stage, phase ^ 1u, abort_flag, args.status)) {
             ok = false;
             break;
           }
           uint8_t* sa = tiles + stage * L::kStageBytes;
+          uint8_t* sb = sa + kATileBytes;
           const uint32_t bar = cluster_map(full + stage, 0);
-          if (leader) mbar_arrive_expect_tx(full + stage, 2 * L::kStageBytes);
-          tma_load_2d_pair(sa, &tmA, bar, kb * BK, ti.a_row, pol);
-          tma_load_2d_pair(sa + kATileBytes, tb, bar, kb * BK, ti.b_row, pol);
+          if (leader) mbar_arrive_expect_tx(full + stage, 2 * cta_bytes);
+          if (!ti.swap_np) {
+            tma_load_2d_pair(sa, &tmA, bar, kb * BK, ti.a_row, pol);
+            tma_load_2d_pair(sb, tb, bar, kb * BK, ti.b_row, pol);
+          } else {
+            // A region: this CTA's 128 weight rows; B region: its N/2 tokens
+            if (P::UP) {
+              tma_load_2d_pair(sa, &tmW0, bar, kb * BK, ti.b_row, pol);
+              tma_load_2d_pair(sa + kATileBytes / 2, &tmW1, bar, kb * BK, ti.b_row, pol);
+            } else {
+              tma_load_2d_pair(sa, &tmB0, bar, kb * BK, ti.b_row, pol);
+            }
+            for (int i = 0; i < nbox; ++i)
+              tma_load_2d_pair(sb + i * kTokBoxRows * BK * 2, &tmT, bar, kb * BK,
+                               ti.a_row + rank * half_n + i * kTokBoxRows, pol);
+          }
           ++issued;
           if (++stage == STAGES) {
             stage = 0;
@@ -1504,6 +1657,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * 256);
         const TileInfo ti = P::tile_info(args, sched, tile, 0);
+        const uint32_t idesc = ti.swap_np ? idesc_bf16_f32(256, ti.swap_np) : IDESC;
         for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
           if (!mbar_wait(full + stage, phase, abort_flag, args.status)) {
             ok = false;
@@ -1515,7 +1669,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t bd = sw128_kmajor_desc(sa + kATileBytes);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
-            tc_mma_bf16_pair(d_tmem, ad + 2u * kk, bd + 2u * kk, IDESC,
+            tc_mma_bf16_pair(d_tmem, ad + 2u * kk, bd + 2u * kk, idesc,
                              (kb != ti.kb0 || kk != 0) ? 1u : 0u);
           tc_commit_pair_mc(empty + stage, 0x3);
           if (++stage == STAGES) {
@@ -1531,12 +1685,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // -------------------------------------------------- epilogue warps (both CTAs)
+    // Warp w reads TMEM lanes 32 (w % 4) .. +32; the two warps of a quadrant
+    // (half 0: warps 2..5, half 1: warps 6..9) split the columns.
     const int q = warp & 3;
     const int row = q * 32 + lane;
+    const int half = (warp - 2) >> 2;
     uint32_t tempty_leader[2];
     tempty_leader[0] = cluster_map(tempty + 0, 0);
     tempty_leader[1] = cluster_map(tempty + 1, 0);
     int it = 0;
+    int nswap = 0;
     for (int tile = pair; tile < total; tile += npairs, ++it) {
       const int acc = it & 1;
       const uint32_t aph = (it >> 1) & 1;
@@ -1548,7 +1706,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const TileInfo ti = P::tile_info(args, sched, tile, rank);
       const uint32_t taddr =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * 256);
-      P::epilogue(args, sched, ti, taddr, row);
+      if (ti.swap_np) {
+        if (!P::epilogue_swap_pair(args, ti, taddr, q, half, xchg, rank, xfull, xempty, nswap,
+                                   abort_flag))
+          break;
+        ++nswap;
+      } else {
+        P::epilogue_staged(args, sched, ti, taddr, row, epi + (warp - 2) * 2048, 4 * half,
+                           4 * half + 4);
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tempty_leader[acc]);
@@ -1622,6 +1788,7 @@ cudaError_t launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMa
 // Launch of the CTA-pair kernel: clusters of 2 CTAs, an even grid.
 template <class P>
 cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
+                        const CUtensorMap& t, const CUtensorMap& w0, const CUtensorMap& w1,
                         const Args& args, int pairs, cudaStream_t s) {
   using L = PairLayout<P>;
   static int configured[64] = {0};
@@ -1636,7 +1803,7 @@ cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUten
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pairs, 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(L::kThreads, 1, 1);
   cfg.dynamicSmemBytes = L::kLaunchBytes;
   cfg.stream = s;
   cudaLaunchAttribute attr[2];
@@ -1648,7 +1815,7 @@ cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUten
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, tc_gemm_pair_kernel<P>, a, b0, b1, args);
+  return cudaLaunchKernelEx(&cfg, tc_gemm_pair_kernel<P>, a, b0, b1, t, w0, w1, args);
 }
 
 }  // namespace tc
@@ -1726,11 +1893,11 @@ static cudaError_t swiglu_tc_impl(const void* a_src, int a_rows, const int32_t* 
   if (!make_tmap(&t1, w1, d, static_cast<uint64_t>(E) * h, 128)) return cudaErrorInvalidValue;
   if (!make_tmap(&t3, w3, d, static_cast<uint64_t>(E) * h, 128)) return cudaErrorInvalidValue;
   if (!make_tmap(&th, H, h, N, BM)) return cudaErrorInvalidValue;
-  // The CTA-pair kernel (256-row tiles, 2/3 of the loads per SM) measured
-  // 5-10% slower than single-CTA 128-row tiles on B200 for segments of ~256
-  // average rows (its 256-row tiles pad to 1.5 tiles per expert) and ~2%
-  // faster at 1024 average rows (Zipf-skewed); it is used from 1024 up.
-  const bool pairs = !gather && N >= 1024 * E;
+  // The CTA-pair kernel (hybrid schedule: 256-row pair tiles, swap-AB pair
+  // tiles for segment tails of at most 128 rows) serves every layer whose
+  // segments average 64 rows or more; shorter segments (decode) stay on the
+  // single-CTA kernel, whose swap-AB tiles stream each weight tile once.
+  const bool pairs = !gather && N >= 64LL * E;
   if (!make_tmap(&t2, w2, h, static_cast<uint64_t>(E) * d, pairs ? 128 : 256))
     return cudaErrorInvalidValue;
   const int max_mt = cdiv(N, BM) + E;   // upper bound on m-tiles over all segments
@@ -1748,16 +1915,22 @@ static cudaError_t swiglu_tc_impl(const void* a_src, int a_rows, const int32_t* 
   a.gather_src = a_src;
   a.gu_out = static_cast<__nv_bfloat16*>(gu);
   if (pairs) {
-    const long long max_pt = cdiv(N, 256) + E;   // upper bound on 256-row pair tiles
+    CUtensorMap txs, t1h, t3h, ths;
+    if (!make_tmap(&txs, a_src, d, a_rows, kTokBoxRows)) return cudaErrorInvalidValue;
+    if (!make_tmap(&t1h, w1, d, static_cast<uint64_t>(E) * h, 64)) return cudaErrorInvalidValue;
+    if (!make_tmap(&t3h, w3, d, static_cast<uint64_t>(E) * h, 64)) return cudaErrorInvalidValue;
+    if (!make_tmap(&ths, H, h, N, kTokBoxRows)) return cudaErrorInvalidValue;
+    const long long max_pt = cdiv(N, 256) + E;   // upper bound on pair tiles per n-tile
     int np = static_cast<int>(std::min<long long>(num_sms() / 2, max_pt * cdiv(h, 128)));
-    cudaError_t e = launch_pair<UpPairPolicy>(tx, t1, t3, a, np, s);
+    cudaError_t e = launch_pair<UpHybridPolicy>(tx, t1, t3, txs, t1h, t3h, a, np, s);
     if (e != cudaSuccess) return e;
     a.K = h;
     a.n_out = d;
     a.out = static_cast<__nv_bfloat16*>(y);
+    a.gu_out = nullptr;
     a.row_scale = row_scale;
     np = static_cast<int>(std::min<long long>(num_sms() / 2, max_pt * cdiv(d, 256)));
-    return launch_pair<DownPairPolicy>(th, t2, t2, a, np, s);
+    return launch_pair<DownHybridPolicy>(th, t2, t2, ths, t2, t2, a, np, s);
   }
   int grid = static_cast<int>(std::min<long long>(num_sms(), 1LL * max_mt * cdiv(h, 128)));
   cudaError_t e = gather ? launch<UpGatherPolicy>(tx, t1, t3, a, grid, s)

@@ -183,9 +183,11 @@ def test_router_options_defaults(L):
     o = m.RouterOptions()
     o.route_scale = 7.0
     o.num_groups = 3
+    o.aux_loss_coef = 2.0
     L.moe_router_options_init(ctypes.byref(o))
     assert (o.score, o.renormalize, o.route_scale, o.expert_bias, o.num_groups, o.topk_groups,
-            o.tokens_per_expert, o.score_before_experts) == (0, 0, 1.0, None, 0, 0, None, 0)
+            o.tokens_per_expert, o.score_before_experts, o.aux_loss, o.aux_loss_coef) == \
+        (0, 0, 1.0, None, 0, 0, None, 0, None, 0.0)
 
 
 def test_shared_expert_workspace_and_checks(L):
@@ -227,13 +229,19 @@ def test_training_entry_points_check_their_arguments(L):
     # E not a multiple of 8
     assert L.moe_forward_train(p, p, None, p, p, p, 4, 64, 12, 2, 64, None, 1, p, p, big,
                                None) == 2
-    o = m.RouterOptions()
-    L.moe_router_options_init(ctypes.byref(o))
-    o.score_before_experts = 1
-    assert L.moe_forward_train(p, p, None, p, p, p, 4, 64, 8, 2, 64, ctypes.byref(o), 1, p, p,
-                               big, None) == 2
-    assert L.moe_backward(p, p, p, p, p, p, 4, 64, 8, 2, 64, ctypes.byref(o), 1, p, p, None, p,
-                          p, p, p, p, big, None) == 2
+    # a shared expert: h % 64 != 0 is unsupported, its weight gradients are
+    # required by the backward, the sizes grow by its state
+    assert L.moe_train_state_size_ex(T, d, E, k, h, 0) == L.moe_train_state_size(T, d, E, k, h)
+    assert L.moe_train_state_size_ex(T, d, E, k, h, 1024) >= \
+        L.moe_train_state_size(T, d, E, k, h) + T * (d + 3 * 1024) * 2
+    assert L.moe_backward_workspace_size_ex(T, d, E, k, h, 1024) >= \
+        L.moe_backward_workspace_size(T, d, E, k, h) + T * (d + 2 * 1024) * 2
+    bad = m.SharedExpert(256, 256, 256, 96)
+    assert L.moe_forward_train_ex(p, p, None, p, p, p, 4, 64, 8, 2, 64, None, ctypes.byref(bad), 1,
+                                  p, p, big, None) == 2
+    sh = m.SharedExpert(256, 256, 256, 64)
+    assert L.moe_backward_ex(p, p, p, p, p, p, 4, 64, 8, 2, 64, None, ctypes.byref(sh), 1, p, p,
+                             None, p, p, p, p, None, None, None, p, big, None) == 1
     # state / workspace too small
     assert L.moe_forward_train(p, p, None, p, p, p, 4, 64, 8, 2, 64, None, 1, p, p, 16,
                                None) == 4

@@ -316,6 +316,30 @@ def test_router_backward_matches_oracle(M, score, renorm, scale, T, E, k, d):
     close_wgrad(dx, rdx)
 
 
+@pytest.mark.parametrize("score,renorm", [("softmax", True), ("sigmoid", False)])
+def test_router_backward_load_balance_gradient(M, score, renorm):
+    """aux_loss_coef: the gradient of coef times the load-balance loss
+    ([HP] _compute_load_balance_loss) joins the routing weights' gradient;
+    against the oracle's router backward fed d_topk_w + coef * the oracle's
+    loss gradient (pinned by finite differences of the loss)."""
+    T, E, k, coef = 300, 16, 4, 0.05
+    L = W.make_logits(T, E, k, seed=11)
+    idx, w, _, _ = O.router_topk_general(k, logits=L, score=score, renormalize=renorm)
+    gw = torch.randn(T, k, generator=torch.Generator().manual_seed(3))
+    dl, _, _, ws = M.router_backward(torch.from_numpy(L).float().cuda(), i32(idx), gw.cuda(),
+                                     score=score, renormalize=renorm, aux_loss_coef=coef)
+    dl0, _, _, _ = M.router_backward(torch.from_numpy(L).float().cuda(), i32(idx), gw.cuda(),
+                                     score=score, renormalize=renorm)
+    torch.cuda.synchronize()
+    assert M.device_status(ws) == 0
+    g = gw.double().numpy() + coef * O.load_balance_loss_grad(idx, E)
+    rdz = O.router_backward(L.astype(np.float32), idx, g, score=score, renormalize=renorm)
+    err = np.abs(f64(dl) - rdz)
+    rowmax = np.abs(rdz).max(axis=1, keepdims=True)
+    assert np.all(err <= 2e-5 * (np.abs(rdz) + rowmax) + 1e-30), err.max()
+    assert not torch.equal(dl, dl0)
+
+
 def test_router_backward_without_gate_gradients(M):
     T, E, k = 50, 16, 2
     L = W.make_logits(T, E, k, seed=1)
@@ -410,7 +434,8 @@ def test_forward_train_and_backward_equal_the_staged_calls(M, cfg_index):
 
 
 @pytest.mark.parametrize("opts", [dict(), dict(score="sigmoid", route_scale=2.5),
-                                  dict(num_groups=4, topk_groups=2)])
+                                  dict(num_groups=4, topk_groups=2),
+                                  dict(aux_loss_coef=0.05)])
 def test_layer_backward_matches_oracle(M, opts):
     """Every gradient of the whole layer (x, w_router, w1, w3, w2, logits)
     on a small layer against the oracle's chain rule, with router options."""
@@ -437,6 +462,8 @@ def test_layer_backward_matches_oracle(M, opts):
     assert np.array_equal(gi.cpu().numpy(), ref["topk_idx"])
     close(out, ref["out"])
     rdy, rdtw = O.combine_backward(dout, ref["y"], ref["dst_pos"], ref["topk_w"])
+    # the load-balance loss's gradient joins the routing weights' gradient
+    rdtw = rdtw + opts.get("aux_loss_coef", 0.0) * O.load_balance_loss_grad(ref["topk_idx"], E)
     rdxp, rw1, rw3, rw2 = O.grouped_swiglu_backward(ref["x_perm"], ref["offsets"], w1, w3, w2,
                                                     rdy)
     rdz, rdwr, rdxr = O.router_backward(ref["logits"], ref["topk_idx"], rdtw,
@@ -465,7 +492,7 @@ def test_layer_backward_matches_oracle(M, opts):
     # a[t, j] = 2^-8 sum_i |dout_i| (|y_i| + 3 rms(y row)) (one bf16 rounding
     # of y and of the hidden activation before it), carried to the logits by
     # the absolute Jacobian: |err[t, e]| <= sum_j |d w_j / d z_e| a[t, j],
-    # plus fp32 slack.
+    # plus fp32 slack (and, for sigmoid scores, the fp32 error of s (1 - s)).
     ydst = ref["y"][ref["dst_pos"]]                                  # [T, k, d]
     yrms = np.sqrt(np.mean(ydst ** 2, axis=2, keepdims=True))
     a = 2.0 ** -8 * np.einsum("ti,tji->tj", np.abs(f64(dout)), np.abs(ydst) + 3 * yrms)
@@ -477,9 +504,103 @@ def test_layer_backward_matches_oracle(M, opts):
                                   renormalize=True, route_scale=ro["route_scale"])
         bound += np.abs(jac_j) * a[:, j:j + 1]
     bound += 1e-5 * np.abs(rdz).max(axis=1, keepdims=True)
+    if ro["score"] == "sigmoid":
+        # the kernel's s (1 - s) in fp32: relative error ~2^-23 / (1 - s),
+        # large where the sigmoid saturates
+        sg = O.sigmoid(ref["logits"])
+        bound += np.abs(rdz) * 2.0 ** -20 / np.maximum(1.0 - sg, 2.0 ** -30)
     wsel = np.asarray(ref["topk_w"]) / ro["route_scale"]
     live = np.all((wsel >= 1e-3) & (wsel <= 1 - 1e-3), axis=1)
     print(f"d logits checked element-wise on {live.sum()} of {T} tokens")
     assert live.sum() >= 30     # 93, 200 and 40 of the 200 tokens for the three options
     err = np.abs(gdz - rdz)[live]
     assert np.all(err <= bound[live]), (err / bound[live]).max()
+
+
+def _small_train_layer(seed, T=200, d=256, E=16, h=192, hs=None):
+    g = torch.Generator().manual_seed(seed)
+    bf = torch.bfloat16
+    x = torch.randn(T, d, generator=g).to(bf)
+    wr = (torch.randn(E, d, generator=g) * 0.5).to(bf)
+    w1 = (torch.randn(E, h, d, generator=g) / math.sqrt(d)).to(bf)
+    w3 = (torch.randn(E, h, d, generator=g) / math.sqrt(d)).to(bf)
+    w2 = (torch.randn(E, d, h, generator=g) / math.sqrt(h)).to(bf)
+    dout = torch.randn(T, d, generator=g).to(bf)
+    sh = None
+    if hs:
+        sh = ((torch.randn(hs, d, generator=g) / math.sqrt(d)).to(bf),
+              (torch.randn(hs, d, generator=g) / math.sqrt(d)).to(bf),
+              (torch.randn(d, hs, generator=g) / math.sqrt(hs)).to(bf))
+    return x, wr, w1, w3, w2, dout, sh
+
+
+def test_layer_backward_score_before_experts(M):
+    """score_before_experts ([HP] MoE.forward): the routed rows are scaled by
+    their weights before the experts and the combine is unweighted.  The
+    training forward equals moe_forward with the option bit for bit; every
+    gradient against the oracle's chain (unweighted combine -> experts ->
+    scaled dispatch -> router), itself pinned by finite differences of the
+    oracle layer."""
+    T, E, k = 200, 16, 4
+    x, wr, w1, w3, w2, dout, _ = _small_train_layer(7, T=T, E=E)
+    c = [t.cuda() for t in (x, wr, w1, w3, w2)]
+    out, state = M.forward_train(*c, k, renormalize=True, score_before_experts=True)
+    grads = M.backward(state, dout.cuda(), *c, want_d_logits=True)
+    torch.cuda.synchronize()
+    assert M.device_status(state["state"]) == 0 and M.device_status(grads["ws"]) == 0
+    assert torch.equal(out, M.forward(*c, k, True, score_before_experts=True))
+    ref = O.moe_forward(x, wr, w1, w3, w2, k, True, score_before_experts=True)
+    close(out, ref["out"])
+    rdy, _ = O.combine_backward(dout, ref["y"], ref["dst_pos"], None)
+    rdxp, rw1, rw3, rw2 = O.grouped_swiglu_backward(ref["x_perm"], ref["offsets"], w1, w3, w2,
+                                                    rdy)
+    rdxs, rdtw = O.scaled_dispatch_backward(rdxp, ref["dst_pos"], ref["topk_w"], x)
+    rdz, rdwr, rdxr = O.router_backward(ref["logits"], ref["topk_idx"], rdtw, renormalize=True,
+                                        x=x, w_router=wr)
+    close(grads["dx"], rdxs + rdxr)
+    for e in range(E):
+        if int(ref["counts"][e]) == 0:
+            continue
+        close_wgrad(grads["dw1"][e], rw1[e])
+        close_wgrad(grads["dw3"][e], rw3[e])
+        close_wgrad(grads["dw2"][e], rw2[e])
+    close_wgrad(grads["dw_router"], rdwr)
+    gdz = f64(grads["d_logits"])
+    assert np.linalg.norm(gdz - rdz) <= 1e-2 * np.linalg.norm(rdz)
+
+
+@pytest.mark.parametrize("hs", [128, 320])
+def test_layer_backward_shared_expert(M, hs):
+    """A shared expert ([HP] MoE.forward: out = routed + shared_expert(x)):
+    the training forward equals moe_forward_ex with it bit for bit; its
+    weight gradients and its share of dx against the oracle (a one-segment
+    SwiGLU backward over every token with the upstream dout, pinned with
+    the rest of the layer by finite differences of the oracle)."""
+    T, E, k = 200, 16, 4
+    x, wr, w1, w3, w2, dout, sh = _small_train_layer(8, T=T, E=E, hs=hs)
+    c = [t.cuda() for t in (x, wr, w1, w3, w2)]
+    shc = tuple(t.cuda() for t in sh)
+    out, state = M.forward_train(*c, k, renormalize=True, shared=shc)
+    grads = M.backward(state, dout.cuda(), *c, shared=shc)
+    torch.cuda.synchronize()
+    assert M.device_status(state["state"]) == 0 and M.device_status(grads["ws"]) == 0
+    assert torch.equal(out, M.forward(*c, k, True, shared=shc))
+    ref = O.moe_forward(x, wr, w1, w3, w2, k, True, shared=sh)
+    close(out, ref["out"])
+    rdy, rdtw = O.combine_backward(dout, ref["y"], ref["dst_pos"], ref["topk_w"])
+    rdxp, _, _, _ = O.grouped_swiglu_backward(ref["x_perm"], ref["offsets"], w1, w3, w2, rdy)
+    _, _, rdxr = O.router_backward(ref["logits"], ref["topk_idx"], rdtw, renormalize=True, x=x,
+                                   w_router=wr)
+    rdxsh, rs1, rs3, rs2 = O.grouped_swiglu_backward(x, np.array([0, T]), sh[0][None],
+                                                     sh[1][None], sh[2][None], dout)
+    # dx is the sum of three shares that are each rounded to bf16 before the
+    # sum (the routed copies', the router's and the shared expert's), so the
+    # bf16 bound applies to the magnitude of the shares, not of their sum
+    parts = [O.dispatch_backward(rdxp, ref["dst_pos"]), rdxr, rdxsh]
+    ref_dx = sum(parts)
+    err = np.abs(f64(grads["dx"]) - ref_dx)
+    assert np.all(err <= 3e-2 * (1 + sum(np.abs(p) for p in parts))), err.max()
+    assert np.linalg.norm(f64(grads["dx"]) - ref_dx) <= 1e-2 * np.linalg.norm(ref_dx)
+    close_wgrad(grads["dws1"], rs1[0])
+    close_wgrad(grads["dws3"], rs3[0])
+    close_wgrad(grads["dws2"], rs2[0])

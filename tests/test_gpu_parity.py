@@ -263,7 +263,7 @@ def test_ep_dispatch_then_regroup(M, T, d, E, k, R):
     assert M.device_status(ws2) == 0
 
 
-@pytest.mark.parametrize("G,R,L,rows_mean", [(8, 8, 16, 32), (1, 2, 2, 3), (3, 5, 7, 1),
+@pytest.mark.parametrize("G,R,L,rows_mean", [(8, 8, 16, 32), (1, 2, 2, 3), (3, 5, 7, 1), (8, 16, 64, 1),
                                              (2, 4, 3, 0)])
 def test_regroup_random_counts(M, G, R, L, rows_mean):
     crm = W.make_rank_counts(G, R, L, rows_mean * G * R * L, seed=G * R + L)
@@ -356,6 +356,31 @@ def test_grouped_swiglu_gather_full_size_sampled(M, cfg):
     c = W.config(cfg)
     swiglu_case(M, c.T, c.d, c.E, c.top_k, c.h, seed=c.seed, dtype=torch.bfloat16, sample=256,
                 gather=True)
+
+
+@pytest.mark.parametrize("counts,d,h", [
+    # 256-row pair tiles, tails of at most 128 rows (swap-AB pair tiles) and
+    # of more (a half-empty pair tile), empty experts, h and d that leave
+    # partial n-tiles
+    ([256, 128, 129, 1, 0, 31, 32, 33, 384, 511], 192, 320),
+    ([600, 200, 90], 320, 448),
+])
+@pytest.mark.parametrize("row_scale", [False, True])
+def test_grouped_swiglu_pair_tile_mix(M, counts, d, h, row_scale):
+    g = torch.Generator().manual_seed(sum(counts) + d)
+    E, N = len(counts), int(sum(counts))
+    bf = torch.bfloat16
+    xp = torch.randn(N, d, generator=g).to(bf)
+    w1 = (torch.randn(E, h, d, generator=g) / math.sqrt(d)).to(bf)
+    w3 = (torch.randn(E, h, d, generator=g) / math.sqrt(d)).to(bf)
+    w2 = (torch.randn(E, d, h, generator=g) / math.sqrt(h)).to(bf)
+    off = np.concatenate([[0], np.cumsum(counts)]).astype(np.int64)
+    rs = torch.rand(N, generator=g) if row_scale else None
+    gy, ws = M.grouped_swiglu(xp.cuda(), i32(off), w1.cuda(), w3.cuda(), w2.cuda(),
+                              None if rs is None else rs.cuda())
+    assert M.device_status(ws) == 0
+    ref = O.grouped_swiglu(xp, off, w1, w3, w2, None if rs is None else rs.numpy())
+    close(gy.cpu(), ref, bf)
 
 
 def test_grouped_swiglu_all_rows_one_expert(M):
