@@ -239,7 +239,7 @@ MOE_API moe_status_t moe_dispatch(const void* x, const int32_t* topk_idx, int T,
  * re-created context is followed; a call on a capturing stream uses the
  * address of the last lookup on that device, so make one call on the device
  * before any capture.  All calls share the array and it keeps the last call's
- * contents (the status word is cleared at the start of each call), so calls
+ * contents (each call rewrites the status word and the table), so calls
  * that overlap on the GPU -- on different streams, or from several host
  * threads -- race; serialise them.  The device status word is not exposed:
  * ids outside [0, E) show up as dst_pos = -1 and offsets[E] < T*k.

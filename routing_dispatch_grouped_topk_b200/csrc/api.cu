@@ -588,10 +588,10 @@ static moe_status_t dispatch_common(const void* x, const int32_t* topk_idx, int 
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int* status = static_cast<int*>(ws);
-  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), s);
-  if (e == cudaSuccess)
-    e = launch_dispatch(p, x, topk_idx, d, dt, counts, offsets, src_row, dst_pos,
-                        x ? x_perm : nullptr, static_cast<char*>(ws) + kStatusBytes, status, s);
+  // the column scan writes the whole status word: nothing to clear first
+  cudaError_t e = launch_dispatch(p, x, topk_idx, d, dt, counts, offsets, src_row, dst_pos,
+                                  x ? x_perm : nullptr, static_cast<char*>(ws) + kStatusBytes,
+                                  status, s, false, nullptr, /*own_status=*/true);
   return cuda_status(e, "moe_dispatch");
 }
 

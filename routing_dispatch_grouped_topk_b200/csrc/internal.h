@@ -119,11 +119,14 @@ cudaError_t launch_lb_loss(const float* lb, int E, int T, int top_k, float* loss
 // hist_done: the histogram table in `ws` was already written (by the router).
 // row_w [T*k] (or null): copy f = t*k + j of row t is multiplied by row_w[f]
 // (fp32 product, one rounding to dt) as it is written to x_perm.
+// own_status: the call's only kernels (the dispatch entry points): the
+// column scan writes the whole status word (MOE_DEV_BAD_EXPERT or 0), so no
+// clearing is needed before the call; otherwise nothing is written to it.
 cudaError_t launch_dispatch(const DispatchPlan& p, const void* x, const int32_t* topk_idx,
                             int d, moe_dtype_t dt, int32_t* counts, int32_t* offsets,
                             int32_t* src_row, int32_t* dst_pos, void* x_perm, void* ws,
                             int* status, cudaStream_t s, bool hist_done = false,
-                            const float* row_w = nullptr);
+                            const float* row_w = nullptr, bool own_status = false);
 
 // ---- regroup ----------------------------------------------------------------
 // One kernel (the segment tables are rebuilt in every block's shared

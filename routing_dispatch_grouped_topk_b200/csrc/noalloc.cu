@@ -79,11 +79,11 @@ extern "C" moe_status_t moe_dispatch_noalloc(const void* x, const int32_t* topk_
     return MOE_ERR_CUDA;
   }
   int* status = static_cast<int*>(base);
-  e = cudaMemsetAsync(status, 0, sizeof(int), s);   // the array keeps the last call's bytes
-  if (e == cudaSuccess)
-    e = launch_dispatch(p, x, topk_idx, d, dt, counts, offsets, src_row, dst_pos,
-                        x ? x_perm : nullptr, static_cast<char*>(base) + kNoAllocStatusBytes,
-                        status, s);
+  // the array keeps the last call's bytes: the histogram kernel rewrites the
+  // whole table and the column scan the whole status word
+  e = launch_dispatch(p, x, topk_idx, d, dt, counts, offsets, src_row, dst_pos,
+                      x ? x_perm : nullptr, static_cast<char*>(base) + kNoAllocStatusBytes,
+                      status, s, false, nullptr, /*own_status=*/true);
   if (e != cudaSuccess) {
     set_last_error("moe_dispatch_noalloc: %s", cudaGetErrorString(e));
     return MOE_ERR_CUDA;

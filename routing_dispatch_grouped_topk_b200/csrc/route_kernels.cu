@@ -17,15 +17,21 @@ namespace moe {
 
 // K1: histogram of the keys of each block of `tb` tokens, stored bin-major
 // (blk[bin * nblk + block]) so that K2 scans contiguous columns.
+// Every block also records in flags[block] (after the table and the column
+// scan's ticket) whether it met an expert id outside [0, E); the column
+// scan's last block turns the flags into the status word, so the dispatch
+// entry points need no cleared status word before them.
 __global__ void dispatch_hist_kernel(const int32_t* __restrict__ idx, int T, int k, int E, int R,
-                                     int L, int S, int tb, int nbins, int32_t* __restrict__ blk,
-                                     int* status) {
+                                     int L, int S, int tb, int nbins, int32_t* __restrict__ blk) {
   pdl_wait();
   pdl_trigger();
   extern __shared__ int hist[];
+  __shared__ int bad;
+  const int nblk = gridDim.x;
+  int32_t* ticket = blk + static_cast<size_t>(nbins) * nblk;
   // the column scan's completion ticket sits after the table
-  if (blockIdx.x == 0 && threadIdx.x == 0)
-    blk[static_cast<size_t>(nbins) * gridDim.x] = 0;
+  if (blockIdx.x == 0 && threadIdx.x == 0) *ticket = 0;
+  if (threadIdx.x == 0) bad = 0;
   for (int i = threadIdx.x; i < nbins; i += blockDim.x) hist[i] = 0;
   __syncthreads();
   const int t0 = blockIdx.x * tb;
@@ -34,15 +40,15 @@ __global__ void dispatch_hist_kernel(const int32_t* __restrict__ idx, int T, int
   for (long long f = f0 + threadIdx.x; f < f1; f += blockDim.x) {
     const int e = idx[f];
     if (static_cast<unsigned>(e) >= static_cast<unsigned>(E)) {
-      set_status(status, MOE_DEV_BAD_EXPERT);
+      bad = 1;
       continue;
     }
     atomicAdd(&hist[dispatch_key(e, static_cast<int>(f / k), R, L, S)], 1);
   }
   __syncthreads();
-  const int nblk = gridDim.x;
   for (int i = threadIdx.x; i < nbins; i += blockDim.x)
     blk[static_cast<size_t>(i) * nblk + blockIdx.x] = hist[i];
+  if (threadIdx.x == 0) ticket[1 + blockIdx.x] = bad;
 }
 
 // Block-wide exclusive scan of `n` ints held in shared memory `a` (in place);
@@ -126,7 +132,8 @@ __device__ int block_scan_value(int v, int* warp_sums, int* total) {
 __global__ void dispatch_colscan_kernel(int32_t* __restrict__ blk, int nblk, int nbins,
                                         int32_t* __restrict__ counts,
                                         int32_t* __restrict__ offsets,
-                                        int32_t* __restrict__ src_row, long long n_slots) {
+                                        int32_t* __restrict__ src_row, long long n_slots,
+                                        int* status_out) {
   pdl_wait();
   pdl_trigger();
   extern __shared__ int osm[];      // nbins (last block only)
@@ -161,6 +168,14 @@ __global__ void dispatch_colscan_kernel(int32_t* __restrict__ blk, int nblk, int
   for (int i = threadIdx.x; i < nbins; i += blockDim.x) offsets[i] = osm[i];
   if (threadIdx.x == 0) offsets[nbins] = total;
   for (long long sl = total + threadIdx.x; sl < n_slots; sl += blockDim.x) src_row[sl] = -1;
+  // the entry point's status word, from the histogram blocks' flags
+  if (status_out) {
+    const int32_t* flags = blk + static_cast<size_t>(nbins) * nblk + 1;
+    int any = 0;
+    for (int b = threadIdx.x; b < nblk; b += blockDim.x) any |= __ldcg(flags + b);
+    any = __syncthreads_or(any);
+    if (threadIdx.x == 0) *status_out = any ? MOE_DEV_BAD_EXPERT : 0;
+  }
 }
 
 // Eight bf16 or four fp32 values times w (fp32 product, rounded once).
@@ -287,26 +302,32 @@ DispatchPlan make_dispatch_plan(int T, int E, int top_k, int R, int max_tb) {
 }
 
 size_t dispatch_ws_bytes(const DispatchPlan& p) {
-  // the histogram table [nbins, nblk], then the column scan's ticket
-  return align_up((static_cast<size_t>(p.nblk) * p.nbins + 1) * sizeof(int32_t), 256);
+  // the histogram table [nbins, nblk], the column scan's ticket, then one
+  // bad-id flag per block
+  return align_up((static_cast<size_t>(p.nblk) * p.nbins + 1 + p.nblk) * sizeof(int32_t), 256);
 }
 
 cudaError_t launch_dispatch(const DispatchPlan& p, const void* x, const int32_t* topk_idx,
                             int d, moe_dtype_t dt, int32_t* counts, int32_t* offsets,
                             int32_t* src_row, int32_t* dst_pos, void* x_perm, void* ws,
-                            int* status, cudaStream_t s, bool hist_done, const float* row_w) {
+                            int* status, cudaStream_t s, bool hist_done, const float* row_w,
+                            bool own_status) {
   int32_t* blk = static_cast<int32_t*>(ws);
   if (p.T == 0) {
     cudaError_t e = cudaMemsetAsync(counts, 0, sizeof(int32_t) * p.nbins, s);
     if (e == cudaSuccess) e = cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (p.nbins + 1), s);
+    if (e == cudaSuccess && own_status) e = cudaMemsetAsync(status, 0, sizeof(int), s);
     return e;
   }
   if (!hist_done)
     launch_k(dispatch_hist_kernel, dim3(p.nblk), dim3(256), p.nbins * sizeof(int), s, topk_idx,
-             p.T, p.k, p.E, p.R, p.L, p.S, p.tb, p.nbins, blk, status);
+             p.T, p.k, p.E, p.R, p.L, p.S, p.tb, p.nbins, blk);
+  // own_status: the histogram kernel ran and the colscan writes the whole
+  // status word from its flags (the entry points clear nothing first);
+  // inside the layer the router wrote the table and the status is shared
   launch_k(dispatch_colscan_kernel, dim3(std::min(p.nbins, num_sms() * 8)), dim3(256),
            p.nbins * sizeof(int), s, blk, p.nblk, p.nbins, counts, offsets, src_row,
-           1LL * p.T * p.k);
+           1LL * p.T * p.k, (!hist_done && own_status) ? status : nullptr);
   const int elt = dt == MOE_BF16 ? 2 : 4;
   const int row_vec = d * elt / 16;
   const size_t sm3 = (p.nbins + p.tb * p.k) * sizeof(int);

@@ -10,13 +10,12 @@
 // memory, not HBM: CTA r owns token rows [r 128 / C, (r + 1) 128 / C) of the
 // tile, every CTA stores its partial rows into their owner's shared memory
 // (st.shared::cluster), and the owner adds the C partials in rank order (a
-// fixed order: the logits do not depend on timing or on the grid).  The C
-// threads of each owned token then split its E experts (thread j takes
-// experts j, j + C, ...), each keeps the top-k of its slice in registers,
-// and k rounds of a shuffle arg-max over the C threads merge the slices
-// (descending key, ties to the lower expert index); the first thread of the
-// token writes the indices and weights, and in the layer forward the
-// dispatch histogram of its token block.  The expert counts of the entry
+// fixed order: the logits do not depend on timing or on the grid).  One warp
+// per owned token then selects the k winners with k rounds of a warp
+// arg-max (two redux.sync reductions on (key, expert): descending key, ties
+// to the lower expert index) and writes the indices and weights; in the
+// layer forward the CTA also writes the dispatch histogram of its token
+// blocks.  The expert counts of the entry
 // point go through a per-CTA table that a second small kernel sums.  The
 // stage memory is sized so that two CTAs fit on an SM (for E <= 128): the
 // scores and top-k of one CTA overlap the loads of the other.
@@ -80,7 +79,7 @@ __device__ __forceinline__ void st_cluster_v4(uint32_t addr, uint32_t a, uint32_
 }
 __device__ __forceinline__ void bar_epi() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
-template <int BN, int KMAX>
+template <int BN>
 __global__ void __launch_bounds__(kThreads, 1)
     router_tc_kernel(const __grid_constant__ CUtensorMap tmX,
                      const __grid_constant__ CUtensorMap tmW, const Args a) {
@@ -225,159 +224,119 @@ __global__ void __launch_bounds__(kThreads, 1)
   cluster_sync_all();
 
   // --------------------------------------------------- scores and top-k
+  // One warp per owned token (the four epilogue warps take every fourth):
+  // lane l holds experts l, l + 32, ... (EPL of them), adds the C partials
+  // in rank order, and the k winners come from k rounds of a warp arg-max
+  // on (key descending, expert ascending) -- two redux.sync reductions each.
+  constexpr int EPL = BN / 32;
   if (warp >= 2) {
     const int i = threadIdx.x - 64;               // 0..127
+    const int ew = warp - 2;                      // epilogue warp 0..3
     const int E = a.E, k = a.k;
     const RouterOptions& opt = a.opt;
-    const int tpt = C;                            // threads per owned token
-    const int it = i / tpt;                       // owned token
-    const int jsl = i - it * tpt;                 // expert slice: e = jsl + tpt m
-    const bool lead = jsl == 0;
     int* dbins = reinterpret_cast<int*>(smem + align_up(static_cast<size_t>(BM) * pitch * 4, 16));
     int* ebins = dbins + (a.blk ? a.nbins : 0);
     float* wsum = reinterpret_cast<float*>(ebins + E);
+    int* tok_e = reinterpret_cast<int*>(wsum + E);   // [own][k] winners, for the histograms
     for (int e = i; e < E; e += 128) {
       ebins[e] = 0;
       wsum[e] = 0.f;
     }
     bar_epi();
     const int t_own0 = tile * BM + rank * own;
-    const int t = t_own0 + it;
-    const bool active = t < a.T;
-    const float* rp = recv + static_cast<size_t>(it) * pitch;
-    const size_t sstride = static_cast<size_t>(own) * pitch;
-    auto zval = [&](int e) {
-      float z = rp[e];
-      for (int s = 1; s < C; ++s) z += rp[s * sstride + e];   // ranks in order
-      return z;
-    };
-    // group reductions over the tpt threads of the token (aligned lanes)
-    auto gmax = [&](float v) {
-      for (int off = 1; off < tpt; off <<= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
-      return v;
-    };
-    auto gsum = [&](float v) {
-      for (int off = 1; off < tpt; off <<= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-      return v;
-    };
     const bool on_logits = opt.bias == nullptr && opt.scale > 0.f;
-    // softmax statistics where the keys or the weights need them
-    float mx = -INFINITY, den = 1.f;
-    const bool need_den = !opt.sigmoid && !(on_logits && a.renorm);
-    if (!on_logits || need_den) {
-      for (int e = jsl; e < E; e += tpt) {
-        float z = zval(e);
-        if (z != z) z = -INFINITY;
-        mx = fmaxf(mx, z);
-      }
-      mx = gmax(mx);
-      if (!opt.sigmoid) {
-        den = 0.f;
-        for (int e = jsl; e < E; e += tpt) {
-          float z = zval(e);
-          if (z != z) z = -INFINITY;
-          den += expf(z - mx);
-        }
-        den = gsum(den);
-      }
-    }
-    // the top-KMAX of this thread's slice (experts ascend within it, so an
-    // equal key never displaces an earlier expert)
-    int keyt[KMAX], idxt[KMAX];
+    const size_t sstride = static_cast<size_t>(own) * pitch;
+    for (int it = ew; it < own; it += 4) {
+      const int t = t_own0 + it;
+      if (t >= a.T) break;                        // warp-uniform
+      const float* rp = recv + static_cast<size_t>(it) * pitch + lane;
+      float sv[EPL];
+      bool avail[EPL];
 #pragma unroll
-    for (int q = 0; q < KMAX; ++q) {
-      keyt[q] = INT_MIN;
-      idxt[q] = -1;
-    }
-    for (int e = jsl; e < E; e += tpt) {
-      float z = zval(e);
-      if (a.logits_out && active) a.logits_out[static_cast<size_t>(t) * E + e] = z;
-      if (z != z) z = -INFINITY;
-      float kv = z;
-      if (!on_logits) {
-        const float ex = opt.sigmoid ? 1.0f / (1.0f + expf(-z)) : expf(z - mx);
-        kv = ex / den * opt.scale;
-        if (opt.bias) {
-          kv += opt.bias[e];
+      for (int q = 0; q < EPL; ++q) {
+        avail[q] = lane + 32 * q < E;
+        float z = 0.f;
+        if (avail[q]) {
+          z = rp[32 * q];
+          for (int sc = 1; sc < C; ++sc) z += rp[sc * sstride + 32 * q];   // ranks in order
+        }
+        sv[q] = z;
+      }
+      float mx = -INFINITY;
+#pragma unroll
+      for (int q = 0; q < EPL; ++q) {
+        if (avail[q] && a.logits_out) a.logits_out[static_cast<size_t>(t) * E + lane + 32 * q] = sv[q];
+        if (sv[q] != sv[q]) sv[q] = -INFINITY;
+        if (avail[q]) mx = fmaxf(mx, sv[q]);
+      }
+      // ex = exp(z - max z) (softmax numerators) or sigmoid(z); s = ex / den
+      float ex[EPL];
+      float den = 1.f;
+      if (opt.sigmoid) {
+#pragma unroll
+        for (int q = 0; q < EPL; ++q) ex[q] = avail[q] ? 1.0f / (1.0f + expf(-sv[q])) : 0.f;
+      } else {
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        den = 0.f;
+#pragma unroll
+        for (int q = 0; q < EPL; ++q) {
+          ex[q] = avail[q] ? expf(sv[q] - mx) : 0.f;
+          den += ex[q];
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
+      }
+      int key[EPL];
+#pragma unroll
+      for (int q = 0; q < EPL; ++q) {
+        float kv = on_logits ? sv[q] : ex[q] / den * opt.scale;
+        if (opt.bias && avail[q]) {
+          kv += opt.bias[lane + 32 * q];
           if (kv != kv) kv = -INFINITY;
         }
+        key[q] = score_key(kv);
       }
-      const int key = score_key(kv);
-      if (key > keyt[KMAX - 1]) {
+      int me = 0;
+      float mxv = 0.f;
+      for (int j = 0; j < k; ++j) {
+        int lk = INT_MIN, li = 0x7fffffff;
+        float lx = 0.f;
 #pragma unroll
-        for (int q = KMAX - 1; q > 0; --q) {
-          const bool shift = keyt[q - 1] < key;
-          const bool place = !shift && keyt[q] < key;
-          const int nk = shift ? keyt[q - 1] : (place ? key : keyt[q]);
-          const int ni = shift ? idxt[q - 1] : (place ? e : idxt[q]);
-          keyt[q] = nk;
-          idxt[q] = ni;
-        }
-        if (keyt[0] < key) {
-          keyt[0] = key;
-          idxt[0] = e;
-        }
-      }
-    }
-    // merge the slices: k rounds of an arg-max over the token's threads on
-    // (key descending, expert ascending); the winner pops its head
-    int sel[KMAX];
-#pragma unroll
-    for (int r = 0; r < KMAX; ++r) {
-      sel[r] = -1;
-      if (r < k) {
-        unsigned long long v =
-            (static_cast<unsigned long long>(static_cast<uint32_t>(keyt[0]) ^ 0x80000000u) << 32) |
-            static_cast<unsigned long long>(0xffffffffu - static_cast<uint32_t>(idxt[0]));
-        for (int off = 1; off < tpt; off <<= 1) {
-          const unsigned long long o = __shfl_xor_sync(0xffffffffu, v, off);
-          v = o > v ? o : v;
-        }
-        const int we = static_cast<int>(0xffffffffu - static_cast<uint32_t>(v & 0xffffffffu));
-        sel[r] = we;
-        if (idxt[0] == we) {
-#pragma unroll
-          for (int q = 0; q < KMAX - 1; ++q) {
-            keyt[q] = keyt[q + 1];
-            idxt[q] = idxt[q + 1];
+        for (int q = 0; q < EPL; ++q)
+          if (avail[q] && key[q] > lk) {   // experts of a lane ascend with q: first max wins
+            lk = key[q];
+            li = lane + 32 * q;
+            lx = ex[q];
           }
-          keyt[KMAX - 1] = INT_MIN;
-          idxt[KMAX - 1] = -1;
+        const int mk = __reduce_max_sync(0xffffffffu, lk);
+        const int be = __reduce_min_sync(0xffffffffu, lk == mk ? li : 0x7fffffff);
+        const float bx = __shfl_sync(0xffffffffu, lx, be & 31);
+#pragma unroll
+        for (int q = 0; q < EPL; ++q)
+          if (lane + 32 * q == be) avail[q] = false;
+        if (lane == j) {
+          me = be;
+          mxv = bx;
         }
+      }
+      // weights: the unbiased score of each winner (renormalised), times the scale
+      const float wx = lane < k ? mxv : 0.f;
+      float sel = wx;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) sel += __shfl_xor_sync(0xffffffffu, sel, off);
+      if (lane < k) {
+        const size_t o = static_cast<size_t>(t) * k + lane;
+        const float wv = wx / (a.renorm ? sel : den) * opt.scale;
+        a.topk_idx[o] = me;
+        a.topk_w[o] = wv;
+        tok_e[it * k + lane] = me;
+        atomicAdd(&ebins[me], 1);
+        if (a.lb) atomicAdd(&wsum[me], wv);
       }
     }
-    // weights: the unbiased score of each winner, renormalised when asked,
-    // times the scale (softmax: exp(z - max) over the denominator)
-    if (lead && active) {
-      if (on_logits && !opt.sigmoid && a.renorm) {
-        mx = zval(sel[0]);          // the largest logit
-        if (mx != mx) mx = -INFINITY;
-      }
-      float exs[KMAX];
-      float ssum = 0.f;
-#pragma unroll
-      for (int r = 0; r < KMAX; ++r) {
-        exs[r] = 0.f;
-        if (r < k) {
-          float z = zval(sel[r]);
-          if (z != z) z = -INFINITY;
-          exs[r] = opt.sigmoid ? 1.0f / (1.0f + expf(-z)) : expf(z - mx);
-          ssum += exs[r];
-        }
-      }
-      const float dv = a.renorm ? ssum : den;
-#pragma unroll
-      for (int r = 0; r < KMAX; ++r) {
-        if (r < k) {
-          const float wv = exs[r] / dv * opt.scale;
-          const size_t o = static_cast<size_t>(t) * k + r;
-          a.topk_idx[o] = sel[r];
-          a.topk_w[o] = wv;
-          atomicAdd(&ebins[sel[r]], 1);
-          if (a.lb) atomicAdd(&wsum[sel[r]], wv);
-        }
-      }
-    }
+    bar_epi();   // the winners of every owned token are in tok_e
     // dispatch histogram of every token block of tb rows this CTA owns
     if (a.blk) {
       if (blockIdx.x == 0 && i == 0)   // the dispatch column scan's ticket
@@ -387,10 +346,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int b = t_own0 / a.tb + jb;
         for (int x = i; x < a.nbins; x += 128) dbins[x] = 0;
         bar_epi();
-        if (lead && active && it / a.tb == jb) {
-#pragma unroll
-          for (int r = 0; r < KMAX; ++r)
-            if (r < k) atomicAdd(&dbins[dispatch_key(sel[r], t, a.R, a.L, a.S)], 1);
+        // the copies of the block's tb tokens, one per thread
+        for (int c = i; c < a.tb * k; c += 128) {
+          const int it = jb * a.tb + c / k;
+          const int t = t_own0 + it;
+          if (t < a.T) atomicAdd(&dbins[dispatch_key(tok_e[it * k + c % k], t, a.R, a.L, a.S)], 1);
         }
         bar_epi();
         if (b < a.nblk)
@@ -432,14 +392,14 @@ __global__ void router_counts_kernel(const int32_t* __restrict__ part, int G, in
   }
 }
 
-template <int BN, int KMAX>
+template <int BN>
 cudaError_t launch_bn(const CUtensorMap& tx, const CUtensorMap& tw, const Args& a, int grid,
                       size_t smem, cudaStream_t s) {
   static int configured[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(router_tc_kernel<BN, KMAX>,
+    cudaError_t e = cudaFuncSetAttribute(router_tc_kernel<BN>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
     if (e != cudaSuccess) return e;
     configured[dev] = 1;
@@ -458,15 +418,7 @@ cudaError_t launch_bn(const CUtensorMap& tx, const CUtensorMap& tw, const Args& 
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, router_tc_kernel<BN, KMAX>, tx, tw, a);
-}
-
-template <int BN>
-cudaError_t launch_k_of(const CUtensorMap& tx, const CUtensorMap& tw, const Args& a, int grid,
-                        size_t smem, cudaStream_t s) {
-  if (a.k <= 4) return launch_bn<BN, 4>(tx, tw, a, grid, smem, s);
-  if (a.k <= 8) return launch_bn<BN, 8>(tx, tw, a, grid, smem, s);
-  return launch_bn<BN, 16>(tx, tw, a, grid, smem, s);
+  return cudaLaunchKernelEx(&cfg, router_tc_kernel<BN>, tx, tw, a);
 }
 
 }  // namespace rtc
@@ -488,7 +440,8 @@ RouterFusedPlan router_fused_plan(int T, int d, int E, const DispatchPlan* plan)
     default: stages = rtc::Layout<256>::kStageRegion; tail = rtc::Layout<256>::kTailBytes; break;
   }
   const size_t exch = align_up(static_cast<size_t>(rtc::BM) * p.pitch * 4, 16) +
-                      (plan ? static_cast<size_t>(plan->nbins) * 4 : 0) + 8 * static_cast<size_t>(E);
+                      (plan ? static_cast<size_t>(plan->nbins) * 4 : 0) + 8 * static_cast<size_t>(E) +
+                      static_cast<size_t>(rtc::BM) * kMaxTopK * 4;   // the owned tokens' winners
   p.region = static_cast<int>(align_up(std::max<size_t>(stages, exch), 1024));
   p.smem = p.region + tail + 1024;   // + slack for the 1 KB alignment
   // two CTAs per SM when they fit (228 KB per SM, 1 KB reserved per CTA)
@@ -557,10 +510,10 @@ cudaError_t launch_router_fused(const void* x, const void* w_router, int T, int 
   a.status = status;
   cudaError_t e;
   switch (p.bn) {
-    case 32: e = rtc::launch_k_of<32>(tx, tw, a, p.grid, p.smem, s); break;
-    case 64: e = rtc::launch_k_of<64>(tx, tw, a, p.grid, p.smem, s); break;
-    case 128: e = rtc::launch_k_of<128>(tx, tw, a, p.grid, p.smem, s); break;
-    default: e = rtc::launch_k_of<256>(tx, tw, a, p.grid, p.smem, s); break;
+    case 32: e = rtc::launch_bn<32>(tx, tw, a, p.grid, p.smem, s); break;
+    case 64: e = rtc::launch_bn<64>(tx, tw, a, p.grid, p.smem, s); break;
+    case 128: e = rtc::launch_bn<128>(tx, tw, a, p.grid, p.smem, s); break;
+    default: e = rtc::launch_bn<256>(tx, tw, a, p.grid, p.smem, s); break;
   }
   if (e == cudaSuccess && counts) {
     launch_k(rtc::router_counts_kernel, dim3(cdiv(E, 256)), dim3(256), 0, s, counts_part, p.grid,

@@ -729,42 +729,135 @@ struct DownStagedPolicy : DownPolicy {
 // covered by 256-row pair tiles: CTA rank r owns rows [256 mt + 128 r, +128)
 // (its A operand and its accumulator lanes) and loads half of the B tile,
 // so a pair moves 64 KB per K block for the work that two single-CTA
-// 128 x 256 tiles do with 96 KB (the kernels are bound by this L2 -> shared
-// memory traffic).  The last m-tile of a segment, when it holds at most 128
-// rows, is a swap-AB pair tile instead: the weights are the M = 256 operand
-// (128 weight rows per SM) and the tile's tokens the N operand (the rows
-// rounded up to 32; each SM loads its N/2 token rows in 16-row boxes), so a
-// short tail costs in proportion to its rows instead of a full tile.
-//   GEMM1 normal tile: rank 0 loads w1 rows [e h + n0, +128), rank 1 the w3
-//     rows of the same hidden units; accumulator columns 0..127 hold G and
-//     128..255 hold U in both CTAs.
-//   GEMM1 swap tile: rank r loads w1 rows [e h + n0 + 64 r, +64) and the w3
-//     rows of the same units (two 64-row boxes): lanes 0..63 hold G and
-//     lanes 64..127 hold U of those 64 hidden units, one column per token.
+// 128 x 256 tiles do with 96 KB.  In GEMM2 the last m-tile of a segment,
+// when it holds at most 128 rows, is a swap-AB pair tile instead: the w2 rows
+// are the M = 256 operand (128 per SM) and the tile's tokens the N operand
+// (the rows rounded up to 32; each SM loads its N/2 token rows in 16-row
+// boxes), so a short tail costs in proportion to its rows.  GEMM1 keeps
+// normal pair tiles for its tails: its swap tiles needed the hidden units' G
+// and U, which land in different TMEM lane quadrants, to meet through 33 KB
+// of shared memory, and the sixth pipeline stage that memory buys measured
+// faster on B200 than the cheaper tails.
+//   GEMM1: rank 0 loads w1 rows [e h + n0, +128), rank 1 the w3 rows of the
+//     same hidden units; accumulator columns 0..127 hold G and 128..255 U.
 //   GEMM2: rank r loads w2 rows [e d + n0 + 128 r, +128), as the B half of a
 //     normal tile or as the A operand of a swap tile.
 constexpr int kPairSwapMaxRows = 128;
 constexpr int kTokBoxRows = 16;          // token rows per TMA box of a swap tile
-constexpr int kXchgPitch = 129;          // fp32 pitch of the swap tile's U exchange
 
+// Work units, taken round-robin by the pairs: the m-tiles of an (expert,
+// n-tile) in order, each its own unit, except that a segment's tail tile
+// joins the normal tile before it (one unit of two tiles run back to back by
+// the same pair, so the tail finds its weight tile in L2).  Units ordered
+// (expert, n-tile, m-tile) keep the tiles that share weight tiles together.
+// (Round-robin over single tiles gave, at ~256-row segments, some pairs a
+// third more work than the mean: normal and tail tiles alternate with the
+// segments and the even number of pairs keeps each pair on one kind;
+// putting every tail after every normal tile balanced it but re-read the
+// weights of the tails from DRAM.)  sched layout: [0] units, [1] n-tiles per
+// expert, [8 .. 8+E] offsets, [8+E+1 .. 8+2E+1] cumulative units per expert.
 template <int NCOLS, int NUM_B_, bool UP_>
 struct HybridPolicy : GroupedSched<256, NUM_B_, NCOLS, 256> {
   using Base = GroupedSched<256, NUM_B_, NCOLS, 256>;
   static constexpr bool UP = UP_;
-  static __device__ TileInfo tile_info(const Args& a, const int* sched, int tile, int rank) {
-    int e, nt, mt, cnt, seg0;
-    Base::locate(a, sched, tile, e, nt, mt, cnt, seg0);
-    TileInfo t;
+
+  // m-tiles of a segment of cnt rows, whether its last one is a tail tile,
+  // and its units per n-tile
+  static __device__ __forceinline__ void seg_tiles(int cnt, int& mt, int& tail, int& mu) {
+    mt = cdiv(max(cnt, 0), 256);
+    tail = (!UP && mt > 0 && cnt - (mt - 1) * 256 <= kPairSwapMaxRows) ? 1 : 0;
+    mu = (tail && mt >= 2) ? mt - 1 : mt;
+  }
+
+  static __device__ void prologue(const Args& a, int* sched) {
+    const int E = a.E;
+    int* off = sched + 8;
+    int* cum = off + E + 1;
+    for (int i = threadIdx.x; i <= E; i += blockDim.x) off[i] = a.offsets[i];
+    __syncthreads();
+    if (threadIdx.x < 32) {
+      const int lane = threadIdx.x;
+      const int nt = cdiv(a.n_out, NCOLS);
+      const int per = cdiv(E, 32);
+      const int e0 = min(E, lane * per), e1 = min(E, e0 + per);
+      int local = 0, bad = 0;
+      for (int e = e0; e < e1; ++e) {
+        const int cnt = off[e + 1] - off[e];
+        bad |= cnt < 0;
+        int mt, tail, mu;
+        seg_tiles(cnt, mt, tail, mu);
+        local += mu * nt;
+      }
+      int incl = local;
+#pragma unroll
+      for (int sh = 1; sh < 32; sh <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, sh);
+        if (lane >= sh) incl += v;
+      }
+      int run = incl - local;
+      for (int e = e0; e < e1; ++e) {
+        cum[e] = run;
+        int mt, tail, mu;
+        seg_tiles(off[e + 1] - off[e], mt, tail, mu);
+        run += mu * nt;
+      }
+      bad = __any_sync(0xffffffffu, bad);
+      const int total = __shfl_sync(0xffffffffu, incl, 31);
+      if (lane == 0) {
+        bad |= (off[0] != 0) || (off[E] != a.M);
+        cum[E] = total;
+        sched[0] = bad ? 0 : total;
+        sched[1] = nt;
+        if (bad && blockIdx.x == 0) set_status(a.status, MOE_DEV_BAD_OFFSETS);
+      }
+    }
+  }
+  static __device__ int num_units(const Args&, const int* sched) { return sched[0]; }
+
+  // unit -> expert e, n-tile, first m-tile; *ntiles = 1 or 2 (normal + tail)
+  static __device__ void locate_unit(const Args& a, const int* sched, int unit, int& e, int& nt,
+                                     int& mt, int& ntiles) {
+    const int E = a.E;
+    const int* off = sched + 8;
+    const int* cum = off + E + 1;
+    int lo = 0, hi = E - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (cum[mid] <= unit) lo = mid; else hi = mid - 1;
+    }
+    e = lo;
+    int mtt, tail, mu;
+    seg_tiles(off[e + 1] - off[e], mtt, tail, mu);
+    const int local = unit - cum[e];
+    nt = local / mu;
+    mt = local - nt * mu;
+    ntiles = (tail && mtt >= 2 && mt == mu - 1) ? 2 : 1;
+  }
+  static __device__ int unit_tiles(const Args& a, const int* sched, int unit) {
+    int e, nt, mt, n;
+    locate_unit(a, sched, unit, e, nt, mt, n);
+    return n;
+  }
+
+  // sub-tile `sub` (0 or 1) of a unit, for CTA `rank` of the pair
+  static __device__ TileInfo tile_info(const Args& a, const int* sched, int unit, int sub,
+                                       int rank) {
+    int e, nt, mt0, n;
+    locate_unit(a, sched, unit, e, nt, mt0, n);
+    const int* off = sched + 8;
+    const int seg0 = off[e], cnt = off[e + 1] - seg0;
+    const int mt = mt0 + sub;
     const int rows = cnt - mt * 256;        // rows from this m-tile to the segment's end
+    TileInfo t;
     t.n0 = nt * NCOLS;
     t.kb0 = 0;
     t.kb1 = cdiv(a.K, BK);
     t.m0 = 0;
-    if (rows <= kPairSwapMaxRows) {
+    if (!UP && rows <= kPairSwapMaxRows) {
       t.a_row = seg0 + mt * 256;            // the tile's first token
       t.m_valid = rows;                     // its tokens
       t.swap_np = (rows + 31) & ~31;        // MMA N of the pair
-      t.b_row = UP ? e * a.n_out + t.n0 + 64 * rank : e * a.n_out + t.n0 + 128 * rank;
+      t.b_row = e * a.n_out + t.n0 + 128 * rank;
     } else {
       const int r0 = mt * 256 + rank * 128;
       t.a_row = seg0 + r0;
@@ -777,71 +870,6 @@ struct HybridPolicy : GroupedSched<256, NUM_B_, NCOLS, 256> {
 };
 
 struct UpHybridPolicy : HybridPolicy<128, 2, true> {
-  // Swap tile: lanes 0..63 (quadrants 0, 1) hold G, lanes 64..127 (quadrants
-  // 2, 3) hold U of hidden units n0 + 64 rank + (lane mod 64), one column per
-  // token.  The U warps pass U through shared memory (fp32, 64 units x N
-  // tokens, odd pitch: conflict-free); the G warps then write H = silu(G) U
-  // (and, in the training forward, G and U) for 32 units per warp and
-  // instruction: 64 contiguous bytes of one token row.  `half` splits the
-  // tokens in chunks of 16 between the two warps of a quadrant.  The hand-off
-  // uses two mbarriers with bounded waits (xfull: the 4 U warps arrive after
-  // writing; xempty: the 4 G warps arrive after reading); `nswap` counts the
-  // swap tiles this warp has handled.  Returns false if a wait gave up.
-  static __device__ bool epilogue_swap_pair(const Args& a, const TileInfo& ti, uint32_t taddr,
-                                            int q, int half, float* xchg, int rank,
-                                            uint64_t* xfull, uint64_t* xempty, int nswap,
-                                            volatile int* abort_flag) {
-    const int lane = threadIdx.x & 31;
-    const int ntok = ti.m_valid;
-    const int h = a.n_out;
-    const uint32_t par = static_cast<uint32_t>(nswap) & 1u;
-    int ok = 1;
-    if (q >= 2) {
-      if (lane == 0) ok = mbar_wait(xempty, par ^ 1u, abort_flag, a.status) ? 1 : 0;
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) return false;
-      float* dst = xchg + ((q - 2) * 32 + lane) * kXchgPitch;
-      for (int t0 = 16 * half; t0 < ntok; t0 += 32) {
-        uint32_t u[16];
-        tmem_ld16(taddr + t0, u);
-        tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 16; ++i) dst[t0 + i] = __uint_as_float(u[i]);
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(xfull);
-      return true;
-    }
-    if (lane == 0) ok = mbar_wait(xfull, par, abort_flag, a.status) ? 1 : 0;
-    ok = __shfl_sync(0xffffffffu, ok, 0);
-    if (!ok) return false;
-    const int ul = q * 32 + lane;
-    const int unit = ti.n0 + 64 * rank + ul;
-    const bool uvalid = unit < h;
-    const float* src = xchg + ul * kXchgPitch;
-    for (int t0 = 16 * half; t0 < ntok; t0 += 32) {
-      uint32_t g[16];
-      tmem_ld16(taddr + t0, g);
-      tmem_ld_wait();
-      if (!uvalid) continue;
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int t = t0 + i;
-        if (t < ntok) {
-          const float gv = __uint_as_float(g[i]), uv = src[t];
-          const size_t r = static_cast<size_t>(ti.a_row + t);
-          a.out[r * h + unit] = __float2bfloat16_rn(silu_f(gv) * uv);
-          if (a.gu_out) {
-            a.gu_out[r * (2 * h) + unit] = __float2bfloat16_rn(gv);
-            a.gu_out[r * (2 * h) + h + unit] = __float2bfloat16_rn(uv);
-          }
-        }
-      }
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(xempty);
-    return true;
-  }
   static __device__ void epilogue_staged(const Args& a, int* s, const TileInfo& ti,
                                          uint32_t taddr, int row, uint8_t* stg, int c0, int c1) {
     UpStagedPolicy::epilogue_staged(a, s, ti, taddr, row, stg, c0, c1);
@@ -853,9 +881,8 @@ struct DownHybridPolicy : HybridPolicy<256, 1, false> {
   // token; a warp writes 32 features (64 contiguous bytes) of one token row
   // per instruction.  Tokens in chunks of 16, split between the two warps of
   // a quadrant by `half`.
-  static __device__ bool epilogue_swap_pair(const Args& a, const TileInfo& ti, uint32_t taddr,
-                                            int q, int half, float*, int rank, uint64_t*,
-                                            uint64_t*, int, volatile int*) {
+  static __device__ void epilogue_swap_pair(const Args& a, const TileInfo& ti, uint32_t taddr,
+                                            int q, int half, int rank) {
     const int lane = threadIdx.x & 31;
     const int f = ti.n0 + 128 * rank + q * 32 + lane;
     const bool fvalid = f < a.n_out;
@@ -875,7 +902,6 @@ struct DownHybridPolicy : HybridPolicy<256, 1, false> {
         }
       }
     }
-    return true;
   }
   static __device__ void epilogue_staged(const Args& a, int* s, const TileInfo& ti,
                                          uint32_t taddr, int row, uint8_t* stg, int c0, int c1) {
@@ -1484,29 +1510,23 @@ __global__ void __launch_bounds__(P::THREADS, 1)
 // TMA producer, warp 1 TMEM owner and (leader) MMA issuer, warps 2..9 the
 // epilogue (two per TMEM lane quadrant, each taking half of the columns).
 // Maps: tmA / tmB0 / tmB1 the normal tiles' operands (128-row boxes; tmB1
-// only for GEMM1), tmT the tokens in 16-row boxes, tmW0 / tmW1 the GEMM1
-// weights in 64-row boxes (swap tiles).
+// only for GEMM1), tmT the tokens of GEMM2's swap tiles in 16-row boxes.
 template <class P>
 struct PairLayout {
   static constexpr int kBHalfBytes = 128 * BK * 2;                  // 16 KB
   static constexpr int kStageBytes = kATileBytes + kBHalfBytes;    // 32 KB per CTA
-  static constexpr int kStages = 5;
+  static constexpr int kStages = 6;
   static constexpr uint32_t kTmemCols = 512;                       // 2 x 256 columns
   static constexpr int kEpiWarps = 8;
   static constexpr int kThreads = 64 + 32 * kEpiWarps;
   static constexpr int kBarOff = kStages * kStageBytes;
-  static constexpr int kNumBars = 2 * kStages + 7;   // + tfull[2], tempty[2], mma_done, xfull, xempty
+  static constexpr int kNumBars = 2 * kStages + 5;   // + tfull[2], tempty[2], mma_done
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSchedOff = (kMiscOff + 16 + 15) / 16 * 16;
   static constexpr int kEpiOff = (kSchedOff + P::SCHED_INTS * 4 + 15) / 16 * 16;
-  // the staged epilogue (2 KB per warp), then a swap tile's U exchange (its
-  // own memory: warps of the next tile may still stage while it is written)
-  static constexpr int kStgBytes = kEpiWarps * 2048;
-  static constexpr int kXchgOff = kEpiOff + kStgBytes;
-  static constexpr int kBytes = kXchgOff + 64 * kXchgPitch * 4;
+  static constexpr int kBytes = kEpiOff + kEpiWarps * 2048;   // the staged epilogue
   static constexpr int kLaunchBytes = kBytes + 1024;
   static_assert(kLaunchBytes <= 227 * 1024, "shared memory budget");
-  static_assert((64 * kXchgPitch * 4) % 16 == 0, "exchange buffer size");
 };
 
 template <class P>
@@ -1514,9 +1534,7 @@ __global__ void __launch_bounds__(PairLayout<P>::kThreads, 1)
     tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB0,
                         const __grid_constant__ CUtensorMap tmB1,
-                        const __grid_constant__ CUtensorMap tmT,
-                        const __grid_constant__ CUtensorMap tmW0,
-                        const __grid_constant__ CUtensorMap tmW1, const Args args) {
+                        const __grid_constant__ CUtensorMap tmT, const Args args) {
   using L = PairLayout<P>;
   constexpr int STAGES = L::kStages;
   constexpr uint32_t IDESC = idesc_bf16_f32(256, 256);
@@ -1530,13 +1548,10 @@ __global__ void __launch_bounds__(PairLayout<P>::kThreads, 1)
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* mma_done = tempty + 2;
-  uint64_t* xfull = mma_done + 1;
-  uint64_t* xempty = xfull + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
   int* sched = reinterpret_cast<int*>(smem + L::kSchedOff);
   uint8_t* epi = smem + L::kEpiOff;
-  float* xchg = reinterpret_cast<float*>(smem + L::kXchgOff);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -1553,20 +1568,16 @@ __global__ void __launch_bounds__(PairLayout<P>::kThreads, 1)
       mbar_init(tempty + a, 2 * L::kEpiWarps);   // every epilogue warp of both CTAs
     }
     mbar_init(mma_done, 1);
-    mbar_init(xfull, 4);    // the four U warps (quadrants 2, 3; both halves)
-    mbar_init(xempty, 4);   // the four G warps (quadrants 0, 1; both halves)
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB0);
-    tma_prefetch_desc(&tmT);
-    if (P::UP) {
+    if (P::UP)
       tma_prefetch_desc(&tmB1);
-      tma_prefetch_desc(&tmW0);
-      tma_prefetch_desc(&tmW1);
-    }
+    else
+      tma_prefetch_desc(&tmT);
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, L::kTmemCols);
@@ -1579,7 +1590,7 @@ __global__ void __launch_bounds__(PairLayout<P>::kThreads, 1)
   cluster_sync_all();   // barriers of both CTAs initialised before any remote arrive
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int total = P::num_tiles(args, sched);
+  const int total = P::num_units(args, sched);
   const int pair = blockIdx.x >> 1;
   const int npairs = gridDim.x >> 1;
 
@@ -1592,8 +1603,9 @@ __global__ void __launch_bounds__(PairLayout<P>::kThreads, 1)
       uint32_t phase = 0;
       int issued = 0;
       bool ok = true;
-      for (int tile = pair; tile < total && ok; tile += npairs) {
-        const TileInfo ti = P::tile_info(args, sched, tile, rank);
+      for (int unit = pair; unit < total && ok; unit += npairs)
+      for (int sub = 0, nsub = P::unit_tiles(args, sched, unit); sub < nsub && ok; ++sub) {
+        const TileInfo ti = P::tile_info(args, sched, unit, sub, rank);
         const int half_n = ti.swap_np / 2;                    // token rows of this CTA
         const int nbox = (half_n + kTokBoxRows - 1) / kTokBoxRows;
         const uint32_t cta_bytes =
@@ -1611,13 +1623,8 @@ __global__ void __launch_bounds__(PairLayout<P>::kThreads, 1)
             tma_load_2d_pair(sa, &tmA, bar, kb * BK, ti.a_row, pol);
             tma_load_2d_pair(sb, tb, bar, kb * BK, ti.b_row, pol);
           } else {
-            // A region: this CTA's 128 weight rows; B region: its N/2 tokens
-            if (P::UP) {
-              tma_load_2d_pair(sa, &tmW0, bar, kb * BK, ti.b_row, pol);
-              tma_load_2d_pair(sa + kATileBytes / 2, &tmW1, bar, kb * BK, ti.b_row, pol);
-            } else {
-              tma_load_2d_pair(sa, &tmB0, bar, kb * BK, ti.b_row, pol);
-            }
+            // A region: this CTA's 128 w2 rows; B region: its N/2 tokens
+            tma_load_2d_pair(sa, &tmB0, bar, kb * BK, ti.b_row, pol);
             for (int i = 0; i < nbox; ++i)
               tma_load_2d_pair(sb + i * kTokBoxRows * BK * 2, &tmT, bar, kb * BK,
                                ti.a_row + rank * half_n + i * kTokBoxRows, pol);
@@ -1650,13 +1657,17 @@ __global__ void __launch_bounds__(PairLayout<P>::kThreads, 1)
       uint32_t phase = 0;
       int it = 0;
       bool ok = true;
-      for (int tile = pair; tile < total && ok; tile += npairs, ++it) {
+      for (int unit = pair; unit < total && ok; unit += npairs)
+      for (int sub = 0, nsub = P::unit_tiles(args, sched, unit); sub < nsub && ok; ++sub, ++it) {
         const int acc = it & 1;
         const uint32_t aph = (it >> 1) & 1;
-        if (!mbar_wait_cluster(tempty + acc, aph ^ 1u, abort_flag, args.status)) break;
+        if (!mbar_wait_cluster(tempty + acc, aph ^ 1u, abort_flag, args.status)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * 256);
-        const TileInfo ti = P::tile_info(args, sched, tile, 0);
+        const TileInfo ti = P::tile_info(args, sched, unit, sub, 0);
         const uint32_t idesc = ti.swap_np ? idesc_bf16_f32(256, ti.swap_np) : IDESC;
         for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
           if (!mbar_wait(full + stage, phase, abort_flag, args.status)) {
@@ -1694,27 +1705,28 @@ __global__ void __launch_bounds__(PairLayout<P>::kThreads, 1)
     tempty_leader[0] = cluster_map(tempty + 0, 0);
     tempty_leader[1] = cluster_map(tempty + 1, 0);
     int it = 0;
-    int nswap = 0;
-    for (int tile = pair; tile < total; tile += npairs, ++it) {
+    bool run = true;
+    for (int unit = pair; unit < total && run; unit += npairs)
+    for (int sub = 0, nsub = P::unit_tiles(args, sched, unit); sub < nsub; ++sub, ++it) {
       const int acc = it & 1;
       const uint32_t aph = (it >> 1) & 1;
       int ok = 1;
       if (lane == 0) ok = mbar_wait(tfull + acc, aph, abort_flag, args.status) ? 1 : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) break;
+      if (!ok) {
+        run = false;
+        break;
+      }
       tc_fence_after();
-      const TileInfo ti = P::tile_info(args, sched, tile, rank);
+      const TileInfo ti = P::tile_info(args, sched, unit, sub, rank);
       const uint32_t taddr =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * 256);
-      if (ti.swap_np) {
-        if (!P::epilogue_swap_pair(args, ti, taddr, q, half, xchg, rank, xfull, xempty, nswap,
-                                   abort_flag))
-          break;
-        ++nswap;
-      } else {
+      if constexpr (!P::UP) {
+        if (ti.swap_np) P::epilogue_swap_pair(args, ti, taddr, q, half, rank);
+      }
+      if (!ti.swap_np)
         P::epilogue_staged(args, sched, ti, taddr, row, epi + (warp - 2) * 2048, 4 * half,
                            4 * half + 4);
-      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tempty_leader[acc]);
@@ -1788,8 +1800,7 @@ cudaError_t launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMa
 // Launch of the CTA-pair kernel: clusters of 2 CTAs, an even grid.
 template <class P>
 cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
-                        const CUtensorMap& t, const CUtensorMap& w0, const CUtensorMap& w1,
-                        const Args& args, int pairs, cudaStream_t s) {
+                        const CUtensorMap& t, const Args& args, int pairs, cudaStream_t s) {
   using L = PairLayout<P>;
   static int configured[64] = {0};
   int dev = 0;
@@ -1815,7 +1826,7 @@ cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUten
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, tc_gemm_pair_kernel<P>, a, b0, b1, t, w0, w1, args);
+  return cudaLaunchKernelEx(&cfg, tc_gemm_pair_kernel<P>, a, b0, b1, t, args);
 }
 
 }  // namespace tc
@@ -1915,14 +1926,11 @@ static cudaError_t swiglu_tc_impl(const void* a_src, int a_rows, const int32_t* 
   a.gather_src = a_src;
   a.gu_out = static_cast<__nv_bfloat16*>(gu);
   if (pairs) {
-    CUtensorMap txs, t1h, t3h, ths;
-    if (!make_tmap(&txs, a_src, d, a_rows, kTokBoxRows)) return cudaErrorInvalidValue;
-    if (!make_tmap(&t1h, w1, d, static_cast<uint64_t>(E) * h, 64)) return cudaErrorInvalidValue;
-    if (!make_tmap(&t3h, w3, d, static_cast<uint64_t>(E) * h, 64)) return cudaErrorInvalidValue;
+    CUtensorMap ths;
     if (!make_tmap(&ths, H, h, N, kTokBoxRows)) return cudaErrorInvalidValue;
     const long long max_pt = cdiv(N, 256) + E;   // upper bound on pair tiles per n-tile
     int np = static_cast<int>(std::min<long long>(num_sms() / 2, max_pt * cdiv(h, 128)));
-    cudaError_t e = launch_pair<UpHybridPolicy>(tx, t1, t3, txs, t1h, t3h, a, np, s);
+    cudaError_t e = launch_pair<UpHybridPolicy>(tx, t1, t3, tx, a, np, s);
     if (e != cudaSuccess) return e;
     a.K = h;
     a.n_out = d;
@@ -1930,7 +1938,7 @@ static cudaError_t swiglu_tc_impl(const void* a_src, int a_rows, const int32_t* 
     a.gu_out = nullptr;
     a.row_scale = row_scale;
     np = static_cast<int>(std::min<long long>(num_sms() / 2, max_pt * cdiv(d, 256)));
-    return launch_pair<DownHybridPolicy>(th, t2, t2, ths, t2, t2, a, np, s);
+    return launch_pair<DownHybridPolicy>(th, t2, t2, ths, a, np, s);
   }
   int grid = static_cast<int>(std::min<long long>(num_sms(), 1LL * max_mt * cdiv(h, 128)));
   cudaError_t e = gather ? launch<UpGatherPolicy>(tx, t1, t3, a, grid, s)
