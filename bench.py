@@ -453,9 +453,40 @@ def other_config(M, idx, dev, stream, flush, pk, steps=10, warmup=3):
     return rec
 
 
+def profile_stage(args):
+    """For ncu captures of one kernel family on a small device footprint:
+    run one stage of the layer three times (no timing, no JSON).  router:
+    only x and w_router are allocated; grouped_swiglu: the layer is routed
+    and dispatched once, then the experts run three times."""
+    import routing_dispatch_grouped_topk_b200 as M
+    M.lib()
+    cfg = W.config(args.config)
+    dev = torch.device("cuda", 0)
+    T, d, E, k = cfg.T, cfg.d, cfg.E, cfg.top_k
+    dt = M.MOE_BF16 if cfg.dtype == "bf16" else M.MOE_F32
+    if args.profile_stage == "router":
+        lay = W.make_layer(cfg, dev, experts=False)
+        idx = torch.empty(T, k, dtype=torch.int32, device=dev)
+        w = torch.empty(T, k, dtype=torch.float32, device=dev)
+        rws = torch.empty(M.router_workspace_size(T, d, E, dt), dtype=torch.uint8, device=dev)
+        for _ in range(3):
+            M.moe_router_topk(lay["x"], lay["w_router"], None, T, d, E, k, M.MOE_SCORE_SOFTMAX,
+                              cfg.renormalize, dt, None, idx, w, None, rws)
+    else:
+        lay = W.make_layer(cfg, dev)
+        idx, w, _, _, _ = M.router_topk(lay["x"], lay["w_router"], k, cfg.renormalize)
+        _, off, _, _, xp, _ = M.dispatch(lay["x"], idx, E)
+        for _ in range(3):
+            M.grouped_swiglu(xp, off, lay["w1"], lay["w3"], lay["w2"])
+    torch.cuda.synchronize()
+
+
 def run_ours(args, ws, rank, local):
     import routing_dispatch_grouped_topk_b200 as M
     M.lib()  # fails loudly if the CUDA library is missing
+    if args.profile and args.profile_stage != "all":
+        profile_stage(args)
+        return
     cfg = W.config(args.config)
     T, d, E, k, h, R = cfg.T, cfg.d, cfg.E, cfg.top_k, cfg.h, cfg.ep_ranks
     dev = torch.device("cuda", local)
@@ -869,6 +900,9 @@ def main():
     ap.add_argument("--profile", action="store_true",
                     help="for ncu captures: run the staged step twice, then moe_forward "
                          "once, and exit (no timing, no JSON)")
+    ap.add_argument("--profile-stage", default="all", choices=["all", "router", "grouped_swiglu"],
+                    help="with --profile: run only this stage three times (small device "
+                         "footprint for multi-pass captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

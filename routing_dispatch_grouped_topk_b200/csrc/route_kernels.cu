@@ -248,16 +248,16 @@ __global__ void __launch_bounds__(1024) dispatch_scatter_kernel(const uint4* __r
   }
   __syncthreads();
   if (!x_perm) return;
-  // Row copies: a warp per token; each lane issues up to four 16-byte loads
+  // Row copies: a warp per token; each lane issues up to eight 16-byte loads
   // of the row before storing them to the token's k slots.
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
   for (int t = t0 + warp; t < t1; t += nw) {
     const uint4* src = x + static_cast<size_t>(t) * row_vec;
     const int* sl = slot + (t - t0) * k;
-    for (int c0 = 0; c0 < row_vec; c0 += 128) {
-      uint4 v[4];
+    for (int c0 = 0; c0 < row_vec; c0 += 256) {
+      uint4 v[8];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < 8; ++u) {
         const int c = c0 + u * 32 + lane;
         if (c < row_vec) v[u] = src[c];
       }
@@ -268,7 +268,7 @@ __global__ void __launch_bounds__(1024) dispatch_scatter_kernel(const uint4* __r
         // [HP] MoE.forward with score_before_experts: routed row times its weight
         const float wj = row_w ? row_w[static_cast<size_t>(t) * k + j] : 1.0f;
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < 8; ++u) {
           const int c = c0 + u * 32 + lane;
           if (c < row_vec) dst[c] = row_w ? scale_vec(v[u], wj, bf16) : v[u];
         }
