@@ -367,6 +367,64 @@ class Layer:
         mark(i + 2)
 
 
+def timed_folded(layer, stream, flush, steps):
+    """CUDA-event times (ms) of moe_grouped_swiglu_combine (the combine
+    folded into GEMM2) on the layer's routed rows, L2 flushed between calls;
+    None where the folded path does not apply (fp32, decode-sized segments).
+    Its dst_pos addresses the expert-major rows the experts read (through
+    the regroup's inverse permutation under simulated EP), composed once
+    before timing from the last staged step."""
+    c, M = layer.cfg, layer.M
+    if layer.dt != M.MOE_BF16 or c.N < 64 * c.E:
+        return None
+    R = c.ep_ranks
+    xe, off = (layer.x_em, layer.oem) if R > 1 else (layer.x_perm, layer.offsets)
+    dst = layer.pinv[layer.dst_pos.long()].int() if R > 1 else layer.dst_pos
+    ws = torch.empty(M.lib().moe_grouped_swiglu_combine_workspace_size(c.T, c.top_k, c.d, c.h,
+                                                                       c.E, layer.dt),
+                     dtype=torch.uint8, device=layer.dev)
+    out = torch.empty_like(layer.out)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps + 2)]
+    torch.cuda.synchronize()
+    for a_ev, b_ev in ev:
+        a_ev.record(stream)
+        M.moe_grouped_swiglu_combine(xe, off, layer.w1, layer.w3, layer.w2, dst, layer.w, c.T,
+                                     c.top_k, c.d, c.h, c.E, layer.dt, out, ws)
+        b_ev.record(stream)
+        flush.zero_()
+    torch.cuda.synchronize()
+    # the folded output against the staged step's (rounding differs: y is
+    # not rounded to bf16 on the folded path)
+    err = (out.float() - layer.out.float()).abs().max().item()
+    ref = layer.out.float().abs().max().item()
+    return [a.elapsed_time(b) for a, b in ev[2:]], err / max(ref, 1e-30)
+
+
+def timed_graph(layer, stream, flush, steps):
+    """CUDA-event times (ms) of replays of one moe_forward call captured in a
+    CUDA graph (the same kernels; no host work per step), L2 flushed between
+    replays, and whether the replay's output equals the direct call's."""
+    layer.forward()
+    torch.cuda.synchronize()
+    ref = layer.fout.clone()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        layer.forward()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps + 2)]
+    torch.cuda.synchronize()
+    for a_ev, b_ev in ev:
+        a_ev.record(stream)
+        g.replay()
+        b_ev.record(stream)
+        flush.zero_()
+    torch.cuda.synchronize()
+    same = bool(torch.equal(layer.fout, ref))
+    del g
+    return [a.elapsed_time(b) for a, b in ev[2:]], same
+
+
 def timed_forward(layer, stream, flush, steps):
     """CUDA-event time (ms) of each moe_forward step; L2 flushed between
     steps, outside the events."""
@@ -624,6 +682,11 @@ def run_ours(args, ws, rank, local):
     e2e_pipe_total = max_over_ranks(t0e.elapsed_time(t1e), ws)
     e2e_pipe_value = job_tokens_per_s(T, ws, args.steps, e2e_pipe_total)
     e2e_match = e2e_match and bool(torch.equal(oh[(args.steps - 1) % 2].to(dev), out))
+    # The combine folded into GEMM2 (moe_grouped_swiglu_combine), timed beside
+    # the unfused grouped SwiGLU + combine of the staged step.
+    folded = timed_folded(layer, stream, flush, min(args.steps, 10))
+    graph_ms, graph_same = timed_graph(layer, stream, flush, args.steps)
+    graph_total = max_over_ranks(sum(graph_ms), ws)
     clocks = sampler.stop() if rank == 0 else None
 
     if rank != 0:
@@ -687,6 +750,18 @@ def run_ours(args, ws, rank, local):
         "clocks": clocks,
         "peaks": pk,
     }
+    line["cuda_graph"] = {
+        "value": job_tokens_per_s(T, ws, args.steps, graph_total), "unit": UNIT,
+        "ms_per_step": graph_total / args.steps, "output_matches_direct_call": graph_same,
+        "what": "the same moe_forward call captured once in a CUDA graph and replayed each "
+                "step (no host work per step); L2 flushed between replays"}
+    if folded is not None:
+        line["folded_combine"] = {
+            "us": 1e3 * statistics.median(folded[0]),
+            "unfused_us": 1e3 * (stage_ms["grouped_swiglu"] + stage_ms["combine"]),
+            "max_diff_vs_staged_rel": folded[1],
+            "what": "moe_grouped_swiglu_combine (fp32 reductions in GEMM2's epilogue, then one "
+                    "bf16 rounding) against moe_grouped_swiglu + moe_combine"}
     if ws == 1 and not args.no_other_configs:
         del layer
         torch.cuda.empty_cache()

@@ -328,6 +328,34 @@ MOE_API moe_status_t moe_grouped_swiglu_gather(const void* x, int T, const int32
                                        size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * moe_grouped_swiglu_combine -- the grouped SwiGLU with the combine folded
+ * into GEMM2's epilogue ([HP] MoE.unpermutation's scatter_add done by the
+ * expert GEMM itself): no y [N, d] is written.
+ *   out[t] = sum_j w[t, j] * (H[s] . w2[e(s)]^T),  s = dst_pos[t, j]
+ * with H as moe_grouped_swiglu (bf16) and w = topk_w (fp32) or 1 when
+ * topk_w == NULL.  Each GEMM2 output row, times its weight, is added in
+ * fp32 into the token's row of an fp32 buffer in the workspace (the order
+ * of the k additions is not fixed, so results may differ run to run in the
+ * last fp32 bits), which is rounded once to bf16 into out [T, d].
+ * x_perm [N, d] with N = T * top_k, offsets [E+1], w1, w3 [E, h, d], w2
+ * [E, d, h], dst_pos [T, top_k] from moe_dispatch (positions outside
+ * [0, N) add nothing).  bf16 only, d % 64 == 0, h % 64 == 0, and only where
+ * the grouped SwiGLU runs on CTA pairs (N >= 64 E); otherwise
+ * MOE_ERR_UNSUPPORTED.  Workspace moe_grouped_swiglu_combine_workspace_size
+ * (status word, H, the fp32 output, the slots' tokens and weights).
+ * moe_forward keeps the deterministic path (moe_grouped_swiglu, then the
+ * gather-reduce of moe_combine); this entry point is the alternative for
+ * callers that accept run-to-run differences in the last bits.
+ * ---------------------------------------------------------------------- */
+MOE_API size_t moe_grouped_swiglu_combine_workspace_size(int T, int top_k, int d, int h, int E,
+                                                 moe_dtype_t dt);
+MOE_API moe_status_t moe_grouped_swiglu_combine(const void* x_perm, const int32_t* offsets,
+                                        const void* w1, const void* w3, const void* w2,
+                                        const int32_t* dst_pos, const float* topk_w, int T,
+                                        int top_k, int d, int h, int E, moe_dtype_t dt,
+                                        void* out, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * moe_combine -- [QO] SpeedupMoeExperts.forward training branch
  * (weighted index_add_); [HP] MoE.unpermutation (scatter_add).
  *
@@ -350,13 +378,14 @@ MOE_API moe_status_t moe_combine(const void* y, const int32_t* dst_pos, const in
  *
  * moe_grouped_swiglu_train -- moe_grouped_swiglu (no row_scale) that also
  * returns what the backward needs:
- *   H [N, h]   = silu(G) * U, rounded to bf16 (the GEMM2 operand)
+ *   H [N, h]   = silu(G) * U, in dt (the GEMM2 operand)
  *   gu [N, 2h] = G | U with G = x_perm[s] . w1[e]^T in columns [0, h) and
  *                U = x_perm[s] . w3[e]^T in [h, 2h), each rounded once to
- *                bf16 from the fp32 accumulator.
- * bf16 only (MOE_ERR_UNSUPPORTED otherwise); shapes and alignment as
- * moe_grouped_swiglu; rows of empty experts are not written.  No workspace
- * beyond a 256-byte device status word (ws, ws_bytes >= 256).
+ *                dt from the fp32 accumulator (bf16: tcgen05; fp32: CUDA
+ *                cores, no rounding).
+ * Shapes and alignment as moe_grouped_swiglu; rows of empty experts are not
+ * written; y is bit-identical to moe_grouped_swiglu's.  No workspace beyond
+ * a 256-byte device status word (ws, ws_bytes >= 256).
  *
  * moe_grouped_swiglu_backward -- for every expert e with rows S (the
  * segment of x_perm), G, U from gu and upstream gradient dY = dy[seg]:
@@ -364,12 +393,13 @@ MOE_API moe_status_t moe_combine(const void* y, const int32_t* dst_pos, const in
  *   dx_perm[seg] = dG . w1[e] + dU . w3[e]                    [N, d]
  *   dw1[e] = dG^T . S,  dw3[e] = dU^T . S                      [E, h, d]
  *   dw2[e] = dY^T . H[seg]                                    [E, d, h]
- * silu'(g) = s(g) (1 + g (1 - s(g))), s the logistic sigmoid.  fp32
- * accumulation on tcgen05 tensor cores; dG and dU are rounded to bf16 once
- * (they are operands of the next products), every output once.  Experts
- * with no rows get zero weight gradients.  bf16 only; d % 64 == 0 and
- * h % 64 == 0; all pointers 16-byte aligned; workspace
- * moe_grouped_swiglu_backward_workspace_size (dG | dU [N, 2h] bf16 plus
+ * silu'(g) = s(g) (1 + g (1 - s(g))), s the logistic sigmoid.  bf16: fp32
+ * accumulation on tcgen05 tensor cores, dG and dU rounded to bf16 once
+ * (they are operands of the next products), every output once; d % 64 == 0
+ * and h % 64 == 0.  fp32: CUDA cores, fp32 throughout; d % 4 == 0 and
+ * h % 4 == 0.  Experts with no rows get zero weight gradients.  All
+ * pointers 16-byte aligned; workspace
+ * moe_grouped_swiglu_backward_workspace_size (dG | dU [N, 2h] in dt plus
  * the status word).  Bad offsets set MOE_DEV_BAD_OFFSETS in the status
  * word (moe_get_device_status) and the outputs are not written.
  *
@@ -399,13 +429,14 @@ MOE_API moe_status_t moe_combine(const void* y, const int32_t* dst_pos, const in
  *   dz = s * (ds - <s, ds>)   (softmax)   or   dz = ds * s * (1 - s)  (sigmoid)
  *   d_logits = dz (fp32, optional), dw_router = dz^T x [E, d] (optional),
  *   dx = dz w_router [T, d] (optional)
- * The gate products run on tcgen05 from dz rounded once to bf16, with fp32
- * accumulation (bf16 x and w_router; dw_router and dx need dt = MOE_BF16,
- * E % 8 == 0 and d % 64 == 0).  dw_router is reduced over token segments
- * into fp32 partials summed in segment order (deterministic).  opts NULL =
+ * dt = MOE_BF16: the gate products run on tcgen05 from dz rounded once to
+ * bf16, with fp32 accumulation (E % 8 == 0 and d % 64 == 0); dw_router is
+ * reduced over token segments into fp32 partials summed in segment order
+ * (deterministic).  dt = MOE_F32: fp32 x, w_router, dw_router and dx; the
+ * products run on CUDA cores from dz in fp32.  opts NULL =
  * defaults (softmax, no renormalisation, scale 1).  E <= 512.  Workspace
- * moe_router_backward_workspace_size (dz in bf16, the partials and the
- * status word).  Entries of topk_idx outside [0, E) are skipped.
+ * moe_router_backward_workspace_size (dz, the partials and the status
+ * word).  Entries of topk_idx outside [0, E) are skipped.
  * ---------------------------------------------------------------------- */
 MOE_API moe_status_t moe_grouped_swiglu_train(const void* x_perm, const int32_t* offsets,
                                       const void* w1, const void* w3, const void* w2, int N,

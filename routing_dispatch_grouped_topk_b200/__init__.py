@@ -36,7 +36,8 @@ __all__ = [
     "EXPORTED_SYMBOLS",
     "moe_router_topk", "moe_dispatch", "moe_ep_dispatch_rank_major", "moe_ep_local_regroup",
     "moe_grouped_swiglu", "moe_grouped_swiglu_gather", "moe_combine", "moe_forward",
-    "moe_get_device_status", "grouped_swiglu_gather",
+    "moe_get_device_status", "grouped_swiglu_gather", "moe_grouped_swiglu_combine",
+    "grouped_swiglu_combine",
     "router_workspace_size", "dispatch_workspace_size", "ep_dispatch_workspace_size",
     "regroup_workspace_size", "grouped_swiglu_workspace_size", "forward_workspace_size",
     "router_topk", "dispatch", "ep_dispatch_rank_major", "ep_local_regroup",
@@ -63,6 +64,7 @@ EXPORTED_SYMBOLS = [
     "moe_ep_dispatch_workspace_size", "moe_ep_dispatch_rank_major",
     "moe_regroup_workspace_size", "moe_ep_local_regroup",
     "moe_grouped_swiglu_workspace_size", "moe_grouped_swiglu", "moe_grouped_swiglu_gather",
+    "moe_grouped_swiglu_combine_workspace_size", "moe_grouped_swiglu_combine",
     "moe_combine",
     "moe_grouped_swiglu_train", "moe_grouped_swiglu_backward_workspace_size",
     "moe_grouped_swiglu_backward", "moe_combine_backward", "moe_dispatch_backward",
@@ -128,6 +130,9 @@ _SIGS = {
     "moe_grouped_swiglu": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _Z, _P]),
     "moe_grouped_swiglu_gather": (_I, [_P, _I, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P,
                                        _P, _Z, _P]),
+    "moe_grouped_swiglu_combine_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I]),
+    "moe_grouped_swiglu_combine": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P,
+                                        _P, _Z, _P]),
     "moe_combine": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P]),
     "moe_grouped_swiglu_train": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _Z,
                                       _P]),
@@ -359,6 +364,15 @@ def moe_grouped_swiglu_gather(x, T, src_row, offsets, w1, w3, w2, row_scale, N, 
         "moe_grouped_swiglu_gather")
 
 
+def moe_grouped_swiglu_combine(x_perm, offsets, w1, w3, w2, dst_pos, topk_w, T, top_k, d, h, E,
+                               dt, out, ws, stream=None):
+    _check(lib().moe_grouped_swiglu_combine(
+        _ptr(x_perm, name="x_perm"), _ptr(offsets, torch.int32, "offsets"), _ptr(w1, name="w1"),
+        _ptr(w3, name="w3"), _ptr(w2, name="w2"), _ptr(dst_pos, torch.int32, "dst_pos"),
+        _ptr(topk_w, torch.float32, "topk_w"), T, top_k, d, h, E, dt, _ptr(out, name="out"),
+        _ptr(ws, name="ws"), _nbytes(ws), _stream(stream)), "moe_grouped_swiglu_combine")
+
+
 def moe_combine(y, dst_pos, row_map, topk_w, T, d, N, top_k, dt, out, stream=None):
     _check(lib().moe_combine(
         _ptr(y, name="y"), _ptr(dst_pos, torch.int32, "dst_pos"),
@@ -587,6 +601,20 @@ def grouped_swiglu(x_perm, offsets, w1, w3, w2, row_scale=None):
     ws = _ws(grouped_swiglu_workspace_size(N, d, h, E, _dt(x_perm)), x_perm.device)
     moe_grouped_swiglu(x_perm, offsets, w1, w3, w2, row_scale, N, d, h, E, _dt(x_perm), y, ws)
     return y, ws
+
+
+def grouped_swiglu_combine(x_perm, offsets, w1, w3, w2, dst_pos, topk_w=None):
+    """The grouped SwiGLU with the combine folded into GEMM2.  Returns
+    (out [T, d], ws)."""
+    T, k = dst_pos.shape
+    d = x_perm.shape[1]
+    E, h, _ = w1.shape
+    dt = _dt(x_perm)
+    out = torch.empty(T, d, dtype=x_perm.dtype, device=x_perm.device)
+    ws = _ws(lib().moe_grouped_swiglu_combine_workspace_size(T, k, d, h, E, dt), x_perm.device)
+    moe_grouped_swiglu_combine(x_perm, offsets, w1, w3, w2, dst_pos, topk_w, T, k, d, h, E, dt,
+                               out, ws)
+    return out, ws
 
 
 def grouped_swiglu_gather(x, src_row, offsets, w1, w3, w2, row_scale=None):

@@ -720,6 +720,83 @@ moe_status_t moe_grouped_swiglu_gather(const void* x, int T, const int32_t* src_
   return cuda_status(e, "moe_grouped_swiglu_gather");
 }
 
+// ------------------------------------------ grouped SwiGLU + folded combine
+namespace {
+// status, H [N, h] bf16, the fp32 output [T, d], slot tokens and weights [N]
+struct FoldWs {
+  int* status;
+  void* H;
+  float* out32;
+  int32_t* slot_tok;
+  float* slot_w;
+  size_t bytes;
+};
+FoldWs carve_fold(void* base, int T, int k, int d, int h) {
+  FoldWs f{};
+  Carve c(base);
+  const size_t N = static_cast<size_t>(T) * k;
+  f.status = c.take<int>(kStatusBytes / sizeof(int));
+  f.H = c.take<char>(N * h * 2);
+  f.out32 = c.take<float>(static_cast<size_t>(T) * d);
+  f.slot_tok = c.take<int32_t>(N);
+  f.slot_w = c.take<float>(N);
+  f.bytes = c.off;
+  return f;
+}
+}  // namespace
+
+size_t moe_grouped_swiglu_combine_workspace_size(int T, int top_k, int d, int h, int E,
+                                                 moe_dtype_t dt) {
+  (void)E;
+  (void)dt;
+  if (T < 0 || top_k < 1 || d < 1 || h < 1) return kStatusBytes;
+  return carve_fold(nullptr, T, top_k, d, h).bytes;
+}
+
+moe_status_t moe_grouped_swiglu_combine(const void* x_perm, const int32_t* offsets,
+                                        const void* w1, const void* w3, const void* w2,
+                                        const int32_t* dst_pos, const float* topk_w, int T,
+                                        int top_k, int d, int h, int E, moe_dtype_t dt, void* out,
+                                        void* ws, size_t ws_bytes, void* stream) {
+  MOE_CHECK_ARG(T >= 0 && top_k >= 1 && top_k <= kMaxTopK, "bad sizes T=%d top_k=%d", T, top_k);
+  const int N = T * top_k;
+  if (moe_status_t st = check_swiglu_shape(N, d, h, E, dt)) return st;
+  if (dt != MOE_BF16 || (N > 0 && !swiglu_tc_uses_pairs(N, E))) {
+    set_last_error("moe_grouped_swiglu_combine: bf16 layers whose segments average 64 rows or "
+                   "more (the CTA-pair GEMM path); N=%d E=%d",
+                   N, E);
+    return MOE_ERR_UNSUPPORTED;
+  }
+  if (T > 0) {
+    MOE_CHECK_ARG(x_perm && offsets && w1 && w3 && w2 && dst_pos && out,
+                  "x_perm, offsets, w1, w3, w2, dst_pos, out are required");
+    MOE_CHECK_ARG(aligned16(x_perm) && aligned16(w1) && aligned16(w3) && aligned16(w2) &&
+                      aligned16(out),
+                  "x_perm, w1, w3, w2, out must be 16-byte aligned");
+  }
+  MOE_CHECK_ARG(ws != nullptr, "ws is required");
+  const size_t need = moe_grouped_swiglu_combine_workspace_size(T, top_k, d, h, E, dt);
+  if (ws_bytes < need) {
+    set_last_error("grouped_swiglu_combine workspace %zu < %zu", ws_bytes, need);
+    return MOE_ERR_WORKSPACE;
+  }
+  const FoldWs f = carve_fold(ws, T, top_k, d, h);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(f.status, 0, sizeof(int), s);
+  if (e == cudaSuccess && T > 0) {
+    // slots no (t, j) points to keep token -1 and add nothing
+    e = cudaMemsetAsync(f.slot_tok, 0xff, static_cast<size_t>(N) * sizeof(int32_t), s);
+    if (e == cudaSuccess) e = launch_slot_map(dst_pos, topk_w, T, top_k, N, f.slot_tok, f.slot_w, s);
+    if (e == cudaSuccess)
+      e = cudaMemsetAsync(f.out32, 0, static_cast<size_t>(T) * d * sizeof(float), s);
+    if (e == cudaSuccess)
+      e = launch_swiglu_tc_combine(x_perm, offsets, w1, w3, w2, N, d, h, E, f.H, f.slot_tok,
+                                   f.slot_w, T, f.out32, f.status, s);
+    if (e == cudaSuccess) e = launch_f32_to_bf16(f.out32, static_cast<size_t>(T) * d, out, s);
+  }
+  return cuda_status(e, "moe_grouped_swiglu_combine");
+}
+
 // ------------------------------------------------------------------ combine
 moe_status_t moe_combine(const void* y, const int32_t* dst_pos, const int32_t* row_map,
                          const float* topk_w, int T, int d, int N, int top_k, moe_dtype_t dt,
@@ -744,10 +821,6 @@ moe_status_t moe_grouped_swiglu_train(const void* x_perm, const int32_t* offsets
                                       moe_dtype_t dt, void* y, void* h_act, void* gu, void* ws,
                                       size_t ws_bytes, void* stream) {
   if (moe_status_t st = check_swiglu_shape(N, d, h, E, dt)) return st;
-  if (dt != MOE_BF16) {
-    set_last_error("moe_grouped_swiglu_train: bf16 only");
-    return MOE_ERR_UNSUPPORTED;
-  }
   if (N > 0) {
     MOE_CHECK_ARG(x_perm && offsets && w1 && w3 && w2 && y && h_act && gu,
                   "x_perm, offsets, w1, w3, w2, y, h_act, gu required");
@@ -763,17 +836,24 @@ moe_status_t moe_grouped_swiglu_train(const void* x_perm, const int32_t* offsets
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int* status = static_cast<int*>(ws);
   cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), s);
-  if (e == cudaSuccess && N > 0)
-    e = launch_swiglu_tc_train(x_perm, offsets, w1, w3, w2, N, d, h, E, y, h_act, gu, status, s);
+  if (e == cudaSuccess && N > 0) {
+    if (dt == MOE_BF16)
+      e = launch_swiglu_tc_train(x_perm, offsets, w1, w3, w2, N, d, h, E, y, h_act, gu, status,
+                                 s);
+    else
+      e = launch_swiglu_simt_f32_train(
+          static_cast<const float*>(x_perm), offsets, static_cast<const float*>(w1),
+          static_cast<const float*>(w3), static_cast<const float*>(w2), N, d, h, E,
+          static_cast<float*>(y), static_cast<float*>(h_act), static_cast<float*>(gu), status, s);
+  }
   return cuda_status(e, "moe_grouped_swiglu_train");
 }
 
 size_t moe_grouped_swiglu_backward_workspace_size(int N, int d, int h, int E, moe_dtype_t dt) {
   (void)d;
   (void)E;
-  (void)dt;
   if (N < 0 || h < 1) return kStatusBytes;
-  return kStatusBytes + align_up(static_cast<size_t>(N) * 2 * h * 2, 256);
+  return kStatusBytes + align_up(static_cast<size_t>(N) * 2 * h * elt_bytes(dt), 256);
 }
 
 moe_status_t moe_grouped_swiglu_backward(const void* x_perm, const int32_t* offsets,
@@ -783,10 +863,6 @@ moe_status_t moe_grouped_swiglu_backward(const void* x_perm, const int32_t* offs
                                          void* dw1, void* dw3, void* dw2, void* ws,
                                          size_t ws_bytes, void* stream) {
   if (moe_status_t st = check_swiglu_shape(N, d, h, E, dt)) return st;
-  if (dt != MOE_BF16) {
-    set_last_error("moe_grouped_swiglu_backward: bf16 only");
-    return MOE_ERR_UNSUPPORTED;
-  }
   MOE_CHECK_ARG(offsets && w1 && w3 && w2 && dw1 && dw3 && dw2,
                 "offsets, w1, w3, w2, dw1, dw3, dw2 required");
   if (N > 0) {
@@ -810,10 +886,18 @@ moe_status_t moe_grouped_swiglu_backward(const void* x_perm, const int32_t* offs
   cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), s);
   if (e == cudaSuccess && N == 0) {
     // no rows: every weight gradient is zero
-    const size_t wbytes = static_cast<size_t>(E) * h * d * 2;
+    const size_t wbytes = static_cast<size_t>(E) * h * d * elt_bytes(dt);
     e = cudaMemsetAsync(dw1, 0, wbytes, s);
     if (e == cudaSuccess) e = cudaMemsetAsync(dw3, 0, wbytes, s);
     if (e == cudaSuccess) e = cudaMemsetAsync(dw2, 0, wbytes, s);
+  } else if (e == cudaSuccess && dt == MOE_F32) {
+    e = launch_swiglu_bwd_simt_f32(
+        static_cast<const float*>(x_perm), offsets, static_cast<const float*>(w1),
+        static_cast<const float*>(w3), static_cast<const float*>(w2),
+        static_cast<const float*>(h_act), static_cast<const float*>(gu),
+        static_cast<const float*>(dy), N, d, h, E, static_cast<float*>(dx_perm),
+        static_cast<float*>(dw1), static_cast<float*>(dw3), static_cast<float*>(dw2),
+        reinterpret_cast<float*>(static_cast<char*>(ws) + kStatusBytes), status, s);
   } else if (e == cudaSuccess) {
     e = launch_swiglu_bwd_tc(x_perm, offsets, w1, w3, w2, h_act, gu, dy, N, d, h, E, dx_perm, dw1,
                              dw3, dw2, static_cast<char*>(ws) + kStatusBytes, status, s);
@@ -863,9 +947,10 @@ moe_status_t moe_dispatch_backward(const void* dx_perm, const int32_t* dst_pos,
 // dw_router [splits, E, d]
 size_t moe_router_backward_workspace_size(int T, int d, int E) {
   if (T < 0 || E < 1 || d < 1) return kStatusBytes;
-  // status, gate segment offsets, dz in bf16, the gate's fp32 partials,
-  // then the expert counts of the load-balance gradient
-  return kStatusBytes + 256 + align_up(static_cast<size_t>(T) * E * 2, 256) +
+  // status, gate segment offsets, dz (bf16 for the tcgen05 gate products,
+  // fp32 for the fp32 ones), the gate's fp32 partials, then the expert
+  // counts of the load-balance gradient
+  return kStatusBytes + 256 + align_up(static_cast<size_t>(T) * E * 4, 256) +
          align_up(static_cast<size_t>(gate_splits(T, d, E)) * E * d * 4, 256) +
          align_up(static_cast<size_t>(E) * 4, 256);
 }
@@ -884,11 +969,9 @@ moe_status_t moe_router_backward(const float* logits, const int32_t* topk_idx,
   MOE_CHECK_ARG(o.score == MOE_SCORE_SOFTMAX || o.score == MOE_SCORE_SIGMOID, "bad score");
   MOE_CHECK_ARG(std::isfinite(o.route_scale) && o.route_scale != 0.0f, "bad route_scale");
   const bool gemm = dw_router || dx;
-  if (gemm) {
-    if (dt != MOE_BF16 || E % 8 != 0 || d % 64 != 0) {
-      set_last_error("router backward gate gradients need bf16, E %% 8 == 0 and d %% 64 == 0");
-      return MOE_ERR_UNSUPPORTED;
-    }
+  if (gemm && dt == MOE_BF16 && (E % 8 != 0 || d % 64 != 0)) {
+    set_last_error("bf16 router backward gate gradients need E %% 8 == 0 and d %% 64 == 0");
+    return MOE_ERR_UNSUPPORTED;
   }
   if (T > 0) {
     MOE_CHECK_ARG(logits && topk_idx && d_topk_w, "logits, topk_idx, d_topk_w required");
@@ -908,7 +991,7 @@ moe_status_t moe_router_backward(const float* logits, const int32_t* topk_idx,
   int32_t* off2 = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + kStatusBytes);
   void* dz16 = static_cast<char*>(ws) + kStatusBytes + 256;
   float* gpart = reinterpret_cast<float*>(static_cast<char*>(dz16) +
-                                          align_up(static_cast<size_t>(T) * E * 2, 256));
+                                          align_up(static_cast<size_t>(T) * E * 4, 256));
   int32_t* lbc = reinterpret_cast<int32_t*>(
       reinterpret_cast<char*>(gpart) +
       align_up(static_cast<size_t>(gate_splits(T, d, E)) * E * d * 4, 256));
@@ -916,7 +999,11 @@ moe_status_t moe_router_backward(const float* logits, const int32_t* topk_idx,
   MOE_CHECK_ARG(std::isfinite(o.aux_loss_coef), "aux_loss_coef must be finite");
   cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), s);
   if (e == cudaSuccess && T == 0 && dw_router)
-    e = cudaMemsetAsync(dw_router, 0, static_cast<size_t>(E) * d * 2, s);
+    e = cudaMemsetAsync(dw_router, 0, static_cast<size_t>(E) * d * elt_bytes(dt), s);
+  // fp32 gate products read dz in fp32: the caller's d_logits, else the
+  // workspace
+  const bool f32 = dt == MOE_F32;
+  float* dz32 = f32 && gemm && !d_logits ? static_cast<float*>(dz16) : d_logits;
   // the load-balance gradient needs the forward's expert counts: recounted
   // from topk_idx
   if (e == cudaSuccess && lb) e = cudaMemsetAsync(lbc, 0, static_cast<size_t>(E) * 4, s);
@@ -924,9 +1011,13 @@ moe_status_t moe_router_backward(const float* logits, const int32_t* topk_idx,
   if (e == cudaSuccess && T > 0)
     e = launch_router_backward(logits, topk_idx, d_topk_w, T, E, top_k,
                                o.score == MOE_SCORE_SIGMOID, o.renormalize, o.route_scale,
-                               d_logits, gemm ? dz16 : nullptr, s, lb ? lbc : nullptr,
+                               dz32, gemm && !f32 ? dz16 : nullptr, s, lb ? lbc : nullptr,
                                lb ? lb_grad_scale(o.aux_loss_coef, E, T, top_k) : 0.f);
-  if (e == cudaSuccess && T > 0 && gemm)
+  if (e == cudaSuccess && T > 0 && gemm && f32)
+    e = launch_gate_backward_f32(dz32, static_cast<const float*>(x),
+                                 static_cast<const float*>(w_router), T, d, E,
+                                 static_cast<float*>(dw_router), static_cast<float*>(dx), s);
+  else if (e == cudaSuccess && T > 0 && gemm)
     e = launch_gate_backward_tc(dz16, x, w_router, T, d, E, dw_router, dx, off2, gpart, status,
                                 s);
   return cuda_status(e, "moe_router_backward");

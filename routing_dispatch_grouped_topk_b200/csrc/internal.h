@@ -202,6 +202,24 @@ cudaError_t launch_swiglu_tc_gather(const void* x, int T, const int32_t* src_row
 cudaError_t launch_swiglu_tc_train(const void* x_perm, const int32_t* offsets, const void* w1,
                                    const void* w3, const void* w2, int N, int d, int h, int E,
                                    void* y, void* H, void* GU, int* status, cudaStream_t s);
+// Whether the bf16 grouped SwiGLU of N rows over E experts runs on the
+// CTA-pair kernel (segments averaging 64 rows or more).
+bool swiglu_tc_uses_pairs(int N, int E);
+// The grouped SwiGLU with the combine folded into GEMM2 (CTA-pair path only,
+// cudaErrorInvalidValue otherwise): out32 [T, d] fp32 (zero before the
+// call) += slot_w[s] * y[s] at row slot_tok[s] for every slot s; H [N, h]
+// is scratch.
+cudaError_t launch_swiglu_tc_combine(const void* x_perm, const int32_t* offsets, const void* w1,
+                                     const void* w3, const void* w2, int N, int d, int h, int E,
+                                     void* H, const int32_t* slot_tok, const float* slot_w,
+                                     int T, float* out32, int* status, cudaStream_t s);
+// slot_tok[dst_pos[t, j]] = t and slot_w[dst_pos[t, j]] = topk_w[t, j] (1
+// when topk_w is null) for every position inside [0, N); slot_tok must be
+// preset to -1.
+cudaError_t launch_slot_map(const int32_t* dst_pos, const float* topk_w, int T, int top_k, int N,
+                            int32_t* slot_tok, float* slot_w, cudaStream_t s);
+// out [n] bf16 = in [n] fp32, rounded to nearest even (n a multiple of 8).
+cudaError_t launch_f32_to_bf16(const float* in, size_t n, void* out, cudaStream_t s);
 // Backward of the grouped SwiGLU (bf16, tcgen05): dX [N, d], dW1/dW3 [E, h, d],
 // dW2 [E, d, h]; dGU [N, 2h] bf16 is scratch.
 cudaError_t launch_swiglu_bwd_tc(const void* x_perm, const int32_t* offsets, const void* w1,
@@ -213,6 +231,22 @@ cudaError_t launch_swiglu_simt_f32(const float* x_perm, const int32_t* offsets,
                                    const float* w1, const float* w3, const float* w2,
                                    const float* row_scale, int N, int d, int h, int E, float* y,
                                    float* H, int* status, cudaStream_t s);
+// fp32 training forward: also writes GU [N, 2h] fp32 (G | U), H is an output.
+cudaError_t launch_swiglu_simt_f32_train(const float* x_perm, const int32_t* offsets,
+                                         const float* w1, const float* w3, const float* w2,
+                                         int N, int d, int h, int E, float* y, float* H,
+                                         float* GU, int* status, cudaStream_t s);
+// fp32 backward of the grouped SwiGLU on CUDA cores; dGU [N, 2h] fp32 scratch.
+cudaError_t launch_swiglu_bwd_simt_f32(const float* x_perm, const int32_t* offsets,
+                                       const float* w1, const float* w3, const float* w2,
+                                       const float* H, const float* GU, const float* dY, int N,
+                                       int d, int h, int E, float* dX, float* dW1, float* dW3,
+                                       float* dW2, float* dGU, int* status, cudaStream_t s);
+// fp32 gate gradients: dw_router = dz^T x [E, d], dx = dz w_router [T, d]
+// (each optional) for dz [T, E] fp32.
+cudaError_t launch_gate_backward_f32(const float* dz, const float* x, const float* w_router,
+                                     int T, int d, int E, float* dw_router, float* dx,
+                                     cudaStream_t s);
 cudaError_t launch_swiglu_simt_f32_gather(const float* x, int x_rows, const int32_t* src_row,
                                           const int32_t* offsets, const float* w1,
                                           const float* w3, const float* w2,

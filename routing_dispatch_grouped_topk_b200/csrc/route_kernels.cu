@@ -949,6 +949,56 @@ cudaError_t launch_sum_partials_bf16(const float* part, int S, size_t n, void* o
   return cudaGetLastError();
 }
 
+// ------------------------------------------- folded combine: slot map, output
+// The inverse of dst_pos: the token and routing weight of every slot.
+__global__ void __launch_bounds__(256) slot_map_kernel(const int32_t* __restrict__ dst_pos,
+                                                       const float* __restrict__ topk_w,
+                                                       long long n, int top_k, int N,
+                                                       int32_t* __restrict__ slot_tok,
+                                                       float* __restrict__ slot_w) {
+  pdl_wait();
+  pdl_trigger();
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int s = dst_pos[i];
+    if (static_cast<unsigned>(s) >= static_cast<unsigned>(N)) continue;
+    slot_tok[s] = static_cast<int32_t>(i / top_k);
+    slot_w[s] = topk_w ? topk_w[i] : 1.0f;
+  }
+}
+
+cudaError_t launch_slot_map(const int32_t* dst_pos, const float* topk_w, int T, int top_k, int N,
+                            int32_t* slot_tok, float* slot_w, cudaStream_t s) {
+  const long long n = 1LL * T * top_k;
+  if (n == 0) return cudaSuccess;
+  const int blocks = static_cast<int>(std::min<long long>((n + 255) / 256, 8LL * num_sms()));
+  launch_k(slot_map_kernel, dim3(blocks), dim3(256), 0, s, dst_pos, topk_w, n, top_k, N,
+           slot_tok, slot_w);
+  return cudaGetLastError();
+}
+
+// out [n] bf16 = in [n] fp32 (RNE), eight values per thread and step.
+__global__ void __launch_bounds__(256) f32_to_bf16_kernel(const float4* __restrict__ in,
+                                                          size_t n8, uint4* __restrict__ out) {
+  pdl_wait();
+  pdl_trigger();
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n8;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const float4 a = in[2 * i], b = in[2 * i + 1];
+    out[i] = make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y),
+                        pack_bf16x2(b.z, b.w));
+  }
+}
+
+cudaError_t launch_f32_to_bf16(const float* in, size_t n, void* out, cudaStream_t s) {
+  const size_t n8 = n / 8;
+  if (n8 == 0) return cudaSuccess;
+  const int blocks = static_cast<int>(std::min<size_t>((n8 + 255) / 256, 8 * num_sms()));
+  launch_k(f32_to_bf16_kernel, dim3(blocks), dim3(256), 0, s, reinterpret_cast<const float4*>(in),
+           n8, static_cast<uint4*>(out));
+  return cudaGetLastError();
+}
+
 // ------------------------------------------------------- fp32 / SIMT router
 template <typename TX>
 __device__ __forceinline__ float to_f(TX v);

@@ -92,6 +92,13 @@ struct Args {
   int split;                 // weight gradient: rows of each expert that go to `out`
   int Ma;                    // weight gradient: output rows per expert
   float* out_f32;            // weight gradient: fp32 output [E, Ma, n_out] instead of bf16
+  // GEMM2 with the combine folded in (CTA-pair kernel): output row s is
+  // scaled by comb_w[s] and added into comb_out[comb_tok[s]] with fp32
+  // reductions instead of being stored
+  float* comb_out;           // [comb_T, n_out] fp32, zero before the launch
+  const int32_t* comb_tok;   // [M] token of every slot (outside [0, comb_T): skipped)
+  const float* comb_w;       // [M] routing weight of every slot
+  int comb_T;
 };
 
 __host__ __device__ constexpr int stages_for(int bn) {
@@ -724,50 +731,35 @@ struct DownStagedPolicy : DownPolicy {
   }
 };
 
-// ------------------------------------------- hybrid CTA-pair tile schedule
+// ------------------------------------------------------ CTA-pair tile schedule
 // The forward GEMMs on CTA pairs (cta_group::2).  Every expert segment is
 // covered by 256-row pair tiles: CTA rank r owns rows [256 mt + 128 r, +128)
 // (its A operand and its accumulator lanes) and loads half of the B tile,
 // so a pair moves 64 KB per K block for the work that two single-CTA
-// 128 x 256 tiles do with 96 KB.  In GEMM2 the last m-tile of a segment,
-// when it holds at most 128 rows, is a swap-AB pair tile instead: the w2 rows
-// are the M = 256 operand (128 per SM) and the tile's tokens the N operand
-// (the rows rounded up to 32; each SM loads its N/2 token rows in 16-row
-// boxes), so a short tail costs in proportion to its rows.  GEMM1 keeps
-// normal pair tiles for its tails: its swap tiles needed the hidden units' G
-// and U, which land in different TMEM lane quadrants, to meet through 33 KB
-// of shared memory, and the sixth pipeline stage that memory buys measured
-// faster on B200 than the cheaper tails.
+// 128 x 256 tiles do with 96 KB.  A segment's last tile may be mostly
+// padding; it is still a plain pair tile.  (Swap-AB pair tiles for tails of
+// at most 128 rows -- weights as the M = 256 operand, the tail's tokens as
+// N -- were built for both GEMMs and measured slower on B200: with them in
+// GEMM2, GEMM1 + GEMM2 took 7 % longer at the Qwen3-30B-A3B sizes, 10 % on
+// the Zipf layer and 19 % at the gpt-oss EP8 sizes (in both GEMMs: 5 %, 12 %
+// and 21 %).  A swap tile streams the whole weight tile for
+// a fraction of the MMA work, its small-N MMAs do not run proportionally
+// faster, and GEMM2's tail, run right after its normal tile, re-read the
+// weight tile from DRAM.)
 //   GEMM1: rank 0 loads w1 rows [e h + n0, +128), rank 1 the w3 rows of the
 //     same hidden units; accumulator columns 0..127 hold G and 128..255 U.
-//   GEMM2: rank r loads w2 rows [e d + n0 + 128 r, +128), as the B half of a
-//     normal tile or as the A operand of a swap tile.
-constexpr int kPairSwapMaxRows = 128;
-constexpr int kTokBoxRows = 16;          // token rows per TMA box of a swap tile
-
-// Work units, taken round-robin by the pairs: the m-tiles of an (expert,
-// n-tile) in order, each its own unit, except that a segment's tail tile
-// joins the normal tile before it (one unit of two tiles run back to back by
-// the same pair, so the tail finds its weight tile in L2).  Units ordered
-// (expert, n-tile, m-tile) keep the tiles that share weight tiles together.
-// (Round-robin over single tiles gave, at ~256-row segments, some pairs a
-// third more work than the mean: normal and tail tiles alternate with the
-// segments and the even number of pairs keeps each pair on one kind;
-// putting every tail after every normal tile balanced it but re-read the
-// weights of the tails from DRAM.)  sched layout: [0] units, [1] n-tiles per
-// expert, [8 .. 8+E] offsets, [8+E+1 .. 8+2E+1] cumulative units per expert.
+//   GEMM2: rank r loads w2 rows [e d + n0 + 128 r, +128).
+//
+// Tiles, taken round-robin by the pairs, are ordered (expert, n-tile,
+// m-tile), so the tiles that run at the same time share weight tiles and
+// token rows in L2.  (Handing tiles out from a global counter instead was
+// measured slower: claimed tiles stay in lock-step, and the pairs working on
+// one expert then read the same lines at the same moment.)  sched layout:
+// [0] tiles, [1] n-tiles per expert, [8 .. 8+E] offsets, [8+E+1 .. 8+2E+1]
+// cumulative tiles per expert.
 template <int NCOLS, int NUM_B_, bool UP_>
-struct HybridPolicy : GroupedSched<256, NUM_B_, NCOLS, 256> {
-  using Base = GroupedSched<256, NUM_B_, NCOLS, 256>;
+struct PairSched : GroupedSched<256, NUM_B_, NCOLS, 256> {
   static constexpr bool UP = UP_;
-
-  // m-tiles of a segment of cnt rows, whether its last one is a tail tile,
-  // and its units per n-tile
-  static __device__ __forceinline__ void seg_tiles(int cnt, int& mt, int& tail, int& mu) {
-    mt = cdiv(max(cnt, 0), 256);
-    tail = (!UP && mt > 0 && cnt - (mt - 1) * 256 <= kPairSwapMaxRows) ? 1 : 0;
-    mu = (tail && mt >= 2) ? mt - 1 : mt;
-  }
 
   static __device__ void prologue(const Args& a, int* sched) {
     const int E = a.E;
@@ -784,9 +776,7 @@ struct HybridPolicy : GroupedSched<256, NUM_B_, NCOLS, 256> {
       for (int e = e0; e < e1; ++e) {
         const int cnt = off[e + 1] - off[e];
         bad |= cnt < 0;
-        int mt, tail, mu;
-        seg_tiles(cnt, mt, tail, mu);
-        local += mu * nt;
+        local += cdiv(max(cnt, 0), 256) * nt;
       }
       int incl = local;
 #pragma unroll
@@ -797,9 +787,7 @@ struct HybridPolicy : GroupedSched<256, NUM_B_, NCOLS, 256> {
       int run = incl - local;
       for (int e = e0; e < e1; ++e) {
         cum[e] = run;
-        int mt, tail, mu;
-        seg_tiles(off[e + 1] - off[e], mt, tail, mu);
-        run += mu * nt;
+        run += cdiv(max(off[e + 1] - off[e], 0), 256) * nt;
       }
       bad = __any_sync(0xffffffffu, bad);
       const int total = __shfl_sync(0xffffffffu, incl, 31);
@@ -812,100 +800,79 @@ struct HybridPolicy : GroupedSched<256, NUM_B_, NCOLS, 256> {
       }
     }
   }
-  static __device__ int num_units(const Args&, const int* sched) { return sched[0]; }
+  static __device__ int num_tiles(const Args&, const int* sched) { return sched[0]; }
 
-  // unit -> expert e, n-tile, first m-tile; *ntiles = 1 or 2 (normal + tail)
-  static __device__ void locate_unit(const Args& a, const int* sched, int unit, int& e, int& nt,
-                                     int& mt, int& ntiles) {
+  // tile -> its half for CTA `rank` of the pair
+  static __device__ TileInfo tile_info(const Args& a, const int* sched, int tile, int rank) {
     const int E = a.E;
     const int* off = sched + 8;
     const int* cum = off + E + 1;
     int lo = 0, hi = E - 1;
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
-      if (cum[mid] <= unit) lo = mid; else hi = mid - 1;
+      if (cum[mid] <= tile) lo = mid; else hi = mid - 1;
     }
-    e = lo;
-    int mtt, tail, mu;
-    seg_tiles(off[e + 1] - off[e], mtt, tail, mu);
-    const int local = unit - cum[e];
-    nt = local / mu;
-    mt = local - nt * mu;
-    ntiles = (tail && mtt >= 2 && mt == mu - 1) ? 2 : 1;
-  }
-  static __device__ int unit_tiles(const Args& a, const int* sched, int unit) {
-    int e, nt, mt, n;
-    locate_unit(a, sched, unit, e, nt, mt, n);
-    return n;
-  }
-
-  // sub-tile `sub` (0 or 1) of a unit, for CTA `rank` of the pair
-  static __device__ TileInfo tile_info(const Args& a, const int* sched, int unit, int sub,
-                                       int rank) {
-    int e, nt, mt0, n;
-    locate_unit(a, sched, unit, e, nt, mt0, n);
-    const int* off = sched + 8;
+    const int e = lo;
     const int seg0 = off[e], cnt = off[e + 1] - seg0;
-    const int mt = mt0 + sub;
-    const int rows = cnt - mt * 256;        // rows from this m-tile to the segment's end
+    const int mtiles = cdiv(cnt, 256);
+    const int local = tile - cum[e];
+    const int nt = local / mtiles, mt = local - nt * mtiles;
+    const int r0 = mt * 256 + rank * 128;
     TileInfo t;
     t.n0 = nt * NCOLS;
     t.kb0 = 0;
     t.kb1 = cdiv(a.K, BK);
     t.m0 = 0;
-    if (!UP && rows <= kPairSwapMaxRows) {
-      t.a_row = seg0 + mt * 256;            // the tile's first token
-      t.m_valid = rows;                     // its tokens
-      t.swap_np = (rows + 31) & ~31;        // MMA N of the pair
-      t.b_row = e * a.n_out + t.n0 + 128 * rank;
-    } else {
-      const int r0 = mt * 256 + rank * 128;
-      t.a_row = seg0 + r0;
-      t.m_valid = max(0, min(BM, cnt - r0));
-      t.swap_np = 0;
-      t.b_row = UP ? e * a.n_out + t.n0 : e * a.n_out + t.n0 + 128 * rank;
-    }
+    t.swap_np = 0;
+    t.a_row = seg0 + r0;
+    t.m_valid = max(0, min(BM, cnt - r0));
+    t.b_row = UP ? e * a.n_out + t.n0 : e * a.n_out + t.n0 + 128 * rank;
     return t;
   }
 };
 
-struct UpHybridPolicy : HybridPolicy<128, 2, true> {
+struct UpPairPolicy : PairSched<128, 2, true> {
   static __device__ void epilogue_staged(const Args& a, int* s, const TileInfo& ti,
                                          uint32_t taddr, int row, uint8_t* stg, int c0, int c1) {
     UpStagedPolicy::epilogue_staged(a, s, ti, taddr, row, stg, c0, c1);
   }
 };
 
-struct DownHybridPolicy : HybridPolicy<256, 1, false> {
-  // Swap tile: lane = output feature n0 + 128 rank + row, one column per
-  // token; a warp writes 32 features (64 contiguous bytes) of one token row
-  // per instruction.  Tokens in chunks of 16, split between the two warps of
-  // a quadrant by `half`.
-  static __device__ void epilogue_swap_pair(const Args& a, const TileInfo& ti, uint32_t taddr,
-                                            int q, int half, int rank) {
-    const int lane = threadIdx.x & 31;
-    const int f = ti.n0 + 128 * rank + q * 32 + lane;
-    const bool fvalid = f < a.n_out;
-    const int ntok = ti.m_valid;
-    for (int t0 = 16 * half; t0 < ntok; t0 += 32) {
-      uint32_t v[16];
-      tmem_ld16(taddr + t0, v);
-      tmem_ld_wait();
-      if (!fvalid) continue;
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int t = t0 + i;
-        if (t < ntok) {
-          const size_t r = static_cast<size_t>(ti.a_row + t);
-          const float sc = a.row_scale ? a.row_scale[r] : 1.0f;
-          a.out[r * a.n_out + f] = __float2bfloat16_rn(__uint_as_float(v[i]) * sc);
-        }
-      }
-    }
-  }
+struct DownPairPolicy : PairSched<256, 1, false> {
   static __device__ void epilogue_staged(const Args& a, int* s, const TileInfo& ti,
                                          uint32_t taddr, int row, uint8_t* stg, int c0, int c1) {
+    if (a.comb_out) {
+      combine_rows(a, ti, taddr, row, c0, c1);
+      return;
+    }
     DownStagedPolicy::epilogue_staged(a, s, ti, taddr, row, stg, c0, c1);
+  }
+  // With the combine folded in: the thread of row s adds its 32 columns of a
+  // chunk, times the slot's weight, into the token's fp32 row as eight
+  // 16-byte reductions.
+  static __device__ void combine_rows(const Args& a, const TileInfo& ti, uint32_t taddr, int row,
+                                      int c0, int c1) {
+    int tok = -1;
+    float w = 0.f;
+    if (row < ti.m_valid) {
+      const size_t r = static_cast<size_t>(ti.a_row + row);
+      tok = a.comb_tok[r];
+      w = a.comb_w[r];
+    }
+    const bool live = static_cast<unsigned>(tok) < static_cast<unsigned>(a.comb_T);
+#pragma unroll 1
+    for (int c = c0; c < c1; ++c) {
+      uint32_t r[32];
+      tmem_ld32(taddr + c * 32, r);
+      tmem_ld_wait();
+      if (ti.n0 + c * 32 >= a.n_out || !live) continue;
+      float* dst = a.comb_out + static_cast<size_t>(tok) * a.n_out + ti.n0 + c * 32;
+#pragma unroll
+      for (int g = 0; g < 8; ++g)
+        red_add_f32x4(dst + 4 * g, __uint_as_float(r[4 * g]) * w,
+                      __uint_as_float(r[4 * g + 1]) * w, __uint_as_float(r[4 * g + 2]) * w,
+                      __uint_as_float(r[4 * g + 3]) * w);
+    }
   }
 };
 
@@ -1509,8 +1476,8 @@ __global__ void __launch_bounds__(P::THREADS, 1)
 // the leader's "tmem empty" barrier.  Roles per CTA (320 threads): warp 0
 // TMA producer, warp 1 TMEM owner and (leader) MMA issuer, warps 2..9 the
 // epilogue (two per TMEM lane quadrant, each taking half of the columns).
-// Maps: tmA / tmB0 / tmB1 the normal tiles' operands (128-row boxes; tmB1
-// only for GEMM1), tmT the tokens of GEMM2's swap tiles in 16-row boxes.
+// Maps: tmA the token rows, tmB0 / tmB1 the weight halves (128-row boxes;
+// tmB1 only for GEMM1).
 template <class P>
 struct PairLayout {
   static constexpr int kBHalfBytes = 128 * BK * 2;                  // 16 KB
@@ -1533,8 +1500,7 @@ template <class P>
 __global__ void __launch_bounds__(PairLayout<P>::kThreads, 1)
     tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB0,
-                        const __grid_constant__ CUtensorMap tmB1,
-                        const __grid_constant__ CUtensorMap tmT, const Args args) {
+                        const __grid_constant__ CUtensorMap tmB1, const Args args) {
   using L = PairLayout<P>;
   constexpr int STAGES = L::kStages;
   constexpr uint32_t IDESC = idesc_bf16_f32(256, 256);
@@ -1574,10 +1540,7 @@ __global__ void __launch_bounds__(PairLayout<P>::kThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB0);
-    if (P::UP)
-      tma_prefetch_desc(&tmB1);
-    else
-      tma_prefetch_desc(&tmT);
+    if (P::UP) tma_prefetch_desc(&tmB1);
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, L::kTmemCols);
@@ -1590,7 +1553,7 @@ __global__ void __launch_bounds__(PairLayout<P>::kThreads, 1)
   cluster_sync_all();   // barriers of both CTAs initialised before any remote arrive
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int total = P::num_units(args, sched);
+  const int total = P::num_tiles(args, sched);
   const int pair = blockIdx.x >> 1;
   const int npairs = gridDim.x >> 1;
 
@@ -1603,13 +1566,8 @@ __global__ void __launch_bounds__(PairLayout<P>::kThreads, 1)
       uint32_t phase = 0;
       int issued = 0;
       bool ok = true;
-      for (int unit = pair; unit < total && ok; unit += npairs)
-      for (int sub = 0, nsub = P::unit_tiles(args, sched, unit); sub < nsub && ok; ++sub) {
-        const TileInfo ti = P::tile_info(args, sched, unit, sub, rank);
-        const int half_n = ti.swap_np / 2;                    // token rows of this CTA
-        const int nbox = (half_n + kTokBoxRows - 1) / kTokBoxRows;
-        const uint32_t cta_bytes =
-            ti.swap_np ? kATileBytes + nbox * kTokBoxRows * BK * 2 : L::kStageBytes;
+      for (int tile = pair; tile < total && ok; tile += npairs) {
+        const TileInfo ti = P::tile_info(args, sched, tile, rank);
         for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
           if (!mbar_wait(empty + stage, phase ^ 1u, abort_flag, args.status)) {
             ok = false;
@@ -1618,17 +1576,9 @@ __global__ void __launch_bounds__(PairLayout<P>::kThreads, 1)
           uint8_t* sa = tiles + stage * L::kStageBytes;
           uint8_t* sb = sa + kATileBytes;
           const uint32_t bar = cluster_map(full + stage, 0);
-          if (leader) mbar_arrive_expect_tx(full + stage, 2 * cta_bytes);
-          if (!ti.swap_np) {
-            tma_load_2d_pair(sa, &tmA, bar, kb * BK, ti.a_row, pol);
-            tma_load_2d_pair(sb, tb, bar, kb * BK, ti.b_row, pol);
-          } else {
-            // A region: this CTA's 128 w2 rows; B region: its N/2 tokens
-            tma_load_2d_pair(sa, &tmB0, bar, kb * BK, ti.b_row, pol);
-            for (int i = 0; i < nbox; ++i)
-              tma_load_2d_pair(sb + i * kTokBoxRows * BK * 2, &tmT, bar, kb * BK,
-                               ti.a_row + rank * half_n + i * kTokBoxRows, pol);
-          }
+          if (leader) mbar_arrive_expect_tx(full + stage, 2 * L::kStageBytes);
+          tma_load_2d_pair(sa, &tmA, bar, kb * BK, ti.a_row, pol);
+          tma_load_2d_pair(sb, tb, bar, kb * BK, ti.b_row, pol);
           ++issued;
           if (++stage == STAGES) {
             stage = 0;
@@ -1657,8 +1607,7 @@ __global__ void __launch_bounds__(PairLayout<P>::kThreads, 1)
       uint32_t phase = 0;
       int it = 0;
       bool ok = true;
-      for (int unit = pair; unit < total && ok; unit += npairs)
-      for (int sub = 0, nsub = P::unit_tiles(args, sched, unit); sub < nsub && ok; ++sub, ++it) {
+      for (int tile = pair; tile < total && ok; tile += npairs, ++it) {
         const int acc = it & 1;
         const uint32_t aph = (it >> 1) & 1;
         if (!mbar_wait_cluster(tempty + acc, aph ^ 1u, abort_flag, args.status)) {
@@ -1667,8 +1616,7 @@ __global__ void __launch_bounds__(PairLayout<P>::kThreads, 1)
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * 256);
-        const TileInfo ti = P::tile_info(args, sched, unit, sub, 0);
-        const uint32_t idesc = ti.swap_np ? idesc_bf16_f32(256, ti.swap_np) : IDESC;
+        const TileInfo ti = P::tile_info(args, sched, tile, 0);
         for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
           if (!mbar_wait(full + stage, phase, abort_flag, args.status)) {
             ok = false;
@@ -1680,7 +1628,7 @@ __global__ void __launch_bounds__(PairLayout<P>::kThreads, 1)
           const uint64_t bd = sw128_kmajor_desc(sa + kATileBytes);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
-            tc_mma_bf16_pair(d_tmem, ad + 2u * kk, bd + 2u * kk, idesc,
+            tc_mma_bf16_pair(d_tmem, ad + 2u * kk, bd + 2u * kk, IDESC,
                              (kb != ti.kb0 || kk != 0) ? 1u : 0u);
           tc_commit_pair_mc(empty + stage, 0x3);
           if (++stage == STAGES) {
@@ -1706,8 +1654,7 @@ __global__ void __launch_bounds__(PairLayout<P>::kThreads, 1)
     tempty_leader[1] = cluster_map(tempty + 1, 0);
     int it = 0;
     bool run = true;
-    for (int unit = pair; unit < total && run; unit += npairs)
-    for (int sub = 0, nsub = P::unit_tiles(args, sched, unit); sub < nsub; ++sub, ++it) {
+    for (int tile = pair; tile < total && run; tile += npairs, ++it) {
       const int acc = it & 1;
       const uint32_t aph = (it >> 1) & 1;
       int ok = 1;
@@ -1718,15 +1665,11 @@ __global__ void __launch_bounds__(PairLayout<P>::kThreads, 1)
         break;
       }
       tc_fence_after();
-      const TileInfo ti = P::tile_info(args, sched, unit, sub, rank);
+      const TileInfo ti = P::tile_info(args, sched, tile, rank);
       const uint32_t taddr =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * 256);
-      if constexpr (!P::UP) {
-        if (ti.swap_np) P::epilogue_swap_pair(args, ti, taddr, q, half, rank);
-      }
-      if (!ti.swap_np)
-        P::epilogue_staged(args, sched, ti, taddr, row, epi + (warp - 2) * 2048, 4 * half,
-                           4 * half + 4);
+      P::epilogue_staged(args, sched, ti, taddr, row, epi + (warp - 2) * 2048, 4 * half,
+                         4 * half + 4);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tempty_leader[acc]);
@@ -1800,7 +1743,7 @@ cudaError_t launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMa
 // Launch of the CTA-pair kernel: clusters of 2 CTAs, an even grid.
 template <class P>
 cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
-                        const CUtensorMap& t, const Args& args, int pairs, cudaStream_t s) {
+                        const Args& args, int pairs, cudaStream_t s) {
   using L = PairLayout<P>;
   static int configured[64] = {0};
   int dev = 0;
@@ -1826,7 +1769,7 @@ cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUten
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, tc_gemm_pair_kernel<P>, a, b0, b1, t, args);
+  return cudaLaunchKernelEx(&cfg, tc_gemm_pair_kernel<P>, a, b0, b1, args);
 }
 
 }  // namespace tc
@@ -1870,11 +1813,19 @@ cudaError_t launch_router_tc(const void* x, const void* w_router, int T, int d, 
 
 // Grouped SwiGLU with GEMM1's A operand gathered from x [T, d] through
 // src_row (no expert-major copy of the tokens in memory).
+// Folded combine of GEMM2 (CTA-pair path only): see Args::comb_out.
+struct FoldedCombine {
+  float* out;           // [T, d] fp32, zero before the call
+  const int32_t* tok;   // [N]
+  const float* w;       // [N]
+  int T;
+};
+
 static cudaError_t swiglu_tc_impl(const void* a_src, int a_rows, const int32_t* src_row,
                                   const int32_t* offsets, const void* w1, const void* w3,
                                   const void* w2, const float* row_scale, int N, int d, int h,
                                   int E, void* y, void* H, int* status, cudaStream_t s,
-                                  void* gu = nullptr);
+                                  void* gu = nullptr, const FoldedCombine* fold = nullptr);
 
 cudaError_t launch_swiglu_tc(const void* x_perm, const int32_t* offsets, const void* w1,
                              const void* w3, const void* w2, const float* row_scale, int N,
@@ -1892,11 +1843,23 @@ cudaError_t launch_swiglu_tc_gather(const void* x, int T, const int32_t* src_row
                         s);
 }
 
+bool swiglu_tc_uses_pairs(int N, int E) { return N >= 64LL * E; }
+
+cudaError_t launch_swiglu_tc_combine(const void* x_perm, const int32_t* offsets, const void* w1,
+                                     const void* w3, const void* w2, int N, int d, int h, int E,
+                                     void* H, const int32_t* slot_tok, const float* slot_w,
+                                     int T, float* out32, int* status, cudaStream_t s) {
+  if (!swiglu_tc_uses_pairs(N, E)) return cudaErrorInvalidValue;
+  const FoldedCombine fold{out32, slot_tok, slot_w, T};
+  return swiglu_tc_impl(x_perm, N, nullptr, offsets, w1, w3, w2, nullptr, N, d, h, E, nullptr,
+                        H, status, s, nullptr, &fold);
+}
+
 static cudaError_t swiglu_tc_impl(const void* a_src, int a_rows, const int32_t* src_row,
                                   const int32_t* offsets, const void* w1, const void* w3,
                                   const void* w2, const float* row_scale, int N, int d, int h,
                                   int E, void* y, void* H, int* status, cudaStream_t s,
-                                  void* gu) {
+                                  void* gu, const FoldedCombine* fold) {
   using namespace tc;
   CUtensorMap tx, t1, t3, th, t2;
   const bool gather = src_row != nullptr;
@@ -1904,11 +1867,11 @@ static cudaError_t swiglu_tc_impl(const void* a_src, int a_rows, const int32_t* 
   if (!make_tmap(&t1, w1, d, static_cast<uint64_t>(E) * h, 128)) return cudaErrorInvalidValue;
   if (!make_tmap(&t3, w3, d, static_cast<uint64_t>(E) * h, 128)) return cudaErrorInvalidValue;
   if (!make_tmap(&th, H, h, N, BM)) return cudaErrorInvalidValue;
-  // The CTA-pair kernel (hybrid schedule: 256-row pair tiles, swap-AB pair
-  // tiles for segment tails of at most 128 rows) serves every layer whose
+  // The CTA-pair kernel (256-row pair tiles) serves every layer whose
   // segments average 64 rows or more; shorter segments (decode) stay on the
   // single-CTA kernel, whose swap-AB tiles stream each weight tile once.
-  const bool pairs = !gather && N >= 64LL * E;
+  const bool pairs = !gather && swiglu_tc_uses_pairs(N, E);
+  if (fold && !pairs) return cudaErrorInvalidValue;
   if (!make_tmap(&t2, w2, h, static_cast<uint64_t>(E) * d, pairs ? 128 : 256))
     return cudaErrorInvalidValue;
   const int max_mt = cdiv(N, BM) + E;   // upper bound on m-tiles over all segments
@@ -1926,19 +1889,23 @@ static cudaError_t swiglu_tc_impl(const void* a_src, int a_rows, const int32_t* 
   a.gather_src = a_src;
   a.gu_out = static_cast<__nv_bfloat16*>(gu);
   if (pairs) {
-    CUtensorMap ths;
-    if (!make_tmap(&ths, H, h, N, kTokBoxRows)) return cudaErrorInvalidValue;
     const long long max_pt = cdiv(N, 256) + E;   // upper bound on pair tiles per n-tile
     int np = static_cast<int>(std::min<long long>(num_sms() / 2, max_pt * cdiv(h, 128)));
-    cudaError_t e = launch_pair<UpHybridPolicy>(tx, t1, t3, tx, a, np, s);
+    cudaError_t e = launch_pair<UpPairPolicy>(tx, t1, t3, a, np, s);
     if (e != cudaSuccess) return e;
     a.K = h;
     a.n_out = d;
     a.out = static_cast<__nv_bfloat16*>(y);
     a.gu_out = nullptr;
     a.row_scale = row_scale;
+    if (fold) {
+      a.comb_out = fold->out;
+      a.comb_tok = fold->tok;
+      a.comb_w = fold->w;
+      a.comb_T = fold->T;
+    }
     np = static_cast<int>(std::min<long long>(num_sms() / 2, max_pt * cdiv(d, 256)));
-    return launch_pair<DownHybridPolicy>(th, t2, t2, ths, a, np, s);
+    return launch_pair<DownPairPolicy>(th, t2, t2, a, np, s);
   }
   int grid = static_cast<int>(std::min<long long>(num_sms(), 1LL * max_mt * cdiv(h, 128)));
   cudaError_t e = gather ? launch<UpGatherPolicy>(tx, t1, t3, a, grid, s)

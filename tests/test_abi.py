@@ -131,6 +131,29 @@ def test_grouped_swiglu_shape_rules(L):
     assert L.moe_grouped_swiglu(p, p, p, p, p, None, 10, 128, 128, 4, 1, p, p, 16, None) == 4
 
 
+def test_grouped_swiglu_combine_rules(L):
+    """The folded combine runs only on the bf16 CTA-pair path (segments
+    averaging >= 64 rows); every rule is checked before any launch."""
+    p = ctypes.c_void_p(256)
+    big = 1 << 30
+    ws = L.moe_grouped_swiglu_combine_workspace_size(512, 4, 128, 128, 8, 1)
+    assert ws >= 256 + 512 * 4 * 128 * 2 + 512 * 128 * 4
+    # fp32 layers, decode-sized segments (N = 16 < 64 E), d not a multiple of 64
+    assert L.moe_grouped_swiglu_combine(p, p, p, p, p, p, None, 512, 4, 128, 128, 8, 0, p, p,
+                                        big, None) == 2
+    assert L.moe_grouped_swiglu_combine(p, p, p, p, p, p, None, 4, 4, 128, 128, 8, 1, p, p, big,
+                                        None) == 2
+    assert L.moe_grouped_swiglu_combine(p, p, p, p, p, p, None, 512, 4, 96, 128, 8, 1, p, p, big,
+                                        None) == 2
+    # bad top_k, missing dst_pos, workspace too small
+    assert L.moe_grouped_swiglu_combine(p, p, p, p, p, p, None, 512, 0, 128, 128, 8, 1, p, p, big,
+                                        None) == 1
+    assert L.moe_grouped_swiglu_combine(p, p, p, p, p, None, None, 512, 4, 128, 128, 8, 1, p, p,
+                                        big, None) == 1
+    assert L.moe_grouped_swiglu_combine(p, p, p, p, p, p, None, 512, 4, 128, 128, 8, 1, p, p, 16,
+                                        None) == 4
+
+
 def test_dispatch_and_regroup_argument_rules(L):
     p = ctypes.c_void_p(256)
     # R must divide E
@@ -250,15 +273,14 @@ def test_training_entry_points_check_their_arguments(L):
 
 
 def test_router_backward_gate_rules(L):
-    """The gate's gradients need bf16, E % 8 == 0 and d % 64 == 0 (the
-    epilogue writes 32-column chunks); d logits alone have no such rule."""
+    """The bf16 gate gradients need E % 8 == 0 and d % 64 == 0 (the tcgen05
+    epilogue writes 32-column chunks); the fp32 ones (CUDA cores) and d
+    logits alone have no such rule (those run on the GPU tests)."""
     p = ctypes.c_void_p(256)
     big = 1 << 30
     assert L.moe_router_backward(p, p, p, p, p, 4, 96, 8, 2, None, 1, None, p, None, p, big,
                                  None) == 2
     assert L.moe_router_backward(p, p, p, p, p, 4, 64, 12, 2, None, 1, None, p, None, p, big,
-                                 None) == 2
-    assert L.moe_router_backward(p, p, p, p, p, 4, 64, 8, 2, None, 0, None, p, None, p, big,
                                  None) == 2
     assert L.moe_router_backward(p, p, p, p, p, 4, 96, 12, 2, None, 0, p, None, None, p, 16,
                                  None) == 4

@@ -359,9 +359,8 @@ def test_grouped_swiglu_gather_full_size_sampled(M, cfg):
 
 
 @pytest.mark.parametrize("counts,d,h", [
-    # 256-row pair tiles, tails of at most 128 rows (swap-AB pair tiles) and
-    # of more (a half-empty pair tile), empty experts, h and d that leave
-    # partial n-tiles
+    # full 256-row pair tiles, short and long tails (pair tiles mostly or
+    # half padding), empty experts, h and d that leave partial n-tiles
     ([256, 128, 129, 1, 0, 31, 32, 33, 384, 511], 192, 320),
     ([600, 200, 90], 320, 448),
 ])
