@@ -275,8 +275,20 @@ def run_reference(args, ws, rank):
 # kernel: gate GEMM, top-k, dispatch histogram), dispatch (column scan,
 # scatter), regroup on the EP layout (one kernel), grouped SwiGLU (GEMM1,
 # GEMM2), combine
+def grouped_gemm_launches(cfg) -> int:
+    """Launches of the grouped SwiGLU: GEMM1 and GEMM2, one each, plus a
+    single-CTA launch over the segments' short last blocks for each GEMM that
+    runs on CTA pairs (bf16, segments averaging >= 64 rows) with a reduction
+    of >= 2560 (d for GEMM1, h for GEMM2)."""
+    if cfg.dtype != "bf16" or cfg.N < 64 * cfg.E:
+        return 2
+    return 2 + (cfg.d >= 2560) + (cfg.h >= 2560)
+
+
 def forward_launches(cfg) -> int:
-    return 1 + 2 + (1 if cfg.ep_ranks > 1 else 0) + 2 + 1
+    # router (its kernel also writes the dispatch histogram), dispatch column
+    # scan and scatter, [regroup], the grouped SwiGLU, combine
+    return 1 + 2 + (1 if cfg.ep_ranks > 1 else 0) + grouped_gemm_launches(cfg) + 1
 
 
 class Layer:
@@ -368,8 +380,9 @@ class Layer:
 
 
 def timed_folded(layer, stream, flush, steps):
-    """CUDA-event times (ms) of moe_grouped_swiglu_combine (the combine
-    folded into GEMM2) on the layer's routed rows, L2 flushed between calls;
+    """CUDA-event times (ms) of moe_grouped_swiglu_combine (the combine folded
+    into GEMM2) and of the unfused moe_grouped_swiglu + moe_combine on the
+    layer's routed rows, alternating in blocks, L2 flushed between calls;
     None where the folded path does not apply (fp32, decode-sized segments).
     Its dst_pos addresses the expert-major rows the experts read (through
     the regroup's inverse permutation under simulated EP), composed once
@@ -379,50 +392,42 @@ def timed_folded(layer, stream, flush, steps):
         return None
     R = c.ep_ranks
     xe, off = (layer.x_em, layer.oem) if R > 1 else (layer.x_perm, layer.offsets)
+    rmap = layer.pinv if R > 1 else None
     dst = layer.pinv[layer.dst_pos.long()].int() if R > 1 else layer.dst_pos
     ws = torch.empty(M.lib().moe_grouped_swiglu_combine_workspace_size(c.T, c.top_k, c.d, c.h,
                                                                        c.E, layer.dt),
                      dtype=torch.uint8, device=layer.dev)
     out = torch.empty_like(layer.out)
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(steps + 2)]
-    torch.cuda.synchronize()
-    for a_ev, b_ev in ev:
-        a_ev.record(stream)
+
+    def folded():
         M.moe_grouped_swiglu_combine(xe, off, layer.w1, layer.w3, layer.w2, dst, layer.w, c.T,
                                      c.top_k, c.d, c.h, c.E, layer.dt, out, ws)
-        b_ev.record(stream)
-        flush.zero_()
-    torch.cuda.synchronize()
-    # the folded output against the staged step's (rounding differs: y is
-    # not rounded to bf16 on the folded path)
+
+    def unfused():
+        M.moe_grouped_swiglu(xe, off, layer.w1, layer.w3, layer.w2, None, c.N, c.d, c.h, c.E,
+                             layer.dt, layer.y, layer.sws)
+        M.moe_combine(layer.y, layer.dst_pos, rmap, layer.w, c.T, c.d, c.N, c.top_k, layer.dt,
+                      layer.out)
+
+    times = {"folded": [], "unfused": []}
+    for blk in range(4):
+        order = (("folded", folded), ("unfused", unfused))
+        for name, fn in (order if blk % 2 == 0 else order[::-1]):
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(steps + 1)]
+            torch.cuda.synchronize()
+            for a_ev, b_ev in ev:
+                a_ev.record(stream)
+                fn()
+                b_ev.record(stream)
+                flush.zero_()
+            torch.cuda.synchronize()
+            times[name] += [a.elapsed_time(b) for a, b in ev[1:]]
+    # the folded output against the unfused one (rounding differs: y is not
+    # rounded to bf16 on the folded path)
     err = (out.float() - layer.out.float()).abs().max().item()
     ref = layer.out.float().abs().max().item()
-    return [a.elapsed_time(b) for a, b in ev[2:]], err / max(ref, 1e-30)
-
-
-def timed_graph(layer, stream, flush, steps):
-    """CUDA-event times (ms) of replays of one moe_forward call captured in a
-    CUDA graph (the same kernels; no host work per step), L2 flushed between
-    replays, and whether the replay's output equals the direct call's."""
-    layer.forward()
-    torch.cuda.synchronize()
-    ref = layer.fout.clone()
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g):
-        layer.forward()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(steps + 2)]
-    torch.cuda.synchronize()
-    for a_ev, b_ev in ev:
-        a_ev.record(stream)
-        g.replay()
-        b_ev.record(stream)
-        flush.zero_()
-    torch.cuda.synchronize()
-    same = bool(torch.equal(layer.fout, ref))
-    del g
-    return [a.elapsed_time(b) for a, b in ev[2:]], same
+    return times, err / max(ref, 1e-30)
 
 
 def timed_forward(layer, stream, flush, steps):
@@ -684,9 +689,7 @@ def run_ours(args, ws, rank, local):
     e2e_match = e2e_match and bool(torch.equal(oh[(args.steps - 1) % 2].to(dev), out))
     # The combine folded into GEMM2 (moe_grouped_swiglu_combine), timed beside
     # the unfused grouped SwiGLU + combine of the staged step.
-    folded = timed_folded(layer, stream, flush, min(args.steps, 10))
-    graph_ms, graph_same = timed_graph(layer, stream, flush, args.steps)
-    graph_total = max_over_ranks(sum(graph_ms), ws)
+    folded = timed_folded(layer, stream, flush, min(args.steps, 5))
     clocks = sampler.stop() if rank == 0 else None
 
     if rank != 0:
@@ -750,18 +753,14 @@ def run_ours(args, ws, rank, local):
         "clocks": clocks,
         "peaks": pk,
     }
-    line["cuda_graph"] = {
-        "value": job_tokens_per_s(T, ws, args.steps, graph_total), "unit": UNIT,
-        "ms_per_step": graph_total / args.steps, "output_matches_direct_call": graph_same,
-        "what": "the same moe_forward call captured once in a CUDA graph and replayed each "
-                "step (no host work per step); L2 flushed between replays"}
     if folded is not None:
         line["folded_combine"] = {
-            "us": 1e3 * statistics.median(folded[0]),
-            "unfused_us": 1e3 * (stage_ms["grouped_swiglu"] + stage_ms["combine"]),
-            "max_diff_vs_staged_rel": folded[1],
+            "us": 1e3 * statistics.median(folded[0]["folded"]),
+            "unfused_us": 1e3 * statistics.median(folded[0]["unfused"]),
+            "max_diff_vs_unfused_rel": folded[1],
             "what": "moe_grouped_swiglu_combine (fp32 reductions in GEMM2's epilogue, then one "
-                    "bf16 rounding) against moe_grouped_swiglu + moe_combine"}
+                    "bf16 rounding) against moe_grouped_swiglu + moe_combine, medians of "
+                    "calls alternating in blocks, L2 flushed between calls"}
     if ws == 1 and not args.no_other_configs:
         del layer
         torch.cuda.empty_cache()
@@ -774,12 +773,14 @@ def run_ours(args, ws, rank, local):
 
 TRAIN_STAGES = ["router", "dispatch", "grouped_swiglu_train", "combine", "combine_backward",
                 "grouped_swiglu_backward", "router_backward", "dispatch_backward"]
-# kernels of ours per two-call training step: router 2 (its top-k kernel also
-# writes the dispatch histogram), dispatch 2, training GEMMs 2, combine 1,
-# combine backward 1, backward GEMMs 4, router backward 6 (scores, token
-# segments, gate weight-gradient partials, their sum, one segment, gate data
-# gradient), dispatch backward 1
-TRAIN_LAUNCHES = 19
+def train_launches(cfg) -> int:
+    """Kernels of ours per two-call training step: router 2 (its top-k kernel
+    also writes the dispatch histogram), dispatch 2, the training GEMMs (as
+    the forward's grouped SwiGLU), combine 1, combine backward 1, backward
+    GEMMs 4, router backward 6 (scores, token segments, gate weight-gradient
+    partials, their sum, one segment, gate data gradient), dispatch
+    backward 1."""
+    return 17 + grouped_gemm_launches(cfg)
 
 
 def run_training(args, ws, rank, local):
@@ -945,11 +946,11 @@ def run_training(args, ws, rank, local):
         "staged_ms_per_step": total_ms_max / args.steps,
         "two_call_matches_staged": matches,
         "device_status": status,
-        "gpu_launches": args.steps * TRAIN_LAUNCHES,
+        "gpu_launches": args.steps * train_launches(cfg),
         "gpu_launches_note": "kernels of libmoe per moe_forward_train + moe_backward step: "
-                             "router 2, dispatch 2, experts forward 2, combine 1, combine "
-                             "backward 1, experts backward 4, router backward 6, dispatch "
-                             "backward 1",
+                             "router 2, dispatch 2, experts forward "
+                             f"{grouped_gemm_launches(cfg)}, combine 1, combine backward 1, "
+                             "experts backward 4, router backward 6, dispatch backward 1",
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)

@@ -343,9 +343,11 @@ MOE_API moe_status_t moe_grouped_swiglu_gather(const void* x, int T, const int32
  * the grouped SwiGLU runs on CTA pairs (N >= 64 E); otherwise
  * MOE_ERR_UNSUPPORTED.  Workspace moe_grouped_swiglu_combine_workspace_size
  * (status word, H, the fp32 output, the slots' tokens and weights).
- * moe_forward keeps the deterministic path (moe_grouped_swiglu, then the
- * gather-reduce of moe_combine); this entry point is the alternative for
- * callers that accept run-to-run differences in the last bits.
+ * Measured slower on B200 than moe_grouped_swiglu + moe_combine (8-32 %
+ * on the bf16 workloads: the fp32 reductions move twice the bytes of the
+ * bf16 rows they replace), and not bitwise reproducible, so moe_forward
+ * keeps the separate gather-reduce; this entry point serves callers that
+ * cannot hold y [N, d].
  * ---------------------------------------------------------------------- */
 MOE_API size_t moe_grouped_swiglu_combine_workspace_size(int T, int top_k, int d, int h, int E,
                                                  moe_dtype_t dt);

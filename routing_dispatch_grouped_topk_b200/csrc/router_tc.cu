@@ -10,8 +10,10 @@
 // memory, not HBM: CTA r owns token rows [r 128 / C, (r + 1) 128 / C) of the
 // tile, every CTA stores its partial rows into their owner's shared memory
 // (st.shared::cluster), and the owner adds the C partials in rank order (a
-// fixed order: the logits do not depend on timing or on the grid).  One warp
-// per owned token then selects the k winners with k rounds of a warp
+// fixed order: the logits do not depend on timing or on the grid; each
+// warp stages its rows so that the remote stores write whole 128-byte row
+// pieces).  One warp per owned token (all six warps of the CTA) then
+// selects the k winners with k rounds of a warp
 // arg-max (two redux.sync reductions on (key, expert): descending key, ties
 // to the lower expert index) and writes the indices and weights; in the
 // layer forward the CTA also writes the dispatch histogram of its token
@@ -78,6 +80,8 @@ __device__ __forceinline__ void st_cluster_v4(uint32_t addr, uint32_t a, uint32_
                : "memory");
 }
 __device__ __forceinline__ void bar_epi() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// floats of one epilogue warp's 32 x 32 staging tile of the exchange (padded rows)
+constexpr int kXchgTile = 32 * 33;
 
 template <int BN>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -198,24 +202,40 @@ __global__ void __launch_bounds__(kThreads, 1)
   cluster_sync_all();
 
   // ------------------------------------------------- partial-logit exchange
+  // Each epilogue warp moves its 32 rows in 32 x 32 chunks: TMEM -> its
+  // staging tile in local shared memory (lane = row) -> read back so that 8
+  // lanes hold one row's 32 columns -> 16-byte remote stores that write 4
+  // whole 128-byte row pieces per instruction.
   float* recv = reinterpret_cast<float*>(smem);   // [C][own][pitch]
   const int pitch = a.pitch;
   if (warp >= 2) {
     const int q = warp & 3;
-    const int row = q * 32 + lane;
-    const int o = row / own, lr = row - o * own;
-    const uint32_t dst =
-        cluster_map(recv, static_cast<uint32_t>(o)) +
-        static_cast<uint32_t>((rank * own + lr) * pitch) * 4u;
+    float* stg = reinterpret_cast<float*>(smem + align_up(static_cast<size_t>(BM) * pitch * 4, 16)) +
+                 (warp - 2) * kXchgTile;        // [32][33]
     const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+    const int sub = lane >> 3, c4 = (lane & 7) * 4;
+    uint32_t dst_row[8];                          // remote address of the row each pass writes
+#pragma unroll
+    for (int pss = 0; pss < 8; ++pss) {
+      const int row = q * 32 + 4 * pss + sub;
+      const int o = row / own, lr = row - o * own;
+      dst_row[pss] = cluster_map(recv, static_cast<uint32_t>(o)) +
+                     static_cast<uint32_t>((rank * own + lr) * pitch + c4) * 4u;
+    }
     for (int c = 0; c * 32 < a.E; ++c) {
       uint32_t v[32];
       tmem_ld32(taddr + c * 32, v);
       tmem_ld_wait();
 #pragma unroll
-      for (int j = 0; j < 8; ++j)
-        st_cluster_v4(dst + static_cast<uint32_t>((c * 32 + 4 * j) * 4), v[4 * j], v[4 * j + 1],
-                      v[4 * j + 2], v[4 * j + 3]);
+      for (int j = 0; j < 32; ++j) stg[lane * 33 + j] = __uint_as_float(v[j]);
+      __syncwarp();
+#pragma unroll
+      for (int pss = 0; pss < 8; ++pss) {
+        const float* src = stg + (4 * pss + sub) * 33 + c4;
+        st_cluster_v4(dst_row[pss] + static_cast<uint32_t>(c * 32 * 4), __float_as_uint(src[0]),
+                      __float_as_uint(src[1]), __float_as_uint(src[2]), __float_as_uint(src[3]));
+      }
+      __syncwarp();
     }
     tc_fence_before();
   }
@@ -224,29 +244,28 @@ __global__ void __launch_bounds__(kThreads, 1)
   cluster_sync_all();
 
   // --------------------------------------------------- scores and top-k
-  // One warp per owned token (the four epilogue warps take every fourth):
+  // One warp per owned token (all six warps, each taking every sixth):
   // lane l holds experts l, l + 32, ... (EPL of them), adds the C partials
   // in rank order, and the k winners come from k rounds of a warp arg-max
   // on (key descending, expert ascending) -- two redux.sync reductions each.
   constexpr int EPL = BN / 32;
-  if (warp >= 2) {
-    const int i = threadIdx.x - 64;               // 0..127
-    const int ew = warp - 2;                      // epilogue warp 0..3
-    const int E = a.E, k = a.k;
-    const RouterOptions& opt = a.opt;
-    int* dbins = reinterpret_cast<int*>(smem + align_up(static_cast<size_t>(BM) * pitch * 4, 16));
-    int* ebins = dbins + (a.blk ? a.nbins : 0);
-    float* wsum = reinterpret_cast<float*>(ebins + E);
-    int* tok_e = reinterpret_cast<int*>(wsum + E);   // [own][k] winners, for the histograms
-    for (int e = i; e < E; e += 128) {
-      ebins[e] = 0;
-      wsum[e] = 0.f;
-    }
-    bar_epi();
-    const int t_own0 = tile * BM + rank * own;
+  const int i = threadIdx.x - 64;                 // epilogue threads: 0..127
+  const int E = a.E, k = a.k;
+  const RouterOptions& opt = a.opt;
+  int* dbins = reinterpret_cast<int*>(smem + align_up(static_cast<size_t>(BM) * pitch * 4, 16));
+  int* ebins = dbins + (a.blk ? a.nbins : 0);
+  float* wsum = reinterpret_cast<float*>(ebins + E);
+  int* tok_e = reinterpret_cast<int*>(wsum + E);   // [own][k] winners, for the histograms
+  const int t_own0 = tile * BM + rank * own;
+  for (int e = threadIdx.x; e < E; e += kThreads) {
+    ebins[e] = 0;
+    wsum[e] = 0.f;
+  }
+  __syncthreads();
+  {
     const bool on_logits = opt.bias == nullptr && opt.scale > 0.f;
     const size_t sstride = static_cast<size_t>(own) * pitch;
-    for (int it = ew; it < own; it += 4) {
+    for (int it = warp; it < own; it += kThreads / 32) {
       const int t = t_own0 + it;
       if (t >= a.T) break;                        // warp-uniform
       const float* rp = recv + static_cast<size_t>(it) * pitch + lane;
@@ -336,7 +355,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (a.lb) atomicAdd(&wsum[me], wv);
       }
     }
-    bar_epi();   // the winners of every owned token are in tok_e
+  }
+  __syncthreads();   // the winners of every owned token are in tok_e
+  if (warp >= 2) {
     // dispatch histogram of every token block of tb rows this CTA owns
     if (a.blk) {
       if (blockIdx.x == 0 && i == 0)   // the dispatch column scan's ticket
@@ -439,9 +460,14 @@ RouterFusedPlan router_fused_plan(int T, int d, int E, const DispatchPlan* plan)
     case 128: stages = rtc::Layout<128>::kStageRegion; tail = rtc::Layout<128>::kTailBytes; break;
     default: stages = rtc::Layout<256>::kStageRegion; tail = rtc::Layout<256>::kTailBytes; break;
   }
-  const size_t exch = align_up(static_cast<size_t>(rtc::BM) * p.pitch * 4, 16) +
-                      (plan ? static_cast<size_t>(plan->nbins) * 4 : 0) + 8 * static_cast<size_t>(E) +
-                      static_cast<size_t>(rtc::BM) * kMaxTopK * 4;   // the owned tokens' winners
+  // (during the exchange the four epilogue warps' staging tiles sit where
+  // the bins go afterwards)
+  const size_t recv = align_up(static_cast<size_t>(rtc::BM) * p.pitch * 4, 16);
+  const size_t exch = recv + std::max<size_t>(
+                                 4 * rtc::kXchgTile * 4,
+                                 (plan ? static_cast<size_t>(plan->nbins) * 4 : 0) +
+                                     8 * static_cast<size_t>(E) +
+                                     static_cast<size_t>(rtc::BM) * kMaxTopK * 4);
   p.region = static_cast<int>(align_up(std::max<size_t>(stages, exch), 1024));
   p.smem = p.region + tail + 1024;   // + slack for the 1 KB alignment
   // two CTAs per SM when they fit (228 KB per SM, 1 KB reserved per CTA)

@@ -92,6 +92,10 @@ struct Args {
   int split;                 // weight gradient: rows of each expert that go to `out`
   int Ma;                    // weight gradient: output rows per expert
   float* out_f32;            // weight gradient: fp32 output [E, Ma, n_out] instead of bf16
+  // Which rows of each expert segment a grouped launch covers (see
+  // pair_head): 0 all of them, 1 the head (CTA-pair launch), 2 the tail
+  // (single-CTA launch).
+  int seg_part;
   // GEMM2 with the combine folded in (CTA-pair kernel): output row s is
   // scaled by comb_w[s] and added into comb_out[comb_tok[s]] with fp32
   // reductions instead of being stored
@@ -172,6 +176,30 @@ struct RouterPolicy {
   static __device__ void finish(const Args&, int*) {}
 };
 
+// The forward's grouped GEMMs split each expert segment of cnt rows between
+// the CTA-pair kernel (256-row pair tiles) and the single-CTA kernel
+// (128-row tiles): a last block of at most 128 rows after at least one full
+// pair tile, or a whole segment of at most 128 rows, goes to the single-CTA
+// kernel, which spends one SM on it where a pair tile would spend two.  The
+// head is the rows the pair kernel covers.
+// Measured on B200: with K = 2880 (64-wide K blocks: 45 per tile) the split
+// took the two GEMMs from 1924 to 1847 us; with K = 2048 and 768 it made
+// them 13 % slower (the second launch waits for the first to finish, and
+// short tiles do not win that back).
+constexpr int kSplitMinK = 2560;
+__host__ __device__ __forceinline__ int pair_head(int cnt) {
+  if (cnt <= 128) return 0;
+  const int mt = cdiv(cnt, 256);
+  return (mt >= 2 && cnt - (mt - 1) * 256 <= 128) ? (mt - 1) * 256 : cnt;
+}
+// First row and length of the part of a segment of cnt rows that a launch
+// with the given seg_part covers.
+__device__ __forceinline__ void split_rows(int part, int cnt, int& start, int& len) {
+  const int head = part ? pair_head(max(cnt, 0)) : 0;
+  start = part == 2 ? head : 0;
+  len = part == 0 ? cnt : part == 1 ? head : cnt - head;
+}
+
 // Grouped problems: schedule over expert segments.  sched layout:
 //   [0] total tiles  [1] n-tiles per m-tile row  [8 .. 8+E]  offsets
 //   [8+E+1 .. 8+2E+1] cumulative tile counts
@@ -204,7 +232,9 @@ struct GroupedSched {
       for (int e = e0; e < e1; ++e) {
         const int cnt = off[e + 1] - off[e];
         bad |= cnt < 0;
-        local += cdiv(max(cnt, 0), MR) * nt;
+        int start, len;
+        split_rows(a.seg_part, cnt, start, len);
+        local += cdiv(max(len, 0), MR) * nt;
       }
       int incl = local;
 #pragma unroll
@@ -215,7 +245,9 @@ struct GroupedSched {
       int run = incl - local;
       for (int e = e0; e < e1; ++e) {
         cum[e] = run;
-        run += cdiv(max(off[e + 1] - off[e], 0), MR) * nt;
+        int start, len;
+        split_rows(a.seg_part, off[e + 1] - off[e], start, len);
+        run += cdiv(max(len, 0), MR) * nt;
       }
       bad = __any_sync(0xffffffffu, bad);
       const int total = __shfl_sync(0xffffffffu, incl, 31);
@@ -241,8 +273,9 @@ struct GroupedSched {
       if (cum[mid] <= tile) lo = mid; else hi = mid - 1;
     }
     e = lo;
-    seg0 = off[e];
-    cnt = off[e + 1] - seg0;
+    int start;
+    split_rows(a.seg_part, off[e + 1] - off[e], start, cnt);
+    seg0 = off[e] + start;
     const int mtiles = cdiv(cnt, MR);
     const int local = tile - cum[e];
     nt = local / mtiles;
@@ -776,7 +809,9 @@ struct PairSched : GroupedSched<256, NUM_B_, NCOLS, 256> {
       for (int e = e0; e < e1; ++e) {
         const int cnt = off[e + 1] - off[e];
         bad |= cnt < 0;
-        local += cdiv(max(cnt, 0), 256) * nt;
+        int start, len;
+        split_rows(a.seg_part, cnt, start, len);
+        local += cdiv(max(len, 0), 256) * nt;
       }
       int incl = local;
 #pragma unroll
@@ -787,7 +822,9 @@ struct PairSched : GroupedSched<256, NUM_B_, NCOLS, 256> {
       int run = incl - local;
       for (int e = e0; e < e1; ++e) {
         cum[e] = run;
-        run += cdiv(max(off[e + 1] - off[e], 0), 256) * nt;
+        int start, len;
+        split_rows(a.seg_part, off[e + 1] - off[e], start, len);
+        run += cdiv(max(len, 0), 256) * nt;
       }
       bad = __any_sync(0xffffffffu, bad);
       const int total = __shfl_sync(0xffffffffu, incl, 31);
@@ -813,7 +850,9 @@ struct PairSched : GroupedSched<256, NUM_B_, NCOLS, 256> {
       if (cum[mid] <= tile) lo = mid; else hi = mid - 1;
     }
     const int e = lo;
-    const int seg0 = off[e], cnt = off[e + 1] - seg0;
+    int start, cnt;
+    split_rows(a.seg_part, off[e + 1] - off[e], start, cnt);
+    const int seg0 = off[e] + start;
     const int mtiles = cdiv(cnt, 256);
     const int local = tile - cum[e];
     const int nt = local / mtiles, mt = local - nt * mtiles;
@@ -1889,10 +1928,30 @@ static cudaError_t swiglu_tc_impl(const void* a_src, int a_rows, const int32_t* 
   a.gather_src = a_src;
   a.gu_out = static_cast<__nv_bfloat16*>(gu);
   if (pairs) {
+    // Each segment's head on CTA pairs and its short last block on the
+    // single-CTA kernel (pair_head), for a GEMM whose reduction is long
+    // enough (kSplitMinK) that the tail tiles' saving outweighs the second
+    // launch; the folded combine keeps whole segments on pairs (only the
+    // pair kernel folds).  The tail launches read what the head launches
+    // read and write other rows.
+    const bool split1 = fold == nullptr && d >= kSplitMinK;
+    const bool split2 = fold == nullptr && h >= kSplitMinK;
+    CUtensorMap t2s;   // w2 in 256-row boxes for the single-CTA GEMM2
+    if (split2 && !make_tmap(&t2s, w2, h, static_cast<uint64_t>(E) * d, 256))
+      return cudaErrorInvalidValue;
     const long long max_pt = cdiv(N, 256) + E;   // upper bound on pair tiles per n-tile
     int np = static_cast<int>(std::min<long long>(num_sms() / 2, max_pt * cdiv(h, 128)));
+    a.seg_part = split1 ? 1 : 0;
     cudaError_t e = launch_pair<UpPairPolicy>(tx, t1, t3, a, np, s);
     if (e != cudaSuccess) return e;
+    if (split1) {   // at most one 128-row tail tile per (expert, n-tile)
+      a.seg_part = 2;
+      e = launch<UpStagedPolicy>(tx, t1, t3, a,
+                                 static_cast<int>(std::min<long long>(
+                                     num_sms(), 1LL * E * cdiv(h, 128))),
+                                 s);
+      if (e != cudaSuccess) return e;
+    }
     a.K = h;
     a.n_out = d;
     a.out = static_cast<__nv_bfloat16*>(y);
@@ -1905,7 +1964,14 @@ static cudaError_t swiglu_tc_impl(const void* a_src, int a_rows, const int32_t* 
       a.comb_T = fold->T;
     }
     np = static_cast<int>(std::min<long long>(num_sms() / 2, max_pt * cdiv(d, 256)));
-    return launch_pair<DownPairPolicy>(th, t2, t2, a, np, s);
+    a.seg_part = split2 ? 1 : 0;
+    e = launch_pair<DownPairPolicy>(th, t2, t2, a, np, s);
+    if (e != cudaSuccess || !split2) return e;
+    a.seg_part = 2;
+    return launch<DownStagedPolicy>(th, t2s, t2s, a,
+                                    static_cast<int>(std::min<long long>(
+                                        num_sms(), 1LL * E * cdiv(d, 256))),
+                                    s);
   }
   int grid = static_cast<int>(std::min<long long>(num_sms(), 1LL * max_mt * cdiv(h, 128)));
   cudaError_t e = gather ? launch<UpGatherPolicy>(tx, t1, t3, a, grid, s)
