@@ -52,20 +52,15 @@ struct TileInfo {
   int m_valid;   // rows of this tile that belong to the problem / expert
   int n0;        // first output column (router: the K split)
   int kb0, kb1;  // K blocks [kb0, kb1) of this tile
-  int swap_np;   // 0, or: swap-AB tile whose MMA N is this many token rows
   int m0;        // weight-gradient tiles: first output row (A column)
 };
 
 // A grouped tile with few valid rows (an expert's last rows, or decode) is
-// computed with A and B swapped: the 128-row weight halves of the B stage
-// become the MMA's M = 128 operand and the tile's token rows (rounded up to
-// 16) its N, as two MMAs of N = np instead of one of N = 256.  The shared
-// memory stages are the same; only the MMA issue and the epilogue differ
-// (accumulator lanes are weight rows, columns are tokens).
-constexpr int kSwapMaxRows = 112;   // 2 * 112 < 256: a swap tile always costs less
-__device__ __forceinline__ void set_swap(TileInfo& t) {
-  t.swap_np = (t.m_valid <= kSwapMaxRows) ? ((max(t.m_valid, 1) + 15) & ~15) : 0;
-}
+// a plain 128-row tile.  (Swap-AB tiles -- the weight halves of the B stage
+// as the MMA's M = 128 operand, the tile's tokens as N -- were measured on
+// B200: no faster for decode, whose grouped GEMMs stream every weight once
+// at the HBM copy rate either way, and 2-6 % slower for segment tails at the
+// gpt-oss EP8 sizes: small-N MMAs do not run proportionally faster.)
 
 struct Args {
   int M;                     // rows of A: T (router) or N (grouped)
@@ -145,7 +140,6 @@ struct RouterPolicy {
     t.n0 = sp;
     t.kb0 = sp * a.kb_per_split;
     t.kb1 = min(cdiv(a.K, BK), t.kb0 + a.kb_per_split);
-    t.swap_np = 0;
     return t;
   }
   static __device__ void epilogue(const Args& a, int*, const TileInfo& ti, uint32_t taddr,
@@ -302,46 +296,10 @@ struct UpPolicyT : GroupedSched<256, 2, 128> {
     t.b_row = e * a.n_out + t.n0;
     t.kb0 = 0;
     t.kb1 = cdiv(a.K, BK);
-    set_swap(t);
     return t;
-  }
-  // Swap-AB tile: lane = hidden unit n0 + row; columns [0, np) hold G and
-  // [np, 2 np) hold U for the tile's tokens.  A warp stores 64 contiguous
-  // bytes of H per token.
-  static __device__ void epilogue_swap(const Args& a, const TileInfo& ti, uint32_t taddr,
-                                       int row) {
-    const int n = ti.n0 + row;
-    const bool nvalid = n < a.n_out;
-    __nv_bfloat16* col = a.out + static_cast<size_t>(ti.a_row) * a.n_out + n;
-    for (int t0 = 0; t0 < ti.m_valid; t0 += 16) {
-      uint32_t g[16], u[16];
-      tmem_ld16(taddr + t0, g);
-      tmem_ld16(taddr + ti.swap_np + t0, u);
-      tmem_ld_wait();
-      if (nvalid) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          if (t0 + i < ti.m_valid) {
-            const float gv = __uint_as_float(g[i]), uv = __uint_as_float(u[i]);
-            col[static_cast<size_t>(t0 + i) * a.n_out] =
-                __float2bfloat16_rn(__fdividef(gv, 1.0f + __expf(-gv)) * uv);
-            if (a.gu_out) {
-              __nv_bfloat16* gu =
-                  a.gu_out + static_cast<size_t>(ti.a_row + t0 + i) * (2 * a.n_out) + n;
-              gu[0] = __float2bfloat16_rn(gv);
-              gu[a.n_out] = __float2bfloat16_rn(uv);
-            }
-          }
-        }
-      }
-    }
   }
   static __device__ void epilogue(const Args& a, int*, const TileInfo& ti, uint32_t taddr,
                                   int row) {
-    if (ti.swap_np) {
-      epilogue_swap(a, ti, taddr, row);
-      return;
-    }
     const bool valid = row < ti.m_valid;
     __nv_bfloat16* dst_row = a.out + static_cast<size_t>(ti.a_row + row) * a.n_out + ti.n0;
 #pragma unroll 1
@@ -400,38 +358,10 @@ struct DownPolicy : GroupedSched<256, 1, 256> {
     t.b_row = e * a.n_out + t.n0;
     t.kb0 = 0;
     t.kb1 = cdiv(a.K, BK);
-    set_swap(t);
     return t;
-  }
-  // Swap-AB tile: lane = output column n0 + row (columns [0, np)) and
-  // n0 + 128 + row (columns [np, 2 np)); columns are the tile's tokens.
-  static __device__ void epilogue_swap(const Args& a, const TileInfo& ti, uint32_t taddr,
-                                       int row) {
-    const int c1 = ti.n0 + row, c2 = ti.n0 + 128 + row;
-    __nv_bfloat16* base = a.out + static_cast<size_t>(ti.a_row) * a.n_out;
-    for (int t0 = 0; t0 < ti.m_valid; t0 += 16) {
-      uint32_t v1[16], v2[16];
-      tmem_ld16(taddr + t0, v1);
-      tmem_ld16(taddr + ti.swap_np + t0, v2);
-      tmem_ld_wait();
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int t = t0 + i;
-        if (t < ti.m_valid) {
-          const float sc = a.row_scale ? a.row_scale[ti.a_row + t] : 1.0f;
-          __nv_bfloat16* r = base + static_cast<size_t>(t) * a.n_out;
-          if (c1 < a.n_out) r[c1] = __float2bfloat16_rn(__uint_as_float(v1[i]) * sc);
-          if (c2 < a.n_out) r[c2] = __float2bfloat16_rn(__uint_as_float(v2[i]) * sc);
-        }
-      }
-    }
   }
   static __device__ void epilogue(const Args& a, int*, const TileInfo& ti, uint32_t taddr,
                                   int row) {
-    if (ti.swap_np) {
-      epilogue_swap(a, ti, taddr, row);
-      return;
-    }
     const bool valid = row < ti.m_valid;
     const size_t grow = static_cast<size_t>(ti.a_row + row);
     const float scale = (valid && a.row_scale) ? a.row_scale[grow] : 1.0f;
@@ -501,7 +431,6 @@ struct DownBwdPolicy : GroupedSched<256, 1, 256> {
     t.b_row = e * a.K;
     t.kb0 = 0;
     t.kb1 = cdiv(a.K, BK);
-    t.swap_np = 0;
     t.m0 = 0;
     return t;
   }
@@ -628,7 +557,6 @@ struct UpBwdPolicy : GroupedSched<256, 2, 256> {
     t.b_row = e * (a.K / 2);
     t.kb0 = 0;
     t.kb1 = cdiv(a.K, BK);
-    t.swap_np = 0;
     t.m0 = 0;
     return t;
   }
@@ -661,12 +589,6 @@ struct UpStagedPolicy : UpPolicyT<false> {
   static constexpr int EPI_STAGE_BYTES = 8 * 2048;
   static __device__ void epilogue_staged(const Args& a, int* s, const TileInfo& ti,
                                          uint32_t taddr, int row, uint8_t* stg, int c0, int c1) {
-    if (ti.swap_np) {
-      // swap-AB tile: one lane per hidden unit; the first warp of each
-      // quadrant writes (the per-row epilogue, as inference)
-      if (c0 == 0) UpPolicyT<false>::epilogue(a, s, ti, taddr, row);
-      return;
-    }
     const int lane = threadIdx.x & 31;
     const int wrow0 = row - lane;
     const int h = a.n_out;
@@ -725,10 +647,6 @@ struct DownStagedPolicy : DownPolicy {
   static constexpr int EPI_STAGE_BYTES = 8 * 2048;
   static __device__ void epilogue_staged(const Args& a, int* s, const TileInfo& ti,
                                          uint32_t taddr, int row, uint8_t* stg, int c0, int c1) {
-    if (ti.swap_np) {
-      if (c0 == 0) DownPolicy::epilogue(a, s, ti, taddr, row);
-      return;
-    }
     const int lane = threadIdx.x & 31;
     const int wrow0 = row - lane;
     const int j = lane & 3;
@@ -862,7 +780,6 @@ struct PairSched : GroupedSched<256, NUM_B_, NCOLS, 256> {
     t.kb0 = 0;
     t.kb1 = cdiv(a.K, BK);
     t.m0 = 0;
-    t.swap_np = 0;
     t.a_row = seg0 + r0;
     t.m_valid = max(0, min(BM, cnt - r0));
     t.b_row = UP ? e * a.n_out + t.n0 : e * a.n_out + t.n0 + 128 * rank;
@@ -930,7 +847,6 @@ struct DgradPolicy : GroupedSched<256, 1, 256> {
     t.b_row = e * a.K;
     t.kb0 = 0;
     t.kb1 = cdiv(a.K, BK);
-    t.swap_np = 0;
     t.m0 = 0;
     return t;
   }
@@ -996,7 +912,6 @@ struct WgradPolicy {
     t.n0 = (r - m * nt) * BN;
     t.kb0 = 0;
     t.kb1 = cdiv(t.m_valid, BK);
-    t.swap_np = 0;
     return t;
   }
   // rows of K block kb that belong to the segment (the rest are zeroed)
@@ -1437,23 +1352,10 @@ __global__ void __launch_bounds__(P::THREADS, 1)
               P::A_MN ? sw128_mnmajor_desc(sa, kMnBoxBytes) : sw128_kmajor_desc(sa);
           const uint64_t bd = P::B_MN ? sw128_mnmajor_desc(sa + kATileBytes, kMnBoxBytes)
                                       : sw128_kmajor_desc(sa + kATileBytes);
-          if (BN == 256 && !P::A_MN && !P::B_MN && ti.swap_np) {
-            // D[:, 0:np) = B[0:128) A^T, D[:, np:2np) = B[128:256) A^T
-            const uint32_t idesc_s = idesc_bf16_f32(128, ti.swap_np);
-            const uint64_t bd_hi = bd + ((128u * 128u) >> 4);   // rows 128.. of the B stage
 #pragma unroll
-            for (int kk = 0; kk < BK / 16; ++kk) {
-              const uint32_t accum = (kb != ti.kb0 || kk != 0) ? 1u : 0u;
-              tc_mma_bf16(d_tmem, bd + 2u * kk, ad + 2u * kk, idesc_s, accum);
-              tc_mma_bf16(d_tmem + static_cast<uint32_t>(ti.swap_np), bd_hi + 2u * kk,
-                          ad + 2u * kk, idesc_s, accum);
-            }
-          } else {
-#pragma unroll
-            for (int kk = 0; kk < BK / 16; ++kk)
-              tc_mma_bf16(d_tmem, ad + A_KSTEP * kk, bd + B_KSTEP * kk, IDESC,
-                          (kb != ti.kb0 || kk != 0) ? 1u : 0u);
-          }
+          for (int kk = 0; kk < BK / 16; ++kk)
+            tc_mma_bf16(d_tmem, ad + A_KSTEP * kk, bd + B_KSTEP * kk, IDESC,
+                        (kb != ti.kb0 || kk != 0) ? 1u : 0u);
           tc_commit(empty + stage);
           if (++stage == STAGES) {
             stage = 0;
@@ -1908,7 +1810,7 @@ static cudaError_t swiglu_tc_impl(const void* a_src, int a_rows, const int32_t* 
   if (!make_tmap(&th, H, h, N, BM)) return cudaErrorInvalidValue;
   // The CTA-pair kernel (256-row pair tiles) serves every layer whose
   // segments average 64 rows or more; shorter segments (decode) stay on the
-  // single-CTA kernel, whose swap-AB tiles stream each weight tile once.
+  // single-CTA kernel, whose 128-row tiles stream each weight tile once.
   const bool pairs = !gather && swiglu_tc_uses_pairs(N, E);
   if (fold && !pairs) return cudaErrorInvalidValue;
   if (!make_tmap(&t2, w2, h, static_cast<uint64_t>(E) * d, pairs ? 128 : 256))
