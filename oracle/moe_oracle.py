@@ -52,7 +52,7 @@ __all__ = [
     "grouped_swiglu", "combine", "moe_forward", "dense_moe", "moe_tokens",
     "silu_grad", "grouped_preactivations", "combine_backward", "grouped_swiglu_backward",
     "dispatch_backward", "router_backward", "load_balance_loss_grad",
-    "scaled_dispatch_backward",
+    "scaled_dispatch_backward", "capacity_drop",
 ]
 
 
@@ -154,7 +154,8 @@ def node_limited_mask(scores, num_groups: int, topk_groups: int) -> np.ndarray:
 
 def router_topk_general(top_k: int, x=None, w_router=None, logits=None, score: str = "softmax",
                         renormalize: bool = False, route_scale: float = 1.0, expert_bias=None,
-                        num_groups: int = 0, topk_groups: int = 0):
+                        num_groups: int = 0, topk_groups: int = 0, capacity: int = 0,
+                        sel_scores=None):
     """Token-choice router with every option of [HP] ``TokenChoiceTopKRouter``,
     in its order: gate logits -> ``score_func`` (softmax over the experts or
     sigmoid) -> times ``route_scale`` -> node-limited group masking ->
@@ -162,8 +163,12 @@ def router_topk_general(top_k: int, x=None, w_router=None, logits=None, score: s
     scores as weights -> bincount.  With ``renormalize`` ([QO]
     ``norm_topk_prob``) the gathered weights are divided by their sum; the
     scale is applied after that division (so that it survives it; without
-    renormalisation this equals gathering the scaled scores).  Returns
-    ``(idx, w, counts, logits)`` like :func:`router_topk`."""
+    renormalisation this equals gathering the scaled scores).  With
+    ``capacity`` > 0 the capacity drop policy (:func:`capacity_drop`) then
+    marks the dropped copies ``idx = -1`` with weight 0; it ranks by
+    ``sel_scores`` [T, k] when given (a caller's copy of the selected scores
+    in its own precision), else by this function's.  Returns ``(idx, w,
+    counts, logits)`` like :func:`router_topk`."""
     L = as_f64(logits) if logits is not None else router_logits(x, w_router)
     E = L.shape[1]
     s = softmax(L) if score == "softmax" else sigmoid(L)
@@ -172,9 +177,14 @@ def router_topk_general(top_k: int, x=None, w_router=None, logits=None, score: s
     keys = for_topk + as_f64(expert_bias)[None, :] if expert_bias is not None else for_topk
     idx = topk_select(keys, top_k)
     w = np.take_along_axis(s, idx, axis=1)
+    sel = w.copy()
     if renormalize:
         w = w / w.sum(axis=1, keepdims=True)
     w = w * route_scale
+    if capacity > 0:
+        keep = capacity_drop(idx, sel if sel_scores is None else sel_scores, capacity)
+        idx = np.where(keep, idx, -1)
+        w = np.where(keep, w, 0.0)
     return idx, w, expert_counts(idx, E), L
 
 
@@ -226,8 +236,34 @@ def load_balance_loss_grad(selected_experts, E: int) -> np.ndarray:
 
 
 def expert_counts(idx, E: int) -> np.ndarray:
-    """``counts[e] = #{(t, j): idx[t, j] == e}`` ([HP] ``torch.bincount``)."""
-    return np.bincount(_i64(idx).ravel(), minlength=E).astype(np.int64)
+    """``counts[e] = #{(t, j): idx[t, j] == e}`` ([HP] ``torch.bincount``);
+    copies marked -1 (dropped by :func:`capacity_drop`) are not counted."""
+    flat = _i64(idx).ravel()
+    return np.bincount(flat[flat >= 0], minlength=E).astype(np.int64)
+
+
+def capacity_drop(idx, sel_scores, capacity: int) -> np.ndarray:
+    """Capacity drop policy ([P4] PaddleFormers ``moe_gate.py``,
+    ``_probs_drop_policy``): a token keeps its assignment to an expert when
+    it is routed there and its score for that expert is among the top
+    ``capacity`` scores for that expert.  Reading taken: the ranking is over
+    the copies routed to the expert (unrouted pairs rank below every routed
+    one), by the router's score of the pair before renormalisation and
+    scale, higher first, equal scores in increasing token order.  Returns
+    the keep mask ``[T, k]``.  ``sel_scores[t, j]`` is the score of the
+    copy ``(t, j)``."""
+    idx = _i64(idx)
+    s = as_f64(sel_scores)
+    T, k = idx.shape
+    keep = np.zeros((T, k), dtype=bool)
+    for e in np.unique(idx):
+        if e < 0:
+            continue
+        tt, jj = np.nonzero(idx == e)
+        order = sorted(range(len(tt)), key=lambda q: (-s[tt[q], jj[q]], tt[q]))
+        for q in order[:max(capacity, 0)]:
+            keep[tt[q], jj[q]] = True
+    return keep
 
 
 # --------------------------------------------------------------------------
@@ -244,17 +280,21 @@ def dispatch(idx, E: int):
     * ``counts[E]``, ``offsets[E+1]`` (exclusive scan, ``offsets[E] = T*k``),
     * ``src_row[N]``: the token of each expert-major slot (``f // k``),
     * ``dst_pos[T, k]``: the slot of each copy (inverse of the sort).
+
+    Copies marked -1 (dropped by the capacity policy) get no slot: their
+    ``dst_pos`` is -1, and ``offsets[E]`` counts the kept copies only.
     """
     idx = _i64(idx)
     T, k = idx.shape
     flat = idx.ravel()
-    order = np.argsort(flat, kind="stable")       # slot -> flat index
-    counts = np.bincount(flat, minlength=E).astype(np.int64)
+    kept = np.nonzero(flat >= 0)[0]
+    order = kept[np.argsort(flat[kept], kind="stable")]   # slot -> flat index
+    counts = np.bincount(flat[kept], minlength=E).astype(np.int64)
     offsets = np.zeros(E + 1, dtype=np.int64)
     offsets[1:] = np.cumsum(counts)
     src_row = order // k
-    dst = np.empty(T * k, dtype=np.int64)
-    dst[order] = np.arange(T * k)
+    dst = np.full(T * k, -1, dtype=np.int64)
+    dst[order] = np.arange(len(order))
     return counts, offsets, src_row, dst.reshape(T, k)
 
 
@@ -399,7 +439,8 @@ def combine(y, dst_pos, topk_w=None) -> np.ndarray:
     out = np.zeros((T, y.shape[1]), dtype=np.float64)
     w = np.ones((T, k)) if topk_w is None else as_f64(topk_w)
     for j in range(k):
-        out += w[:, j:j + 1] * y[dp[:, j]]
+        live = dp[:, j] >= 0           # a dropped copy (-1) adds nothing
+        out[live] += w[live, j:j + 1] * y[dp[live, j]]
     return out
 
 
