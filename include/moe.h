@@ -21,6 +21,10 @@
  *   [EP] huggingface/transformers PR #41053 "Qwen3 moe":
  *        Ep2DpParallel._token_dispatch (rank-major received buffer that has to
  *        be reshuffled back into expert order).
+ *   [PF] PaddlePaddle/PaddleFormers PR #2702 "[Unified MoE Layer]: Add MoE
+ *        Layer with DeepEP EP Support; Add Qwen3MoE EP", review of
+ *        paddleformers/nn/moe_deepep/moe_gate.py: _probs_drop_policy (the
+ *        capacity drop policy).
  *
  * Conventions shared by every entry point
  * ---------------------------------------
@@ -170,6 +174,21 @@ MOE_API moe_status_t moe_router_topk(const void* x, const void* w_router, const 
  * weight of a copy routed to expert e receives aux_loss_coef * E * f_e / T
  * (f_e as above; the counts carry no gradient), added to d_topk_w before the
  * router's backward.  0 (the default) adds nothing.
+ *
+ * capacity ([PF] PaddleFormers moe_gate.py, _probs_drop_policy): 0 (the
+ * default) keeps every copy.  With capacity > 0 a token keeps its copy for
+ * expert e only if its score for e is among the `capacity` highest scores of
+ * the copies routed to e (the score before renormalisation and route_scale;
+ * equal scores to the lower token index): a dropped copy gets topk_idx = -1
+ * and topk_w = 0, the kept weights are unchanged, and `counts` counts the
+ * kept copies (tokens_per_expert and aux_loss still count the routed ones).
+ * moe_dispatch skips -1 without an error; moe_combine and the backward
+ * entry points skip the positions of dropped copies.  moe_forward_ex: bf16
+ * and ep_ranks = 1 only; the training entry points take no capacity.
+ *
+ * topk_scores (output, [T, k] fp32 device, or NULL): the score of each
+ * selected expert before renormalisation and route_scale (softmax or
+ * sigmoid of the logits), the key the capacity policy ranks by.
  * ---------------------------------------------------------------------- */
 typedef struct moe_router_options {
   moe_score_t score;
@@ -182,6 +201,8 @@ typedef struct moe_router_options {
   int score_before_experts;
   float* aux_loss;
   float aux_loss_coef;
+  int capacity;
+  float* topk_scores;
 } moe_router_options_t;
 
 MOE_API void moe_router_options_init(moe_router_options_t* opts);
@@ -209,7 +230,9 @@ MOE_API moe_status_t moe_router_topk_ex(const void* x, const void* w_router,
  * The order inside an expert segment is increasing f, so the result is
  * unique and bit-exact.  topk_idx [T, k] int32; counts [E]; offsets [E+1];
  * src_row [T*k]; dst_pos [T, k]; x [T, d] and x_perm [T*k, d] dt.
- * Ids outside [0, E) set MOE_DEV_BAD_EXPERT; such copies get dst_pos = -1,
+ * An id of -1 is a copy the capacity policy dropped: it is skipped (dst_pos
+ * = -1, no slot) without an error.  Other ids outside [0, E) set
+ * MOE_DEV_BAD_EXPERT; such copies get dst_pos = -1,
  * take no slot, and the unused tail slots of src_row are -1.
  * ---------------------------------------------------------------------- */
 MOE_API size_t moe_dispatch_workspace_size(int T, int E, int top_k);

@@ -243,7 +243,7 @@ def expert_counts(idx, E: int) -> np.ndarray:
 
 
 def capacity_drop(idx, sel_scores, capacity: int) -> np.ndarray:
-    """Capacity drop policy ([P4] PaddleFormers ``moe_gate.py``,
+    """Capacity drop policy ([PF] PaddleFormers ``moe_gate.py``,
     ``_probs_drop_policy``): a token keeps its assignment to an expert when
     it is routed there and its score for that expert is among the top
     ``capacity`` scores for that expert.  Reading taken: the ranking is over

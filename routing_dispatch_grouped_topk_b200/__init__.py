@@ -95,6 +95,8 @@ class RouterOptions(ctypes.Structure):
         ("score_before_experts", ctypes.c_int),
         ("aux_loss", ctypes.c_void_p),
         ("aux_loss_coef", ctypes.c_float),
+        ("capacity", ctypes.c_int),
+        ("topk_scores", ctypes.c_void_p),
     ]
 
 
@@ -280,13 +282,15 @@ def moe_router_options_init() -> RouterOptions:
 def router_options(score="softmax", renormalize=False, route_scale=1.0, expert_bias=None,
                    num_groups=0, topk_groups=0, tokens_per_expert=None,
                    score_before_experts=False, aux_loss=None,
-                   aux_loss_coef=0.0) -> RouterOptions:
+                   aux_loss_coef=0.0, capacity=0, topk_scores=None) -> RouterOptions:
     """A RouterOptions from keyword values ([HP] TokenChoiceTopKRouter's
     settings).  expert_bias / tokens_per_expert are fp32 CUDA tensors [E],
-    aux_loss an fp32 CUDA tensor of one element, or None; they must stay
-    alive while the call that takes the options runs.  aux_loss_coef (the
-    backward entry points) adds the gradient of aux_loss_coef times the
-    load-balance loss to the routing weights' gradient."""
+    aux_loss an fp32 CUDA tensor of one element, topk_scores an fp32 CUDA
+    tensor [T, k] (output), or None; they must stay alive while the call
+    that takes the options runs.  aux_loss_coef (the backward entry points)
+    adds the gradient of aux_loss_coef times the load-balance loss to the
+    routing weights' gradient.  capacity > 0 applies the capacity drop
+    policy (dropped copies: topk_idx -1, weight 0)."""
     o = moe_router_options_init()
     o.score = {"softmax": MOE_SCORE_SOFTMAX, "sigmoid": MOE_SCORE_SIGMOID}[score]
     o.renormalize = int(bool(renormalize))
@@ -298,6 +302,8 @@ def router_options(score="softmax", renormalize=False, route_scale=1.0, expert_b
     o.score_before_experts = int(bool(score_before_experts))
     o.aux_loss = _ptr(aux_loss, torch.float32, "aux_loss")
     o.aux_loss_coef = float(aux_loss_coef)
+    o.capacity = int(capacity or 0)
+    o.topk_scores = _ptr(topk_scores, torch.float32, "topk_scores")
     return o
 
 

@@ -85,12 +85,21 @@ float lb_grad_scale(float coef, int E, int T, int k) {
                : 0.f;
 }
 
-// Status word, the load-balance statistics, then the fp32 logit scratch:
-// [ksplit, T, E] partial logits of the tensor-core GEMM, or [T, E] logits of
-// the CUDA-core path.
-size_t router_ws(int T, int d, int E, moe_dtype_t dt) {
+// Status word, the load-balance statistics, the fp32 logit scratch ([ksplit,
+// T, E] partial logits of the tensor-core GEMM, or [T, E] logits of the
+// CUDA-core path), then the capacity policy's scratch: the selected scores
+// [T, kMaxTopK] and one 64-bit threshold per expert.
+size_t logit_scratch_bytes(int T, int d, int E, moe_dtype_t dt) {
   const size_t planes = router_uses_tc(E, dt) ? router_plan(T, d).ksplit : 1;
-  return kStatusBytes + lb_bytes(E) + align_up(planes * T * E * sizeof(float), 256);
+  return align_up(planes * T * E * sizeof(float), 256);
+}
+size_t capacity_scratch_bytes(int T, int E) {
+  return align_up(static_cast<size_t>(T) * kMaxTopK * sizeof(float), 256) +
+         align_up(static_cast<size_t>(E) * 8, 256);
+}
+size_t router_ws(int T, int d, int E, moe_dtype_t dt) {
+  return kStatusBytes + lb_bytes(E) + logit_scratch_bytes(T, d, E, dt) +
+         capacity_scratch_bytes(T, E);
 }
 
 moe_router_options_t default_options() {
@@ -105,6 +114,8 @@ moe_router_options_t default_options() {
   o.score_before_experts = 0;
   o.aux_loss = nullptr;
   o.aux_loss_coef = 0.0f;
+  o.capacity = 0;
+  o.topk_scores = nullptr;
   return o;
 }
 
@@ -120,6 +131,7 @@ moe_status_t check_router(const void* x, const void* w_router, const float* logi
                 top_k, kMaxTopK);
   MOE_CHECK_ARG(std::isfinite(o.route_scale) && o.route_scale != 0.0f,
                 "route_scale must be finite and non-zero");
+  MOE_CHECK_ARG(o.capacity >= 0, "capacity=%d must be >= 0", o.capacity);
   if (o.num_groups != 0) {
     MOE_CHECK_ARG(o.num_groups >= 1 && o.num_groups <= 32 && E % o.num_groups == 0,
                   "num_groups=%d must be in [1, 32] and divide E=%d", o.num_groups, E);
@@ -175,6 +187,7 @@ RouterOptions kernel_options(const moe_router_options_t& o) {
   k.bias = o.expert_bias;
   k.groups = o.num_groups;
   k.topk_groups = o.num_groups ? o.topk_groups : 0;
+  k.scores_out = o.topk_scores;
   return k;
 }
 
@@ -197,11 +210,21 @@ cudaError_t run_router(const void* x, const void* w_router, const float* logits_
                        void* scratch, int* status, cudaStream_t s,
                        const DispatchPlan* plan = nullptr, int32_t* blk = nullptr,
                        bool own_status = false) {
-  const RouterOptions ko = kernel_options(o);
+  RouterOptions ko = kernel_options(o);
   const int renorm = o.renormalize;
   float* tpe = o.tokens_per_expert;
   float* lb = o.aux_loss ? static_cast<float*>(scratch) : nullptr;
   float* part = reinterpret_cast<float*>(static_cast<char*>(scratch) + lb_bytes(E));
+  // The capacity policy ranks the copies by their scores, kept by the router
+  // (the caller's topk_scores or the scratch), and changes the routing after
+  // the router: the dispatch histogram is then the dispatch's own.
+  const bool cap = o.capacity > 0 && T > 0;
+  char* cap_scratch = static_cast<char*>(scratch) + lb_bytes(E) + logit_scratch_bytes(T, d, E, dt);
+  if (cap && !ko.scores_out) ko.scores_out = reinterpret_cast<float*>(cap_scratch);
+  if (cap) {
+    plan = nullptr;
+    blk = nullptr;
+  }
   cudaError_t e = cudaSuccess;
   if (lb) e = cudaMemsetAsync(lb, 0, 2 * sizeof(float) * E, s);
   const bool fused = router_is_fused(logits_in, T, d, E, o, dt, plan);
@@ -227,6 +250,16 @@ cudaError_t run_router(const void* x, const void* w_router, const float* logits_
         e = launch_router_topk(L, 1, T, E, top_k, renorm, ko, nullptr, topk_idx, topk_w, counts,
                                tpe, plan, blk, s, lb);
     }
+  }
+  // [PF] PaddleFormers moe_gate _probs_drop_policy; the counts then count
+  // the kept copies (tokens_per_expert and the load-balance statistics keep
+  // the routed ones: they measure the router, which the capacity then caps)
+  if (e == cudaSuccess && cap) {
+    unsigned long long* thr = reinterpret_cast<unsigned long long*>(
+        cap_scratch + align_up(static_cast<size_t>(T) * kMaxTopK * sizeof(float), 256));
+    e = launch_capacity_drop(topk_idx, topk_w, ko.scores_out, T, top_k, E, o.capacity, thr, s);
+    if (e == cudaSuccess && counts) e = cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, s);
+    if (e == cudaSuccess && counts) e = launch_expert_hist(topk_idx, 1LL * T * top_k, E, counts, s);
   }
   // [HP] _compute_load_balance_loss of this call (0 for no tokens)
   if (e == cudaSuccess && lb) e = launch_lb_loss(lb, E, T, top_k, o.aux_loss, s);
@@ -450,6 +483,10 @@ moe_status_t check_train(int T, int d, int E, int top_k, int h, const moe_router
                          moe_dtype_t dt) {
   if (dt != MOE_BF16) {
     set_last_error("training entry points: bf16 only");
+    return MOE_ERR_UNSUPPORTED;
+  }
+  if (o.capacity != 0) {
+    set_last_error("training entry points: no capacity policy");
     return MOE_ERR_UNSUPPORTED;
   }
   MOE_CHECK_ARG(T >= 0 && E >= 1 && E <= kMaxExperts && top_k >= 1 && top_k <= kMaxTopK &&
@@ -1247,6 +1284,10 @@ moe_status_t moe_forward_ex(const void* x, const void* w_router, const float* lo
     return st;
   const int N = T * top_k;
   if (moe_status_t st = check_swiglu_shape(N, d, h, E, dt)) return st;
+  if (o.capacity > 0 && (ep_ranks != 1 || dt != MOE_BF16)) {
+    set_last_error("moe_forward_ex: the capacity policy needs ep_ranks = 1 and bf16");
+    return MOE_ERR_UNSUPPORTED;
+  }
   MOE_CHECK_ARG(ep_ranks >= 1 && E % ep_ranks == 0 && E * ep_ranks <= kMaxBins &&
                     1LL * ep_ranks * E <= kMaxSegments,
                 "ep_ranks=%d must divide E with E*ep_ranks <= %d", ep_ranks, kMaxBins);
@@ -1270,7 +1311,9 @@ moe_status_t moe_forward_ex(const void* x, const void* w_router, const float* lo
   const int R = ep_ranks;
   cudaError_t e = cudaMemsetAsync(f.status, 0, sizeof(int), s);
   const DispatchPlan p = layer_dispatch_plan(T, d, E, top_k, R, dt);
-  // The router's top-k kernel also writes the dispatch histogram table.
+  // The router's top-k kernel also writes the dispatch histogram table,
+  // unless the capacity policy changes the routing after it.
+  const bool cap = o.capacity > 0;
   if (e == cudaSuccess)
     e = run_router(x, w_router, logits_in, T, d, E, top_k, o, dt, logits_out, idx, w, nullptr,
                    f.router_scratch, f.status, s, &p, static_cast<int32_t*>(f.disp_ws));
@@ -1285,7 +1328,7 @@ moe_status_t moe_forward_ex(const void* x, const void* w_router, const float* lo
   // weight and the combine below is unweighted.
   const bool before = o.score_before_experts != 0;
   e = launch_dispatch(p, x, idx, d, dt, cnt_a, f.offsets_a, f.src_row, f.dst_pos, f.x_a,
-                      f.disp_ws, f.status, s, /*hist_done=*/T > 0, before ? w : nullptr);
+                      f.disp_ws, f.status, s, /*hist_done=*/T > 0 && !cap, before ? w : nullptr);
   if (e != cudaSuccess) return cuda_status(e, "moe_forward/dispatch");
   const void* xe = f.x_a;
   const int32_t* off = f.offsets_a;
@@ -1299,7 +1342,13 @@ moe_status_t moe_forward_ex(const void* x, const void* w_router, const float* lo
     off = f.offsets_em;
     row_map = f.perm_inv;
   }
-  e = run_swiglu(xe, off, w1, w3, w2, nullptr, N, d, h, E, dt, f.y, f.H, f.status, s);
+  // with the capacity policy the kept copies fill the first offsets[E] < N
+  // slots
+  e = N == 0 ? cudaSuccess
+             : cap ? launch_swiglu_tc(xe, off, w1, w3, w2, nullptr, N, d, h, E, f.y, f.H,
+                                      f.status, s, /*rows_upto=*/true)
+                   : run_swiglu(xe, off, w1, w3, w2, nullptr, N, d, h, E, dt, f.y, f.H, f.status,
+                                s);
   if (e != cudaSuccess) return cuda_status(e, "moe_forward/grouped_swiglu");
   // [HP] MoE.forward: shared_expert(x_flat), added to the routed output in
   // the combine.

@@ -77,6 +77,8 @@ __device__ __forceinline__ float key_score(int k) { return __int_as_float(k ^ ((
 // Bin of a routed copy in the dispatch: the expert (R = 1), or on the
 // rank-major EP layout (destination rank g, source rank r = t / S, local
 // expert l) numbered (g * R + r) * L + l.
+// topk_idx value of a copy the capacity drop policy removed
+constexpr int kDroppedCopy = -1;
 __device__ __forceinline__ int dispatch_key(int e, int t, int R, int L, int S) {
   if (R == 1) return e;
   const int g = e / L, l = e - g * L, r = t / S;

@@ -98,6 +98,9 @@ struct RouterOptions {
   const float* bias = nullptr;
   int groups = 0;
   int topk_groups = 0;
+  // [T, k] or null: the score of each selected expert before renormalisation
+  // and scale (the key of the capacity drop policy)
+  float* scores_out = nullptr;
 };
 
 // Sum of `nsplit` partial logit arrays [nsplit, T, E] (in split order), then
@@ -163,6 +166,13 @@ cudaError_t launch_router_backward(const float* logits, const int32_t* topk_idx,
                                    int renorm, float scale, float* dz32, void* dz16,
                                    cudaStream_t s, const int32_t* lb_counts = nullptr,
                                    float lb_scale = 0.f);
+// Capacity drop policy: for every expert with more than `capacity` routed
+// copies, keep the `capacity` of them with the highest score (scores [T, k],
+// the router's scores_out), equal scores to the lower token; the others get
+// topk_idx = -1 and topk_w = 0.  thr is device scratch for E 64-bit keys.
+cudaError_t launch_capacity_drop(int32_t* topk_idx, float* topk_w, const float* scores, int T,
+                                 int k, int E, int capacity, unsigned long long* thr,
+                                 cudaStream_t s);
 // counts [E] += histogram of idx [n] (counts cleared by the caller).
 cudaError_t launch_expert_hist(const int32_t* idx, long long n, int E, int32_t* counts,
                                cudaStream_t s);
@@ -188,10 +198,12 @@ cudaError_t launch_single_segment(int32_t* offsets, int n, cudaStream_t s);
 
 // ---- grouped SwiGLU -----------------------------------------------------
 // bf16 tcgen05 path: H (bf16 [N, h]) is scratch.
+// rows_upto: offsets[E] may be below N (the rows past it are dropped copies
+// and stay uncomputed).
 cudaError_t launch_swiglu_tc(const void* x_perm, const int32_t* offsets, const void* w1,
                              const void* w3, const void* w2, const float* row_scale, int N,
                              int d, int h, int E, void* y, void* H, int* status,
-                             cudaStream_t s);
+                             cudaStream_t s, bool rows_upto = false);
 // Same with GEMM1's rows read from x [T, d] through src_row [N] (TMA gather4).
 cudaError_t launch_swiglu_tc_gather(const void* x, int T, const int32_t* src_row,
                                     const int32_t* offsets, const void* w1, const void* w3,

@@ -40,7 +40,7 @@ __global__ void dispatch_hist_kernel(const int32_t* __restrict__ idx, int T, int
   for (long long f = f0 + threadIdx.x; f < f1; f += blockDim.x) {
     const int e = idx[f];
     if (static_cast<unsigned>(e) >= static_cast<unsigned>(E)) {
-      bad = 1;
+      bad |= e != kDroppedCopy;   // a copy the capacity policy dropped is no error
       continue;
     }
     atomicAdd(&hist[dispatch_key(e, static_cast<int>(f / k), R, L, S)], 1);
@@ -746,6 +746,101 @@ cudaError_t launch_router_backward(const float* logits, const int32_t* topk_idx,
   return cudaGetLastError();
 }
 
+// ------------------------------------------------------- capacity drop
+// [PF] PaddleFormers moe_gate.py, _probs_drop_policy: a token keeps its
+// assignment to an expert when it is routed there and its score is among the
+// top `capacity` scores for that expert (ranked over the expert's routed
+// copies; equal scores to the lower token).  Every copy gets a unique 64-bit
+// key, (score, then the token reversed), and one block per expert finds the
+// capacity-th largest key of its copies by an 8-bit radix select over the
+// flat copy list (eight passes); the copies below it are dropped.
+__device__ __forceinline__ unsigned long long capacity_key(float s, int t) {
+  const unsigned hi = static_cast<unsigned>(score_key(s != s ? -INFINITY : s)) ^ 0x80000000u;
+  return (static_cast<unsigned long long>(hi) << 32) | (0xFFFFFFFFu - static_cast<unsigned>(t));
+}
+
+__global__ void __launch_bounds__(512) capacity_select_kernel(
+    const int32_t* __restrict__ idx, const float* __restrict__ scores, long long n, int k,
+    int capacity, unsigned long long* __restrict__ thr) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ unsigned hist[256];
+  __shared__ unsigned long long prefix_s;
+  __shared__ int want_s, count_s;
+  const int e = blockIdx.x;
+  if (threadIdx.x == 0) count_s = 0;
+  __syncthreads();
+  int mine = 0;
+  for (long long i = threadIdx.x; i < n; i += blockDim.x) mine += idx[i] == e;
+  atomicAdd(&count_s, mine);
+  __syncthreads();
+  const int count = count_s;
+  if (count <= capacity) {   // nothing to drop: keep every key
+    if (threadIdx.x == 0) thr[e] = 0ull;
+    return;
+  }
+  if (threadIdx.x == 0) {
+    prefix_s = 0ull;
+    want_s = capacity;   // rank (1 = largest) of the key wanted among those left
+  }
+  for (int shift = 56; shift >= 0; shift -= 8) {
+    for (int b = threadIdx.x; b < 256; b += blockDim.x) hist[b] = 0;
+    __syncthreads();
+    const unsigned long long prefix = prefix_s;
+    const unsigned long long hi_mask = shift == 56 ? 0ull : ~0ull << (shift + 8);
+    for (long long i = threadIdx.x; i < n; i += blockDim.x) {
+      if (idx[i] != e) continue;
+      const unsigned long long key = capacity_key(scores[i], static_cast<int>(i / k));
+      if ((key & hi_mask) == (prefix & hi_mask))
+        atomicAdd(&hist[(key >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int want = want_s, cum = 0;
+      for (int b = 255; b >= 0; --b) {
+        const int c = static_cast<int>(hist[b]);
+        if (cum + c >= want) {
+          prefix_s = prefix | (static_cast<unsigned long long>(b) << shift);
+          want_s = want - cum;
+          break;
+        }
+        cum += c;
+      }
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) thr[e] = prefix_s;   // the capacity-th largest key: keep keys >= it
+}
+
+__global__ void capacity_apply_kernel(int32_t* __restrict__ idx, float* __restrict__ w,
+                                      const float* __restrict__ scores, long long n, int k, int E,
+                                      const unsigned long long* __restrict__ thr) {
+  pdl_wait();
+  pdl_trigger();
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int e = idx[i];
+    if (static_cast<unsigned>(e) >= static_cast<unsigned>(E)) continue;
+    const unsigned long long t = thr[e];
+    if (t && capacity_key(scores[i], static_cast<int>(i / k)) < t) {
+      idx[i] = kDroppedCopy;
+      w[i] = 0.f;
+    }
+  }
+}
+
+cudaError_t launch_capacity_drop(int32_t* topk_idx, float* topk_w, const float* scores, int T,
+                                 int k, int E, int capacity, unsigned long long* thr,
+                                 cudaStream_t s) {
+  const long long n = 1LL * T * k;
+  if (n == 0) return cudaSuccess;
+  launch_k(capacity_select_kernel, dim3(E), dim3(512), 0, s, topk_idx, scores, n, k, capacity, thr);
+  const int blocks = static_cast<int>(std::min<long long>((n + 255) / 256, 8LL * num_sms()));
+  launch_k(capacity_apply_kernel, dim3(blocks), dim3(256), 0, s, topk_idx, topk_w, scores, n, k,
+           E, static_cast<const unsigned long long*>(thr));
+  return cudaGetLastError();
+}
+
 // counts[e] += number of entries of idx [n] equal to e (entries outside
 // [0, E) skipped); counts cleared by the caller.
 __global__ void expert_hist_kernel(const int32_t* __restrict__ idx, long long n, int E,
@@ -1220,6 +1315,7 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
       topk_idx[o] = my_e;
       const float wout = wx / (renorm ? sel : den) * opt.scale;
       topk_w[o] = wout;
+      if (opt.scores_out) opt.scores_out[o] = wx / den;
       if (blk) atomicAdd(&dbins[dispatch_key(my_e, t, R, L, S)], 1);
       if (tally_e) atomicAdd(&ebins[my_e], 1);
       if (lb) atomicAdd(&wsum[my_e], wout);

@@ -350,6 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float wv = wx / (a.renorm ? sel : den) * opt.scale;
         a.topk_idx[o] = me;
         a.topk_w[o] = wv;
+        if (opt.scores_out) opt.scores_out[o] = wx / den;
         tok_e[it * k + lane] = me;
         atomicAdd(&ebins[me], 1);
         if (a.lb) atomicAdd(&wsum[me], wv);

@@ -91,6 +91,9 @@ struct Args {
   // pair_head): 0 all of them, 1 the head (CTA-pair launch), 2 the tail
   // (single-CTA launch).
   int seg_part;
+  // Grouped launches: offsets[E] may be below M (rows past it are copies the
+  // capacity policy dropped, left uncomputed); else it must equal M.
+  int rows_upto;
   // GEMM2 with the combine folded in (CTA-pair kernel): output row s is
   // scaled by comb_w[s] and added into comb_out[comb_tok[s]] with fp32
   // reductions instead of being stored
@@ -246,7 +249,7 @@ struct GroupedSched {
       bad = __any_sync(0xffffffffu, bad);
       const int total = __shfl_sync(0xffffffffu, incl, 31);
       if (lane == 0) {
-        bad |= (off[0] != 0) || (off[E] != a.M);
+        bad |= (off[0] != 0) || (a.rows_upto ? off[E] > a.M : off[E] != a.M);
         cum[E] = total;
         sched[0] = bad ? 0 : total;
         sched[1] = nt;
@@ -747,7 +750,7 @@ struct PairSched : GroupedSched<256, NUM_B_, NCOLS, 256> {
       bad = __any_sync(0xffffffffu, bad);
       const int total = __shfl_sync(0xffffffffu, incl, 31);
       if (lane == 0) {
-        bad |= (off[0] != 0) || (off[E] != a.M);
+        bad |= (off[0] != 0) || (a.rows_upto ? off[E] > a.M : off[E] != a.M);
         cum[E] = total;
         sched[0] = bad ? 0 : total;
         sched[1] = nt;
@@ -887,7 +890,7 @@ struct WgradPolicy {
       for (int e = threadIdx.x; e < E; e += 32) bad |= off[e + 1] < off[e];
       bad = __any_sync(0xffffffffu, bad);
       if (threadIdx.x == 0) {
-        bad |= (off[0] != 0) || (off[E] != a.M);
+        bad |= (off[0] != 0) || (a.rows_upto ? off[E] > a.M : off[E] != a.M);
         const int mt = cdiv(a.Ma, BM), nt = cdiv(a.n_out, BN);
         sched[0] = bad ? 0 : E * mt * nt;
         sched[1] = mt;
@@ -1766,14 +1769,15 @@ static cudaError_t swiglu_tc_impl(const void* a_src, int a_rows, const int32_t* 
                                   const int32_t* offsets, const void* w1, const void* w3,
                                   const void* w2, const float* row_scale, int N, int d, int h,
                                   int E, void* y, void* H, int* status, cudaStream_t s,
-                                  void* gu = nullptr, const FoldedCombine* fold = nullptr);
+                                  void* gu = nullptr, const FoldedCombine* fold = nullptr,
+                                  bool rows_upto = false);
 
 cudaError_t launch_swiglu_tc(const void* x_perm, const int32_t* offsets, const void* w1,
                              const void* w3, const void* w2, const float* row_scale, int N,
                              int d, int h, int E, void* y, void* H, int* status,
-                             cudaStream_t s) {
+                             cudaStream_t s, bool rows_upto) {
   return swiglu_tc_impl(x_perm, N, nullptr, offsets, w1, w3, w2, row_scale, N, d, h, E, y, H,
-                        status, s);
+                        status, s, nullptr, nullptr, rows_upto);
 }
 
 cudaError_t launch_swiglu_tc_gather(const void* x, int T, const int32_t* src_row,
@@ -1800,7 +1804,7 @@ static cudaError_t swiglu_tc_impl(const void* a_src, int a_rows, const int32_t* 
                                   const int32_t* offsets, const void* w1, const void* w3,
                                   const void* w2, const float* row_scale, int N, int d, int h,
                                   int E, void* y, void* H, int* status, cudaStream_t s,
-                                  void* gu, const FoldedCombine* fold) {
+                                  void* gu, const FoldedCombine* fold, bool rows_upto) {
   using namespace tc;
   CUtensorMap tx, t1, t3, th, t2;
   const bool gather = src_row != nullptr;
@@ -1821,6 +1825,7 @@ static cudaError_t swiglu_tc_impl(const void* a_src, int a_rows, const int32_t* 
   a.E = E;
   a.offsets = offsets;
   a.status = status;
+  a.rows_upto = rows_upto ? 1 : 0;
   // GEMM1: H = silu(x w1^T) * (x w3^T)
   a.K = d;
   a.n_out = h;

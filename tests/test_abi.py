@@ -207,10 +207,32 @@ def test_router_options_defaults(L):
     o.route_scale = 7.0
     o.num_groups = 3
     o.aux_loss_coef = 2.0
+    o.capacity = 5
+    o.topk_scores = 64
     L.moe_router_options_init(ctypes.byref(o))
     assert (o.score, o.renormalize, o.route_scale, o.expert_bias, o.num_groups, o.topk_groups,
-            o.tokens_per_expert, o.score_before_experts, o.aux_loss, o.aux_loss_coef) == \
-        (0, 0, 1.0, None, 0, 0, None, 0, None, 0.0)
+            o.tokens_per_expert, o.score_before_experts, o.aux_loss, o.aux_loss_coef,
+            o.capacity, o.topk_scores) == (0, 0, 1.0, None, 0, 0, None, 0, None, 0.0, 0, None)
+
+
+def test_capacity_rules(L):
+    """A negative capacity is rejected; the layer forward takes the capacity
+    policy only in bf16 with ep_ranks = 1, the training forward not at all
+    (all before any launch)."""
+    import routing_dispatch_grouped_topk_b200 as m
+    o = m.RouterOptions()
+    L.moe_router_options_init(ctypes.byref(o))
+    p = ctypes.c_void_p(256)
+    o.capacity = -1
+    assert L.moe_router_topk_ex(p, p, None, 4, 64, 8, 2, ctypes.byref(o), 1, None, p, p, None, p,
+                                1 << 20, None) == 1
+    o.capacity = 3
+    assert L.moe_forward_ex(p, p, None, p, p, p, 4, 64, 8, 2, 64, ctypes.byref(o), None, 2, 1, p,
+                            None, None, None, None, p, 1 << 30, None) == 2
+    assert L.moe_forward_ex(p, p, None, p, p, p, 4, 64, 8, 2, 64, ctypes.byref(o), None, 1, 0, p,
+                            None, None, None, None, p, 1 << 30, None) == 2
+    assert L.moe_forward_train(p, p, None, p, p, p, 4, 64, 8, 2, 64, ctypes.byref(o), 1, p, p,
+                               1 << 30, None) == 2
 
 
 def test_shared_expert_workspace_and_checks(L):

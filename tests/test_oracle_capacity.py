@@ -1,4 +1,4 @@
-"""Pins of the oracle's capacity drop policy ([P4] PaddleFormers moe_gate.py,
+"""Pins of the oracle's capacity drop policy ([PF] PaddleFormers moe_gate.py,
 _probs_drop_policy) and of the dispatch and combine of dropped copies.
 
 Pins that do not restate the oracle's sort:
