@@ -12,10 +12,10 @@
 // (st.shared::cluster), and the owner adds the C partials in rank order (a
 // fixed order: the logits do not depend on timing or on the grid; each
 // warp stages its rows so that the remote stores write whole 128-byte row
-// pieces).  One warp per owned token (all six warps of the CTA) then
-// selects the k winners with k rounds of a warp
-// arg-max (two redux.sync reductions on (key, expert): descending key, ties
-// to the lower expert index) and writes the indices and weights; in the
+// pieces).  The owner's 128 epilogue threads, C per token, then select the
+// k winners (sorted register lists of each thread's experts merged by k
+// shuffle arg-max rounds: descending key, ties to the lower expert index)
+// and write the indices and weights; in the
 // layer forward the CTA also writes the dispatch histogram of its token
 // blocks.  The expert counts of the entry
 // point go through a per-CTA table that a second small kernel sums.  The
@@ -82,6 +82,203 @@ __device__ __forceinline__ void st_cluster_v4(uint32_t addr, uint32_t a, uint32_
 __device__ __forceinline__ void bar_epi() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 // floats of one epilogue warp's 32 x 32 staging tile of the exchange (padded rows)
 constexpr int kXchgTile = 32 * 33;
+
+// Sorted list of the KM largest (key, expert) pairs a thread has seen, key
+// descending; a thread meets its experts in ascending order, so an equal key
+// never displaces an entry (ties go to the lower expert).
+template <int KM>
+__device__ __forceinline__ void topk_insert(int (&kk)[KM], int (&ee)[KM], float (&vv)[KM], int key,
+                                            int e, float v) {
+  if (key <= kk[KM - 1]) return;
+#pragma unroll
+  for (int j = KM - 1; j >= 0; --j) {
+    if (kk[j] < key) {
+      if (j > 0 && kk[j - 1] < key) {
+        kk[j] = kk[j - 1];
+        ee[j] = ee[j - 1];
+        vv[j] = vv[j - 1];
+      } else {
+        kk[j] = key;
+        ee[j] = e;
+        vv[j] = v;
+      }
+    }
+  }
+}
+
+// Logits of experts 4j .. 4j+3 of a token: its C partial rows (rank r at
+// row + r rstride) added in rank order.
+__device__ __forceinline__ float4 partial_sum4(const float* row, size_t rstride, int C, int j) {
+  float4 z = *reinterpret_cast<const float4*>(row + 4 * j);
+  for (int r = 1; r < C; ++r) {
+    const float4 q = *reinterpret_cast<const float4*>(row + r * rstride + 4 * j);
+    z.x += q.x;
+    z.y += q.y;
+    z.z += q.z;
+    z.w += q.w;
+  }
+  return z;
+}
+
+__device__ __forceinline__ float f4_at(const float4& v, int c) {
+  return c == 0 ? v.x : c == 1 ? v.y : c == 2 ? v.z : v.w;
+}
+
+// Scores, top-k and weights of the tokens a CTA owns, on its 128 epilogue
+// threads: G = 128 / own threads per token (G = C), thread g taking the
+// expert quads g, g + G, ... of the token's row.  Each thread keeps the KM
+// best (key, expert) pairs of its experts; k rounds of a G-way arg-max
+// (xor shuffles on (key descending, expert ascending)) merge them.  The
+// partial-logit rows are read as 16-byte vectors; the row pitch
+// (4 G mod 32 floats) puts the eight threads of each load phase on distinct
+// banks.  Arithmetic: z = partials in rank order; max and denominator over
+// the experts of a thread in ascending order, then across the G threads by
+// the xor butterfly; the renormalising sum over the winners in rank order.
+template <int KM>
+__device__ __forceinline__ void score_owned(const Args& a, const float* recv, int own, int C,
+                                            int t_own0, int* tok_e, float* tok_w, int* ebins,
+                                            float* wsum) {
+  const int i = static_cast<int>(threadIdx.x) - 64;
+  const int G = BM / own;
+  const int it = i / G, g = i - it * G;
+  const int t = t_own0 + it;
+  const bool live = t < a.T;   // the G threads of a token agree; every thread takes part
+  const int E = a.E, k = a.k;
+  const RouterOptions& opt = a.opt;
+  const bool on_logits = opt.bias == nullptr && opt.scale > 0.f;
+  const size_t rstride = static_cast<size_t>(own) * a.pitch;
+  const float* row = recv + static_cast<size_t>(it) * a.pitch;
+  const int nq = (E + 3) >> 2;
+
+  // Softmax scores as keys (bias or a non-positive scale): the maximum and
+  // the denominator first.
+  float mx = -INFINITY, den = 1.f;
+  if (!on_logits && !opt.sigmoid) {
+    for (int j = g; j < nq; j += G) {
+      const float4 z4 = partial_sum4(row, rstride, C, j);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const float z = f4_at(z4, c);
+        if (4 * j + c < E && z == z) mx = fmaxf(mx, z);
+      }
+    }
+    for (int sh = 1; sh < G; sh <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, sh));
+    float dn = 0.f;
+    for (int j = g; j < nq; j += G) {
+      const float4 z4 = partial_sum4(row, rstride, C, j);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float z = f4_at(z4, c);
+        if (z != z) z = -INFINITY;
+        if (4 * j + c < E) dn += expf(z - mx);
+      }
+    }
+    for (int sh = 1; sh < G; sh <<= 1) dn += __shfl_xor_sync(0xffffffffu, dn, sh);
+    den = dn;
+  }
+
+  // selection: every expert of the thread into its sorted list; a winner
+  // carries its logit (keys on the logits) or its score
+  int kk[KM], ee[KM];
+  float vv[KM];
+#pragma unroll
+  for (int q = 0; q < KM; ++q) {
+    kk[q] = INT_MIN;
+    ee[q] = INT_MAX;
+    vv[q] = 0.f;
+  }
+  for (int j = g; j < nq; j += G) {
+    const float4 z4 = partial_sum4(row, rstride, C, j);
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      const int e = 4 * j + c;
+      if (e >= E) break;
+      float z = f4_at(z4, c);
+      if (a.logits_out && live) a.logits_out[static_cast<size_t>(t) * E + e] = z;
+      if (z != z) z = -INFINITY;
+      float kv = z, v = z;
+      if (!on_logits) {
+        v = opt.sigmoid ? 1.0f / (1.0f + expf(-z)) : expf(z - mx);
+        kv = v / den * opt.scale;
+        if (opt.bias) {
+          kv += opt.bias[e];
+          if (kv != kv) kv = -INFINITY;
+        }
+      }
+      topk_insert<KM>(kk, ee, vv, score_key(kv), e, v);
+    }
+  }
+
+  // merge: round r takes the best head of the G lists and pops it; the
+  // winner's expert goes to tok_e and its unbiased score to tok_w (with keys
+  // on the logits: the softmax numerator exp(z - max z), max z being the
+  // first winner's logit, or sigmoid(z)); sel sums them in round order
+  float sel = 0.f;
+  for (int r = 0; r < k; ++r) {
+    int bk = kk[0], be = ee[0];
+    float bv = vv[0];
+    for (int sh = 1; sh < G; sh <<= 1) {
+      const int ok = __shfl_xor_sync(0xffffffffu, bk, sh);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, sh);
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, sh);
+      if (ok > bk || (ok == bk && oe < be)) {
+        bk = ok;
+        be = oe;
+        bv = ov;
+      }
+    }
+    if (ee[0] == be) {
+#pragma unroll
+      for (int q = 0; q + 1 < KM; ++q) {
+        kk[q] = kk[q + 1];
+        ee[q] = ee[q + 1];
+        vv[q] = vv[q + 1];
+      }
+      kk[KM - 1] = INT_MIN;
+      ee[KM - 1] = INT_MAX;
+    }
+    if (on_logits) {
+      if (r == 0) mx = bv;
+      bv = opt.sigmoid ? 1.0f / (1.0f + expf(-bv)) : expf(bv - mx);
+    }
+    sel += bv;
+    if (g == 0) {
+      tok_e[it * k + r] = be;
+      tok_w[it * k + r] = bv;
+    }
+  }
+  // softmax with keys on the logits: the denominator when it is asked for
+  if (on_logits && !opt.sigmoid && (!a.renorm || opt.scores_out)) {
+    float dn = 0.f;
+    for (int j = g; j < nq; j += G) {
+      const float4 z4 = partial_sum4(row, rstride, C, j);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float z = f4_at(z4, c);
+        if (z != z) z = -INFINITY;
+        if (4 * j + c < E) dn += expf(z - mx);
+      }
+    }
+    for (int sh = 1; sh < G; sh <<= 1) dn += __shfl_xor_sync(0xffffffffu, dn, sh);
+    den = dn;
+  }
+  __syncwarp();
+  // weights: the winners' scores (renormalised), times the scale; thread g
+  // writes the winners r = g, g + G, ...
+  if (live) {
+    for (int r = g; r < k; r += G) {
+      const size_t o = static_cast<size_t>(t) * k + r;
+      const int e = tok_e[it * k + r];
+      const float wx = tok_w[it * k + r];
+      const float wv = wx / (a.renorm ? sel : den) * opt.scale;
+      a.topk_idx[o] = e;
+      a.topk_w[o] = wv;
+      if (opt.scores_out) opt.scores_out[o] = wx / den;
+      atomicAdd(&ebins[e], 1);
+      if (a.lb) atomicAdd(&wsum[e], wv);
+    }
+  }
+}
 
 template <int BN>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -244,118 +441,28 @@ __global__ void __launch_bounds__(kThreads, 1)
   cluster_sync_all();
 
   // --------------------------------------------------- scores and top-k
-  // One warp per owned token (all six warps, each taking every sixth):
-  // lane l holds experts l, l + 32, ... (EPL of them), adds the C partials
-  // in rank order, and the k winners come from k rounds of a warp arg-max
-  // on (key descending, expert ascending) -- two redux.sync reductions each.
-  constexpr int EPL = BN / 32;
+  // The 128 epilogue threads score the owned tokens (score_owned); warps 0
+  // and 1 wait at the barrier below.
   const int i = threadIdx.x - 64;                 // epilogue threads: 0..127
   const int E = a.E, k = a.k;
-  const RouterOptions& opt = a.opt;
   int* dbins = reinterpret_cast<int*>(smem + align_up(static_cast<size_t>(BM) * pitch * 4, 16));
   int* ebins = dbins + (a.blk ? a.nbins : 0);
   float* wsum = reinterpret_cast<float*>(ebins + E);
   int* tok_e = reinterpret_cast<int*>(wsum + E);   // [own][k] winners, for the histograms
+  float* tok_w = reinterpret_cast<float*>(tok_e + BM * kMaxTopK);   // [own][k] their scores
   const int t_own0 = tile * BM + rank * own;
   for (int e = threadIdx.x; e < E; e += kThreads) {
     ebins[e] = 0;
     wsum[e] = 0.f;
   }
   __syncthreads();
-  {
-    const bool on_logits = opt.bias == nullptr && opt.scale > 0.f;
-    const size_t sstride = static_cast<size_t>(own) * pitch;
-    for (int it = warp; it < own; it += kThreads / 32) {
-      const int t = t_own0 + it;
-      if (t >= a.T) break;                        // warp-uniform
-      const float* rp = recv + static_cast<size_t>(it) * pitch + lane;
-      float sv[EPL];
-      bool avail[EPL];
-#pragma unroll
-      for (int q = 0; q < EPL; ++q) {
-        avail[q] = lane + 32 * q < E;
-        float z = 0.f;
-        if (avail[q]) {
-          z = rp[32 * q];
-          for (int sc = 1; sc < C; ++sc) z += rp[sc * sstride + 32 * q];   // ranks in order
-        }
-        sv[q] = z;
-      }
-      float mx = -INFINITY;
-#pragma unroll
-      for (int q = 0; q < EPL; ++q) {
-        if (avail[q] && a.logits_out) a.logits_out[static_cast<size_t>(t) * E + lane + 32 * q] = sv[q];
-        if (sv[q] != sv[q]) sv[q] = -INFINITY;
-        if (avail[q]) mx = fmaxf(mx, sv[q]);
-      }
-      // ex = exp(z - max z) (softmax numerators) or sigmoid(z); s = ex / den
-      float ex[EPL];
-      float den = 1.f;
-      if (opt.sigmoid) {
-#pragma unroll
-        for (int q = 0; q < EPL; ++q) ex[q] = avail[q] ? 1.0f / (1.0f + expf(-sv[q])) : 0.f;
-      } else {
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1)
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-        den = 0.f;
-#pragma unroll
-        for (int q = 0; q < EPL; ++q) {
-          ex[q] = avail[q] ? expf(sv[q] - mx) : 0.f;
-          den += ex[q];
-        }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
-      }
-      int key[EPL];
-#pragma unroll
-      for (int q = 0; q < EPL; ++q) {
-        float kv = on_logits ? sv[q] : ex[q] / den * opt.scale;
-        if (opt.bias && avail[q]) {
-          kv += opt.bias[lane + 32 * q];
-          if (kv != kv) kv = -INFINITY;
-        }
-        key[q] = score_key(kv);
-      }
-      int me = 0;
-      float mxv = 0.f;
-      for (int j = 0; j < k; ++j) {
-        int lk = INT_MIN, li = 0x7fffffff;
-        float lx = 0.f;
-#pragma unroll
-        for (int q = 0; q < EPL; ++q)
-          if (avail[q] && key[q] > lk) {   // experts of a lane ascend with q: first max wins
-            lk = key[q];
-            li = lane + 32 * q;
-            lx = ex[q];
-          }
-        const int mk = __reduce_max_sync(0xffffffffu, lk);
-        const int be = __reduce_min_sync(0xffffffffu, lk == mk ? li : 0x7fffffff);
-        const float bx = __shfl_sync(0xffffffffu, lx, be & 31);
-#pragma unroll
-        for (int q = 0; q < EPL; ++q)
-          if (lane + 32 * q == be) avail[q] = false;
-        if (lane == j) {
-          me = be;
-          mxv = bx;
-        }
-      }
-      // weights: the unbiased score of each winner (renormalised), times the scale
-      const float wx = lane < k ? mxv : 0.f;
-      float sel = wx;
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) sel += __shfl_xor_sync(0xffffffffu, sel, off);
-      if (lane < k) {
-        const size_t o = static_cast<size_t>(t) * k + lane;
-        const float wv = wx / (a.renorm ? sel : den) * opt.scale;
-        a.topk_idx[o] = me;
-        a.topk_w[o] = wv;
-        if (opt.scores_out) opt.scores_out[o] = wx / den;
-        tok_e[it * k + lane] = me;
-        atomicAdd(&ebins[me], 1);
-        if (a.lb) atomicAdd(&wsum[me], wv);
-      }
-    }
+  if (warp >= 2) {
+    if (a.k <= 4)
+      score_owned<4>(a, recv, own, C, t_own0, tok_e, tok_w, ebins, wsum);
+    else if (a.k <= 8)
+      score_owned<8>(a, recv, own, C, t_own0, tok_e, tok_w, ebins, wsum);
+    else
+      score_owned<16>(a, recv, own, C, t_own0, tok_e, tok_w, ebins, wsum);
   }
   __syncthreads();   // the winners of every owned token are in tok_e
   if (warp >= 2) {
@@ -451,7 +558,9 @@ RouterFusedPlan router_fused_plan(int T, int d, int E, const DispatchPlan* plan)
   p.bn = E <= 32 ? 32 : E <= 64 ? 64 : E <= 128 ? 128 : 256;
   p.tiles = std::max(1, cdiv(T, rtc::BM));
   p.kb_total = std::max(1, cdiv(d, rtc::BK));
-  p.pitch = (E + 31) / 32 * 32 + 4;
+  // the row pitch is (E rounded up to 32) + 4 C mod 32 floats (conflict-free
+  // 16-byte reads in score_owned); the memory is sized for the widest one
+  const int pitch_max = (E + 31) / 32 * 32 + 16;
   // shared memory: the stages, or after the K loop the partial logits of the
   // cluster, the dispatch bins and the expert bins, whichever is larger
   int stages = 0, tail = 0;
@@ -463,12 +572,12 @@ RouterFusedPlan router_fused_plan(int T, int d, int E, const DispatchPlan* plan)
   }
   // (during the exchange the four epilogue warps' staging tiles sit where
   // the bins go afterwards)
-  const size_t recv = align_up(static_cast<size_t>(rtc::BM) * p.pitch * 4, 16);
+  const size_t recv = align_up(static_cast<size_t>(rtc::BM) * pitch_max * 4, 16);
   const size_t exch = recv + std::max<size_t>(
                                  4 * rtc::kXchgTile * 4,
                                  (plan ? static_cast<size_t>(plan->nbins) * 4 : 0) +
                                      8 * static_cast<size_t>(E) +
-                                     static_cast<size_t>(rtc::BM) * kMaxTopK * 4);
+                                     static_cast<size_t>(rtc::BM) * kMaxTopK * 8);
   p.region = static_cast<int>(align_up(std::max<size_t>(stages, exch), 1024));
   p.smem = p.region + tail + 1024;   // + slack for the 1 KB alignment
   // two CTAs per SM when they fit (228 KB per SM, 1 KB reserved per CTA)
@@ -482,6 +591,7 @@ RouterFusedPlan router_fused_plan(int T, int d, int E, const DispatchPlan* plan)
   while (C < 8 && p.tiles * C * 2 <= per_sm * kRouterTargetTiles && 2 * C <= p.kb_total) C *= 2;
   while (C > 1 && (C - 1) * cdiv(p.kb_total, C) >= p.kb_total) C /= 2;
   p.C = C;
+  p.pitch = (E + 31) / 32 * 32 + (4 * C) % 32;
   p.kb_per_cta = cdiv(p.kb_total, C);
   p.grid = p.tiles * C;
   p.ok = p.smem <= 227 * 1024 && (!plan || rtc::BM / C >= plan->tb);
