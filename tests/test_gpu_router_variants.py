@@ -74,8 +74,9 @@ def on_logits(opts):
     return opts.get("expert_bias") is None and opts.get("route_scale", 1.0) > 0
 
 
-def check_router(gi, gw, L, k, renorm, opts):
-    """GPU (gi, gw) against the oracle on fp32 logits L [T, E]."""
+def check_router(gi, gw, L, k, renorm, opts, min_sure=0.8):
+    """GPU (gi, gw) against the oracle on fp32 logits L [T, E]; at least
+    ``min_sure`` of the tokens must have a top-k the margin decides."""
     T, E = L.shape
     L64 = O.as_f64(L)
     idx, w, _, _ = O.router_topk_general(k, logits=L, renormalize=renorm, **opts)
@@ -95,7 +96,7 @@ def check_router(gi, gw, L, k, renorm, opts):
             tg = opts["topk_groups"]
             if tg < G:
                 sure &= (gmax[:, tg - 1] - gmax[:, tg]) > margin
-        assert sure.mean() > 0.8, sure.mean()
+        assert sure.mean() > min_sure, sure.mean()
         assert np.array_equal(gi[sure], idx[sure])
         # elsewhere: distinct experts whose keys reach the k-th key within the margin
         for t in np.nonzero(~sure)[0]:
@@ -317,3 +318,36 @@ def test_load_balance_loss_in_forward_and_empty(M):
     L0 = torch.zeros(0, 16, device="cuda")
     M.router_topk(logits_in=L0, top_k=2, aux_loss=aux)
     assert aux.item() == 0.0
+
+
+# Shapes that put the fused tcgen05 router on each cluster size C (= threads
+# per token in its scoring): (T, d, E, k) -> C = 8, 4, 2, 1; E not a multiple
+# of 4 and k = 1 / 16 included.
+FUSED_SHAPES = [(200, 1024, 61, 5), (2500, 512, 130, 16), (3000, 128, 37, 3), (129, 64, 255, 1)]
+FUSED_VARIANTS = [dict(), VARIANTS[0], VARIANTS[2], VARIANTS[5], VARIANTS[7]]
+
+
+@pytest.mark.parametrize("T,d,E,k", FUSED_SHAPES)
+@pytest.mark.parametrize("vi", range(len(FUSED_VARIANTS)))
+@pytest.mark.parametrize("renorm", [False, True])
+def test_fused_router_options(M, T, d, E, k, vi, renorm):
+    """The fused router (bf16 gate, no groups) with the options: indices and
+    weights against the oracle's general router on the GPU's own fp32
+    logits, and the selected experts' unbiased scores (topk_scores)."""
+    g = torch.Generator().manual_seed(T + d + E + k)
+    x = torch.randn(T, d, generator=g).to(torch.bfloat16).cuda()
+    wr = (torch.randn(E, d, generator=g) * (2.0 / d ** 0.5)).to(torch.bfloat16).cuda()
+    o, go = materialize(dict(FUSED_VARIANTS[vi]), E, seed=vi)
+    sc = torch.empty(T, k, dtype=torch.float32, device="cuda")
+    gi, gw, gc, logits, ws = M.router_topk(x, wr, k, renorm, want_logits=True, topk_scores=sc,
+                                           **go)
+    torch.cuda.synchronize()
+    assert M.device_status(ws) == 0
+    gi = gi.cpu().numpy()
+    L = logits.cpu().numpy()
+    # A negative scale selects the smallest scores: their gaps fall below the
+    # margin (which scales with the token's largest key) more often.
+    check_router(gi, gw.cpu(), L, k, renorm, o, min_sure=0.5 if o.get("route_scale", 1) < 0 else 0.8)
+    assert np.array_equal(gc.cpu().numpy(), np.bincount(gi.ravel(), minlength=E))
+    s, _, _ = oracle_keys(O.as_f64(L), o)
+    close(sc.cpu(), np.take_along_axis(s, gi.astype(np.int64), axis=1), torch.float32)
