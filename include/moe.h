@@ -89,7 +89,9 @@ typedef enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID = 1 } moe_score_t;
 /* Bits of the device status word. */
 #define MOE_DEV_BAD_EXPERT 1   /* dispatch: expert id outside [0, E)            */
 #define MOE_DEV_BAD_COUNTS 2   /* regroup: counts negative or not summing to rows */
-#define MOE_DEV_BAD_OFFSETS 4  /* grouped_swiglu: offsets not 0..N non-decreasing */
+#define MOE_DEV_BAD_OFFSETS 4  /* grouped_swiglu: offsets not 0..N non-decreasing;
+                                  dispatch: a slot outside [0, T k) (its workspace
+                                  changed while the call ran) */
 #define MOE_DEV_TIMEOUT 8      /* a pipeline wait exceeded its time limit        */
 
 /* Limits of this build. */

@@ -202,7 +202,8 @@ __global__ void __launch_bounds__(1024) dispatch_scatter_kernel(const uint4* __r
                                         const int32_t* __restrict__ offsets,
                                         int32_t* __restrict__ src_row,
                                         int32_t* __restrict__ dst_pos, uint4* __restrict__ x_perm,
-                                        int row_vec, const float* __restrict__ row_w, int bf16) {
+                                        int row_vec, const float* __restrict__ row_w, int bf16,
+                                        int* status) {
   pdl_wait();
   pdl_trigger();
   extern __shared__ int sm[];
@@ -235,6 +236,12 @@ __global__ void __launch_bounds__(1024) dispatch_scatter_kernel(const uint4* __r
       const int leader = __ffs(peers) - 1;
       int sl = -1;
       if (key >= 0) sl = run[key] + rank;
+      // a slot outside [0, T k) can only come from a table overwritten while
+      // the call ran: skip the copy, flag it, keep every access in bounds
+      if (static_cast<unsigned long long>(static_cast<unsigned>(sl)) >= 1ULL * T * k && sl != -1) {
+        sl = -1;
+        if (status) set_status(status, MOE_DEV_BAD_OFFSETS);
+      }
       __syncwarp();
       if (key >= 0 && lane == leader) run[key] += __popc(peers);
       __syncwarp();
@@ -336,7 +343,7 @@ cudaError_t launch_dispatch(const DispatchPlan& p, const void* x, const int32_t*
   launch_k(dispatch_scatter_kernel, dim3(p.nblk), dim3(threads), sm3, s,
            static_cast<const uint4*>(x), topk_idx, p.T, p.k, p.E, p.R, p.L, p.S, p.tb, p.nbins,
            blk, offsets, src_row, dst_pos, static_cast<uint4*>(x_perm), row_vec, row_w,
-           dt == MOE_BF16 ? 1 : 0);
+           dt == MOE_BF16 ? 1 : 0, status);
   return cudaGetLastError();
 }
 

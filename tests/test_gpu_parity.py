@@ -363,6 +363,9 @@ def test_grouped_swiglu_gather_full_size_sampled(M, cfg):
     # half padding), empty experts, h and d that leave partial n-tiles
     ([256, 128, 129, 1, 0, 31, 32, 33, 384, 511], 192, 320),
     ([600, 200, 90], 320, 448),
+    # last blocks of 1, 44 and 128 rows after full pair tiles (computed with
+    # their pair tile), one of 129 rows (a pair tile of its own)
+    ([257, 300, 640, 385, 130, 2], 128, 192),
 ])
 @pytest.mark.parametrize("row_scale", [False, True])
 def test_grouped_swiglu_pair_tile_mix(M, counts, d, h, row_scale):
