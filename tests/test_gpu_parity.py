@@ -385,6 +385,45 @@ def test_grouped_swiglu_pair_tile_mix(M, counts, d, h, row_scale):
     close(gy.cpu(), ref, bf)
 
 
+def test_grouped_swiglu_long_reduction_tails(M):
+    """Reductions of 2624 in both GEMMs (the long-reduction path): a
+    segment's short last block after its full 256-row pair tiles runs in the
+    single-CTA launch (last blocks of 1, 44, 64, 65 and 128 rows), a
+    129-row last block and segments of at most 128 rows are pair tiles of
+    their own; 2624 hidden units and output columns leave partial n-tiles.
+    Sampled rows (every segment's first and last rows, the rows around each
+    256-row boundary, a random few) against the oracle's per-expert SwiGLU,
+    with a row scale."""
+    counts = [257, 300, 320, 321, 384, 385, 640, 130, 2, 0]
+    d = h = 2624
+    g = torch.Generator().manual_seed(11)
+    E, N = len(counts), int(sum(counts))
+    bf = torch.bfloat16
+    xp = torch.randn(N, d, generator=g).to(bf)
+    w1 = (torch.randn(E, h, d, generator=g) / math.sqrt(d)).to(bf)
+    w3 = (torch.randn(E, h, d, generator=g) / math.sqrt(d)).to(bf)
+    w2 = (torch.randn(E, d, h, generator=g) / math.sqrt(h)).to(bf)
+    off = np.concatenate([[0], np.cumsum(counts)]).astype(np.int64)
+    rs = torch.rand(N, generator=g)
+    gy, ws = M.grouped_swiglu(xp.cuda(), i32(off), w1.cuda(), w3.cuda(), w2.cuda(), rs.cuda())
+    assert M.device_status(ws) == 0
+    gy = gy.cpu()
+    assert torch.isfinite(gy.float()).all()
+    rng = np.random.default_rng(3)
+    for e in range(E):
+        lo, hi = int(off[e]), int(off[e + 1])
+        if hi == lo:
+            continue
+        rows = {lo, hi - 1, min(lo + 1, hi - 1), max(hi - 2, lo)}
+        for b in range(256, hi - lo, 256):
+            rows |= {lo + b - 1, lo + b, min(lo + b + 63, hi - 1), min(lo + b + 64, hi - 1)}
+        rows |= set(rng.integers(lo, hi, size=4).tolist())
+        r = torch.tensor(sorted(rows))
+        ref = O.grouped_swiglu(xp[r], np.array([0, len(r)]), w1[e:e + 1], w3[e:e + 1],
+                               w2[e:e + 1], rs[r].numpy())
+        close(gy[r], ref, bf)
+
+
 def test_grouped_swiglu_all_rows_one_expert(M):
     T, E, k = 1500, 8, 1
     L = W.make_logits(T, E, k, seed=3)
