@@ -552,3 +552,71 @@ def test_forward_edge_shapes(M, T, d, E, k, h, ep):
     x, wr, w1, w3, w2 = small_layer(T, d, E, k, h, seed=T + 1)
     wr = (wr.float() * 50).to(torch.bfloat16)
     forward_check(M, x, wr, w1, w3, w2, k, True, ep, sample=None)
+
+
+# ---------------------------------------------------------- NaN scores
+def test_router_nan_logits_from_logits(M):
+    """Logits with NaN entries: a NaN score never wins over a number (it is
+    taken as -inf for the selection), so the routing equals the oracle's on
+    the same logits with NaN set to -inf; weights of rows with a finite
+    winner stay finite."""
+    T, E, k = 300, 64, 6
+    L = W.make_logits(T, E, k, seed=21)
+    rng = np.random.default_rng(21)
+    mask = rng.random((T, E)) < 0.1
+    L[mask] = np.nan
+    gi, gw, gc, _, ws = M.router_topk(logits_in=torch.from_numpy(L).cuda(), top_k=k,
+                                      renormalize=True)
+    torch.cuda.synchronize()
+    assert M.device_status(ws) == 0
+    Lr = np.where(np.isnan(L), -np.inf, L)
+    idx, w, counts, _ = O.router_topk(k, True, logits=Lr)
+    assert np.array_equal(gi.cpu().numpy(), idx)
+    assert np.array_equal(gc.cpu().numpy(), counts)
+    close(gw, w, torch.float32)
+
+
+def test_router_nan_tokens_fused_gate(M):
+    """The fused router on tokens whose x holds a NaN (all their logits
+    NaN): every key ties at -inf, so the k lowest expert ids are selected;
+    the other tokens route as without them."""
+    T, d, E, k = 512, 256, 32, 4
+    g = torch.Generator().manual_seed(5)
+    x = torch.randn(T, d, generator=g).to(torch.bfloat16)
+    wr = (torch.randn(E, d, generator=g) * 0.1).to(torch.bfloat16)
+    bad = torch.tensor([0, 17, 255, 511])
+    xn = x.clone()
+    xn[bad, 3] = float("nan")
+    gi, gw, gc, _, ws = M.router_topk(xn.cuda(), wr.cuda(), top_k=k, renormalize=True)
+    gi0, gw0, _, _, _ = M.router_topk(x.cuda(), wr.cuda(), top_k=k, renormalize=True)
+    torch.cuda.synchronize()
+    assert M.device_status(ws) == 0
+    gi, gi0 = gi.cpu().numpy(), gi0.cpu().numpy()
+    assert (gi[bad.numpy()] == np.arange(k)[None, :]).all()
+    good = np.setdiff1d(np.arange(T), bad.numpy())
+    assert np.array_equal(gi[good], gi0[good])
+    assert torch.equal(gw.cpu()[good], gw0.cpu()[good])
+    assert np.array_equal(gc.cpu().numpy(), np.bincount(gi.ravel(), minlength=E))
+
+
+def test_router_nan_expert_fused_gate(M):
+    """A NaN in one row of w_router: that expert's logit is NaN for every
+    token and is never selected; the routing equals the oracle's on the
+    GPU's own logits with NaN set to -inf."""
+    T, d, E, k = 700, 512, 48, 5
+    g = torch.Generator().manual_seed(6)
+    x = torch.randn(T, d, generator=g).to(torch.bfloat16)
+    wr = (torch.randn(E, d, generator=g) * 0.1).to(torch.bfloat16)
+    wr[7, 11] = float("nan")
+    gi, gw, gc, gl, ws = M.router_topk(x.cuda(), wr.cuda(), top_k=k, renormalize=True,
+                                       want_logits=True)
+    torch.cuda.synchronize()
+    assert M.device_status(ws) == 0
+    L = gl.cpu().numpy()
+    assert np.isnan(L[:, 7]).all() and np.isfinite(np.delete(L, 7, axis=1)).all()
+    idx, w, counts, _ = O.router_topk(k, True, logits=np.where(np.isnan(L), -np.inf, L))
+    gi = gi.cpu().numpy()
+    assert not (gi == 7).any()
+    assert np.array_equal(gi, idx)
+    assert np.array_equal(gc.cpu().numpy(), counts)
+    close(gw, w, torch.float32)
