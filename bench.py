@@ -521,9 +521,17 @@ def profile_stage(args):
     run one stage of the layer three times (no timing, no JSON).  router:
     only x and w_router are allocated; grouped_swiglu: the layer is routed
     and dispatched once, then the experts run three times."""
+    import dataclasses
     import routing_dispatch_grouped_topk_b200 as M
     M.lib()
     cfg = W.config(args.config)
+    if args.profile_experts:
+        # the same layer with fewer experts and as many rows per expert (the
+        # same kernels, reduction lengths and segment tails on a device
+        # footprint small enough for multi-pass captures)
+        E2 = args.profile_experts
+        cfg = dataclasses.replace(cfg, E=E2, T=cfg.T * E2 // cfg.E, ep_ranks=1,
+                                  name=f"{cfg.name}_E{E2}")
     dev = torch.device("cuda", 0)
     T, d, E, k = cfg.T, cfg.d, cfg.E, cfg.top_k
     dt = M.MOE_BF16 if cfg.dtype == "bf16" else M.MOE_F32
@@ -979,6 +987,9 @@ def main():
     ap.add_argument("--profile-stage", default="all", choices=["all", "router", "grouped_swiglu"],
                     help="with --profile: run only this stage three times (small device "
                          "footprint for multi-pass captures)")
+    ap.add_argument("--profile-experts", type=int, default=0,
+                    help="with --profile-stage: the workload with this many experts and the "
+                         "token count scaled to keep the rows per expert")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
