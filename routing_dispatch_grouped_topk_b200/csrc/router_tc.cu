@@ -19,8 +19,8 @@
 // layer forward the CTA also writes the dispatch histogram of its token
 // blocks.  The expert counts of the entry
 // point go through a per-CTA table that a second small kernel sums.  The
-// stage memory is sized so that two CTAs fit on an SM (for E <= 128): the
-// scores and top-k of one CTA overlap the loads of the other.
+// stage memory is sized so that two CTAs fit on an SM (for E <= 128): twice
+// the loads in flight and twice the scoring threads per SM.
 //
 // Every mbarrier wait is bounded (2 s) and unwinds by setting
 // MOE_DEV_TIMEOUT; the control flow after the K loop is the same in every
