@@ -379,6 +379,68 @@ class Layer:
         mark(i + 2)
 
 
+def timed_next_rows(layer, stream, flush, steps):
+    """CUDA-event medians (us; L2 flushed after every call, calls of one kind
+    back to back) of the layer's NEXT-row options at its sizes: the router
+    entry point with each router option ([HP] TokenChoiceTopKRouter's score
+    function, selection-only bias, node-limited groups) and with the capacity
+    drop policy ([PF] moe_gate _probs_drop_policy), and the single-device layer
+    forward (ep_ranks = 1) with and without the capacity.  The capacity is the
+    mean load per expert, so the copies routed past it to busier experts are
+    dropped.  None for fp32 layers."""
+    c, M = layer.cfg, layer.M
+    if layer.dt != M.MOE_BF16:
+        return None
+    T, d, E, k, h, dt, dev = c.T, c.d, c.E, c.top_k, c.h, layer.dt, layer.dev
+    cap = -(-T * k // E)
+    bias = torch.linspace(-0.05, 0.05, E, device=dev)
+    idx = torch.empty(T, k, dtype=torch.int32, device=dev)
+    w = torch.empty(T, k, dtype=torch.float32, device=dev)
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    rws = torch.empty(M.router_workspace_size(T, d, E, dt), dtype=torch.uint8, device=dev)
+    out1 = torch.empty_like(layer.out)
+    fws = torch.empty(M.forward_ex_workspace_size(T, d, E, k, h, 1, dt), dtype=torch.uint8,
+                      device=dev)
+
+    def timed(fn):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps + 1)]
+        torch.cuda.synchronize()
+        for a_ev, b_ev in ev:
+            a_ev.record(stream)
+            fn()
+            b_ev.record(stream)
+            flush.zero_()
+        torch.cuda.synchronize()
+        return 1e3 * statistics.median(a.elapsed_time(b) for a, b in ev[1:])
+
+    router = {}
+    variants = {"softmax": {}, "sigmoid": {"score": "sigmoid"}, "expert_bias": {"expert_bias": bias},
+                "node_limited_groups": {"num_groups": 8, "topk_groups": 4}, "capacity": {"capacity": cap}}
+    for name, o in variants.items():
+        if name == "node_limited_groups" and E % 8:
+            continue
+        opts = M.router_options(renormalize=c.renormalize, **o)
+        router[name] = timed(lambda opts=opts: M.moe_router_topk_ex(
+            layer.x, layer.wr, None, T, d, E, k, opts, dt, None, idx, w, counts, rws))
+    M.moe_router_topk_ex(layer.x, layer.wr, None, T, d, E, k,
+                         M.router_options(renormalize=c.renormalize, capacity=cap), dt, None, idx,
+                         w, counts, rws)
+    torch.cuda.synchronize()
+    dropped = int((idx < 0).sum())
+    fwd = {}
+    for name, o in (("forward_ep1_us", {}), ("forward_ep1_capacity_us", {"capacity": cap})):
+        opts = M.router_options(renormalize=c.renormalize, **o)
+        fwd[name] = timed(lambda opts=opts: M.moe_forward_ex(
+            layer.x, layer.wr, None, layer.w1, layer.w3, layer.w2, T, d, E, k, h, opts, None, 1,
+            dt, out1, None, None, None, None, fws))
+    return {"router_us": router,
+            "capacity": dict(capacity=cap, dropped_copies=dropped, copies=T * k, **fwd),
+            "what": "moe_router_topk_ex with each option and moe_forward_ex (ep_ranks 1) with and "
+                    "without the capacity at the headline sizes; medians of calls of one kind, "
+                    "L2 flushed after each call"}
+
+
 def timed_folded(layer, stream, flush, steps):
     """CUDA-event times (ms) of moe_grouped_swiglu_combine (the combine folded
     into GEMM2) and of the unfused moe_grouped_swiglu + moe_combine on the
@@ -699,6 +761,7 @@ def run_ours(args, ws, rank, local):
     # the unfused grouped SwiGLU + combine of the staged step.
     folded = timed_folded(layer, stream, flush, min(args.steps, 5))
     clocks = sampler.stop() if rank == 0 else None
+    next_rows = timed_next_rows(layer, stream, flush, min(args.steps, 5))
 
     if rank != 0:
         return
@@ -769,6 +832,8 @@ def run_ours(args, ws, rank, local):
             "what": "moe_grouped_swiglu_combine (fp32 reductions in GEMM2's epilogue, then one "
                     "bf16 rounding) against moe_grouped_swiglu + moe_combine, medians of "
                     "calls alternating in blocks, L2 flushed between calls"}
+    if next_rows is not None:
+        line["next_rows"] = next_rows
     if ws == 1 and not args.no_other_configs:
         del layer
         torch.cuda.empty_cache()

@@ -759,11 +759,57 @@ cudaError_t launch_router_backward(const float* logits, const int32_t* topk_idx,
 // top `capacity` scores for that expert (ranked over the expert's routed
 // copies; equal scores to the lower token).  Every copy gets a unique 64-bit
 // key, (score, then the token reversed), and one block per expert finds the
-// capacity-th largest key of its copies by an 8-bit radix select over the
-// flat copy list (eight passes); the copies below it are dropped.
+// capacity-th largest key of its copies by an 8-bit radix select (eight
+// passes over the keys it gathered in shared memory in one scan of the flat
+// copy list, or over that list when they do not fit); the copies below it
+// are dropped.
 __device__ __forceinline__ unsigned long long capacity_key(float s, int t) {
   const unsigned hi = static_cast<unsigned>(score_key(s != s ? -INFINITY : s)) ^ 0x80000000u;
   return (static_cast<unsigned long long>(hi) << 32) | (0xFFFFFFFFu - static_cast<unsigned>(t));
+}
+
+// An expert's routed copies gathered in shared memory by the select kernel
+// (more than this: its passes scan the flat copy list instead).
+constexpr int kCapKeys = 4096;
+
+// Warp 0 of the select kernel: the bin of hist[0..255] (taken from the top)
+// that holds the want-th largest key, and how many keys lie in higher bins.
+// Lane l holds bins 8l .. 8l+7; a suffix sum over the lanes finds the lane,
+// its own bins the bin.
+__device__ __forceinline__ void capacity_find_bin(const unsigned* hist, int want, int& bin,
+                                                  int& above) {
+  const int lane = threadIdx.x & 31;
+  unsigned c[8], sum = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    c[j] = hist[8 * lane + j];
+    sum += c[j];
+  }
+  unsigned suf = sum;   // keys in bins >= 8 lane
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const unsigned v = __shfl_down_sync(0xffffffffu, suf, off);
+    if (lane + off < 32) suf += v;
+  }
+  const unsigned w = static_cast<unsigned>(want);
+  const unsigned excl = suf - sum;   // keys in higher lanes' bins
+  const unsigned ball = __ballot_sync(0xffffffffu, excl < w && w <= suf);
+  const int owner = __ffs(ball) - 1;
+  int b = 0, a = 0;
+  if (lane == owner) {
+    unsigned cum = excl;
+#pragma unroll
+    for (int j = 7; j >= 0; --j) {
+      if (cum + c[j] >= w) {
+        b = 8 * lane + j;
+        a = static_cast<int>(cum);
+        break;
+      }
+      cum += c[j];
+    }
+  }
+  bin = __shfl_sync(0xffffffffu, b, owner & 31);
+  above = __shfl_sync(0xffffffffu, a, owner & 31);
 }
 
 __global__ void __launch_bounds__(512) capacity_select_kernel(
@@ -771,21 +817,27 @@ __global__ void __launch_bounds__(512) capacity_select_kernel(
     int capacity, unsigned long long* __restrict__ thr) {
   pdl_wait();
   pdl_trigger();
+  __shared__ unsigned long long keys_s[kCapKeys];
   __shared__ unsigned hist[256];
   __shared__ unsigned long long prefix_s;
   __shared__ int want_s, count_s;
   const int e = blockIdx.x;
   if (threadIdx.x == 0) count_s = 0;
   __syncthreads();
-  int mine = 0;
-  for (long long i = threadIdx.x; i < n; i += blockDim.x) mine += idx[i] == e;
-  atomicAdd(&count_s, mine);
+  // one scan of the copy list: count the expert's copies, keep their keys
+  // while they fit (their order does not matter: the keys are distinct)
+  for (long long i = threadIdx.x; i < n; i += blockDim.x)
+    if (idx[i] == e) {
+      const int p = atomicAdd(&count_s, 1);
+      if (p < kCapKeys) keys_s[p] = capacity_key(scores[i], static_cast<int>(i / k));
+    }
   __syncthreads();
   const int count = count_s;
   if (count <= capacity) {   // nothing to drop: keep every key
     if (threadIdx.x == 0) thr[e] = 0ull;
     return;
   }
+  const bool in_smem = count <= kCapKeys;
   if (threadIdx.x == 0) {
     prefix_s = 0ull;
     want_s = capacity;   // rank (1 = largest) of the key wanted among those left
@@ -795,23 +847,25 @@ __global__ void __launch_bounds__(512) capacity_select_kernel(
     __syncthreads();
     const unsigned long long prefix = prefix_s;
     const unsigned long long hi_mask = shift == 56 ? 0ull : ~0ull << (shift + 8);
-    for (long long i = threadIdx.x; i < n; i += blockDim.x) {
-      if (idx[i] != e) continue;
-      const unsigned long long key = capacity_key(scores[i], static_cast<int>(i / k));
-      if ((key & hi_mask) == (prefix & hi_mask))
-        atomicAdd(&hist[(key >> shift) & 255u], 1u);
+    if (in_smem) {
+      for (int j = threadIdx.x; j < count; j += blockDim.x) {
+        const unsigned long long key = keys_s[j];
+        if ((key & hi_mask) == (prefix & hi_mask)) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+      }
+    } else {
+      for (long long i = threadIdx.x; i < n; i += blockDim.x) {
+        if (idx[i] != e) continue;
+        const unsigned long long key = capacity_key(scores[i], static_cast<int>(i / k));
+        if ((key & hi_mask) == (prefix & hi_mask)) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+      }
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-      int want = want_s, cum = 0;
-      for (int b = 255; b >= 0; --b) {
-        const int c = static_cast<int>(hist[b]);
-        if (cum + c >= want) {
-          prefix_s = prefix | (static_cast<unsigned long long>(b) << shift);
-          want_s = want - cum;
-          break;
-        }
-        cum += c;
+    if (threadIdx.x < 32) {
+      int bin = 0, above = 0;
+      capacity_find_bin(hist, want_s, bin, above);
+      if (threadIdx.x == 0) {
+        prefix_s = prefix | (static_cast<unsigned long long>(bin) << shift);
+        want_s -= above;
       }
     }
     __syncthreads();
