@@ -257,9 +257,8 @@ cudaError_t run_router(const void* x, const void* w_router, const float* logits_
   if (e == cudaSuccess && cap) {
     unsigned long long* thr = reinterpret_cast<unsigned long long*>(
         cap_scratch + align_up(static_cast<size_t>(T) * kMaxTopK * sizeof(float), 256));
-    e = launch_capacity_drop(topk_idx, topk_w, ko.scores_out, T, top_k, E, o.capacity, thr, s);
-    if (e == cudaSuccess && counts) e = cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, s);
-    if (e == cudaSuccess && counts) e = launch_expert_hist(topk_idx, 1LL * T * top_k, E, counts, s);
+    e = launch_capacity_drop(topk_idx, topk_w, ko.scores_out, T, top_k, E, o.capacity, thr,
+                             counts, s);
   }
   // [HP] _compute_load_balance_loss of this call (0 for no tokens)
   if (e == cudaSuccess && lb) e = launch_lb_loss(lb, E, T, top_k, o.aux_loss, s);

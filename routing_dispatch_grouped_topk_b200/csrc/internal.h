@@ -169,10 +169,11 @@ cudaError_t launch_router_backward(const float* logits, const int32_t* topk_idx,
 // Capacity drop policy: for every expert with more than `capacity` routed
 // copies, keep the `capacity` of them with the highest score (scores [T, k],
 // the router's scores_out), equal scores to the lower token; the others get
-// topk_idx = -1 and topk_w = 0.  thr is device scratch for E 64-bit keys.
+// topk_idx = -1 and topk_w = 0.  thr is device scratch for E 64-bit keys;
+// counts [E] (or null) receives the copies each expert keeps.
 cudaError_t launch_capacity_drop(int32_t* topk_idx, float* topk_w, const float* scores, int T,
                                  int k, int E, int capacity, unsigned long long* thr,
-                                 cudaStream_t s);
+                                 int32_t* counts, cudaStream_t s);
 // counts [E] += histogram of idx [n] (counts cleared by the caller).
 cudaError_t launch_expert_hist(const int32_t* idx, long long n, int E, int32_t* counts,
                                cudaStream_t s);

@@ -814,7 +814,7 @@ __device__ __forceinline__ void capacity_find_bin(const unsigned* hist, int want
 
 __global__ void __launch_bounds__(512) capacity_select_kernel(
     const int32_t* __restrict__ idx, const float* __restrict__ scores, long long n, int k,
-    int capacity, unsigned long long* __restrict__ thr) {
+    int capacity, unsigned long long* __restrict__ thr, int32_t* __restrict__ counts) {
   pdl_wait();
   pdl_trigger();
   __shared__ unsigned long long keys_s[kCapKeys];
@@ -833,6 +833,8 @@ __global__ void __launch_bounds__(512) capacity_select_kernel(
     }
   __syncthreads();
   const int count = count_s;
+  // the copies the expert keeps: all of them, or the `capacity` largest keys
+  if (threadIdx.x == 0 && counts) counts[e] = min(count, capacity);
   if (count <= capacity) {   // nothing to drop: keep every key
     if (threadIdx.x == 0) thr[e] = 0ull;
     return;
@@ -892,10 +894,11 @@ __global__ void capacity_apply_kernel(int32_t* __restrict__ idx, float* __restri
 
 cudaError_t launch_capacity_drop(int32_t* topk_idx, float* topk_w, const float* scores, int T,
                                  int k, int E, int capacity, unsigned long long* thr,
-                                 cudaStream_t s) {
+                                 int32_t* counts, cudaStream_t s) {
   const long long n = 1LL * T * k;
   if (n == 0) return cudaSuccess;
-  launch_k(capacity_select_kernel, dim3(E), dim3(512), 0, s, topk_idx, scores, n, k, capacity, thr);
+  launch_k(capacity_select_kernel, dim3(E), dim3(512), 0, s, topk_idx, scores, n, k, capacity, thr,
+           counts);
   const int blocks = static_cast<int>(std::min<long long>((n + 255) / 256, 8LL * num_sms()));
   launch_k(capacity_apply_kernel, dim3(blocks), dim3(256), 0, s, topk_idx, topk_w, scores, n, k,
            E, static_cast<const unsigned long long*>(thr));
