@@ -358,3 +358,27 @@ def test_fused_router_options(M, T, d, E, k, vi, renorm):
     assert np.array_equal(gc.cpu().numpy(), np.bincount(gi.ravel(), minlength=E))
     s, _, _ = oracle_keys(O.as_f64(L), o)
     close(sc.cpu(), np.take_along_axis(s, gi.astype(np.int64), axis=1), torch.float32)
+
+
+# Node-limited groups on the tensor-core router (split-K gate and the
+# warp-per-token top-k) over token counts, reductions and expert counts
+GROUP_SHAPES = [(200, 1024, 64, 5), (6000, 512, 128, 16), (3000, 128, 32, 3), (129, 64, 256, 1)]
+
+
+@pytest.mark.parametrize("T,d,E,k", GROUP_SHAPES)
+@pytest.mark.parametrize("vi", [3, 4, 6])
+@pytest.mark.parametrize("renorm", [False, True])
+def test_router_node_limited_groups_gemm(M, T, d, E, k, vi, renorm):
+    """Group-limited routing (8 groups; 3 or 4 kept) on the bf16 gate, with
+    sigmoid scores, a scale and a selection-only bias: indices and weights
+    against the oracle's general router on the GPU's own logits."""
+    g = torch.Generator().manual_seed(T + d + E + k + vi)
+    x = torch.randn(T, d, generator=g).to(torch.bfloat16).cuda()
+    wr = (torch.randn(E, d, generator=g) * (2.0 / d ** 0.5)).to(torch.bfloat16).cuda()
+    o, go = materialize(dict(VARIANTS[vi]), E, seed=vi)
+    gi, gw, gc, logits, ws = M.router_topk(x, wr, k, renorm, want_logits=True, **go)
+    torch.cuda.synchronize()
+    assert M.device_status(ws) == 0
+    gi = gi.cpu().numpy()
+    check_router(gi, gw.cpu(), logits.cpu().numpy(), k, renorm, o)
+    assert np.array_equal(gc.cpu().numpy(), np.bincount(gi.ravel(), minlength=E))
